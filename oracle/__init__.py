@@ -1,0 +1,215 @@
+"""CPU oracle for the rotated W4A4 linear layer (test infrastructure only).
+
+Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's CPU
+baseline import this package.  The product library never does, and nothing
+here touches the CUDA path: this is a ctypes wrapper around the plain C file
+``convrot_oracle.c`` (see its header for what each step computes and which
+page section it follows).
+
+Arrays are numpy; bf16 values travel as ``uint16`` bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "convrot_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+# Plain IEEE semantics: no fast-math, no contraction of a*b+c into an FMA.
+_CFLAGS = ["-O2", "-std=c99", "-fPIC", "-shared", "-fopenmp", "-fno-fast-math",
+           "-ffp-contract=off"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc if the shared object is missing or stale."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *_CFLAGS, _SRC, "-o", tmp, "-lm"], check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        I = ctypes.c_int
+        sig = {
+            "oracle_bf16_to_double": [P, I64, P],
+            "oracle_float_to_bf16": [P, I64, P],
+            "oracle_hadamard": [I, P],
+            "oracle_hadamard_kron": [I, P],
+            "oracle_rotate": [P, I64, I64, I, P],
+            "oracle_quantize_rows": [P, I64, I64, P, P],
+            "oracle_pack": [P, I64, I64, P],
+            "oracle_unpack": [P, I64, I64, P],
+            "oracle_gemm": [P, P, I64, I64, I64, P],
+            "oracle_epilogue": [P, P, P, P, I64, I64, P],
+            "oracle_prepare_rows": [P, I64, I64, I, P, P],
+            "oracle_linear_prepared_w": [P, P, P, P, I64, I64, I64, I, P],
+            "oracle_num_threads": [],
+        }
+        for name, args in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ctypes.c_int
+        L.oracle_set_num_threads.argtypes = [I]
+        L.oracle_set_num_threads.restype = None
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle buffers must be contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise ValueError(f"{what}: oracle rejected the arguments (rc={rc})")
+
+
+def set_num_threads(t: int) -> None:
+    lib().oracle_set_num_threads(int(t))
+
+
+def num_threads() -> int:
+    return int(lib().oracle_num_threads())
+
+
+# --------------------------------------------------------------------------
+# bf16 helpers
+# --------------------------------------------------------------------------
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    out = np.empty(bits.shape, dtype=np.float64)
+    _check(lib().oracle_bf16_to_double(_ptr(bits), bits.size, _ptr(out)), "bf16_to_f64")
+    return out
+
+
+def f32_to_bf16(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, dtype=np.uint16)
+    _check(lib().oracle_float_to_bf16(_ptr(x), x.size, _ptr(out)), "f32_to_bf16")
+    return out
+
+
+# --------------------------------------------------------------------------
+# The method's steps
+# --------------------------------------------------------------------------
+
+def hadamard(n: int) -> np.ndarray:
+    H = np.empty((n, n), dtype=np.float64)
+    _check(lib().oracle_hadamard(n, _ptr(H)), "hadamard")
+    return H
+
+
+def hadamard_kron(n: int) -> np.ndarray:
+    H = np.empty((n, n), dtype=np.float64)
+    _check(lib().oracle_hadamard_kron(n, _ptr(H)), "hadamard_kron")
+    return H
+
+
+def rotate(x_bf16: np.ndarray, group: int) -> np.ndarray:
+    """fp64 rows of x (I_G (x) H_group)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    rows, K = x.shape
+    y = np.empty((rows, K), dtype=np.float64)
+    _check(lib().oracle_rotate(_ptr(x), rows, K, group, _ptr(y)), "rotate")
+    return y
+
+
+def quantize_rows(y: np.ndarray):
+    """(codes int8 [rows][K], scales fp32 [rows]) from fp64 rotated rows."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    rows, K = y.shape
+    q = np.empty((rows, K), dtype=np.int8)
+    s = np.empty((rows,), dtype=np.float32)
+    _check(lib().oracle_quantize_rows(_ptr(y), rows, K, _ptr(q), _ptr(s)), "quantize_rows")
+    return q, s
+
+
+def pack(q: np.ndarray) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    rows, K = q.shape
+    p = np.empty((rows, K // 2), dtype=np.uint8)
+    _check(lib().oracle_pack(_ptr(q), rows, K, _ptr(p)), "pack")
+    return p
+
+
+def unpack(p: np.ndarray, K: int) -> np.ndarray:
+    p = np.ascontiguousarray(p, dtype=np.uint8)
+    rows = p.shape[0]
+    q = np.empty((rows, K), dtype=np.int8)
+    _check(lib().oracle_unpack(_ptr(p), rows, K, _ptr(q)), "unpack")
+    return q
+
+
+def gemm(qx: np.ndarray, qw: np.ndarray, K: int) -> np.ndarray:
+    """int64 acc[m][n] = sum_k qx[m][k] qw[n][k] from packed operands."""
+    qx = np.ascontiguousarray(qx, dtype=np.uint8)
+    qw = np.ascontiguousarray(qw, dtype=np.uint8)
+    M, N = qx.shape[0], qw.shape[0]
+    acc = np.empty((M, N), dtype=np.int64)
+    _check(lib().oracle_gemm(_ptr(qx), _ptr(qw), M, N, K, _ptr(acc)), "gemm")
+    return acc
+
+
+def epilogue(acc: np.ndarray, sx: np.ndarray, sw: np.ndarray, bias_bf16: np.ndarray | None):
+    acc = np.ascontiguousarray(acc, dtype=np.int64)
+    sx = np.ascontiguousarray(sx, dtype=np.float32)
+    sw = np.ascontiguousarray(sw, dtype=np.float32)
+    b = None if bias_bf16 is None else np.ascontiguousarray(bias_bf16, dtype=np.uint16)
+    M, N = acc.shape
+    y = np.empty((M, N), dtype=np.uint16)
+    _check(lib().oracle_epilogue(_ptr(acc), _ptr(sx), _ptr(sw), _ptr(b), M, N, _ptr(y)),
+           "epilogue")
+    return y
+
+
+def prepare_rows(x_bf16: np.ndarray, group: int):
+    """(packed uint8 [rows][K/2], scales fp32 [rows]): rotate, quantise, pack."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    rows, K = x.shape
+    p = np.empty((rows, K // 2), dtype=np.uint8)
+    s = np.empty((rows,), dtype=np.float32)
+    _check(lib().oracle_prepare_rows(_ptr(x), rows, K, group, _ptr(p), _ptr(s)), "prepare_rows")
+    return p, s
+
+
+def linear_prepared_w(x_bf16, qw, sw, bias_bf16, group: int) -> np.ndarray:
+    """bf16 bits y [M][N] of the whole layer given prepared weights."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    qw = np.ascontiguousarray(qw, dtype=np.uint8)
+    sw = np.ascontiguousarray(sw, dtype=np.float32)
+    b = None if bias_bf16 is None else np.ascontiguousarray(bias_bf16, dtype=np.uint16)
+    M, K = x.shape
+    N = qw.shape[0]
+    y = np.empty((M, N), dtype=np.uint16)
+    _check(lib().oracle_linear_prepared_w(_ptr(x), _ptr(qw), _ptr(sw), _ptr(b), M, N, K, group,
+                                          _ptr(y)), "linear_prepared_w")
+    return y
+
+
+def tie_band(y: np.ndarray, s: np.ndarray, band: float = 1e-5) -> np.ndarray:
+    """Mask of positions whose fp64 y/s lies within ``band`` of a .5 rounding
+    boundary: the only positions where a code may legitimately differ between
+    two fp32 evaluations of the rotation (different summation order)."""
+    s64 = s.astype(np.float64)[:, None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = np.where(s64 > 0, y / np.where(s64 > 0, s64, 1.0), 0.0)
+    a = np.abs(v)
+    return np.abs(a - (np.floor(a) + 0.5)) < band

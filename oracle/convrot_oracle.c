@@ -1,0 +1,369 @@
+/*
+ * convrot_oracle.c -- plain, slow CPU oracle for the rotated W4A4 linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links, loads or calls
+ * this file; only the test suite, the smoke check and the benchmark's CPU
+ * baseline do.  It shares no code, header, table or constant with the CUDA
+ * library and is written to be checked against the pages by eye: dense
+ * matrices, scalar loops, fp64 wherever the pages leave the precision open.
+ *
+ * What it computes (sources are the pages' titles and sections):
+ *
+ *  - H_n, the normalised regular Hadamard matrix of order n = 4^k.
+ *    "convrot-mlx" README, "What is included": normalised regular-Hadamard
+ *    rotation for groups of 64 and 256.  Comfy-Org/comfy-quants issue
+ *    "convrot is exactly same as ... QuaRot Stage 1c", section 2 ("The
+ *    equivalent Hadamard matrix"): the regular matrix is used for N_0 = 4^k.
+ *    Reading: H_n = (J - 2I)^{(x)k} / sqrt(n), the k-th Kronecker power of the
+ *    order-4 regular Hadamard J - 2I, normalised so that H H^T = I.
+ *    Entry (i, j) is (-1)^{number of base-4 digit positions where i and j
+ *    agree} / sqrt(n).  oracle_hadamard builds it from that digit rule;
+ *    oracle_hadamard_kron builds it by literal repeated Kronecker products.
+ *
+ *  - The block rotation R = I_G (x) H_n.  Same issue, section 1 ("Both apply
+ *    'group-wise' operator"): X R = [X_1 H, ..., X_G H], one Hadamard per
+ *    K-group of n channels.  Written here as a dense fp64 mat-vec per group.
+ *
+ *  - Rowwise symmetric absmax INT4 in [-7, 7].  "convrot-mlx" README, "What is
+ *    included".  One scale per row (per token for activations, per output
+ *    channel for weights); the group size only affects the rotation.
+ *    Readings (the pages leave these open): the decision is taken in fp32,
+ *      a   = fp32(max_k |y_k|)         (y the fp64 rotated row)
+ *      s   = a / 7                      (fp32, IEEE division; the stored scale)
+ *      inv = 7 / a                      (fp32, IEEE division)
+ *      v_k = fp32(y_k) * inv            (one fp32 multiply)
+ *      q_k = clamp(round_half_away(v_k), -7, 7);  a == 0 gives s = 0, q = 0.
+ *
+ *  - Packing, two codes per byte, low nibble = even k, 4-bit two's complement.
+ *    "convrot-mlx" README, "What is included" (N x packed-K layout); nibble
+ *    order per "mlx-nf4" README, "What it provides" (low-first intake).
+ *
+ *  - The integer GEMM acc[m][n] = sum_k qx[m][k] * qw[n][k] in int64, and the
+ *    epilogue y = bf16_rne(((float)acc * sx[m]) * sw[n] + (float)b[n]) in
+ *    fp32 in that order.  "convrot-mlx" README, "Install and test": the
+ *    complete path is rotation, activation quantisation, the integer product,
+ *    scaling and bias.
+ *
+ * Every function returns 0 on success or a negative number for bad
+ * arguments.  Buffers are caller-owned, row-major and contiguous.
+ * bf16 values travel as their raw 16-bit patterns (uint16_t).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ----------------------------------------------------------------------- */
+/* bf16 <-> float, written out by hand.                                     */
+/* ----------------------------------------------------------------------- */
+
+/* A bf16 pattern is the top half of an IEEE binary32 pattern. */
+static double bf16_bits_to_double(uint16_t h) {
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Round a finite binary32 to bf16, nearest-even on the 16 dropped bits. */
+static uint16_t float_to_bf16_bits_rne(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7F800000u) == 0x7F800000u) {            /* inf / nan: keep */
+        uint16_t h = (uint16_t)(u >> 16);
+        if (u & 0x007FFFFFu) h |= 0x0040u;              /* quiet nan */
+        return h;
+    }
+    uint32_t dropped = u & 0xFFFFu;
+    uint32_t kept = u >> 16;
+    if (dropped > 0x8000u || (dropped == 0x8000u && (kept & 1u))) kept += 1u;
+    return (uint16_t)kept;
+}
+
+int oracle_bf16_to_double(const uint16_t *in, int64_t count, double *out) {
+    if (!in || !out || count < 0) return -1;
+    for (int64_t i = 0; i < count; ++i) out[i] = bf16_bits_to_double(in[i]);
+    return 0;
+}
+
+int oracle_float_to_bf16(const float *in, int64_t count, uint16_t *out) {
+    if (!in || !out || count < 0) return -1;
+    for (int64_t i = 0; i < count; ++i) out[i] = float_to_bf16_bits_rne(in[i]);
+    return 0;
+}
+
+/* ----------------------------------------------------------------------- */
+/* The regular Hadamard matrix.                                             */
+/* ----------------------------------------------------------------------- */
+
+/* k such that n == 4^k, or -1. */
+static int log4_exact(int n) {
+    int k = 0;
+    if (n < 1) return -1;
+    while (n > 1) {
+        if (n % 4) return -1;
+        n /= 4;
+        ++k;
+    }
+    return k;
+}
+
+/* H[i*n + j] = (-1)^{#digits where i and j agree} / sqrt(n). */
+int oracle_hadamard(int n, double *H) {
+    int k = log4_exact(n);
+    if (k < 0 || !H) return -1;
+    double norm = 1.0 / sqrt((double)n);
+    for (int i = 0; i < n; ++i) {
+        for (int j = 0; j < n; ++j) {
+            int agree = 0, a = i, b = j;
+            for (int d = 0; d < k; ++d) {
+                if (a % 4 == b % 4) ++agree;
+                a /= 4;
+                b /= 4;
+            }
+            H[(int64_t)i * n + j] = (agree % 2 ? -1.0 : 1.0) * norm;
+        }
+    }
+    return 0;
+}
+
+/* The same matrix by literal Kronecker products: start from the 1x1 matrix
+ * [1] and k times form P <- P (x) T with T = (J - 2I) / 2. */
+int oracle_hadamard_kron(int n, double *H) {
+    int k = log4_exact(n);
+    if (k < 0 || !H) return -1;
+    double T[4][4];
+    for (int a = 0; a < 4; ++a)
+        for (int b = 0; b < 4; ++b) T[a][b] = (a == b ? -1.0 : 1.0) / 2.0;
+    double *P = (double *)malloc(sizeof(double) * (size_t)n * n);
+    double *Q = (double *)malloc(sizeof(double) * (size_t)n * n);
+    if (!P || !Q) { free(P); free(Q); return -2; }
+    int m = 1;
+    P[0] = 1.0;
+    for (int step = 0; step < k; ++step) {
+        int m4 = m * 4;
+        /* (P (x) T)[r*4 + a][c*4 + b] = P[r][c] * T[a][b] */
+        for (int r = 0; r < m; ++r)
+            for (int c = 0; c < m; ++c)
+                for (int a = 0; a < 4; ++a)
+                    for (int b = 0; b < 4; ++b)
+                        Q[(int64_t)(r * 4 + a) * m4 + (c * 4 + b)] = P[(int64_t)r * m + c] * T[a][b];
+        double *t = P; P = Q; Q = t;
+        m = m4;
+    }
+    memcpy(H, P, sizeof(double) * (size_t)n * n);
+    free(P);
+    free(Q);
+    return 0;
+}
+
+/* ----------------------------------------------------------------------- */
+/* Block rotation X -> X (I_G (x) H_n).                                      */
+/* ----------------------------------------------------------------------- */
+
+/* y[r][g*n + i] = sum_j x[r][g*n + j] * H[j][i], all in fp64.
+ * x is bf16 (rows x K); K must be a multiple of n. */
+int oracle_rotate(const uint16_t *x, int64_t rows, int64_t K, int n, double *y) {
+    if (!x || !y || rows < 0 || K <= 0 || log4_exact(n) < 0 || K % n) return -1;
+    double *H = (double *)malloc(sizeof(double) * (size_t)n * n);
+    if (!H) return -2;
+    oracle_hadamard(n, H);
+    int64_t G = K / n;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        double *xg = (double *)malloc(sizeof(double) * (size_t)n);
+        for (int64_t g = 0; g < G; ++g) {
+            const uint16_t *src = x + r * K + g * n;
+            for (int j = 0; j < n; ++j) xg[j] = bf16_bits_to_double(src[j]);
+            double *dst = y + r * K + g * n;
+            for (int i = 0; i < n; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < n; ++j) acc += xg[j] * H[(int64_t)j * n + i];
+                dst[i] = acc;
+            }
+        }
+        free(xg);
+    }
+    free(H);
+    return 0;
+}
+
+/* ----------------------------------------------------------------------- */
+/* Rowwise symmetric absmax quantisation to [-7, 7].                         */
+/* ----------------------------------------------------------------------- */
+
+/* Round half away from zero, written from its definition: the integer
+ * nearest to v, and on an exact tie the one of larger magnitude. */
+static int round_half_away(float v) {
+    double a = fabs((double)v);
+    double f = floor(a);
+    double frac = a - f;                  /* exact in double */
+    int mag = (int)f + (frac >= 0.5 ? 1 : 0);
+    return v < 0.0f ? -mag : mag;
+}
+
+int oracle_quantize_rows(const double *y, int64_t rows, int64_t K, int8_t *q, float *s) {
+    if (!y || !q || !s || rows < 0 || K <= 0) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const double *yr = y + r * K;
+        double amax = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            double t = fabs(yr[k]);
+            if (t > amax) amax = t;
+        }
+        float a = (float)amax;
+        if (a == 0.0f) {
+            s[r] = 0.0f;
+            memset(q + r * K, 0, (size_t)K);
+            continue;
+        }
+        float sr = a / 7.0f;
+        float inv = 7.0f / a;
+        s[r] = sr;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = (float)yr[k] * inv;
+            int c = round_half_away(v);
+            if (c > 7) c = 7;
+            if (c < -7) c = -7;
+            q[r * K + k] = (int8_t)c;
+        }
+    }
+    return 0;
+}
+
+/* ----------------------------------------------------------------------- */
+/* Nibble packing.                                                           */
+/* ----------------------------------------------------------------------- */
+
+/* byte[j] = (q[2j] & 0xF) | ((q[2j+1] & 0xF) << 4).  K must be even. */
+int oracle_pack(const int8_t *q, int64_t rows, int64_t K, uint8_t *p) {
+    if (!q || !p || rows < 0 || K <= 0 || K % 2) return -1;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < K / 2; ++j) {
+            uint8_t lo = (uint8_t)q[r * K + 2 * j] & 0x0Fu;
+            uint8_t hi = (uint8_t)q[r * K + 2 * j + 1] & 0x0Fu;
+            p[r * (K / 2) + j] = (uint8_t)(lo | (hi << 4));
+        }
+    return 0;
+}
+
+/* A 4-bit two's complement nibble back to a signed integer. */
+static int nibble_to_int(unsigned v) {
+    v &= 0x0Fu;
+    return v >= 8u ? (int)v - 16 : (int)v;
+}
+
+int oracle_unpack(const uint8_t *p, int64_t rows, int64_t K, int8_t *q) {
+    if (!p || !q || rows < 0 || K <= 0 || K % 2) return -1;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < K / 2; ++j) {
+            uint8_t b = p[r * (K / 2) + j];
+            q[r * K + 2 * j] = (int8_t)nibble_to_int(b);
+            q[r * K + 2 * j + 1] = (int8_t)nibble_to_int(b >> 4);
+        }
+    return 0;
+}
+
+/* ----------------------------------------------------------------------- */
+/* Integer GEMM and epilogue.                                                */
+/* ----------------------------------------------------------------------- */
+
+/* acc[m][n] = sum_k qx[m][k] * qw[n][k]; both operands packed [rows][K/2]. */
+int oracle_gemm(const uint8_t *qx, const uint8_t *qw, int64_t M, int64_t N, int64_t K,
+                int64_t *acc) {
+    if (!qx || !qw || !acc || M < 0 || N < 0 || K <= 0 || K % 2) return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; ++m) {
+        int8_t *a = (int8_t *)malloc((size_t)K);
+        int8_t *b = (int8_t *)malloc((size_t)K);
+        oracle_unpack(qx + m * (K / 2), 1, K, a);
+        for (int64_t n = 0; n < N; ++n) {
+            oracle_unpack(qw + n * (K / 2), 1, K, b);
+            int64_t s = 0;
+            for (int64_t k = 0; k < K; ++k) s += (int64_t)a[k] * (int64_t)b[k];
+            acc[m * N + n] = s;
+        }
+        free(a);
+        free(b);
+    }
+    return 0;
+}
+
+/* y[m][n] = bf16_rne( ((float)acc * sx[m]) * sw[n] + (float)bias[n] ), fp32,
+ * no fused multiply-add; bias may be NULL (zeros). */
+int oracle_epilogue(const int64_t *acc, const float *sx, const float *sw, const uint16_t *bias,
+                    int64_t M, int64_t N, uint16_t *y) {
+    if (!acc || !sx || !sw || !y || M < 0 || N < 0) return -1;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            float t = (float)acc[m * N + n];
+            t = t * sx[m];
+            t = t * sw[n];
+            float b = bias ? (float)bf16_bits_to_double(bias[n]) : 0.0f;
+            t = t + b;
+            y[m * N + n] = float_to_bf16_bits_rne(t);
+        }
+    return 0;
+}
+
+/* ----------------------------------------------------------------------- */
+/* Composite steps.                                                          */
+/* ----------------------------------------------------------------------- */
+
+/* Rotate, quantise and pack rows of a bf16 matrix: the per-row preparation
+ * shared by weights (offline) and activations (per call). */
+int oracle_prepare_rows(const uint16_t *x, int64_t rows, int64_t K, int n, uint8_t *packed,
+                        float *scale) {
+    if (!x || !packed || !scale || rows < 0 || K <= 0 || log4_exact(n) < 0 || K % n) return -1;
+    if (rows == 0) return 0;
+    double *y = (double *)malloc(sizeof(double) * (size_t)rows * (size_t)K);
+    int8_t *q = (int8_t *)malloc((size_t)rows * (size_t)K);
+    if (!y || !q) { free(y); free(q); return -2; }
+    int rc = oracle_rotate(x, rows, K, n, y);
+    if (!rc) rc = oracle_quantize_rows(y, rows, K, q, scale);
+    if (!rc) rc = oracle_pack(q, rows, K, packed);
+    free(y);
+    free(q);
+    return rc;
+}
+
+/* The whole layer on bf16 inputs: prepare x, take the prepared weights, run
+ * the integer product and the epilogue. */
+int oracle_linear_prepared_w(const uint16_t *x, const uint8_t *qw, const float *sw,
+                             const uint16_t *bias, int64_t M, int64_t N, int64_t K, int n,
+                             uint16_t *y) {
+    if (!x || !qw || !sw || !y || M < 0 || N < 0 || K <= 0) return -1;
+    if (M == 0 || N == 0) return 0;
+    uint8_t *qx = (uint8_t *)malloc((size_t)M * (size_t)(K / 2));
+    float *sx = (float *)malloc(sizeof(float) * (size_t)M);
+    int64_t *acc = (int64_t *)malloc(sizeof(int64_t) * (size_t)M * (size_t)N);
+    if (!qx || !sx || !acc) { free(qx); free(sx); free(acc); return -2; }
+    int rc = oracle_prepare_rows(x, M, K, n, qx, sx);
+    if (!rc) rc = oracle_gemm(qx, qw, M, N, K, acc);
+    if (!rc) rc = oracle_epilogue(acc, sx, sw, bias, M, N, y);
+    free(qx);
+    free(sx);
+    free(acc);
+    return rc;
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_num_threads(int t) {
+#ifdef _OPENMP
+    if (t > 0) omp_set_num_threads(t);
+#else
+    (void)t;
+#endif
+}

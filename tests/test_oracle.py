@@ -1,0 +1,390 @@
+"""Pins for the CPU oracle (no GPU).
+
+The oracle is trusted only after it agrees with things fixed independently of
+it: the pages' definitions written out as golden fixtures, closed forms
+(orthogonality, row sums, fixed points), an independent algorithm for the
+same operator (the Kronecker power applied digit by digit, numpy.kron),
+exhaustive search for the rounding rule, and brute force on tiny inputs.
+Each test names what a plausible mistake in the oracle would break.
+"""
+import itertools
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from rotated_w4a4_quantized_b200 import workloads as wl
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _load_matrix(name):
+    rows = []
+    for line in open(os.path.join(GOLD, name)):
+        line = line.split("#")[0].strip()
+        if line:
+            rows.append([float(t) for t in line.split()])
+    return np.array(rows)
+
+
+def _rand_bf16(shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    t = (torch.randn(*shape, generator=g) * scale).to(torch.bfloat16)
+    return wl.bf16_bits(t)
+
+
+# ---------------------------------------------------------------------------
+# H_n
+# ---------------------------------------------------------------------------
+
+def test_h4_matches_golden(oracle):
+    gold = _load_matrix("regular_hadamard_4.txt")
+    assert np.array_equal(oracle.hadamard(4), gold)
+    assert np.array_equal(oracle.hadamard_kron(4), gold)
+
+
+@pytest.mark.parametrize("n", [4, 16, 64, 256])
+def test_h_is_normalised_regular_hadamard(oracle, n):
+    H = oracle.hadamard(n)
+    # entries exactly +-1/sqrt(n) (a power of two here, so exact in fp64)
+    assert np.all(np.abs(H) == 1.0 / np.sqrt(n))
+    # symmetric and orthogonal: H H^T = I exactly (all products are exact)
+    assert np.array_equal(H, H.T)
+    assert np.array_equal(H @ H.T, np.eye(n))
+    # regular: constant row and column sums sqrt(n) before normalisation
+    U = np.rint(H * np.sqrt(n)).astype(np.int64)
+    assert np.all(U.sum(axis=1) == int(np.sqrt(n)))
+    assert np.all(U.sum(axis=0) == int(np.sqrt(n)))
+    assert np.array_equal(U @ U.T, n * np.eye(n, dtype=np.int64))
+
+
+@pytest.mark.parametrize("n", [16, 64, 256])
+def test_h_digit_rule_equals_kronecker_power(oracle, n):
+    # two builders inside the oracle and numpy.kron outside it must agree
+    T = (np.ones((4, 4)) - 2 * np.eye(4)) / 2
+    P = np.ones((1, 1))
+    while P.shape[0] < n:
+        P = np.kron(P, T)
+    assert np.array_equal(oracle.hadamard(n), P)
+    assert np.array_equal(oracle.hadamard_kron(n), P)
+
+
+def test_h4_equivalent_to_sylvester_up_to_signed_permutations(oracle):
+    # Comfy-Org/comfy-quants issue, section 2: H_reg = P H_sylv Q with P, Q
+    # signed permutations.  Brute force over all 384 x 384 pairs for n = 4.
+    R = np.rint(oracle.hadamard(4) * 2).astype(int)
+    S2 = np.array([[1, 1], [1, -1]])
+    S = np.kron(S2, S2)
+    signed_perms = []
+    for perm in itertools.permutations(range(4)):
+        for signs in itertools.product((1, -1), repeat=4):
+            M = np.zeros((4, 4), dtype=int)
+            for i, j in enumerate(perm):
+                M[i, j] = signs[i]
+            signed_perms.append(M)
+    target = {R.tobytes()}
+    found = False
+    for P in signed_perms:
+        PS = P @ S
+        for Q in signed_perms:
+            if (PS @ Q).tobytes() in target:
+                found = True
+                break
+        if found:
+            break
+    assert found
+
+
+# ---------------------------------------------------------------------------
+# Rotation
+# ---------------------------------------------------------------------------
+
+def _digitwise_rotate(x, n):
+    """x (rows, K) fp64 times I_G (x) H_n, applying (J-2I)/2 along each base-4
+    digit of the within-group index: an algorithm independent of the oracle's
+    dense mat-vec."""
+    rows, K = x.shape
+    k = int(round(np.log(n) / np.log(4)))
+    T = (np.ones((4, 4)) - 2 * np.eye(4)) / 2
+    t = x.reshape(rows, K // n, *([4] * k))
+    for ax in range(k):
+        t = np.moveaxis(np.tensordot(t, T, axes=([2 + ax], [0])), -1, 2 + ax)
+    return t.reshape(rows, K)
+
+
+@pytest.mark.parametrize("n", [4, 16, 64, 256])
+def test_rotation_equals_digitwise_transform(oracle, n):
+    x = _rand_bf16((5, 4 * n), seed=n)
+    y = oracle.rotate(x, n)
+    ref = _digitwise_rotate(oracle.bf16_to_f64(x), n)
+    assert np.allclose(y, ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("n", [64, 256])
+def test_rotation_preserves_norm_and_block_structure(oracle, n):
+    x = _rand_bf16((7, 3 * n), seed=11)
+    xd = oracle.bf16_to_f64(x)
+    y = oracle.rotate(x, n)
+    for g in range(3):
+        a = np.linalg.norm(xd[:, g * n:(g + 1) * n], axis=1)
+        b = np.linalg.norm(y[:, g * n:(g + 1) * n], axis=1)
+        assert np.allclose(a, b, rtol=1e-12, atol=0)
+    # one-hot input: reproduces one row of H inside its own group only
+    H = oracle.hadamard(n)
+    j, g = 5, 1
+    e = np.zeros((1, 3 * n), dtype=np.uint16)
+    e[0, g * n + j] = 0x3F80  # bf16 1.0
+    ye = oracle.rotate(e, n)
+    expect = np.zeros(3 * n)
+    expect[g * n:(g + 1) * n] = H[j]
+    assert np.array_equal(ye[0], expect)
+
+
+@pytest.mark.parametrize("n", [64, 256])
+def test_rotating_both_operands_preserves_the_product(oracle, n):
+    # Comfy-Org/comfy-quants issue, section 1: Y = sum_i RHT(X_i) RHT(W_i)^T
+    # equals X W^T because H is orthogonal.
+    X = _rand_bf16((6, 4 * n), seed=3)
+    W = _rand_bf16((9, 4 * n), seed=4, scale=0.02)
+    ref = oracle.bf16_to_f64(X) @ oracle.bf16_to_f64(W).T
+    RX, RW = oracle.rotate(X, n), oracle.rotate(W, n)
+    chunked = sum(RX[:, i * n:(i + 1) * n] @ RW[:, i * n:(i + 1) * n].T for i in range(4))
+    assert np.allclose(chunked, ref, rtol=0, atol=1e-12 * np.abs(ref).max())
+
+
+def test_all_ones_is_a_fixed_point(oracle):
+    x = np.full((1, 256), 0x3F80, dtype=np.uint16)
+    for n in (4, 16, 64, 256):
+        assert np.array_equal(oracle.rotate(x, n), np.ones((1, 256)))
+
+
+# ---------------------------------------------------------------------------
+# Quantisation
+# ---------------------------------------------------------------------------
+
+def _nearest_half_away_by_search(v):
+    """argmin_c |v - c| over c in [-7, 7]; on a tie the larger |c|."""
+    best = None
+    for c in range(-7, 8):
+        d = abs(float(v) - c)
+        if best is None or d < best[0] - 0.0 or (d == best[0] and abs(c) > abs(best[1])):
+            best = (d, c)
+    return best[1]
+
+
+def test_quantize_matches_exhaustive_search(oracle):
+    y = oracle.bf16_to_f64(_rand_bf16((4, 256), seed=5)) * 3.0
+    q, s = oracle.quantize_rows(y)
+    for r in range(y.shape[0]):
+        a = np.float32(np.abs(y[r]).max())
+        assert s[r] == np.float32(a / np.float32(7))
+        inv = np.float32(np.float32(7) / a)
+        for k in range(y.shape[1]):
+            v = np.float32(np.float32(y[r, k]) * inv)
+            assert q[r, k] == _nearest_half_away_by_search(v)
+        # the largest magnitude maps to +-7
+        kmax = int(np.argmax(np.abs(y[r])))
+        assert abs(int(q[r, kmax])) == 7
+    assert np.abs(q).max() <= 7
+
+
+def test_quantize_edge_rows(oracle):
+    # with absmax 7, inv = 1 exactly and v = y: exact .5 ties round away
+    # (the decision is taken on fp32(y): 3.4999999 would round to fp32 3.5,
+    # so the value just below 3.5 is the fp32 neighbour itself)
+    below = float(np.nextafter(np.float32(3.5), np.float32(0)))
+    ties = np.array([[7.0, 0.5, 1.5, 2.5, -0.5, -2.5, below, -6.5, 6.5, 0.0, -7.0, 0.49]])
+    q, s = oracle.quantize_rows(ties)
+    assert s[0] == np.float32(1.0)
+    assert q[0].tolist() == [7, 1, 2, 3, -1, -3, 3, -7, 7, 0, -7, 0]
+    q0, s0 = oracle.quantize_rows(np.zeros((2, 64)))
+    assert np.all(s0 == 0) and np.all(q0 == 0)
+    one = np.zeros((1, 64))
+    one[0, 17] = -0.003
+    q1, s1 = oracle.quantize_rows(one)
+    assert q1[0, 17] == -7 and np.count_nonzero(q1) == 1
+    flat = np.full((1, 64), 2.5)
+    qf, _ = oracle.quantize_rows(flat)
+    assert np.all(qf == 7)
+
+
+# ---------------------------------------------------------------------------
+# Packing
+# ---------------------------------------------------------------------------
+
+def test_pack_matches_golden_bytes(oracle):
+    rows = []
+    for line in open(os.path.join(GOLD, "nibble_pack.txt")):
+        line = line.split("#")[0].strip()
+        if line:
+            a, b, h = line.split()
+            rows.append((int(a), int(b), int(h, 16)))
+    q = np.array([[c for a, b, _ in rows for c in (a, b)]], dtype=np.int8)
+    p = oracle.pack(q)
+    assert p[0].tolist() == [h for _, _, h in rows]
+
+
+def test_pack_unpack_round_trip_all_pairs(oracle):
+    codes = [(a, b) for a in range(-7, 8) for b in range(-7, 8)]
+    q = np.array([[c for pair in codes for c in pair]], dtype=np.int8)
+    p = oracle.pack(q)
+    assert len(set(p[0].tolist())) == 225
+    assert np.array_equal(oracle.unpack(p, q.shape[1]), q)
+
+
+# ---------------------------------------------------------------------------
+# Integer GEMM and epilogue
+# ---------------------------------------------------------------------------
+
+def test_gemm_matches_numpy_int64(oracle):
+    rng = np.random.default_rng(0)
+    for (M, K, N) in [(4, 16, 16), (5, 64, 7), (3, 512, 9)]:
+        a = rng.integers(-7, 8, size=(M, K)).astype(np.int8)
+        b = rng.integers(-7, 8, size=(N, K)).astype(np.int8)
+        acc = oracle.gemm(oracle.pack(a), oracle.pack(b), K)
+        assert np.array_equal(acc, a.astype(np.int64) @ b.astype(np.int64).T)
+
+
+def test_gemm_saturation(oracle):
+    K = 12288
+    a = np.full((2, K), 7, dtype=np.int8)
+    a[1] = -7
+    b = np.full((3, K), 7, dtype=np.int8)
+    acc = oracle.gemm(oracle.pack(a), oracle.pack(b), K)
+    assert np.all(acc[0] == 49 * K) and np.all(acc[1] == -49 * K)
+    assert 49 * K < 2 ** 31
+
+
+def _bf16_to_f64_np(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def test_epilogue_exact_values_and_one_ulp(oracle):
+    acc = np.array([[3, -12544, 0, 1 << 20]], dtype=np.int64)
+    sx = np.array([0.5], dtype=np.float32)
+    sw = np.array([0.25, 1.0 / 49.0, 0.125, 2.0 ** -20], dtype=np.float32)
+    bias = np.array([0x3F80, 0x0000, 0xBF00, 0x0000], dtype=np.uint16)  # 1, 0, -0.5, 0
+    y = oracle.epilogue(acc, sx, sw, bias)
+    # 3*0.5*0.25 + 1 = 1.375 exactly -> 0x3FB0; 0*... - 0.5 -> 0xBF00;
+    # 2^20 * 0.5 * 2^-20 = 0.5 -> 0x3F00
+    assert y[0, 0] == 0x3FB0 and y[0, 2] == 0xBF00 and y[0, 3] == 0x3F00
+    # a second evaluation in fp64 rounded once agrees within one bf16 ulp
+    rng = np.random.default_rng(1)
+    acc = rng.integers(-600000, 600000, size=(16, 32)).astype(np.int64)
+    sx = rng.uniform(1e-3, 1.0, size=16).astype(np.float32)
+    sw = rng.uniform(1e-5, 1e-2, size=32).astype(np.float32)
+    bias = wl.bf16_bits(torch.randn(32, generator=torch.Generator().manual_seed(2)).to(torch.bfloat16))
+    y = _bf16_to_f64_np(oracle.epilogue(acc, sx, sw, bias))
+    ref = acc * sx.astype(np.float64)[:, None] * sw.astype(np.float64)[None, :] + _bf16_to_f64_np(bias)
+    ulp = 2.0 ** (np.floor(np.log2(np.abs(ref))) - 7)
+    assert np.all(np.abs(y - ref) <= ulp)
+
+
+def test_epilogue_null_bias_is_zero_bias(oracle):
+    acc = np.arange(12, dtype=np.int64).reshape(3, 4) - 5
+    sx = np.array([0.1, 0.2, 0.3], dtype=np.float32)
+    sw = np.array([1.0, 2.0, 3.0, 4.0], dtype=np.float32)
+    assert np.array_equal(oracle.epilogue(acc, sx, sw, None),
+                          oracle.epilogue(acc, sx, sw, np.zeros(4, dtype=np.uint16)))
+
+
+# ---------------------------------------------------------------------------
+# Whole layer
+# ---------------------------------------------------------------------------
+
+def _brute_force_layer(x_bits, w_bits, b_bits, n):
+    """Everything again from scratch in numpy for tiny shapes: numpy.kron for
+    H, float32 decisions, codes, int64 dot, float32 epilogue."""
+    T = (np.ones((4, 4)) - 2 * np.eye(4)) / 2
+    H = np.ones((1, 1))
+    while H.shape[0] < n:
+        H = np.kron(H, T)
+    R = np.kron(np.eye(x_bits.shape[1] // n), H)
+
+    def prep(bits):
+        y = _bf16_to_f64_np(bits) @ R
+        codes, scales = [], []
+        for row in y:
+            a = np.float32(np.abs(row).max())
+            if a == 0:
+                codes.append(np.zeros(len(row), dtype=np.int64))
+                scales.append(np.float32(0))
+                continue
+            inv = np.float32(np.float32(7) / a)
+            v = (row.astype(np.float32) * inv).astype(np.float32)
+            c = np.array([_nearest_half_away_by_search(t) for t in v])
+            codes.append(c)
+            scales.append(np.float32(a / np.float32(7)))
+        return np.array(codes), np.array(scales, dtype=np.float32)
+
+    qx, sx = prep(x_bits)
+    qw, sw = prep(w_bits)
+    acc = qx @ qw.T
+    t = acc.astype(np.float32) * sx[:, None]
+    t = t.astype(np.float32) * sw[None, :]
+    t = t.astype(np.float32) + _bf16_to_f64_np(b_bits).astype(np.float32)[None, :]
+    return t.astype(np.float32), qx, sx, qw, sw
+
+
+@pytest.mark.parametrize("n", [4, 16])
+def test_layer_brute_force_tiny(oracle, n):
+    x = _rand_bf16((4, 16), seed=20 + n)
+    w = _rand_bf16((16, 16), seed=30 + n, scale=0.02)
+    b = _rand_bf16((16,), seed=40 + n, scale=0.02)
+    t, qx, sx, qw, sw = _brute_force_layer(x, w, b, n)
+    px, ox = oracle.prepare_rows(x, n)
+    pw, ow = oracle.prepare_rows(w, n)
+    assert np.array_equal(oracle.unpack(px, 16), qx) and np.array_equal(ox, sx)
+    assert np.array_equal(oracle.unpack(pw, 16), qw) and np.array_equal(ow, sw)
+    y = oracle.linear_prepared_w(x, pw, ow, b, n)
+    assert np.array_equal(y, oracle.f32_to_bf16(t))
+
+
+def test_worked_examples(oracle):
+    for line in open(os.path.join(GOLD, "worked_examples.txt")):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        name, K, n, acc, ybits = line.split()
+        K, n, acc, ybits = int(K), int(n), int(acc), int(ybits, 16)
+        if name == "onehot":
+            x = np.zeros((1, K), dtype=np.uint16)
+            x[0, 0] = 0x3F80
+            w = x.copy()
+            b = None
+        else:
+            x = np.full((1, K), 0x3F80, dtype=np.uint16)
+            w = x.copy()
+            b = np.array([0xBF00 if name == "ones_bias" else 0], dtype=np.uint16)
+        px, sx = oracle.prepare_rows(x, n)
+        pw, sw = oracle.prepare_rows(w, n)
+        assert oracle.gemm(px, pw, K)[0, 0] == acc, name
+        assert oracle.linear_prepared_w(x, pw, sw, b, n)[0, 0] == ybits, name
+
+
+def test_rotation_reduces_outlier_error(oracle):
+    # Rotation spreads channel outliers over each group before the rowwise
+    # quantiser sees them; with identity rotation (group 1 is not allowed, so
+    # compare against quantising the unrotated rows directly) the error is
+    # larger.  Scaled-down version of the outlier workload.
+    lt = wl.make_random_layer(32, 512, 48, 64, seed=9, bias=False)
+    x = lt.x.float()
+    ch = torch.randperm(512, generator=torch.Generator().manual_seed(1))[:5]
+    x[:, ch] *= 50
+    xb = wl.bf16_bits(x.to(torch.bfloat16))
+    wb = wl.bf16_bits(lt.w)
+    dense = _bf16_to_f64_np(xb) @ _bf16_to_f64_np(wb).T
+
+    def err(group):
+        pw, sw = oracle.prepare_rows(wb, group)
+        y = _bf16_to_f64_np(oracle.linear_prepared_w(xb, pw, sw, None, group))
+        return np.linalg.norm(y - dense) / np.linalg.norm(dense)
+
+    qx, sx = oracle.quantize_rows(_bf16_to_f64_np(xb))
+    qw, sw = oracle.quantize_rows(_bf16_to_f64_np(wb))
+    acc = qx.astype(np.int64) @ qw.astype(np.int64).T
+    plain = acc * sx.astype(np.float64)[:, None] * sw.astype(np.float64)[None, :]
+    e_plain = np.linalg.norm(plain - dense) / np.linalg.norm(dense)
+    assert err(64) < e_plain
+    assert err(256) < e_plain
