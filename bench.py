@@ -1,0 +1,443 @@
+"""Benchmark of the rotated W4A4 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step is one pass of the whole path over one batch: the fused prep kernel
+(rotation, rowwise absmax INT4 quantisation, packing) and the tcgen05 GEMM
+with its scale/bias/bf16 epilogue (two kernels per linear layer).  Weights are
+prepared once before timing (the offline step).  The L2 cache is flushed
+(a 256 MiB write) before every timed step, outside the timed interval; each
+step is bracketed by CUDA events on the launching stream.  Under torchrun
+every rank runs its own batch (weak scaling, no collective on the data path);
+the reported time is the maximum over ranks.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
+instead, on bounded samples of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from rotated_w4a4_quantized_b200 import workloads as wl  # noqa: E402
+
+METRIC = "W4A4 linear end-to-end TOPS and % of INT8 tensor peak; prep kernel HBM GB/s"
+L2_FLUSH_BYTES = 256 << 20
+# Bytes a prep launch must move per row: 2K read (bf16), K/2 + 4 written.
+PREP_BYTES_PER_ROW = lambda K: 2 * K + K // 2 + 4  # noqa: E731
+INT8_PER_BF16 = 2.0   # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm": float(p["hbm_gbs"]), "bf16": float(p["bf16_tflops"]),
+                "bf16_sustained": float(p["bf16_tflops_sustained"]), "src": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "src": "fallback"}
+
+
+def _src_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "rotated_w4a4_quantized_b200", "csrc")
+    for name in sorted(os.listdir(d)):
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(workload, kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("src_hash") != _src_hash():
+        return None
+    return t.get("per_launch_bytes", {}).get(workload, {}).get(kernel)
+
+
+class ClockSampler:
+    """nvidia-smi samples of one GPU while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: str):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 6:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[2:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def aggregate(local_ms: float, local_ops: float, device=None):
+    """(max time over ranks, total ops over ranks); control plane only."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return local_ms, local_ops
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    o = torch.tensor([local_ops], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(o, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(o.item())
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+
+def run_gpu(args):
+    import torch.distributed as dist
+
+    import rotated_w4a4_quantized_b200 as cr
+    from rotated_w4a4_quantized_b200 import build
+    build.build()
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    name = args.workload
+    spec = wl.WORKLOADS[name]
+    layers = wl.make_workload(name, seed=spec.seed + rank)
+    stream = torch.cuda.current_stream()
+
+    # offline step: prepare the weights once
+    prepared = []
+    for lt in layers:
+        w = lt.w.to(dev)
+        qw, sw = cr.convrot_quantize_weight(w, lt.spec.group)
+        b = None if lt.b is None else lt.b.to(dev)
+        del w
+        prepared.append((lt.spec, qw, sw, b))
+    x0 = layers[0].x.to(dev)
+    acts, ws = [], []
+    for i, (sp, qw, sw, b) in enumerate(prepared):
+        acts.append(x0 if i == 0 else torch.empty(sp.M, sp.K, dtype=torch.bfloat16, device=dev))
+        ws.append((torch.empty(sp.M, sp.K // 2, dtype=torch.uint8, device=dev),
+                   torch.empty(sp.M, dtype=torch.float32, device=dev)))
+    outs = [torch.empty(sp.M, sp.N, dtype=torch.bfloat16, device=dev) for sp, *_ in prepared]
+    for i in range(1, len(prepared)):
+        acts[i] = outs[i - 1]          # chained layers: next input is this output
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    nl = len(prepared)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nl + 1)] for _ in range(args.steps)]
+
+    def step(events=None):
+        for i, (sp, qw, sw, b) in enumerate(prepared):
+            if events is not None:
+                events[2 * i].record(stream)
+            cr.convrot_prepare_act(acts[i], sp.group, ws[i][0], ws[i][1])
+            if events is not None:
+                events[2 * i + 1].record(stream)
+            cr.convrot_linear_prepared(ws[i][0], ws[i][1], qw, sw, b, sp.K, out=outs[i])
+        if events is not None:
+            events[2 * nl].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if cr.convrot_check_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = str(local)
+    with ClockSampler(gpu_id) as clocks:
+        for k in range(args.steps):
+            flush.zero_()
+            step(ev[k])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    status = cr.convrot_check_device_error()
+    if status != 0:
+        raise RuntimeError(f"device error status {status} in the timed region")
+
+    step_ms = [e[0].elapsed_time(e[-1]) for e in ev]
+    prep_ms = [[e[2 * i].elapsed_time(e[2 * i + 1]) for e in ev] for i in range(nl)]
+    gemm_ms = [[e[2 * i + 1].elapsed_time(e[2 * i + 2]) for e in ev] for i in range(nl)]
+    local_ms = sum(step_ms)
+    ops_step = spec.ops
+    t_max, ops_total = aggregate(local_ms, ops_step * args.steps, dev)
+    value = ops_total / (t_max * 1e-3) / 1e12                      # TOPS, whole job
+    tokens_s = spec.tokens * world * args.steps / (t_max * 1e-3)
+
+    peaks = _peaks()
+    int8_peak = peaks["bf16"] * INT8_PER_BF16
+    gemm_avg = [statistics.fmean(g) for g in gemm_ms]
+    prep_avg = [statistics.fmean(p) for p in prep_ms]
+    gemm_tops = [2 * sp.M * sp.N * sp.K / (g * 1e-3) / 1e12 for (sp, *_), g in zip(prepared, gemm_avg)]
+    prep_gbs = [sp.M * PREP_BYTES_PER_ROW(sp.K) / (p * 1e-3) / 1e9 for (sp, *_), p in zip(prepared, prep_avg)]
+    gemm_total, prep_total = sum(map(sum, gemm_ms)), sum(map(sum, prep_ms))
+    if gemm_total >= prep_total:
+        i = max(range(nl), key=lambda j: sum(gemm_ms[j]))
+        sp = prepared[i][0]
+        roof = {"kernel": "gemm_kernel", "bound": "tensor", "achieved": round(gemm_tops[i], 2),
+                "peak": round(int8_peak, 1), "unit": "TFLOP/s",
+                "frac": round(gemm_tops[i] / int8_peak, 4),
+                "traffic": _traffic(name, "gemm_kernel"),
+                "note": "integer tensor ops (2 per multiply-add); peak = measured bf16 burst "
+                        f"x {INT8_PER_BF16} nominal int8/bf16 ratio ({peaks['src']})"}
+    else:
+        i = max(range(nl), key=lambda j: sum(prep_ms[j]))
+        roof = {"kernel": "prep_kernel", "bound": "hbm", "achieved": round(prep_gbs[i], 1),
+                "peak": peaks["hbm"], "unit": "GB/s", "frac": round(prep_gbs[i] / peaks["hbm"], 4),
+                "traffic": _traffic(name, "prep_kernel"),
+                "note": f"HBM peak {peaks['src']}"}
+
+    # end to end through the public call, host buffers, copies inside the interval
+    e2e = run_e2e(cr, prepared, spec, dev, stream, flush, args)
+    t_e2e, ops_e2e = aggregate(e2e["ms"], ops_step * e2e["steps"], dev)
+
+    launches = 2 * nl * args.steps
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "s8",
+        "data": "synthetic (seeded bf16, shapes and distributions of the workload; no weights)",
+        "config": {"workload": name, "layers": [f"{l.M}x{l.K}->{l.N} g{l.group}" for l in spec.layers],
+                   "tokens_per_rank": spec.tokens, "l2": "flushed (256 MiB write) before each step",
+                   "parallelism": f"dp{world}"},
+        "tokens_per_s": round(tokens_s, 1),
+        "int8_peak_frac_path": round(value / world / int8_peak, 4),
+        "gemm_tops": [round(v, 2) for v in gemm_tops],
+        "prep_gbs": [round(v, 1) for v in prep_gbs],
+        "prep_hbm_frac": [round(v / peaks["hbm"], 4) for v in prep_gbs],
+        "roofline": roof,
+        "e2e": {"value": round(ops_e2e / (t_e2e * 1e-3) / 1e12, 3), "unit": "TOPS",
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0:
+        line["cpu_baseline"] = cpu_baseline(name, args.cpu_seconds) if world == 1 and not args.no_cpu else None
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(cr, prepared, spec, dev, stream, flush, args):
+    """The public call on pinned host buffers: H2D of x, convrot_linear per
+    layer, D2H of y, all inside the event interval."""
+    sp0 = prepared[0][0]
+    x_host = wl.make_workload(args.workload)[0].x.pin_memory()
+    y_host = torch.empty(prepared[-1][0].M, prepared[-1][0].N, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x_host, device=dev)
+    wss = [torch.empty(max(1, cr.convrot_linear_workspace_size(sp.M, sp.K)), dtype=torch.uint8,
+                       device=dev) for sp, *_ in prepared]
+    outs = [torch.empty(sp.M, sp.N, dtype=torch.bfloat16, device=dev) for sp, *_ in prepared]
+    steps = max(3, min(args.steps, 200))
+
+    def one():
+        x_dev.copy_(x_host, non_blocking=True)
+        inp = x_dev
+        for i, (sp, qw, sw, b) in enumerate(prepared):
+            cr.convrot_linear(inp, qw, sw, b, sp.group, wss[i], outs[i])
+            inp = outs[i]
+        y_host.copy_(outs[-1], non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    total = 0.0
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        one()
+        b.record(stream)
+        b.synchronize()
+        total += a.elapsed_time(b)
+    return {"ms": total, "steps": steps, "h2d": sp0.M * sp0.K * 2,
+            "d2h": prepared[-1][0].M * prepared[-1][0].N * 2}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle as a timed baseline
+# ---------------------------------------------------------------------------
+
+class OracleSampler:
+    """The oracle's per-call work on a sample of token rows: prepare those
+    activation rows, integer GEMM against the prepared weights, epilogue.
+    Weight preparation is offline (done once here, untimed), as on the GPU."""
+
+    def __init__(self, name):
+        import oracle as O
+        O.build()
+        self.O = O
+        self.spec = wl.WORKLOADS[name]
+        l0 = wl.make_workload(name)[0]
+        self.sp = l0.spec
+        self.pw, self.sw = O.prepare_rows(wl.bf16_bits(l0.w), self.sp.group)
+        self.bb = None if l0.b is None else wl.bf16_bits(l0.b)
+        self.xb = wl.bf16_bits(l0.x)
+        self.cores = O.num_threads()
+        self.layer = f"{self.sp.M}x{self.sp.K}->{self.sp.N} g{self.sp.group}"
+
+    def run(self, rows):
+        O, sp = self.O, self.sp
+        t0 = time.perf_counter()
+        px, sx = O.prepare_rows(self.xb[:rows], sp.group)
+        O.epilogue(O.gemm(px, self.pw, sp.K), sx, self.sw, self.bb)
+        return time.perf_counter() - t0
+
+    def calibrate(self, seconds):
+        """Rows such that one run takes about `seconds` (at least 1 row)."""
+        rows, t = 1, self.run(1)
+        while t < seconds / 8 and rows < self.sp.M:
+            rows = min(self.sp.M, rows * 4)
+            t = self.run(rows)
+        if t < seconds and rows < self.sp.M:
+            rows = min(self.sp.M, max(rows, int(rows * seconds / max(t, 1e-6))))
+        return rows
+
+    def ops(self, rows):
+        return 2 * rows * self.sp.N * self.sp.K
+
+
+def cpu_baseline(name, seconds):
+    s = OracleSampler(name)
+    rows = s.calibrate(seconds)
+    t = s.run(rows)
+    return {"value": round(s.ops(rows) / t / 1e12, 9), "unit": "TOPS", "cores": s.cores,
+            "kind": "oracle",
+            "sample": f"{rows} of {s.sp.M} token rows of layer {s.layer} (prep + int64 GEMM + "
+                      f"epilogue, weights prepared offline), {t:.1f} s"}
+
+
+def run_reference(args):
+    world, rank, _ = _dist()
+    if rank != 0:
+        return
+    name = args.workload
+    s = OracleSampler(name)
+    # the whole run (warm-up + steps) stays within about --cpu-seconds x 8
+    per_step = args.cpu_seconds * 8 / (args.steps + args.warmup)
+    rows = s.calibrate(per_step)
+    total = 0.0
+    for k in range(args.warmup + args.steps):
+        t = s.run(rows)
+        if k >= args.warmup:
+            total += t
+    value = s.ops(rows) * args.steps / total / 1e12
+    spec = wl.WORKLOADS[name]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 9), "unit": "TOPS",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "s8",
+        "data": "synthetic (seeded bf16, same workload)",
+        "config": {"workload": name, "layers": [f"{l.M}x{l.K}->{l.N} g{l.group}" for l in spec.layers],
+                   "tokens_per_rank": spec.tokens, "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(value, 9), "unit": "TOPS", "cores": s.cores, "kind": "oracle",
+                         "sample": f"each step: {rows} of {s.sp.M} token rows of layer {s.layer} "
+                                   "(prep + int64 GEMM + epilogue, weights prepared offline)"},
+        "e2e": {"value": round(value, 9), "unit": "TOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=wl.DEFAULT_BENCH, choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU time budget of the oracle baseline")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,145 @@
+/*
+ * convrot.h -- C ABI of the B200 (sm_100a) rotated W4A4 linear layer.
+ *
+ * The layer (pages: "convrot-mlx" README, "What is included" and "Install and
+ * test"; Comfy-Org/comfy-quants issue "convrot is exactly same as or a wrapper
+ * around QuaRot Stage 1c", sections 1 and 2):
+ *
+ *   1. every K-group of n in {64, 256} channels of a bf16 row is multiplied by
+ *      the normalised regular Hadamard matrix H_n = (J - 2I)^{(x)log4 n}/sqrt(n),
+ *      i.e. the row is multiplied by the block-diagonal R = I_G (x) H_n;
+ *   2. the rotated row is quantised with ONE symmetric absmax scale per row to
+ *      signed INT4 codes in [-7, 7]:
+ *          a = max|y|,  s = a / 7,  q = round_half_away(y * (7 / a))   (fp32)
+ *      (a == 0 gives s = 0 and all codes 0), and packed two codes per byte,
+ *      low nibble = even channel, 4-bit two's complement;
+ *   3. activations and offline-prepared weights are multiplied with exact
+ *      integer accumulation, acc[m][n] = sum_k qx[m][k] qw[n][k], and
+ *   4. the epilogue writes y[m][n] = bf16_rne((float(acc) * sx[m]) * sw[n] + b[n])
+ *      evaluated in fp32 in that order.
+ *
+ * Conventions for every entry point:
+ *   - All pointers are DEVICE pointers on the current CUDA device unless stated
+ *     otherwise, row-major and contiguous, 16-byte aligned (CONVROT_ERR_ALIGN
+ *     otherwise).  bf16 tensors are passed as const void* to raw bf16 data.
+ *   - Ownership stays with the caller: the library allocates nothing, frees
+ *     nothing, never synchronises and never changes the current device.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default).
+ *   - Arguments are validated before anything is launched: a non-OK status
+ *     means nothing was enqueued, except CONVROT_ERR_CUDA (a launch failed).
+ *   - Shapes: M, N >= 1 (M = 0 or N = 0 is a no-op returning OK), K a
+ *     multiple of `group`, 64 <= K <= CONVROT_MAX_K; group is 64 or 256.
+ *   - Results are deterministic: identical inputs give identical bytes.
+ *   - Device-side waits are bounded; a wait that runs out records
+ *     CONVROT_ERR_DEVICE_TIMEOUT, which convrot_check_device_error reports.
+ */
+#ifndef CONVROT_H_
+#define CONVROT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                        /* the CUDA runtime's stream type */
+typedef struct CUstream_st *convrot_stream_t;  /* same object as cudaStream_t */
+
+#define CONVROT_MAX_K 32768
+
+typedef enum {
+    CONVROT_OK = 0,
+    CONVROT_ERR_NULL = 1,            /* a required pointer is NULL */
+    CONVROT_ERR_GROUP = 2,           /* group is not 64 or 256 */
+    CONVROT_ERR_SHAPE = 3,           /* negative dim, K % group, K out of range */
+    CONVROT_ERR_ALIGN = 4,           /* a pointer is not 16-byte aligned */
+    CONVROT_ERR_WORKSPACE = 5,       /* workspace smaller than required */
+    CONVROT_ERR_CUDA = 6,            /* a CUDA runtime call or launch failed */
+    CONVROT_ERR_DEVICE_TIMEOUT = 7,  /* a bounded device wait ran out */
+    CONVROT_ERR_UNSUPPORTED = 8      /* device is not sm_100 */
+} convrot_status;
+
+/* Human-readable name of a status (static storage, never NULL). */
+const char *convrot_status_string(convrot_status s);
+
+/*
+ * Steps 1-2 on weights (offline).  w_bf16: [N][K] bf16.  Writes qw: [N][K/2]
+ * bytes (packed codes) and sw: [N] fp32 scales.  Source: "convrot-mlx"
+ * README, "Install and test" (quantize_convrot_weight -> qweight, scales).
+ */
+convrot_status convrot_quantize_weight(const void *w_bf16, int64_t N, int64_t K, int group,
+                                       uint8_t *qw, float *sw, convrot_stream_t stream);
+
+/*
+ * Steps 1-2 on activations: the fused prep kernel (one CTA per row).
+ * x_bf16: [M][K] bf16.  Writes qx: [M][K/2] bytes and sx: [M] fp32.
+ * Source: "convrot-mlx" README, "What is included" (fused activation prep).
+ */
+convrot_status convrot_prepare_act(const void *x_bf16, int64_t M, int64_t K, int group,
+                                   uint8_t *qx, float *sx, convrot_stream_t stream);
+
+/* Bytes of workspace convrot_linear needs: packed codes and scales of x,
+ * each region rounded up to 256 bytes. */
+size_t convrot_linear_workspace_size(int64_t M, int64_t K);
+
+/*
+ * Steps 1-4, the whole layer: prep kernel into `workspace`, then the
+ * tcgen05 INT GEMM with the fused scale/bias/bf16 epilogue.
+ * x_bf16 [M][K] bf16; qw [N][K/2] and sw [N] from convrot_quantize_weight
+ * with the same group; bias_bf16 [N] bf16 or NULL (zeros); y_bf16 [M][N].
+ * workspace: ws_bytes >= convrot_linear_workspace_size(M, K), 256-byte
+ * aligned.  Source: "convrot-mlx" README, "Install and test" (the complete
+ * path is rotation, activation quantisation, the integer product, scaling
+ * and bias).
+ */
+convrot_status convrot_linear(const void *x_bf16, const uint8_t *qw, const float *sw,
+                              const void *bias_bf16, int64_t M, int64_t N, int64_t K, int group,
+                              void *workspace, size_t ws_bytes, void *y_bf16,
+                              convrot_stream_t stream);
+
+/*
+ * Steps 3-4 only, on prepared operands: qx [M][K/2], sx [M], qw [N][K/2],
+ * sw [N], bias [N] bf16 or NULL, y [M][N] bf16.  K is the unpacked length
+ * (a multiple of 64).
+ */
+convrot_status convrot_linear_prepared(const uint8_t *qx, const float *sx, const uint8_t *qw,
+                                       const float *sw, const void *bias_bf16, int64_t M,
+                                       int64_t N, int64_t K, void *y_bf16,
+                                       convrot_stream_t stream);
+
+/*
+ * Test hook: step 1 alone, through the same prep kernel.  Writes the
+ * normalised rotated rows y_rot [M][K] as fp32.
+ */
+convrot_status convrot_debug_rotate_f32(const void *x_bf16, int64_t M, int64_t K, int group,
+                                        float *y_rot, convrot_stream_t stream);
+
+/*
+ * Test hook: step 3 alone, through the same GEMM kernel.  Writes the exact
+ * integer accumulators acc [M][N] as int32 (|acc| <= 49 K always fits).
+ */
+convrot_status convrot_debug_gemm_s32(const uint8_t *qx, const uint8_t *qw, int64_t M, int64_t N,
+                                      int64_t K, int32_t *acc, convrot_stream_t stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device error word of the
+ * current device: CONVROT_ERR_DEVICE_TIMEOUT if a bounded wait in any kernel
+ * of this library ran out since the last check, CONVROT_ERR_CUDA if the
+ * synchronisation itself failed, CONVROT_OK otherwise.
+ */
+convrot_status convrot_check_device_error(convrot_stream_t stream);
+
+/*
+ * Test hook for the timeout path: launches one CTA that waits on a
+ * shared-memory barrier nothing ever signals, giving up after timeout_ns
+ * nanoseconds (clamped to [1e3, 5e9]); it then records
+ * CONVROT_ERR_DEVICE_TIMEOUT in the device error word and returns normally.
+ */
+convrot_status convrot_debug_timeout_probe(int64_t timeout_ns, convrot_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CONVROT_H_ */

@@ -170,8 +170,12 @@ int oracle_hadamard_kron(int n, double *H) {
 int oracle_rotate(const uint16_t *x, int64_t rows, int64_t K, int n, double *y) {
     if (!x || !y || rows < 0 || K <= 0 || log4_exact(n) < 0 || K % n) return -1;
     double *H = (double *)malloc(sizeof(double) * (size_t)n * n);
-    if (!H) return -2;
+    double *Ht = (double *)malloc(sizeof(double) * (size_t)n * n);
+    if (!H || !Ht) { free(H); free(Ht); return -2; }
     oracle_hadamard(n, H);
+    /* Ht[i][j] = H[j][i]: the same products in the same order, read row-wise */
+    for (int i = 0; i < n; ++i)
+        for (int j = 0; j < n; ++j) Ht[(int64_t)i * n + j] = H[(int64_t)j * n + i];
     int64_t G = K / n;
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t r = 0; r < rows; ++r) {
@@ -182,13 +186,14 @@ int oracle_rotate(const uint16_t *x, int64_t rows, int64_t K, int n, double *y) 
             double *dst = y + r * K + g * n;
             for (int i = 0; i < n; ++i) {
                 double acc = 0.0;
-                for (int j = 0; j < n; ++j) acc += xg[j] * H[(int64_t)j * n + i];
+                for (int j = 0; j < n; ++j) acc += xg[j] * Ht[(int64_t)i * n + j];
                 dst[i] = acc;
             }
         }
         free(xg);
     }
     free(H);
+    free(Ht);
     return 0;
 }
 
@@ -277,20 +282,21 @@ int oracle_unpack(const uint8_t *p, int64_t rows, int64_t K, int8_t *q) {
 int oracle_gemm(const uint8_t *qx, const uint8_t *qw, int64_t M, int64_t N, int64_t K,
                 int64_t *acc) {
     if (!qx || !qw || !acc || M < 0 || N < 0 || K <= 0 || K % 2) return -1;
+    int8_t *a = (int8_t *)malloc((size_t)M * (size_t)K + 1);
+    int8_t *b = (int8_t *)malloc((size_t)N * (size_t)K + 1);
+    if (!a || !b) { free(a); free(b); return -2; }
+    oracle_unpack(qx, M, K, a);
+    oracle_unpack(qw, N, K, b);
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t m = 0; m < M; ++m) {
-        int8_t *a = (int8_t *)malloc((size_t)K);
-        int8_t *b = (int8_t *)malloc((size_t)K);
-        oracle_unpack(qx + m * (K / 2), 1, K, a);
         for (int64_t n = 0; n < N; ++n) {
-            oracle_unpack(qw + n * (K / 2), 1, K, b);
             int64_t s = 0;
-            for (int64_t k = 0; k < K; ++k) s += (int64_t)a[k] * (int64_t)b[k];
+            for (int64_t k = 0; k < K; ++k) s += (int64_t)a[m * K + k] * (int64_t)b[n * K + k];
             acc[m * N + n] = s;
         }
-        free(a);
-        free(b);
     }
+    free(a);
+    free(b);
     return 0;
 }
 

@@ -1,0 +1,199 @@
+"""B200-native rotated W4A4 (ConvRot-style) linear layer.
+
+A thin ctypes binding over the C ABI in ``include/convrot.h`` (the library
+``libconvrot.so`` built in this directory by ``build.py``).  Every step of the
+layer runs in that library's CUDA kernels; this module only marshals torch
+tensors (device memory and the current stream) into pointers and sizes and
+turns status codes into exceptions.  There is no CPU fallback: if the
+library is missing, importing the ops raises.
+
+Names follow the C ABI: ``convrot_quantize_weight``, ``convrot_prepare_act``,
+``convrot_linear``, ``convrot_linear_prepared`` (plus the test hooks).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libconvrot.so")
+
+STATUS = {
+    0: "CONVROT_OK", 1: "CONVROT_ERR_NULL", 2: "CONVROT_ERR_GROUP", 3: "CONVROT_ERR_SHAPE",
+    4: "CONVROT_ERR_ALIGN", 5: "CONVROT_ERR_WORKSPACE", 6: "CONVROT_ERR_CUDA",
+    7: "CONVROT_ERR_DEVICE_TIMEOUT", 8: "CONVROT_ERR_UNSUPPORTED",
+}
+MAX_K = 32768
+
+
+class ConvRotError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m rotated_w4a4_quantized_b200.build` "
+                "(there is no fallback path)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, I, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        sigs = {
+            "convrot_quantize_weight": [P, I64, I64, I, P, P, P],
+            "convrot_prepare_act": [P, I64, I64, I, P, P, P],
+            "convrot_linear": [P, P, P, P, I64, I64, I64, I, P, SZ, P, P],
+            "convrot_linear_prepared": [P, P, P, P, P, I64, I64, I64, P, P],
+            "convrot_debug_rotate_f32": [P, I64, I64, I, P, P],
+            "convrot_debug_gemm_s32": [P, P, I64, I64, I64, P, P],
+            "convrot_check_device_error": [P],
+            "convrot_debug_timeout_probe": [I64, P],
+        }
+        for name, args in sigs.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ctypes.c_int
+        L.convrot_linear_workspace_size.argtypes = [I64, I64]
+        L.convrot_linear_workspace_size.restype = SZ
+        L.convrot_status_string.argtypes = [I]
+        L.convrot_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _p(t: torch.Tensor | None):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise ConvRotError(rc, what)
+
+
+def _need(t: torch.Tensor, dtype, name: str):
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+
+
+# ---------------------------------------------------------------------------
+# the C ABI, one wrapper each
+# ---------------------------------------------------------------------------
+
+def convrot_quantize_weight(w: torch.Tensor, group: int, qw=None, sw=None, stream=None):
+    """bf16 [N, K] -> (packed codes uint8 [N, K/2], fp32 scales [N])."""
+    _need(w, torch.bfloat16, "w")
+    N, K = w.shape
+    qw = torch.empty(N, K // 2, dtype=torch.uint8, device=w.device) if qw is None else qw
+    sw = torch.empty(N, dtype=torch.float32, device=w.device) if sw is None else sw
+    _check(lib().convrot_quantize_weight(_p(w), N, K, group, _p(qw), _p(sw), _stream(stream)),
+           "convrot_quantize_weight")
+    return qw, sw
+
+
+def convrot_prepare_act(x: torch.Tensor, group: int, qx=None, sx=None, stream=None):
+    """bf16 [M, K] -> (packed codes uint8 [M, K/2], fp32 scales [M])."""
+    _need(x, torch.bfloat16, "x")
+    M, K = x.shape
+    qx = torch.empty(M, K // 2, dtype=torch.uint8, device=x.device) if qx is None else qx
+    sx = torch.empty(M, dtype=torch.float32, device=x.device) if sx is None else sx
+    _check(lib().convrot_prepare_act(_p(x), M, K, group, _p(qx), _p(sx), _stream(stream)),
+           "convrot_prepare_act")
+    return qx, sx
+
+
+def convrot_linear_workspace_size(M: int, K: int) -> int:
+    return int(lib().convrot_linear_workspace_size(M, K))
+
+
+def convrot_linear(x, qw, sw, bias, group: int, workspace=None, out=None, stream=None):
+    """The whole layer: bf16 x [M, K] -> bf16 y [M, N]."""
+    _need(x, torch.bfloat16, "x")
+    M, K = x.shape
+    N = qw.shape[0]
+    if workspace is None:
+        workspace = torch.empty(max(1, convrot_linear_workspace_size(M, K)), dtype=torch.uint8,
+                                device=x.device)
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
+    _check(lib().convrot_linear(_p(x), _p(qw), _p(sw), _p(bias), M, N, K, group, _p(workspace),
+                                workspace.numel(), _p(out), _stream(stream)), "convrot_linear")
+    return out
+
+
+def convrot_linear_prepared(qx, sx, qw, sw, bias, K: int, out=None, stream=None):
+    M, N = qx.shape[0], qw.shape[0]
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=qx.device) if out is None else out
+    _check(lib().convrot_linear_prepared(_p(qx), _p(sx), _p(qw), _p(sw), _p(bias), M, N, K,
+                                         _p(out), _stream(stream)), "convrot_linear_prepared")
+    return out
+
+
+def convrot_debug_rotate_f32(x, group: int, out=None, stream=None):
+    M, K = x.shape
+    out = torch.empty(M, K, dtype=torch.float32, device=x.device) if out is None else out
+    _check(lib().convrot_debug_rotate_f32(_p(x), M, K, group, _p(out), _stream(stream)),
+           "convrot_debug_rotate_f32")
+    return out
+
+
+def convrot_debug_gemm_s32(qx, qw, K: int, out=None, stream=None):
+    M, N = qx.shape[0], qw.shape[0]
+    out = torch.empty(M, N, dtype=torch.int32, device=qx.device) if out is None else out
+    _check(lib().convrot_debug_gemm_s32(_p(qx), _p(qw), M, N, K, _p(out), _stream(stream)),
+           "convrot_debug_gemm_s32")
+    return out
+
+
+def convrot_check_device_error(stream=None) -> int:
+    """Synchronise the stream; return (and clear) the device error status."""
+    return int(lib().convrot_check_device_error(_stream(stream)))
+
+
+def convrot_debug_timeout_probe(timeout_ns: int, stream=None):
+    _check(lib().convrot_debug_timeout_probe(int(timeout_ns), _stream(stream)),
+           "convrot_debug_timeout_probe")
+
+
+class ConvRotLinear:
+    """A linear layer held as rotated, row-quantised, packed INT4 weights.
+
+    ``ConvRotLinear.from_dense(weight, bias, group)`` prepares the weights once
+    (offline step); calling the layer runs the whole fused path on the current
+    stream.  It mirrors the page's ``ConvRotLinear`` / ``quantize_convrot_weight``
+    pair ("convrot-mlx" README, "Install and test").
+    """
+
+    def __init__(self, qweight, scales, bias, group: int, in_features: int):
+        self.qweight, self.scales, self.bias = qweight, scales, bias
+        self.group, self.in_features = group, in_features
+        self.out_features = qweight.shape[0]
+        self._ws = None
+
+    @classmethod
+    def from_dense(cls, weight: torch.Tensor, bias: torch.Tensor | None, group: int = 256):
+        qw, sw = convrot_quantize_weight(weight.contiguous(), group)
+        b = None if bias is None else bias.to(torch.bfloat16).contiguous()
+        return cls(qw, sw, b, group, weight.shape[1])
+
+    def __call__(self, x: torch.Tensor) -> torch.Tensor:
+        lead = x.shape[:-1]
+        x2 = x.reshape(-1, self.in_features).contiguous()
+        need = convrot_linear_workspace_size(x2.shape[0], self.in_features)
+        if self._ws is None or self._ws.numel() < need or self._ws.device != x2.device:
+            self._ws = torch.empty(max(1, need), dtype=torch.uint8, device=x2.device)
+        y = convrot_linear(x2, self.qweight, self.scales, self.bias, self.group, self._ws)
+        return y.reshape(*lead, self.out_features)

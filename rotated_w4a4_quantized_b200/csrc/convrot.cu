@@ -1,0 +1,329 @@
+// convrot.cu -- the C ABI declared in include/convrot.h: argument checks,
+// launch configuration and TMA descriptors around the prep and GEMM kernels.
+// One translation unit, so the device error word is a single symbol.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include <mutex>
+
+#include "../../include/convrot.h"
+#include "gemm.cuh"
+#include "prep.cuh"
+#include "ptx.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool ready = false;
+    convrot_status status = CONVROT_OK;
+    int num_sms = 0;
+};
+
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mu;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+template <class F>
+bool set_smem(F *kernel, int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+           cudaSuccess;
+}
+
+// Per-device one-time set-up: capability check, SM count, kernel attributes.
+convrot_status device_setup(int *dev_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CONVROT_ERR_CUDA;
+    *dev_out = dev;
+    DeviceState &st = g_dev[dev];
+    if (st.ready) return st.status;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (st.ready) return st.status;
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        st.status = CONVROT_ERR_CUDA;
+        st.ready = true;
+        return st.status;
+    }
+    if (major != 10 || minor != 0) {
+        st.status = CONVROT_ERR_UNSUPPORTED;
+        st.ready = true;
+        return st.status;
+    }
+    if (!g_encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                             &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn) {
+            st.status = CONVROT_ERR_CUDA;
+            st.ready = true;
+            return st.status;
+        }
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    bool ok = true;
+    ok &= set_smem(gemm::gemm_kernel<256, false, false>, gemm::Cfg<256>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<256, false, true>, gemm::Cfg<256>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<16, true, false>, gemm::Cfg<16>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<32, true, false>, gemm::Cfg<32>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<64, true, false>, gemm::Cfg<64>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<128, true, false>, gemm::Cfg<128>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<16, true, true>, gemm::Cfg<16>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<32, true, true>, gemm::Cfg<32>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<64, true, true>, gemm::Cfg<64>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<128, true, true>, gemm::Cfg<128>::SMEM_BYTES);
+    st.num_sms = sms;
+    st.status = ok ? CONVROT_OK : CONVROT_ERR_CUDA;
+    st.ready = true;
+    return st.status;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+convrot_status check_shape(int64_t rows, int64_t K, int group) {
+    if (group != 64 && group != 256) return CONVROT_ERR_GROUP;
+    if (rows < 0 || K < 64 || K > CONVROT_MAX_K || K % group) return CONVROT_ERR_SHAPE;
+    if (rows > (int64_t(1) << 30)) return CONVROT_ERR_SHAPE;
+    return CONVROT_OK;
+}
+
+convrot_status launch_prep(const void *x, int64_t rows, int64_t K, int group, uint8_t *q, float *s,
+                           float *yrot, cudaStream_t stream) {
+    if (rows == 0) return CONVROT_OK;
+    const dim3 grid(static_cast<unsigned>(rows));
+    const dim3 block(static_cast<unsigned>(K / prep::kElemsPerThread));
+    const uint16_t *xx = static_cast<const uint16_t *>(x);
+    const int k = static_cast<int>(K);
+    if (yrot) {
+        if (group == 64) prep::prep_kernel<64, 1><<<grid, block, 0, stream>>>(xx, k, q, s, yrot);
+        else prep::prep_kernel<256, 1><<<grid, block, 0, stream>>>(xx, k, q, s, yrot);
+    } else {
+        if (group == 64) prep::prep_kernel<64, 0><<<grid, block, 0, stream>>>(xx, k, q, s, yrot);
+        else prep::prep_kernel<256, 0><<<grid, block, 0, stream>>>(xx, k, q, s, yrot);
+    }
+    return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
+}
+
+bool make_map(CUtensorMap *map, const uint8_t *base, int64_t rows, int64_t K, int box_rows) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(gemm::BKP), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, bool SWAP, bool OUT_S32>
+convrot_status launch_gemm_cfg(int num_sms, const uint8_t *qA, const uint8_t *qB, int64_t rowsA,
+                               int64_t rowsB, int64_t K, const float *sx, const float *sw,
+                               const void *bias, void *out, int64_t M, int64_t N,
+                               cudaStream_t stream) {
+    CUtensorMap tmA, tmB;
+    if (!make_map(&tmA, qA, rowsA, K, gemm::BM) || !make_map(&tmB, qB, rowsB, K, BN))
+        return CONVROT_ERR_CUDA;
+    const int64_t tiles = ((rowsA + gemm::BM - 1) / gemm::BM) * ((rowsB + BN - 1) / BN);
+    const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+    gemm::gemm_kernel<BN, SWAP, OUT_S32><<<grid, gemm::kThreads, gemm::Cfg<BN>::SMEM_BYTES, stream>>>(
+        tmA, tmB, static_cast<int>(rowsA), static_cast<int>(rowsB), static_cast<int>(K), sx, sw,
+        static_cast<const uint16_t *>(bias), out, static_cast<int>(M), static_cast<int>(N));
+    return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
+}
+
+// Path choice: up to 128 tokens the weights take the 128-row MMA side
+// (skinny form, N-side tile = tokens rounded up to 16); otherwise 128 x 256
+// tiles with tokens on the M side.
+template <bool OUT_S32>
+convrot_status launch_gemm(int num_sms, const uint8_t *qx, const float *sx, const uint8_t *qw,
+                           const float *sw, const void *bias, int64_t M, int64_t N, int64_t K,
+                           void *out, cudaStream_t stream) {
+    if (M <= 128) {
+        if (M <= 16)
+            return launch_gemm_cfg<16, true, OUT_S32>(num_sms, qw, qx, N, M, K, sx, sw, bias, out, M,
+                                                      N, stream);
+        if (M <= 32)
+            return launch_gemm_cfg<32, true, OUT_S32>(num_sms, qw, qx, N, M, K, sx, sw, bias, out, M,
+                                                      N, stream);
+        if (M <= 64)
+            return launch_gemm_cfg<64, true, OUT_S32>(num_sms, qw, qx, N, M, K, sx, sw, bias, out, M,
+                                                      N, stream);
+        return launch_gemm_cfg<128, true, OUT_S32>(num_sms, qw, qx, N, M, K, sx, sw, bias, out, M, N,
+                                                   stream);
+    }
+    return launch_gemm_cfg<256, false, OUT_S32>(num_sms, qx, qw, M, N, K, sx, sw, bias, out, M, N,
+                                                stream);
+}
+
+convrot_status check_gemm_args(const uint8_t *qx, const uint8_t *qw, int64_t M, int64_t N,
+                               int64_t K) {
+    if (!qx || !qw) return CONVROT_ERR_NULL;
+    if (M < 0 || N < 0 || K < 64 || K > CONVROT_MAX_K || K % 64) return CONVROT_ERR_SHAPE;
+    if (M > (int64_t(1) << 30) || N > (int64_t(1) << 30) || M * N > (int64_t(1) << 40))
+        return CONVROT_ERR_SHAPE;
+    if (!aligned16(qx) || !aligned16(qw)) return CONVROT_ERR_ALIGN;
+    return CONVROT_OK;
+}
+
+inline size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+extern "C" {
+
+const char *convrot_status_string(convrot_status s) {
+    switch (s) {
+        case CONVROT_OK: return "CONVROT_OK";
+        case CONVROT_ERR_NULL: return "CONVROT_ERR_NULL: a required pointer is NULL";
+        case CONVROT_ERR_GROUP: return "CONVROT_ERR_GROUP: group must be 64 or 256";
+        case CONVROT_ERR_SHAPE: return "CONVROT_ERR_SHAPE: bad shape (K % group, K range, sizes)";
+        case CONVROT_ERR_ALIGN: return "CONVROT_ERR_ALIGN: pointer not 16-byte aligned";
+        case CONVROT_ERR_WORKSPACE: return "CONVROT_ERR_WORKSPACE: workspace too small or misaligned";
+        case CONVROT_ERR_CUDA: return "CONVROT_ERR_CUDA: a CUDA call or launch failed";
+        case CONVROT_ERR_DEVICE_TIMEOUT: return "CONVROT_ERR_DEVICE_TIMEOUT: a bounded device wait ran out";
+        case CONVROT_ERR_UNSUPPORTED: return "CONVROT_ERR_UNSUPPORTED: needs an sm_100 device";
+    }
+    return "CONVROT_ERR_UNKNOWN";
+}
+
+convrot_status convrot_quantize_weight(const void *w_bf16, int64_t N, int64_t K, int group,
+                                       uint8_t *qw, float *sw, convrot_stream_t stream) {
+    convrot_status st = check_shape(N, K, group);
+    if (st != CONVROT_OK) return st;
+    if (N == 0) return CONVROT_OK;
+    if (!w_bf16 || !qw || !sw) return CONVROT_ERR_NULL;
+    if (!aligned16(w_bf16) || !aligned16(qw) || (reinterpret_cast<uintptr_t>(sw) & 3u))
+        return CONVROT_ERR_ALIGN;
+    int dev;
+    if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    return launch_prep(w_bf16, N, K, group, qw, sw, nullptr, stream);
+}
+
+convrot_status convrot_prepare_act(const void *x_bf16, int64_t M, int64_t K, int group, uint8_t *qx,
+                                   float *sx, convrot_stream_t stream) {
+    return convrot_quantize_weight(x_bf16, M, K, group, qx, sx, stream);
+}
+
+size_t convrot_linear_workspace_size(int64_t M, int64_t K) {
+    if (M <= 0 || K <= 0) return 0;
+    return round256(static_cast<size_t>(M) * static_cast<size_t>(K / 2)) +
+           round256(static_cast<size_t>(M) * sizeof(float));
+}
+
+convrot_status convrot_linear_prepared(const uint8_t *qx, const float *sx, const uint8_t *qw,
+                                       const float *sw, const void *bias_bf16, int64_t M, int64_t N,
+                                       int64_t K, void *y_bf16, convrot_stream_t stream) {
+    if (M < 0 || N < 0) return CONVROT_ERR_SHAPE;
+    if (M == 0 || N == 0) return CONVROT_OK;
+    convrot_status st = check_gemm_args(qx, qw, M, N, K);
+    if (st != CONVROT_OK) return st;
+    if (!sx || !sw || !y_bf16) return CONVROT_ERR_NULL;
+    if (!aligned16(sx) || !aligned16(sw) || !aligned16(y_bf16) ||
+        (bias_bf16 && !aligned16(bias_bf16)))
+        return CONVROT_ERR_ALIGN;
+    int dev;
+    if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    return launch_gemm<false>(g_dev[dev].num_sms, qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream);
+}
+
+convrot_status convrot_linear(const void *x_bf16, const uint8_t *qw, const float *sw,
+                              const void *bias_bf16, int64_t M, int64_t N, int64_t K, int group,
+                              void *workspace, size_t ws_bytes, void *y_bf16,
+                              convrot_stream_t stream) {
+    convrot_status st = check_shape(M, K, group);
+    if (st != CONVROT_OK) return st;
+    if (N < 0) return CONVROT_ERR_SHAPE;
+    if (M == 0 || N == 0) return CONVROT_OK;
+    if (!x_bf16 || !qw || !sw || !y_bf16 || !workspace) return CONVROT_ERR_NULL;
+    if (ws_bytes < convrot_linear_workspace_size(M, K) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return CONVROT_ERR_WORKSPACE;
+    if (!aligned16(x_bf16) || !aligned16(qw) || !aligned16(sw) || !aligned16(y_bf16) ||
+        (bias_bf16 && !aligned16(bias_bf16)))
+        return CONVROT_ERR_ALIGN;
+    if ((st = check_gemm_args(qw, qw, M, N, K)) != CONVROT_OK) return st;
+    int dev;
+    if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    uint8_t *qx = static_cast<uint8_t *>(workspace);
+    float *sx = reinterpret_cast<float *>(qx + round256(static_cast<size_t>(M) * (K / 2)));
+    if ((st = launch_prep(x_bf16, M, K, group, qx, sx, nullptr, stream)) != CONVROT_OK) return st;
+    return launch_gemm<false>(g_dev[dev].num_sms, qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream);
+}
+
+convrot_status convrot_debug_rotate_f32(const void *x_bf16, int64_t M, int64_t K, int group,
+                                        float *y_rot, convrot_stream_t stream) {
+    convrot_status st = check_shape(M, K, group);
+    if (st != CONVROT_OK) return st;
+    if (M == 0) return CONVROT_OK;
+    if (!x_bf16 || !y_rot) return CONVROT_ERR_NULL;
+    if (!aligned16(x_bf16) || !aligned16(y_rot)) return CONVROT_ERR_ALIGN;
+    int dev;
+    if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    return launch_prep(x_bf16, M, K, group, nullptr, nullptr, y_rot, stream);
+}
+
+convrot_status convrot_debug_gemm_s32(const uint8_t *qx, const uint8_t *qw, int64_t M, int64_t N,
+                                      int64_t K, int32_t *acc, convrot_stream_t stream) {
+    if (M < 0 || N < 0) return CONVROT_ERR_SHAPE;
+    if (M == 0 || N == 0) return CONVROT_OK;
+    convrot_status st = check_gemm_args(qx, qw, M, N, K);
+    if (st != CONVROT_OK) return st;
+    if (!acc) return CONVROT_ERR_NULL;
+    if (!aligned16(acc)) return CONVROT_ERR_ALIGN;
+    int dev;
+    if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    return launch_gemm<true>(g_dev[dev].num_sms, qx, nullptr, qw, nullptr, nullptr, M, N, K, acc,
+                             stream);
+}
+
+convrot_status convrot_check_device_error(convrot_stream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return CONVROT_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_convrot_error, sizeof v) != cudaSuccess) return CONVROT_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_convrot_error, &zero, sizeof zero) != cudaSuccess)
+            return CONVROT_ERR_CUDA;
+        return static_cast<convrot_status>(v);
+    }
+    return CONVROT_OK;
+}
+
+}  // extern "C"
+
+// The timeout probe: one thread waits on a barrier nothing signals.
+__global__ void timeout_probe_kernel(uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    const uint32_t b = ptx::smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(b, 1);
+        abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) ptx::mbar_wait(b, 0, &abort_flag, limit_ns);
+}
+
+extern "C" convrot_status convrot_debug_timeout_probe(int64_t timeout_ns,
+                                                      convrot_stream_t stream) {
+    int dev;
+    convrot_status st = device_setup(&dev);
+    if (st != CONVROT_OK) return st;
+    if (timeout_ns < 1000) timeout_ns = 1000;
+    if (timeout_ns > 5000000000ll) timeout_ns = 5000000000ll;
+    timeout_probe_kernel<<<1, 32, 0, stream>>>(static_cast<uint64_t>(timeout_ns));
+    return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
+}

@@ -1,0 +1,362 @@
+// gemm.cuh -- packed INT4 x INT4 GEMM on the sm_100a tensor cores, with the
+// fused scale / bias / bf16 epilogue.
+//
+// What it computes ("convrot-mlx" README, "What is included" and "Install and
+// test"): acc[m][n] = sum_k qx[m][k] qw[n][k] exactly, then
+// y[m][n] = bf16_rne((float(acc) * sx[m]) * sw[n] + b[n]).
+//
+// The tensor pipe has no 4-bit integer operand, so packed tiles are widened
+// to int8 in shared memory and fed to tcgen05.mma kind::i8 (s8 x s8 -> s32,
+// accumulators in TMEM).  Widening: a packed byte holds code c0 in its low
+// nibble and c1 in its high nibble (two's complement).  (byte & 0xF0) read
+// as int8 is exactly 16 c1, and ((byte << 4) & 0xF0) is exactly 16 c0, so a
+// 32-bit word of 8 codes widens with one AND, one SHIFT and one AND into two
+// words of four int8 each: no sign-extension work.  Both operands are
+// widened the same way, so the tensor cores accumulate 256 * acc; the
+// epilogue shifts right by 8 (exact: |256 acc| <= 256 * 49 * 32768 < 2^31).
+// The widened K order inside every 32-code block is [even codes, odd codes];
+// it is the same permutation for both operands, so the dot products are
+// unchanged.
+//
+// CTA organisation (one CTA per SM, persistent over output tiles):
+//   warp 0       TMA producer: packed A [128 x 64 B] and B [BN x 64 B] tiles
+//                per K-block into a ring of packed stages;
+//   warp 1       TMEM allocator and MMA issuer (one thread): 4 MMAs of K = 32
+//                per K-block into one of two TMEM accumulators;
+//   warps 2..5   epilogue: tcgen05.ld, shift, scale, bias, bf16, store;
+//   warps 6..13  widening: packed stage -> int8 stage in the 128-byte
+//                swizzled K-major layout the MMA descriptors describe.
+// Accumulators are double-buffered in TMEM so the epilogue of one tile runs
+// under the main loop of the next.
+//
+// SWAP selects the skinny-M form: the weights become the 128-row MMA operand
+// and the few token rows the N-side operand (BN = 16 .. 128), so the weight
+// stream is split over many CTAs; the epilogue writes the transposed tile.
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+#include "ptx.cuh"
+
+namespace gemm {
+
+constexpr int BM = 128;          // MMA M: rows of operand A per tile
+constexpr int BKP = 64;          // packed bytes per row per K-block
+constexpr int BK = 128;          // int8 values per row per K-block
+constexpr int kThreads = 448;    // 14 warps
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpEpi0 = 2, kWarpUnp0 = 6;
+constexpr int kUnpWarps = 8;
+
+template <int BN>
+struct Cfg {
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "kind::i8 with M=128 needs N%16==0");
+    static constexpr int SP = (BN == 256) ? 3 : 4;     // packed stages
+    static constexpr int SU = (BN == 256) ? 3 : 4;     // widened stages
+    static constexpr int PA = BM * BKP;
+    static constexpr int PB = BN * BKP;
+    static constexpr int UA = BM * BK;
+    static constexpr int UB = BN * BK;
+    static constexpr int OFF_UA = 0;                   // 1024-aligned tiles first
+    static constexpr int OFF_UB = OFF_UA + SU * UA;
+    static constexpr int OFF_PA = OFF_UB + SU * UB;
+    static constexpr int OFF_PB = OFF_PA + SP * PA;
+    static constexpr int OFF_BAR = OFF_PB + SP * PB;
+    static constexpr int NUM_BARS = 2 * SP + 2 * SU + 5;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + slack for 1024 alignment
+    // Each accumulator buffer is read 32 columns at a time, so buffers are at
+    // least 32 columns apart and the allocation covers two of them.
+    static constexpr int ACC_STRIDE = BN < 32 ? 32 : BN;
+    static constexpr int TMEM_COLS = 2 * ACC_STRIDE;        // 64 .. 512, a power of two
+    static constexpr int JW = BN < 32 ? BN : 32;             // valid columns per 32-wide read
+    static_assert(UB % 1024 == 0, "widened B tiles must stay 1024-aligned");
+    static_assert(SMEM_BYTES <= 232448, "exceeds the per-CTA shared memory limit");
+};
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "r"(addr));
+    return r;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                       uint32_t d) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t h) {
+    return __uint_as_float(static_cast<uint32_t>(h) << 16);
+}
+
+__device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
+    __nv_bfloat16 h = __float2bfloat16_rn(f);
+    return *reinterpret_cast<uint16_t *>(&h);
+}
+
+// The epilogue arithmetic, in the fixed order of the definition.
+__device__ __forceinline__ float epi(uint32_t raw, float sx, float sw, float b) {
+    const int acc = static_cast<int>(raw) >> 8;
+    float t = __fmul_rn(__int2float_rn(acc), sx);
+    t = __fmul_rn(t, sw);
+    return __fadd_rn(t, b);
+}
+
+// OUT_S32: write the integer accumulators (test hook) instead of bf16.
+template <int BN, bool SWAP, bool OUT_S32>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+            int rowsA, int rowsB, int K, const float *__restrict__ sx,
+            const float *__restrict__ sw, const uint16_t *__restrict__ bias,
+            void *__restrict__ out, int M, int N) {
+    using C = Cfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = ptx::smem_u32(smem);
+    const uint32_t bar0 = sbase + C::OFF_BAR;
+    auto full_p = [&](int s) { return bar0 + 8u * s; };
+    auto empty_p = [&](int s) { return bar0 + 8u * (C::SP + s); };
+    auto full_u = [&](int s) { return bar0 + 8u * (2 * C::SP + s); };
+    auto empty_u = [&](int s) { return bar0 + 8u * (2 * C::SP + C::SU + s); };
+    auto acc_full = [&](int b) { return bar0 + 8u * (2 * C::SP + 2 * C::SU + b); };
+    auto acc_empty = [&](int b) { return bar0 + 8u * (2 * C::SP + 2 * C::SU + 2 + b); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * C::SP + 2 * C::SU + 4);
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::SP; ++s) {
+            ptx::mbar_init(full_p(s), 1);
+            ptx::mbar_init(empty_p(s), kUnpWarps);
+        }
+        for (int s = 0; s < C::SU; ++s) {
+            ptx::mbar_init(full_u(s), kUnpWarps);
+            ptx::mbar_init(empty_u(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(acc_full(b), 1);
+            ptx::mbar_init(acc_empty(b), 4);
+        }
+        ptx::mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == kWarpTma && lane == 0) {
+        ptx::tma_prefetch_desc(&tmA);
+        ptx::tma_prefetch_desc(&tmB);
+    }
+    if (warp == kWarpMma) {
+        ptx::tmem_alloc(sbase + C::OFF_MISC, C::TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int tiles_a = (rowsA + BM - 1) / BM;
+    const int tiles_b = (rowsB + BN - 1) / BN;
+    const int num_tiles = tiles_a * tiles_b;
+    const int num_kb = (K / 2 + BKP - 1) / BKP;
+
+    if (warp == kWarpTma) {
+        if (lane == 0) {
+            int ps = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int ta = tile % tiles_a, tb = tile / tiles_a;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!ptx::mbar_wait(empty_p(ps), ph ^ 1, abort_flag)) { ok = false; break; }
+                    ptx::mbar_arrive_expect_tx(full_p(ps), C::PA + C::PB);
+                    ptx::tma_load_2d(sbase + C::OFF_PA + ps * C::PA, &tmA, full_p(ps), kb * BKP,
+                                     ta * BM);
+                    ptx::tma_load_2d(sbase + C::OFF_PB + ps * C::PB, &tmB, full_p(ps), kb * BKP,
+                                     tb * BN);
+                    if (++ps == C::SP) { ps = 0; ph ^= 1; }
+                }
+            }
+            if (!ok) {
+                // Let copies already in flight land before the CTA exits.
+                for (int s = 0; s < C::SP; ++s) {
+                    volatile int never = 0;
+                    ptx::mbar_wait(full_p(s), ph ^ (s < ps ? 0u : 1u), &never, 10000000ull);
+                }
+            }
+        }
+    } else if (warp == kWarpMma) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = ptx::idesc_i8(BM, BN);
+            int us = 0;
+            uint32_t ph = 0;
+            int local = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+                const int b = local & 1;
+                const uint32_t aph = (local >> 1) & 1;
+                if (!ptx::mbar_wait(acc_empty(b), aph ^ 1, abort_flag)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t d = tmem_base + static_cast<uint32_t>(b * C::ACC_STRIDE);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!ptx::mbar_wait(full_u(us), ph, abort_flag)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    const uint32_t a0 = sbase + C::OFF_UA + us * C::UA;
+                    const uint32_t b0 = sbase + C::OFF_UB + us * C::UB;
+#pragma unroll
+                    for (int j = 0; j < BK / 32; ++j)
+                        ptx::mma_i8_ss(d, ptx::sw128_kmajor_desc(a0 + 32 * j),
+                                       ptx::sw128_kmajor_desc(b0 + 32 * j), idesc,
+                                       (kb | j) != 0 ? 1u : 0u);
+                    ptx::tc_commit(empty_u(us));
+                    if (++us == C::SU) { us = 0; ph ^= 1; }
+                }
+                if (ok) ptx::tc_commit(acc_full(b));
+            }
+            // Wait for every MMA this thread issued before TMEM is released.
+            ptx::tc_commit(drain_bar);
+            volatile int never = 0;
+            ptx::mbar_wait(drain_bar, 0, &never, 100000000ull);
+        }
+    } else if (warp < kWarpEpi0 + 4) {
+        const int quarter = warp & 3;                 // TMEM lanes 32*quarter ..
+        const int r = quarter * 32 + lane;            // row of the accumulator tile
+        int local = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+            const int ta = tile % tiles_a, tb = tile / tiles_a;
+            const int b = local & 1;
+            const uint32_t aph = (local >> 1) & 1;
+            if (!ptx::mbar_wait(acc_full(b), aph, abort_flag)) break;
+            ptx::tc_fence_after();
+            const int arow = ta * BM + r;             // A row of this lane
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t v[32];
+                __syncwarp();   // tcgen05.ld is warp-collective
+                ptx::tmem_ld_32x32b_x32(
+                    tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                        static_cast<uint32_t>(b * C::ACC_STRIDE + c0),
+                    v);
+                ptx::tmem_ld_wait();
+                const int bcol0 = tb * BN + c0;       // first B row of these 32 columns
+                if (!SWAP) {
+                    // lane = output row m, columns = output columns n
+                    const int m = arow;
+                    if (m >= M) continue;
+                    const int n0 = bcol0;
+                    if (OUT_S32) {
+                        int32_t *o = reinterpret_cast<int32_t *>(out) + static_cast<size_t>(m) * N;
+                        for (int j = 0; j < C::JW; ++j)
+                            if (n0 + j < N) o[n0 + j] = static_cast<int32_t>(v[j]) >> 8;
+                    } else {
+                        const float sxm = sx[m];
+                        uint16_t *o = reinterpret_cast<uint16_t *>(out) + static_cast<size_t>(m) * N;
+                        if (C::JW == 32 && n0 + 32 <= N && (N & 7) == 0) {
+                            uint32_t pk[16];
+#pragma unroll
+                            for (int j = 0; j < 32; j += 2) {
+                                const float b0 = bias ? bf16_to_f32(bias[n0 + j]) : 0.0f;
+                                const float b1 = bias ? bf16_to_f32(bias[n0 + j + 1]) : 0.0f;
+                                const uint16_t h0 = f32_to_bf16_rne(epi(v[j], sxm, sw[n0 + j], b0));
+                                const uint16_t h1 =
+                                    f32_to_bf16_rne(epi(v[j + 1], sxm, sw[n0 + j + 1], b1));
+                                pk[j / 2] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+                            }
+                            uint4 *o4 = reinterpret_cast<uint4 *>(o + n0);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                o4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                        } else {
+                            for (int j = 0; j < C::JW; ++j) {
+                                const int n = n0 + j;
+                                if (n >= N) break;
+                                const float bb = bias ? bf16_to_f32(bias[n]) : 0.0f;
+                                o[n] = f32_to_bf16_rne(epi(v[j], sxm, sw[n], bb));
+                            }
+                        }
+                    }
+                } else {
+                    // lane = output column n (a weight row), columns = tokens m
+                    const int n = arow;
+                    if (n >= N) continue;
+                    if (OUT_S32) {
+                        int32_t *o = reinterpret_cast<int32_t *>(out);
+                        for (int j = 0; j < C::JW; ++j) {
+                            const int m = bcol0 + j;
+                            if (m >= M) break;
+                            o[static_cast<size_t>(m) * N + n] = static_cast<int32_t>(v[j]) >> 8;
+                        }
+                    } else {
+                        const float swn = sw[n];
+                        const float bn = bias ? bf16_to_f32(bias[n]) : 0.0f;
+                        uint16_t *o = reinterpret_cast<uint16_t *>(out);
+                        for (int j = 0; j < C::JW; ++j) {
+                            const int m = bcol0 + j;
+                            if (m >= M) break;
+                            o[static_cast<size_t>(m) * N + n] = f32_to_bf16_rne(epi(v[j], sx[m], swn, bn));
+                        }
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(acc_empty(b));
+        }
+    } else {
+        // widening warps
+        const int ut = threadIdx.x - kWarpUnp0 * 32;   // 0 .. 255
+        constexpr int kChunks = (BM + BN) * 4;          // 16-byte packed chunks per stage
+        int ps = 0, us = 0;
+        uint32_t pph = 0, uph = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            for (int kb = 0; kb < num_kb; ++kb) {
+                if (!ptx::mbar_wait(full_p(ps), pph, abort_flag)) { ok = false; break; }
+                if (!ptx::mbar_wait(empty_u(us), uph ^ 1, abort_flag)) { ok = false; break; }
+                const uint32_t pa = sbase + C::OFF_PA + ps * C::PA;
+                const uint32_t pb = sbase + C::OFF_PB + ps * C::PB;
+                const uint32_t ua = sbase + C::OFF_UA + us * C::UA;
+                const uint32_t ub = sbase + C::OFF_UB + us * C::UB;
+#pragma unroll 2
+                for (int idx = ut; idx < kChunks; idx += kUnpWarps * 32) {
+                    const int row = idx >> 2, c = idx & 3;
+                    const bool in_a = row < BM;
+                    const int rr = in_a ? row : row - BM;
+                    const uint32_t src = (in_a ? pa : pb) + rr * 64 + c * 16;
+                    const uint32_t dst = (in_a ? ua : ub) + rr * 128;
+                    const uint32_t sw8 = static_cast<uint32_t>(rr & 7);
+                    const uint4 w = lds128(src);
+                    const uint32_t hm = 0xF0F0F0F0u;
+                    sts128(dst + (((2u * c) ^ sw8) << 4), (w.x << 4) & hm, (w.y << 4) & hm,
+                           (w.z << 4) & hm, (w.w << 4) & hm);
+                    sts128(dst + (((2u * c + 1u) ^ sw8) << 4), w.x & hm, w.y & hm, w.z & hm,
+                           w.w & hm);
+                }
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    ptx::mbar_arrive(empty_p(ps));
+                    ptx::mbar_arrive(full_u(us));
+                }
+                if (++ps == C::SP) { ps = 0; pph ^= 1; }
+                if (++us == C::SU) { us = 0; uph ^= 1; }
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == kWarpMma) {
+        __syncwarp();
+        ptx::tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+}  // namespace gemm

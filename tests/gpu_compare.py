@@ -1,0 +1,105 @@
+"""Comparison helpers for the GPU parity tests (test infrastructure).
+
+Gates (fixed here, used by every GPU test):
+  - rotated values: |y_gpu - y_oracle| <= 1e-5 * max|y_oracle| per row
+    (fp32 butterflies against the fp64 dense product);
+  - scales: relative difference <= 1e-5;
+  - codes and packed bytes: identical, except at positions whose oracle
+    y/s lies within 1e-5 of a .5 rounding boundary (the "tie band"), where
+    the two fp32 evaluations of the rotation may round apart by one code;
+  - integer accumulators: identical when both sides start from the same
+    codes;
+  - bf16 outputs: within 1 bf16 ulp of the oracle's fp32 epilogue when both
+    sides start from the same codes and scales; with independently prepared
+    codes, within 1 ulp plus the exact effect of the tie-band code
+    differences the oracle itself identifies (each moves acc by at most the
+    other operand's code magnitude + 1).
+
+GPU bytes are decoded here with numpy, never by the oracle.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+TIE_BAND = 1e-5
+ROT_TOL = 1e-5
+SCALE_RTOL = 1e-5
+
+
+def to_np_u16(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def decode_codes(packed: np.ndarray) -> np.ndarray:
+    """uint8 [rows][K/2] -> int8 [rows][K], low nibble first, two's complement."""
+    p = packed.astype(np.int16)
+    lo = p & 0xF
+    hi = (p >> 4) & 0xF
+    lo = np.where(lo >= 8, lo - 16, lo)
+    hi = np.where(hi >= 8, hi - 16, hi)
+    out = np.empty((packed.shape[0], packed.shape[1] * 2), dtype=np.int8)
+    out[:, 0::2] = lo
+    out[:, 1::2] = hi
+    return out
+
+
+def bf16_f64(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def bf16_ulp(v: np.ndarray) -> np.ndarray:
+    a = np.abs(v)
+    e = np.floor(np.log2(np.where(a > 0, a, 1e-38)))
+    return np.where(a > 0, 2.0 ** (e - 7), 2.0 ** -133)
+
+
+def check_rotation(y_gpu: np.ndarray, y_ref: np.ndarray):
+    amax = np.abs(y_ref).max(axis=1, keepdims=True)
+    err = np.abs(y_gpu.astype(np.float64) - y_ref)
+    bad = err > ROT_TOL * np.maximum(amax, 1e-30)
+    assert not bad.any(), f"rotation off at {np.argwhere(bad)[:5]}, max rel {(err / np.maximum(amax, 1e-30)).max()}"
+
+
+def check_prepared(q_gpu_packed, s_gpu, q_ref_packed, s_ref, tie):
+    """Codes/bytes equal outside the tie band; scales within SCALE_RTOL."""
+    s_gpu = np.asarray(s_gpu, dtype=np.float64)
+    s_ref = np.asarray(s_ref, dtype=np.float64)
+    rel = np.abs(s_gpu - s_ref) / np.maximum(np.abs(s_ref), 1e-30)
+    assert np.all((s_ref == 0) == (s_gpu == 0)), "zero-scale rows differ"
+    assert rel.max() <= SCALE_RTOL, f"scale rel err {rel.max()}"
+    cg = decode_codes(q_gpu_packed)
+    cr = decode_codes(q_ref_packed)
+    diff = cg != cr
+    outside = diff & ~tie
+    assert not outside.any(), f"{outside.sum()} codes differ outside the tie band, e.g. {np.argwhere(outside)[:5]}"
+    assert np.all(np.abs(cg.astype(int) - cr.astype(int)) <= 1), "a code moved by more than one step"
+    # bytes whose two codes agree must be identical
+    same_pair = ~(diff[:, 0::2] | diff[:, 1::2])
+    assert np.array_equal(q_gpu_packed[same_pair], q_ref_packed[same_pair])
+    return int(diff.sum())
+
+
+def output_tolerance(y_ref_bits, qx_ref, qw_ref, sx, sw, tie_x, tie_w):
+    """Per-element allowance: 1 bf16 ulp, plus the largest acc change the
+    oracle's tie-band positions allow, times the scales, plus one more ulp
+    for the re-rounding when that term is nonzero."""
+    y = bf16_f64(y_ref_bits)
+    cx = np.abs(decode_codes(qx_ref).astype(np.int64)) + 1
+    cw = np.abs(decode_codes(qw_ref).astype(np.int64)) + 1
+    dacc = (tie_x.astype(np.int64) @ cw.T) + (cx @ tie_w.astype(np.int64).T)
+    extra = dacc * np.asarray(sx, np.float64)[:, None] * np.asarray(sw, np.float64)[None, :] * 1.001
+    tol = bf16_ulp(y) + extra + np.where(dacc > 0, bf16_ulp(np.abs(y) + extra), 0.0)
+    return tol
+
+
+def check_outputs(y_gpu_bits, y_ref_bits, tol=None):
+    g = bf16_f64(y_gpu_bits)
+    r = bf16_f64(y_ref_bits)
+    if tol is None:
+        tol = bf16_ulp(r)
+    err = np.abs(g - r)
+    bad = err > tol
+    assert not bad.any(), (f"{bad.sum()} outputs outside tolerance, e.g. at {np.argwhere(bad)[:5]}: "
+                           f"gpu {g[bad][:5]} ref {r[bad][:5]}")
+    return int((err > 0).sum())

@@ -1,0 +1,93 @@
+"""The C ABI library without a GPU: it loads, exports every symbol the header
+declares, and rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import rotated_w4a4_quantized_b200 as cr
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "convrot.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from rotated_w4a4_quantized_b200 import build
+    build.build()
+    return cr.lib()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(convrot_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for required in ("convrot_quantize_weight", "convrot_prepare_act", "convrot_linear",
+                     "convrot_linear_prepared", "convrot_linear_workspace_size",
+                     "convrot_debug_rotate_f32", "convrot_debug_gemm_s32",
+                     "convrot_status_string", "convrot_check_device_error",
+                     "convrot_debug_timeout_probe"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code in range(9):
+        s = L.convrot_status_string(code).decode()
+        assert s.startswith("CONVROT_")
+    assert L.convrot_status_string(123).decode() == "CONVROT_ERR_UNKNOWN"
+
+
+def test_workspace_size(L):
+    assert cr.convrot_linear_workspace_size(0, 1024) == 0
+    assert cr.convrot_linear_workspace_size(3, 1024) == 1536 + 256
+    assert cr.convrot_linear_workspace_size(1, 64) == 256 + 256
+    assert cr.convrot_linear_workspace_size(1024, 3072) == 1024 * 1536 + 4096
+
+
+A = ctypes.c_void_p(0x10000)    # fake, aligned, never dereferenced: checks fail first
+B = ctypes.c_void_p(0x20000)
+U = ctypes.c_void_p(0x20008)    # 8-byte aligned only
+
+
+def test_host_validation_without_device(L):
+    s = None
+    # group / shape
+    assert L.convrot_quantize_weight(A, 4, 1024, 128, B, B, s) == 2
+    assert L.convrot_quantize_weight(A, 4, 1000, 64, B, B, s) == 3
+    assert L.convrot_quantize_weight(A, 4, 32768 + 256, 256, B, B, s) == 3
+    assert L.convrot_quantize_weight(A, -1, 1024, 64, B, B, s) == 3
+    assert L.convrot_prepare_act(A, 4, 64, 256, B, B, s) == 3      # K % group
+    # empty work is a no-op, even with NULL pointers
+    assert L.convrot_prepare_act(None, 0, 1024, 64, None, None, s) == 0
+    assert L.convrot_linear(None, None, None, None, 0, 8, 1024, 64, None, 0, None, s) == 0
+    # NULL and alignment
+    assert L.convrot_prepare_act(None, 4, 1024, 64, B, B, s) == 1
+    assert L.convrot_prepare_act(U, 4, 1024, 64, B, B, s) == 4
+    ws = cr.convrot_linear_workspace_size(4, 1024)
+    assert L.convrot_linear(A, B, B, None, 4, 8, 1024, 64, A, ws - 1, B, s) == 5
+    assert L.convrot_linear(A, B, B, None, 4, 8, 1024, 64, U, ws, B, s) == 5
+    assert L.convrot_linear(A, B, U, None, 4, 8, 1024, 64, A, ws, B, s) == 4
+    assert L.convrot_linear(A, B, B, U, 4, 8, 1024, 64, A, ws, B, s) == 4
+    assert L.convrot_linear_prepared(A, B, A, B, None, 4, 8, 1000, B, s) == 3
+    assert L.convrot_linear_prepared(None, B, A, B, None, 4, 8, 1024, B, s) == 1
+    assert L.convrot_debug_gemm_s32(A, B, 4, 8, 96, B, s) == 3
+    assert L.convrot_debug_gemm_s32(A, B, 4, 8, 128, U, s) == 4
+    assert L.convrot_debug_rotate_f32(A, 4, 512, 256, None, s) == 1
+
+
+def test_valid_call_without_gpu_reports_cuda_error(L):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    # Arguments pass validation; the device set-up then fails cleanly.
+    assert L.convrot_prepare_act(A, 4, 1024, 64, B, B, None) == 6

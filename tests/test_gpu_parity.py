@@ -1,0 +1,247 @@
+"""GPU parity: the CUDA path against the CPU oracle, element by element, on
+the same seeded inputs (gates in tests/gpu_compare.py).
+
+Small cases span several tiles and a ragged tail in every dimension; the
+full-size workloads run in the same launch configuration as the benchmark
+and are compared on sampled rows and columns the oracle computes one by one
+(rows of a linear layer are independent, so the oracle prepares only the
+sampled activation rows and weight rows)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import rotated_w4a4_quantized_b200 as cr
+from rotated_w4a4_quantized_b200 import workloads as wl
+from tests import gpu_compare as gc
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from rotated_w4a4_quantized_b200 import build
+    build.build()
+    O.build()
+
+
+def _dev(t):
+    return t.cuda()
+
+
+def _layer(M, K, N, group, seed, bias=True, zero_rows=()):
+    lt = wl.make_random_layer(M, K, N, group, seed, bias=bias)
+    if zero_rows:
+        x = lt.x.clone()
+        x[list(zero_rows)] = 0
+        lt.x = x
+    return lt
+
+
+# ---------------------------------------------------------------------------
+# step by step
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("group", [64, 256])
+@pytest.mark.parametrize("M,K", [(1, 256), (7, 1024), (33, 3072), (5, 12288), (3, 32768)])
+def test_rotation_matches_oracle(group, M, K):
+    x = wl.make_random_layer(M, K, 1, group, seed=M + K).x
+    y = cr.convrot_debug_rotate_f32(_dev(x), group)
+    torch.cuda.synchronize()
+    gc.check_rotation(y.cpu().numpy(), O.rotate(wl.bf16_bits(x), group))
+
+
+@pytest.mark.parametrize("group", [64, 256])
+@pytest.mark.parametrize("M,K", [(1, 256), (9, 1024), (130, 3072), (4, 12288), (2, 32768)])
+def test_prepare_matches_oracle(group, M, K):
+    x = _layer(M, K, 1, group, seed=3 * M + K, zero_rows=(0,) if M > 2 else ()).x
+    xb = wl.bf16_bits(x)
+    qx, sx = cr.convrot_prepare_act(_dev(x), group)
+    torch.cuda.synchronize()
+    y = O.rotate(xb, group)
+    q_ref, s_ref = O.prepare_rows(xb, group)
+    tie = O.tie_band(y, s_ref, gc.TIE_BAND)
+    gc.check_prepared(qx.cpu().numpy(), sx.cpu().numpy(), q_ref, s_ref, tie)
+    if M > 2:
+        assert sx[0].item() == 0.0 and int(qx[0].abs().sum()) == 0
+
+
+def test_prepare_edge_rows():
+    # exact ties and saturation: absmax 7 after rotation makes inv = 1
+    K, group = 256, 256
+    rows = []
+    # all ones -> rotated all ones -> all codes 7
+    rows.append(np.full(K, 0x3F80, dtype=np.uint16))
+    # one-hot -> one row of H (entries +-1/16) -> all codes +-7
+    e = np.zeros(K, dtype=np.uint16)
+    e[3] = 0x4000  # 2.0
+    rows.append(e)
+    # zeros
+    rows.append(np.zeros(K, dtype=np.uint16))
+    xb = np.stack(rows)
+    x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16)
+    qx, sx = cr.convrot_prepare_act(_dev(x), group)
+    q_ref, s_ref = O.prepare_rows(xb, group)
+    assert np.array_equal(qx.cpu().numpy(), q_ref)
+    assert np.array_equal(sx.cpu().numpy(), s_ref)
+    assert np.all(qx.cpu().numpy()[0] == 0x77)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 16, 64), (5, 72, 192), (16, 128, 1024), (17, 300, 512),
+                                   (64, 1000, 768), (100, 256, 256), (128, 384, 1024),
+                                   (129, 257, 320), (300, 600, 1536), (513, 96, 128)])
+def test_gemm_s32_bit_exact(M, N, K):
+    rng = np.random.default_rng(M * 7 + N)
+    a = rng.integers(-7, 8, size=(M, K)).astype(np.int8)
+    b = rng.integers(-7, 8, size=(N, K)).astype(np.int8)
+    if M > 3:
+        a[2] = 7
+        b[min(3, N - 1)] = -7
+    pa, pb = O.pack(a), O.pack(b)
+    acc = cr.convrot_debug_gemm_s32(_dev(torch.from_numpy(pa)), _dev(torch.from_numpy(pb)), K)
+    torch.cuda.synchronize()
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), O.gemm(pa, pb, K))
+
+
+@pytest.mark.parametrize("M,N,K,bias", [(3, 48, 256, True), (40, 200, 1024, False),
+                                        (130, 520, 768, True), (300, 13, 256, True)])
+def test_linear_prepared_one_ulp(M, N, K, bias):
+    lt = _layer(M, K, N, 64, seed=M + N, bias=bias)
+    xb, wb = wl.bf16_bits(lt.x), wl.bf16_bits(lt.w)
+    bb = None if lt.b is None else wl.bf16_bits(lt.b)
+    px, sx = O.prepare_rows(xb, 64)
+    pw, sw = O.prepare_rows(wb, 64)
+    y_ref = O.epilogue(O.gemm(px, pw, K), sx, sw, bb)
+    t = lambda a: _dev(torch.from_numpy(a))
+    y = cr.convrot_linear_prepared(t(px), t(sx), t(pw), t(sw), None if lt.b is None else _dev(lt.b), K)
+    torch.cuda.synchronize()
+    gc.check_outputs(gc.to_np_u16(y), y_ref)
+
+
+# ---------------------------------------------------------------------------
+# the whole layer
+# ---------------------------------------------------------------------------
+
+def _full_path_case(lt, group, rows=None, cols=None):
+    """Run the GPU path on the whole layer; compare rows x cols with the
+    oracle computed from the same seeded bf16 inputs."""
+    x, w = _dev(lt.x), _dev(lt.w)
+    b = None if lt.b is None else _dev(lt.b)
+    qw, sw = cr.convrot_quantize_weight(w, group)
+    y = cr.convrot_linear(x, qw, sw, b, group)
+    torch.cuda.synchronize()
+    assert cr.convrot_check_device_error() == 0
+    M, K = lt.x.shape
+    N = lt.w.shape[0]
+    rows = np.arange(M) if rows is None else np.asarray(rows)
+    cols = np.arange(N) if cols is None else np.asarray(cols)
+    xb = wl.bf16_bits(lt.x)[rows]
+    wb = wl.bf16_bits(lt.w)[cols]
+    bb = None if lt.b is None else wl.bf16_bits(lt.b)[cols]
+    px, sx = O.prepare_rows(xb, group)
+    pw, swr = O.prepare_rows(wb, group)
+    tie_x = O.tie_band(O.rotate(xb, group), sx, gc.TIE_BAND)
+    tie_w = O.tie_band(O.rotate(wb, group), swr, gc.TIE_BAND)
+    gc.check_prepared(qw.cpu().numpy()[cols], sw.cpu().numpy()[cols], pw, swr, tie_w)
+    y_ref = O.epilogue(O.gemm(px, pw, K), sx, swr, bb)
+    tol = gc.output_tolerance(y_ref, px, pw, sx, swr, tie_x, tie_w)
+    gc.check_outputs(gc.to_np_u16(y)[np.ix_(rows, cols)], y_ref, tol)
+    return y
+
+
+@pytest.mark.parametrize("group", [64, 256])
+@pytest.mark.parametrize("M,K,N", [(1, 256, 16), (2, 512, 200), (63, 1024, 130), (64, 768, 1024),
+                                   (65, 1536, 72), (128, 1024, 256), (129, 512, 600),
+                                   (300, 1536, 600), (1000, 256, 40)])
+def test_linear_matches_oracle(group, M, K, N):
+    lt = _layer(M, K, N, group, seed=M * 31 + N + group, zero_rows=(M // 2,) if M > 4 else ())
+    _full_path_case(lt, group)
+
+
+def test_zero_rows_give_exactly_the_bias():
+    lt = _layer(140, 512, 96, 256, seed=5, zero_rows=(0, 77, 139))
+    y = _full_path_case(lt, 256)
+    yb = y.cpu()
+    for r in (0, 77, 139):
+        assert torch.equal(yb[r], lt.b)
+
+
+def test_linear_deterministic():
+    lt = _layer(700, 2048, 1100, 64, seed=8)
+    x, w, b = _dev(lt.x), _dev(lt.w), _dev(lt.b)
+    qw, sw = cr.convrot_quantize_weight(w, 64)
+    y1 = cr.convrot_linear(x, qw, sw, b, 64)
+    y2 = cr.convrot_linear(x, qw, sw, b, 64)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, sampled outputs
+# ---------------------------------------------------------------------------
+
+def _sample(n, k, seed):
+    rng = np.random.default_rng(seed)
+    pick = set(rng.choice(n, size=min(n, k), replace=False).tolist())
+    pick |= {0, n - 1, min(n - 1, 127), min(n - 1, 128), min(n - 1, 255), min(n - 1, 256)}
+    return np.array(sorted(pick))
+
+
+@pytest.mark.parametrize("name", ["small_g256", "outlier_g64", "qkv_g256", "square_g256",
+                                  "skinny_m1_g64", "skinny_m16_g64", "skinny_m128_g64",
+                                  "skinny_m512_g64"])
+def test_workload_full_size_sampled(name):
+    lt = wl.make_workload(name)[0]
+    M, N = lt.x.shape[0], lt.w.shape[0]
+    _full_path_case(lt, lt.spec.group, rows=_sample(M, 48, 1), cols=_sample(N, 48, 2))
+
+
+def test_dit_mlp_pair_full_size_sampled():
+    up, down = wl.make_workload("dit_mlp_g256")
+    group = 256
+    rows = _sample(up.x.shape[0], 32, 3)
+    # up-projection, sampled
+    _full_path_case(up, group, rows=rows, cols=_sample(up.w.shape[0], 48, 4))
+    # down-projection: its input rows at the sampled positions are the
+    # oracle's own up-projection output; other rows are seeded noise of the
+    # same spread.  The GPU runs the full 1536 x 12288 -> 3072 layer.
+    xb = wl.bf16_bits(up.x)[rows]
+    px, sx = O.prepare_rows(xb, group)
+    pw, sw = O.prepare_rows(wl.bf16_bits(up.w), group)
+    h_rows = O.epilogue(O.gemm(px, pw, up.spec.K), sx, sw, wl.bf16_bits(up.b))
+    g = torch.Generator().manual_seed(11)
+    h = (torch.randn(up.x.shape[0], up.w.shape[0], generator=g) * 1.1).to(torch.bfloat16)
+    h_np = wl.bf16_bits(h).copy()
+    h_np[rows] = h_rows
+    down.x = torch.from_numpy(h_np.view(np.int16)).view(torch.bfloat16)
+    _full_path_case(down, group, rows=rows, cols=_sample(down.w.shape[0], 48, 5))
+
+
+# ---------------------------------------------------------------------------
+# failure detection without faulting the GPU
+# ---------------------------------------------------------------------------
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    assert cr.convrot_check_device_error() == 0
+    cr.convrot_debug_timeout_probe(2_000_000)      # 2 ms, nothing ever arrives
+    assert cr.convrot_check_device_error() == 7    # CONVROT_ERR_DEVICE_TIMEOUT
+    assert cr.convrot_check_device_error() == 0    # cleared
+    lt = _layer(8, 256, 32, 64, seed=1)
+    _full_path_case(lt, 64)
+
+
+def test_bad_arguments_raise():
+    x = torch.zeros(4, 1000, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(cr.ConvRotError) as e:
+        cr.convrot_prepare_act(x, 64)
+    assert e.value.status == 3
+    x = torch.zeros(4, 1024, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(cr.ConvRotError) as e:
+        cr.convrot_prepare_act(x, 32)
+    assert e.value.status == 2
+    misaligned = x.view(-1)[1:1025].view(1, 1024)      # starts 2 bytes past a boundary
+    with pytest.raises(cr.ConvRotError) as e:
+        cr.convrot_debug_rotate_f32(misaligned, 64)
+    assert e.value.status == 4
