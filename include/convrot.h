@@ -57,7 +57,8 @@ typedef enum {
     CONVROT_ERR_WORKSPACE = 5,       /* workspace smaller than required */
     CONVROT_ERR_CUDA = 6,            /* a CUDA runtime call or launch failed */
     CONVROT_ERR_DEVICE_TIMEOUT = 7,  /* a bounded device wait ran out */
-    CONVROT_ERR_UNSUPPORTED = 8      /* device is not sm_100 */
+    CONVROT_ERR_UNSUPPORTED = 8,     /* device is not sm_100 */
+    CONVROT_ERR_SCRATCH_LIMIT = 9    /* needs more than the built-in scratch array */
 } convrot_status;
 
 /* Human-readable name of a status (static storage, never NULL). */
@@ -121,6 +122,37 @@ convrot_status convrot_debug_rotate_f32(const void *x_bf16, int64_t M, int64_t K
  */
 convrot_status convrot_debug_gemm_s32(const uint8_t *qx, const uint8_t *qw, int64_t M, int64_t N,
                                       int64_t K, int32_t *acc, convrot_stream_t stream);
+
+/*
+ * The whole layer, like convrot_linear, for callers that cannot give the
+ * library any device memory of their own: a plugin called by a host runtime
+ * that owns every allocation and passes no workspace, or a caller on a
+ * latency-critical path that must not call cudaMalloc (it can synchronise the
+ * device and take milliseconds).  The pages have no counterpart to this
+ * entry point; it exists only for such callers.
+ *
+ * Instead of a caller-provided workspace it uses one fixed array of
+ * CONVROT_NOALLOC_SCRATCH_BYTES in the library's own device memory.  Every
+ * GPU that loads the library holds that array until the process exits.
+ * Requests needing more (round256(M*K/2) + round256(4*M) bytes, the same
+ * layout as convrot_linear_workspace_size) fail with
+ * CONVROT_ERR_SCRATCH_LIMIT before anything is launched; e.g. M = 4096 with
+ * K = 4096 fits (8 MiB), M = 8192 with K = 4096 (16 MiB + 32 KiB) does not.
+ *
+ * The array is shared by every call on a device and keeps the last call's
+ * contents; the prep kernel overwrites every byte the GEMM then reads, so
+ * nothing needs clearing between calls.  Calls whose work overlaps on the
+ * GPU (for example on two streams without ordering between them) race on the
+ * array and give undefined results: order them.  The first call on each
+ * device looks up the array's device address once (cudaGetSymbolAddress with
+ * that device current); make that first call before any stream capture.
+ * Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ * Arguments, layouts and errors are otherwise those of convrot_linear.
+ */
+#define CONVROT_NOALLOC_SCRATCH_BYTES (16u << 20)
+convrot_status convrot_linear_noalloc(const void *x_bf16, const uint8_t *qw, const float *sw,
+                                      const void *bias_bf16, int64_t M, int64_t N, int64_t K,
+                                      int group, void *y_bf16, convrot_stream_t stream);
 
 /*
  * Synchronises `stream`, then returns and clears the device error word of the

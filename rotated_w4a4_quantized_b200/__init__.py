@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libconvrot.so")
 STATUS = {
     0: "CONVROT_OK", 1: "CONVROT_ERR_NULL", 2: "CONVROT_ERR_GROUP", 3: "CONVROT_ERR_SHAPE",
     4: "CONVROT_ERR_ALIGN", 5: "CONVROT_ERR_WORKSPACE", 6: "CONVROT_ERR_CUDA",
-    7: "CONVROT_ERR_DEVICE_TIMEOUT", 8: "CONVROT_ERR_UNSUPPORTED",
+    7: "CONVROT_ERR_DEVICE_TIMEOUT", 8: "CONVROT_ERR_UNSUPPORTED", 9: "CONVROT_ERR_SCRATCH_LIMIT",
 }
 MAX_K = 32768
 
@@ -56,6 +56,7 @@ def lib() -> ctypes.CDLL:
             "convrot_debug_gemm_s32": [P, P, I64, I64, I64, P, P],
             "convrot_check_device_error": [P],
             "convrot_debug_timeout_probe": [I64, P],
+            "convrot_linear_noalloc": [P, P, P, P, I64, I64, I64, I, P, P],
         }
         for name, args in sigs.items():
             f = getattr(L, name)
@@ -131,6 +132,21 @@ def convrot_linear(x, qw, sw, bias, group: int, workspace=None, out=None, stream
     out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
     _check(lib().convrot_linear(_p(x), _p(qw), _p(sw), _p(bias), M, N, K, group, _p(workspace),
                                 workspace.numel(), _p(out), _stream(stream)), "convrot_linear")
+    return out
+
+
+def convrot_linear_noalloc(x, qw, sw, bias, group: int, out=None, stream=None):
+    """The whole layer without a caller workspace: the library's fixed
+    16 MiB scratch array holds the packed activations instead.  Meant for
+    callers that cannot allocate device memory (a plugin whose host runtime
+    owns every allocation, or a path that must not call cudaMalloc).  Calls
+    that overlap on the GPU share that array and race; order them."""
+    _need(x, torch.bfloat16, "x")
+    M, K = x.shape
+    N = qw.shape[0]
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
+    _check(lib().convrot_linear_noalloc(_p(x), _p(qw), _p(sw), _p(bias), M, N, K, group, _p(out),
+                                        _stream(stream)), "convrot_linear_noalloc")
     return out
 
 

@@ -7,6 +7,7 @@
 #include <stdint.h>
 #include <stdio.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/convrot.h"
@@ -194,6 +195,8 @@ const char *convrot_status_string(convrot_status s) {
         case CONVROT_ERR_CUDA: return "CONVROT_ERR_CUDA: a CUDA call or launch failed";
         case CONVROT_ERR_DEVICE_TIMEOUT: return "CONVROT_ERR_DEVICE_TIMEOUT: a bounded device wait ran out";
         case CONVROT_ERR_UNSUPPORTED: return "CONVROT_ERR_UNSUPPORTED: needs an sm_100 device";
+        case CONVROT_ERR_SCRATCH_LIMIT:
+            return "CONVROT_ERR_SCRATCH_LIMIT: larger than the built-in scratch array";
     }
     return "CONVROT_ERR_UNKNOWN";
 }
@@ -326,4 +329,66 @@ extern "C" convrot_status convrot_debug_timeout_probe(int64_t timeout_ns,
     if (timeout_ns > 5000000000ll) timeout_ns = 5000000000ll;
     timeout_probe_kernel<<<1, 32, 0, stream>>>(static_cast<uint64_t>(timeout_ns));
     return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// convrot_linear_noalloc: the whole layer with the library's own scratch.
+//
+// For callers that cannot hand out device memory (a plugin inside a runtime
+// that owns all allocations, or a path that must not call cudaMalloc because
+// it can synchronise the device).  The packed activation codes and scales
+// live in this fixed file-scope array instead of a caller's workspace.  In
+// host code `g_noalloc_scratch` names only a host-side stand-in for the
+// symbol, so its real device address is looked up once per device with
+// cudaGetSymbolAddress and that address is what the kernels receive.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_noalloc_scratch[CONVROT_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::atomic<void *> g_noalloc_addr[kMaxDevices];
+
+// Device address of the scratch array on `dev` (the current device).  The
+// first call on a device performs the lookup; it must not run during stream
+// capture.
+convrot_status noalloc_scratch(int dev, uint8_t **out) {
+    void *p = g_noalloc_addr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        std::lock_guard<std::mutex> lock(g_mu);
+        p = g_noalloc_addr[dev].load(std::memory_order_relaxed);
+        if (!p) {
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+                return CONVROT_ERR_CUDA;
+            g_noalloc_addr[dev].store(p, std::memory_order_release);
+        }
+    }
+    *out = static_cast<uint8_t *>(p);
+    return CONVROT_OK;
+}
+}  // namespace
+
+extern "C" convrot_status convrot_linear_noalloc(const void *x_bf16, const uint8_t *qw,
+                                                 const float *sw, const void *bias_bf16, int64_t M,
+                                                 int64_t N, int64_t K, int group, void *y_bf16,
+                                                 convrot_stream_t stream) {
+    convrot_status st = check_shape(M, K, group);
+    if (st != CONVROT_OK) return st;
+    if (N < 0) return CONVROT_ERR_SHAPE;
+    if (M == 0 || N == 0) return CONVROT_OK;
+    if (!x_bf16 || !qw || !sw || !y_bf16) return CONVROT_ERR_NULL;
+    if (!aligned16(x_bf16) || !aligned16(qw) || !aligned16(sw) || !aligned16(y_bf16) ||
+        (bias_bf16 && !aligned16(bias_bf16)))
+        return CONVROT_ERR_ALIGN;
+    if ((st = check_gemm_args(qw, qw, M, N, K)) != CONVROT_OK) return st;
+    if (convrot_linear_workspace_size(M, K) > CONVROT_NOALLOC_SCRATCH_BYTES)
+        return CONVROT_ERR_SCRATCH_LIMIT;
+    int dev;
+    if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    uint8_t *qx = nullptr;
+    if ((st = noalloc_scratch(dev, &qx)) != CONVROT_OK) return st;
+    // Every byte of qx and sx read by the GEMM is written by the prep kernel
+    // first, so leftovers of an earlier call never reach the result.
+    float *sx = reinterpret_cast<float *>(qx + round256(static_cast<size_t>(M) * (K / 2)));
+    if ((st = launch_prep(x_bf16, M, K, group, qx, sx, nullptr, stream)) != CONVROT_OK) return st;
+    return launch_gemm<false>(g_dev[dev].num_sms, qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16,
+                              stream);
 }
