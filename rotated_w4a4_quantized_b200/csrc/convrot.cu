@@ -75,16 +75,20 @@ convrot_status device_setup(int *dev_out) {
         g_encode = reinterpret_cast<EncodeTiledFn>(fn);
     }
     bool ok = true;
-    ok &= set_smem(gemm::gemm_kernel<256, false, false>, gemm::Cfg<256>::SMEM_BYTES);
-    ok &= set_smem(gemm::gemm_kernel<256, false, true>, gemm::Cfg<256>::SMEM_BYTES);
-    ok &= set_smem(gemm::gemm_kernel<16, true, false>, gemm::Cfg<16>::SMEM_BYTES);
-    ok &= set_smem(gemm::gemm_kernel<32, true, false>, gemm::Cfg<32>::SMEM_BYTES);
-    ok &= set_smem(gemm::gemm_kernel<64, true, false>, gemm::Cfg<64>::SMEM_BYTES);
-    ok &= set_smem(gemm::gemm_kernel<128, true, false>, gemm::Cfg<128>::SMEM_BYTES);
-    ok &= set_smem(gemm::gemm_kernel<16, true, true>, gemm::Cfg<16>::SMEM_BYTES);
-    ok &= set_smem(gemm::gemm_kernel<32, true, true>, gemm::Cfg<32>::SMEM_BYTES);
-    ok &= set_smem(gemm::gemm_kernel<64, true, true>, gemm::Cfg<64>::SMEM_BYTES);
-    ok &= set_smem(gemm::gemm_kernel<128, true, true>, gemm::Cfg<128>::SMEM_BYTES);
+    ok &= set_smem(prep::prep_kernel<64, 0>, CONVROT_MAX_K * 2);
+    ok &= set_smem(prep::prep_kernel<256, 0>, CONVROT_MAX_K * 2);
+    ok &= set_smem(prep::prep_kernel<64, 1>, CONVROT_MAX_K * 2);
+    ok &= set_smem(prep::prep_kernel<256, 1>, CONVROT_MAX_K * 2);
+    ok &= set_smem(gemm::gemm_kernel<256, false, false>, gemm::Cfg<256, false>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<256, false, true>, gemm::Cfg<256, false>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<16, true, false>, gemm::Cfg<16, true>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<32, true, false>, gemm::Cfg<32, true>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<64, true, false>, gemm::Cfg<64, true>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<128, true, false>, gemm::Cfg<128, true>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<16, true, true>, gemm::Cfg<16, true>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<32, true, true>, gemm::Cfg<32, true>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<64, true, true>, gemm::Cfg<64, true>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<128, true, true>, gemm::Cfg<128, true>::SMEM_BYTES);
     st.num_sms = sms;
     st.status = ok ? CONVROT_OK : CONVROT_ERR_CUDA;
     st.ready = true;
@@ -107,12 +111,13 @@ convrot_status launch_prep(const void *x, int64_t rows, int64_t K, int group, ui
     const dim3 block(static_cast<unsigned>(K / prep::kElemsPerThread));
     const uint16_t *xx = static_cast<const uint16_t *>(x);
     const int k = static_cast<int>(K);
+    const size_t smem = static_cast<size_t>(K) * 2;     // one bf16 row, staged
     if (yrot) {
-        if (group == 64) prep::prep_kernel<64, 1><<<grid, block, 0, stream>>>(xx, k, q, s, yrot);
-        else prep::prep_kernel<256, 1><<<grid, block, 0, stream>>>(xx, k, q, s, yrot);
+        if (group == 64) prep::prep_kernel<64, 1><<<grid, block, smem, stream>>>(xx, k, q, s, yrot);
+        else prep::prep_kernel<256, 1><<<grid, block, smem, stream>>>(xx, k, q, s, yrot);
     } else {
-        if (group == 64) prep::prep_kernel<64, 0><<<grid, block, 0, stream>>>(xx, k, q, s, yrot);
-        else prep::prep_kernel<256, 0><<<grid, block, 0, stream>>>(xx, k, q, s, yrot);
+        if (group == 64) prep::prep_kernel<64, 0><<<grid, block, smem, stream>>>(xx, k, q, s, yrot);
+        else prep::prep_kernel<256, 0><<<grid, block, smem, stream>>>(xx, k, q, s, yrot);
     }
     return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
@@ -128,19 +133,42 @@ bool make_map(CUtensorMap *map, const uint8_t *base, int64_t rows, int64_t K, in
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 output y [M][N] for the epilogue's TMA stores: 32 x 32 boxes,
+// 64-byte swizzle (needs N % 8 == 0 so that rows start 16-byte aligned).
+bool make_out_map(CUtensorMap *map, void *y, int64_t M, int64_t N) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(gemm::kStoreBox),
+                               static_cast<cuuint32_t>(gemm::kStoreBox)};
+    const cuuint32_t estr[2] = {1, 1};
+    return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int BN, bool SWAP, bool OUT_S32>
 convrot_status launch_gemm_cfg(int num_sms, const uint8_t *qA, const uint8_t *qB, int64_t rowsA,
                                int64_t rowsB, int64_t K, const float *sx, const float *sw,
                                const void *bias, void *out, int64_t M, int64_t N,
                                cudaStream_t stream) {
-    CUtensorMap tmA, tmB;
+    CUtensorMap tmA, tmB, tmY;
     if (!make_map(&tmA, qA, rowsA, K, gemm::BM) || !make_map(&tmB, qB, rowsB, K, BN))
         return CONVROT_ERR_CUDA;
+    int use_tma_store = 0;
+    if (!SWAP && !OUT_S32 && N % 8 == 0) {
+        if (!make_out_map(&tmY, out, M, N)) return CONVROT_ERR_CUDA;
+        use_tma_store = 1;
+    } else {
+        tmY = tmA;   // unused by the kernel
+    }
     const int64_t tiles = ((rowsA + gemm::BM - 1) / gemm::BM) * ((rowsB + BN - 1) / BN);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-    gemm::gemm_kernel<BN, SWAP, OUT_S32><<<grid, gemm::kThreads, gemm::Cfg<BN>::SMEM_BYTES, stream>>>(
-        tmA, tmB, static_cast<int>(rowsA), static_cast<int>(rowsB), static_cast<int>(K), sx, sw,
-        static_cast<const uint16_t *>(bias), out, static_cast<int>(M), static_cast<int>(N));
+    gemm::gemm_kernel<BN, SWAP, OUT_S32>
+        <<<grid, gemm::kThreads, gemm::Cfg<BN, SWAP>::SMEM_BYTES, stream>>>(
+            tmA, tmB, tmY, use_tma_store, static_cast<int>(rowsA), static_cast<int>(rowsB),
+            static_cast<int>(K), sx, sw, static_cast<const uint16_t *>(bias), out,
+            static_cast<int>(M), static_cast<int>(N));
     return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 

@@ -19,22 +19,27 @@
 // unchanged.
 //
 // CTA organisation (one CTA per SM, persistent over output tiles):
-//   warp 0       TMA producer: packed A [128 x 64 B] and B [BN x 64 B] tiles
-//                per K-block into a ring of packed stages;
-//   warp 1       TMEM allocator and MMA issuer (one thread): 4 MMAs of K = 32
-//                per K-block into one of two TMEM accumulators;
-//   warps 2..5   epilogue: tcgen05.ld, shift, scale, bias, bf16, store;
-//   warps 6..13  widening: packed stage -> int8 stage in the 128-byte
-//                swizzled K-major layout the MMA descriptors describe.
+//   warp 0        TMA producer: packed A [128 x 64 B] and B [BN x 64 B] tiles
+//                 per K-block into a ring of packed stages;
+//   warp 1        TMEM allocator and MMA issuer (one thread): 4 MMAs of K = 32
+//                 per K-block into one of two TMEM accumulators;
+//   warps 2..9    epilogue, two warps per TMEM lane quarter (each takes half
+//                 of the tile's columns): tcgen05.ld, shift, scale, bias,
+//                 bf16; full tiles leave through a swizzled shared-memory
+//                 box and a TMA store;
+//   warps 10..17  widening: packed stage -> int8 stage in the 128-byte
+//                 swizzled K-major layout the MMA descriptors describe.
 // Accumulators are double-buffered in TMEM so the epilogue of one tile runs
 // under the main loop of the next.
 //
 // SWAP selects the skinny-M form: the weights become the 128-row MMA operand
 // and the few token rows the N-side operand (BN = 16 .. 128), so the weight
-// stream is split over many CTAs; the epilogue writes the transposed tile.
+// stream is split over many CTAs; the epilogue writes the transposed tile
+// with direct stores.
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 #include "ptx.cuh"
@@ -44,22 +49,28 @@ namespace gemm {
 constexpr int BM = 128;          // MMA M: rows of operand A per tile
 constexpr int BKP = 64;          // packed bytes per row per K-block
 constexpr int BK = 128;          // int8 values per row per K-block
-constexpr int kThreads = 448;    // 14 warps
-constexpr int kWarpTma = 0, kWarpMma = 1, kWarpEpi0 = 2, kWarpUnp0 = 6;
-constexpr int kUnpWarps = 8;
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpEpi0 = 2, kEpiWarps = 8;
+constexpr int kWarpUnp0 = kWarpEpi0 + kEpiWarps, kUnpWarps = 8;
+constexpr int kThreads = (kWarpUnp0 + kUnpWarps) * 32;    // 576
+constexpr int kStoreBox = 32;    // epilogue TMA-store box: 32 rows x 32 bf16
 
-template <int BN>
+template <int BN, bool SWAP>
 struct Cfg {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "kind::i8 with M=128 needs N%16==0");
-    static constexpr int SP = (BN == 256) ? 3 : 4;     // packed stages
-    static constexpr int SU = (BN == 256) ? 3 : 4;     // widened stages
+    // Packed stages keep HBM loads in flight; the narrow (skinny) tiles are
+    // bound by the weight stream, so they trade widened stages for more
+    // packed ones.  The wide tile keeps room for the epilogue's store boxes.
+    static constexpr int SP = BN == 256 ? 4 : BN == 128 ? 6 : BN == 64 ? 10 : 12;
+    static constexpr int SU = BN == 256 ? 2 : 3;
     static constexpr int PA = BM * BKP;
     static constexpr int PB = BN * BKP;
     static constexpr int UA = BM * BK;
     static constexpr int UB = BN * BK;
+    static constexpr int ST = SWAP ? 0 : kEpiWarps * 2 * kStoreBox * kStoreBox * 2;  // store boxes
     static constexpr int OFF_UA = 0;                   // 1024-aligned tiles first
     static constexpr int OFF_UB = OFF_UA + SU * UA;
-    static constexpr int OFF_PA = OFF_UB + SU * UB;
+    static constexpr int OFF_ST = OFF_UB + SU * UB;
+    static constexpr int OFF_PA = OFF_ST + ST;
     static constexpr int OFF_PB = OFF_PA + SP * PA;
     static constexpr int OFF_BAR = OFF_PB + SP * PB;
     static constexpr int NUM_BARS = 2 * SP + 2 * SU + 5;
@@ -71,6 +82,7 @@ struct Cfg {
     static constexpr int TMEM_COLS = 2 * ACC_STRIDE;        // 64 .. 512, a power of two
     static constexpr int JW = BN < 32 ? BN : 32;             // valid columns per 32-wide read
     static_assert(UB % 1024 == 0, "widened B tiles must stay 1024-aligned");
+    static_assert(ST % 1024 == 0, "store boxes must stay 1024-aligned");
     static_assert(SMEM_BYTES <= 232448, "exceeds the per-CTA shared memory limit");
 };
 
@@ -106,14 +118,32 @@ __device__ __forceinline__ float epi(uint32_t raw, float sx, float sw, float b) 
     return __fadd_rn(t, b);
 }
 
+// The same arithmetic for two adjacent columns, returning their bf16 pair
+// (low half = first column).  float(acc) is formed exactly without the
+// conversion unit: for |acc| < 2^22 the bit pattern 0x4B400000 + acc is the
+// float 1.5 * 2^23 + acc, and subtracting 1.5 * 2^23 is exact.
+__device__ __forceinline__ uint32_t epi_pair(uint32_t r0, uint32_t r1, float sx, float sw0,
+                                             float sw1, float b0, float b1) {
+    float f0 = __int_as_float((static_cast<int>(r0) >> 8) + 0x4B400000);
+    float f1 = __int_as_float((static_cast<int>(r1) >> 8) + 0x4B400000);
+    ptx::add2(f0, f1, f0, f1, -12582912.0f, -12582912.0f);
+    ptx::mul2(f0, f1, f0, f1, sx, sx);
+    ptx::mul2(f0, f1, f0, f1, sw0, sw1);
+    ptx::add2(f0, f1, f0, f1, b0, b1);
+    const __nv_bfloat162 h = __floats2bfloat162_rn(f0, f1);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
 // OUT_S32: write the integer accumulators (test hook) instead of bf16.
+// tmY (used when !SWAP && !OUT_S32 && use_tma_store): bf16 y [M][N], box
+// 32 x 32, 64-byte swizzle.
 template <int BN, bool SWAP, bool OUT_S32>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-            int rowsA, int rowsB, int K, const float *__restrict__ sx,
-            const float *__restrict__ sw, const uint16_t *__restrict__ bias,
-            void *__restrict__ out, int M, int N) {
-    using C = Cfg<BN>;
+            const __grid_constant__ CUtensorMap tmY, int use_tma_store, int rowsA, int rowsB,
+            int K, const float *__restrict__ sx, const float *__restrict__ sw,
+            const uint16_t *__restrict__ bias, void *__restrict__ out, int M, int N) {
+    using C = Cfg<BN, SWAP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -142,7 +172,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(acc_full(b), 1);
-            ptx::mbar_init(acc_empty(b), 4);
+            ptx::mbar_init(acc_empty(b), kEpiWarps);
         }
         ptx::mbar_init(drain_bar, 1);
         *abort_flag = 0;
@@ -151,6 +181,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     if (warp == kWarpTma && lane == 0) {
         ptx::tma_prefetch_desc(&tmA);
         ptx::tma_prefetch_desc(&tmB);
+        if (!SWAP && !OUT_S32 && use_tma_store) ptx::tma_prefetch_desc(&tmY);
     }
     if (warp == kWarpMma) {
         ptx::tmem_alloc(sbase + C::OFF_MISC, C::TMEM_COLS);
@@ -224,9 +255,18 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             volatile int never = 0;
             ptx::mbar_wait(drain_bar, 0, &never, 100000000ull);
         }
-    } else if (warp < kWarpEpi0 + 4) {
+    } else if (warp < kWarpUnp0) {
+        // ------------------------------------------------------------ epilogue
+        const int e = warp - kWarpEpi0;               // 0 .. 7
         const int quarter = warp & 3;                 // TMEM lanes 32*quarter ..
+        const int half = e >> 2;                      // which half of the columns
         const int r = quarter * 32 + lane;            // row of the accumulator tile
+        constexpr int kCols = BN >= 64 ? BN / 2 : BN; // columns this warp covers
+        const int col_begin = BN >= 64 ? half * kCols : 0;
+        const bool active = BN >= 64 || half == 0;
+        const bool tma_out = !SWAP && !OUT_S32 && use_tma_store;
+        const uint32_t box0 = sbase + C::OFF_ST + e * (2 * kStoreBox * kStoreBox * 2);
+        int nstores = 0;
         int local = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             const int ta = tile % tiles_a, tb = tile / tiles_a;
@@ -235,44 +275,78 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             if (!ptx::mbar_wait(acc_full(b), aph, abort_flag)) break;
             ptx::tc_fence_after();
             const int arow = ta * BM + r;             // A row of this lane
+            if (active) {
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                uint32_t v[32];
-                __syncwarp();   // tcgen05.ld is warp-collective
-                ptx::tmem_ld_32x32b_x32(
-                    tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                        static_cast<uint32_t>(b * C::ACC_STRIDE + c0),
-                    v);
-                ptx::tmem_ld_wait();
-                const int bcol0 = tb * BN + c0;       // first B row of these 32 columns
-                if (!SWAP) {
-                    // lane = output row m, columns = output columns n
-                    const int m = arow;
-                    if (m >= M) continue;
-                    const int n0 = bcol0;
-                    if (OUT_S32) {
-                        int32_t *o = reinterpret_cast<int32_t *>(out) + static_cast<size_t>(m) * N;
-                        for (int j = 0; j < C::JW; ++j)
-                            if (n0 + j < N) o[n0 + j] = static_cast<int32_t>(v[j]) >> 8;
-                    } else {
-                        const float sxm = sx[m];
-                        uint16_t *o = reinterpret_cast<uint16_t *>(out) + static_cast<size_t>(m) * N;
-                        if (C::JW == 32 && n0 + 32 <= N && (N & 7) == 0) {
-                            uint32_t pk[16];
+                for (int c0 = col_begin; c0 < col_begin + kCols; c0 += 32) {
+                    const int bcol0 = tb * BN + c0;   // first B row of these 32 columns
+                    uint32_t v[32];
+                    __syncwarp();   // tcgen05.ld is warp-collective
+                    ptx::tmem_ld_32x32b_x32(
+                        tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                            static_cast<uint32_t>(b * C::ACC_STRIDE + c0),
+                        v);
+                    ptx::tmem_ld_wait();
+                    if (!SWAP && !OUT_S32 && tma_out) {
+                        // 32 rows x 32 columns through a swizzled box, one TMA store
+                        const int n0 = bcol0;
+                        const bool full_cols = n0 + 32 <= N;
+                        const float sxm = arow < M ? sx[arow] : 0.0f;
+                        uint32_t pk[16];
+                        if (full_cols) {
+                            const float4 *s4 = reinterpret_cast<const float4 *>(sw + n0);
+                            const uint4 *b4 = reinterpret_cast<const uint4 *>(bias + n0);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const float4 fa = __ldg(s4 + 2 * i), fb = __ldg(s4 + 2 * i + 1);
+                                const uint4 u = bias ? __ldg(b4 + i) : make_uint4(0, 0, 0, 0);
+                                const uint32_t bw[4] = {u.x, u.y, u.z, u.w};
+                                const float swv[8] = {fa.x, fa.y, fa.z, fa.w, fb.x, fb.y, fb.z, fb.w};
+#pragma unroll
+                                for (int j = 0; j < 4; ++j)
+                                    pk[4 * i + j] = epi_pair(v[8 * i + 2 * j], v[8 * i + 2 * j + 1], sxm,
+                                                             swv[2 * j], swv[2 * j + 1],
+                                                             __uint_as_float(bw[j] << 16),
+                                                             __uint_as_float(bw[j] & 0xFFFF0000u));
+                            }
+                        } else {
 #pragma unroll
                             for (int j = 0; j < 32; j += 2) {
-                                const float b0 = bias ? bf16_to_f32(bias[n0 + j]) : 0.0f;
-                                const float b1 = bias ? bf16_to_f32(bias[n0 + j + 1]) : 0.0f;
-                                const uint16_t h0 = f32_to_bf16_rne(epi(v[j], sxm, sw[n0 + j], b0));
-                                const uint16_t h1 =
-                                    f32_to_bf16_rne(epi(v[j + 1], sxm, sw[n0 + j + 1], b1));
-                                pk[j / 2] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+                                const int n = n0 + j;
+                                const float s0 = n < N ? sw[n] : 0.0f;
+                                const float s1 = n + 1 < N ? sw[n + 1] : 0.0f;
+                                const float b0 = (bias && n < N) ? bf16_to_f32(bias[n]) : 0.0f;
+                                const float b1 = (bias && n + 1 < N) ? bf16_to_f32(bias[n + 1]) : 0.0f;
+                                pk[j / 2] = epi_pair(v[j], v[j + 1], sxm, s0, s1, b0, b1);
                             }
-                            uint4 *o4 = reinterpret_cast<uint4 *>(o + n0);
+                        }
+                        const uint32_t box = box0 + (nstores & 1) * (kStoreBox * kStoreBox * 2);
+                        if (lane == 0) ptx::bulk_wait_read<1>();   // this box's previous store
+                        __syncwarp();
 #pragma unroll
-                            for (int i = 0; i < 4; ++i)
-                                o4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                        for (int c = 0; c < 4; ++c) {
+                            const uint32_t sw16 = static_cast<uint32_t>(c ^ ((lane >> 1) & 3));
+                            sts128(box + lane * 64 + sw16 * 16, pk[4 * c], pk[4 * c + 1],
+                                   pk[4 * c + 2], pk[4 * c + 3]);
+                        }
+                        ptx::fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            ptx::tma_store_2d(&tmY, box, n0, ta * BM + quarter * 32);
+                            ptx::bulk_commit();
+                        }
+                        ++nstores;
+                    } else if (!SWAP) {
+                        // lane = output row m, columns = output columns n
+                        const int m = arow;
+                        if (m >= M) continue;
+                        const int n0 = bcol0;
+                        if (OUT_S32) {
+                            int32_t *o = reinterpret_cast<int32_t *>(out) + static_cast<size_t>(m) * N;
+                            for (int j = 0; j < C::JW; ++j)
+                                if (n0 + j < N) o[n0 + j] = static_cast<int32_t>(v[j]) >> 8;
                         } else {
+                            const float sxm = sx[m];
+                            uint16_t *o = reinterpret_cast<uint16_t *>(out) + static_cast<size_t>(m) * N;
                             for (int j = 0; j < C::JW; ++j) {
                                 const int n = n0 + j;
                                 if (n >= N) break;
@@ -280,26 +354,27 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                                 o[n] = f32_to_bf16_rne(epi(v[j], sxm, sw[n], bb));
                             }
                         }
-                    }
-                } else {
-                    // lane = output column n (a weight row), columns = tokens m
-                    const int n = arow;
-                    if (n >= N) continue;
-                    if (OUT_S32) {
-                        int32_t *o = reinterpret_cast<int32_t *>(out);
-                        for (int j = 0; j < C::JW; ++j) {
-                            const int m = bcol0 + j;
-                            if (m >= M) break;
-                            o[static_cast<size_t>(m) * N + n] = static_cast<int32_t>(v[j]) >> 8;
-                        }
                     } else {
-                        const float swn = sw[n];
-                        const float bn = bias ? bf16_to_f32(bias[n]) : 0.0f;
-                        uint16_t *o = reinterpret_cast<uint16_t *>(out);
-                        for (int j = 0; j < C::JW; ++j) {
-                            const int m = bcol0 + j;
-                            if (m >= M) break;
-                            o[static_cast<size_t>(m) * N + n] = f32_to_bf16_rne(epi(v[j], sx[m], swn, bn));
+                        // lane = output column n (a weight row), columns = tokens m
+                        const int n = arow;
+                        if (n >= N) continue;
+                        if (OUT_S32) {
+                            int32_t *o = reinterpret_cast<int32_t *>(out);
+                            for (int j = 0; j < C::JW; ++j) {
+                                const int m = bcol0 + j;
+                                if (m >= M) break;
+                                o[static_cast<size_t>(m) * N + n] = static_cast<int32_t>(v[j]) >> 8;
+                            }
+                        } else {
+                            const float swn = sw[n];
+                            const float bn = bias ? bf16_to_f32(bias[n]) : 0.0f;
+                            uint16_t *o = reinterpret_cast<uint16_t *>(out);
+                            for (int j = 0; j < C::JW; ++j) {
+                                const int m = bcol0 + j;
+                                if (m >= M) break;
+                                o[static_cast<size_t>(m) * N + n] =
+                                    f32_to_bf16_rne(epi(v[j], sx[m], swn, bn));
+                            }
                         }
                     }
                 }
@@ -308,10 +383,19 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(acc_empty(b));
         }
+        if (tma_out && lane == 0) ptx::bulk_wait_all();
     } else {
-        // widening warps
+        // ------------------------------------------------------------ widening
+        // Thread ut widens 16-byte packed chunks ut, ut + 256, ...; since 256 is
+        // a multiple of 4 chunks per row and of 8 rows per swizzle group, its
+        // chunk column and swizzle phase are the same for every one of them.
         const int ut = threadIdx.x - kWarpUnp0 * 32;   // 0 .. 255
         constexpr int kChunks = (BM + BN) * 4;          // 16-byte packed chunks per stage
+        constexpr int kPer = (kChunks + kUnpWarps * 32 - 1) / (kUnpWarps * 32);
+        const uint32_t c = static_cast<uint32_t>(ut & 3);
+        const uint32_t sw8 = static_cast<uint32_t>((ut >> 2) & 7);
+        const uint32_t lo_off = ((2u * c) ^ sw8) << 4;
+        const uint32_t hi_off = ((2u * c + 1u) ^ sw8) << 4;
         int ps = 0, us = 0;
         uint32_t pph = 0, uph = 0;
         bool ok = true;
@@ -323,20 +407,25 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 const uint32_t pb = sbase + C::OFF_PB + ps * C::PB;
                 const uint32_t ua = sbase + C::OFF_UA + us * C::UA;
                 const uint32_t ub = sbase + C::OFF_UB + us * C::UB;
-#pragma unroll 2
-                for (int idx = ut; idx < kChunks; idx += kUnpWarps * 32) {
-                    const int row = idx >> 2, c = idx & 3;
-                    const bool in_a = row < BM;
-                    const int rr = in_a ? row : row - BM;
-                    const uint32_t src = (in_a ? pa : pb) + rr * 64 + c * 16;
-                    const uint32_t dst = (in_a ? ua : ub) + rr * 128;
-                    const uint32_t sw8 = static_cast<uint32_t>(rr & 7);
-                    const uint4 w = lds128(src);
-                    const uint32_t hm = 0xF0F0F0F0u;
-                    sts128(dst + (((2u * c) ^ sw8) << 4), (w.x << 4) & hm, (w.y << 4) & hm,
-                           (w.z << 4) & hm, (w.w << 4) & hm);
-                    sts128(dst + (((2u * c + 1u) ^ sw8) << 4), w.x & hm, w.y & hm, w.z & hm,
-                           w.w & hm);
+                uint4 w[kPer];
+#pragma unroll
+                for (int i = 0; i < kPer; ++i) {
+                    const int row = (ut >> 2) + 64 * i;   // rows of A, then rows of B
+                    if (row < BM + BN) {
+                        const uint32_t src = row < BM ? pa + row * 64 : pb + (row - BM) * 64;
+                        w[i] = lds128(src + c * 16);
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < kPer; ++i) {
+                    const int row = (ut >> 2) + 64 * i;
+                    if (row < BM + BN) {
+                        const uint32_t dst = row < BM ? ua + row * 128 : ub + (row - BM) * 128;
+                        const uint32_t hm = 0xF0F0F0F0u;
+                        sts128(dst + lo_off, (w[i].x << 4) & hm, (w[i].y << 4) & hm,
+                               (w[i].z << 4) & hm, (w[i].w << 4) & hm);
+                        sts128(dst + hi_off, w[i].x & hm, w[i].y & hm, w[i].z & hm, w[i].w & hm);
+                    }
                 }
                 ptx::fence_proxy_async_smem();
                 __syncwarp();

@@ -21,15 +21,22 @@
 //   v = u * inv, q = round_half_away(v).
 // Because 2^-k scaling is exact, u * (7 / a_u) is bit-identical to
 // y * (7 / max|y|).  round_half_away(v) for |v| < 8 is computed as
-// trunc(|v| + (0.5 - 2^-25)) with the sign of v: adding the largest float
-// below 0.5 (instead of 0.5) is exactly round-half-away-from-zero on fp32
-// inputs of this range, and |v| <= 7 (1 + 2^-24) by construction, so no
-// clamp is needed.  Codes are packed two per byte, low nibble = even channel.
+// trunc(v + sign(v) (0.5 - 2^-25)): adding the largest float below 0.5
+// (instead of 0.5) is exactly round-half-away-from-zero on fp32 inputs of
+// this range (IEEE addition is symmetric in sign), and |v| <= 7 (1 + 2^-24)
+// by construction, so no clamp is needed.  Codes are packed two per byte,
+// low nibble = even channel.
 #pragma once
 
 #include <stdint.h>
 
+#include "ptx.cuh"
+
 namespace prep {
+
+using ptx::add2;
+using ptx::bfly2;
+using ptx::mul2;
 
 constexpr int kElemsPerThread = 64;
 constexpr int kMaxThreads = 512;   // K <= 32768
@@ -42,29 +49,42 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4 *p) {
     return r;
 }
 
-// One radix-4 butterfly stage along the digit whose stride is S (1, 4, 16).
-template <int S>
-__device__ __forceinline__ void radix4_stage(float (&v)[kElemsPerThread]) {
-#pragma unroll
-    for (int b = 0; b < kElemsPerThread; ++b) {
-        if ((b / S) % 4 != 0) continue;
-        const float a0 = v[b], a1 = v[b + S], a2 = v[b + 2 * S], a3 = v[b + 3 * S];
-        const float sum = (a0 + a1) + (a2 + a3);
-        v[b] = fmaf(-2.0f, a0, sum);
-        v[b + S] = fmaf(-2.0f, a1, sum);
-        v[b + 2 * S] = fmaf(-2.0f, a2, sum);
-        v[b + 3 * S] = fmaf(-2.0f, a3, sum);
-    }
+// Two signed codes into one byte of the running word:
+// result = (acc << 8) | ((hi & 0xF) << 4) | (lo & 0xF), saturating to [-8, 7]
+// (codes here are already in [-7, 7]).
+__device__ __forceinline__ uint32_t pack_nibbles(int hi, int lo, uint32_t acc) {
+    uint32_t d;
+    asm("cvt.pack.sat.s4.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(hi), "r"(lo), "r"(acc));
+    return d;
 }
 
-__device__ __forceinline__ int quant_code(float u, float inv) {
-    const float v = __fmul_rn(u, inv);
-    const float mag = __fadd_rn(fabsf(v), __int_as_float(0x3EFFFFFF));   // 0.5 - 2^-25
-    return __float2int_rz(copysignf(mag, v));
+// One radix-4 butterfly stage along the digit whose stride is S (1, 4, 16),
+// two quadruples at a time.  Quadruples start at the indices b whose digit of
+// stride S is 0; they are paired as (b, b + P) with P = 4 for S = 1 and
+// P = 1 otherwise, so both members of a pair are quadruple starts.
+template <int S>
+__device__ __forceinline__ void radix4_stage(float (&v)[kElemsPerThread]) {
+    constexpr int P = (S == 1) ? 4 : 1;
+#pragma unroll
+    for (int b = 0; b < kElemsPerThread; ++b) {
+        if ((b / S) % 4 != 0 || (b / P) % 2 != 0) continue;
+        const int c = b + P;
+        float s01a, s01b, s23a, s23b, suma, sumb;
+        add2(s01a, s01b, v[b], v[c], v[b + S], v[c + S]);
+        add2(s23a, s23b, v[b + 2 * S], v[c + 2 * S], v[b + 3 * S], v[c + 3 * S]);
+        add2(suma, sumb, s01a, s01b, s23a, s23b);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) bfly2(v[b + j * S], v[c + j * S], suma, sumb);
+    }
 }
 
 // MODE 0: quantise + pack (q, s).  MODE 1: write the normalised rotated row
 // as fp32 (yrot) instead.
+//
+// Loads: the row is read with coalesced 128-bit loads (consecutive threads,
+// consecutive 16-byte chunks) and written to shared memory so that chunk c of
+// thread t's 128-byte slice sits at position c ^ (t mod 8); each thread then
+// reads its own 64 channels back with conflict-free 128-bit loads.
 template <int G, int MODE>
 __global__ void __launch_bounds__(kMaxThreads)
 prep_kernel(const uint16_t *__restrict__ x, int K, uint8_t *__restrict__ q,
@@ -73,24 +93,35 @@ prep_kernel(const uint16_t *__restrict__ x, int K, uint8_t *__restrict__ q,
     constexpr int kDigits = (G == 64) ? 3 : 4;
     constexpr float kNorm = (G == 64) ? 0.125f : 0.0625f;   // 2^-kDigits
 
+    extern __shared__ uint4 stage[];                     // K * 2 bytes
     __shared__ uint32_t red[kMaxThreads / 32];
 
     const int row = blockIdx.x;
     const int t = threadIdx.x;
-    const int nthreads = blockDim.x;
+    const int nthreads = blockDim.x;                     // K / 64
     const int warp = t >> 5, lane = t & 31;
     const int warp_lanes = min(32, nthreads - warp * 32);
     const uint32_t mask = warp_lanes == 32 ? 0xFFFFFFFFu : ((1u << warp_lanes) - 1u);
 
-    const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(row) * K) + t * 8;
-    uint4 raw[8];
+    {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(row) * K);
+        uint4 r[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) raw[i] = ldg_stream(src + i);
+        for (int j = 0; j < 8; ++j) r[j] = ldg_stream(src + t + j * nthreads);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int g = t + j * nthreads;              // chunk index in the row
+            const int owner = g >> 3, c = g & 7;
+            stage[owner * 8 + (c ^ (owner & 7))] = r[j];
+        }
+    }
+    __syncthreads();
 
     float v[kElemsPerThread];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+        const uint4 raw = stage[t * 8 + (i ^ (t & 7))];
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
@@ -104,10 +135,12 @@ prep_kernel(const uint16_t *__restrict__ x, int K, uint8_t *__restrict__ q,
     if (kDigits == 4) {
         // digit 3 = lane bits 0..1: the 4 threads of this 256-channel group
 #pragma unroll
-        for (int e = 0; e < kElemsPerThread; ++e) {
-            float sum = v[e] + __shfl_xor_sync(mask, v[e], 1);
-            sum = sum + __shfl_xor_sync(mask, sum, 2);
-            v[e] = fmaf(-2.0f, v[e], sum);
+        for (int e = 0; e < kElemsPerThread; e += 2) {
+            float s0, s1;
+            add2(s0, s1, v[e], v[e + 1], __shfl_xor_sync(mask, v[e], 1),
+                 __shfl_xor_sync(mask, v[e + 1], 1));
+            add2(s0, s1, s0, s1, __shfl_xor_sync(mask, s0, 2), __shfl_xor_sync(mask, s1, 2));
+            bfly2(v[e], v[e + 1], s0, s1);
         }
     }
 
@@ -137,11 +170,22 @@ prep_kernel(const uint16_t *__restrict__ x, int K, uint8_t *__restrict__ q,
     uint32_t packed[8];
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
-        uint32_t word = 0;
+        int code[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            word |= (static_cast<uint32_t>(quant_code(v[8 * w + j], inv)) & 0xFu) << (4 * j);
-        packed[w] = word;
+        for (int j = 0; j < 8; j += 2) {
+            float p0, p1, h0, h1;
+            mul2(p0, p1, v[8 * w + j], v[8 * w + j + 1], inv, inv);
+            // add (0.5 - 2^-25) with the sign of the product, truncate
+            const float c0 = __uint_as_float((__float_as_uint(p0) & 0x80000000u) | 0x3EFFFFFFu);
+            const float c1 = __uint_as_float((__float_as_uint(p1) & 0x80000000u) | 0x3EFFFFFFu);
+            add2(h0, h1, p0, p1, c0, c1);
+            code[j] = __float2int_rz(h0);
+            code[j + 1] = __float2int_rz(h1);
+        }
+        uint32_t word = pack_nibbles(code[7], code[6], 0u);
+        word = pack_nibbles(code[5], code[4], word);
+        word = pack_nibbles(code[3], code[2], word);
+        packed[w] = pack_nibbles(code[1], code[0], word);
     }
     uint4 *dst = reinterpret_cast<uint4 *>(q + static_cast<size_t>(row) * (K / 2)) + t * 2;
     dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
