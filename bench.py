@@ -2,14 +2,17 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
-One step is one pass of the whole path over one batch: the fused prep kernel
-(rotation, rowwise absmax INT4 quantisation, packing) and the tcgen05 GEMM
-with its scale/bias/bf16 epilogue (two kernels per linear layer).  Weights are
-prepared once before timing (the offline step).  The L2 cache is flushed
-(a 256 MiB write) before every timed step, outside the timed interval; each
-step is bracketed by CUDA events on the launching stream.  Under torchrun
-every rank runs its own batch (weak scaling, no collective on the data path);
-the reported time is the maximum over ranks.
+One step is one pass of the whole path over one batch through the public
+call convrot_linear: the fused prep kernel (rotation, rowwise absmax INT4
+quantisation, packing) and the tcgen05 GEMM with its scale/bias/bf16
+epilogue (two kernels per linear layer).  Weights are prepared once before
+timing (the offline step).  The L2 cache is flushed (a 256 MiB write) before
+every timed step, outside the timed interval; each step is bracketed by CUDA
+events on the launching stream.  A second pass of the same number of steps
+runs the two kernels through the split calls with an event between them to
+time each kernel for the roofline.  Under torchrun every rank runs its own
+batch (weak scaling, no collective on the data path); the reported time is
+the maximum over ranks.
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
 instead, on bounded samples of the same workload, on the host cores.
@@ -184,29 +187,34 @@ def run_gpu(args):
         del w
         prepared.append((lt.spec, qw, sw, b))
     x0 = layers[0].x.to(dev)
-    acts, ws = [], []
+    acts, ws, lws = [], [], []
     for i, (sp, qw, sw, b) in enumerate(prepared):
         acts.append(x0 if i == 0 else torch.empty(sp.M, sp.K, dtype=torch.bfloat16, device=dev))
         ws.append((torch.empty(sp.M, sp.K // 2, dtype=torch.uint8, device=dev),
                    torch.empty(sp.M, dtype=torch.float32, device=dev)))
+        lws.append(torch.empty(max(1, cr.convrot_linear_workspace_size(sp.M, sp.K)),
+                               dtype=torch.uint8, device=dev))
     outs = [torch.empty(sp.M, sp.N, dtype=torch.bfloat16, device=dev) for sp, *_ in prepared]
     for i in range(1, len(prepared)):
         acts[i] = outs[i - 1]          # chained layers: next input is this output
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     nl = len(prepared)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nl + 1)] for _ in range(args.steps)]
 
-    def step(events=None):
+    def step():
+        # the public whole-layer call: prep kernel + GEMM kernel per layer
         for i, (sp, qw, sw, b) in enumerate(prepared):
-            if events is not None:
-                events[2 * i].record(stream)
+            cr.convrot_linear(acts[i], qw, sw, b, sp.group, lws[i], outs[i])
+
+    def step_split(events):
+        # the same two kernels through the split calls, with an event between
+        # them, to time each kernel on its own
+        for i, (sp, qw, sw, b) in enumerate(prepared):
+            events[2 * i].record(stream)
             cr.convrot_prepare_act(acts[i], sp.group, ws[i][0], ws[i][1])
-            if events is not None:
-                events[2 * i + 1].record(stream)
+            events[2 * i + 1].record(stream)
             cr.convrot_linear_prepared(ws[i][0], ws[i][1], qw, sw, b, sp.K, out=outs[i])
-        if events is not None:
-            events[2 * nl].record(stream)
+        events[2 * nl].record(stream)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -215,6 +223,9 @@ def run_gpu(args):
     if cr.convrot_check_device_error() != 0:
         raise RuntimeError("device error during warm-up")
 
+    # timed region: whole steps, L2 flushed before each (outside the interval)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -225,7 +236,9 @@ def run_gpu(args):
     with ClockSampler(gpu_id) as clocks:
         for k in range(args.steps):
             flush.zero_()
-            step(ev[k])
+            ev[k][0].record(stream)
+            step()
+            ev[k][1].record(stream)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -233,8 +246,16 @@ def run_gpu(args):
     status = cr.convrot_check_device_error()
     if status != 0:
         raise RuntimeError(f"device error status {status} in the timed region")
+    step_ms = [a.elapsed_time(b) for a, b in ev]
 
-    step_ms = [e[0].elapsed_time(e[-1]) for e in ev]
+    # per-kernel durations over the same number of steps
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nl + 1)]
+           for _ in range(args.steps)]
+    for k in range(args.steps):
+        flush.zero_()
+        step_split(kev[k])
+    torch.cuda.synchronize()
+    ev = kev
     prep_ms = [[e[2 * i].elapsed_time(e[2 * i + 1]) for e in ev] for i in range(nl)]
     gemm_ms = [[e[2 * i + 1].elapsed_time(e[2 * i + 2]) for e in ev] for i in range(nl)]
     local_ms = sum(step_ms)

@@ -164,12 +164,25 @@ convrot_status launch_gemm_cfg(int num_sms, const uint8_t *qA, const uint8_t *qB
     }
     const int64_t tiles = ((rowsA + gemm::BM - 1) / gemm::BM) * ((rowsB + BN - 1) / BN);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-    gemm::gemm_kernel<BN, SWAP, OUT_S32>
-        <<<grid, gemm::kThreads, gemm::Cfg<BN, SWAP>::SMEM_BYTES, stream>>>(
-            tmA, tmB, tmY, use_tma_store, static_cast<int>(rowsA), static_cast<int>(rowsB),
-            static_cast<int>(K), sx, sw, static_cast<const uint16_t *>(bias), out,
-            static_cast<int>(M), static_cast<int>(N));
-    return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
+    // Programmatic dependent launch: the GEMM's set-up (barriers, TMEM,
+    // descriptor prefetch) overlaps the end of the preceding kernel on the
+    // stream (normally the prep kernel); the kernel waits for that grid's
+    // results before its first load.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(gemm::kThreads);
+    cfg.dynamicSmemBytes = gemm::Cfg<BN, SWAP>::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(
+        &cfg, gemm::gemm_kernel<BN, SWAP, OUT_S32>, tmA, tmB, tmY, use_tma_store,
+        static_cast<int>(rowsA), static_cast<int>(rowsB), static_cast<int>(K), sx, sw,
+        static_cast<const uint16_t *>(bias), out, static_cast<int>(M), static_cast<int>(N));
+    return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 
 // Path choice: up to 128 tokens the weights take the 128-row MMA side

@@ -60,7 +60,7 @@ struct Cfg {
     // Packed stages keep HBM loads in flight; the narrow (skinny) tiles are
     // bound by the weight stream, so they trade widened stages for more
     // packed ones.  The wide tile keeps room for the epilogue's store boxes.
-    static constexpr int SP = BN == 256 ? 4 : BN == 128 ? 6 : BN == 64 ? 10 : 12;
+    static constexpr int SP = BN == 256 ? 3 : BN == 128 ? 6 : BN == 64 ? 10 : 12;
     static constexpr int SU = BN == 256 ? 2 : 3;
     static constexpr int PA = BM * BKP;
     static constexpr int PB = BN * BKP;
@@ -70,7 +70,13 @@ struct Cfg {
     static constexpr int OFF_UA = 0;                   // 1024-aligned tiles first
     static constexpr int OFF_UB = OFF_UA + SU * UA;
     static constexpr int OFF_ST = OFF_UB + SU * UB;
-    static constexpr int OFF_PA = OFF_ST + ST;
+    // per-warp copies of the tile's column parameters (sw as fp32, bias as
+    // bf16) for the columns that warp covers, two tiles deep
+    static constexpr int CP_COLS = BN >= 64 ? BN / 2 : BN;
+    static constexpr int CP_WARP = 2 * CP_COLS * 6;
+    static constexpr int CP = SWAP ? 0 : kEpiWarps * CP_WARP;
+    static constexpr int OFF_CP = OFF_ST + ST;
+    static constexpr int OFF_PA = OFF_CP + ((CP + 1023) / 1024) * 1024;
     static constexpr int OFF_PB = OFF_PA + SP * PA;
     static constexpr int OFF_BAR = OFF_PB + SP * PB;
     static constexpr int NUM_BARS = 2 * SP + 2 * SU + 5;
@@ -191,6 +197,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // Everything above overlaps the tail of the kernel that produced the
+    // operands (programmatic dependent launch); nothing below may run before
+    // that kernel's results are visible.
+    ptx::grid_dependency_wait();
 
     const int tiles_a = (rowsA + BM - 1) / BM;
     const int tiles_b = (rowsB + BN - 1) / BN;
@@ -272,9 +282,27 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             const int ta = tile % tiles_a, tb = tile / tiles_a;
             const int b = local & 1;
             const uint32_t aph = (local >> 1) & 1;
+            const int arow = ta * BM + r;             // A row of this lane
+            // The tile's column scales and bias go to shared memory (and the
+            // row scale to a register) while the main loop still runs, so the
+            // epilogue never waits on these loads.
+            // Each warp keeps its own copy of its columns' parameters, so no
+            // synchronisation beyond the warp is needed.
+            float *cp_sw = reinterpret_cast<float *>(smem + C::OFF_CP + e * C::CP_WARP +
+                                                     b * (C::CP_COLS * 6));
+            uint16_t *cp_b = reinterpret_cast<uint16_t *>(cp_sw + C::CP_COLS);
+            float sxm = 0.0f;
+            if (tma_out && active) {
+                for (int i = lane; i < kCols; i += 32) {
+                    const int n = tb * BN + col_begin + i;
+                    cp_sw[i] = n < N ? sw[n] : 0.0f;
+                    cp_b[i] = (bias && n < N) ? bias[n] : static_cast<uint16_t>(0);
+                }
+                sxm = arow < M ? sx[arow] : 0.0f;
+                __syncwarp();
+            }
             if (!ptx::mbar_wait(acc_full(b), aph, abort_flag)) break;
             ptx::tc_fence_after();
-            const int arow = ta * BM + r;             // A row of this lane
             if (active) {
 #pragma unroll 1
                 for (int c0 = col_begin; c0 < col_begin + kCols; c0 += 32) {
@@ -289,35 +317,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     if (!SWAP && !OUT_S32 && tma_out) {
                         // 32 rows x 32 columns through a swizzled box, one TMA store
                         const int n0 = bcol0;
-                        const bool full_cols = n0 + 32 <= N;
-                        const float sxm = arow < M ? sx[arow] : 0.0f;
                         uint32_t pk[16];
-                        if (full_cols) {
-                            const float4 *s4 = reinterpret_cast<const float4 *>(sw + n0);
-                            const uint4 *b4 = reinterpret_cast<const uint4 *>(bias + n0);
+                        const float4 *s4 = reinterpret_cast<const float4 *>(cp_sw + (c0 - col_begin));
+                        const uint4 *b4 = reinterpret_cast<const uint4 *>(cp_b + (c0 - col_begin));
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const float4 fa = __ldg(s4 + 2 * i), fb = __ldg(s4 + 2 * i + 1);
-                                const uint4 u = bias ? __ldg(b4 + i) : make_uint4(0, 0, 0, 0);
-                                const uint32_t bw[4] = {u.x, u.y, u.z, u.w};
-                                const float swv[8] = {fa.x, fa.y, fa.z, fa.w, fb.x, fb.y, fb.z, fb.w};
+                        for (int i = 0; i < 4; ++i) {
+                            const float4 fa = s4[2 * i], fb = s4[2 * i + 1];
+                            const uint4 u = b4[i];
+                            const uint32_t bw[4] = {u.x, u.y, u.z, u.w};
+                            const float swv[8] = {fa.x, fa.y, fa.z, fa.w, fb.x, fb.y, fb.z, fb.w};
 #pragma unroll
-                                for (int j = 0; j < 4; ++j)
-                                    pk[4 * i + j] = epi_pair(v[8 * i + 2 * j], v[8 * i + 2 * j + 1], sxm,
-                                                             swv[2 * j], swv[2 * j + 1],
-                                                             __uint_as_float(bw[j] << 16),
-                                                             __uint_as_float(bw[j] & 0xFFFF0000u));
-                            }
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 32; j += 2) {
-                                const int n = n0 + j;
-                                const float s0 = n < N ? sw[n] : 0.0f;
-                                const float s1 = n + 1 < N ? sw[n + 1] : 0.0f;
-                                const float b0 = (bias && n < N) ? bf16_to_f32(bias[n]) : 0.0f;
-                                const float b1 = (bias && n + 1 < N) ? bf16_to_f32(bias[n + 1]) : 0.0f;
-                                pk[j / 2] = epi_pair(v[j], v[j + 1], sxm, s0, s1, b0, b1);
-                            }
+                            for (int j = 0; j < 4; ++j)
+                                pk[4 * i + j] = epi_pair(v[8 * i + 2 * j], v[8 * i + 2 * j + 1], sxm,
+                                                         swv[2 * j], swv[2 * j + 1],
+                                                         __uint_as_float(bw[j] << 16),
+                                                         __uint_as_float(bw[j] & 0xFFFF0000u));
                         }
                         const uint32_t box = box0 + (nstores & 1) * (kStoreBox * kStoreBox * 2);
                         if (lane == 0) ptx::bulk_wait_read<1>();   // this box's previous store

@@ -190,6 +190,9 @@ prep_kernel(const uint16_t *__restrict__ x, int K, uint8_t *__restrict__ q,
     uint4 *dst = reinterpret_cast<uint4 *>(q + static_cast<size_t>(row) * (K / 2)) + t * 2;
     dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+    // The GEMM that consumes these rows may be scheduled now; it still waits
+    // for this whole grid to complete before reading them.
+    ptx::launch_dependents();
 }
 
 }  // namespace prep
