@@ -18,6 +18,9 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr int kSmemOptin = 232448;   // per-CTA shared memory limit (sm_100)
+// dynamic shared memory the prep kernels may use (their static part is < 1 KB)
+constexpr int kPrepSmemMax = kSmemOptin - 1024;
 
 struct DeviceState {
     bool ready = false;
@@ -75,10 +78,10 @@ convrot_status device_setup(int *dev_out) {
         g_encode = reinterpret_cast<EncodeTiledFn>(fn);
     }
     bool ok = true;
-    ok &= set_smem(prep::prep_kernel<64, 0>, CONVROT_MAX_K * 2);
-    ok &= set_smem(prep::prep_kernel<256, 0>, CONVROT_MAX_K * 2);
-    ok &= set_smem(prep::prep_kernel<64, 1>, CONVROT_MAX_K * 2);
-    ok &= set_smem(prep::prep_kernel<256, 1>, CONVROT_MAX_K * 2);
+    ok &= set_smem(prep::prep_kernel<64, 0>, kPrepSmemMax);
+    ok &= set_smem(prep::prep_kernel<256, 0>, kPrepSmemMax);
+    ok &= set_smem(prep::prep_kernel<64, 1>, kPrepSmemMax);
+    ok &= set_smem(prep::prep_kernel<256, 1>, kPrepSmemMax);
     ok &= set_smem(gemm::gemm_kernel<256, false, false>, gemm::Cfg<256, false>::SMEM_BYTES);
     ok &= set_smem(gemm::gemm_kernel<256, false, true>, gemm::Cfg<256, false>::SMEM_BYTES);
     ok &= set_smem(gemm::gemm_kernel<16, true, false>, gemm::Cfg<16, true>::SMEM_BYTES);
@@ -104,20 +107,48 @@ convrot_status check_shape(int64_t rows, int64_t K, int group) {
     return CONVROT_OK;
 }
 
-convrot_status launch_prep(const void *x, int64_t rows, int64_t K, int group, uint8_t *q, float *s,
-                           float *yrot, cudaStream_t stream) {
+// Shared memory of one prep CTA: one staged bf16 row (+ the group-256
+// exchange area of 4 bytes per channel).
+size_t prep_smem(int64_t K, int group) {
+    return static_cast<size_t>(K) * (group == 256 ? 6 : 2);
+}
+
+// Resident prep CTAs per SM for a (group, mode, K) launch, cached.
+int prep_ctas_per_sm(int group, int mode, int64_t K) {
+    static int cache[2][2][prep::kMaxThreads + 1];
+    const int T = static_cast<int>(K / prep::kElemsPerThread);
+    int &slot = cache[group == 256][mode][T];
+    if (slot == 0) {
+        int n = 0;
+        cudaError_t e;
+        const size_t smem = prep_smem(K, group);
+        if (group == 64)
+            e = mode ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, prep::prep_kernel<64, 1>, T, smem)
+                     : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, prep::prep_kernel<64, 0>, T, smem);
+        else
+            e = mode ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, prep::prep_kernel<256, 1>, T, smem)
+                     : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, prep::prep_kernel<256, 0>, T, smem);
+        slot = (e == cudaSuccess && n > 0) ? n : 1;
+    }
+    return slot;
+}
+
+convrot_status launch_prep(int num_sms, const void *x, int64_t rows, int64_t K, int group,
+                           uint8_t *q, float *s, float *yrot, cudaStream_t stream) {
     if (rows == 0) return CONVROT_OK;
-    const dim3 grid(static_cast<unsigned>(rows));
+    const int mode = yrot ? 1 : 0;
+    const size_t smem = prep_smem(K, group);
+    const int64_t resident = static_cast<int64_t>(num_sms) * prep_ctas_per_sm(group, mode, K);
+    const dim3 grid(static_cast<unsigned>(rows < resident ? rows : resident));
     const dim3 block(static_cast<unsigned>(K / prep::kElemsPerThread));
     const uint16_t *xx = static_cast<const uint16_t *>(x);
-    const int k = static_cast<int>(K);
-    const size_t smem = static_cast<size_t>(K) * 2;     // one bf16 row, staged
+    const int m = static_cast<int>(rows), k = static_cast<int>(K);
     if (yrot) {
-        if (group == 64) prep::prep_kernel<64, 1><<<grid, block, smem, stream>>>(xx, k, q, s, yrot);
-        else prep::prep_kernel<256, 1><<<grid, block, smem, stream>>>(xx, k, q, s, yrot);
+        if (group == 64) prep::prep_kernel<64, 1><<<grid, block, smem, stream>>>(xx, m, k, q, s, yrot);
+        else prep::prep_kernel<256, 1><<<grid, block, smem, stream>>>(xx, m, k, q, s, yrot);
     } else {
-        if (group == 64) prep::prep_kernel<64, 0><<<grid, block, smem, stream>>>(xx, k, q, s, yrot);
-        else prep::prep_kernel<256, 0><<<grid, block, smem, stream>>>(xx, k, q, s, yrot);
+        if (group == 64) prep::prep_kernel<64, 0><<<grid, block, smem, stream>>>(xx, m, k, q, s, yrot);
+        else prep::prep_kernel<256, 0><<<grid, block, smem, stream>>>(xx, m, k, q, s, yrot);
     }
     return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
@@ -252,7 +283,7 @@ convrot_status convrot_quantize_weight(const void *w_bf16, int64_t N, int64_t K,
         return CONVROT_ERR_ALIGN;
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
-    return launch_prep(w_bf16, N, K, group, qw, sw, nullptr, stream);
+    return launch_prep(g_dev[dev].num_sms, w_bf16, N, K, group, qw, sw, nullptr, stream);
 }
 
 convrot_status convrot_prepare_act(const void *x_bf16, int64_t M, int64_t K, int group, uint8_t *qx,
@@ -302,7 +333,8 @@ convrot_status convrot_linear(const void *x_bf16, const uint8_t *qw, const float
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
     uint8_t *qx = static_cast<uint8_t *>(workspace);
     float *sx = reinterpret_cast<float *>(qx + round256(static_cast<size_t>(M) * (K / 2)));
-    if ((st = launch_prep(x_bf16, M, K, group, qx, sx, nullptr, stream)) != CONVROT_OK) return st;
+    if ((st = launch_prep(g_dev[dev].num_sms, x_bf16, M, K, group, qx, sx, nullptr, stream)) != CONVROT_OK)
+        return st;
     return launch_gemm<false>(g_dev[dev].num_sms, qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream);
 }
 
@@ -315,7 +347,7 @@ convrot_status convrot_debug_rotate_f32(const void *x_bf16, int64_t M, int64_t K
     if (!aligned16(x_bf16) || !aligned16(y_rot)) return CONVROT_ERR_ALIGN;
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
-    return launch_prep(x_bf16, M, K, group, nullptr, nullptr, y_rot, stream);
+    return launch_prep(g_dev[dev].num_sms, x_bf16, M, K, group, nullptr, nullptr, y_rot, stream);
 }
 
 convrot_status convrot_debug_gemm_s32(const uint8_t *qx, const uint8_t *qw, int64_t M, int64_t N,
@@ -429,7 +461,8 @@ extern "C" convrot_status convrot_linear_noalloc(const void *x_bf16, const uint8
     // Every byte of qx and sx read by the GEMM is written by the prep kernel
     // first, so leftovers of an earlier call never reach the result.
     float *sx = reinterpret_cast<float *>(qx + round256(static_cast<size_t>(M) * (K / 2)));
-    if ((st = launch_prep(x_bf16, M, K, group, qx, sx, nullptr, stream)) != CONVROT_OK) return st;
+    if ((st = launch_prep(g_dev[dev].num_sms, x_bf16, M, K, group, qx, sx, nullptr, stream)) != CONVROT_OK)
+        return st;
     return launch_gemm<false>(g_dev[dev].num_sms, qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16,
                               stream);
 }

@@ -1,7 +1,7 @@
 // prep.cuh -- fused rotation + rowwise absmax INT4 quantisation + packing.
 //
-// One CTA per row, K/64 threads; thread t owns the 64 consecutive channels
-// [64t, 64t + 64) of its row, loaded with eight 128-bit loads.
+// K/64 threads per CTA, persistent over rows; thread t owns the 64
+// consecutive channels [64t, 64t + 64) of each row it helps with.
 //
 // Rotation.  Within a group of n = 4^k channels the normalised regular
 // Hadamard is H_n = T^{(x)k} / 2^k with T = J - 2I (Comfy-Org/comfy-quants
@@ -11,9 +11,10 @@
 // that differ only in digit d, y_i = (x_0 + x_1 + x_2 + x_3) - 2 x_i.  The k
 // butterflies commute (every factor is the same symmetric T), so they run in
 // any order: digits 0, 1, 2 live inside one thread's 64 registers; for
-// n = 256 digit 3 spans the 4 threads of the group and is done with two
-// XOR shuffles.  The 1/2^k normalisation is exact and is folded into the
-// scale (see below), so the butterflies run on unnormalised values.
+// n = 256 digit 3 spans the 4 threads of the group, which swap quarters of
+// their data through shared memory so that digit 3 also becomes a register
+// stride.  The 1/2^k normalisation is exact and is folded into the scale
+// (see below), so the butterflies run on unnormalised values.
 //
 // Quantisation ("convrot-mlx" README, "What is included": symmetric rowwise
 // absmax to [-7, 7]).  With u the unnormalised rotated row and y = u 2^-k:
@@ -41,14 +42,6 @@ using ptx::mul2;
 constexpr int kElemsPerThread = 64;
 constexpr int kMaxThreads = 512;   // K <= 32768
 
-__device__ __forceinline__ uint4 ldg_stream(const uint4 *p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
-
 // Two signed codes into one byte of the running word:
 // result = (acc << 8) | ((hi & 0xF) << 4) | (lo & 0xF), saturating to [-8, 7]
 // (codes here are already in [-7, 7]).
@@ -58,138 +51,215 @@ __device__ __forceinline__ uint32_t pack_nibbles(int hi, int lo, uint32_t acc) {
     return d;
 }
 
-// One radix-4 butterfly stage along the digit whose stride is S (1, 4, 16),
-// two quadruples at a time.  Quadruples start at the indices b whose digit of
-// stride S is 0; they are paired as (b, b + P) with P = 4 for S = 1 and
-// P = 1 otherwise, so both members of a pair are quadruple starts.
+// Radix-4 butterflies with packed two-wide arithmetic.  Every packed
+// operation works on the register pair (v[2i], v[2i+1]) so that values stay
+// in the same aligned register pair through all stages.
+//
+// Digit 0 (stride 1): the quadruple {4q .. 4q+3} is two pairs; their packed
+// sum gives (v0+v2, v1+v3), one scalar add completes the quadruple sum.
+__device__ __forceinline__ void radix4_digit0(float (&v)[kElemsPerThread]) {
+#pragma unroll
+    for (int b = 0; b < kElemsPerThread; b += 4) {
+        float p0, p1;
+        add2(p0, p1, v[b], v[b + 1], v[b + 2], v[b + 3]);
+        const float sum = p0 + p1;
+        bfly2(v[b], v[b + 1], sum, sum);
+        bfly2(v[b + 2], v[b + 3], sum, sum);
+    }
+}
+
+// Digits with stride S = 4 or 16: the quadruples starting at b and b + 1
+// (b even) run side by side in the two halves of each packed operation.
 template <int S>
 __device__ __forceinline__ void radix4_stage(float (&v)[kElemsPerThread]) {
-    constexpr int P = (S == 1) ? 4 : 1;
 #pragma unroll
-    for (int b = 0; b < kElemsPerThread; ++b) {
-        if ((b / S) % 4 != 0 || (b / P) % 2 != 0) continue;
-        const int c = b + P;
+    for (int b = 0; b < kElemsPerThread; b += 2) {
+        if ((b / S) % 4 != 0) continue;
         float s01a, s01b, s23a, s23b, suma, sumb;
-        add2(s01a, s01b, v[b], v[c], v[b + S], v[c + S]);
-        add2(s23a, s23b, v[b + 2 * S], v[c + 2 * S], v[b + 3 * S], v[c + 3 * S]);
+        add2(s01a, s01b, v[b], v[b + 1], v[b + S], v[b + 1 + S]);
+        add2(s23a, s23b, v[b + 2 * S], v[b + 1 + 2 * S], v[b + 3 * S], v[b + 1 + 3 * S]);
         add2(suma, sumb, s01a, s01b, s23a, s23b);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) bfly2(v[b + j * S], v[c + j * S], suma, sumb);
+        for (int j = 0; j < 4; ++j) bfly2(v[b + j * S], v[b + 1 + j * S], suma, sumb);
     }
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 // MODE 0: quantise + pack (q, s).  MODE 1: write the normalised rotated row
 // as fp32 (yrot) instead.
 //
-// Loads: the row is read with coalesced 128-bit loads (consecutive threads,
-// consecutive 16-byte chunks) and written to shared memory so that chunk c of
-// thread t's 128-byte slice sits at position c ^ (t mod 8); each thread then
-// reads its own 64 channels back with conflict-free 128-bit loads.
+// Persistent: CTA b handles rows b, b + gridDim.x, ...  Loads are
+// asynchronous: while a row is rotated and quantised, the next row of the
+// same CTA is already on its way into the stage buffer.  Each row is read with coalesced 16-byte copies (consecutive
+// threads, consecutive chunks) that land so that chunk c of thread t's
+// 128-byte slice sits at position c ^ (t mod 8); each thread then reads its
+// own 64 channels with conflict-free 128-bit loads.
 template <int G, int MODE>
 __global__ void __launch_bounds__(kMaxThreads)
-prep_kernel(const uint16_t *__restrict__ x, int K, uint8_t *__restrict__ q,
+prep_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ q,
             float *__restrict__ s, float *__restrict__ yrot) {
     static_assert(G == 64 || G == 256, "group 64 or 256");
     constexpr int kDigits = (G == 64) ? 3 : 4;
     constexpr float kNorm = (G == 64) ? 0.125f : 0.0625f;   // 2^-kDigits
 
-    extern __shared__ uint4 stage[];                     // K * 2 bytes
+    // K * 2 bytes of stage buffer, then (group 256) K * 4 bytes of exchange
+    extern __shared__ uint4 stage[];
     __shared__ uint32_t red[kMaxThreads / 32];
 
-    const int row = blockIdx.x;
     const int t = threadIdx.x;
     const int nthreads = blockDim.x;                     // K / 64
     const int warp = t >> 5, lane = t & 31;
     const int warp_lanes = min(32, nthreads - warp * 32);
     const uint32_t mask = warp_lanes == 32 ? 0xFFFFFFFFu : ((1u << warp_lanes) - 1u);
+    const int row_chunks = nthreads * 8;                 // 16-byte chunks per row
+    const uint32_t stage_s = ptx::smem_u32(stage);
 
-    {
-        const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(row) * K);
-        uint4 r[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) r[j] = ldg_stream(src + t + j * nthreads);
+    auto issue_row = [&](int r, int buf) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(r) * K);
+        const uint32_t base = stage_s;
+        (void)buf;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int g = t + j * nthreads;              // chunk index in the row
             const int owner = g >> 3, c = g & 7;
-            stage[owner * 8 + (c ^ (owner & 7))] = r[j];
+            cp_async16(base + static_cast<uint32_t>((owner * 8 + (c ^ (owner & 7))) * 16), src + g);
+        }
+    };
+
+    // One stage buffer: a row is read into registers, then (after a barrier)
+    // the next row of this CTA is requested into the same buffer, so the copy
+    // overlaps all of the arithmetic on the current row.
+    int row = blockIdx.x;
+    if (row < M) issue_row(row, 0);
+    cp_async_commit();
+    for (; row < M; row += gridDim.x) {
+        const int next = row + gridDim.x;
+        cp_async_wait_all();      // this row's copies (by this thread) have landed
+        __syncthreads();          // ... and everyone else's
+
+        float v[kElemsPerThread];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint4 raw = stage[t * 8 + (i ^ (t & 7))];
+            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+                v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+            }
+        }
+        __syncthreads();          // the stage buffer is free again
+        if (next < M) issue_row(next, 0);
+        cp_async_commit();
+
+        radix4_digit0(v);
+        radix4_stage<4>(v);
+        radix4_stage<16>(v);
+        // For n = 256 the four threads of a group hold digit 3 = 0..3.  They
+        // swap quarters through shared memory so that each thread then holds,
+        // for its j = t mod 4, the channels 64 d3 + 16 j + r (d3 = 0..3,
+        // r = 0..15): digit 3 becomes a register stride of 16 and the last
+        // butterfly runs in registers.  Chunk i = 4a + b (4 floats) of thread t
+        // is stored at slot (4b + a) ^ (t mod 16) of t's 16-slot row, which
+        // keeps both the stores and the transposed loads free of bank conflicts.
+        if (kDigits == 4) {
+            float4 *xb = reinterpret_cast<float4 *>(stage + row_chunks);
+            const int key = t & 15;
+            __syncwarp(mask);     // the group finished reading the previous row's swap
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                xb[t * 16 + ((((i & 3) << 2) | (i >> 2)) ^ key)] =
+                    make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            __syncwarp(mask);
+            const int j = t & 3, gb = t & ~3;
+#pragma unroll
+            for (int d3 = 0; d3 < 4; ++d3) {
+                const int w = gb + d3;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float4 f = xb[w * 16 + (((c << 2) | j) ^ (w & 15))];
+                    v[16 * d3 + 4 * c] = f.x;
+                    v[16 * d3 + 4 * c + 1] = f.y;
+                    v[16 * d3 + 4 * c + 2] = f.z;
+                    v[16 * d3 + 4 * c + 3] = f.w;
+                }
+            }
+            radix4_stage<16>(v);
+        }
+        // Position in the row of register e of this thread.
+        auto chan = [&](int e) -> int {
+            if (kDigits == 3) return t * 64 + e;
+            return (t & ~3) * 64 + 64 * (e >> 4) + 16 * (t & 3) + (e & 15);
+        };
+
+        if (MODE == 1) {
+            float *dst = yrot + static_cast<size_t>(row) * K;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                *reinterpret_cast<float4 *>(dst + chan(4 * i)) =
+                    make_float4(v[4 * i] * kNorm, v[4 * i + 1] * kNorm, v[4 * i + 2] * kNorm,
+                                v[4 * i + 3] * kNorm);
+            continue;
+        }
+
+        float m = 0.0f;
+#pragma unroll
+        for (int e = 0; e < kElemsPerThread; ++e) m = fmaxf(m, fabsf(v[e]));
+        // non-negative floats order like their bit patterns
+        uint32_t mb = __reduce_max_sync(mask, __float_as_uint(m));
+        if (lane == 0) red[warp] = mb;
+        __syncthreads();
+        const int nwarps = (nthreads + 31) >> 5;
+        for (int w = 0; w < nwarps; ++w) mb = max(mb, red[w]);
+        const float a_u = __uint_as_float(mb);
+
+        const float inv = a_u > 0.0f ? __fdiv_rn(7.0f, a_u) : 0.0f;
+        if (t == 0) s[row] = __fdiv_rn(a_u * kNorm, 7.0f);
+
+        uint32_t packed[8];
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            int code[8];
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+                float p0, p1, h0, h1;
+                mul2(p0, p1, v[8 * w + j], v[8 * w + j + 1], inv, inv);
+                // add (0.5 - 2^-25) with the sign of the product, truncate
+                const float c0 = __uint_as_float((__float_as_uint(p0) & 0x80000000u) | 0x3EFFFFFFu);
+                const float c1 = __uint_as_float((__float_as_uint(p1) & 0x80000000u) | 0x3EFFFFFFu);
+                add2(h0, h1, p0, p1, c0, c1);
+                code[j] = __float2int_rz(h0);
+                code[j + 1] = __float2int_rz(h1);
+            }
+            uint32_t word = pack_nibbles(code[7], code[6], 0u);
+            word = pack_nibbles(code[5], code[4], word);
+            word = pack_nibbles(code[3], code[2], word);
+            packed[w] = pack_nibbles(code[1], code[0], word);
+        }
+        uint8_t *qrow = q + static_cast<size_t>(row) * (K / 2);
+        if (kDigits == 3) {
+            uint4 *dst = reinterpret_cast<uint4 *>(qrow + t * 32);
+            dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+        } else {
+            // registers 16 d3 .. 16 d3 + 15 are 16 consecutive channels: 8 bytes
+#pragma unroll
+            for (int d3 = 0; d3 < 4; ++d3)
+                *reinterpret_cast<uint2 *>(qrow + chan(16 * d3) / 2) =
+                    make_uint2(packed[2 * d3], packed[2 * d3 + 1]);
         }
     }
-    __syncthreads();
-
-    float v[kElemsPerThread];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const uint4 raw = stage[t * 8 + (i ^ (t & 7))];
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
-            v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-        }
-    }
-
-    radix4_stage<1>(v);
-    radix4_stage<4>(v);
-    radix4_stage<16>(v);
-    if (kDigits == 4) {
-        // digit 3 = lane bits 0..1: the 4 threads of this 256-channel group
-#pragma unroll
-        for (int e = 0; e < kElemsPerThread; e += 2) {
-            float s0, s1;
-            add2(s0, s1, v[e], v[e + 1], __shfl_xor_sync(mask, v[e], 1),
-                 __shfl_xor_sync(mask, v[e + 1], 1));
-            add2(s0, s1, s0, s1, __shfl_xor_sync(mask, s0, 2), __shfl_xor_sync(mask, s1, 2));
-            bfly2(v[e], v[e + 1], s0, s1);
-        }
-    }
-
-    if (MODE == 1) {
-        float4 *dst = reinterpret_cast<float4 *>(yrot + static_cast<size_t>(row) * K) + t * 16;
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-            dst[i] = make_float4(v[4 * i] * kNorm, v[4 * i + 1] * kNorm, v[4 * i + 2] * kNorm,
-                                 v[4 * i + 3] * kNorm);
-        return;
-    }
-
-    float m = 0.0f;
-#pragma unroll
-    for (int e = 0; e < kElemsPerThread; ++e) m = fmaxf(m, fabsf(v[e]));
-    // non-negative floats order like their bit patterns
-    uint32_t mb = __reduce_max_sync(mask, __float_as_uint(m));
-    if (lane == 0) red[warp] = mb;
-    __syncthreads();
-    const int nwarps = (nthreads + 31) >> 5;
-    for (int w = 0; w < nwarps; ++w) mb = max(mb, red[w]);
-    const float a_u = __uint_as_float(mb);
-
-    const float inv = a_u > 0.0f ? __fdiv_rn(7.0f, a_u) : 0.0f;
-    if (t == 0) s[row] = __fdiv_rn(a_u * kNorm, 7.0f);
-
-    uint32_t packed[8];
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-        int code[8];
-#pragma unroll
-        for (int j = 0; j < 8; j += 2) {
-            float p0, p1, h0, h1;
-            mul2(p0, p1, v[8 * w + j], v[8 * w + j + 1], inv, inv);
-            // add (0.5 - 2^-25) with the sign of the product, truncate
-            const float c0 = __uint_as_float((__float_as_uint(p0) & 0x80000000u) | 0x3EFFFFFFu);
-            const float c1 = __uint_as_float((__float_as_uint(p1) & 0x80000000u) | 0x3EFFFFFFu);
-            add2(h0, h1, p0, p1, c0, c1);
-            code[j] = __float2int_rz(h0);
-            code[j + 1] = __float2int_rz(h1);
-        }
-        uint32_t word = pack_nibbles(code[7], code[6], 0u);
-        word = pack_nibbles(code[5], code[4], word);
-        word = pack_nibbles(code[3], code[2], word);
-        packed[w] = pack_nibbles(code[1], code[0], word);
-    }
-    uint4 *dst = reinterpret_cast<uint4 *>(q + static_cast<size_t>(row) * (K / 2)) + t * 2;
-    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
     // The GEMM that consumes these rows may be scheduled now; it still waits
     // for this whole grid to complete before reading them.
     ptx::launch_dependents();
