@@ -6,13 +6,16 @@ One step is one pass of the whole path over one batch through the public
 call convrot_linear: the fused prep kernel (rotation, rowwise absmax INT4
 quantisation, packing) and the tcgen05 GEMM with its scale/bias/bf16
 epilogue (two kernels per linear layer).  Weights are prepared once before
-timing (the offline step).  The L2 cache is flushed (a 256 MiB write) before
-every timed step, outside the timed interval; each step is bracketed by CUDA
-events on the launching stream.  A second pass of the same number of steps
-runs the two kernels through the split calls with an event between them to
-time each kernel for the roofline.  Under torchrun every rank runs its own
-batch (weak scaling, no collective on the data path); the reported time is
-the maximum over ranks.
+timing (the offline step).  Caches stay cold without a flush kernel: the
+steps cycle through enough full copies of the step's data (activations,
+workspace, weights, outputs) that the copies together exceed twice the L2
+size.  Each step is one CUDA graph replay; K replays run back to back between
+two CUDA events on the launching stream.  Two more passes of K replays time
+the prep kernel alone and the GEMM alone for the roofline.  The end-to-end
+figure calls convrot_linear on pinned host buffers with the copies inside the
+timed interval (L2 flushed before each of those steps).  Under torchrun every
+rank runs its own batch (weak scaling, no collective on the data path); the
+reported time is the maximum over ranks.
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
 instead, on bounded samples of the same workload, on the host cores.
@@ -94,13 +97,23 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            # wait (up to 3 s) until the sampler runs, so the window is covered
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 3.0 and self.proc.poll() is None:
+                time.sleep(0.01)
         except OSError:
             self.proc = None
+        self.first = len(self.lines)
         return self
+
+    def mark_end(self):
+        """Call when the timed work is done; later samples are not used."""
+        time.sleep(0.03)             # let the sample covering the end arrive
+        self.last = len(self.lines)
 
     def _read(self):
         for line in self.proc.stdout:
@@ -118,7 +131,9 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        lo = max(0, getattr(self, "first", 0) - 1)
+        hi = getattr(self, "last", len(self.lines))
+        for line in self.lines[lo:hi]:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) != 6:
                 continue
@@ -177,6 +192,7 @@ def run_gpu(args):
     spec = wl.WORKLOADS[name]
     layers = wl.make_workload(name, seed=spec.seed + rank)
     stream = torch.cuda.current_stream()
+    nl = len(layers)
 
     # offline step: prepare the weights once
     prepared = []
@@ -187,45 +203,84 @@ def run_gpu(args):
         del w
         prepared.append((lt.spec, qw, sw, b))
     x0 = layers[0].x.to(dev)
-    acts, ws, lws = [], [], []
-    for i, (sp, qw, sw, b) in enumerate(prepared):
-        acts.append(x0 if i == 0 else torch.empty(sp.M, sp.K, dtype=torch.bfloat16, device=dev))
-        ws.append((torch.empty(sp.M, sp.K // 2, dtype=torch.uint8, device=dev),
-                   torch.empty(sp.M, dtype=torch.float32, device=dev)))
-        lws.append(torch.empty(max(1, cr.convrot_linear_workspace_size(sp.M, sp.K)),
-                               dtype=torch.uint8, device=dev))
-    outs = [torch.empty(sp.M, sp.N, dtype=torch.bfloat16, device=dev) for sp, *_ in prepared]
-    for i in range(1, len(prepared)):
-        acts[i] = outs[i - 1]          # chained layers: next input is this output
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    nl = len(prepared)
+    # Cold caches without a flush kernel: the steps cycle through R full copies
+    # of everything a step touches (activations, workspace, weights, outputs),
+    # with R copies together at least twice the L2 size, so no step finds its
+    # data in L2 from an earlier one.
+    step_bytes = sum(sp.M * sp.K * 2 + cr.convrot_linear_workspace_size(sp.M, sp.K)
+                     + sp.N * (sp.K // 2 + 6) + sp.M * sp.N * 2 for sp, *_ in prepared)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = 1 if step_bytes >= 2 * l2 else min(64, -(-2 * l2 // step_bytes))
 
-    def step():
+    class Copy:
+        pass
+
+    copies = []
+    for r in range(R):
+        c = Copy()
+        c.w = [(sp, qw.clone(), sw.clone(), None if b is None else b.clone())
+               for sp, qw, sw, b in prepared]
+        c.acts = [x0.clone()]
+        c.ws, c.lws, c.outs = [], [], []
+        for i, (sp, *_) in enumerate(prepared):
+            c.ws.append((torch.empty(sp.M, sp.K // 2, dtype=torch.uint8, device=dev),
+                         torch.empty(sp.M, dtype=torch.float32, device=dev)))
+            c.lws.append(torch.empty(max(1, cr.convrot_linear_workspace_size(sp.M, sp.K)),
+                                     dtype=torch.uint8, device=dev))
+            c.outs.append(torch.empty(sp.M, sp.N, dtype=torch.bfloat16, device=dev))
+            if i + 1 < nl:
+                c.acts.append(c.outs[i])   # chained layers: next input is this output
+        copies.append(c)
+
+    def step(c):
         # the public whole-layer call: prep kernel + GEMM kernel per layer
-        for i, (sp, qw, sw, b) in enumerate(prepared):
-            cr.convrot_linear(acts[i], qw, sw, b, sp.group, lws[i], outs[i])
+        for i, (sp, qw, sw, b) in enumerate(c.w):
+            cr.convrot_linear(c.acts[i], qw, sw, b, sp.group, c.lws[i], c.outs[i])
 
-    def step_split(events):
-        # the same two kernels through the split calls, with an event between
-        # them, to time each kernel on its own
-        for i, (sp, qw, sw, b) in enumerate(prepared):
-            events[2 * i].record(stream)
-            cr.convrot_prepare_act(acts[i], sp.group, ws[i][0], ws[i][1])
-            events[2 * i + 1].record(stream)
-            cr.convrot_linear_prepared(ws[i][0], ws[i][1], qw, sw, b, sp.K, out=outs[i])
-        events[2 * nl].record(stream)
+    def prep_only(c, i):
+        sp, qw, sw, b = c.w[i]
+        cr.convrot_prepare_act(c.acts[i], sp.group, c.ws[i][0], c.ws[i][1])
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
+    def gemm_only(c, i):
+        sp, qw, sw, b = c.w[i]
+        cr.convrot_linear_prepared(c.ws[i][0], c.ws[i][1], qw, sw, b, sp.K, out=c.outs[i])
+
+    for k in range(max(args.warmup, R)):
+        step(copies[k % R])
+        for i in range(nl):
+            prep_only(copies[k % R], i)
+            gemm_only(copies[k % R], i)
     torch.cuda.synchronize()
     if cr.convrot_check_device_error() != 0:
         raise RuntimeError("device error during warm-up")
 
-    # timed region: whole steps, L2 flushed before each (outside the interval)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+    # One CUDA graph per copy and per program (whole step, prep only, GEMM
+    # only): the timed loops replay them back to back, so host launch cost is
+    # not in the device timing.
+    def capture(fn, *a):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn(*a)
+        return g
+
+    g_step = [capture(step, c) for c in copies]
+    g_prep = [[capture(prep_only, c, i) for c in copies] for i in range(nl)]
+    g_gemm = [[capture(gemm_only, c, i) for c in copies] for i in range(nl)]
+    for g in g_step + sum(g_prep, []) + sum(g_gemm, []):
+        g.replay()
+    torch.cuda.synchronize()
+
+    def timed(graphs, steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for k in range(steps):
+            graphs[k % R].replay()
+        b.record()
+        b.synchronize()
+        return a.elapsed_time(b)
+
+    # timed region: K whole steps
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -234,31 +289,20 @@ def run_gpu(args):
     except Exception:
         gpu_id = str(local)
     with ClockSampler(gpu_id) as clocks:
-        for k in range(args.steps):
-            flush.zero_()
-            ev[k][0].record(stream)
-            step()
-            ev[k][1].record(stream)
+        local_ms = timed(g_step, args.steps)
         torch.cuda.synchronize()
+        clocks.mark_end()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     status = cr.convrot_check_device_error()
     if status != 0:
         raise RuntimeError(f"device error status {status} in the timed region")
-    step_ms = [a.elapsed_time(b) for a, b in ev]
 
-    # per-kernel durations over the same number of steps
-    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nl + 1)]
-           for _ in range(args.steps)]
-    for k in range(args.steps):
-        flush.zero_()
-        step_split(kev[k])
-    torch.cuda.synchronize()
-    ev = kev
-    prep_ms = [[e[2 * i].elapsed_time(e[2 * i + 1]) for e in ev] for i in range(nl)]
-    gemm_ms = [[e[2 * i + 1].elapsed_time(e[2 * i + 2]) for e in ev] for i in range(nl)]
-    local_ms = sum(step_ms)
+    # per-kernel durations: K back-to-back launches of one kernel of one layer
+    prep_ms = [[timed(g_prep[i], args.steps) / args.steps] * args.steps for i in range(nl)]
+    gemm_ms = [[timed(g_gemm[i], args.steps) / args.steps] * args.steps for i in range(nl)]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)   # e2e pass only
     ops_step = spec.ops
     t_max, ops_total = aggregate(local_ms, ops_step * args.steps, dev)
     value = ops_total / (t_max * 1e-3) / 1e12                      # TOPS, whole job
@@ -298,7 +342,10 @@ def run_gpu(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "s8",
         "data": "synthetic (seeded bf16, shapes and distributions of the workload; no weights)",
         "config": {"workload": name, "layers": [f"{l.M}x{l.K}->{l.N} g{l.group}" for l in spec.layers],
-                   "tokens_per_rank": spec.tokens, "l2": "flushed (256 MiB write) before each step",
+                   "tokens_per_rank": spec.tokens,
+                   "l2": f"cold: steps cycle through {R} copies of all step data "
+                         f"({R * step_bytes / 2**20:.0f} MiB >= 2 x L2)",
+                   "launch": "CUDA graph per step, replayed back to back",
                    "parallelism": f"dp{world}"},
         "tokens_per_s": round(tokens_s, 1),
         "int8_peak_frac_path": round(value / world / int8_peak, 4),
@@ -342,15 +389,17 @@ def run_e2e(cr, prepared, spec, dev, stream, flush, args):
     for _ in range(3):
         one()
     torch.cuda.synchronize()
-    total = 0.0
-    for _ in range(steps):
+    # Steps are enqueued ahead (no per-step synchronisation), so the interval
+    # of each step holds its copies and kernels, not host enqueue gaps.
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for a, b in ev:
         flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         one()
         b.record(stream)
-        b.synchronize()
-        total += a.elapsed_time(b)
+    torch.cuda.synchronize()
+    total = sum(a.elapsed_time(b) for a, b in ev)
     return {"ms": total, "steps": steps, "h2d": sp0.M * sp0.K * 2,
             "d2h": prepared[-1][0].M * prepared[-1][0].N * 2}
 
@@ -444,7 +493,7 @@ def run_reference(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=10000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=wl.DEFAULT_BENCH, choices=sorted(wl.WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])

@@ -84,6 +84,8 @@ convrot_status device_setup(int *dev_out) {
     ok &= set_smem(prep::prep_kernel<256, 1>, kPrepSmemMax);
     ok &= set_smem(gemm::gemm_kernel<256, false, false>, gemm::Cfg<256, false>::SMEM_BYTES);
     ok &= set_smem(gemm::gemm_kernel<256, false, true>, gemm::Cfg<256, false>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<192, false, false>, gemm::Cfg<192, false>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<192, false, true>, gemm::Cfg<192, false>::SMEM_BYTES);
     ok &= set_smem(gemm::gemm_kernel<16, true, false>, gemm::Cfg<16, true>::SMEM_BYTES);
     ok &= set_smem(gemm::gemm_kernel<32, true, false>, gemm::Cfg<32, true>::SMEM_BYTES);
     ok &= set_smem(gemm::gemm_kernel<64, true, false>, gemm::Cfg<64, true>::SMEM_BYTES);
@@ -153,10 +155,11 @@ convrot_status launch_prep(int num_sms, const void *x, int64_t rows, int64_t K, 
     return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 
-bool make_map(CUtensorMap *map, const uint8_t *base, int64_t rows, int64_t K, int box_rows) {
+bool make_map(CUtensorMap *map, const uint8_t *base, int64_t rows, int64_t K, int box_bytes,
+              int box_rows) {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(gemm::BKP), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_bytes), static_cast<cuuint32_t>(box_rows)};
     const cuuint32_t estr[2] = {1, 1};
     return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -184,7 +187,8 @@ convrot_status launch_gemm_cfg(int num_sms, const uint8_t *qA, const uint8_t *qB
                                const void *bias, void *out, int64_t M, int64_t N,
                                cudaStream_t stream) {
     CUtensorMap tmA, tmB, tmY;
-    if (!make_map(&tmA, qA, rowsA, K, gemm::BM) || !make_map(&tmB, qB, rowsB, K, BN))
+    constexpr int pkb = gemm::Cfg<BN, SWAP>::PKB;
+    if (!make_map(&tmA, qA, rowsA, K, pkb, gemm::BM) || !make_map(&tmB, qB, rowsB, K, pkb, BN))
         return CONVROT_ERR_CUDA;
     int use_tma_store = 0;
     if (!SWAP && !OUT_S32 && N % 8 == 0) {
@@ -236,6 +240,17 @@ convrot_status launch_gemm(int num_sms, const uint8_t *qx, const float *sx, cons
         return launch_gemm_cfg<128, true, OUT_S32>(num_sms, qw, qx, N, M, K, sx, sw, bias, out, M, N,
                                                    stream);
     }
+    // Wider tiles need fewer widened bytes per output, but a tile count just
+    // above a multiple of the SM count wastes most of a wave.  The widening
+    // work of a tile is proportional to its rows of A plus B (128 + BN).
+    const int64_t mt = (M + gemm::BM - 1) / gemm::BM;
+    const auto cost = [&](int64_t bn) {
+        const int64_t tiles = mt * ((N + bn - 1) / bn);
+        return ((tiles + num_sms - 1) / num_sms) * (gemm::BM + bn);
+    };
+    if (cost(192) < cost(256))
+        return launch_gemm_cfg<192, false, OUT_S32>(num_sms, qx, qw, M, N, K, sx, sw, bias, out, M,
+                                                    N, stream);
     return launch_gemm_cfg<256, false, OUT_S32>(num_sms, qx, qw, M, N, K, sx, sw, bias, out, M, N,
                                                 stream);
 }

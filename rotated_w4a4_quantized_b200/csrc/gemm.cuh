@@ -28,7 +28,8 @@
 //                 bf16; full tiles leave through a swizzled shared-memory
 //                 box and a TMA store;
 //   warps 10..17  widening: packed stage -> int8 stage in the 128-byte
-//                 swizzled K-major layout the MMA descriptors describe.
+//                 swizzled K-major layout the MMA descriptors describe; the
+//                 warps form groups that take alternate stages.
 // Accumulators are double-buffered in TMEM so the epilogue of one tile runs
 // under the main loop of the next.
 //
@@ -47,7 +48,7 @@
 namespace gemm {
 
 constexpr int BM = 128;          // MMA M: rows of operand A per tile
-constexpr int BKP = 64;          // packed bytes per row per K-block
+constexpr int BKP = 64;          // packed bytes per row per 128-deep K-block
 constexpr int BK = 128;          // int8 values per row per K-block
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpEpi0 = 2, kEpiWarps = 8;
 constexpr int kWarpUnp0 = kWarpEpi0 + kEpiWarps, kUnpWarps = 8;
@@ -57,13 +58,27 @@ constexpr int kStoreBox = 32;    // epilogue TMA-store box: 32 rows x 32 bf16
 template <int BN, bool SWAP>
 struct Cfg {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "kind::i8 with M=128 needs N%16==0");
+    static_assert(BN < 64 || (BN / 2) % 32 == 0, "each epilogue half covers whole 32-column reads");
     // Packed stages keep HBM loads in flight; the narrow (skinny) tiles are
     // bound by the weight stream, so they trade widened stages for more
     // packed ones.  The wide tile keeps room for the epilogue's store boxes.
-    static constexpr int SP = BN == 256 ? 3 : BN == 128 ? 6 : BN == 64 ? 10 : 12;
-    static constexpr int SU = BN == 256 ? 2 : 3;
-    static constexpr int PA = BM * BKP;
-    static constexpr int PB = BN * BKP;
+    // A widened slot comes back only after its MMAs complete (~500 cycles)
+    // and the next widening (~700 cycles) is done, so narrow tiles, whose
+    // MMAs are short, keep more widened slots; the packed ring keeps 100+ KB
+    // of the weight stream in flight.
+    static constexpr int SP = BN == 256 ? 3 : BN == 192 ? 5 : BN == 128 ? 3 : BN == 64 ? 4 : BN == 32 ? 5 : 3;
+    static constexpr int SU = BN >= 192 ? 2 : BN == 128 ? 4 : BN == 64 ? 5 : 6;
+    // The widening warps split into UG groups that take alternate stages, so
+    // the hand-off latency of one stage overlaps the widening of the next.
+    static constexpr int UG = BN >= 192 ? 1 : 2;
+    static_assert(SU >= UG, "each group needs a widened stage of its own");
+    // Packed stages of the narrow tiles carry PKB bytes of each row (PSUB
+    // K-blocks), so the weight stream is read in longer contiguous pieces;
+    // the widening turns each packed stage into PSUB widened K-blocks.
+    static constexpr int PKB = (!SWAP && BN >= 192) ? 64 : BN == 16 ? 256 : 128;
+    static constexpr int PSUB = PKB / BKP;
+    static constexpr int PA = BM * PKB;
+    static constexpr int PB = BN * PKB;
     static constexpr int UA = BM * BK;
     static constexpr int UB = BN * BK;
     static constexpr int ST = SWAP ? 0 : kEpiWarps * 2 * kStoreBox * kStoreBox * 2;  // store boxes
@@ -85,7 +100,8 @@ struct Cfg {
     // Each accumulator buffer is read 32 columns at a time, so buffers are at
     // least 32 columns apart and the allocation covers two of them.
     static constexpr int ACC_STRIDE = BN < 32 ? 32 : BN;
-    static constexpr int TMEM_COLS = 2 * ACC_STRIDE;        // 64 .. 512, a power of two
+    static constexpr int TMEM_COLS = 2 * ACC_STRIDE <= 64 ? 64 : 2 * ACC_STRIDE <= 128 ? 128
+                                     : 2 * ACC_STRIDE <= 256 ? 256 : 512;   // power of two
     static constexpr int JW = BN < 32 ? BN : 32;             // valid columns per 32-wide read
     static_assert(UB % 1024 == 0, "widened B tiles must stay 1024-aligned");
     static_assert(ST % 1024 == 0, "store boxes must stay 1024-aligned");
@@ -170,10 +186,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::SP; ++s) {
             ptx::mbar_init(full_p(s), 1);
-            ptx::mbar_init(empty_p(s), kUnpWarps);
+            ptx::mbar_init(empty_p(s), C::PSUB * (kUnpWarps / C::UG));
         }
         for (int s = 0; s < C::SU; ++s) {
-            ptx::mbar_init(full_u(s), kUnpWarps);
+            ptx::mbar_init(full_u(s), kUnpWarps / C::UG);
             ptx::mbar_init(empty_u(s), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -205,66 +221,76 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     const int tiles_a = (rowsA + BM - 1) / BM;
     const int tiles_b = (rowsB + BN - 1) / BN;
     const int num_tiles = tiles_a * tiles_b;
-    const int num_kb = (K / 2 + BKP - 1) / BKP;
+    const int num_kp = (K / 2 + C::PKB - 1) / C::PKB;   // packed stages per tile
+    const int num_kb = num_kp * C::PSUB;                // widened K-blocks per tile
 
+    // The producer and MMA warps run their loops with all 32 lanes (so the
+    // addresses and descriptors stay warp-uniform) and let one elected lane
+    // issue each TMA copy, MMA and commit.
     if (warp == kWarpTma) {
-        if (lane == 0) {
-            int ps = 0;
-            uint32_t ph = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                const int ta = tile % tiles_a, tb = tile / tiles_a;
-                for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!ptx::mbar_wait(empty_p(ps), ph ^ 1, abort_flag)) { ok = false; break; }
+        const bool leader = ptx::elect_one();
+        int ps = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            const int ta = tile % tiles_a, tb = tile / tiles_a;
+            for (int kp = 0; kp < num_kp; ++kp) {
+                if (!ptx::mbar_wait(empty_p(ps), ph ^ 1, abort_flag)) { ok = false; break; }
+                if (leader) {
                     ptx::mbar_arrive_expect_tx(full_p(ps), C::PA + C::PB);
-                    ptx::tma_load_2d(sbase + C::OFF_PA + ps * C::PA, &tmA, full_p(ps), kb * BKP,
+                    ptx::tma_load_2d(sbase + C::OFF_PA + ps * C::PA, &tmA, full_p(ps), kp * C::PKB,
                                      ta * BM);
-                    ptx::tma_load_2d(sbase + C::OFF_PB + ps * C::PB, &tmB, full_p(ps), kb * BKP,
+                    ptx::tma_load_2d(sbase + C::OFF_PB + ps * C::PB, &tmB, full_p(ps), kp * C::PKB,
                                      tb * BN);
-                    if (++ps == C::SP) { ps = 0; ph ^= 1; }
                 }
+                __syncwarp();
+                if (++ps == C::SP) { ps = 0; ph ^= 1; }
             }
-            if (!ok) {
-                // Let copies already in flight land before the CTA exits.
-                for (int s = 0; s < C::SP; ++s) {
-                    volatile int never = 0;
-                    ptx::mbar_wait(full_p(s), ph ^ (s < ps ? 0u : 1u), &never, 10000000ull);
-                }
+        }
+        if (!ok && leader) {
+            // Let copies already in flight land before the CTA exits.
+            for (int s = 0; s < C::SP; ++s) {
+                volatile int never = 0;
+                ptx::mbar_wait(full_p(s), ph ^ (s < ps ? 0u : 1u), &never, 10000000ull);
             }
         }
     } else if (warp == kWarpMma) {
-        if (lane == 0) {
-            constexpr uint32_t idesc = ptx::idesc_i8(BM, BN);
-            int us = 0;
-            uint32_t ph = 0;
-            int local = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
-                const int b = local & 1;
-                const uint32_t aph = (local >> 1) & 1;
-                if (!ptx::mbar_wait(acc_empty(b), aph ^ 1, abort_flag)) { ok = false; break; }
+        const bool leader = ptx::elect_one();
+        constexpr uint32_t idesc = ptx::idesc_i8(BM, BN);
+        int us = 0;
+        uint32_t ph = 0;
+        int local = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+            const int b = local & 1;
+            const uint32_t aph = (local >> 1) & 1;
+            if (!ptx::mbar_wait(acc_empty(b), aph ^ 1, abort_flag)) { ok = false; break; }
+            ptx::tc_fence_after();
+            const uint32_t d = tmem_base + static_cast<uint32_t>(b * C::ACC_STRIDE);
+            for (int kb = 0; kb < num_kb; ++kb) {
+                if (!ptx::mbar_wait(full_u(us), ph, abort_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
-                const uint32_t d = tmem_base + static_cast<uint32_t>(b * C::ACC_STRIDE);
-                for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!ptx::mbar_wait(full_u(us), ph, abort_flag)) { ok = false; break; }
-                    ptx::tc_fence_after();
-                    const uint32_t a0 = sbase + C::OFF_UA + us * C::UA;
-                    const uint32_t b0 = sbase + C::OFF_UB + us * C::UB;
+                const uint32_t a0 = sbase + C::OFF_UA + us * C::UA;
+                const uint32_t b0 = sbase + C::OFF_UB + us * C::UB;
+                if (leader) {
 #pragma unroll
                     for (int j = 0; j < BK / 32; ++j)
                         ptx::mma_i8_ss(d, ptx::sw128_kmajor_desc(a0 + 32 * j),
                                        ptx::sw128_kmajor_desc(b0 + 32 * j), idesc,
                                        (kb | j) != 0 ? 1u : 0u);
                     ptx::tc_commit(empty_u(us));
-                    if (++us == C::SU) { us = 0; ph ^= 1; }
                 }
-                if (ok) ptx::tc_commit(acc_full(b));
+                __syncwarp();
+                if (++us == C::SU) { us = 0; ph ^= 1; }
             }
-            // Wait for every MMA this thread issued before TMEM is released.
-            ptx::tc_commit(drain_bar);
-            volatile int never = 0;
-            ptx::mbar_wait(drain_bar, 0, &never, 100000000ull);
+            if (ok && leader) ptx::tc_commit(acc_full(b));
+            __syncwarp();
         }
+        // Wait for every MMA this warp issued before TMEM is released.
+        if (leader) ptx::tc_commit(drain_bar);
+        __syncwarp();
+        volatile int never = 0;
+        ptx::mbar_wait(drain_bar, 0, &never, 100000000ull);
     } else if (warp < kWarpUnp0) {
         // ------------------------------------------------------------ epilogue
         const int e = warp - kWarpEpi0;               // 0 .. 7
@@ -400,55 +426,60 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         if (tma_out && lane == 0) ptx::bulk_wait_all();
     } else {
         // ------------------------------------------------------------ widening
-        // Thread ut widens 16-byte packed chunks ut, ut + 256, ...; since 256 is
-        // a multiple of 4 chunks per row and of 8 rows per swizzle group, its
-        // chunk column and swizzle phase are the same for every one of them.
-        const int ut = threadIdx.x - kWarpUnp0 * 32;   // 0 .. 255
+        // Group g of UG takes stages g, g + UG, g + 2 UG, ... (counted over all
+        // tiles and K-blocks of this CTA).  Within a group, thread ut widens
+        // 16-byte packed chunks ut, ut + GT, ... (GT threads per group); GT is
+        // a multiple of 4 chunks per row and of 8 rows per swizzle group, so a
+        // thread's chunk column and swizzle phase never change.
+        constexpr int GT = kUnpWarps * 32 / C::UG;
+        const int ug = (threadIdx.x - kWarpUnp0 * 32) / GT;
+        const int ut = (threadIdx.x - kWarpUnp0 * 32) % GT;
         constexpr int kChunks = (BM + BN) * 4;          // 16-byte packed chunks per stage
-        constexpr int kPer = (kChunks + kUnpWarps * 32 - 1) / (kUnpWarps * 32);
+        constexpr int kPer = (kChunks + GT - 1) / GT;
+        constexpr int kRowStep = GT / 4;
         const uint32_t c = static_cast<uint32_t>(ut & 3);
         const uint32_t sw8 = static_cast<uint32_t>((ut >> 2) & 7);
         const uint32_t lo_off = ((2u * c) ^ sw8) << 4;
         const uint32_t hi_off = ((2u * c + 1u) ^ sw8) << 4;
-        int ps = 0, us = 0;
-        uint32_t pph = 0, uph = 0;
-        bool ok = true;
-        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-            for (int kb = 0; kb < num_kb; ++kb) {
-                if (!ptx::mbar_wait(full_p(ps), pph, abort_flag)) { ok = false; break; }
-                if (!ptx::mbar_wait(empty_u(us), uph ^ 1, abort_flag)) { ok = false; break; }
-                const uint32_t pa = sbase + C::OFF_PA + ps * C::PA;
-                const uint32_t pb = sbase + C::OFF_PB + ps * C::PB;
-                const uint32_t ua = sbase + C::OFF_UA + us * C::UA;
-                const uint32_t ub = sbase + C::OFF_UB + us * C::UB;
-                uint4 w[kPer];
+        const int my_tiles = num_tiles > static_cast<int>(blockIdx.x)
+                                 ? (num_tiles - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1
+                                 : 0;
+        const int total = my_tiles * num_kb;            // stages this CTA runs
+        for (int n = ug; n < total; n += C::UG) {
+            const int np = n / C::PSUB, sub = n % C::PSUB;   // packed stage, K-block in it
+            const int ps = np % C::SP, us = n % C::SU;
+            const uint32_t pph = (np / C::SP) & 1, uph = (n / C::SU) & 1;
+            if (!ptx::mbar_wait(full_p(ps), pph, abort_flag)) break;
+            if (!ptx::mbar_wait(empty_u(us), uph ^ 1, abort_flag)) break;
+            const uint32_t pa = sbase + C::OFF_PA + ps * C::PA;
+            const uint32_t pb = sbase + C::OFF_PB + ps * C::PB;
+            const uint32_t ua = sbase + C::OFF_UA + us * C::UA;
+            const uint32_t ub = sbase + C::OFF_UB + us * C::UB;
+            uint4 w[kPer];
 #pragma unroll
-                for (int i = 0; i < kPer; ++i) {
-                    const int row = (ut >> 2) + 64 * i;   // rows of A, then rows of B
-                    if (row < BM + BN) {
-                        const uint32_t src = row < BM ? pa + row * 64 : pb + (row - BM) * 64;
-                        w[i] = lds128(src + c * 16);
-                    }
+            for (int i = 0; i < kPer; ++i) {
+                const int row = (ut >> 2) + kRowStep * i;   // rows of A, then rows of B
+                if (row < BM + BN) {
+                    const uint32_t src = row < BM ? pa + row * C::PKB : pb + (row - BM) * C::PKB;
+                    w[i] = lds128(src + sub * BKP + c * 16);
                 }
+            }
 #pragma unroll
-                for (int i = 0; i < kPer; ++i) {
-                    const int row = (ut >> 2) + 64 * i;
-                    if (row < BM + BN) {
-                        const uint32_t dst = row < BM ? ua + row * 128 : ub + (row - BM) * 128;
-                        const uint32_t hm = 0xF0F0F0F0u;
-                        sts128(dst + lo_off, (w[i].x << 4) & hm, (w[i].y << 4) & hm,
-                               (w[i].z << 4) & hm, (w[i].w << 4) & hm);
-                        sts128(dst + hi_off, w[i].x & hm, w[i].y & hm, w[i].z & hm, w[i].w & hm);
-                    }
+            for (int i = 0; i < kPer; ++i) {
+                const int row = (ut >> 2) + kRowStep * i;
+                if (row < BM + BN) {
+                    const uint32_t dst = row < BM ? ua + row * 128 : ub + (row - BM) * 128;
+                    const uint32_t hm = 0xF0F0F0F0u;
+                    sts128(dst + lo_off, (w[i].x << 4) & hm, (w[i].y << 4) & hm,
+                           (w[i].z << 4) & hm, (w[i].w << 4) & hm);
+                    sts128(dst + hi_off, w[i].x & hm, w[i].y & hm, w[i].z & hm, w[i].w & hm);
                 }
-                ptx::fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    ptx::mbar_arrive(empty_p(ps));
-                    ptx::mbar_arrive(full_u(us));
-                }
-                if (++ps == C::SP) { ps = 0; pph ^= 1; }
-                if (++us == C::SU) { us = 0; uph ^= 1; }
+            }
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                ptx::mbar_arrive(empty_p(ps));
+                ptx::mbar_arrive(full_u(us));
             }
         }
     }

@@ -91,7 +91,8 @@ def test_prepare_edge_rows():
 
 @pytest.mark.parametrize("M,N,K", [(1, 16, 64), (5, 72, 192), (16, 128, 1024), (17, 300, 512),
                                    (64, 1000, 768), (100, 256, 256), (128, 384, 1024),
-                                   (129, 257, 320), (300, 600, 1536), (513, 96, 128)])
+                                   (129, 257, 320), (300, 600, 1536), (513, 96, 128),
+                                   (1024, 4096, 128)])
 def test_gemm_s32_bit_exact(M, N, K):
     rng = np.random.default_rng(M * 7 + N)
     a = rng.integers(-7, 8, size=(M, K)).astype(np.int8)
