@@ -184,6 +184,82 @@ def convrot_debug_timeout_probe(timeout_ns: int, stream=None):
            "convrot_debug_timeout_probe")
 
 
+class HostPipeline:
+    """The layer (or a chain of layers) on pinned host buffers, with the
+    copies overlapped with the compute.
+
+    Rows are independent, so the batch is cut into row chunks: chunk i is
+    copied host -> device on one stream, run through ``convrot_linear`` for
+    each layer on the caller's stream, and copied back on a third stream,
+    while chunk i+1 is already being copied in.  The results are identical
+    to one whole-batch call.  Device buffers are allocated once here.
+
+    ``layers`` is a list of (qweight, scales, bias or None, group) with each
+    layer's in_features equal to the previous layer's out_features.
+
+    With ``graph=True`` the first call runs eagerly and the second call for
+    the same host buffers captures the whole multi-stream sequence into one
+    CUDA graph, which later calls replay (one launch per call instead of a
+    dozen stream operations per chunk).
+    """
+
+    def __init__(self, M: int, K: int, layers, chunks: int = 8, device=None, graph: bool = True):
+        self.M, self.K, self.layers = M, K, layers
+        self.use_graph, self._graph, self._key, self._calls = graph, None, None, 0
+        dev = torch.device("cuda") if device is None else torch.device(device)
+        widths = [K] + [qw.shape[0] for qw, *_ in layers]
+        # chunk rows keep every row slice 16-byte aligned (N % 8 == 0 for all outputs)
+        if any(w % 8 for w in widths[1:]):
+            chunks = 1
+        step = max(1, -(-M // max(1, chunks)))
+        self.ranges = [(r, min(M, r + step)) for r in range(0, M, step)]
+        self.acts = [torch.empty(M, w, dtype=torch.bfloat16, device=dev) for w in widths]
+        self.ws = [torch.empty(max(1, convrot_linear_workspace_size(step, widths[i])),
+                               dtype=torch.uint8, device=dev) for i in range(len(layers))]
+        self.s_in = torch.cuda.Stream(device=dev)
+        self.s_out = torch.cuda.Stream(device=dev)
+        n = len(self.ranges)
+        self.e_start = torch.cuda.Event()
+        self.e_in = [torch.cuda.Event() for _ in range(n)]
+        self.e_done = [torch.cuda.Event() for _ in range(n)]
+        self.e_out = torch.cuda.Event()
+
+    def __call__(self, x_host: torch.Tensor, y_host: torch.Tensor, stream=None):
+        main = torch.cuda.current_stream() if stream is None else stream
+        key = (x_host.data_ptr(), y_host.data_ptr())
+        if self.use_graph and self._calls >= 1:
+            if self._graph is None or self._key != key:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    self._enqueue(x_host, y_host, torch.cuda.current_stream())
+                self._graph, self._key = g, key
+            with torch.cuda.stream(main):
+                self._graph.replay()
+            return y_host
+        self._calls += 1
+        return self._enqueue(x_host, y_host, main)
+
+    def _enqueue(self, x_host, y_host, main):
+        self.e_start.record(main)
+        self.s_in.wait_event(self.e_start)
+        self.s_out.wait_event(self.e_start)
+        for i, (r0, r1) in enumerate(self.ranges):
+            with torch.cuda.stream(self.s_in):
+                self.acts[0][r0:r1].copy_(x_host[r0:r1], non_blocking=True)
+                self.e_in[i].record(self.s_in)
+            main.wait_event(self.e_in[i])
+            for l, (qw, sw, b, group) in enumerate(self.layers):
+                convrot_linear(self.acts[l][r0:r1], qw, sw, b, group, self.ws[l],
+                               out=self.acts[l + 1][r0:r1], stream=main)
+            self.e_done[i].record(main)
+            self.s_out.wait_event(self.e_done[i])
+            with torch.cuda.stream(self.s_out):
+                y_host[r0:r1].copy_(self.acts[-1][r0:r1], non_blocking=True)
+        self.e_out.record(self.s_out)
+        main.wait_event(self.e_out)
+        return y_host
+
+
 class ConvRotLinear:
     """A linear layer held as rotated, row-quantised, packed INT4 weights.
 

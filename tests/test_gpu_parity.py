@@ -246,3 +246,25 @@ def test_bad_arguments_raise():
     with pytest.raises(cr.ConvRotError) as e:
         cr.convrot_debug_rotate_f32(misaligned, 64)
     assert e.value.status == 4
+
+
+# ---------------------------------------------------------------------------
+# host-buffer pipeline
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,chunks", [(1000, 8), (37, 4), (256, 1)])
+def test_host_pipeline_matches_device_call(M, chunks):
+    up = _layer(M, 512, 320, 64, seed=M)
+    # chain of two layers: 512 -> 320 -> 96
+    w1 = _layer(M, 512, 320, 64, seed=M + 2)
+    w2 = _layer(M, 320, 96, 64, seed=M + 3)
+    qw1, sw1 = cr.convrot_quantize_weight(_dev(w1.w), 64)
+    qw2, sw2 = cr.convrot_quantize_weight(_dev(w2.w), 64)
+    b1, b2 = _dev(w1.b), _dev(w2.b)
+    x = up.x
+    ref = cr.convrot_linear(cr.convrot_linear(_dev(x), qw1, sw1, b1, 64), qw2, sw2, b2, 64)
+    pipe = cr.HostPipeline(M, 512, [(qw1, sw1, b1, 64), (qw2, sw2, b2, 64)], chunks=chunks)
+    y_host = torch.empty(M, 96, dtype=torch.bfloat16).pin_memory()
+    pipe(x.pin_memory(), y_host)
+    torch.cuda.synchronize()
+    assert torch.equal(y_host, ref.cpu())
