@@ -124,6 +124,23 @@ convrot_status convrot_debug_gemm_s32(const uint8_t *qx, const uint8_t *qw, int6
                                       int64_t K, int32_t *acc, convrot_stream_t stream);
 
 /*
+ * Test hook: steps 3-4 (out_s32 = 0: y [M][N] bf16, as convrot_linear_prepared)
+ * or step 3 alone (out_s32 = 1: acc [M][N] int32, sx / sw / bias unused) with
+ * the token-major GEMM forced to one tile shape, so that each shape can be
+ * checked whatever the automatic choice for (M, N, K) would be:
+ *   tiles = 0  automatic (as the entry points above);
+ *           1  128 x 256 tiles, both operands widened in shared memory;
+ *           2  128 x 192 tiles, A widened into TMEM;
+ *           3  256 x 192 tiles on CTA pairs (cta_group::2).
+ * Returns CONVROT_ERR_SHAPE for any other value and CONVROT_ERR_UNSUPPORTED
+ * when the device cannot co-schedule CTA pairs (tiles = 3).
+ */
+convrot_status convrot_debug_gemm_tiles(const uint8_t *qx, const float *sx, const uint8_t *qw,
+                                        const float *sw, const void *bias_bf16, int64_t M,
+                                        int64_t N, int64_t K, int tiles, int out_s32, void *out,
+                                        convrot_stream_t stream);
+
+/*
  * The whole layer, like convrot_linear, for callers that cannot give the
  * library any device memory of their own: a plugin called by a host runtime
  * that owns every allocation and passes no workspace, or a caller on a

@@ -57,6 +57,7 @@ def lib() -> ctypes.CDLL:
             "convrot_check_device_error": [P],
             "convrot_debug_timeout_probe": [I64, P],
             "convrot_linear_noalloc": [P, P, P, P, I64, I64, I64, I, P, P],
+            "convrot_debug_gemm_tiles": [P, P, P, P, P, I64, I64, I64, I, I, P, P],
         }
         for name, args in sigs.items():
             f = getattr(L, name)
@@ -171,6 +172,23 @@ def convrot_debug_gemm_s32(qx, qw, K: int, out=None, stream=None):
     out = torch.empty(M, N, dtype=torch.int32, device=qx.device) if out is None else out
     _check(lib().convrot_debug_gemm_s32(_p(qx), _p(qw), M, N, K, _p(out), _stream(stream)),
            "convrot_debug_gemm_s32")
+    return out
+
+
+# tile shapes of the token-major GEMM (convrot_debug_gemm_tiles)
+TILES_AUTO, TILES_128x256, TILES_128x192, TILES_256x192_PAIR = 0, 1, 2, 3
+
+
+def convrot_debug_gemm_tiles(qx, sx, qw, sw, bias, K: int, tiles: int, out_s32: bool = False,
+                             out=None, stream=None):
+    """Steps 3-4 (bf16 y) or step 3 alone (int32 acc, out_s32=True) with the
+    GEMM forced to one tile shape (TILES_*)."""
+    M, N = qx.shape[0], qw.shape[0]
+    dt = torch.int32 if out_s32 else torch.bfloat16
+    out = torch.empty(M, N, dtype=dt, device=qx.device) if out is None else out
+    _check(lib().convrot_debug_gemm_tiles(_p(qx), _p(sx), _p(qw), _p(sw), _p(bias), M, N, K,
+                                          int(tiles), int(bool(out_s32)), _p(out),
+                                          _stream(stream)), "convrot_debug_gemm_tiles")
     return out
 
 

@@ -26,6 +26,7 @@ struct DeviceState {
     bool ready = false;
     convrot_status status = CONVROT_OK;
     int num_sms = 0;
+    int pair_clusters = 0;   // co-resident 2-CTA clusters of the pair GEMM (0: none)
 };
 
 DeviceState g_dev[kMaxDevices];
@@ -94,6 +95,30 @@ convrot_status device_setup(int *dev_out) {
     ok &= set_smem(gemm::gemm_kernel<32, true, true>, gemm::Cfg<32, true>::SMEM_BYTES);
     ok &= set_smem(gemm::gemm_kernel<64, true, true>, gemm::Cfg<64, true>::SMEM_BYTES);
     ok &= set_smem(gemm::gemm_kernel<128, true, true>, gemm::Cfg<128, true>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<192, false, false, true>, gemm::Cfg<192, false, true>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<192, false, true, true>, gemm::Cfg<192, false, true>::SMEM_BYTES);
+    if (ok) {
+        // How many CTA pairs fit on the device at once (pairs need two SMs
+        // of one GPC); the pair GEMM's persistent grid is that many clusters.
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1));
+        cfg.blockDim = dim3(gemm::kThreads);
+        cfg.dynamicSmemBytes = gemm::Cfg<192, false, true>::SMEM_BYTES;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, gemm::gemm_kernel<192, false, false, true>, &cfg) !=
+            cudaSuccess) {
+            cudaGetLastError();   // clear it: the 1-CTA kernels remain
+            n = 0;
+        }
+        st.pair_clusters = n;
+    }
     st.num_sms = sms;
     st.status = ok ? CONVROT_OK : CONVROT_ERR_CUDA;
     st.ready = true;
@@ -156,13 +181,13 @@ convrot_status launch_prep(int num_sms, const void *x, int64_t rows, int64_t K, 
 }
 
 bool make_map(CUtensorMap *map, const uint8_t *base, int64_t rows, int64_t K, int box_bytes,
-              int box_rows) {
+              int box_rows, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE) {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_bytes), static_cast<cuuint32_t>(box_rows)};
     const cuuint32_t estr[2] = {1, 1};
     return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(base), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -181,14 +206,18 @@ bool make_out_map(CUtensorMap *map, void *y, int64_t M, int64_t N) {
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool SWAP, bool OUT_S32>
-convrot_status launch_gemm_cfg(int num_sms, const uint8_t *qA, const uint8_t *qB, int64_t rowsA,
+// slots: CTAs (CTA pairs when PAIR) the persistent grid may use.
+template <int BN, bool SWAP, bool OUT_S32, bool PAIR = false>
+convrot_status launch_gemm_cfg(int slots, const uint8_t *qA, const uint8_t *qB, int64_t rowsA,
                                int64_t rowsB, int64_t K, const float *sx, const float *sw,
                                const void *bias, void *out, int64_t M, int64_t N,
                                cudaStream_t stream) {
+    using C = gemm::Cfg<BN, SWAP, PAIR>;
     CUtensorMap tmA, tmB, tmY;
-    constexpr int pkb = gemm::Cfg<BN, SWAP>::PKB;
-    if (!make_map(&tmA, qA, rowsA, K, pkb, gemm::BM) || !make_map(&tmB, qB, rowsB, K, pkb, BN))
+    constexpr int pkb = C::PKB;
+    // A widened into TMEM reads its packed rows 64-byte swizzled.
+    const CUtensorMapSwizzle swa = C::ATM ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE;
+    if (!make_map(&tmA, qA, rowsA, K, pkb, gemm::BM, swa) || !make_map(&tmB, qB, rowsB, K, pkb, C::BR))
         return CONVROT_ERR_CUDA;
     int use_tma_store = 0;
     if (!SWAP && !OUT_S32 && N % 8 == 0) {
@@ -197,8 +226,8 @@ convrot_status launch_gemm_cfg(int num_sms, const uint8_t *qA, const uint8_t *qB
     } else {
         tmY = tmA;   // unused by the kernel
     }
-    const int64_t tiles = ((rowsA + gemm::BM - 1) / gemm::BM) * ((rowsB + BN - 1) / BN);
-    const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+    const int64_t tiles = ((rowsA + C::TM - 1) / C::TM) * ((rowsB + BN - 1) / BN);
+    const int grid = static_cast<int>(tiles < slots ? tiles : slots) * C::CG;
     // Programmatic dependent launch: the GEMM's set-up (barriers, TMEM,
     // descriptor prefetch) overlaps the end of the preceding kernel on the
     // stream (normally the prep kernel); the kernel waits for that grid's
@@ -206,28 +235,37 @@ convrot_status launch_gemm_cfg(int num_sms, const uint8_t *qA, const uint8_t *qB
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(gemm::kThreads);
-    cfg.dynamicSmemBytes = gemm::Cfg<BN, SWAP>::SMEM_BYTES;
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = C::CG;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = PAIR ? 2 : 1;
     const cudaError_t e = cudaLaunchKernelEx(
-        &cfg, gemm::gemm_kernel<BN, SWAP, OUT_S32>, tmA, tmB, tmY, use_tma_store,
+        &cfg, gemm::gemm_kernel<BN, SWAP, OUT_S32, PAIR>, tmA, tmB, tmY, use_tma_store,
         static_cast<int>(rowsA), static_cast<int>(rowsB), static_cast<int>(K), sx, sw,
         static_cast<const uint16_t *>(bias), out, static_cast<int>(M), static_cast<int>(N));
     return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 
+// Tile shapes of the token-major path (more than 128 tokens).
+enum TileChoice { kTilesAuto = 0, kTiles128x256 = 1, kTiles128x192 = 2, kTiles256x192Pair = 3 };
+
 // Path choice: up to 128 tokens the weights take the 128-row MMA side
-// (skinny form, N-side tile = tokens rounded up to 16); otherwise 128 x 256
-// tiles with tokens on the M side.
+// (skinny form, N-side tile = tokens rounded up to 16); otherwise tokens on
+// the M side, with the tile shape that finishes first.
 template <bool OUT_S32>
-convrot_status launch_gemm(int num_sms, const uint8_t *qx, const float *sx, const uint8_t *qw,
-                           const float *sw, const void *bias, int64_t M, int64_t N, int64_t K,
-                           void *out, cudaStream_t stream) {
-    if (M <= 128) {
+convrot_status launch_gemm(const DeviceState &ds, const uint8_t *qx, const float *sx,
+                           const uint8_t *qw, const float *sw, const void *bias, int64_t M,
+                           int64_t N, int64_t K, void *out, cudaStream_t stream,
+                           int tiles = kTilesAuto) {
+    const int num_sms = ds.num_sms;
+    if (tiles == kTilesAuto && M <= 128) {
         if (M <= 16)
             return launch_gemm_cfg<16, true, OUT_S32>(num_sms, qw, qx, N, M, K, sx, sw, bias, out, M,
                                                       N, stream);
@@ -240,19 +278,35 @@ convrot_status launch_gemm(int num_sms, const uint8_t *qx, const float *sx, cons
         return launch_gemm_cfg<128, true, OUT_S32>(num_sms, qw, qx, N, M, K, sx, sw, bias, out, M, N,
                                                    stream);
     }
-    // Wider tiles need fewer widened bytes per output, but a tile count just
-    // above a multiple of the SM count wastes most of a wave.  The widening
-    // work of a tile is proportional to its rows of A plus B (128 + BN).
-    const int64_t mt = (M + gemm::BM - 1) / gemm::BM;
-    const auto cost = [&](int64_t bn) {
-        const int64_t tiles = mt * ((N + bn - 1) / bn);
-        return ((tiles + num_sms - 1) / num_sms) * (gemm::BM + bn);
-    };
-    if (cost(192) < cost(256))
+    if (tiles == kTilesAuto) {
+        // Time of one K-block step of a wave of tiles, in cycles, as measured
+        // on these kernels: the 128 x 256 tile widens both operands through
+        // shared memory (~940); the 128 x 192 tile keeps A in TMEM (~670);
+        // the 256 x 192 pair splits B between two SMs, so each SM moves 40%
+        // fewer shared-memory bytes per MMA (~620 for twice the rows).
+        // A tile count just above a multiple of the slots wastes a wave.
+        const auto waves = [](int64_t t, int64_t slots) { return (t + slots - 1) / slots; };
+        const int64_t n192 = (N + 191) / 192, n256 = (N + 255) / 256;
+        const int64_t c_ss = waves(((M + 127) / 128) * n256, num_sms) * 940;
+        const int64_t c_atm = waves(((M + 127) / 128) * n192, num_sms) * 670;
+        const int64_t c_pair =
+            ds.pair_clusters > 0 ? waves(((M + 255) / 256) * n192, ds.pair_clusters) * 620 : INT64_MAX;
+        tiles = c_pair <= c_atm && c_pair <= c_ss ? kTiles256x192Pair
+                : c_atm <= c_ss                   ? kTiles128x192
+                                                  : kTiles128x256;
+    }
+    if (tiles == kTiles256x192Pair) {
+        if (ds.pair_clusters <= 0) return CONVROT_ERR_UNSUPPORTED;
+        return launch_gemm_cfg<192, false, OUT_S32, true>(ds.pair_clusters, qx, qw, M, N, K, sx, sw,
+                                                          bias, out, M, N, stream);
+    }
+    if (tiles == kTiles128x192)
         return launch_gemm_cfg<192, false, OUT_S32>(num_sms, qx, qw, M, N, K, sx, sw, bias, out, M,
                                                     N, stream);
-    return launch_gemm_cfg<256, false, OUT_S32>(num_sms, qx, qw, M, N, K, sx, sw, bias, out, M, N,
-                                                stream);
+    if (tiles == kTiles128x256)
+        return launch_gemm_cfg<256, false, OUT_S32>(num_sms, qx, qw, M, N, K, sx, sw, bias, out, M,
+                                                    N, stream);
+    return CONVROT_ERR_SHAPE;
 }
 
 convrot_status check_gemm_args(const uint8_t *qx, const uint8_t *qw, int64_t M, int64_t N,
@@ -325,7 +379,7 @@ convrot_status convrot_linear_prepared(const uint8_t *qx, const float *sx, const
         return CONVROT_ERR_ALIGN;
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
-    return launch_gemm<false>(g_dev[dev].num_sms, qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream);
+    return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream);
 }
 
 convrot_status convrot_linear(const void *x_bf16, const uint8_t *qw, const float *sw,
@@ -350,7 +404,7 @@ convrot_status convrot_linear(const void *x_bf16, const uint8_t *qw, const float
     float *sx = reinterpret_cast<float *>(qx + round256(static_cast<size_t>(M) * (K / 2)));
     if ((st = launch_prep(g_dev[dev].num_sms, x_bf16, M, K, group, qx, sx, nullptr, stream)) != CONVROT_OK)
         return st;
-    return launch_gemm<false>(g_dev[dev].num_sms, qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream);
+    return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream);
 }
 
 convrot_status convrot_debug_rotate_f32(const void *x_bf16, int64_t M, int64_t K, int group,
@@ -375,8 +429,29 @@ convrot_status convrot_debug_gemm_s32(const uint8_t *qx, const uint8_t *qw, int6
     if (!aligned16(acc)) return CONVROT_ERR_ALIGN;
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
-    return launch_gemm<true>(g_dev[dev].num_sms, qx, nullptr, qw, nullptr, nullptr, M, N, K, acc,
+    return launch_gemm<true>(g_dev[dev], qx, nullptr, qw, nullptr, nullptr, M, N, K, acc,
                              stream);
+}
+
+convrot_status convrot_debug_gemm_tiles(const uint8_t *qx, const float *sx, const uint8_t *qw,
+                                        const float *sw, const void *bias_bf16, int64_t M,
+                                        int64_t N, int64_t K, int tiles, int out_s32, void *out,
+                                        convrot_stream_t stream) {
+    if (M < 0 || N < 0) return CONVROT_ERR_SHAPE;
+    if (tiles < kTilesAuto || tiles > kTiles256x192Pair) return CONVROT_ERR_SHAPE;
+    if (M == 0 || N == 0) return CONVROT_OK;
+    convrot_status st = check_gemm_args(qx, qw, M, N, K);
+    if (st != CONVROT_OK) return st;
+    if (!out || (!out_s32 && (!sx || !sw))) return CONVROT_ERR_NULL;
+    if (!aligned16(out) || (!out_s32 && (!aligned16(sx) || !aligned16(sw) ||
+                                         (bias_bf16 && !aligned16(bias_bf16)))))
+        return CONVROT_ERR_ALIGN;
+    int dev;
+    if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    if (out_s32)
+        return launch_gemm<true>(g_dev[dev], qx, nullptr, qw, nullptr, nullptr, M, N, K, out, stream,
+                                 tiles);
+    return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, out, stream, tiles);
 }
 
 convrot_status convrot_check_device_error(convrot_stream_t stream) {
@@ -478,6 +553,6 @@ extern "C" convrot_status convrot_linear_noalloc(const void *x_bf16, const uint8
     float *sx = reinterpret_cast<float *>(qx + round256(static_cast<size_t>(M) * (K / 2)));
     if ((st = launch_prep(g_dev[dev].num_sms, x_bf16, M, K, group, qx, sx, nullptr, stream)) != CONVROT_OK)
         return st;
-    return launch_gemm<false>(g_dev[dev].num_sms, qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16,
+    return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16,
                               stream);
 }

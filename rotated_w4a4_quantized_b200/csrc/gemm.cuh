@@ -55,9 +55,16 @@ constexpr int kWarpUnp0 = kWarpEpi0 + kEpiWarps, kUnpWarps = 8;
 constexpr int kThreads = (kWarpUnp0 + kUnpWarps) * 32;    // 576
 constexpr int kStoreBox = 32;    // epilogue TMA-store box: 32 rows x 32 bf16
 
-template <int BN, bool SWAP>
+// PAIR: a 2-CTA cluster computes one 256 x BN tile with cta_group::2 MMAs;
+// each CTA holds 128 rows of A (in its TMEM), BN / 2 rows of B (in its
+// shared memory) and 128 rows of the accumulator.
+template <int BN, bool SWAP, bool PAIR = false>
 struct Cfg {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "kind::i8 with M=128 needs N%16==0");
+    static_assert(!PAIR || (!SWAP && BN == 192), "the CTA pair runs 256 x 192 tiles");
+    static constexpr int CG = PAIR ? 2 : 1;          // tcgen05 CTA group
+    static constexpr int TM = PAIR ? 2 * BM : BM;    // rows of A per tile
+    static constexpr int BR = PAIR ? BN / 2 : BN;    // rows of B per CTA
     static_assert(BN < 64 || (BN / 2) % 32 == 0, "each epilogue half covers whole 32-column reads");
     // Packed stages keep HBM loads in flight; the narrow (skinny) tiles are
     // bound by the weight stream, so they trade widened stages for more
@@ -66,8 +73,12 @@ struct Cfg {
     // and the next widening (~700 cycles) is done, so narrow tiles, whose
     // MMAs are short, keep more widened slots; the packed ring keeps 100+ KB
     // of the weight stream in flight.
-    static constexpr int SP = BN == 256 ? 3 : BN == 192 ? 5 : BN == 128 ? 3 : BN == 64 ? 4 : BN == 32 ? 5 : 3;
-    static constexpr int SU = BN >= 192 ? 2 : BN == 128 ? 4 : BN == 64 ? 5 : 6;
+    // ATM: the 128 x 192 tile widens operand A straight into TMEM (the MMA
+    // reads A from there), so only B passes through widened shared memory;
+    // TMEM holds two 192-column accumulators plus SU 32-column A stages.
+    static constexpr bool ATM = PAIR || (!SWAP && BN == 192);
+    static constexpr int SP = PAIR ? 8 : ATM ? 4 : BN == 256 ? 3 : BN == 192 ? 5 : BN == 128 ? 3 : BN == 64 ? 4 : BN == 32 ? 5 : 3;
+    static constexpr int SU = ATM ? 4 : BN >= 192 ? 2 : BN == 128 ? 4 : BN == 64 ? 5 : 6;
     // The widening warps split into UG groups that take alternate stages, so
     // the hand-off latency of one stage overlaps the widening of the next.
     static constexpr int UG = BN >= 192 ? 1 : 2;
@@ -78,10 +89,11 @@ struct Cfg {
     static constexpr int PKB = (!SWAP && BN >= 192) ? 64 : BN == 16 ? 256 : 128;
     static constexpr int PSUB = PKB / BKP;
     static constexpr int PA = BM * PKB;
-    static constexpr int PB = BN * PKB;
-    static constexpr int UA = BM * BK;
-    static constexpr int UB = BN * BK;
-    static constexpr int ST = SWAP ? 0 : kEpiWarps * 2 * kStoreBox * kStoreBox * 2;  // store boxes
+    static constexpr int PB = BR * PKB;
+    static constexpr int UA = ATM ? 0 : BM * BK;
+    static constexpr int UB = BR * BK;
+    static constexpr int SB = 2;   // store boxes per epilogue warp
+    static constexpr int ST = SWAP ? 0 : kEpiWarps * SB * kStoreBox * kStoreBox * 2;
     static constexpr int OFF_UA = 0;                   // 1024-aligned tiles first
     static constexpr int OFF_UB = OFF_UA + SU * UA;
     static constexpr int OFF_ST = OFF_UB + SU * UB;
@@ -100,8 +112,12 @@ struct Cfg {
     // Each accumulator buffer is read 32 columns at a time, so buffers are at
     // least 32 columns apart and the allocation covers two of them.
     static constexpr int ACC_STRIDE = BN < 32 ? 32 : BN;
-    static constexpr int TMEM_COLS = 2 * ACC_STRIDE <= 64 ? 64 : 2 * ACC_STRIDE <= 128 ? 128
-                                     : 2 * ACC_STRIDE <= 256 ? 256 : 512;   // power of two
+    static constexpr int A_OFF = 2 * ACC_STRIDE;              // first A-stage column (ATM)
+    static constexpr int TMEM_NEED = A_OFF + (ATM ? SU * (BK / 4) : 0);
+    static constexpr int TMEM_COLS = TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
+                                     : TMEM_NEED <= 256 ? 256 : 512;   // power of two
+    static_assert(TMEM_NEED <= 512, "TMEM holds 512 columns");
+    static_assert(!ATM || (PSUB == 1 && PKB == 64), "A-in-TMEM reads 64-byte swizzled packed rows");
     static constexpr int JW = BN < 32 ? BN : 32;             // valid columns per 32-wide read
     static_assert(UB % 1024 == 0, "widened B tiles must stay 1024-aligned");
     static_assert(ST % 1024 == 0, "store boxes must stay 1024-aligned");
@@ -159,13 +175,13 @@ __device__ __forceinline__ uint32_t epi_pair(uint32_t r0, uint32_t r1, float sx,
 // OUT_S32: write the integer accumulators (test hook) instead of bf16.
 // tmY (used when !SWAP && !OUT_S32 && use_tma_store): bf16 y [M][N], box
 // 32 x 32, 64-byte swizzle.
-template <int BN, bool SWAP, bool OUT_S32>
+template <int BN, bool SWAP, bool OUT_S32, bool PAIR = false>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmY, int use_tma_store, int rowsA, int rowsB,
             int K, const float *__restrict__ sx, const float *__restrict__ sw,
             const uint16_t *__restrict__ bias, void *__restrict__ out, int M, int N) {
-    using C = Cfg<BN, SWAP>;
+    using C = Cfg<BN, SWAP, PAIR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -182,6 +198,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // Rank in the CTA pair (0 issues the MMAs; the barriers that gather both
+    // CTAs' work live in CTA 0).
+    const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0u;
+    // Arrive on a barrier of CTA 0 (remote for CTA 1 of a pair).
+    auto arrive_leader = [&](uint32_t bar) {
+        if (PAIR && rank != 0) ptx::mbar_arrive_remote(ptx::mapa_shared(bar, 0));
+        else ptx::mbar_arrive(bar);
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::SP; ++s) {
@@ -189,12 +213,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             ptx::mbar_init(empty_p(s), C::PSUB * (kUnpWarps / C::UG));
         }
         for (int s = 0; s < C::SU; ++s) {
-            ptx::mbar_init(full_u(s), kUnpWarps / C::UG);
+            ptx::mbar_init(full_u(s), (PAIR ? 2 : 1) * kUnpWarps / C::UG);
             ptx::mbar_init(empty_u(s), 1);
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(acc_full(b), 1);
-            ptx::mbar_init(acc_empty(b), kEpiWarps);
+            ptx::mbar_init(acc_empty(b), (PAIR ? 2 : 1) * kEpiWarps);
         }
         ptx::mbar_init(drain_bar, 1);
         *abort_flag = 0;
@@ -206,11 +230,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         if (!SWAP && !OUT_S32 && use_tma_store) ptx::tma_prefetch_desc(&tmY);
     }
     if (warp == kWarpMma) {
-        ptx::tmem_alloc(sbase + C::OFF_MISC, C::TMEM_COLS);
-        ptx::tmem_relinquish();
+        ptx::tmem_alloc<C::CG>(sbase + C::OFF_MISC, C::TMEM_COLS);
+        ptx::tmem_relinquish<C::CG>();
     }
     ptx::tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) ptx::cluster_sync();   // the peer's barriers are initialised
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     // Everything above overlaps the tail of the kernel that produced the
@@ -218,9 +243,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     // that kernel's results are visible.
     ptx::grid_dependency_wait();
 
-    const int tiles_a = (rowsA + BM - 1) / BM;
+    const int tiles_a = (rowsA + C::TM - 1) / C::TM;
     const int tiles_b = (rowsB + BN - 1) / BN;
     const int num_tiles = tiles_a * tiles_b;
+    // Persistent schedule: tile t goes to CTA (pair) t mod the grid.
+    const int first_tile = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int tile_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
     const int num_kp = (K / 2 + C::PKB - 1) / C::PKB;   // packed stages per tile
     const int num_kb = num_kp * C::PSUB;                // widened K-blocks per tile
 
@@ -232,16 +260,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         int ps = 0;
         uint32_t ph = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        for (int tile = first_tile; tile < num_tiles && ok; tile += tile_step) {
             const int ta = tile % tiles_a, tb = tile / tiles_a;
             for (int kp = 0; kp < num_kp; ++kp) {
                 if (!ptx::mbar_wait(empty_p(ps), ph ^ 1, abort_flag)) { ok = false; break; }
                 if (leader) {
                     ptx::mbar_arrive_expect_tx(full_p(ps), C::PA + C::PB);
                     ptx::tma_load_2d(sbase + C::OFF_PA + ps * C::PA, &tmA, full_p(ps), kp * C::PKB,
-                                     ta * BM);
+                                     ta * C::TM + static_cast<int>(rank) * BM);
                     ptx::tma_load_2d(sbase + C::OFF_PB + ps * C::PB, &tmB, full_p(ps), kp * C::PKB,
-                                     tb * BN);
+                                     tb * BN + static_cast<int>(rank) * C::BR);
                 }
                 __syncwarp();
                 if (++ps == C::SP) { ps = 0; ph ^= 1; }
@@ -255,42 +283,58 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             }
         }
     } else if (warp == kWarpMma) {
+        // In a pair only CTA 0 issues; its commits arrive on the barriers of
+        // both CTAs.
+        const bool issuer = !PAIR || rank == 0;
         const bool leader = ptx::elect_one();
-        constexpr uint32_t idesc = ptx::idesc_i8(BM, BN);
+        constexpr uint32_t idesc = ptx::idesc_i8(C::TM, BN);
+        auto commit_both = [&](uint32_t bar) {
+            ptx::tc_commit<C::CG>(bar);
+            if constexpr (PAIR) ptx::tc_commit<C::CG>(ptx::mapa_shared(bar, 1));
+        };
         int us = 0;
         uint32_t ph = 0;
         int local = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+        for (int tile = first_tile; issuer && tile < num_tiles && ok; tile += tile_step, ++local) {
             const int b = local & 1;
             const uint32_t aph = (local >> 1) & 1;
-            if (!ptx::mbar_wait(acc_empty(b), aph ^ 1, abort_flag)) { ok = false; break; }
+            if (!ptx::mbar_wait<PAIR>(acc_empty(b), aph ^ 1, abort_flag)) { ok = false; break; }
             ptx::tc_fence_after();
             const uint32_t d = tmem_base + static_cast<uint32_t>(b * C::ACC_STRIDE);
             for (int kb = 0; kb < num_kb; ++kb) {
-                if (!ptx::mbar_wait(full_u(us), ph, abort_flag)) { ok = false; break; }
+                if (!ptx::mbar_wait<PAIR>(full_u(us), ph, abort_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
                 const uint32_t a0 = sbase + C::OFF_UA + us * C::UA;
                 const uint32_t b0 = sbase + C::OFF_UB + us * C::UB;
                 if (leader) {
 #pragma unroll
-                    for (int j = 0; j < BK / 32; ++j)
-                        ptx::mma_i8_ss(d, ptx::sw128_kmajor_desc(a0 + 32 * j),
-                                       ptx::sw128_kmajor_desc(b0 + 32 * j), idesc,
-                                       (kb | j) != 0 ? 1u : 0u);
-                    ptx::tc_commit(empty_u(us));
+                    for (int j = 0; j < BK / 32; ++j) {
+                        if constexpr (C::ATM)
+                            // A stage: 8 columns (32 int8 of each row) per MMA
+                            ptx::mma_i8_ts<C::CG>(
+                                d, tmem_base + static_cast<uint32_t>(C::A_OFF + us * (BK / 4) + 8 * j),
+                                ptx::sw128_kmajor_desc(b0 + 32 * j), idesc, (kb | j) != 0 ? 1u : 0u);
+                        else
+                            ptx::mma_i8_ss(d, ptx::sw128_kmajor_desc(a0 + 32 * j),
+                                           ptx::sw128_kmajor_desc(b0 + 32 * j), idesc,
+                                           (kb | j) != 0 ? 1u : 0u);
+                    }
+                    commit_both(empty_u(us));
                 }
                 __syncwarp();
                 if (++us == C::SU) { us = 0; ph ^= 1; }
             }
-            if (ok && leader) ptx::tc_commit(acc_full(b));
+            if (ok && leader) commit_both(acc_full(b));
             __syncwarp();
         }
         // Wait for every MMA this warp issued before TMEM is released.
-        if (leader) ptx::tc_commit(drain_bar);
-        __syncwarp();
-        volatile int never = 0;
-        ptx::mbar_wait(drain_bar, 0, &never, 100000000ull);
+        if (issuer) {
+            if (leader) ptx::tc_commit<C::CG>(drain_bar);
+            __syncwarp();
+            volatile int never = 0;
+            ptx::mbar_wait(drain_bar, 0, &never, 100000000ull);
+        }
     } else if (warp < kWarpUnp0) {
         // ------------------------------------------------------------ epilogue
         const int e = warp - kWarpEpi0;               // 0 .. 7
@@ -301,14 +345,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         const int col_begin = BN >= 64 ? half * kCols : 0;
         const bool active = BN >= 64 || half == 0;
         const bool tma_out = !SWAP && !OUT_S32 && use_tma_store;
-        const uint32_t box0 = sbase + C::OFF_ST + e * (2 * kStoreBox * kStoreBox * 2);
+        const uint32_t box0 = sbase + C::OFF_ST + e * (C::SB * kStoreBox * kStoreBox * 2);
         int nstores = 0;
         int local = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+        for (int tile = first_tile; tile < num_tiles; tile += tile_step, ++local) {
             const int ta = tile % tiles_a, tb = tile / tiles_a;
             const int b = local & 1;
             const uint32_t aph = (local >> 1) & 1;
-            const int arow = ta * BM + r;             // A row of this lane
+            const int row0 = ta * C::TM + static_cast<int>(rank) * BM;   // this CTA's first A row
+            const int arow = row0 + r;                // A row of this lane
             // The tile's column scales and bias go to shared memory (and the
             // row scale to a register) while the main loop still runs, so the
             // epilogue never waits on these loads.
@@ -327,7 +372,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 sxm = arow < M ? sx[arow] : 0.0f;
                 __syncwarp();
             }
-            if (!ptx::mbar_wait(acc_full(b), aph, abort_flag)) break;
+            if (!ptx::mbar_wait<PAIR>(acc_full(b), aph, abort_flag)) break;
             ptx::tc_fence_after();
             if (active) {
 #pragma unroll 1
@@ -359,8 +404,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                                                          __uint_as_float(bw[j] << 16),
                                                          __uint_as_float(bw[j] & 0xFFFF0000u));
                         }
-                        const uint32_t box = box0 + (nstores & 1) * (kStoreBox * kStoreBox * 2);
-                        if (lane == 0) ptx::bulk_wait_read<1>();   // this box's previous store
+                        const uint32_t box = box0 + (nstores % C::SB) * (kStoreBox * kStoreBox * 2);
+                        if (lane == 0) ptx::bulk_wait_read<C::SB - 1>();   // this box's previous store
                         __syncwarp();
 #pragma unroll
                         for (int c = 0; c < 4; ++c) {
@@ -371,7 +416,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                         ptx::fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) {
-                            ptx::tma_store_2d(&tmY, box, n0, ta * BM + quarter * 32);
+                            ptx::tma_store_2d(&tmY, box, n0, row0 + quarter * 32);
                             ptx::bulk_commit();
                         }
                         ++nstores;
@@ -421,9 +466,95 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             }
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(acc_empty(b));
+            if (lane == 0) arrive_leader(acc_empty(b));
         }
         if (tma_out && lane == 0) ptx::bulk_wait_all();
+    } else if constexpr (C::ATM) {
+        // ------------------------------------------------- widening, A in TMEM
+        // Warps 0..3 of the group widen A: thread = one A row (TMEM lane), its
+        // 64 packed bytes arrive 64-byte swizzled (16-byte chunk c of row r at
+        // c ^ ((r >> 1) & 3)), so eight consecutive rows hit all banks once;
+        // the 128 int8 go to the row's 32 columns of the A stage with one
+        // tcgen05.st.  Warps 4..7 widen B into the swizzled shared-memory
+        // stage.  Column 8c + x (x < 4) of an A stage holds the even codes of
+        // packed word x of chunk c and column 8c + 4 + x its odd codes: the
+        // same K order as the B rows' [even, odd] 16-byte halves.
+        const int uw = warp - kWarpUnp0;
+        const int my_tiles = num_tiles > first_tile ? (num_tiles - 1 - first_tile) / tile_step + 1 : 0;
+        const int total = my_tiles * num_kb;
+        const uint32_t hm = 0xF0F0F0F0u;
+        if (uw < 4) {
+            const int quarter = warp & 3;             // TMEM lanes 32*quarter ..
+            const int r = quarter * 32 + lane;
+            const uint32_t rsw = static_cast<uint32_t>((r >> 1) & 3);
+            const uint32_t trow = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                  static_cast<uint32_t>(C::A_OFF);
+            for (int n = 0; n < total; ++n) {
+                const int ps = n % C::SP, us = n % C::SU;
+                const uint32_t pph = (n / C::SP) & 1, uph = (n / C::SU) & 1;
+                if (!ptx::mbar_wait(full_p(ps), pph, abort_flag)) break;
+                if (!ptx::mbar_wait<PAIR>(empty_u(us), uph ^ 1, abort_flag)) break;
+                ptx::tc_fence_after();
+                const uint32_t src = sbase + C::OFF_PA + ps * C::PA + r * BKP;
+                uint32_t t[32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 w = lds128(src + ((static_cast<uint32_t>(c) ^ rsw) << 4));
+                    t[8 * c + 0] = (w.x << 4) & hm;
+                    t[8 * c + 1] = (w.y << 4) & hm;
+                    t[8 * c + 2] = (w.z << 4) & hm;
+                    t[8 * c + 3] = (w.w << 4) & hm;
+                    t[8 * c + 4] = w.x & hm;
+                    t[8 * c + 5] = w.y & hm;
+                    t[8 * c + 6] = w.z & hm;
+                    t[8 * c + 7] = w.w & hm;
+                }
+                __syncwarp();   // tcgen05.st is warp-collective
+                ptx::tmem_st_32x32b_x32(trow + static_cast<uint32_t>(us * (BK / 4)), t);
+                ptx::tmem_st_wait();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    ptx::mbar_arrive(empty_p(ps));
+                    arrive_leader(full_u(us));
+                }
+            }
+        } else {
+            // 128 threads over BN rows x 4 chunks: thread bt takes chunk bt & 3
+            // of rows bt / 4 + 32 i; 32 is a multiple of the 8-row swizzle
+            // period, so the swizzle phase of a thread never changes.
+            const int bt = threadIdx.x - (kWarpUnp0 + 4) * 32;
+            constexpr int kPerB = C::BR / 32;
+            const uint32_t c = static_cast<uint32_t>(bt & 3);
+            const int row0 = bt >> 2;
+            const uint32_t sw8 = static_cast<uint32_t>(row0 & 7);
+            const uint32_t lo_off = ((2u * c) ^ sw8) << 4;
+            const uint32_t hi_off = ((2u * c + 1u) ^ sw8) << 4;
+            for (int n = 0; n < total; ++n) {
+                const int ps = n % C::SP, us = n % C::SU;
+                const uint32_t pph = (n / C::SP) & 1, uph = (n / C::SU) & 1;
+                if (!ptx::mbar_wait(full_p(ps), pph, abort_flag)) break;
+                if (!ptx::mbar_wait<PAIR>(empty_u(us), uph ^ 1, abort_flag)) break;
+                const uint32_t pb = sbase + C::OFF_PB + ps * C::PB + row0 * BKP + c * 16;
+                const uint32_t ub = sbase + C::OFF_UB + us * C::UB + row0 * 128;
+                uint4 w[kPerB];
+#pragma unroll
+                for (int i = 0; i < kPerB; ++i) w[i] = lds128(pb + i * 32 * BKP);
+#pragma unroll
+                for (int i = 0; i < kPerB; ++i) {
+                    const uint32_t dst = ub + i * 32 * 128;
+                    sts128(dst + lo_off, (w[i].x << 4) & hm, (w[i].y << 4) & hm,
+                           (w[i].z << 4) & hm, (w[i].w << 4) & hm);
+                    sts128(dst + hi_off, w[i].x & hm, w[i].y & hm, w[i].z & hm, w[i].w & hm);
+                }
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    ptx::mbar_arrive(empty_p(ps));
+                    arrive_leader(full_u(us));
+                }
+            }
+        }
     } else {
         // ------------------------------------------------------------ widening
         // Group g of UG takes stages g, g + UG, g + 2 UG, ... (counted over all
@@ -441,9 +572,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         const uint32_t sw8 = static_cast<uint32_t>((ut >> 2) & 7);
         const uint32_t lo_off = ((2u * c) ^ sw8) << 4;
         const uint32_t hi_off = ((2u * c + 1u) ^ sw8) << 4;
-        const int my_tiles = num_tiles > static_cast<int>(blockIdx.x)
-                                 ? (num_tiles - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1
-                                 : 0;
+        const int my_tiles = num_tiles > first_tile ? (num_tiles - 1 - first_tile) / tile_step + 1 : 0;
         const int total = my_tiles * num_kb;            // stages this CTA runs
         for (int n = ug; n < total; n += C::UG) {
             const int np = n / C::PSUB, sub = n % C::PSUB;   // packed stage, K-block in it
@@ -486,10 +615,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 
     ptx::tc_fence_before();
     __syncthreads();
+    // A pair's CTAs leave together: CTA 0's MMAs read CTA 1's shared memory
+    // and TMEM, and CTA 1 arrives on CTA 0's barriers.
+    if constexpr (PAIR) ptx::cluster_sync();
     ptx::tc_fence_after();
     if (warp == kWarpMma) {
         __syncwarp();
-        ptx::tmem_dealloc(tmem_base, C::TMEM_COLS);
+        ptx::tmem_dealloc<C::CG>(tmem_base, C::TMEM_COLS);
     }
 }
 

@@ -106,6 +106,48 @@ def test_gemm_s32_bit_exact(M, N, K):
     assert np.array_equal(acc.cpu().numpy().astype(np.int64), O.gemm(pa, pb, K))
 
 
+# Every token-major tile shape on its own, whatever the automatic choice:
+# ragged M, N and K tails, several tiles per CTA (the persistent loop and the
+# double-buffered accumulator), and an odd tile count for the CTA pairs.
+TILE_SHAPES = [cr.TILES_128x256, cr.TILES_128x192, cr.TILES_256x192_PAIR]
+TILE_IDS = ["128x256", "128x192tmem", "256x192pair"]
+TILE_CASES = [(1, 16, 64), (100, 200, 192), (257, 385, 1088), (384, 576, 2048),
+              (1000, 2000, 512), (2304, 3072, 256), (2304, 3072, 3072)]
+
+
+@pytest.mark.parametrize("tiles", TILE_SHAPES, ids=TILE_IDS)
+@pytest.mark.parametrize("M,N,K", TILE_CASES)
+def test_gemm_tiles_s32_bit_exact(tiles, M, N, K):
+    rng = np.random.default_rng(M * 13 + N + tiles)
+    a = rng.integers(-7, 8, size=(M, K)).astype(np.int8)
+    b = rng.integers(-7, 8, size=(N, K)).astype(np.int8)
+    if M > 3:
+        a[2] = 7
+        b[min(3, N - 1)] = -7
+    pa, pb = O.pack(a), O.pack(b)
+    acc = cr.convrot_debug_gemm_tiles(_dev(torch.from_numpy(pa)), None, _dev(torch.from_numpy(pb)),
+                                      None, None, K, tiles, out_s32=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), O.gemm(pa, pb, K))
+
+
+@pytest.mark.parametrize("tiles", TILE_SHAPES, ids=TILE_IDS)
+@pytest.mark.parametrize("M,N,K,bias", [(130, 520, 768, True), (600, 1000, 1024, False),
+                                        (1100, 392, 3072, True)])
+def test_gemm_tiles_epilogue_one_ulp(tiles, M, N, K, bias):
+    lt = _layer(M, K, N, 64, seed=M + N + tiles, bias=bias)
+    xb, wb = wl.bf16_bits(lt.x), wl.bf16_bits(lt.w)
+    bb = None if lt.b is None else wl.bf16_bits(lt.b)
+    px, sx = O.prepare_rows(xb, 64)
+    pw, sw = O.prepare_rows(wb, 64)
+    y_ref = O.epilogue(O.gemm(px, pw, K), sx, sw, bb)
+    t = lambda a: _dev(torch.from_numpy(a))
+    y = cr.convrot_debug_gemm_tiles(t(px), t(sx), t(pw), t(sw),
+                                    None if lt.b is None else _dev(lt.b), K, tiles)
+    torch.cuda.synchronize()
+    gc.check_outputs(gc.to_np_u16(y), y_ref)
+
+
 @pytest.mark.parametrize("M,N,K,bias", [(3, 48, 256, True), (40, 200, 1024, False),
                                         (130, 520, 768, True), (300, 13, 256, True)])
 def test_linear_prepared_one_ulp(M, N, K, bias):
