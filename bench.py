@@ -255,27 +255,43 @@ def run_gpu(args):
     if cr.convrot_check_device_error() != 0:
         raise RuntimeError("device error during warm-up")
 
-    # One CUDA graph per copy and per program (whole step, prep only, GEMM
-    # only): the timed loops replay them back to back, so host launch cost is
-    # not in the device timing.
+    # CUDA graphs per program (whole step, prep only, GEMM only): one graph
+    # per copy, and one graph that runs every copy once in turn (R steps), so
+    # a replay launches R steps and host launch cost stays out of the device
+    # timing even for layers that take a few microseconds.
     def capture(fn, *a):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             fn(*a)
         return g
 
-    g_step = [capture(step, c) for c in copies]
-    g_prep = [[capture(prep_only, c, i) for c in copies] for i in range(nl)]
-    g_gemm = [[capture(gemm_only, c, i) for c in copies] for i in range(nl)]
-    for g in g_step + sum(g_prep, []) + sum(g_gemm, []):
-        g.replay()
+    def capture_all(fn, *a):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for c in copies:
+                fn(c, *a)
+        return g
+
+    progs = {"step": (step, ())}
+    for i in range(nl):
+        progs[("prep", i)] = (prep_only, (i,))
+        progs[("gemm", i)] = (gemm_only, (i,))
+    graphs = {k: ([capture(fn, c, *a) for c in copies], capture_all(fn, *a))
+              for k, (fn, a) in progs.items()}
+    for one, every in graphs.values():
+        for g in one + [every]:
+            g.replay()
     torch.cuda.synchronize()
 
-    def timed(graphs, steps):
+    def timed(key, steps):
+        """Device time of exactly `steps` back-to-back steps of one program."""
+        one, every = graphs[key]
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        for k in range(steps):
-            graphs[k % R].replay()
+        for _ in range(steps // R):
+            every.replay()
+        for k in range(steps % R):
+            one[k].replay()
         b.record()
         b.synchronize()
         return a.elapsed_time(b)
@@ -289,7 +305,7 @@ def run_gpu(args):
     except Exception:
         gpu_id = str(local)
     with ClockSampler(gpu_id) as clocks:
-        local_ms = timed(g_step, args.steps)
+        local_ms = timed("step", args.steps)
         torch.cuda.synchronize()
         clocks.mark_end()
     if world > 1:
@@ -300,8 +316,8 @@ def run_gpu(args):
         raise RuntimeError(f"device error status {status} in the timed region")
 
     # per-kernel durations: K back-to-back launches of one kernel of one layer
-    prep_ms = [[timed(g_prep[i], args.steps) / args.steps] * args.steps for i in range(nl)]
-    gemm_ms = [[timed(g_gemm[i], args.steps) / args.steps] * args.steps for i in range(nl)]
+    prep_ms = [[timed(("prep", i), args.steps) / args.steps] * args.steps for i in range(nl)]
+    gemm_ms = [[timed(("gemm", i), args.steps) / args.steps] * args.steps for i in range(nl)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)   # e2e pass only
     ops_step = spec.ops
     t_max, ops_total = aggregate(local_ms, ops_step * args.steps, dev)
@@ -345,7 +361,7 @@ def run_gpu(args):
                    "tokens_per_rank": spec.tokens,
                    "l2": f"cold: steps cycle through {R} copies of all step data "
                          f"({R * step_bytes / 2**20:.0f} MiB >= 2 x L2)",
-                   "launch": "CUDA graph per step, replayed back to back",
+                   "launch": f"CUDA graphs of {R} steps (each copy once), replayed back to back",
                    "parallelism": f"dp{world}"},
         "tokens_per_s": round(tokens_s, 1),
         "int8_peak_frac_path": round(value / world / int8_peak, 4),

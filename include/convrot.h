@@ -131,9 +131,13 @@ convrot_status convrot_debug_gemm_s32(const uint8_t *qx, const uint8_t *qw, int6
  *   tiles = 0  automatic (as the entry points above);
  *           1  128 x 256 tiles, both operands widened in shared memory;
  *           2  128 x 192 tiles, A widened into TMEM;
- *           3  256 x 192 tiles on CTA pairs (cta_group::2).
- * Returns CONVROT_ERR_SHAPE for any other value and CONVROT_ERR_UNSUPPORTED
- * when the device cannot co-schedule CTA pairs (tiles = 3).
+ *           3  256 x 192 tiles on CTA pairs (cta_group::2);
+ *           4  few-token form (M <= 128): weights widened into TMEM, one
+ *              CTA per slice of weight rows (the automatic choice there);
+ *           5  few-token form with both operands widened in shared memory.
+ * Returns CONVROT_ERR_SHAPE for any other value or for 4 / 5 with M > 128,
+ * and CONVROT_ERR_UNSUPPORTED when the device cannot co-schedule CTA pairs
+ * (tiles = 3).
  */
 convrot_status convrot_debug_gemm_tiles(const uint8_t *qx, const float *sx, const uint8_t *qw,
                                         const float *sw, const void *bias_bf16, int64_t M,

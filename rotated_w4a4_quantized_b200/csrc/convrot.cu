@@ -14,6 +14,7 @@
 #include "gemm.cuh"
 #include "prep.cuh"
 #include "ptx.cuh"
+#include "skinny.cuh"
 
 namespace {
 
@@ -97,6 +98,14 @@ convrot_status device_setup(int *dev_out) {
     ok &= set_smem(gemm::gemm_kernel<128, true, true>, gemm::Cfg<128, true>::SMEM_BYTES);
     ok &= set_smem(gemm::gemm_kernel<192, false, false, true>, gemm::Cfg<192, false, true>::SMEM_BYTES);
     ok &= set_smem(gemm::gemm_kernel<192, false, true, true>, gemm::Cfg<192, false, true>::SMEM_BYTES);
+    ok &= set_smem(skinny::skinny_kernel<16, false>, skinny::Cfg<16>::SMEM_BYTES);
+    ok &= set_smem(skinny::skinny_kernel<32, false>, skinny::Cfg<32>::SMEM_BYTES);
+    ok &= set_smem(skinny::skinny_kernel<64, false>, skinny::Cfg<64>::SMEM_BYTES);
+    ok &= set_smem(skinny::skinny_kernel<128, false>, skinny::Cfg<128>::SMEM_BYTES);
+    ok &= set_smem(skinny::skinny_kernel<16, true>, skinny::Cfg<16>::SMEM_BYTES);
+    ok &= set_smem(skinny::skinny_kernel<32, true>, skinny::Cfg<32>::SMEM_BYTES);
+    ok &= set_smem(skinny::skinny_kernel<64, true>, skinny::Cfg<64>::SMEM_BYTES);
+    ok &= set_smem(skinny::skinny_kernel<128, true>, skinny::Cfg<128>::SMEM_BYTES);
     if (ok) {
         // How many CTA pairs fit on the device at once (pairs need two SMs
         // of one GPC); the pair GEMM's persistent grid is that many clusters.
@@ -253,19 +262,77 @@ convrot_status launch_gemm_cfg(int slots, const uint8_t *qA, const uint8_t *qB, 
     return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 
-// Tile shapes of the token-major path (more than 128 tokens).
-enum TileChoice { kTilesAuto = 0, kTiles128x256 = 1, kTiles128x192 = 2, kTiles256x192Pair = 3 };
+// Skinny GEMM (M <= 128): one CTA per slice of R weight rows, weights
+// widened into TMEM.  weights_ready: the weights were complete before the
+// preceding kernel on the stream (the prep kernel of the same call) started,
+// so the kernel may start streaming them before that kernel finishes.
+template <int BN, bool OUT_S32>
+convrot_status launch_skinny_cfg(int num_sms, const uint8_t *qx, const float *sx,
+                                 const uint8_t *qw, const float *sw, const void *bias, int64_t M,
+                                 int64_t N, int64_t K, void *out, bool weights_ready,
+                                 cudaStream_t stream) {
+    const int R = skinny::rows_per_cta(N, num_sms);
+    CUtensorMap tmA, tmB;
+    if (!make_map(&tmA, qw, N, K, skinny::kPKB, R, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tmB, qx, M, K, skinny::kPKB, BN))
+        return CONVROT_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((N + R - 1) / R));
+    cfg.blockDim = dim3(skinny::kThreads);
+    cfg.dynamicSmemBytes = skinny::Cfg<BN>::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(
+        &cfg, skinny::skinny_kernel<BN, OUT_S32>, tmA, tmB, R, weights_ready ? 1 : 0,
+        static_cast<int>(K), sx, sw, static_cast<const uint16_t *>(bias), out, static_cast<int>(M),
+        static_cast<int>(N));
+    return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
+}
 
-// Path choice: up to 128 tokens the weights take the 128-row MMA side
-// (skinny form, N-side tile = tokens rounded up to 16); otherwise tokens on
-// the M side, with the tile shape that finishes first.
+template <bool OUT_S32>
+convrot_status launch_skinny(int num_sms, const uint8_t *qx, const float *sx, const uint8_t *qw,
+                             const float *sw, const void *bias, int64_t M, int64_t N, int64_t K,
+                             void *out, bool weights_ready, cudaStream_t stream) {
+    if (M <= 16)
+        return launch_skinny_cfg<16, OUT_S32>(num_sms, qx, sx, qw, sw, bias, M, N, K, out,
+                                              weights_ready, stream);
+    if (M <= 32)
+        return launch_skinny_cfg<32, OUT_S32>(num_sms, qx, sx, qw, sw, bias, M, N, K, out,
+                                              weights_ready, stream);
+    if (M <= 64)
+        return launch_skinny_cfg<64, OUT_S32>(num_sms, qx, sx, qw, sw, bias, M, N, K, out,
+                                              weights_ready, stream);
+    return launch_skinny_cfg<128, OUT_S32>(num_sms, qx, sx, qw, sw, bias, M, N, K, out,
+                                           weights_ready, stream);
+}
+
+// GEMM forms: the automatic choice, the three token-major tile shapes, and
+// the two few-token forms (M <= 128).
+enum TileChoice {
+    kTilesAuto = 0, kTiles128x256 = 1, kTiles128x192 = 2, kTiles256x192Pair = 3,
+    kSkinnyTmem = 4, kSkinnySmem = 5
+};
+
+// Path choice: up to 128 tokens the few-token form (weights on the 128-row
+// MMA side, widened into TMEM, one CTA per slice of weight rows); otherwise
+// tokens on the M side, with the tile shape that finishes first.
 template <bool OUT_S32>
 convrot_status launch_gemm(const DeviceState &ds, const uint8_t *qx, const float *sx,
                            const uint8_t *qw, const float *sw, const void *bias, int64_t M,
                            int64_t N, int64_t K, void *out, cudaStream_t stream,
-                           int tiles = kTilesAuto) {
+                           int tiles = kTilesAuto, bool weights_ready = false) {
     const int num_sms = ds.num_sms;
-    if (tiles == kTilesAuto && M <= 128) {
+    if (tiles == kTilesAuto && M <= 128) tiles = kSkinnyTmem;
+    if (tiles == kSkinnyTmem && M > 128) return CONVROT_ERR_SHAPE;
+    if (tiles == kSkinnySmem && M > 128) return CONVROT_ERR_SHAPE;
+    if (tiles == kSkinnyTmem)
+        return launch_skinny<OUT_S32>(num_sms, qx, sx, qw, sw, bias, M, N, K, out, weights_ready,
+                                      stream);
+    if (tiles == kSkinnySmem) {
         if (M <= 16)
             return launch_gemm_cfg<16, true, OUT_S32>(num_sms, qw, qx, N, M, K, sx, sw, bias, out, M,
                                                       N, stream);
@@ -404,7 +471,8 @@ convrot_status convrot_linear(const void *x_bf16, const uint8_t *qw, const float
     float *sx = reinterpret_cast<float *>(qx + round256(static_cast<size_t>(M) * (K / 2)));
     if ((st = launch_prep(g_dev[dev].num_sms, x_bf16, M, K, group, qx, sx, nullptr, stream)) != CONVROT_OK)
         return st;
-    return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream);
+    return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream,
+                              kTilesAuto, true);
 }
 
 convrot_status convrot_debug_rotate_f32(const void *x_bf16, int64_t M, int64_t K, int group,
@@ -438,7 +506,7 @@ convrot_status convrot_debug_gemm_tiles(const uint8_t *qx, const float *sx, cons
                                         int64_t N, int64_t K, int tiles, int out_s32, void *out,
                                         convrot_stream_t stream) {
     if (M < 0 || N < 0) return CONVROT_ERR_SHAPE;
-    if (tiles < kTilesAuto || tiles > kTiles256x192Pair) return CONVROT_ERR_SHAPE;
+    if (tiles < kTilesAuto || tiles > kSkinnySmem) return CONVROT_ERR_SHAPE;
     if (M == 0 || N == 0) return CONVROT_OK;
     convrot_status st = check_gemm_args(qx, qw, M, N, K);
     if (st != CONVROT_OK) return st;
@@ -554,5 +622,5 @@ extern "C" convrot_status convrot_linear_noalloc(const void *x_bf16, const uint8
     if ((st = launch_prep(g_dev[dev].num_sms, x_bf16, M, K, group, qx, sx, nullptr, stream)) != CONVROT_OK)
         return st;
     return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16,
-                              stream);
+                              stream, kTilesAuto, true);
 }

@@ -143,6 +143,12 @@ prep_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ 
     int row = blockIdx.x;
     if (row < M) issue_row(row, 0);
     cp_async_commit();
+    // The GEMM that follows may be scheduled on the SMs this grid leaves
+    // free from now on (all of this grid's CTAs are resident: the grid is
+    // sized to the resident capacity).  It sets up, and streams weights that
+    // do not depend on this grid, but reads these rows only after its
+    // griddepcontrol.wait, which waits for this whole grid to complete.
+    ptx::launch_dependents();
     for (; row < M; row += gridDim.x) {
         const int next = row + gridDim.x;
         cp_async_wait_all();      // this row's copies (by this thread) have landed
@@ -260,9 +266,6 @@ prep_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ 
                     make_uint2(packed[2 * d3], packed[2 * d3 + 1]);
         }
     }
-    // The GEMM that consumes these rows may be scheduled now; it still waits
-    // for this whole grid to complete before reading them.
-    ptx::launch_dependents();
 }
 
 }  // namespace prep

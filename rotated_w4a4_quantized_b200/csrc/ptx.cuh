@@ -90,6 +90,13 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                  : "memory");
 }
 
+// try_wait suspends the waiting thread in hardware until the phase completes
+// or this many nanoseconds pass, so a waiting warp issues no instructions
+// (without the hint the suspend window is short, and spinning warps slow the
+// barrier operations of the warps doing the work).  The bounded-wait loop
+// below re-checks its limit and the abort flag after every window.
+constexpr uint32_t kSuspendHintNs = 1000000;
+
 // CL = true: acquire at cluster scope, for barriers that the peer CTA of a
 // cluster arrives on.
 template <bool CL = false>
@@ -98,18 +105,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     if constexpr (!CL)
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
             "selp.u32 %0, 1, 0, p;\n\t}"
             : "=r"(ok)
-            : "r"(bar), "r"(parity)
+            : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
             : "memory");
     else
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
             "selp.u32 %0, 1, 0, p;\n\t}"
             : "=r"(ok)
-            : "r"(bar), "r"(parity)
+            : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
             : "memory");
     return ok != 0;
 }

@@ -131,6 +131,53 @@ def test_gemm_tiles_s32_bit_exact(tiles, M, N, K):
     assert np.array_equal(acc.cpu().numpy().astype(np.int64), O.gemm(pa, pb, K))
 
 
+# The two few-token forms (M <= 128): token tiles of 16 .. 128 with ragged
+# token counts, weight-row slices with a ragged last slice, K tails.
+SKINNY_FORMS = [cr.SKINNY_TMEM, cr.SKINNY_SMEM]
+SKINNY_IDS = ["tmem", "smem"]
+SKINNY_CASES = [(1, 16, 64), (1, 14336, 4096), (5, 300, 1088), (16, 1000, 512), (17, 257, 192),
+                (33, 4000, 3072), (64, 1024, 1024), (100, 777, 2048), (128, 14336, 256)]
+
+
+@pytest.mark.parametrize("form", SKINNY_FORMS, ids=SKINNY_IDS)
+@pytest.mark.parametrize("M,N,K", SKINNY_CASES)
+def test_gemm_skinny_s32_bit_exact(form, M, N, K):
+    rng = np.random.default_rng(M * 17 + N + form)
+    a = rng.integers(-7, 8, size=(M, K)).astype(np.int8)
+    b = rng.integers(-7, 8, size=(N, K)).astype(np.int8)
+    a[0] = 7
+    b[N - 1] = -7
+    pa, pb = O.pack(a), O.pack(b)
+    acc = cr.convrot_debug_gemm_tiles(_dev(torch.from_numpy(pa)), None, _dev(torch.from_numpy(pb)),
+                                      None, None, K, form, out_s32=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), O.gemm(pa, pb, K))
+
+
+@pytest.mark.parametrize("form", SKINNY_FORMS, ids=SKINNY_IDS)
+@pytest.mark.parametrize("M,N,K,bias", [(1, 4096, 1024, True), (16, 1000, 768, False),
+                                        (77, 520, 3072, True), (128, 2048, 512, True)])
+def test_gemm_skinny_epilogue_one_ulp(form, M, N, K, bias):
+    lt = _layer(M, K, N, 64, seed=M + N + form, bias=bias)
+    xb, wb = wl.bf16_bits(lt.x), wl.bf16_bits(lt.w)
+    bb = None if lt.b is None else wl.bf16_bits(lt.b)
+    px, sx = O.prepare_rows(xb, 64)
+    pw, sw = O.prepare_rows(wb, 64)
+    y_ref = O.epilogue(O.gemm(px, pw, K), sx, sw, bb)
+    t = lambda a: _dev(torch.from_numpy(a))
+    y = cr.convrot_debug_gemm_tiles(t(px), t(sx), t(pw), t(sw),
+                                    None if lt.b is None else _dev(lt.b), K, form)
+    torch.cuda.synchronize()
+    gc.check_outputs(gc.to_np_u16(y), y_ref)
+
+
+def test_gemm_skinny_forms_reject_many_tokens():
+    q = torch.zeros(129, 64, dtype=torch.uint8, device="cuda")
+    for form in SKINNY_FORMS:
+        with pytest.raises(cr.ConvRotError):
+            cr.convrot_debug_gemm_tiles(q, None, q, None, None, 128, form, out_s32=True)
+
+
 @pytest.mark.parametrize("tiles", TILE_SHAPES, ids=TILE_IDS)
 @pytest.mark.parametrize("M,N,K,bias", [(130, 520, 768, True), (600, 1000, 1024, False),
                                         (1100, 392, 3072, True)])
