@@ -224,8 +224,8 @@ convrot_status launch_gemm_cfg(int slots, const uint8_t *qA, const uint8_t *qB, 
     using C = gemm::Cfg<BN, SWAP, PAIR>;
     CUtensorMap tmA, tmB, tmY;
     constexpr int pkb = C::PKB;
-    // A widened into TMEM reads its packed rows 64-byte swizzled.
-    const CUtensorMapSwizzle swa = C::ATM ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE;
+    // A widened into TMEM reads its packed rows 128-byte swizzled.
+    const CUtensorMapSwizzle swa = C::ATM ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
     if (!make_map(&tmA, qA, rowsA, K, pkb, gemm::BM, swa) || !make_map(&tmB, qB, rowsB, K, pkb, C::BR))
         return CONVROT_ERR_CUDA;
     int use_tma_store = 0;

@@ -75,10 +75,15 @@ struct Cfg {
     // of the weight stream in flight.
     // ATM: the 128 x 192 tile widens operand A straight into TMEM (the MMA
     // reads A from there), so only B passes through widened shared memory;
-    // TMEM holds two 192-column accumulators plus SU 32-column A stages.
+    // TMEM holds two 192-column accumulators plus SU 64-column A stages.
+    // Its stages are two K-blocks deep (KS = 2, 128 packed bytes per row):
+    // every TMA issue, barrier operation and TMEM store wait is paid once per
+    // 256 codes, which the single-thread issue loops need to keep up with
+    // the tensor cores.
     static constexpr bool ATM = PAIR || (!SWAP && BN == 192);
-    static constexpr int SP = PAIR ? 8 : ATM ? 4 : BN == 256 ? 3 : BN == 192 ? 5 : BN == 128 ? 3 : BN == 64 ? 4 : BN == 32 ? 5 : 3;
-    static constexpr int SU = ATM ? 4 : BN >= 192 ? 2 : BN == 128 ? 4 : BN == 64 ? 5 : 6;
+    static constexpr int KS = ATM ? 2 : 1;           // K-blocks per widened stage
+    static constexpr int SP = PAIR ? 4 : ATM ? 2 : BN == 256 ? 3 : BN == 192 ? 5 : BN == 128 ? 3 : BN == 64 ? 4 : BN == 32 ? 5 : 3;
+    static constexpr int SU = ATM ? 2 : BN >= 192 ? 2 : BN == 128 ? 4 : BN == 64 ? 5 : 6;
     // The widening warps split into UG groups that take alternate stages, so
     // the hand-off latency of one stage overlaps the widening of the next.
     static constexpr int UG = BN >= 192 ? 1 : 2;
@@ -86,12 +91,13 @@ struct Cfg {
     // Packed stages of the narrow tiles carry PKB bytes of each row (PSUB
     // K-blocks), so the weight stream is read in longer contiguous pieces;
     // the widening turns each packed stage into PSUB widened K-blocks.
-    static constexpr int PKB = (!SWAP && BN >= 192) ? 64 : BN == 16 ? 256 : 128;
-    static constexpr int PSUB = PKB / BKP;
+    static constexpr int PKB = ATM ? 128 : (!SWAP && BN >= 192) ? 64 : BN == 16 ? 256 : 128;
+    static constexpr int PSUB = ATM ? 1 : PKB / BKP;
     static constexpr int PA = BM * PKB;
     static constexpr int PB = BR * PKB;
     static constexpr int UA = ATM ? 0 : BM * BK;
-    static constexpr int UB = BR * BK;
+    static constexpr int UBH = BR * BK;               // widened B tile of one K-block
+    static constexpr int UB = KS * UBH;
     static constexpr int SB = 2;   // store boxes per epilogue warp
     static constexpr int ST = SWAP ? 0 : kEpiWarps * SB * kStoreBox * kStoreBox * 2;
     static constexpr int OFF_UA = 0;                   // 1024-aligned tiles first
@@ -113,11 +119,12 @@ struct Cfg {
     // least 32 columns apart and the allocation covers two of them.
     static constexpr int ACC_STRIDE = BN < 32 ? 32 : BN;
     static constexpr int A_OFF = 2 * ACC_STRIDE;              // first A-stage column (ATM)
-    static constexpr int TMEM_NEED = A_OFF + (ATM ? SU * (BK / 4) : 0);
+    static constexpr int A_COLS = KS * BK / 4;                 // TMEM columns of an A stage
+    static constexpr int TMEM_NEED = A_OFF + (ATM ? SU * A_COLS : 0);
     static constexpr int TMEM_COLS = TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
                                      : TMEM_NEED <= 256 ? 256 : 512;   // power of two
     static_assert(TMEM_NEED <= 512, "TMEM holds 512 columns");
-    static_assert(!ATM || (PSUB == 1 && PKB == 64), "A-in-TMEM reads 64-byte swizzled packed rows");
+    static_assert(!ATM || (PSUB == 1 && PKB == 128), "A-in-TMEM reads 128-byte swizzled packed rows");
     static constexpr int JW = BN < 32 ? BN : 32;             // valid columns per 32-wide read
     static_assert(UB % 1024 == 0, "widened B tiles must stay 1024-aligned");
     static_assert(ST % 1024 == 0, "store boxes must stay 1024-aligned");
@@ -252,30 +259,25 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     const int num_kp = (K / 2 + C::PKB - 1) / C::PKB;   // packed stages per tile
     const int num_kb = num_kp * C::PSUB;                // widened K-blocks per tile
 
-    // The producer and MMA warps run their loops with all 32 lanes (so the
-    // addresses and descriptors stay warp-uniform) and let one elected lane
-    // issue each TMA copy, MMA and commit.
+    // The producer and MMA loops run in one thread each (lane 0): a warp-wide
+    // mbarrier operation costs a multiple of one thread's.
     if (warp == kWarpTma) {
-        const bool leader = ptx::elect_one();
         int ps = 0;
         uint32_t ph = 0;
         bool ok = true;
-        for (int tile = first_tile; tile < num_tiles && ok; tile += tile_step) {
+        for (int tile = first_tile; lane == 0 && tile < num_tiles && ok; tile += tile_step) {
             const int ta = tile % tiles_a, tb = tile / tiles_a;
             for (int kp = 0; kp < num_kp; ++kp) {
                 if (!ptx::mbar_wait(empty_p(ps), ph ^ 1, abort_flag)) { ok = false; break; }
-                if (leader) {
-                    ptx::mbar_arrive_expect_tx(full_p(ps), C::PA + C::PB);
-                    ptx::tma_load_2d(sbase + C::OFF_PA + ps * C::PA, &tmA, full_p(ps), kp * C::PKB,
-                                     ta * C::TM + static_cast<int>(rank) * BM);
-                    ptx::tma_load_2d(sbase + C::OFF_PB + ps * C::PB, &tmB, full_p(ps), kp * C::PKB,
-                                     tb * BN + static_cast<int>(rank) * C::BR);
-                }
-                __syncwarp();
+                ptx::mbar_arrive_expect_tx(full_p(ps), C::PA + C::PB);
+                ptx::tma_load_2d(sbase + C::OFF_PA + ps * C::PA, &tmA, full_p(ps), kp * C::PKB,
+                                 ta * C::TM + static_cast<int>(rank) * BM);
+                ptx::tma_load_2d(sbase + C::OFF_PB + ps * C::PB, &tmB, full_p(ps), kp * C::PKB,
+                                 tb * BN + static_cast<int>(rank) * C::BR);
                 if (++ps == C::SP) { ps = 0; ph ^= 1; }
             }
         }
-        if (!ok && leader) {
+        if (!ok) {
             // Let copies already in flight land before the CTA exits.
             for (int s = 0; s < C::SP; ++s) {
                 volatile int never = 0;
@@ -285,8 +287,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     } else if (warp == kWarpMma) {
         // In a pair only CTA 0 issues; its commits arrive on the barriers of
         // both CTAs.
-        const bool issuer = !PAIR || rank == 0;
-        const bool leader = ptx::elect_one();
+        const bool issuer = (!PAIR || rank == 0) && lane == 0;
         constexpr uint32_t idesc = ptx::idesc_i8(C::TM, BN);
         auto commit_both = [&](uint32_t bar) {
             ptx::tc_commit<C::CG>(bar);
@@ -307,31 +308,28 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 ptx::tc_fence_after();
                 const uint32_t a0 = sbase + C::OFF_UA + us * C::UA;
                 const uint32_t b0 = sbase + C::OFF_UB + us * C::UB;
-                if (leader) {
 #pragma unroll
-                    for (int j = 0; j < BK / 32; ++j) {
-                        if constexpr (C::ATM)
-                            // A stage: 8 columns (32 int8 of each row) per MMA
-                            ptx::mma_i8_ts<C::CG>(
-                                d, tmem_base + static_cast<uint32_t>(C::A_OFF + us * (BK / 4) + 8 * j),
-                                ptx::sw128_kmajor_desc(b0 + 32 * j), idesc, (kb | j) != 0 ? 1u : 0u);
-                        else
-                            ptx::mma_i8_ss(d, ptx::sw128_kmajor_desc(a0 + 32 * j),
-                                           ptx::sw128_kmajor_desc(b0 + 32 * j), idesc,
-                                           (kb | j) != 0 ? 1u : 0u);
-                    }
-                    commit_both(empty_u(us));
+                for (int j = 0; j < C::KS * BK / 32; ++j) {
+                    if constexpr (C::ATM)
+                        // A stage: 8 columns (32 int8 of each row) per MMA; B
+                        // K-block j / 4 is its own 128-byte swizzled tile
+                        ptx::mma_i8_ts<C::CG>(
+                            d, tmem_base + static_cast<uint32_t>(C::A_OFF + us * C::A_COLS + 8 * j),
+                            ptx::sw128_kmajor_desc(b0 + (j >> 2) * C::UBH + 32 * (j & 3)), idesc,
+                            (kb | j) != 0 ? 1u : 0u);
+                    else
+                        ptx::mma_i8_ss(d, ptx::sw128_kmajor_desc(a0 + 32 * j),
+                                       ptx::sw128_kmajor_desc(b0 + 32 * j), idesc,
+                                       (kb | j) != 0 ? 1u : 0u);
                 }
-                __syncwarp();
+                commit_both(empty_u(us));
                 if (++us == C::SU) { us = 0; ph ^= 1; }
             }
-            if (ok && leader) commit_both(acc_full(b));
-            __syncwarp();
+            if (ok) commit_both(acc_full(b));
         }
-        // Wait for every MMA this warp issued before TMEM is released.
+        // Wait for every MMA this thread issued before TMEM is released.
         if (issuer) {
-            if (leader) ptx::tc_commit<C::CG>(drain_bar);
-            __syncwarp();
+            ptx::tc_commit<C::CG>(drain_bar);
             volatile int never = 0;
             ptx::mbar_wait(drain_bar, 0, &never, 100000000ull);
         }
@@ -471,14 +469,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         if (tma_out && lane == 0) ptx::bulk_wait_all();
     } else if constexpr (C::ATM) {
         // ------------------------------------------------- widening, A in TMEM
-        // Warps 0..3 of the group widen A: thread = one A row (TMEM lane), its
-        // 64 packed bytes arrive 64-byte swizzled (16-byte chunk c of row r at
-        // c ^ ((r >> 1) & 3)), so eight consecutive rows hit all banks once;
-        // the 128 int8 go to the row's 32 columns of the A stage with one
-        // tcgen05.st.  Warps 4..7 widen B into the swizzled shared-memory
-        // stage.  Column 8c + x (x < 4) of an A stage holds the even codes of
-        // packed word x of chunk c and column 8c + 4 + x its odd codes: the
-        // same K order as the B rows' [even, odd] 16-byte halves.
+        // A stage = two K-blocks.  Warps 0..3 of the group widen A: thread =
+        // one A row (TMEM lane); its 128 packed bytes arrive 128-byte swizzled
+        // (16-byte chunk p of row r at p ^ (r & 7)), so eight consecutive rows
+        // reading the same logical chunk hit all banks once.  Chunk p = 4 h + c
+        // is in K-block h; column 32 h + 8 c + x (x < 4) of the stage holds the
+        // even codes of packed word x of the chunk and column 32 h + 8 c + 4 + x
+        // its odd codes: the K order of the B rows' [even, odd] 16-byte halves.
+        // Warps 4..7 widen B into the swizzled shared-memory stage, one
+        // 128-byte-row tile per K-block.
         const int uw = warp - kWarpUnp0;
         const int my_tiles = num_tiles > first_tile ? (num_tiles - 1 - first_tile) / tile_step + 1 : 0;
         const int total = my_tiles * num_kb;
@@ -486,7 +485,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         if (uw < 4) {
             const int quarter = warp & 3;             // TMEM lanes 32*quarter ..
             const int r = quarter * 32 + lane;
-            const uint32_t rsw = static_cast<uint32_t>((r >> 1) & 3);
+            const uint32_t rsw = static_cast<uint32_t>(r & 7);
             const uint32_t trow = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                   static_cast<uint32_t>(C::A_OFF);
             for (int n = 0; n < total; ++n) {
@@ -495,22 +494,26 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 if (!ptx::mbar_wait(full_p(ps), pph, abort_flag)) break;
                 if (!ptx::mbar_wait<PAIR>(empty_u(us), uph ^ 1, abort_flag)) break;
                 ptx::tc_fence_after();
-                const uint32_t src = sbase + C::OFF_PA + ps * C::PA + r * BKP;
-                uint32_t t[32];
+                const uint32_t src = sbase + C::OFF_PA + ps * C::PA + r * C::PKB;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint4 w = lds128(src + ((static_cast<uint32_t>(c) ^ rsw) << 4));
-                    t[8 * c + 0] = (w.x << 4) & hm;
-                    t[8 * c + 1] = (w.y << 4) & hm;
-                    t[8 * c + 2] = (w.z << 4) & hm;
-                    t[8 * c + 3] = (w.w << 4) & hm;
-                    t[8 * c + 4] = w.x & hm;
-                    t[8 * c + 5] = w.y & hm;
-                    t[8 * c + 6] = w.z & hm;
-                    t[8 * c + 7] = w.w & hm;
+                for (int h = 0; h < C::KS; ++h) {
+                    uint32_t t[32];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const uint32_t chunk = static_cast<uint32_t>(4 * h + c) ^ rsw;
+                        const uint4 w = lds128(src + (chunk << 4));
+                        t[8 * c + 0] = (w.x << 4) & hm;
+                        t[8 * c + 1] = (w.y << 4) & hm;
+                        t[8 * c + 2] = (w.z << 4) & hm;
+                        t[8 * c + 3] = (w.w << 4) & hm;
+                        t[8 * c + 4] = w.x & hm;
+                        t[8 * c + 5] = w.y & hm;
+                        t[8 * c + 6] = w.z & hm;
+                        t[8 * c + 7] = w.w & hm;
+                    }
+                    __syncwarp();   // tcgen05.st is warp-collective
+                    ptx::tmem_st_32x32b_x32(trow + static_cast<uint32_t>(us * C::A_COLS + 32 * h), t);
                 }
-                __syncwarp();   // tcgen05.st is warp-collective
-                ptx::tmem_st_32x32b_x32(trow + static_cast<uint32_t>(us * (BK / 4)), t);
                 ptx::tmem_st_wait();
                 ptx::tc_fence_before();
                 __syncwarp();
@@ -520,32 +523,43 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 }
             }
         } else {
-            // 128 threads over BN rows x 4 chunks: thread bt takes chunk bt & 3
-            // of rows bt / 4 + 32 i; 32 is a multiple of the 8-row swizzle
-            // period, so the swizzle phase of a thread never changes.
+            // 128 threads over BR rows x 2 K-blocks x 4 chunks of 16 bytes:
+            // thread bt takes chunk c = bt & 3 of K-block h = (bt >> 2) & 1, of
+            // rows 32 j + 2 q + (h ^ i) for i = 0, 1 (q = bt >> 3).  The eight
+            // threads of a quarter warp then touch one row's K-block 0 and an
+            // adjacent row's K-block 1: 128 distinct bytes on the packed read,
+            // and chunk sets of opposite swizzle parity on the widened writes,
+            // so neither access has bank conflicts.
             const int bt = threadIdx.x - (kWarpUnp0 + 4) * 32;
-            constexpr int kPerB = C::BR / 32;
+            constexpr int kRowBlocks = C::BR / 32;
             const uint32_t c = static_cast<uint32_t>(bt & 3);
-            const int row0 = bt >> 2;
-            const uint32_t sw8 = static_cast<uint32_t>(row0 & 7);
-            const uint32_t lo_off = ((2u * c) ^ sw8) << 4;
-            const uint32_t hi_off = ((2u * c + 1u) ^ sw8) << 4;
+            const int h = (bt >> 2) & 1;
+            const int q2 = 2 * (bt >> 3);
             for (int n = 0; n < total; ++n) {
                 const int ps = n % C::SP, us = n % C::SU;
                 const uint32_t pph = (n / C::SP) & 1, uph = (n / C::SU) & 1;
                 if (!ptx::mbar_wait(full_p(ps), pph, abort_flag)) break;
                 if (!ptx::mbar_wait<PAIR>(empty_u(us), uph ^ 1, abort_flag)) break;
-                const uint32_t pb = sbase + C::OFF_PB + ps * C::PB + row0 * BKP + c * 16;
-                const uint32_t ub = sbase + C::OFF_UB + us * C::UB + row0 * 128;
-                uint4 w[kPerB];
+                const uint32_t pb = sbase + C::OFF_PB + ps * C::PB + h * BKP + c * 16;
+                const uint32_t ub = sbase + C::OFF_UB + us * C::UB + h * C::UBH;
 #pragma unroll
-                for (int i = 0; i < kPerB; ++i) w[i] = lds128(pb + i * 32 * BKP);
+                for (int j = 0; j < kRowBlocks; ++j) {
+                    uint4 w[2];
+                    int row[2];
 #pragma unroll
-                for (int i = 0; i < kPerB; ++i) {
-                    const uint32_t dst = ub + i * 32 * 128;
-                    sts128(dst + lo_off, (w[i].x << 4) & hm, (w[i].y << 4) & hm,
-                           (w[i].z << 4) & hm, (w[i].w << 4) & hm);
-                    sts128(dst + hi_off, w[i].x & hm, w[i].y & hm, w[i].z & hm, w[i].w & hm);
+                    for (int i = 0; i < 2; ++i) {
+                        row[i] = 32 * j + q2 + (h ^ i);
+                        w[i] = lds128(pb + row[i] * C::PKB);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const uint32_t sw8 = static_cast<uint32_t>(row[i] & 7);
+                        const uint32_t dst = ub + row[i] * 128;
+                        sts128(dst + (((2u * c) ^ sw8) << 4), (w[i].x << 4) & hm, (w[i].y << 4) & hm,
+                               (w[i].z << 4) & hm, (w[i].w << 4) & hm);
+                        sts128(dst + (((2u * c + 1u) ^ sw8) << 4), w[i].x & hm, w[i].y & hm,
+                               w[i].z & hm, w[i].w & hm);
+                    }
                 }
                 ptx::fence_proxy_async_smem();
                 __syncwarp();
