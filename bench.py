@@ -43,6 +43,10 @@ METRIC = "W4A4 linear end-to-end TOPS and % of INT8 tensor peak; prep kernel HBM
 L2_FLUSH_BYTES = 256 << 20
 # Bytes a prep launch must move per row: 2K read (bf16), K/2 + 4 written.
 PREP_BYTES_PER_ROW = lambda K: 2 * K + K // 2 + 4  # noqa: E731
+# GEMM algorithmic bytes: packed codes of both operands, both scale vectors,
+# bias, bf16 output
+GEMM_BYTES = lambda M, N, K: M * K // 2 + N * K // 2 + 4 * (M + N) + 2 * N + 2 * M * N  # noqa: E731
+SKINNY_MAX_M = 128   # the GEMM's few-token form (weight stream, HBM-bound) up to here
 INT8_PER_BF16 = 2.0   # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 
 
@@ -334,12 +338,20 @@ def run_gpu(args):
     if gemm_total >= prep_total:
         i = max(range(nl), key=lambda j: sum(gemm_ms[j]))
         sp = prepared[i][0]
-        roof = {"kernel": "gemm_kernel", "bound": "tensor", "achieved": round(gemm_tops[i], 2),
-                "peak": round(int8_peak, 1), "unit": "TFLOP/s",
-                "frac": round(gemm_tops[i] / int8_peak, 4),
-                "traffic": _traffic(name, "gemm_kernel"),
-                "note": "integer tensor ops (2 per multiply-add); peak = measured bf16 burst "
-                        f"x {INT8_PER_BF16} nominal int8/bf16 ratio ({peaks['src']})"}
+        if sp.M <= SKINNY_MAX_M:
+            gbs = GEMM_BYTES(sp.M, sp.N, sp.K) / (gemm_avg[i] * 1e-3) / 1e9
+            roof = {"kernel": "skinny_kernel", "bound": "hbm", "achieved": round(gbs, 1),
+                    "peak": peaks["hbm"], "unit": "GB/s", "frac": round(gbs / peaks["hbm"], 4),
+                    "traffic": _traffic(name, "skinny_kernel"),
+                    "note": "algorithmic bytes M K/2 + N K/2 + 4(M+N) + 2N + 2MN (the packed "
+                            f"weight stream dominates); HBM peak {peaks['src']}"}
+        else:
+            roof = {"kernel": "gemm_kernel", "bound": "tensor", "achieved": round(gemm_tops[i], 2),
+                    "peak": round(int8_peak, 1), "unit": "TFLOP/s",
+                    "frac": round(gemm_tops[i] / int8_peak, 4),
+                    "traffic": _traffic(name, "gemm_kernel"),
+                    "note": "integer tensor ops (2 per multiply-add); peak = measured bf16 burst "
+                            f"x {INT8_PER_BF16} nominal int8/bf16 ratio ({peaks['src']})"}
     else:
         i = max(range(nl), key=lambda j: sum(prep_ms[j]))
         roof = {"kernel": "prep_kernel", "bound": "hbm", "achieved": round(prep_gbs[i], 1),
@@ -366,6 +378,8 @@ def run_gpu(args):
         "tokens_per_s": round(tokens_s, 1),
         "int8_peak_frac_path": round(value / world / int8_peak, 4),
         "gemm_tops": [round(v, 2) for v in gemm_tops],
+        "gemm_gbs": [round(GEMM_BYTES(sp.M, sp.N, sp.K) / (g * 1e-3) / 1e9, 1)
+                     for (sp, *_), g in zip(prepared, gemm_avg)],
         "prep_gbs": [round(v, 1) for v in prep_gbs],
         "prep_hbm_frac": [round(v / peaks["hbm"], 4) for v in prep_gbs],
         "roofline": roof,

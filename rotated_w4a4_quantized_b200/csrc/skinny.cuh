@@ -55,7 +55,7 @@ template <int BN>
 struct Cfg {
     static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128, "token tile of 16..128");
     // Packed stages in flight: ~100+ KB of the weight stream per SM.
-    static constexpr int SP = BN == 16 ? 8 : BN == 32 ? 7 : BN == 64 ? 6 : 3;
+    static constexpr int SP = BN == 16 ? 11 : BN == 32 ? 9 : BN == 64 ? 6 : 3;
     static constexpr int SU = BN == 128 ? 3 : 4;      // TMEM A stages = widened B stages
     static constexpr int PA = kMaxRows * kPKB;        // packed weight stage (up to 128 rows)
     static constexpr int PB = BN * kPKB;              // packed token stage
@@ -116,7 +116,14 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     const int num_kp = (K / 2 + kPKB - 1) / kPKB;        // stages; K tails are zero-filled
     const uint32_t stage_tx = static_cast<uint32_t>((R + BN) * kPKB);
 
+    // Thread 0 is also the producer: it sets up the barriers and, when the
+    // weights may be read early, requests the first stages of them before
+    // the rest of the set-up (TMEM allocation, the CTA barrier), so the
+    // weight stream starts as early as the CTA does.
+    const int early = early_a ? (num_kp < C::SP ? num_kp : C::SP) : 0;
     if (threadIdx.x == 0) {
+        ptx::tma_prefetch_desc(&tmA);
+        ptx::tma_prefetch_desc(&tmB);
         for (int s = 0; s < C::SP; ++s) {
             ptx::mbar_init(full_p(s), 1);
             ptx::mbar_init(empty_p(s), 8);    // 4 token + 4 weight widening warps
@@ -128,10 +135,10 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         ptx::mbar_init(acc_full, 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
-    }
-    if (warp == kWarpTma && lane == 0) {
-        ptx::tma_prefetch_desc(&tmA);
-        ptx::tma_prefetch_desc(&tmB);
+        for (int kp = 0; kp < early; ++kp) {
+            ptx::mbar_arrive_expect_tx(full_p(kp), stage_tx);
+            ptx::tma_load_2d(sbase + C::OFF_PA + kp * C::PA, &tmA, full_p(kp), kp * kPKB, n0);
+        }
     }
     if (warp == kWarpMma) {
         ptx::tmem_alloc(sbase + C::OFF_MISC, C::TMEM_COLS);
@@ -145,11 +152,6 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     // The producer and MMA loops run in one thread each.
     if (warp == kWarpTma) {
         if (lane == 0) {
-            const int early = early_a ? (num_kp < C::SP ? num_kp : C::SP) : 0;
-            for (int kp = 0; kp < early; ++kp) {
-                ptx::mbar_arrive_expect_tx(full_p(kp), stage_tx);
-                ptx::tma_load_2d(sbase + C::OFF_PA + kp * C::PA, &tmA, full_p(kp), kp * kPKB, n0);
-            }
             ptx::grid_dependency_wait();   // the tokens come from the preceding kernel
             int ps = 0;
             uint32_t ph = 0;
