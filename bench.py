@@ -47,6 +47,8 @@ PREP_BYTES_PER_ROW = lambda K: 2 * K + K // 2 + 4  # noqa: E731
 # bias, bf16 output
 GEMM_BYTES = lambda M, N, K: M * K // 2 + N * K // 2 + 4 * (M + N) + 2 * N + 2 * M * N  # noqa: E731
 SKINNY_MAX_M = 128   # the GEMM's few-token form (weight stream, HBM-bound) up to here
+# whole-layer algorithmic bytes when the layer runs as one kernel
+LAYER_BYTES = lambda M, N, K: 2 * M * K + N * K // 2 + 4 * N + 2 * N + 2 * M * N  # noqa: E731
 INT8_PER_BF16 = 2.0   # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 
 
@@ -335,7 +337,18 @@ def run_gpu(args):
     gemm_tops = [2 * sp.M * sp.N * sp.K / (g * 1e-3) / 1e12 for (sp, *_), g in zip(prepared, gemm_avg)]
     prep_gbs = [sp.M * PREP_BYTES_PER_ROW(sp.K) / (p * 1e-3) / 1e9 for (sp, *_), p in zip(prepared, prep_avg)]
     gemm_total, prep_total = sum(map(sum, gemm_ms)), sum(map(sum, prep_ms))
-    if gemm_total >= prep_total:
+    single = [cr.convrot_linear_single_kernel(sp.M, sp.K, sp.group) for sp, *_ in prepared]
+    if all(single):
+        # the whole step is one decode kernel per layer (token preparation
+        # fused into a CUDA-core GEMV): its algorithmic bytes over the step time
+        byts = sum(LAYER_BYTES(sp.M, sp.N, sp.K) for sp, *_ in prepared)
+        gbs = byts * args.steps / (t_max * 1e-3) / 1e9
+        roof = {"kernel": "decode_kernel", "bound": "hbm", "achieved": round(gbs, 1),
+                "peak": peaks["hbm"], "unit": "GB/s", "frac": round(gbs / peaks["hbm"], 4),
+                "traffic": _traffic(name, "decode_kernel"),
+                "note": "whole layer in one kernel; algorithmic bytes 2MK (x) + NK/2 + 4N + 2N "
+                        f"+ 2MN (y) per step; HBM peak {peaks['src']}"}
+    elif gemm_total >= prep_total:
         i = max(range(nl), key=lambda j: sum(gemm_ms[j]))
         sp = prepared[i][0]
         if sp.M <= SKINNY_MAX_M:
@@ -363,7 +376,7 @@ def run_gpu(args):
     e2e = run_e2e(cr, prepared, spec, dev, stream, flush, args)
     t_e2e, ops_e2e = aggregate(e2e["ms"], ops_step * e2e["steps"], dev)
 
-    launches = 2 * nl * args.steps
+    launches = sum(1 if s1 else 2 for s1 in single) * args.steps
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 5),

@@ -124,6 +124,16 @@ convrot_status convrot_debug_gemm_s32(const uint8_t *qx, const uint8_t *qw, int6
                                       int64_t K, int32_t *acc, convrot_stream_t stream);
 
 /*
+ * Whether convrot_linear runs a layer of this shape as one kernel: 1 when
+ * 1 <= M <= 4, K is a multiple of 2048 and the few token rows can be
+ * prepared inside the GEMM kernel (activation preparation fused into a
+ * CUDA-core GEMV; the workspace is then not touched), 0 when it runs the
+ * prep kernel and the GEMM.  Host-only, no device work; invalid arguments
+ * give 0.  Both forms give bit-identical results.
+ */
+int convrot_linear_single_kernel(int64_t M, int64_t K, int group);
+
+/*
  * Test hook: steps 3-4 (out_s32 = 0: y [M][N] bf16, as convrot_linear_prepared)
  * or step 3 alone (out_s32 = 1: acc [M][N] int32, sx / sw / bias unused) with
  * the token-major GEMM forced to one tile shape, so that each shape can be

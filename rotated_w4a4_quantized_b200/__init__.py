@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
             f = getattr(L, name)
             f.argtypes = args
             f.restype = ctypes.c_int
+        L.convrot_linear_single_kernel.argtypes = [I64, I64, I]
+        L.convrot_linear_single_kernel.restype = I
         L.convrot_linear_workspace_size.argtypes = [I64, I64]
         L.convrot_linear_workspace_size.restype = SZ
         L.convrot_status_string.argtypes = [I]
@@ -116,6 +118,11 @@ def convrot_prepare_act(x: torch.Tensor, group: int, qx=None, sx=None, stream=No
     _check(lib().convrot_prepare_act(_p(x), M, K, group, _p(qx), _p(sx), _stream(stream)),
            "convrot_prepare_act")
     return qx, sx
+
+
+def convrot_linear_single_kernel(M: int, K: int, group: int) -> bool:
+    """True when convrot_linear runs this shape as one kernel (1..4 tokens)."""
+    return bool(lib().convrot_linear_single_kernel(M, K, group))
 
 
 def convrot_linear_workspace_size(M: int, K: int) -> int:

@@ -18,7 +18,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "csrc", "convrot.cu")
 DEPS = [os.path.join(HERE, "csrc", f) for f in ("convrot.cu", "gemm.cuh", "prep.cuh", "ptx.cuh",
-                                                     "skinny.cuh")]
+                                                     "skinny.cuh", "decode.cuh")]
 HEADER = os.path.join(os.path.dirname(HERE), "include", "convrot.h")
 LIB = os.path.join(HERE, "libconvrot.so")
 

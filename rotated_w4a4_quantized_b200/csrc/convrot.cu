@@ -15,6 +15,7 @@
 #include "prep.cuh"
 #include "ptx.cuh"
 #include "skinny.cuh"
+#include "decode.cuh"
 
 namespace {
 
@@ -106,6 +107,12 @@ convrot_status device_setup(int *dev_out) {
     ok &= set_smem(skinny::skinny_kernel<32, true>, skinny::Cfg<32>::SMEM_BYTES);
     ok &= set_smem(skinny::skinny_kernel<64, true>, skinny::Cfg<64>::SMEM_BYTES);
     ok &= set_smem(skinny::skinny_kernel<128, true>, skinny::Cfg<128>::SMEM_BYTES);
+    ok &= set_smem(decode::decode_kernel<1, 64>, kPrepSmemMax);
+    ok &= set_smem(decode::decode_kernel<2, 64>, kPrepSmemMax);
+    ok &= set_smem(decode::decode_kernel<4, 64>, kPrepSmemMax);
+    ok &= set_smem(decode::decode_kernel<1, 256>, kPrepSmemMax);
+    ok &= set_smem(decode::decode_kernel<2, 256>, kPrepSmemMax);
+    ok &= set_smem(decode::decode_kernel<4, 256>, kPrepSmemMax);
     if (ok) {
         // How many CTA pairs fit on the device at once (pairs need two SMs
         // of one GPC); the pair GEMM's persistent grid is that many clusters.
@@ -376,6 +383,53 @@ convrot_status launch_gemm(const DeviceState &ds, const uint8_t *qx, const float
     return CONVROT_ERR_SHAPE;
 }
 
+// The one-kernel path for 1..4 tokens (decode.cuh): token rows prepared in
+// every CTA, GEMV on the CUDA cores.  Returns the ring depth (stages of 16 KB)
+// that fits, or 0 when the shape takes the two-kernel path.
+// R: weight rows per CTA (the ring slots are R x 128 bytes).
+int decode_stages(int64_t M, int64_t K, int group, int R = decode::kRows) {
+    if (M < 1 || M > 4 || K % 2048 != 0) return 0;
+    const int MT = M <= 1 ? 1 : M <= 2 ? 2 : 4;
+    if (MT * (K / prep::kElemsPerThread) > decode::kConsumerWarps * 32) return 0;
+    // A ring of ~6 slots (~80 KB per SM in flight) streams fastest: deeper
+    // rings (up to the whole slice at once) measured 5-8% slower.
+    const int num_kp = static_cast<int>(K / (2 * decode::kPKB));
+    int sp = num_kp < 6 ? num_kp : 6;
+    while (sp >= 2 && decode::smem_bytes(MT, group, static_cast<int>(K), sp, R) + 1024 >
+                          static_cast<size_t>(kPrepSmemMax))
+        --sp;
+    return sp >= 2 ? sp : 0;
+}
+
+template <int MT, int G>
+convrot_status launch_decode_cfg(int num_sms, int SP, const void *x, const uint8_t *qw,
+                                 const float *sw, const void *bias, int64_t M, int64_t N,
+                                 int64_t K, void *y, cudaStream_t stream) {
+    const int R = skinny::rows_per_cta(N, num_sms);
+    CUtensorMap tmW;
+    if (!make_map(&tmW, qw, N, K, decode::kPKB, R, CU_TENSOR_MAP_SWIZZLE_128B)) return CONVROT_ERR_CUDA;
+    const size_t smem = decode::smem_bytes(MT, G, static_cast<int>(K), SP, R) + 1024;
+    const dim3 grid(static_cast<unsigned>((N + R - 1) / R));
+    decode::decode_kernel<MT, G><<<grid, decode::kThreads, smem, stream>>>(
+        tmW, static_cast<const uint16_t *>(x), static_cast<int>(M), static_cast<int>(N),
+        static_cast<int>(K), R, SP, sw, static_cast<const uint16_t *>(bias),
+        static_cast<uint16_t *>(y));
+    return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
+}
+
+convrot_status launch_decode(int num_sms, int SP, const void *x, const uint8_t *qw, const float *sw,
+                             const void *bias, int64_t M, int64_t N, int64_t K, int group, void *y,
+                             cudaStream_t stream) {
+    if (group == 64) {
+        if (M <= 1) return launch_decode_cfg<1, 64>(num_sms, SP, x, qw, sw, bias, M, N, K, y, stream);
+        if (M <= 2) return launch_decode_cfg<2, 64>(num_sms, SP, x, qw, sw, bias, M, N, K, y, stream);
+        return launch_decode_cfg<4, 64>(num_sms, SP, x, qw, sw, bias, M, N, K, y, stream);
+    }
+    if (M <= 1) return launch_decode_cfg<1, 256>(num_sms, SP, x, qw, sw, bias, M, N, K, y, stream);
+    if (M <= 2) return launch_decode_cfg<2, 256>(num_sms, SP, x, qw, sw, bias, M, N, K, y, stream);
+    return launch_decode_cfg<4, 256>(num_sms, SP, x, qw, sw, bias, M, N, K, y, stream);
+}
+
 convrot_status check_gemm_args(const uint8_t *qx, const uint8_t *qw, int64_t M, int64_t N,
                                int64_t K) {
     if (!qx || !qw) return CONVROT_ERR_NULL;
@@ -467,12 +521,21 @@ convrot_status convrot_linear(const void *x_bf16, const uint8_t *qw, const float
     if ((st = check_gemm_args(qw, qw, M, N, K)) != CONVROT_OK) return st;
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    // 1..4 tokens: one kernel (the workspace is not touched)
+    if (const int sp = decode_stages(M, K, group, skinny::rows_per_cta(N, g_dev[dev].num_sms)))
+        return launch_decode(g_dev[dev].num_sms, sp, x_bf16, qw, sw, bias_bf16, M, N, K, group,
+                             y_bf16, stream);
     uint8_t *qx = static_cast<uint8_t *>(workspace);
     float *sx = reinterpret_cast<float *>(qx + round256(static_cast<size_t>(M) * (K / 2)));
     if ((st = launch_prep(g_dev[dev].num_sms, x_bf16, M, K, group, qx, sx, nullptr, stream)) != CONVROT_OK)
         return st;
     return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream,
                               kTilesAuto, true);
+}
+
+int convrot_linear_single_kernel(int64_t M, int64_t K, int group) {
+    if (check_shape(M, K, group) != CONVROT_OK) return 0;
+    return decode_stages(M, K, group) > 0 ? 1 : 0;
 }
 
 convrot_status convrot_debug_rotate_f32(const void *x_bf16, int64_t M, int64_t K, int group,

@@ -103,6 +103,109 @@ __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
+// ------------------------------------------------------------------------
+// The steps of one row, shared by prep_kernel and the fused decode kernel
+// (same instructions in the same order, so both give identical codes).
+// t is the thread's index among the K/64 threads that handle the row.
+
+// Registers v[0..63] <- the thread's 64 channels of a staged bf16 row (the
+// stage layout: chunk c of thread t's 128-byte slice at position c ^ (t & 7)).
+__device__ __forceinline__ void load_row(const uint4 *__restrict__ sb, int t,
+                                         float (&v)[kElemsPerThread]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint4 raw = sb[t * 8 + (i ^ (t & 7))];
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+            v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+    }
+}
+
+// The unnormalised rotation of the thread's channels: digits 0-2 in
+// registers; for n = 256 the four threads of a group (lanes of one warp)
+// hold digit 3 = 0..3 and swap quarters through xb (16 float4 per thread)
+// so that each thread then holds, for its j = t mod 4, the channels
+// 64 d3 + 16 j + r (d3 = 0..3, r = 0..15): digit 3 becomes a register
+// stride of 16 and the last butterfly runs in registers.  Chunk i = 4a + b
+// (4 floats) of thread t is stored at slot (4b + a) ^ (t mod 16) of t's
+// 16-slot row, which keeps both the stores and the transposed loads free of
+// bank conflicts.  mask: the lanes of the warp that take part.
+template <int G>
+__device__ __forceinline__ void rotate_row(float (&v)[kElemsPerThread], float4 *__restrict__ xb,
+                                           int t, uint32_t mask) {
+    radix4_digit0(v);
+    radix4_stage<4>(v);
+    radix4_stage<16>(v);
+    if (G == 256) {
+        const int key = t & 15;
+        __syncwarp(mask);     // the group finished reading the previous swap
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            xb[t * 16 + ((((i & 3) << 2) | (i >> 2)) ^ key)] =
+                make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        __syncwarp(mask);
+        const int j = t & 3, gb = t & ~3;
+#pragma unroll
+        for (int d3 = 0; d3 < 4; ++d3) {
+            const int w = gb + d3;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float4 f = xb[w * 16 + (((c << 2) | j) ^ (w & 15))];
+                v[16 * d3 + 4 * c] = f.x;
+                v[16 * d3 + 4 * c + 1] = f.y;
+                v[16 * d3 + 4 * c + 2] = f.z;
+                v[16 * d3 + 4 * c + 3] = f.w;
+            }
+        }
+        radix4_stage<16>(v);
+    }
+}
+
+// Channel of register e of thread t after rotate_row.
+template <int G>
+__device__ __forceinline__ int row_chan(int t, int e) {
+    if (G == 64) return t * 64 + e;
+    return (t & ~3) * 64 + 64 * (e >> 4) + 16 * (t & 3) + (e & 15);
+}
+
+// The thread's max |v|: four independent chains of three-input maxima.
+__device__ __forceinline__ float thread_absmax(const float (&v)[kElemsPerThread]) {
+    float mk[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int e = 0; e < kElemsPerThread; e += 8)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) mk[k] = max3(mk[k], fabsf(v[e + 2 * k]), fabsf(v[e + 2 * k + 1]));
+    return max3(mk[0], mk[1], fmaxf(mk[2], mk[3]));
+}
+
+// Codes q = round_half_away(v * inv), packed two per byte (low nibble =
+// even register): packed[w] holds registers 8w .. 8w + 7.
+__device__ __forceinline__ void quantize_pack(const float (&v)[kElemsPerThread], float inv,
+                                              uint32_t (&packed)[8]) {
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+        int code[8];
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+            float p0, p1, h0, h1;
+            mul2(p0, p1, v[8 * w + j], v[8 * w + j + 1], inv, inv);
+            // add (0.5 - 2^-25) with the sign of the product, truncate
+            const float c0 = __uint_as_float((__float_as_uint(p0) & 0x80000000u) | 0x3EFFFFFFu);
+            const float c1 = __uint_as_float((__float_as_uint(p1) & 0x80000000u) | 0x3EFFFFFFu);
+            add2(h0, h1, p0, p1, c0, c1);
+            code[j] = __float2int_rz(h0);
+            code[j + 1] = __float2int_rz(h1);
+        }
+        uint32_t word = pack_nibbles(code[7], code[6], 0u);
+        word = pack_nibbles(code[5], code[4], word);
+        word = pack_nibbles(code[3], code[2], word);
+        packed[w] = pack_nibbles(code[1], code[0], word);
+    }
+}
+
 // MODE 0: quantise + pack (q, s).  MODE 1: write the normalised rotated row
 // as fp32 (yrot) instead.
 //
@@ -162,59 +265,13 @@ prep_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ 
         __syncthreads();          // ... and everyone else's
 
         float v[kElemsPerThread];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint4 raw = stage[t * 8 + (i ^ (t & 7))];
-            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
-                v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-            }
-        }
+        load_row(stage, t, v);
         __syncthreads();          // the stage buffer is free again
         if (next < M) issue_row(next, 0);
         cp_async_commit();
 
-        radix4_digit0(v);
-        radix4_stage<4>(v);
-        radix4_stage<16>(v);
-        // For n = 256 the four threads of a group hold digit 3 = 0..3.  They
-        // swap quarters through shared memory so that each thread then holds,
-        // for its j = t mod 4, the channels 64 d3 + 16 j + r (d3 = 0..3,
-        // r = 0..15): digit 3 becomes a register stride of 16 and the last
-        // butterfly runs in registers.  Chunk i = 4a + b (4 floats) of thread t
-        // is stored at slot (4b + a) ^ (t mod 16) of t's 16-slot row, which
-        // keeps both the stores and the transposed loads free of bank conflicts.
-        if (kDigits == 4) {
-            float4 *xb = reinterpret_cast<float4 *>(stage + row_chunks);
-            const int key = t & 15;
-            __syncwarp(mask);     // the group finished reading the previous row's swap
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                xb[t * 16 + ((((i & 3) << 2) | (i >> 2)) ^ key)] =
-                    make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-            __syncwarp(mask);
-            const int j = t & 3, gb = t & ~3;
-#pragma unroll
-            for (int d3 = 0; d3 < 4; ++d3) {
-                const int w = gb + d3;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const float4 f = xb[w * 16 + (((c << 2) | j) ^ (w & 15))];
-                    v[16 * d3 + 4 * c] = f.x;
-                    v[16 * d3 + 4 * c + 1] = f.y;
-                    v[16 * d3 + 4 * c + 2] = f.z;
-                    v[16 * d3 + 4 * c + 3] = f.w;
-                }
-            }
-            radix4_stage<16>(v);
-        }
-        // Position in the row of register e of this thread.
-        auto chan = [&](int e) -> int {
-            if (kDigits == 3) return t * 64 + e;
-            return (t & ~3) * 64 + 64 * (e >> 4) + 16 * (t & 3) + (e & 15);
-        };
+        rotate_row<G>(v, reinterpret_cast<float4 *>(stage + row_chunks), t, mask);
+        auto chan = [&](int e) -> int { return row_chan<G>(t, e); };
 
         if (MODE == 1) {
             float *dst = yrot + static_cast<size_t>(row) * K;
@@ -226,14 +283,7 @@ prep_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ 
             continue;
         }
 
-        // Row absmax: four independent chains of three-input maxima (16 deep
-        // instead of one chain 64 deep).
-        float mk[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-        for (int e = 0; e < kElemsPerThread; e += 8)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) mk[k] = max3(mk[k], fabsf(v[e + 2 * k]), fabsf(v[e + 2 * k + 1]));
-        float m = max3(mk[0], mk[1], fmaxf(mk[2], mk[3]));
+        const float m = thread_absmax(v);
         // non-negative floats order like their bit patterns
         uint32_t mb = __reduce_max_sync(mask, __float_as_uint(m));
         if (lane == 0) red[warp] = mb;
@@ -246,25 +296,7 @@ prep_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ 
         if (t == 0) s[row] = __fdiv_rn(a_u * kNorm, 7.0f);
 
         uint32_t packed[8];
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            int code[8];
-#pragma unroll
-            for (int j = 0; j < 8; j += 2) {
-                float p0, p1, h0, h1;
-                mul2(p0, p1, v[8 * w + j], v[8 * w + j + 1], inv, inv);
-                // add (0.5 - 2^-25) with the sign of the product, truncate
-                const float c0 = __uint_as_float((__float_as_uint(p0) & 0x80000000u) | 0x3EFFFFFFu);
-                const float c1 = __uint_as_float((__float_as_uint(p1) & 0x80000000u) | 0x3EFFFFFFu);
-                add2(h0, h1, p0, p1, c0, c1);
-                code[j] = __float2int_rz(h0);
-                code[j + 1] = __float2int_rz(h1);
-            }
-            uint32_t word = pack_nibbles(code[7], code[6], 0u);
-            word = pack_nibbles(code[5], code[4], word);
-            word = pack_nibbles(code[3], code[2], word);
-            packed[w] = pack_nibbles(code[1], code[0], word);
-        }
+        quantize_pack(v, inv, packed);
         uint8_t *qrow = q + static_cast<size_t>(row) * (K / 2);
         if (kDigits == 3) {
             uint4 *dst = reinterpret_cast<uint4 *>(qrow + t * 32);

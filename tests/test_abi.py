@@ -93,6 +93,20 @@ def test_host_validation_without_device(L):
     assert L.convrot_debug_gemm_tiles(None, None, None, None, None, 0, 8, 128, 3, 1, None, s) == 0
 
 
+def test_single_kernel_rule(L):
+    # one kernel for 1..4 tokens when K is a multiple of 2048 and the token
+    # rows fit one round of in-kernel preparation (M * K / 64 <= 256 threads)
+    assert L.convrot_linear_single_kernel(1, 4096, 64) == 1
+    assert L.convrot_linear_single_kernel(4, 4096, 256) == 1
+    assert L.convrot_linear_single_kernel(2, 8192, 64) == 1
+    assert L.convrot_linear_single_kernel(1, 16384, 256) == 1
+    assert L.convrot_linear_single_kernel(3, 8192, 64) == 0      # 4 x 128 threads
+    assert L.convrot_linear_single_kernel(5, 4096, 64) == 0
+    assert L.convrot_linear_single_kernel(0, 4096, 64) == 0
+    assert L.convrot_linear_single_kernel(1, 3072, 64) == 0      # K % 2048
+    assert L.convrot_linear_single_kernel(1, 4096, 128) == 0     # bad group
+
+
 def test_valid_call_without_gpu_reports_cuda_error(L):
     import torch
     if torch.cuda.is_available():

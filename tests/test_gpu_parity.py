@@ -250,6 +250,35 @@ def test_linear_matches_oracle(group, M, K, N):
     _full_path_case(lt, group)
 
 
+# The one-kernel path for 1..4 tokens (K a multiple of 2048, M * K <= 16384
+# for 4 tokens' worth of preparation threads): against the oracle, and
+# bit-identical to the two-kernel path (prep kernel + GEMM) on the same inputs.
+DECODE_CASES = [(1, 2048, 1000, 64, True), (1, 4096, 14336, 64, False), (2, 4096, 777, 256, True),
+                (3, 4096, 1024, 256, True), (4, 4096, 3000, 64, True), (1, 16384, 520, 256, False),
+                (2, 8192, 384, 64, True), (4, 2048, 130, 256, False)]
+
+
+@pytest.mark.parametrize("M,K,N,group,bias", DECODE_CASES)
+def test_decode_path_matches_oracle(M, K, N, group, bias):
+    lt = _layer(M, K, N, group, seed=M * 7 + K + N, bias=bias, zero_rows=(1,) if M > 2 else ())
+    cols = None if N <= 4096 else np.r_[0:300, N - 300:N]
+    _full_path_case(lt, group, cols=cols)
+
+
+@pytest.mark.parametrize("M,K,N,group,bias", DECODE_CASES)
+def test_decode_path_equals_two_kernel_path(M, K, N, group, bias):
+    lt = _layer(M, K, N, group, seed=M * 11 + K + N, bias=bias)
+    x, w = _dev(lt.x), _dev(lt.w)
+    b = None if lt.b is None else _dev(lt.b)
+    qw, sw = cr.convrot_quantize_weight(w, group)
+    y1 = cr.convrot_linear(x, qw, sw, b, group)
+    qx, sx = cr.convrot_prepare_act(x, group)
+    y2 = cr.convrot_linear_prepared(qx, sx, qw, sw, b, K)
+    torch.cuda.synchronize()
+    assert cr.convrot_check_device_error() == 0
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
 def test_zero_rows_give_exactly_the_bias():
     lt = _layer(140, 512, 96, 256, seed=5, zero_rows=(0, 77, 139))
     y = _full_path_case(lt, 256)
