@@ -144,10 +144,11 @@ int convrot_linear_single_kernel(int64_t M, int64_t K, int group);
  *           3  256 x 192 tiles on CTA pairs (cta_group::2);
  *           4  few-token form (M <= 128): weights widened into TMEM, one
  *              CTA per slice of weight rows (the automatic choice there);
- *           5  few-token form with both operands widened in shared memory.
+ *           5  few-token form with both operands widened in shared memory;
+ *           6  256 x 128 tiles on CTA pairs (four TMEM A stages).
  * Returns CONVROT_ERR_SHAPE for any other value or for 4 / 5 with M > 128,
  * and CONVROT_ERR_UNSUPPORTED when the device cannot co-schedule CTA pairs
- * (tiles = 3).
+ * (tiles = 3, 6).
  */
 convrot_status convrot_debug_gemm_tiles(const uint8_t *qx, const float *sx, const uint8_t *qw,
                                         const float *sw, const void *bias_bf16, int64_t M,

@@ -99,6 +99,8 @@ convrot_status device_setup(int *dev_out) {
     ok &= set_smem(gemm::gemm_kernel<128, true, true>, gemm::Cfg<128, true>::SMEM_BYTES);
     ok &= set_smem(gemm::gemm_kernel<192, false, false, true>, gemm::Cfg<192, false, true>::SMEM_BYTES);
     ok &= set_smem(gemm::gemm_kernel<192, false, true, true>, gemm::Cfg<192, false, true>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<128, false, false, true>, gemm::Cfg<128, false, true>::SMEM_BYTES);
+    ok &= set_smem(gemm::gemm_kernel<128, false, true, true>, gemm::Cfg<128, false, true>::SMEM_BYTES);
     ok &= set_smem(skinny::skinny_kernel<16, false>, skinny::Cfg<16>::SMEM_BYTES);
     ok &= set_smem(skinny::skinny_kernel<32, false>, skinny::Cfg<32>::SMEM_BYTES);
     ok &= set_smem(skinny::skinny_kernel<64, false>, skinny::Cfg<64>::SMEM_BYTES);
@@ -321,7 +323,7 @@ convrot_status launch_skinny(int num_sms, const uint8_t *qx, const float *sx, co
 // the two few-token forms (M <= 128).
 enum TileChoice {
     kTilesAuto = 0, kTiles128x256 = 1, kTiles128x192 = 2, kTiles256x192Pair = 3,
-    kSkinnyTmem = 4, kSkinnySmem = 5
+    kSkinnyTmem = 4, kSkinnySmem = 5, kTiles256x128Pair = 6
 };
 
 // Path choice: up to 128 tokens the few-token form (weights on the 128-row
@@ -353,21 +355,28 @@ convrot_status launch_gemm(const DeviceState &ds, const uint8_t *qx, const float
                                                    stream);
     }
     if (tiles == kTilesAuto) {
-        // Time of one K-block step of a wave of tiles, in cycles, as measured
-        // on these kernels: the 128 x 256 tile widens both operands through
-        // shared memory (~940); the 128 x 192 tile keeps A in TMEM (~670);
-        // the 256 x 192 pair splits B between two SMs, so each SM moves 40%
-        // fewer shared-memory bytes per MMA (~620 for twice the rows).
-        // A tile count just above a multiple of the slots wastes a wave.
-        const auto waves = [](int64_t t, int64_t slots) { return (t + slots - 1) / slots; };
-        const int64_t n192 = (N + 191) / 192, n256 = (N + 255) / 256;
-        const int64_t c_ss = waves(((M + 127) / 128) * n256, num_sms) * 940;
-        const int64_t c_atm = waves(((M + 127) / 128) * n192, num_sms) * 670;
-        const int64_t c_pair =
-            ds.pair_clusters > 0 ? waves(((M + 255) / 256) * n192, ds.pair_clusters) * 620 : INT64_MAX;
-        tiles = c_pair <= c_atm && c_pair <= c_ss ? kTiles256x192Pair
-                : c_atm <= c_ss                   ? kTiles128x192
-                                                  : kTiles128x256;
+        // Measured on layers of 1024-8192 tokens and K 3072-12288: the
+        // 256 x 192 pair beats both single-CTA shapes everywhere (each SM
+        // widens half of B and the tensor core reads A from TMEM), and the
+        // 256 x 128 pair (four TMEM A stages instead of two) was within a few
+        // per cent either way, so the pair runs 256 x 192.  Without CTA
+        // pairs the cost is wave-weighted (a tile count just above a multiple
+        // of the SMs wastes a wave): one 256-code stage of a wave takes ~1880
+        // cycles on 128 x 256 tiles (both operands widened in shared memory)
+        // and ~1340 on 128 x 192 (A in TMEM).
+        if (ds.pair_clusters > 0) {
+            tiles = kTiles256x192Pair;
+        } else {
+            const auto waves = [](int64_t t, int64_t slots) { return (t + slots - 1) / slots; };
+            const int64_t c_ss = waves(((M + 127) / 128) * ((N + 255) / 256), num_sms) * 1880;
+            const int64_t c_atm = waves(((M + 127) / 128) * ((N + 191) / 192), num_sms) * 1340;
+            tiles = c_atm <= c_ss ? kTiles128x192 : kTiles128x256;
+        }
+    }
+    if (tiles == kTiles256x128Pair) {
+        if (ds.pair_clusters <= 0) return CONVROT_ERR_UNSUPPORTED;
+        return launch_gemm_cfg<128, false, OUT_S32, true>(ds.pair_clusters, qx, qw, M, N, K, sx, sw,
+                                                          bias, out, M, N, stream);
     }
     if (tiles == kTiles256x192Pair) {
         if (ds.pair_clusters <= 0) return CONVROT_ERR_UNSUPPORTED;
@@ -569,7 +578,7 @@ convrot_status convrot_debug_gemm_tiles(const uint8_t *qx, const float *sx, cons
                                         int64_t N, int64_t K, int tiles, int out_s32, void *out,
                                         convrot_stream_t stream) {
     if (M < 0 || N < 0) return CONVROT_ERR_SHAPE;
-    if (tiles < kTilesAuto || tiles > kSkinnySmem) return CONVROT_ERR_SHAPE;
+    if (tiles < kTilesAuto || tiles > kTiles256x128Pair) return CONVROT_ERR_SHAPE;
     if (M == 0 || N == 0) return CONVROT_OK;
     convrot_status st = check_gemm_args(qx, qw, M, N, K);
     if (st != CONVROT_OK) return st;

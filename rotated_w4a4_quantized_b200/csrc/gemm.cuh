@@ -61,7 +61,7 @@ constexpr int kStoreBox = 32;    // epilogue TMA-store box: 32 rows x 32 bf16
 template <int BN, bool SWAP, bool PAIR = false>
 struct Cfg {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "kind::i8 with M=128 needs N%16==0");
-    static_assert(!PAIR || (!SWAP && BN == 192), "the CTA pair runs 256 x 192 tiles");
+    static_assert(!PAIR || (!SWAP && (BN == 192 || BN == 128)), "the CTA pair runs 256 x 192 or 256 x 128 tiles");
     static constexpr int CG = PAIR ? 2 : 1;          // tcgen05 CTA group
     static constexpr int TM = PAIR ? 2 * BM : BM;    // rows of A per tile
     static constexpr int BR = PAIR ? BN / 2 : BN;    // rows of B per CTA
@@ -83,10 +83,12 @@ struct Cfg {
     static constexpr bool ATM = PAIR || (!SWAP && BN == 192);
     static constexpr int KS = ATM ? 2 : 1;           // K-blocks per widened stage
     static constexpr int SP = PAIR ? 4 : ATM ? 2 : BN == 256 ? 3 : BN == 192 ? 5 : BN == 128 ? 3 : BN == 64 ? 4 : BN == 32 ? 5 : 3;
-    static constexpr int SU = ATM ? 2 : BN >= 192 ? 2 : BN == 128 ? 4 : BN == 64 ? 5 : 6;
+    // the 256 x 128 pair has room in TMEM for four A stages (2 x 128
+    // accumulator columns + 4 x 64), the 192-wide tiles for two
+    static constexpr int SU = (PAIR && BN == 128) ? 4 : ATM ? 2 : BN >= 192 ? 2 : BN == 128 ? 4 : BN == 64 ? 5 : 6;
     // The widening warps split into UG groups that take alternate stages, so
     // the hand-off latency of one stage overlaps the widening of the next.
-    static constexpr int UG = BN >= 192 ? 1 : 2;
+    static constexpr int UG = (ATM || BN >= 192) ? 1 : 2;   // the TMEM-A widening runs as one group
     static_assert(SU >= UG, "each group needs a widened stage of its own");
     // Packed stages of the narrow tiles carry PKB bytes of each row (PSUB
     // K-blocks), so the weight stream is read in longer contiguous pieces;
@@ -166,15 +168,19 @@ __device__ __forceinline__ float epi(uint32_t raw, float sx, float sw, float b) 
 // The same arithmetic for two adjacent columns, returning their bf16 pair
 // (low half = first column).  float(acc) is formed exactly without the
 // conversion unit: for |acc| < 2^22 the bit pattern 0x4B400000 + acc is the
-// float 1.5 * 2^23 + acc, and subtracting 1.5 * 2^23 is exact.
+// float 1.5 * 2^23 + acc, and subtracting 1.5 * 2^23 is exact.  The last
+// multiply and the bias add are scalar round-to-nearest operations: ptxas
+// fuses a packed mul.rn.f32x2 feeding an add.rn.f32x2 into one fused
+// multiply-add (measured on sm_100a), which rounds once instead of twice
+// and, where the bias cancels the product, changes the bf16 result.
 __device__ __forceinline__ uint32_t epi_pair(uint32_t r0, uint32_t r1, float sx, float sw0,
                                              float sw1, float b0, float b1) {
     float f0 = __int_as_float((static_cast<int>(r0) >> 8) + 0x4B400000);
     float f1 = __int_as_float((static_cast<int>(r1) >> 8) + 0x4B400000);
     ptx::add2(f0, f1, f0, f1, -12582912.0f, -12582912.0f);
     ptx::mul2(f0, f1, f0, f1, sx, sx);
-    ptx::mul2(f0, f1, f0, f1, sw0, sw1);
-    ptx::add2(f0, f1, f0, f1, b0, b1);
+    f0 = __fadd_rn(__fmul_rn(f0, sw0), b0);
+    f1 = __fadd_rn(__fmul_rn(f1, sw1), b1);
     const __nv_bfloat162 h = __floats2bfloat162_rn(f0, f1);
     return *reinterpret_cast<const uint32_t *>(&h);
 }

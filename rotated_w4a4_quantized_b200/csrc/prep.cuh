@@ -189,15 +189,15 @@ __device__ __forceinline__ void quantize_pack(const float (&v)[kElemsPerThread],
     for (int w = 0; w < 8; ++w) {
         int code[8];
 #pragma unroll
-        for (int j = 0; j < 8; j += 2) {
-            float p0, p1, h0, h1;
-            mul2(p0, p1, v[8 * w + j], v[8 * w + j + 1], inv, inv);
+        for (int j = 0; j < 8; ++j) {
+            // the product is rounded to fp32 before the offset is added: scalar
+            // round-to-nearest operations, which ptxas does not fuse (a packed
+            // mul.rn.f32x2 feeding an add.rn.f32x2 becomes one fused
+            // multiply-add on sm_100a)
+            const float p = __fmul_rn(v[8 * w + j], inv);
             // add (0.5 - 2^-25) with the sign of the product, truncate
-            const float c0 = __uint_as_float((__float_as_uint(p0) & 0x80000000u) | 0x3EFFFFFFu);
-            const float c1 = __uint_as_float((__float_as_uint(p1) & 0x80000000u) | 0x3EFFFFFFu);
-            add2(h0, h1, p0, p1, c0, c1);
-            code[j] = __float2int_rz(h0);
-            code[j + 1] = __float2int_rz(h1);
+            const float c = __uint_as_float((__float_as_uint(p) & 0x80000000u) | 0x3EFFFFFFu);
+            code[j] = __float2int_rz(__fadd_rn(p, c));
         }
         uint32_t word = pack_nibbles(code[7], code[6], 0u);
         word = pack_nibbles(code[5], code[4], word);

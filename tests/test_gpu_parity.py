@@ -109,8 +109,8 @@ def test_gemm_s32_bit_exact(M, N, K):
 # Every token-major tile shape on its own, whatever the automatic choice:
 # ragged M, N and K tails, several tiles per CTA (the persistent loop and the
 # double-buffered accumulator), and an odd tile count for the CTA pairs.
-TILE_SHAPES = [cr.TILES_128x256, cr.TILES_128x192, cr.TILES_256x192_PAIR]
-TILE_IDS = ["128x256", "128x192tmem", "256x192pair"]
+TILE_SHAPES = [cr.TILES_128x256, cr.TILES_128x192, cr.TILES_256x192_PAIR, cr.TILES_256x128_PAIR]
+TILE_IDS = ["128x256", "128x192tmem", "256x192pair", "256x128pair"]
 TILE_CASES = [(1, 16, 64), (100, 200, 192), (257, 385, 1088), (384, 576, 2048),
               (1000, 2000, 512), (2304, 3072, 256), (2304, 3072, 3072)]
 
@@ -193,6 +193,34 @@ def test_gemm_tiles_epilogue_one_ulp(tiles, M, N, K, bias):
                                     None if lt.b is None else _dev(lt.b), K, tiles)
     torch.cuda.synchronize()
     gc.check_outputs(gc.to_np_u16(y), y_ref)
+
+
+# acc * s_x * s_w nearly cancels the bias here: rounding the product to fp32
+# before adding the bias (the definition) gives bf16 0x33f0, a fused
+# multiply-add gives 0x33f3.  Every GEMM form and both store paths (TMA boxes
+# for N % 8 == 0, direct stores otherwise) must round twice.
+@pytest.mark.parametrize("M,N", [(1, 16), (1, 7), (5, 40), (200, 16), (200, 9), (130, 520)])
+def test_epilogue_rounds_product_before_bias(M, N):
+    K = 64
+    a = np.zeros((M, K), np.int8)
+    b = np.zeros((N, K), np.int8)
+    a[:, 0], b[:, 0] = 2, 4                                  # acc = 8 everywhere
+    pa, pb = O.pack(a), O.pack(b)
+    sx = np.full(M, 0.47859192, np.float32)
+    sw = np.full(N, 0.008799647, np.float32)
+    bias = np.full(N, 0xBD0A, np.uint16)                      # -0.033691406
+    y_ref = O.epilogue(O.gemm(pa, pb, K), sx, sw, bias)
+    assert np.all(y_ref == 0x33F0)
+    t = lambda v: _dev(torch.from_numpy(v))
+    bt = t(bias.view(np.int16)).view(torch.bfloat16)
+    forms = [cr.TILES_AUTO] + (TILE_SHAPES + [cr.SKINNY_SMEM] if M <= 128 else TILE_SHAPES)
+    for form in forms + ([cr.SKINNY_TMEM] if M <= 128 else []):
+        y = cr.convrot_debug_gemm_tiles(t(pa), t(sx), t(pb), t(sw), bt, K, form)
+        torch.cuda.synchronize()
+        assert np.array_equal(gc.to_np_u16(y), y_ref), form
+    y = cr.convrot_linear_prepared(t(pa), t(sx), t(pb), t(sw), bt, K)
+    torch.cuda.synchronize()
+    assert np.array_equal(gc.to_np_u16(y), y_ref)
 
 
 @pytest.mark.parametrize("M,N,K,bias", [(3, 48, 256, True), (40, 200, 1024, False),
