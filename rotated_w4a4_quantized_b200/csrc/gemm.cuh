@@ -100,7 +100,9 @@ struct Cfg {
     static constexpr int UA = ATM ? 0 : BM * BK;
     static constexpr int UBH = BR * BK;               // widened B tile of one K-block
     static constexpr int UB = KS * UBH;
-    static constexpr int SB = 2;   // store boxes per epilogue warp
+    // store boxes per epilogue warp: three let the pair's epilogue (3 boxes
+    // per tile and warp) issue every store without waiting for a box
+    static constexpr int SB = PAIR ? 3 : 2;
     static constexpr int ST = SWAP ? 0 : kEpiWarps * SB * kStoreBox * kStoreBox * 2;
     static constexpr int OFF_UA = 0;                   // 1024-aligned tiles first
     static constexpr int OFF_UB = OFF_UA + SU * UA;
@@ -472,7 +474,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             __syncwarp();
             if (lane == 0) arrive_leader(acc_empty(b));
         }
-        if (tma_out && lane == 0) ptx::bulk_wait_all();
+        // The boxes must have been read before the CTA's shared memory goes;
+        // the global writes complete with the grid.
+        if (tma_out && lane == 0) ptx::bulk_wait_read<0>();
     } else if constexpr (C::ATM) {
         // ------------------------------------------------- widening, A in TMEM
         // A stage = two K-blocks.  Warps 0..3 of the group widen A: thread =
