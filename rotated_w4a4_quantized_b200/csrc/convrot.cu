@@ -400,10 +400,10 @@ int decode_stages(int64_t M, int64_t K, int group, int R = decode::kRows) {
     if (M < 1 || M > 4 || K % 2048 != 0) return 0;
     const int MT = M <= 1 ? 1 : M <= 2 ? 2 : 4;
     if (MT * (K / prep::kElemsPerThread) > decode::kConsumerWarps * 32) return 0;
-    // A ring of ~6 slots (~80 KB per SM in flight) streams fastest: deeper
-    // rings (up to the whole slice at once) measured 5-8% slower.
-    const int num_kp = static_cast<int>(K / (2 * decode::kPKB));
-    int sp = num_kp < 6 ? num_kp : 6;
+    // Three slots of 512 bytes per row (~160 KB per SM in flight) stream as
+    // fast as the whole slice at once and leave room for long rows.
+    const int num_kp = static_cast<int>(K / (2 * decode::kPKB * decode::kBlocks));
+    int sp = num_kp < 3 ? num_kp : 3;
     while (sp >= 2 && decode::smem_bytes(MT, group, static_cast<int>(K), sp, R) + 1024 >
                           static_cast<size_t>(kPrepSmemMax))
         --sp;

@@ -14,17 +14,23 @@
 // no hand-off:
 //   * CTA i owns weight rows [i R, i R + R) over the whole of K (R as for the
 //     few-token GEMM: the multiple of 8 that spreads N over the SMs); warp 8
-//     issues TMA copies of its packed rows, 256 codes (128 bytes) per row per
-//     stage, 128-byte swizzled, into a ring of SP R-row slots whose stages
-//     are all requested at kernel start, right after the token rows;
+//     issues TMA copies of its packed rows into a ring of SP slots, a stage
+//     being 512 contiguous bytes (1024 codes) of each of the R rows, loaded
+//     as four 128-byte swizzled column blocks on one barrier.  The first SP
+//     stages are requested at kernel start, right after the token rows.
+//     Wide stages matter: with 128 bytes per row per stage the one-shot
+//     29 MB stream of a 4096 x 14336 layer measured 3.9 TB/s, with 512
+//     bytes about 5.5 TB/s;
 //   * warps 0-7 first prepare the tokens: token m is handled by K/64 threads
 //     exactly as in prep_kernel (staged bf16 row, radix-4 butterflies,
 //     absmax, round-half-away, nibble packing), then widen the packed codes
 //     to int8 words in shared memory (16 x code, even and odd codes of each
 //     packed word apart, as the GEMM widens them);
 //   * then thread (r, h) of warps 0-7 takes weight row r and K-block h of
-//     every stage: it widens its 64 packed bytes and accumulates
-//     sum 256 q_w q_x with dp4a (s8 x s8 -> s32) on the CUDA cores, exactly;
+//     each column block: it widens its 64 packed bytes and accumulates
+//     sum 256 q_w q_x with dp4a (s8 x s8 -> s32) on the CUDA cores, exactly,
+//     in four independent chains (integer sums: any order gives the same
+//     result) so that the dp4a latency does not serialise the stage;
 //     with <= 4 tokens the tensor core would spend its ~75-cycle minimum per
 //     128-row MMA on 1-4 useful columns, while dp4a needs about one
 //     instruction per weight byte per token;
@@ -45,16 +51,17 @@ constexpr int kConsumerWarps = 8;                        // 128 rows x 2 K-block
 constexpr int kWarpTma = kConsumerWarps;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;      // 288
 constexpr int kRows = skinny::kMaxRows;                  // weight rows per CTA at most
-constexpr int kPKB = skinny::kPKB;                       // packed bytes per row per stage
+constexpr int kPKB = skinny::kPKB;                       // packed bytes per row per column block
+constexpr int kBlocks = 4;                               // column blocks per stage
 constexpr int kBarConsumers = 15;                        // named barrier: warps 0-7
 
 // Shared memory of a launch (bytes, without the 1024 alignment slack):
-// ring of SP slots of R x 128 bytes | widened tokens (MT x K) | token prep
+// ring of SP slots of R x 512 bytes | widened tokens (MT x K) | token prep
 // areas | K-half partial sums | barriers.  R is a multiple of 8, so every
 // slot stays aligned to the 1024-byte swizzle atom.
 inline size_t smem_bytes(int MT, int G, int K, int SP, int R) {
     const size_t prep_per_tok = static_cast<size_t>(K) * (G == 256 ? 4 : 2);
-    return static_cast<size_t>(SP) * R * kPKB + static_cast<size_t>(MT) * K +
+    return static_cast<size_t>(SP) * kBlocks * R * kPKB + static_cast<size_t>(MT) * K +
            MT * prep_per_tok + static_cast<size_t>(kRows) * MT * 4 + 2 * SP * 8 + 16;
 }
 
@@ -76,7 +83,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t *__restric
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = ptx::smem_u32(smem);
     const size_t prep_per_tok = static_cast<size_t>(K) * (G == 256 ? 4 : 2);
-    const int slot = R * kPKB;                           // ring slot bytes
+    const int blk = R * kPKB;                            // one column block of a stage
+    const int slot = kBlocks * blk;                      // ring slot bytes
     uint32_t *xw = reinterpret_cast<uint32_t *>(smem + static_cast<size_t>(SP) * slot);
     uint8_t *prep_area = reinterpret_cast<uint8_t *>(xw) + static_cast<size_t>(MT) * K;
     int32_t *accs = reinterpret_cast<int32_t *>(prep_area + MT * prep_per_tok);
@@ -90,8 +98,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t *__restric
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = static_cast<int>(blockIdx.x) * R;
-    const int num_kp = K / (2 * kPKB);                   // K is a multiple of 2048
-    const uint32_t stage_tx = static_cast<uint32_t>(R * kPKB);
+    const int num_kp = K / (2 * kPKB * kBlocks);         // K is a multiple of 2048
+    const uint32_t stage_tx = static_cast<uint32_t>(slot);
     const uint32_t hm = 0xF0F0F0F0u;
 
     // The token rows are requested first, ahead of the weight burst, so that
@@ -122,7 +130,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t *__restric
         // The whole ring at once: the weights are this call's input.
         for (int kp = 0; kp < SP && kp < num_kp; ++kp) {
             ptx::mbar_arrive_expect_tx(full_p(kp), stage_tx);
-            ptx::tma_load_2d(sbase + kp * slot, &tmW, full_p(kp), kp * kPKB, n0);
+            for (int q = 0; q < kBlocks; ++q)
+                ptx::tma_load_2d(sbase + kp * slot + q * blk, &tmW, full_p(kp),
+                                 (kp * kBlocks + q) * kPKB, n0);
         }
     }
     __syncthreads();
@@ -134,7 +144,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t *__restric
                 const int s = kp % SP;
                 if (!ptx::mbar_wait(empty_p(s), ((kp / SP) - 1) & 1, abort_flag)) break;
                 ptx::mbar_arrive_expect_tx(full_p(s), stage_tx);
-                ptx::tma_load_2d(sbase + s * slot, &tmW, full_p(s), kp * kPKB, n0);
+                for (int q = 0; q < kBlocks; ++q)
+                    ptx::tma_load_2d(sbase + s * slot + q * blk, &tmW, full_p(s),
+                                     (kp * kBlocks + q) * kPKB, n0);
             }
         }
         return;
@@ -181,36 +193,48 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t *__restric
     const int r = threadIdx.x & (kRows - 1);             // weight row in the slice
     const int h = threadIdx.x >> 7;                      // K-block of each stage
     const uint32_t rsw = static_cast<uint32_t>(r & 7);
-    int acc[MT];
+    int a4[MT][4];                                       // chain c: words 4c .. 4c + 3
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[m] = 0;
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) a4[m][c] = 0;
     bool ok = true;
     for (int kp = 0; kp < num_kp; ++kp) {
         const int s = kp % SP;
         if (!ptx::mbar_wait(full_p(s), (kp / SP) & 1, abort_flag)) { ok = false; break; }
-        const uint32_t src = sbase + s * slot + r * kPKB;
-        const uint32_t xk = ptx::smem_u32(xw) + static_cast<uint32_t>((2 * kp + h) * 128);
+        if (r < R) {                                     // rows past the slice only wait
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            if (r >= R) break;                           // rows past the slice
-            const uint4 wv = gemm::lds128(src + ((static_cast<uint32_t>(4 * h + c) ^ rsw) << 4));
-            const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+            for (int q = 0; q < kBlocks; ++q) {
+                const uint32_t src = sbase + s * slot + q * blk + r * kPKB;
+                const uint32_t xk = ptx::smem_u32(xw) +
+                                    static_cast<uint32_t>((2 * (kp * kBlocks + q) + h) * 128);
 #pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                // words 4c .. 4c + 3 of the K-block: (even, odd) pairs
-                const uint32_t xa = xk + static_cast<uint32_t>(m * K + 32 * c);
-                const uint4 x0 = gemm::lds128(xa), x1 = gemm::lds128(xa + 16);
-                const uint32_t xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 wv = gemm::lds128(src + ((static_cast<uint32_t>(4 * h + c) ^ rsw) << 4));
+                    const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    acc[m] = __dp4a(static_cast<int>((ww[j] << 4) & hm), static_cast<int>(xv[2 * j]), acc[m]);
-                    acc[m] = __dp4a(static_cast<int>(ww[j] & hm), static_cast<int>(xv[2 * j + 1]), acc[m]);
+                    for (int m = 0; m < MT; ++m) {
+                        // words 4c .. 4c + 3 of the K-block: (even, odd) pairs
+                        const uint32_t xa = xk + static_cast<uint32_t>(m * K + 32 * c);
+                        const uint4 x0 = gemm::lds128(xa), x1 = gemm::lds128(xa + 16);
+                        const uint32_t xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            a4[m][c] = __dp4a(static_cast<int>((ww[j] << 4) & hm),
+                                              static_cast<int>(xv[2 * j]), a4[m][c]);
+                            a4[m][c] = __dp4a(static_cast<int>(ww[j] & hm),
+                                              static_cast<int>(xv[2 * j + 1]), a4[m][c]);
+                        }
+                    }
                 }
             }
         }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(empty_p(s));
     }
+    int acc[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) acc[m] = (a4[m][0] + a4[m][1]) + (a4[m][2] + a4[m][3]);
 
     // ------------------------------------------------------------ epilogue
     if (h == 1)
