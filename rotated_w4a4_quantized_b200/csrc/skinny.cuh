@@ -303,24 +303,32 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             const bool store = live && n < N;
             const float swn = store ? sw[n] : 0.0f;
             const float bn = (store && bias) ? gemm::bf16_to_f32(bias[n]) : 0.0f;
+            constexpr int JW = BN < 32 ? BN : 32;
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t v[32];
                 __syncwarp();   // tcgen05.ld is warp-collective
                 ptx::tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(c0), v);
+                // The token scales of the chunk, as independent loads issued
+                // together (one dependent load per token would serialise
+                // the epilogue on the load latency).
+                float sxv[JW];
+#pragma unroll
+                for (int j = 0; j < JW; ++j)
+                    sxv[j] = (!OUT_S32 && store && c0 + j < M) ? __ldg(sx + c0 + j) : 0.0f;
                 ptx::tmem_ld_wait();
                 if (!store) continue;
-                constexpr int JW = BN < 32 ? BN : 32;
 #pragma unroll
                 for (int j = 0; j < JW; ++j) {
                     const int m = c0 + j;
-                    if (m >= M) break;
-                    if (OUT_S32)
-                        reinterpret_cast<int32_t *>(out)[static_cast<size_t>(m) * N + n] =
-                            static_cast<int32_t>(v[j]) >> 8;
-                    else
-                        reinterpret_cast<uint16_t *>(out)[static_cast<size_t>(m) * N + n] =
-                            gemm::f32_to_bf16_rne(gemm::epi(v[j], sx[m], swn, bn));
+                    if (m < M) {
+                        if (OUT_S32)
+                            reinterpret_cast<int32_t *>(out)[static_cast<size_t>(m) * N + n] =
+                                static_cast<int32_t>(v[j]) >> 8;
+                        else
+                            reinterpret_cast<uint16_t *>(out)[static_cast<size_t>(m) * N + n] =
+                                gemm::f32_to_bf16_rne(gemm::epi(v[j], sxv[j], swn, bn));
+                    }
                 }
             }
         }
