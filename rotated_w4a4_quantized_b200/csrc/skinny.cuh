@@ -67,7 +67,8 @@ struct Cfg {
     static constexpr int OFF_BAR = OFF_PB + SP * PB;
     static constexpr int NUM_BARS = 2 * SP + 2 * SU + 1;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;     // TMEM base, abort flag
-    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;     // + slack for 1024 alignment
+    static constexpr int OFF_SX = OFF_MISC + 16;                 // token scales (fp32 x BN)
+    static constexpr int SMEM_BYTES = OFF_SX + 4 * BN + 1024;   // + slack for 1024 alignment
     static constexpr int ACC_COLS = BN < 32 ? 32 : BN;          // read 32 columns at a time
     static constexpr int A_COLS = kSKB * BK / 4;                // TMEM columns of an A stage (64)
     static constexpr int A_OFF = ACC_COLS;                      // first A-stage column
@@ -250,6 +251,10 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         ptx::grid_dependency_wait();
         const int quarter = warp & 3;                  // TMEM lanes 32 quarter ..
         const int r = quarter * 32 + lane;
+        // The token scales are staged in shared memory now, long before the
+        // epilogue needs them.
+        float *sxs = reinterpret_cast<float *>(smem + C::OFF_SX);
+        if (!OUT_S32 && r < BN) sxs[r] = r < M ? sx[r] : 0.0f;
         const bool live = r < R;
         const uint32_t rsw = static_cast<uint32_t>(r & 7);
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -297,6 +302,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         }
         // ------------------------------------------------------------ epilogue
         // lane = output column n (a weight row), accumulator columns = tokens m
+        asm volatile("bar.sync 1, 128;" ::: "memory");   // warps 6-9: sxs is written
         if (ok && ptx::mbar_wait(acc_full, 0, abort_flag)) {
             ptx::tc_fence_after();
             const int n = n0 + r;
@@ -309,13 +315,6 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 uint32_t v[32];
                 __syncwarp();   // tcgen05.ld is warp-collective
                 ptx::tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(c0), v);
-                // The token scales of the chunk, as independent loads issued
-                // together (one dependent load per token would serialise
-                // the epilogue on the load latency).
-                float sxv[JW];
-#pragma unroll
-                for (int j = 0; j < JW; ++j)
-                    sxv[j] = (!OUT_S32 && store && c0 + j < M) ? __ldg(sx + c0 + j) : 0.0f;
                 ptx::tmem_ld_wait();
                 if (!store) continue;
 #pragma unroll
@@ -327,7 +326,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                                 static_cast<int32_t>(v[j]) >> 8;
                         else
                             reinterpret_cast<uint16_t *>(out)[static_cast<size_t>(m) * N + n] =
-                                gemm::f32_to_bf16_rne(gemm::epi(v[j], sxv[j], swn, bn));
+                                gemm::f32_to_bf16_rne(gemm::epi(v[j], sxs[m], swn, bn));
                     }
                 }
             }
