@@ -183,10 +183,11 @@ def convrot_debug_gemm_s32(qx, qw, K: int, out=None, stream=None):
 
 
 # GEMM forms of convrot_debug_gemm_tiles: the token-major tile shapes and the
-# two few-token forms (M <= 128)
+# three few-token forms (M <= 128)
 TILES_AUTO, TILES_128x256, TILES_128x192, TILES_256x192_PAIR = 0, 1, 2, 3
 SKINNY_TMEM, SKINNY_SMEM = 4, 5
 TILES_256x128_PAIR = 6
+SKINNY_PAIR = 7
 
 
 def convrot_debug_gemm_tiles(qx, sx, qw, sw, bias, K: int, tiles: int, out_s32: bool = False,

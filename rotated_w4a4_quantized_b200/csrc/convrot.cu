@@ -109,6 +109,12 @@ convrot_status device_setup(int *dev_out) {
     ok &= set_smem(skinny::skinny_kernel<32, true>, skinny::Cfg<32>::SMEM_BYTES);
     ok &= set_smem(skinny::skinny_kernel<64, true>, skinny::Cfg<64>::SMEM_BYTES);
     ok &= set_smem(skinny::skinny_kernel<128, true>, skinny::Cfg<128>::SMEM_BYTES);
+    ok &= set_smem(skinny::skinny_kernel<32, false, true>, skinny::Cfg<32, true>::SMEM_BYTES);
+    ok &= set_smem(skinny::skinny_kernel<64, false, true>, skinny::Cfg<64, true>::SMEM_BYTES);
+    ok &= set_smem(skinny::skinny_kernel<128, false, true>, skinny::Cfg<128, true>::SMEM_BYTES);
+    ok &= set_smem(skinny::skinny_kernel<32, true, true>, skinny::Cfg<32, true>::SMEM_BYTES);
+    ok &= set_smem(skinny::skinny_kernel<64, true, true>, skinny::Cfg<64, true>::SMEM_BYTES);
+    ok &= set_smem(skinny::skinny_kernel<128, true, true>, skinny::Cfg<128, true>::SMEM_BYTES);
     ok &= set_smem(decode::decode_kernel<1, 64>, kPrepSmemMax);
     ok &= set_smem(decode::decode_kernel<2, 64>, kPrepSmemMax);
     ok &= set_smem(decode::decode_kernel<4, 64>, kPrepSmemMax);
@@ -275,28 +281,35 @@ convrot_status launch_gemm_cfg(int slots, const uint8_t *qA, const uint8_t *qB, 
 // widened into TMEM.  weights_ready: the weights were complete before the
 // preceding kernel on the stream (the prep kernel of the same call) started,
 // so the kernel may start streaming them before that kernel finishes.
-template <int BN, bool OUT_S32>
+template <int BN, bool OUT_S32, bool PAIR = false>
 convrot_status launch_skinny_cfg(int num_sms, const uint8_t *qx, const float *sx,
                                  const uint8_t *qw, const float *sw, const void *bias, int64_t M,
                                  int64_t N, int64_t K, void *out, bool weights_ready,
                                  cudaStream_t stream) {
+    using C = skinny::Cfg<BN, PAIR>;
     const int R = skinny::rows_per_cta(N, num_sms);
     CUtensorMap tmA, tmB;
     if (!make_map(&tmA, qw, N, K, skinny::kPKB, R, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&tmB, qx, M, K, skinny::kPKB, BN))
+        !make_map(&tmB, qx, M, K, skinny::kPKB, C::BR))
         return CONVROT_ERR_CUDA;
+    int64_t ctas = (N + R - 1) / R;
+    if (PAIR) ctas += ctas & 1;   // whole pairs (a trailing CTA past N only waits and exits)
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>((N + R - 1) / R));
+    cfg.gridDim = dim3(static_cast<unsigned>(ctas));
     cfg.blockDim = dim3(skinny::kThreads);
-    cfg.dynamicSmemBytes = skinny::Cfg<BN>::SMEM_BYTES;
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = PAIR ? 2 : 1;
     const cudaError_t e = cudaLaunchKernelEx(
-        &cfg, skinny::skinny_kernel<BN, OUT_S32>, tmA, tmB, R, weights_ready ? 1 : 0,
+        &cfg, skinny::skinny_kernel<BN, OUT_S32, PAIR>, tmA, tmB, R, weights_ready ? 1 : 0,
         static_cast<int>(K), sx, sw, static_cast<const uint16_t *>(bias), out, static_cast<int>(M),
         static_cast<int>(N));
     return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
@@ -305,7 +318,17 @@ convrot_status launch_skinny_cfg(int num_sms, const uint8_t *qx, const float *sx
 template <bool OUT_S32>
 convrot_status launch_skinny(int num_sms, const uint8_t *qx, const float *sx, const uint8_t *qw,
                              const float *sw, const void *bias, int64_t M, int64_t N, int64_t K,
-                             void *out, bool weights_ready, cudaStream_t stream) {
+                             void *out, bool weights_ready, cudaStream_t stream, bool pair = false) {
+    if (pair) {
+        if (M <= 32)
+            return launch_skinny_cfg<32, OUT_S32, true>(num_sms, qx, sx, qw, sw, bias, M, N, K, out,
+                                                        weights_ready, stream);
+        if (M <= 64)
+            return launch_skinny_cfg<64, OUT_S32, true>(num_sms, qx, sx, qw, sw, bias, M, N, K, out,
+                                                        weights_ready, stream);
+        return launch_skinny_cfg<128, OUT_S32, true>(num_sms, qx, sx, qw, sw, bias, M, N, K, out,
+                                                     weights_ready, stream);
+    }
     if (M <= 16)
         return launch_skinny_cfg<16, OUT_S32>(num_sms, qx, sx, qw, sw, bias, M, N, K, out,
                                               weights_ready, stream);
@@ -323,7 +346,7 @@ convrot_status launch_skinny(int num_sms, const uint8_t *qx, const float *sx, co
 // the two few-token forms (M <= 128).
 enum TileChoice {
     kTilesAuto = 0, kTiles128x256 = 1, kTiles128x192 = 2, kTiles256x192Pair = 3,
-    kSkinnyTmem = 4, kSkinnySmem = 5, kTiles256x128Pair = 6
+    kSkinnyTmem = 4, kSkinnySmem = 5, kTiles256x128Pair = 6, kSkinnyPair = 7
 };
 
 // Path choice: up to 128 tokens the few-token form (weights on the 128-row
@@ -338,9 +361,11 @@ convrot_status launch_gemm(const DeviceState &ds, const uint8_t *qx, const float
     if (tiles == kTilesAuto && M <= 128) tiles = kSkinnyTmem;
     if (tiles == kSkinnyTmem && M > 128) return CONVROT_ERR_SHAPE;
     if (tiles == kSkinnySmem && M > 128) return CONVROT_ERR_SHAPE;
-    if (tiles == kSkinnyTmem)
+    if (tiles == kSkinnyPair && M > 128) return CONVROT_ERR_SHAPE;
+    if (tiles == kSkinnyPair && ds.pair_clusters <= 0) return CONVROT_ERR_UNSUPPORTED;
+    if (tiles == kSkinnyTmem || tiles == kSkinnyPair)
         return launch_skinny<OUT_S32>(num_sms, qx, sx, qw, sw, bias, M, N, K, out, weights_ready,
-                                      stream);
+                                      stream, tiles == kSkinnyPair);
     if (tiles == kSkinnySmem) {
         if (M <= 16)
             return launch_gemm_cfg<16, true, OUT_S32>(num_sms, qw, qx, N, M, K, sx, sw, bias, out, M,
@@ -578,7 +603,7 @@ convrot_status convrot_debug_gemm_tiles(const uint8_t *qx, const float *sx, cons
                                         int64_t N, int64_t K, int tiles, int out_s32, void *out,
                                         convrot_stream_t stream) {
     if (M < 0 || N < 0) return CONVROT_ERR_SHAPE;
-    if (tiles < kTilesAuto || tiles > kTiles256x128Pair) return CONVROT_ERR_SHAPE;
+    if (tiles < kTilesAuto || tiles > kSkinnyPair) return CONVROT_ERR_SHAPE;
     if (M == 0 || N == 0) return CONVROT_OK;
     convrot_status st = check_gemm_args(qx, qw, M, N, K);
     if (st != CONVROT_OK) return st;

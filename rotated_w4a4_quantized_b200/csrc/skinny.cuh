@@ -51,15 +51,22 @@ constexpr int kMaxRows = 128;       // weight rows per CTA: the TMEM lanes
 constexpr int kSKB = 2;             // K-blocks per stage
 constexpr int kPKB = kSKB * BKP;    // packed bytes per row per stage (128)
 
-template <int BN>
+// PAIR: two CTAs (a cluster) share each MMA (cta_group::2, M = 256): each
+// keeps its own R weight rows in its own TMEM lanes and half of the token
+// columns in its shared memory; CTA 0 issues the MMAs for both.  Half the
+// MMA instructions per weight byte of the one-CTA form.
+template <int BN, bool PAIR = false>
 struct Cfg {
     static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128, "token tile of 16..128");
+    static_assert(!PAIR || BN >= 32, "cta_group::2 MMAs with A in TMEM need N >= 32");
+    static constexpr int CG = PAIR ? 2 : 1;           // tcgen05 CTA group
+    static constexpr int BR = PAIR ? BN / 2 : BN;     // token rows held by this CTA
     // Packed stages in flight: ~100+ KB of the weight stream per SM.
-    static constexpr int SP = BN == 16 ? 11 : BN == 32 ? 9 : BN == 64 ? 6 : 3;
-    static constexpr int SU = BN == 128 ? 3 : 4;      // TMEM A stages = widened B stages
+    static constexpr int SP = BR == 16 ? 11 : BR == 32 ? 9 : BR == 64 ? 6 : 3;
+    static constexpr int SU = (BN == 128 && !PAIR) ? 3 : 4;   // TMEM A stages = widened B stages
     static constexpr int PA = kMaxRows * kPKB;        // packed weight stage (up to 128 rows)
-    static constexpr int PB = BN * kPKB;              // packed token stage
-    static constexpr int UBH = BN * BK;               // widened token tile of one K-block
+    static constexpr int PB = BR * kPKB;              // packed token stage
+    static constexpr int UBH = BR * BK;               // widened token tile of one K-block
     static constexpr int UB = kSKB * UBH;             // widened token stage
     static constexpr int OFF_UB = 0;                  // 1024-aligned tiles first
     static constexpr int OFF_PA = OFF_UB + SU * UB;
@@ -69,6 +76,7 @@ struct Cfg {
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;     // TMEM base, abort flag
     static constexpr int OFF_SX = OFF_MISC + 16;                 // token scales (fp32 x BN)
     static constexpr int SMEM_BYTES = OFF_SX + 4 * BN + 1024;   // + slack for 1024 alignment
+    static constexpr uint32_t IDESC = ptx::idesc_i8(PAIR ? 256 : 128, BN);
     static constexpr int ACC_COLS = BN < 32 ? 32 : BN;          // read 32 columns at a time
     static constexpr int A_COLS = kSKB * BK / 4;                // TMEM columns of an A stage (64)
     static constexpr int A_OFF = ACC_COLS;                      // first A-stage column
@@ -88,17 +96,17 @@ inline int rows_per_cta(int64_t N, int num_sms) {
 }
 
 // tmA: packed weights [N][K/2], box 128 B x R rows, 128-byte swizzle.
-// tmB: packed tokens [M][K/2], box 128 B x BN rows.
+// tmB: packed tokens [M][K/2], box 128 B x Cfg::BR rows.
 // early_a: the weights were complete before the preceding kernel on the
 // stream started, so they may be loaded before waiting for it.
 // OUT_S32: write the integer accumulators (test hook) instead of bf16.
-template <int BN, bool OUT_S32>
+template <int BN, bool OUT_S32, bool PAIR = false>
 __global__ void __launch_bounds__(kThreads, 1)
 skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               int R, int early_a, int K, const float *__restrict__ sx,
               const float *__restrict__ sw, const uint16_t *__restrict__ bias,
               void *__restrict__ out, int M, int N) {
-    using C = Cfg<BN>;
+    using C = Cfg<BN, PAIR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -115,7 +123,14 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = static_cast<int>(blockIdx.x) * R;     // first weight row of this CTA
     const int num_kp = (K / 2 + kPKB - 1) / kPKB;        // stages; K tails are zero-filled
-    const uint32_t stage_tx = static_cast<uint32_t>((R + BN) * kPKB);
+    const uint32_t stage_tx = static_cast<uint32_t>((R + C::BR) * kPKB);
+    // Rank in the pair: CTA 0 issues the MMAs and holds the barrier that
+    // gathers both CTAs' widened stages; its commits reach both CTAs.
+    const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0u;
+    auto arrive_leader = [&](uint32_t bar) {
+        if (PAIR && rank != 0) ptx::mbar_arrive_remote(ptx::mapa_shared(bar, 0));
+        else ptx::mbar_arrive(bar);
+    };
 
     // Thread 0 is also the producer: it sets up the barriers and, when the
     // weights may be read early, requests the first stages of them before
@@ -130,7 +145,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             ptx::mbar_init(empty_p(s), 8);    // 4 token + 4 weight widening warps
         }
         for (int s = 0; s < C::SU; ++s) {
-            ptx::mbar_init(full_u(s), 8);
+            ptx::mbar_init(full_u(s), (PAIR ? 2 : 1) * 8);
             ptx::mbar_init(empty_u(s), 1);
         }
         ptx::mbar_init(acc_full, 1);
@@ -142,11 +157,12 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         }
     }
     if (warp == kWarpMma) {
-        ptx::tmem_alloc(sbase + C::OFF_MISC, C::TMEM_COLS);
-        ptx::tmem_relinquish();
+        ptx::tmem_alloc<C::CG>(sbase + C::OFF_MISC, C::TMEM_COLS);
+        ptx::tmem_relinquish<C::CG>();
     }
     ptx::tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) ptx::cluster_sync();   // the peer's barriers are initialised
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
@@ -163,7 +179,8 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                     ptx::mbar_arrive_expect_tx(full_p(ps), stage_tx);
                     ptx::tma_load_2d(sbase + C::OFF_PA + ps * C::PA, &tmA, full_p(ps), kp * kPKB, n0);
                 }
-                ptx::tma_load_2d(sbase + C::OFF_PB + ps * C::PB, &tmB, full_p(ps), kp * kPKB, 0);
+                ptx::tma_load_2d(sbase + C::OFF_PB + ps * C::PB, &tmB, full_p(ps), kp * kPKB,
+                                 static_cast<int>(rank) * C::BR);
                 if (++ps == C::SP) { ps = 0; ph ^= 1; }
             }
             if (!ok) {
@@ -175,28 +192,31 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             }
         }
     } else if (warp == kWarpMma) {
-        if (lane == 0) {
+        if (lane == 0 && rank == 0) {
+            auto commit_both = [&](uint32_t bar) {
+                ptx::tc_commit<C::CG>(bar);
+                if constexpr (PAIR) ptx::tc_commit<C::CG>(ptx::mapa_shared(bar, 1));
+            };
             ptx::grid_dependency_wait();
-            constexpr uint32_t idesc = ptx::idesc_i8(kMaxRows, BN);
             int us = 0;
             uint32_t ph = 0;
             for (int kp = 0; kp < num_kp; ++kp) {
-                if (!ptx::mbar_wait(full_u(us), ph, abort_flag)) break;
+                if (!ptx::mbar_wait<PAIR>(full_u(us), ph, abort_flag)) break;
                 ptx::tc_fence_after();
                 const uint32_t a0 = tmem_base + static_cast<uint32_t>(C::A_OFF + us * C::A_COLS);
                 const uint32_t b0 = sbase + C::OFF_UB + us * C::UB;
 #pragma unroll
                 for (int j = 0; j < kSKB * BK / 32; ++j)   // A stage: 8 columns per MMA
-                    ptx::mma_i8_ts(tmem_base, a0 + static_cast<uint32_t>(8 * j),
-                                   ptx::sw128_kmajor_desc(b0 + (j >> 2) * C::UBH + 32 * (j & 3)),
-                                   idesc, (kp | j) != 0 ? 1u : 0u);
-                ptx::tc_commit(empty_u(us));
+                    ptx::mma_i8_ts<C::CG>(tmem_base, a0 + static_cast<uint32_t>(8 * j),
+                                          ptx::sw128_kmajor_desc(b0 + (j >> 2) * C::UBH + 32 * (j & 3)),
+                                          C::IDESC, (kp | j) != 0 ? 1u : 0u);
+                commit_both(empty_u(us));
                 if (++us == C::SU) { us = 0; ph ^= 1; }
             }
             // Also the drain: TMEM is released only after every MMA completed.
-            ptx::tc_commit(acc_full);
+            commit_both(acc_full);
             volatile int never = 0;
-            ptx::mbar_wait(acc_full, 0, &never, 100000000ull);
+            ptx::mbar_wait<PAIR>(acc_full, 0, &never, 100000000ull);
         }
     } else if (warp < kWarpA0) {
         // ------------------------------------------------------ token widening
@@ -206,7 +226,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         // phase is fixed.
         ptx::grid_dependency_wait();
         const int bt = static_cast<int>(threadIdx.x) - kWarpB0 * 32;
-        constexpr int kPerB = BN / 16;
+        constexpr int kPerB = C::BR / 16;
         const uint32_t c8 = static_cast<uint32_t>(bt & 7);
         const uint32_t h = c8 >> 2, c = c8 & 3;
         const int row0 = bt >> 3;
@@ -218,7 +238,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             const int ps = kp % C::SP, us = kp % C::SU;
             const uint32_t pph = (kp / C::SP) & 1, uph = (kp / C::SU) & 1;
             if (!ptx::mbar_wait(full_p(ps), pph, abort_flag)) break;
-            if (!ptx::mbar_wait(empty_u(us), uph ^ 1, abort_flag)) break;
+            if (!ptx::mbar_wait<PAIR>(empty_u(us), uph ^ 1, abort_flag)) break;
             const uint32_t pb = sbase + C::OFF_PB + ps * C::PB + row0 * kPKB + c8 * 16;
             const uint32_t ub = sbase + C::OFF_UB + us * C::UB + h * C::UBH + row0 * 128;
             uint4 w[kPerB];
@@ -235,7 +255,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             __syncwarp();
             if (lane == 0) {
                 ptx::mbar_arrive(empty_p(ps));
-                ptx::mbar_arrive(full_u(us));
+                arrive_leader(full_u(us));
             }
         }
     } else {
@@ -264,7 +284,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             const int ps = kp % C::SP, us = kp % C::SU;
             const uint32_t pph = (kp / C::SP) & 1, uph = (kp / C::SU) & 1;
             if (!ptx::mbar_wait(full_p(ps), pph, abort_flag)) { ok = false; break; }
-            if (!ptx::mbar_wait(empty_u(us), uph ^ 1, abort_flag)) { ok = false; break; }
+            if (!ptx::mbar_wait<PAIR>(empty_u(us), uph ^ 1, abort_flag)) { ok = false; break; }
             ptx::tc_fence_after();
             const uint32_t src = sbase + C::OFF_PA + ps * C::PA + r * kPKB;
 #pragma unroll
@@ -297,13 +317,13 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             __syncwarp();
             if (lane == 0) {
                 ptx::mbar_arrive(empty_p(ps));
-                ptx::mbar_arrive(full_u(us));
+                arrive_leader(full_u(us));
             }
         }
         // ------------------------------------------------------------ epilogue
         // lane = output column n (a weight row), accumulator columns = tokens m
         asm volatile("bar.sync 1, 128;" ::: "memory");   // warps 6-9: sxs is written
-        if (ok && ptx::mbar_wait(acc_full, 0, abort_flag)) {
+        if (ok && ptx::mbar_wait<PAIR>(acc_full, 0, abort_flag)) {
             ptx::tc_fence_after();
             const int n = n0 + r;
             const bool store = live && n < N;
@@ -335,10 +355,11 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
 
     ptx::tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) ptx::cluster_sync();   // the peer's MMAs and arrivals are done
     ptx::tc_fence_after();
     if (warp == kWarpMma) {
         __syncwarp();
-        ptx::tmem_dealloc(tmem_base, C::TMEM_COLS);
+        ptx::tmem_dealloc<C::CG>(tmem_base, C::TMEM_COLS);
     }
 }
 

@@ -83,8 +83,8 @@ def test_host_validation_without_device(L):
     assert L.convrot_debug_gemm_s32(A, B, 4, 8, 96, B, s) == 3
     assert L.convrot_debug_gemm_s32(A, B, 4, 8, 128, U, s) == 4
     assert L.convrot_debug_rotate_f32(A, 4, 512, 256, None, s) == 1
-    # forced tile shapes: only 0..3, and the same argument checks
-    assert L.convrot_debug_gemm_tiles(A, B, A, B, None, 4, 8, 128, 7, 0, B, s) == 3
+    # forced tile shapes: only 0..7, and the same argument checks
+    assert L.convrot_debug_gemm_tiles(A, B, A, B, None, 4, 8, 128, 8, 0, B, s) == 3
     assert L.convrot_debug_gemm_tiles(A, B, A, B, None, 4, 8, 128, -1, 1, B, s) == 3
     assert L.convrot_debug_gemm_tiles(A, B, A, B, None, 4, 8, 96, 2, 1, B, s) == 3
     assert L.convrot_debug_gemm_tiles(A, None, A, B, None, 4, 8, 128, 2, 0, B, s) == 1

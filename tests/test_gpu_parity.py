@@ -131,10 +131,11 @@ def test_gemm_tiles_s32_bit_exact(tiles, M, N, K):
     assert np.array_equal(acc.cpu().numpy().astype(np.int64), O.gemm(pa, pb, K))
 
 
-# The two few-token forms (M <= 128): token tiles of 16 .. 128 with ragged
-# token counts, weight-row slices with a ragged last slice, K tails.
-SKINNY_FORMS = [cr.SKINNY_TMEM, cr.SKINNY_SMEM]
-SKINNY_IDS = ["tmem", "smem"]
+# The three few-token forms (M <= 128): token tiles of 16 .. 128 with ragged
+# token counts, weight-row slices with a ragged last slice (and, on CTA
+# pairs, a last pair with one slice past N), K tails.
+SKINNY_FORMS = [cr.SKINNY_TMEM, cr.SKINNY_SMEM, cr.SKINNY_PAIR]
+SKINNY_IDS = ["tmem", "smem", "pair"]
 SKINNY_CASES = [(1, 16, 64), (1, 14336, 4096), (5, 300, 1088), (16, 1000, 512), (17, 257, 192),
                 (33, 4000, 3072), (64, 1024, 1024), (100, 777, 2048), (128, 14336, 256)]
 
@@ -214,7 +215,7 @@ def test_epilogue_rounds_product_before_bias(M, N):
     t = lambda v: _dev(torch.from_numpy(v))
     bt = t(bias.view(np.int16)).view(torch.bfloat16)
     forms = [cr.TILES_AUTO] + (TILE_SHAPES + [cr.SKINNY_SMEM] if M <= 128 else TILE_SHAPES)
-    for form in forms + ([cr.SKINNY_TMEM] if M <= 128 else []):
+    for form in forms + ([cr.SKINNY_TMEM, cr.SKINNY_PAIR] if M <= 128 else []):
         y = cr.convrot_debug_gemm_tiles(t(pa), t(sx), t(pb), t(sw), bt, K, form)
         torch.cuda.synchronize()
         assert np.array_equal(gc.to_np_u16(y), y_ref), form
