@@ -143,14 +143,12 @@ int convrot_linear_single_kernel(int64_t M, int64_t K, int group);
  *           2  128 x 192 tiles, A widened into TMEM;
  *           3  256 x 192 tiles on CTA pairs (cta_group::2);
  *           4  few-token form (M <= 128): weights widened into TMEM, one
- *              CTA per slice of weight rows (the automatic choice up to 64
- *              tokens);
+ *              CTA per slice of weight rows (the automatic choice there);
  *           5  few-token form with both operands widened in shared memory;
  *           6  256 x 128 tiles on CTA pairs (four TMEM A stages);
  *           7  few-token form on CTA pairs (M <= 128): each CTA widens its
  *              slice of weight rows into its TMEM and holds half of the
- *              token columns; one cta_group::2 MMA covers both slices (the
- *              automatic choice for 65 to 128 tokens).
+ *              token columns; one cta_group::2 MMA covers both slices.
  * Returns CONVROT_ERR_SHAPE for any other value or for 4 / 5 / 7 with
  * M > 128, and CONVROT_ERR_UNSUPPORTED when the device cannot co-schedule
  * CTA pairs (tiles = 3, 6, 7).

@@ -358,11 +358,10 @@ convrot_status launch_gemm(const DeviceState &ds, const uint8_t *qx, const float
                            int64_t N, int64_t K, void *out, cudaStream_t stream,
                            int tiles = kTilesAuto, bool weights_ready = false) {
     const int num_sms = ds.num_sms;
-    // Few tokens: the weight-streaming forms.  Above 64 tokens (128-column
-    // token tiles) the CTA-pair form is faster (its smaller per-CTA token
-    // share leaves room for twice the packed stages, and half the MMAs).
-    if (tiles == kTilesAuto && M <= 128)
-        tiles = (M > 64 && ds.pair_clusters > 0) ? kSkinnyPair : kSkinnyTmem;
+    // Few tokens: the weight-streaming form.  (The CTA-pair form measured
+    // the same at 128 tokens and slower below: each SM's tensor core does
+    // the same work per weight byte either way.)
+    if (tiles == kTilesAuto && M <= 128) tiles = kSkinnyTmem;
     if (tiles == kSkinnyTmem && M > 128) return CONVROT_ERR_SHAPE;
     if (tiles == kSkinnySmem && M > 128) return CONVROT_ERR_SHAPE;
     if (tiles == kSkinnyPair && M > 128) return CONVROT_ERR_SHAPE;

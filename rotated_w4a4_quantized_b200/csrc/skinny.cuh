@@ -29,8 +29,11 @@
 // gemm.cuh (the epilogue shifts the accumulator right by 8).
 //
 // CTA organisation (one CTA per SM, one tile):
-//   warp 0      TMA producer (one thread): packed weight tile [R x 128 B]
-//               (128-byte swizzle) and packed token tile [BN x 128 B];
+//   warp 0      weight TMA producer (one thread): packed weight tiles
+//               [R x 128 B] (128-byte swizzle), in a ring as deep as shared
+//               memory allows;
+//   warp 10     token TMA producer (one thread): packed token tiles
+//               [BN x 128 B], a ring of three (they come from L2);
 //   warp 1      TMEM allocator and MMA issuer (one thread): 8 MMAs of K = 32
 //               per stage, A from TMEM, B from shared memory;
 //   warps 2..5  token widening into the swizzled B stages;
@@ -45,8 +48,8 @@ namespace skinny {
 
 using gemm::BK;
 using gemm::BKP;
-constexpr int kWarpTma = 0, kWarpMma = 1, kWarpB0 = 2, kWarpA0 = 6;
-constexpr int kThreads = 10 * 32;
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpB0 = 2, kWarpA0 = 6, kWarpTmaB = 10;
+constexpr int kThreads = 11 * 32;
 constexpr int kMaxRows = 128;       // weight rows per CTA: the TMEM lanes
 constexpr int kSKB = 2;             // K-blocks per stage
 constexpr int kPKB = kSKB * BKP;    // packed bytes per row per stage (128)
@@ -61,18 +64,23 @@ struct Cfg {
     static_assert(!PAIR || BN >= 32, "cta_group::2 MMAs with A in TMEM need N >= 32");
     static constexpr int CG = PAIR ? 2 : 1;           // tcgen05 CTA group
     static constexpr int BR = PAIR ? BN / 2 : BN;     // token rows held by this CTA
-    // Packed stages in flight: ~100+ KB of the weight stream per SM.
-    static constexpr int SP = BR == 16 ? 11 : BR == 32 ? 9 : BR == 64 ? 6 : 3;
     static constexpr int SU = (BN == 128 && !PAIR) ? 3 : 4;   // TMEM A stages = widened B stages
     static constexpr int PA = kMaxRows * kPKB;        // packed weight stage (up to 128 rows)
     static constexpr int PB = BR * kPKB;              // packed token stage
+    // Tokens and weights have rings of their own: the tokens come from L2
+    // and need few stages in flight, the weight stream from HBM as many as
+    // the rest of shared memory holds (up to 12: ~160 KB in flight per SM).
+    static constexpr int SB = 3;
+    static constexpr int SP_FIT = (232448 - (SU * kSKB * BR * BK + SB * PB + 4096)) / PA;
+    static constexpr int SP = SP_FIT > 12 ? 12 : SP_FIT;
+    static_assert(SP >= 3, "at least three weight stages in flight");
     static constexpr int UBH = BR * BK;               // widened token tile of one K-block
     static constexpr int UB = kSKB * UBH;             // widened token stage
     static constexpr int OFF_UB = 0;                  // 1024-aligned tiles first
     static constexpr int OFF_PA = OFF_UB + SU * UB;
     static constexpr int OFF_PB = OFF_PA + SP * PA;
-    static constexpr int OFF_BAR = OFF_PB + SP * PB;
-    static constexpr int NUM_BARS = 2 * SP + 2 * SU + 1;
+    static constexpr int OFF_BAR = OFF_PB + SB * PB;
+    static constexpr int NUM_BARS = 2 * SP + 2 * SB + 2 * SU + 1;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;     // TMEM base, abort flag
     static constexpr int OFF_SX = OFF_MISC + 16;                 // token scales (fp32 x BN)
     static constexpr int SMEM_BYTES = OFF_SX + 4 * BN + 1024;   // + slack for 1024 alignment
@@ -112,18 +120,22 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = ptx::smem_u32(smem);
     const uint32_t bar0 = sbase + C::OFF_BAR;
-    auto full_p = [&](int s) { return bar0 + 8u * s; };
-    auto empty_p = [&](int s) { return bar0 + 8u * (C::SP + s); };
-    auto full_u = [&](int s) { return bar0 + 8u * (2 * C::SP + s); };
-    auto empty_u = [&](int s) { return bar0 + 8u * (2 * C::SP + C::SU + s); };
-    const uint32_t acc_full = bar0 + 8u * (2 * C::SP + 2 * C::SU);
+    auto full_a = [&](int s) { return bar0 + 8u * s; };                 // weight stages
+    auto empty_a = [&](int s) { return bar0 + 8u * (C::SP + s); };
+    auto full_b = [&](int s) { return bar0 + 8u * (2 * C::SP + s); };   // token stages
+    auto empty_b = [&](int s) { return bar0 + 8u * (2 * C::SP + C::SB + s); };
+    const uint32_t bar_u = bar0 + 8u * (2 * C::SP + 2 * C::SB);
+    auto full_u = [&](int s) { return bar_u + 8u * s; };                // TMEM A / widened B
+    auto empty_u = [&](int s) { return bar_u + 8u * (C::SU + s); };
+    const uint32_t acc_full = bar_u + 8u * (2 * C::SU);
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = static_cast<int>(blockIdx.x) * R;     // first weight row of this CTA
     const int num_kp = (K / 2 + kPKB - 1) / kPKB;        // stages; K tails are zero-filled
-    const uint32_t stage_tx = static_cast<uint32_t>((R + C::BR) * kPKB);
+    const uint32_t a_tx = static_cast<uint32_t>(R * kPKB);        // bytes of a weight stage
+    const uint32_t b_tx = static_cast<uint32_t>(C::BR * kPKB);    // bytes of a token stage
     // Rank in the pair: CTA 0 issues the MMAs and holds the barrier that
     // gathers both CTAs' widened stages; its commits reach both CTAs.
     const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0u;
@@ -132,17 +144,21 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         else ptx::mbar_arrive(bar);
     };
 
-    // Thread 0 is also the producer: it sets up the barriers and, when the
-    // weights may be read early, requests the first stages of them before
-    // the rest of the set-up (TMEM allocation, the CTA barrier), so the
-    // weight stream starts as early as the CTA does.
+    // Thread 0 is also the weight producer: it sets up the barriers and,
+    // when the weights may be read early, requests the first stages of them
+    // before the rest of the set-up (TMEM allocation, the CTA barrier), so
+    // the weight stream starts as early as the CTA does.
     const int early = early_a ? (num_kp < C::SP ? num_kp : C::SP) : 0;
     if (threadIdx.x == 0) {
         ptx::tma_prefetch_desc(&tmA);
         ptx::tma_prefetch_desc(&tmB);
         for (int s = 0; s < C::SP; ++s) {
-            ptx::mbar_init(full_p(s), 1);
-            ptx::mbar_init(empty_p(s), 8);    // 4 token + 4 weight widening warps
+            ptx::mbar_init(full_a(s), 1);
+            ptx::mbar_init(empty_a(s), 4);    // the 4 weight widening warps
+        }
+        for (int s = 0; s < C::SB; ++s) {
+            ptx::mbar_init(full_b(s), 1);
+            ptx::mbar_init(empty_b(s), 4);    // the 4 token widening warps
         }
         for (int s = 0; s < C::SU; ++s) {
             ptx::mbar_init(full_u(s), (PAIR ? 2 : 1) * 8);
@@ -152,8 +168,8 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         *abort_flag = 0;
         ptx::fence_mbar_init();
         for (int kp = 0; kp < early; ++kp) {
-            ptx::mbar_arrive_expect_tx(full_p(kp), stage_tx);
-            ptx::tma_load_2d(sbase + C::OFF_PA + kp * C::PA, &tmA, full_p(kp), kp * kPKB, n0);
+            ptx::mbar_arrive_expect_tx(full_a(kp), a_tx);
+            ptx::tma_load_2d(sbase + C::OFF_PA + kp * C::PA, &tmA, full_a(kp), kp * kPKB, n0);
         }
     }
     if (warp == kWarpMma) {
@@ -166,30 +182,43 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
+    // Let a producer's copies already in flight land before the CTA exits:
+    // `issued` stages went into a ring of S slots.
+    auto drain = [&](auto full, int issued, int S) {
+        const int ps = issued % S;
+        const uint32_t ph = static_cast<uint32_t>(issued / S) & 1u;
+        for (int s = 0; s < S; ++s) {
+            volatile int never = 0;
+            ptx::mbar_wait(full(s), ph ^ (s < ps ? 0u : 1u), &never, 10000000ull);
+        }
+    };
+
     // The producer and MMA loops run in one thread each.
     if (warp == kWarpTma) {
         if (lane == 0) {
+            // Weights that may come from the preceding kernel wait for it.
+            if (!early_a) ptx::grid_dependency_wait();
+            int kp = early;
+            for (; kp < num_kp; ++kp) {
+                const int s = kp % C::SP;
+                if (!ptx::mbar_wait(empty_a(s), ((kp / C::SP) & 1) ^ 1, abort_flag)) break;
+                ptx::mbar_arrive_expect_tx(full_a(s), a_tx);
+                ptx::tma_load_2d(sbase + C::OFF_PA + s * C::PA, &tmA, full_a(s), kp * kPKB, n0);
+            }
+            if (kp < num_kp) drain(full_a, kp, C::SP);
+        }
+    } else if (warp == kWarpTmaB) {
+        if (lane == 0) {
             ptx::grid_dependency_wait();   // the tokens come from the preceding kernel
-            int ps = 0;
-            uint32_t ph = 0;
-            bool ok = true;
-            for (int kp = 0; kp < num_kp; ++kp) {
-                if (kp >= early) {
-                    if (!ptx::mbar_wait(empty_p(ps), ph ^ 1, abort_flag)) { ok = false; break; }
-                    ptx::mbar_arrive_expect_tx(full_p(ps), stage_tx);
-                    ptx::tma_load_2d(sbase + C::OFF_PA + ps * C::PA, &tmA, full_p(ps), kp * kPKB, n0);
-                }
-                ptx::tma_load_2d(sbase + C::OFF_PB + ps * C::PB, &tmB, full_p(ps), kp * kPKB,
+            int kp = 0;
+            for (; kp < num_kp; ++kp) {
+                const int s = kp % C::SB;
+                if (!ptx::mbar_wait(empty_b(s), ((kp / C::SB) & 1) ^ 1, abort_flag)) break;
+                ptx::mbar_arrive_expect_tx(full_b(s), b_tx);
+                ptx::tma_load_2d(sbase + C::OFF_PB + s * C::PB, &tmB, full_b(s), kp * kPKB,
                                  static_cast<int>(rank) * C::BR);
-                if (++ps == C::SP) { ps = 0; ph ^= 1; }
             }
-            if (!ok) {
-                // Let copies already in flight land before the CTA exits.
-                for (int s = 0; s < C::SP; ++s) {
-                    volatile int never = 0;
-                    ptx::mbar_wait(full_p(s), ph ^ (s < ps ? 0u : 1u), &never, 10000000ull);
-                }
-            }
+            if (kp < num_kp) drain(full_b, kp, C::SB);
         }
     } else if (warp == kWarpMma) {
         if (lane == 0 && rank == 0) {
@@ -235,9 +264,9 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         const uint32_t hi_off = ((2u * c + 1u) ^ sw8) << 4;
         const uint32_t hm = 0xF0F0F0F0u;
         for (int kp = 0; kp < num_kp; ++kp) {
-            const int ps = kp % C::SP, us = kp % C::SU;
-            const uint32_t pph = (kp / C::SP) & 1, uph = (kp / C::SU) & 1;
-            if (!ptx::mbar_wait(full_p(ps), pph, abort_flag)) break;
+            const int ps = kp % C::SB, us = kp % C::SU;
+            const uint32_t pph = (kp / C::SB) & 1, uph = (kp / C::SU) & 1;
+            if (!ptx::mbar_wait(full_b(ps), pph, abort_flag)) break;
             if (!ptx::mbar_wait<PAIR>(empty_u(us), uph ^ 1, abort_flag)) break;
             const uint32_t pb = sbase + C::OFF_PB + ps * C::PB + row0 * kPKB + c8 * 16;
             const uint32_t ub = sbase + C::OFF_UB + us * C::UB + h * C::UBH + row0 * 128;
@@ -254,7 +283,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             ptx::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                ptx::mbar_arrive(empty_p(ps));
+                ptx::mbar_arrive(empty_b(ps));
                 arrive_leader(full_u(us));
             }
         }
@@ -283,7 +312,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         for (int kp = 0; kp < num_kp; ++kp) {
             const int ps = kp % C::SP, us = kp % C::SU;
             const uint32_t pph = (kp / C::SP) & 1, uph = (kp / C::SU) & 1;
-            if (!ptx::mbar_wait(full_p(ps), pph, abort_flag)) { ok = false; break; }
+            if (!ptx::mbar_wait(full_a(ps), pph, abort_flag)) { ok = false; break; }
             if (!ptx::mbar_wait<PAIR>(empty_u(us), uph ^ 1, abort_flag)) { ok = false; break; }
             ptx::tc_fence_after();
             const uint32_t src = sbase + C::OFF_PA + ps * C::PA + r * kPKB;
@@ -316,7 +345,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                ptx::mbar_arrive(empty_p(ps));
+                ptx::mbar_arrive(empty_a(ps));
                 arrive_leader(full_u(us));
             }
         }
