@@ -187,6 +187,21 @@ __device__ __forceinline__ uint32_t epi_pair(uint32_t r0, uint32_t r1, float sx,
     return *reinterpret_cast<const uint32_t *>(&h);
 }
 
+// The same arithmetic for two tokens of one output column (the few-token
+// forms, where accumulator columns are tokens): their own token scales,
+// the column's weight scale and bias.
+__device__ __forceinline__ uint32_t epi_pair_tok(uint32_t r0, uint32_t r1, float sx0, float sx1,
+                                                 float sw, float b) {
+    float f0 = __int_as_float((static_cast<int>(r0) >> 8) + 0x4B400000);
+    float f1 = __int_as_float((static_cast<int>(r1) >> 8) + 0x4B400000);
+    ptx::add2(f0, f1, f0, f1, -12582912.0f, -12582912.0f);
+    ptx::mul2(f0, f1, f0, f1, sx0, sx1);
+    f0 = __fadd_rn(__fmul_rn(f0, sw), b);
+    f1 = __fadd_rn(__fmul_rn(f1, sw), b);
+    const __nv_bfloat162 h = __floats2bfloat162_rn(f0, f1);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
 // OUT_S32: write the integer accumulators (test hook) instead of bf16.
 // tmY (used when !SWAP && !OUT_S32 && use_tma_store): bf16 y [M][N], box
 // 32 x 32, 64-byte swizzle.

@@ -366,16 +366,29 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 ptx::tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(c0), v);
                 ptx::tmem_ld_wait();
                 if (!store) continue;
+                if (OUT_S32) {
 #pragma unroll
-                for (int j = 0; j < JW; ++j) {
-                    const int m = c0 + j;
-                    if (m < M) {
-                        if (OUT_S32)
+                    for (int j = 0; j < JW; ++j) {
+                        const int m = c0 + j;
+                        if (m < M)
                             reinterpret_cast<int32_t *>(out)[static_cast<size_t>(m) * N + n] =
                                 static_cast<int32_t>(v[j]) >> 8;
-                        else
-                            reinterpret_cast<uint16_t *>(out)[static_cast<size_t>(m) * N + n] =
-                                gemm::f32_to_bf16_rne(gemm::epi(v[j], sxs[m], swn, bn));
+                    }
+                } else {
+                    // Two tokens at a time with the packed arithmetic (and no
+                    // int-to-float conversions: the conversion unit's rate,
+                    // not the stores, bounded this loop).
+                    uint16_t *y = reinterpret_cast<uint16_t *>(out);
+#pragma unroll
+                    for (int j = 0; j < JW; j += 2) {
+                        const int m = c0 + j;
+                        if (m < M) {
+                            const uint32_t pr =
+                                gemm::epi_pair_tok(v[j], v[j + 1], sxs[m], sxs[m + 1], swn, bn);
+                            y[static_cast<size_t>(m) * N + n] = static_cast<uint16_t>(pr);
+                            if (m + 1 < M)
+                                y[static_cast<size_t>(m + 1) * N + n] = static_cast<uint16_t>(pr >> 16);
+                        }
                     }
                 }
             }
