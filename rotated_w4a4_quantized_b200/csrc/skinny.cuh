@@ -308,12 +308,11 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         const uint32_t rsw = static_cast<uint32_t>(r & 7);
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
         const uint32_t hm = 0xF0F0F0F0u;
-        bool ok = true;
         for (int kp = 0; kp < num_kp; ++kp) {
             const int ps = kp % C::SP, us = kp % C::SU;
             const uint32_t pph = (kp / C::SP) & 1, uph = (kp / C::SU) & 1;
-            if (!ptx::mbar_wait(full_a(ps), pph, abort_flag)) { ok = false; break; }
-            if (!ptx::mbar_wait<PAIR>(empty_u(us), uph ^ 1, abort_flag)) { ok = false; break; }
+            if (!ptx::mbar_wait(full_a(ps), pph, abort_flag)) break;
+            if (!ptx::mbar_wait<PAIR>(empty_u(us), uph ^ 1, abort_flag)) break;
             ptx::tc_fence_after();
             const uint32_t src = sbase + C::OFF_PA + ps * C::PA + r * kPKB;
 #pragma unroll
@@ -349,18 +348,32 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 arrive_leader(full_u(us));
             }
         }
-        // ------------------------------------------------------------ epilogue
-        // lane = output column n (a weight row), accumulator columns = tokens m
-        asm volatile("bar.sync 1, 128;" ::: "memory");   // warps 6-9: sxs is written
-        if (ok && ptx::mbar_wait<PAIR>(acc_full, 0, abort_flag)) {
+    }
+
+    // ---------------------------------------------------------------- epilogue
+    // Warps 2-9, two per TMEM lane quarter: lane = output column n (a weight
+    // row), accumulator columns = tokens m.  With 64 or more token columns
+    // the weight warps take the even 32-column chunks and the token warps
+    // the odd ones.
+    if (warp >= kWarpB0 && warp < kWarpTmaB) {
+        asm volatile("bar.sync 1, 256;" ::: "memory");   // sxs is written, both loops are done
+        const bool wgrp = warp >= kWarpA0;
+        constexpr int kStep = BN >= 64 ? 64 : 32;
+        const int cbeg = (BN >= 64 && !wgrp) ? 32 : 0;
+        const bool active = BN >= 64 || wgrp;
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+        const float *sxs = reinterpret_cast<const float *>(smem + C::OFF_SX);
+        if (active && !*abort_flag && ptx::mbar_wait<PAIR>(acc_full, 0, abort_flag)) {
             ptx::tc_fence_after();
             const int n = n0 + r;
-            const bool store = live && n < N;
-            const float swn = store ? sw[n] : 0.0f;
-            const float bn = (store && bias) ? gemm::bf16_to_f32(bias[n]) : 0.0f;
+            const bool store = r < R && n < N;
+            const float swn = (!OUT_S32 && store) ? sw[n] : 0.0f;
+            const float bn = (!OUT_S32 && store && bias) ? gemm::bf16_to_f32(bias[n]) : 0.0f;
             constexpr int JW = BN < 32 ? BN : 32;
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
+            for (int c0 = cbeg; c0 < BN; c0 += kStep) {
                 uint32_t v[32];
                 __syncwarp();   // tcgen05.ld is warp-collective
                 ptx::tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(c0), v);
