@@ -385,15 +385,21 @@ convrot_status launch_gemm(const DeviceState &ds, const uint8_t *qx, const float
     if (tiles == kTilesAuto) {
         // Measured on layers of 1024-8192 tokens and K 3072-12288: the
         // 256 x 192 pair beats both single-CTA shapes everywhere (each SM
-        // widens half of B and the tensor core reads A from TMEM), and the
-        // 256 x 128 pair (four TMEM A stages instead of two) was within a few
-        // per cent either way, so the pair runs 256 x 192.  Without CTA
+        // widens half of B and the tensor core reads A from TMEM).  Without CTA
         // pairs the cost is wave-weighted (a tile count just above a multiple
         // of the SMs wastes a wave): one 256-code stage of a wave takes ~1880
         // cycles on 128 x 256 tiles (both operands widened in shared memory)
         // and ~1340 on 128 x 192 (A in TMEM).
         if (ds.pair_clusters > 0) {
-            tiles = kTiles256x192Pair;
+            // A 256 x 128 pair tile takes ~0.9 of a 256 x 192 one's time
+            // (measured on 1024-8192 tokens), so the narrower tile wins only
+            // where the 192-wide grid wastes most of a last wave: e.g. 96
+            // tiles on 74 pairs (1536 x 3072) against 144.
+            const auto waves = [](int64_t t, int64_t slots) { return (t + slots - 1) / slots; };
+            const int64_t ta = (M + 255) / 256;
+            const int64_t c192 = waves(ta * ((N + 191) / 192), ds.pair_clusters) * 10;
+            const int64_t c128 = waves(ta * ((N + 127) / 128), ds.pair_clusters) * 9;
+            tiles = c128 < c192 ? kTiles256x128Pair : kTiles256x192Pair;
         } else {
             const auto waves = [](int64_t t, int64_t slots) { return (t + slots - 1) / slots; };
             const int64_t c_ss = waves(((M + 127) / 128) * ((N + 255) / 256), num_sms) * 1880;
