@@ -125,11 +125,13 @@ convrot_status convrot_debug_gemm_s32(const uint8_t *qx, const uint8_t *qw, int6
 
 /*
  * Whether convrot_linear runs a layer of this shape as one kernel: 1 when
- * 1 <= M <= 4, K is a multiple of 2048 and the few token rows can be
+ * 1 <= M <= 4, K is a multiple of 2048 up to 16384 and the few token rows'
+ * buffers fit in shared memory beside the weight ring, so the rows are
  * prepared inside the GEMM kernel (activation preparation fused into a
- * CUDA-core GEMV; the workspace is then not touched), 0 when it runs the
- * prep kernel and the GEMM.  Host-only, no device work; invalid arguments
- * give 0.  Both forms give bit-identical results.
+ * CUDA-core GEMV; the workspace is then not touched); 0 when it runs the
+ * prep kernel and the GEMM.  Depends on (M, K, group) only.  Host-only, no
+ * device work; invalid arguments give 0.  Both forms give bit-identical
+ * results.
  */
 int convrot_linear_single_kernel(int64_t M, int64_t K, int group);
 

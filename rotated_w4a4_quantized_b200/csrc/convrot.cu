@@ -433,7 +433,7 @@ convrot_status launch_gemm(const DeviceState &ds, const uint8_t *qx, const float
 int decode_stages(int64_t M, int64_t K, int group, int R = decode::kRows) {
     if (M < 1 || M > 4 || K % 2048 != 0) return 0;
     const int MT = M <= 1 ? 1 : M <= 2 ? 2 : 4;
-    if (MT * (K / prep::kElemsPerThread) > decode::kConsumerWarps * 32) return 0;
+    if (K / prep::kElemsPerThread > decode::kConsumerWarps * 32) return 0;   // K <= 16384
     // Three slots of 512 bytes per row (~160 KB per SM in flight) stream as
     // fast as the whole slice at once and leave room for long rows.
     const int num_kp = static_cast<int>(K / (2 * decode::kPKB * decode::kBlocks));
@@ -564,10 +564,14 @@ convrot_status convrot_linear(const void *x_bf16, const uint8_t *qw, const float
     if ((st = check_gemm_args(qw, qw, M, N, K)) != CONVROT_OK) return st;
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
-    // 1..4 tokens: one kernel (the workspace is not touched)
-    if (const int sp = decode_stages(M, K, group, skinny::rows_per_cta(N, g_dev[dev].num_sms)))
-        return launch_decode(g_dev[dev].num_sms, sp, x_bf16, qw, sw, bias_bf16, M, N, K, group,
-                             y_bf16, stream);
+    // 1..4 tokens: one kernel (the workspace is not touched).  Eligibility
+    // is decided for the largest slice (128 rows), so that it depends on
+    // (M, K, group) alone, as convrot_linear_single_kernel reports it; the
+    // ring then takes what the actual slice leaves.
+    if (decode_stages(M, K, group) > 0)
+        if (const int sp = decode_stages(M, K, group, skinny::rows_per_cta(N, g_dev[dev].num_sms)))
+            return launch_decode(g_dev[dev].num_sms, sp, x_bf16, qw, sw, bias_bf16, M, N, K,
+                                 group, y_bf16, stream);
     uint8_t *qx = static_cast<uint8_t *>(workspace);
     float *sx = reinterpret_cast<float *>(qx + round256(static_cast<size_t>(M) * (K / 2)));
     if ((st = launch_prep(g_dev[dev].num_sms, x_bf16, M, K, group, qx, sx, nullptr, stream)) != CONVROT_OK)

@@ -36,9 +36,10 @@
 //     instruction per weight byte per token;
 //   * the two K halves of each row are added and the epilogue (the GEMM's,
 //     same arithmetic) writes y.
-// Eligible shapes: M <= 4, K a multiple of 2048 and MT * K / 64 <= 256 (one
-// round of token preparation by the 256 threads); others take the two-kernel
-// path.
+// Eligible shapes: M <= 4, K a multiple of 2048 up to 16384 (at most 256
+// threads per token row; rows beyond what 256 threads hold at once are
+// prepared in further rounds), and the rows' buffers fit in shared memory
+// beside two ring slots; others take the two-kernel path.
 #pragma once
 
 #include "gemm.cuh"
@@ -103,19 +104,22 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t *__restric
     const uint32_t hm = 0xF0F0F0F0u;
 
     // The token rows are requested first, ahead of the weight burst, so that
-    // their preparation is not queued behind it.
+    // their preparation is not queued behind it.  Token m is prepared by the
+    // K/64 threads of slot m mod tpr, in round m / tpr.
     const int gt = K / prep::kElemsPerThread;            // threads per token (multiple of 32)
-    const int tok = threadIdx.x / gt, t = threadIdx.x % gt;
-    uint4 *stg = reinterpret_cast<uint4 *>(prep_area + tok * prep_per_tok);
-    if (warp < kWarpTma && tok < M) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(tok) * K);
-        const uint32_t stg_s = ptx::smem_u32(stg);
+    const int tpr = (kConsumerWarps * 32) / gt;          // tokens per round (K <= 16384)
+    const int slot_tok = threadIdx.x / gt, t = threadIdx.x % gt;
+    if (warp < kWarpTma && slot_tok < tpr) {
+        for (int tok = slot_tok; tok < M; tok += tpr) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(tok) * K);
+            const uint32_t stg_s = ptx::smem_u32(prep_area + tok * prep_per_tok);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int g = t + j * gt;                    // chunk index in the row
-            const int owner = g >> 3, c = g & 7;
-            prep::cp_async16(stg_s + static_cast<uint32_t>((owner * 8 + (c ^ (owner & 7))) * 16),
-                             src + g);
+            for (int j = 0; j < 8; ++j) {
+                const int g = t + j * gt;                // chunk index in the row
+                const int owner = g >> 3, c = g & 7;
+                prep::cp_async16(stg_s + static_cast<uint32_t>((owner * 8 + (c ^ (owner & 7))) * 16),
+                                 src + g);
+            }
         }
         prep::cp_async_commit();
     }
@@ -153,18 +157,22 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t *__restric
     }
 
     // ------------------------------------------------------ token preparation
-    {
+    for (int tok0 = 0; tok0 < MT; tok0 += tpr) {
+        const int tok = tok0 + slot_tok;
+        const int bid = 1 + slot_tok;                    // named barrier of the slot
+        uint4 *stg = reinterpret_cast<uint4 *>(prep_area + tok * prep_per_tok);
+        if (slot_tok >= tpr || tok >= MT) continue;
         if (tok < M) {
             prep::cp_async_wait_all();
-            bar_named(1 + tok, gt);                      // the row has landed
+            bar_named(bid, gt);                          // the row has landed
             float v[prep::kElemsPerThread];
             prep::load_row(stg, t, v);
-            bar_named(1 + tok, gt);                      // the stage may be overwritten
+            bar_named(bid, gt);                          // the stage may be overwritten
             prep::rotate_row<G>(v, reinterpret_cast<float4 *>(stg), t, 0xFFFFFFFFu);
             const float m = prep::thread_absmax(v);
             uint32_t mb = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m));
             if (lane == 0) red[tok][t >> 5] = mb;
-            bar_named(1 + tok, gt);
+            bar_named(bid, gt);
             for (int w = 0; w < gt / 32; ++w) mb = max(mb, red[tok][w]);
             const float a_u = __uint_as_float(mb);
             const float inv = a_u > 0.0f ? __fdiv_rn(7.0f, a_u) : 0.0f;
@@ -181,13 +189,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t *__restric
                 *reinterpret_cast<uint2 *>(xt + kb * 32 + 2 * i) =
                     make_uint2((packed[w] << 4) & hm, packed[w] & hm);
             }
-        } else if (tok < MT) {
+        } else {
             // tokens M .. MT-1 multiply as zeros
             uint4 *xt = reinterpret_cast<uint4 *>(xw + static_cast<size_t>(tok) * (K / 4));
             for (int i = t; i < K / 16; i += gt) xt[i] = make_uint4(0u, 0u, 0u, 0u);
         }
-        bar_named(kBarConsumers, kConsumerWarps * 32);   // all tokens are ready
     }
+    bar_named(kBarConsumers, kConsumerWarps * 32);       // all tokens are ready
 
     // ---------------------------------------------------------------- GEMV
     const int r = threadIdx.x & (kRows - 1);             // weight row in the slice

@@ -94,13 +94,20 @@ def test_host_validation_without_device(L):
 
 
 def test_single_kernel_rule(L):
-    # one kernel for 1..4 tokens when K is a multiple of 2048 and the token
-    # rows fit one round of in-kernel preparation (M * K / 64 <= 256 threads)
+    # one kernel for 1..4 tokens when K is a multiple of 2048 up to 16384 and
+    # the token rows' buffers (1 + 2 bytes per element for group 64, 1 + 4 for
+    # group 256, for 1, 2 or 4 rows) fit beside two 64 KB ring slots
     assert L.convrot_linear_single_kernel(1, 4096, 64) == 1
     assert L.convrot_linear_single_kernel(4, 4096, 256) == 1
     assert L.convrot_linear_single_kernel(2, 8192, 64) == 1
     assert L.convrot_linear_single_kernel(1, 16384, 256) == 1
-    assert L.convrot_linear_single_kernel(3, 8192, 64) == 0      # 4 x 128 threads
+    assert L.convrot_linear_single_kernel(2, 12288, 64) == 1     # two rounds of 192 threads
+    assert L.convrot_linear_single_kernel(2, 14336, 64) == 1
+    assert L.convrot_linear_single_kernel(4, 6144, 64) == 1      # two rounds of 2 x 96 threads
+    assert L.convrot_linear_single_kernel(3, 8192, 64) == 0      # 4 x 24 KB of rows
+    assert L.convrot_linear_single_kernel(2, 16384, 64) == 0
+    assert L.convrot_linear_single_kernel(4, 8192, 256) == 0
+    assert L.convrot_linear_single_kernel(1, 18432, 64) == 0     # > 256 threads per row
     assert L.convrot_linear_single_kernel(5, 4096, 64) == 0
     assert L.convrot_linear_single_kernel(0, 4096, 64) == 0
     assert L.convrot_linear_single_kernel(1, 3072, 64) == 0      # K % 2048

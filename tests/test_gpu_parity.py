@@ -284,11 +284,14 @@ def test_linear_matches_oracle(group, M, K, N):
 # bit-identical to the two-kernel path (prep kernel + GEMM) on the same inputs.
 DECODE_CASES = [(1, 2048, 1000, 64, True), (1, 4096, 14336, 64, False), (2, 4096, 777, 256, True),
                 (3, 4096, 1024, 256, True), (4, 4096, 3000, 64, True), (1, 16384, 520, 256, False),
-                (2, 8192, 384, 64, True), (4, 2048, 130, 256, False)]
+                (2, 8192, 384, 64, True), (4, 2048, 130, 256, False),
+                # token rows prepared in two rounds
+                (2, 12288, 600, 64, True), (3, 6144, 1040, 64, False), (2, 14336, 272, 64, True)]
 
 
 @pytest.mark.parametrize("M,K,N,group,bias", DECODE_CASES)
 def test_decode_path_matches_oracle(M, K, N, group, bias):
+    assert cr.convrot_linear_single_kernel(M, K, group)      # the one-kernel path runs
     lt = _layer(M, K, N, group, seed=M * 7 + K + N, bias=bias, zero_rows=(1,) if M > 2 else ())
     cols = None if N <= 4096 else np.r_[0:300, N - 300:N]
     _full_path_case(lt, group, cols=cols)
