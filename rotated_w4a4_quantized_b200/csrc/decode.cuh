@@ -63,11 +63,78 @@ constexpr int kBarConsumers = 15;                        // named barrier: warps
 inline size_t smem_bytes(int MT, int G, int K, int SP, int R) {
     const size_t prep_per_tok = static_cast<size_t>(K) * (G == 256 ? 4 : 2);
     return static_cast<size_t>(SP) * kBlocks * R * kPKB + static_cast<size_t>(MT) * K +
-           MT * prep_per_tok + static_cast<size_t>(kRows) * MT * 4 + 2 * SP * 8 + 16;
+           MT * prep_per_tok + static_cast<size_t>(kConsumerWarps * 32) * MT * 4 + 2 * SP * 8 + 16;
 }
+
+// Consumer threads per weight row: 2 for slices of more than 64 rows, 4 for
+// 33..64, 8 for up to 32 (small N), so that all 256 consumer threads work.
+inline __host__ __device__ int threads_per_row(int R) { return R > 64 ? 2 : R > 32 ? 4 : 8; }
 
 __device__ __forceinline__ void bar_named(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// The GEMV over the weight ring with NH consumer threads per weight row:
+// thread (r = t mod 256/NH, h = t / (256/NH)) takes row r and the 8/NH
+// 16-byte chunks h*8/NH .. of every 128-byte column block (chunks 0-3 are
+// the block's first K-block of 128 codes, 4-7 its second), widens them and
+// accumulates sum 256 q_w q_x with dp4a in four independent chains (integer
+// sums: any order gives the same result).  Returns false if a wait gave up.
+template <int MT, int NH>
+__device__ __forceinline__ bool gemv(uint32_t sbase, int slot, int blk, uint32_t xw_s, int K,
+                                     int R, int num_kp, int SP, uint32_t bar0,
+                                     volatile int *abort_flag, int (&acc)[MT]) {
+    constexpr int RR = kConsumerWarps * 32 / NH;         // rows covered
+    constexpr int CPT = 8 / NH;                          // chunks per thread per block
+    const int r = threadIdx.x % RR, h = threadIdx.x / RR;
+    const uint32_t rsw = static_cast<uint32_t>(r & 7);
+    const uint32_t hm = 0xF0F0F0F0u;
+    int a4[MT][4];
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) a4[m][c] = 0;
+    bool ok = true;
+    for (int kp = 0; kp < num_kp; ++kp) {
+        const int s = kp % SP;
+        if (!ptx::mbar_wait(bar0 + 8u * s, (kp / SP) & 1, abort_flag)) { ok = false; break; }
+        if (r < R) {                                     // rows past the slice only wait
+#pragma unroll
+            for (int q = 0; q < kBlocks; ++q) {
+                const uint32_t src = sbase + s * slot + q * blk + r * kPKB;
+                // widened tokens of the block: 2 K-blocks x 128 bytes per token
+                const uint32_t xb = xw_s + static_cast<uint32_t>((kp * kBlocks + q) * 256);
+#pragma unroll
+                for (int cc = 0; cc < CPT; ++cc) {
+                    const int p = h * CPT + cc;          // chunk of the block
+                    const int kbp = p >> 2, c = p & 3;
+                    const uint4 wv = gemm::lds128(src + ((static_cast<uint32_t>(p) ^ rsw) << 4));
+                    const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+                    constexpr int kChains = 4;
+                    const int ch = (q * CPT + cc) % kChains;
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) {
+                        // words 4c .. 4c + 3 of K-block kbp: (even, odd) pairs
+                        const uint32_t xa = xb + static_cast<uint32_t>(m * K + kbp * 128 + 32 * c);
+                        const uint4 x0 = gemm::lds128(xa), x1 = gemm::lds128(xa + 16);
+                        const uint32_t xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            a4[m][ch] = __dp4a(static_cast<int>((ww[j] << 4) & hm),
+                                               static_cast<int>(xv[2 * j]), a4[m][ch]);
+                            a4[m][ch] = __dp4a(static_cast<int>(ww[j] & hm),
+                                               static_cast<int>(xv[2 * j + 1]), a4[m][ch]);
+                        }
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(bar0 + 8u * (SP + s));
+    }
+#pragma unroll
+    for (int m = 0; m < MT; ++m) acc[m] = (a4[m][0] + a4[m][1]) + (a4[m][2] + a4[m][3]);
+    return ok;
 }
 
 // tmW: packed weights [N][K/2], box 128 B x R rows, 128-byte swizzle.
@@ -89,7 +156,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t *__restric
     uint32_t *xw = reinterpret_cast<uint32_t *>(smem + static_cast<size_t>(SP) * slot);
     uint8_t *prep_area = reinterpret_cast<uint8_t *>(xw) + static_cast<size_t>(MT) * K;
     int32_t *accs = reinterpret_cast<int32_t *>(prep_area + MT * prep_per_tok);
-    const uint32_t bar0 = ptx::smem_u32(accs + kRows * MT);
+    const uint32_t bar0 = ptx::smem_u32(accs + kConsumerWarps * 32 * MT);
     auto full_p = [&](int s) { return bar0 + 8u * s; };
     auto empty_p = [&](int s) { return bar0 + 8u * (SP + s); };
     __shared__ uint32_t red[MT][kConsumerWarps];
@@ -198,56 +265,24 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t *__restric
     bar_named(kBarConsumers, kConsumerWarps * 32);       // all tokens are ready
 
     // ---------------------------------------------------------------- GEMV
-    const int r = threadIdx.x & (kRows - 1);             // weight row in the slice
-    const int h = threadIdx.x >> 7;                      // K-block of each stage
-    const uint32_t rsw = static_cast<uint32_t>(r & 7);
-    int a4[MT][4];                                       // chain c: words 4c .. 4c + 3
-#pragma unroll
-    for (int m = 0; m < MT; ++m)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) a4[m][c] = 0;
-    bool ok = true;
-    for (int kp = 0; kp < num_kp; ++kp) {
-        const int s = kp % SP;
-        if (!ptx::mbar_wait(full_p(s), (kp / SP) & 1, abort_flag)) { ok = false; break; }
-        if (r < R) {                                     // rows past the slice only wait
-#pragma unroll
-            for (int q = 0; q < kBlocks; ++q) {
-                const uint32_t src = sbase + s * slot + q * blk + r * kPKB;
-                const uint32_t xk = ptx::smem_u32(xw) +
-                                    static_cast<uint32_t>((2 * (kp * kBlocks + q) + h) * 128);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint4 wv = gemm::lds128(src + ((static_cast<uint32_t>(4 * h + c) ^ rsw) << 4));
-                    const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) {
-                        // words 4c .. 4c + 3 of the K-block: (even, odd) pairs
-                        const uint32_t xa = xk + static_cast<uint32_t>(m * K + 32 * c);
-                        const uint4 x0 = gemm::lds128(xa), x1 = gemm::lds128(xa + 16);
-                        const uint32_t xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            a4[m][c] = __dp4a(static_cast<int>((ww[j] << 4) & hm),
-                                              static_cast<int>(xv[2 * j]), a4[m][c]);
-                            a4[m][c] = __dp4a(static_cast<int>(ww[j] & hm),
-                                              static_cast<int>(xv[2 * j + 1]), a4[m][c]);
-                        }
-                    }
-                }
-            }
-        }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(empty_p(s));
-    }
+    // Thread (r, h): weight row r of the slice and part h of every 128-byte
+    // column block, with NH threads per row (threads_per_row).
+    const int nh = threads_per_row(R);
     int acc[MT];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) acc[m] = (a4[m][0] + a4[m][1]) + (a4[m][2] + a4[m][3]);
+    bool ok;
+    if (nh == 2)
+        ok = gemv<MT, 2>(sbase, slot, blk, ptx::smem_u32(xw), K, R, num_kp, SP, bar0, abort_flag, acc);
+    else if (nh == 4)
+        ok = gemv<MT, 4>(sbase, slot, blk, ptx::smem_u32(xw), K, R, num_kp, SP, bar0, abort_flag, acc);
+    else
+        ok = gemv<MT, 8>(sbase, slot, blk, ptx::smem_u32(xw), K, R, num_kp, SP, bar0, abort_flag, acc);
 
     // ------------------------------------------------------------ epilogue
-    if (h == 1)
+    // The NH parts of each row are added (exact integers) by its part 0.
+    const int rr = (kConsumerWarps * 32) / nh;
+    const int r = threadIdx.x % rr, h = threadIdx.x / rr;
 #pragma unroll
-        for (int m = 0; m < MT; ++m) accs[r * MT + m] = acc[m];
+    for (int m = 0; m < MT; ++m) accs[threadIdx.x * MT + m] = acc[m];
     bar_named(kBarConsumers, kConsumerWarps * 32);
     const int n = n0 + r;
     if (ok && h == 0 && r < R && n < N) {
@@ -256,7 +291,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t *__restric
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
             if (m >= M) break;
-            const int32_t total = acc[m] + accs[r * MT + m];
+            int32_t total = acc[m];
+            for (int p = 1; p < nh; ++p) total += accs[(p * rr + r) * MT + m];
             y[static_cast<size_t>(m) * N + n] =
                 gemm::f32_to_bf16_rne(gemm::epi(static_cast<uint32_t>(total), sxs[m], swn, bn));
         }

@@ -286,7 +286,9 @@ DECODE_CASES = [(1, 2048, 1000, 64, True), (1, 4096, 14336, 64, False), (2, 4096
                 (3, 4096, 1024, 256, True), (4, 4096, 3000, 64, True), (1, 16384, 520, 256, False),
                 (2, 8192, 384, 64, True), (4, 2048, 130, 256, False),
                 # token rows prepared in two rounds
-                (2, 12288, 600, 64, True), (3, 6144, 1040, 64, False), (2, 14336, 272, 64, True)]
+                (2, 12288, 600, 64, True), (3, 6144, 1040, 64, False), (2, 14336, 272, 64, True),
+                # slices of 33..64 rows (four consumer threads per weight row)
+                (2, 4096, 6144, 256, True), (4, 2048, 8000, 64, False)]
 
 
 @pytest.mark.parametrize("M,K,N,group,bias", DECODE_CASES)
