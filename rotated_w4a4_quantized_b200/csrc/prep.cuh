@@ -1,7 +1,9 @@
 // prep.cuh -- fused rotation + rowwise absmax INT4 quantisation + packing.
 //
-// K/64 threads per CTA, persistent over rows; thread t owns the 64
-// consecutive channels [64t, 64t + 64) of each row it helps with.
+// prep_kernel: K/64 threads per CTA, persistent over rows; thread t owns the
+// 64 consecutive channels [64t, 64t + 64) of each row it helps with.
+// prep16_kernel (end of file): the same steps with 16 channels per thread,
+// for launches of up to 1024 rows, where each row's latency is the cost.
 //
 // Rotation.  Within a group of n = 4^k channels the normalised regular
 // Hadamard is H_n = T^{(x)k} / 2^k with T = J - 2I (Comfy-Org/comfy-quants
@@ -57,9 +59,10 @@ __device__ __forceinline__ uint32_t pack_nibbles(int hi, int lo, uint32_t acc) {
 //
 // Digit 0 (stride 1): the quadruple {4q .. 4q+3} is two pairs; their packed
 // sum gives (v0+v2, v1+v3), one scalar add completes the quadruple sum.
-__device__ __forceinline__ void radix4_digit0(float (&v)[kElemsPerThread]) {
+template <int E>
+__device__ __forceinline__ void radix4_digit0(float (&v)[E]) {
 #pragma unroll
-    for (int b = 0; b < kElemsPerThread; b += 4) {
+    for (int b = 0; b < E; b += 4) {
         float p0, p1;
         add2(p0, p1, v[b], v[b + 1], v[b + 2], v[b + 3]);
         const float sum = p0 + p1;
@@ -70,10 +73,10 @@ __device__ __forceinline__ void radix4_digit0(float (&v)[kElemsPerThread]) {
 
 // Digits with stride S = 4 or 16: the quadruples starting at b and b + 1
 // (b even) run side by side in the two halves of each packed operation.
-template <int S>
-__device__ __forceinline__ void radix4_stage(float (&v)[kElemsPerThread]) {
+template <int S, int E>
+__device__ __forceinline__ void radix4_stage(float (&v)[E]) {
 #pragma unroll
-    for (int b = 0; b < kElemsPerThread; b += 2) {
+    for (int b = 0; b < E; b += 2) {
         if ((b / S) % 4 != 0) continue;
         float s01a, s01b, s23a, s23b, suma, sumb;
         add2(s01a, s01b, v[b], v[b + 1], v[b + S], v[b + 1 + S]);
@@ -172,10 +175,11 @@ __device__ __forceinline__ int row_chan(int t, int e) {
 }
 
 // The thread's max |v|: four independent chains of three-input maxima.
-__device__ __forceinline__ float thread_absmax(const float (&v)[kElemsPerThread]) {
+template <int E>
+__device__ __forceinline__ float thread_absmax(const float (&v)[E]) {
     float mk[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-    for (int e = 0; e < kElemsPerThread; e += 8)
+    for (int e = 0; e < E; e += 8)
 #pragma unroll
         for (int k = 0; k < 4; ++k) mk[k] = max3(mk[k], fabsf(v[e + 2 * k]), fabsf(v[e + 2 * k + 1]));
     return max3(mk[0], mk[1], fmaxf(mk[2], mk[3]));
@@ -183,10 +187,11 @@ __device__ __forceinline__ float thread_absmax(const float (&v)[kElemsPerThread]
 
 // Codes q = round_half_away(v * inv), packed two per byte (low nibble =
 // even register): packed[w] holds registers 8w .. 8w + 7.
-__device__ __forceinline__ void quantize_pack(const float (&v)[kElemsPerThread], float inv,
-                                              uint32_t (&packed)[8]) {
+template <int E>
+__device__ __forceinline__ void quantize_pack(const float (&v)[E], float inv,
+                                              uint32_t (&packed)[E / 8]) {
 #pragma unroll
-    for (int w = 0; w < 8; ++w) {
+    for (int w = 0; w < E / 8; ++w) {
         int code[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -309,6 +314,88 @@ prep_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ 
                 *reinterpret_cast<uint2 *>(qrow + chan(16 * d3) / 2) =
                     make_uint2(packed[2 * d3], packed[2 * d3 + 1]);
         }
+    }
+}
+
+
+// ------------------------------------------------------------------------
+// The same preparation with 16 channels per thread (K/16 threads per row),
+// for latency-bound launches (few rows per SM): a quarter of the per-thread
+// work per row and no shared-memory exchange.  Thread t owns channels
+// [16t, 16t + 16), loaded straight from global memory (32 contiguous bytes
+// per thread, coalesced).  Digits 0 and 1 of the rotation run in registers;
+// digit 2 spans lanes t ^ 1, t ^ 2 (the four threads of a 64-group) and,
+// for n = 256, digit 3 lanes t ^ 4, t ^ 8, as shuffles: lane l forms
+// (x_l + x_l^1) + (x_l^2 + x_l^3), the same sums in the same order as the
+// register butterfly (x_0 + x_1) + (x_2 + x_3) (addition commutes bitwise),
+// so codes, scales and rotated values are bit-identical to prep_kernel's.
+__device__ __forceinline__ void radix4_lanes(float (&v)[16], int m1, int m2) {
+#pragma unroll
+    for (int e = 0; e < 16; e += 2) {
+        float a0 = v[e] + __shfl_xor_sync(0xFFFFFFFFu, v[e], m1);
+        float a1 = v[e + 1] + __shfl_xor_sync(0xFFFFFFFFu, v[e + 1], m1);
+        const float s0 = a0 + __shfl_xor_sync(0xFFFFFFFFu, a0, m2);
+        const float s1 = a1 + __shfl_xor_sync(0xFFFFFFFFu, a1, m2);
+        bfly2(v[e], v[e + 1], s0, s1);
+    }
+}
+
+template <int G, int MODE>
+__global__ void __launch_bounds__(1024)
+prep16_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ q,
+              float *__restrict__ s, float *__restrict__ yrot) {
+    static_assert(G == 64 || G == 256, "group 64 or 256");
+    constexpr float kNorm = (G == 64) ? 0.125f : 0.0625f;   // 2^-digits
+    __shared__ uint32_t red[2][32];
+    // blockDim.x = K/16 rounded up to whole warps; K is a multiple of 256, so
+    // the padding lanes form whole 16-lane groups: they hold zeros, take part
+    // in the shuffles and the maximum, and store nothing.
+    const int t = threadIdx.x;
+    const bool act = t < K / 16;
+    const int nwarps = blockDim.x >> 5;
+    const int warp = t >> 5, lane = t & 31;
+    int it = 0;
+    for (int row = blockIdx.x; row < M; row += gridDim.x, ++it) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(row) * K) + 2 * t;
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        const uint4 r0 = act ? src[0] : z, r1 = act ? src[1] : z;
+        // As in prep_kernel: the GEMM that follows may be scheduled (and
+        // stream its weights) from now on; it reads these rows only after
+        // its griddepcontrol.wait.
+        if (it == 0) ptx::launch_dependents();
+        float v[16];
+        const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            v[2 * j] = __uint_as_float(w[j] << 16);
+            v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+        radix4_digit0(v);
+        radix4_stage<4>(v);
+        radix4_lanes(v, 1, 2);                           // digit 2
+        if (G == 256) radix4_lanes(v, 4, 8);             // digit 3
+        if (MODE == 1) {
+            if (!act) continue;
+            float4 *dst = reinterpret_cast<float4 *>(yrot + static_cast<size_t>(row) * K) + 4 * t;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                dst[i] = make_float4(v[4 * i] * kNorm, v[4 * i + 1] * kNorm, v[4 * i + 2] * kNorm,
+                                     v[4 * i + 3] * kNorm);
+            continue;
+        }
+        const float m = thread_absmax(v);
+        uint32_t mb = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m));
+        if (lane == 0) red[it & 1][warp] = mb;           // two buffers: one barrier per row
+        __syncthreads();
+        for (int wi = 0; wi < nwarps; ++wi) mb = max(mb, red[it & 1][wi]);
+        const float a_u = __uint_as_float(mb);
+        const float inv = a_u > 0.0f ? __fdiv_rn(7.0f, a_u) : 0.0f;
+        if (t == 0) s[row] = __fdiv_rn(a_u * kNorm, 7.0f);
+        uint32_t packed[2];
+        quantize_pack(v, inv, packed);
+        if (act)
+            *reinterpret_cast<uint2 *>(q + static_cast<size_t>(row) * (K / 2) + 8 * t) =
+                make_uint2(packed[0], packed[1]);
     }
 }
 

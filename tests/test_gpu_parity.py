@@ -45,7 +45,8 @@ def _layer(M, K, N, group, seed, bias=True, zero_rows=()):
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("group", [64, 256])
-@pytest.mark.parametrize("M,K", [(1, 256), (7, 1024), (33, 3072), (5, 12288), (3, 32768)])
+@pytest.mark.parametrize("M,K", [(1, 256), (7, 1024), (33, 3072), (5, 12288), (3, 32768),
+                                 (1030, 512)])
 def test_rotation_matches_oracle(group, M, K):
     x = wl.make_random_layer(M, K, 1, group, seed=M + K).x
     y = cr.convrot_debug_rotate_f32(_dev(x), group)
@@ -54,7 +55,8 @@ def test_rotation_matches_oracle(group, M, K):
 
 
 @pytest.mark.parametrize("group", [64, 256])
-@pytest.mark.parametrize("M,K", [(1, 256), (9, 1024), (130, 3072), (4, 12288), (2, 32768)])
+@pytest.mark.parametrize("M,K", [(1, 256), (9, 1024), (130, 3072), (4, 12288), (2, 32768),
+                                 (1100, 768)])
 def test_prepare_matches_oracle(group, M, K):
     x = _layer(M, K, 1, group, seed=3 * M + K, zero_rows=(0,) if M > 2 else ()).x
     xb = wl.bf16_bits(x)
