@@ -5,7 +5,8 @@
 One step is one pass of the whole path over one batch through the public
 call convrot_linear: the fused prep kernel (rotation, rowwise absmax INT4
 quantisation, packing) and the tcgen05 GEMM with its scale/bias/bf16
-epilogue (two kernels per linear layer).  Weights are prepared once before
+epilogue (two kernels per linear layer; for 1-4 tokens one kernel that does
+both).  Weights are prepared once before
 timing (the offline step).  Caches stay cold without a flush kernel: the
 steps cycle through enough full copies of the step's data (activations,
 workspace, weights, outputs) that the copies together exceed twice the L2

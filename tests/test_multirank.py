@@ -1,0 +1,73 @@
+"""The multi-rank benchmark path on the CPU (gloo, world size 2).
+
+The layer partitions over tokens: every rank runs its own batch with
+replicated weights and no data-path collective; the only cross-rank
+operations are the timing reduction (max of the step time, sum of the work)
+and, for the reference arm, that only rank 0 runs and prints.
+"""
+import argparse
+import os
+import socket
+import tempfile
+
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+from rotated_w4a4_quantized_b200 import workloads as wl
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _aggregate_rank(rank: int, world: int, port: int, out_dir: str):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        ms, ops = bench.aggregate(1.5 + rank, 10.0 * (rank + 1))
+        with open(os.path.join(out_dir, f"rank{rank}.txt"), "w") as f:
+            f.write(f"{ms} {ops}\n")
+    finally:
+        dist.destroy_process_group()
+
+
+def test_aggregate_takes_max_time_and_total_work_over_two_ranks():
+    port = _free_port()
+    with tempfile.TemporaryDirectory() as d:
+        mp.start_processes(_aggregate_rank, args=(2, port, d), nprocs=2, join=True,
+                           start_method="spawn")
+        for rank in range(2):
+            with open(os.path.join(d, f"rank{rank}.txt")) as f:
+                ms, ops = map(float, f.read().split())
+            assert ms == 2.5            # the slowest rank's time
+            assert ops == 30.0          # every rank's work
+
+
+def test_aggregate_is_local_without_a_process_group():
+    assert not dist.is_initialized()
+    assert bench.aggregate(3.25, 7.0) == (3.25, 7.0)
+
+
+def test_each_rank_runs_its_own_batch_of_the_same_shape():
+    name = "small_g256"
+    seed = wl.WORKLOADS[name].seed
+    r0 = wl.make_workload(name, seed=seed + 0)
+    r1 = wl.make_workload(name, seed=seed + 1)
+    assert [l.spec for l in r0] == [l.spec for l in r1]
+    for a, b in zip(r0, r1):
+        assert a.x.shape == b.x.shape and a.w.shape == b.w.shape
+        assert not torch.equal(a.x, b.x)
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    args = argparse.Namespace(workload="small_g256", steps=3, warmup=3, cpu_seconds=0.1)
+    assert bench.run_reference(args) is None
+    assert capsys.readouterr().out == ""
