@@ -341,7 +341,7 @@ __device__ __forceinline__ void radix4_lanes(float (&v)[16], int m1, int m2) {
 }
 
 template <int G, int MODE>
-__global__ void __launch_bounds__(1024)
+__global__ void __maxnreg__(40)
 prep16_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ q,
               float *__restrict__ s, float *__restrict__ yrot) {
     static_assert(G == 64 || G == 256, "group 64 or 256");
