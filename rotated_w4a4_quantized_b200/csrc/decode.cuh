@@ -23,19 +23,21 @@
 //     bytes about 5.5 TB/s;
 //   * warps 0-7 first prepare the tokens: token m is handled by K/64 threads
 //     exactly as in prep_kernel (staged bf16 row, radix-4 butterflies,
-//     absmax, round-half-away, nibble packing), then widen the packed codes
-//     to int8 words in shared memory (16 x code, even and odd codes of each
-//     packed word apart, as the GEMM widens them);
-//   * then thread (r, h) of warps 0-7 takes weight row r and K-block h of
-//     each column block: it widens its 64 packed bytes and accumulates
-//     sum 256 q_w q_x with dp4a (s8 x s8 -> s32) on the CUDA cores, exactly,
-//     in four independent chains (integer sums: any order gives the same
-//     result) so that the dp4a latency does not serialise the stage;
-//     with <= 4 tokens the tensor core would spend its ~75-cycle minimum per
-//     128-row MMA on 1-4 useful columns, while dp4a needs about one
-//     instruction per weight byte per token;
-//   * the two K halves of each row are added and the epilogue (the GEMM's,
-//     same arithmetic) writes y.
+//     absmax, round-half-away, nibble packing), in rounds when the rows need
+//     more than 256 threads, then widen the packed codes to int8 words in
+//     shared memory (16 x code, even and odd codes of each packed word
+//     apart, as the GEMM widens them);
+//   * then thread (r, h) of warps 0-7 takes weight row r and part h of each
+//     128-byte column block (2, 4 or 8 threads per row: see gemv), widens
+//     its packed bytes and accumulates sum 256 q_w q_x with dp4a
+//     (s8 x s8 -> s32) on the CUDA cores, exactly, in four independent
+//     chains (integer sums: any order gives the same result) so that the
+//     dp4a latency does not serialise the stage; with <= 4 tokens the tensor
+//     core would spend its ~75-cycle minimum per 128-row MMA on 1-4 useful
+//     columns, while dp4a needs about one instruction per weight byte per
+//     token;
+//   * the parts of each row are added and the epilogue (the GEMM's, same
+//     arithmetic) writes y.
 // Eligible shapes: M <= 4, K a multiple of 2048 up to 16384 (at most 256
 // threads per token row; rows beyond what 256 threads hold at once are
 // prepared in further rounds), and the rows' buffers fit in shared memory

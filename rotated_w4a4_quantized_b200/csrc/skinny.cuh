@@ -38,8 +38,10 @@
 //               per stage, A from TMEM, B from shared memory;
 //   warps 2..5  token widening into the swizzled B stages;
 //   warps 6..9  weight widening into the TMEM A stages (thread = weight row
-//               = TMEM lane), then the epilogue (tcgen05.ld, scale, bias,
-//               bf16) for the same lanes.
+//               = TMEM lane);
+//   warps 2..9  then the epilogue (tcgen05.ld, scale, bias, bf16), two warps
+//               per TMEM lane quarter, two tokens at a time.
+// The CTA-pair form (PAIR) shares each MMA between two CTAs (see Cfg).
 #pragma once
 
 #include "gemm.cuh"
