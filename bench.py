@@ -483,14 +483,28 @@ class OracleSampler:
         return 2 * rows * self.sp.N * self.sp.K
 
 
+# workloads whose baseline also gets a one-thread figure
+ONE_THREAD_BASELINE = ("small_g256", "outlier_g64")
+
+
 def cpu_baseline(name, seconds):
     s = OracleSampler(name)
     rows = s.calibrate(seconds)
     t = s.run(rows)
-    return {"value": round(s.ops(rows) / t / 1e12, 9), "unit": "TOPS", "cores": s.cores,
-            "kind": "oracle",
-            "sample": f"{rows} of {s.sp.M} token rows of layer {s.layer} (prep + int64 GEMM + "
-                      f"epilogue, weights prepared offline), {t:.1f} s"}
+    out = {"value": round(s.ops(rows) / t / 1e12, 9), "unit": "TOPS", "cores": s.cores,
+           "kind": "oracle",
+           "sample": f"{rows} of {s.sp.M} token rows of layer {s.layer} (prep + int64 GEMM + "
+                     f"epilogue, weights prepared offline), {t:.1f} s"}
+    if name in ONE_THREAD_BASELINE:
+        s.O.set_num_threads(1)
+        try:
+            rows1 = s.calibrate(seconds / 4)
+            t1 = s.run(rows1)
+        finally:
+            s.O.set_num_threads(s.cores)
+        out["value_1thread"] = round(s.ops(rows1) / t1 / 1e12, 9)
+        out["sample_1thread"] = f"{rows1} token rows on one thread, {t1:.1f} s"
+    return out
 
 
 def run_reference(args):
