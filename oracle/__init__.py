@@ -57,6 +57,11 @@ def lib():
             "oracle_epilogue": [P, P, P, P, I64, I64, P],
             "oracle_prepare_rows": [P, I64, I64, I, P, P],
             "oracle_linear_prepared_w": [P, P, P, P, I64, I64, I64, I, P],
+            "oracle_round_bf16": [P, I64, P],
+            "oracle_w4a16_rotate_act": [P, I64, I64, I, P],
+            "oracle_w4a16_gemm": [P, P, I64, I64, I64, P, P, P],
+            "oracle_w4a16_epilogue": [P, P, P, I64, I64, P, P],
+            "oracle_w4a16_linear": [P, P, P, P, I64, I64, I64, I, P],
             "oracle_num_threads": [],
         }
         for name, args in sig.items():
@@ -213,3 +218,86 @@ def tie_band(y: np.ndarray, s: np.ndarray, band: float = 1e-5) -> np.ndarray:
         v = np.where(s64 > 0, y / np.where(s64 > 0, s64, 1.0), 0.0)
     a = np.abs(v)
     return np.abs(a - (np.floor(a) + 0.5)) < band
+
+
+# --------------------------------------------------------------------------
+# The W4A16 variant
+# --------------------------------------------------------------------------
+
+def round_bf16(y: np.ndarray) -> np.ndarray:
+    """bf16 bits of fp64 values, rounded once to nearest, ties to even."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    out = np.empty(y.shape, dtype=np.uint16)
+    _check(lib().oracle_round_bf16(_ptr(y), y.size, _ptr(out)), "round_bf16")
+    return out
+
+
+def w4a16_rotate_act(x_bf16: np.ndarray, group: int) -> np.ndarray:
+    """bf16 bits of the rotated rows, each value rounded once."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    rows, K = x.shape
+    xr = np.empty((rows, K), dtype=np.uint16)
+    _check(lib().oracle_w4a16_rotate_act(_ptr(x), rows, K, group, _ptr(xr)), "w4a16_rotate_act")
+    return xr
+
+
+def w4a16_gemm(xr_bf16: np.ndarray, qw: np.ndarray, K: int):
+    """(acc, l1, p16) fp64 [M][N]: sum_k xr q, sum_k |xr q|, and the sum of
+    |partial sums| at every 16th K position (packed weights)."""
+    xr = np.ascontiguousarray(xr_bf16, dtype=np.uint16)
+    qw = np.ascontiguousarray(qw, dtype=np.uint8)
+    M, N = xr.shape[0], qw.shape[0]
+    acc = np.empty((M, N), dtype=np.float64)
+    l1 = np.empty((M, N), dtype=np.float64)
+    p16 = np.empty((M, N), dtype=np.float64)
+    _check(lib().oracle_w4a16_gemm(_ptr(xr), _ptr(qw), M, N, K, _ptr(acc), _ptr(l1), _ptr(p16)),
+           "w4a16_gemm")
+    return acc, l1, p16
+
+
+def w4a16_epilogue(acc: np.ndarray, sw: np.ndarray, bias_bf16: np.ndarray | None):
+    """(t fp64, y bf16 bits): t = acc sw + b exactly, y = bf16_rne(t)."""
+    acc = np.ascontiguousarray(acc, dtype=np.float64)
+    sw = np.ascontiguousarray(sw, dtype=np.float32)
+    b = None if bias_bf16 is None else np.ascontiguousarray(bias_bf16, dtype=np.uint16)
+    M, N = acc.shape
+    t = np.empty((M, N), dtype=np.float64)
+    y = np.empty((M, N), dtype=np.uint16)
+    _check(lib().oracle_w4a16_epilogue(_ptr(acc), _ptr(sw), _ptr(b), M, N, _ptr(t), _ptr(y)),
+           "w4a16_epilogue")
+    return t, y
+
+
+def w4a16_linear(x_bf16, qw, sw, bias_bf16, group: int) -> np.ndarray:
+    """bf16 bits y [M][N] of the whole W4A16 layer given prepared weights."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    qw = np.ascontiguousarray(qw, dtype=np.uint8)
+    sw = np.ascontiguousarray(sw, dtype=np.float32)
+    b = None if bias_bf16 is None else np.ascontiguousarray(bias_bf16, dtype=np.uint16)
+    M, K = x.shape
+    N = qw.shape[0]
+    y = np.empty((M, N), dtype=np.uint16)
+    _check(lib().oracle_w4a16_linear(_ptr(x), _ptr(qw), _ptr(sw), _ptr(b), M, N, K, group,
+                                     _ptr(y)), "w4a16_linear")
+    return y
+
+
+def bf16_spacing(y: np.ndarray) -> np.ndarray:
+    """Distance between the two bf16 values around |y| (2^-133 below the
+    normal range)."""
+    a = np.abs(np.asarray(y, dtype=np.float64))
+    _, e = np.frexp(a)
+    q = np.where(e - 1 < -126, -133, e - 8)
+    return np.ldexp(1.0, q)
+
+
+def bf16_tie_band(y: np.ndarray, band: float = 1e-5) -> np.ndarray:
+    """Mask of fp64 values lying within ``band`` x (the row's max |y|) of a
+    bf16 rounding midpoint: where two fp32 evaluations of the rotation may
+    round to neighbouring bf16 values."""
+    y = np.asarray(y, dtype=np.float64)
+    a = np.abs(y)
+    sp = bf16_spacing(a)
+    mid = (np.floor(a / sp) + 0.5) * sp
+    amax = a.max(axis=-1, keepdims=True) if a.ndim > 1 else a.max()
+    return np.abs(a - mid) <= band * amax

@@ -44,6 +44,14 @@
  *    complete path is rotation, activation quantisation, the integer product,
  *    scaling and bias.
  *
+ *  - The W4A16 variant.  "convrot-mlx" README, "What is included" (a W4A16
+ *    TensorOps path beside W4A4) and "Requirements" (BF16 x INT4 products).
+ *    The pages give no formula; reading: the weights are the W4A4 ones
+ *    (rotated, quantised, packed), the activations are rotated by the same
+ *    R and each rotated value is rounded once to bf16 (the operand type),
+ *    and y = bf16_rne(sum_k xr[m][k] q[n][k] * sw[n] + b[n]) with the sum,
+ *    the scaling and the bias exact (fp64 here), rounded once at the end.
+ *
  * Every function returns 0 on success or a negative number for bad
  * arguments.  Buffers are caller-owned, row-major and contiguous.
  * bf16 values travel as their raw 16-bit patterns (uint16_t).
@@ -354,6 +362,119 @@ int oracle_linear_prepared_w(const uint16_t *x, const uint8_t *qw, const float *
     if (!rc) rc = oracle_epilogue(acc, sx, sw, bias, M, N, y);
     free(qx);
     free(sx);
+    free(acc);
+    return rc;
+}
+
+/* ----------------------------------------------------------------------- */
+/* The W4A16 variant.                                                        */
+/* ----------------------------------------------------------------------- */
+
+/* Round a finite double to the nearest bf16 (8 significant bits), ties to
+ * even, in one step: scale |v| by a power of two so that the bf16 spacing
+ * becomes 1, round that to an integer, scale back.  (Going through fp32
+ * first would round twice.)  Below the normal range the spacing is that of
+ * the subnormals, 2^-133; above it the result overflows to infinity. */
+static uint16_t double_to_bf16_bits_rne(double v) {
+    if (v == 0.0) return signbit(v) ? (uint16_t)0x8000u : (uint16_t)0;
+    if (!isfinite(v)) return float_to_bf16_bits_rne((float)v);
+    double a = fabs(v);
+    int e;
+    frexp(a, &e);                        /* a = f 2^e, 0.5 <= f < 1 */
+    int q = e - 8;                       /* spacing 2^(e-1) * 2^-7 */
+    if (e - 1 < -126) q = -133;          /* subnormal spacing */
+    double scaled = ldexp(a, -q);        /* exact */
+    double f = floor(scaled);
+    double frac = scaled - f;            /* exact */
+    if (frac > 0.5 || (frac == 0.5 && fmod(f, 2.0) != 0.0)) f += 1.0;
+    float rf = (float)ldexp(f, q);       /* exact: at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &rf, sizeof u);
+    uint16_t h = (uint16_t)(u >> 16);
+    return v < 0.0 ? (uint16_t)(h | 0x8000u) : h;
+}
+
+int oracle_round_bf16(const double *in, int64_t count, uint16_t *out) {
+    if (!in || !out || count < 0) return -1;
+    for (int64_t i = 0; i < count; ++i) out[i] = double_to_bf16_bits_rne(in[i]);
+    return 0;
+}
+
+/* xr = bf16_rne(x R): the fp64 rotation above, each value rounded once. */
+int oracle_w4a16_rotate_act(const uint16_t *x, int64_t rows, int64_t K, int n, uint16_t *xr) {
+    if (!x || !xr || rows < 0 || K <= 0 || log4_exact(n) < 0 || K % n) return -1;
+    if (rows == 0) return 0;
+    double *y = (double *)malloc(sizeof(double) * (size_t)rows * (size_t)K);
+    if (!y) return -2;
+    int rc = oracle_rotate(x, rows, K, n, y);
+    if (!rc) rc = oracle_round_bf16(y, rows * K, xr);
+    free(y);
+    return rc;
+}
+
+/* acc[m][n] = sum_k xr[m][k] q[n][k] in fp64 (every product is exact; so is
+ * the sum while the row's values span fewer than about 40 binades), and two
+ * magnitudes that bound the rounding of any evaluation that adds the terms
+ * in K order, 16 at a time:
+ *   l1[m][n]  = sum_k |xr[m][k] q[n][k]|,
+ *   p16[m][n] = sum_j |partial sum over k < min(16 j, K)|, j = 1 .. ceil(K/16).
+ * l1 and p16 may be NULL. */
+int oracle_w4a16_gemm(const uint16_t *xr, const uint8_t *qw, int64_t M, int64_t N, int64_t K,
+                      double *acc, double *l1, double *p16) {
+    if (!xr || !qw || !acc || M < 0 || N < 0 || K <= 0 || K % 2) return -1;
+    int8_t *b = (int8_t *)malloc((size_t)N * (size_t)K + 1);
+    double *a = (double *)malloc(sizeof(double) * ((size_t)M * (size_t)K + 1));
+    if (!a || !b) { free(a); free(b); return -2; }
+    oracle_unpack(qw, N, K, b);
+    for (int64_t i = 0; i < M * K; ++i) a[i] = bf16_bits_to_double(xr[i]);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double s = 0.0, s1 = 0.0, sp = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double t = a[m * K + k] * (double)b[n * K + k];
+                s += t;
+                s1 += fabs(t);
+                if (k % 16 == 15 || k == K - 1) sp += fabs(s);
+            }
+            acc[m * N + n] = s;
+            if (l1) l1[m * N + n] = s1;
+            if (p16) p16[m * N + n] = sp;
+        }
+    }
+    free(a);
+    free(b);
+    return 0;
+}
+
+/* t[m][n] = acc[m][n] * sw[n] + b[n] in fp64 and y = bf16_rne(t); bias may
+ * be NULL (zeros); t may be NULL. */
+int oracle_w4a16_epilogue(const double *acc, const float *sw, const uint16_t *bias, int64_t M,
+                          int64_t N, double *t, uint16_t *y) {
+    if (!acc || !sw || !y || M < 0 || N < 0) return -1;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double v = acc[m * N + n] * (double)sw[n];
+            v += bias ? bf16_bits_to_double(bias[n]) : 0.0;
+            if (t) t[m * N + n] = v;
+            y[m * N + n] = double_to_bf16_bits_rne(v);
+        }
+    return 0;
+}
+
+/* The whole W4A16 layer on bf16 inputs, given the prepared weights. */
+int oracle_w4a16_linear(const uint16_t *x, const uint8_t *qw, const float *sw,
+                        const uint16_t *bias, int64_t M, int64_t N, int64_t K, int n,
+                        uint16_t *y) {
+    if (!x || !qw || !sw || !y || M < 0 || N < 0 || K <= 0) return -1;
+    if (M == 0 || N == 0) return 0;
+    uint16_t *xr = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)M * (size_t)K);
+    double *acc = (double *)malloc(sizeof(double) * (size_t)M * (size_t)N);
+    if (!xr || !acc) { free(xr); free(acc); return -2; }
+    int rc = oracle_w4a16_rotate_act(x, M, K, n, xr);
+    if (!rc) rc = oracle_w4a16_gemm(xr, qw, M, N, K, acc, NULL, NULL);
+    if (!rc) rc = oracle_w4a16_epilogue(acc, sw, bias, M, N, NULL, y);
+    free(xr);
     free(acc);
     return rc;
 }
