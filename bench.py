@@ -20,6 +20,10 @@ reported time is the maximum over ranks.
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
 instead, on bounded samples of the same workload, on the host cores.
+
+``--variant w4a16`` measures the W4A16 variant the same way instead (public
+call convrot_w4a16_linear: the rotation kernel writing bf16, then the bf16 x
+INT4 tcgen05 GEMM), reported in bf16 tensor TFLOP/s.
 """
 from __future__ import annotations
 
@@ -51,6 +55,11 @@ SKINNY_MAX_M = 128   # the GEMM's few-token form (weight stream, HBM-bound) up t
 # whole-layer algorithmic bytes when the layer runs as one kernel
 LAYER_BYTES = lambda M, N, K: 2 * M * K + N * K // 2 + 4 * N + 2 * N + 2 * M * N  # noqa: E731
 INT8_PER_BF16 = 2.0   # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+METRIC_W4A16 = "W4A16 linear end-to-end TFLOP/s (bf16 x INT4 tensor ops); rotation kernel HBM GB/s"
+# W4A16 algorithmic bytes: the rotation reads x and writes xr (bf16 each);
+# the GEMM reads xr, the packed weights, scales and bias and writes y
+ROT16_BYTES = lambda M, K: 4 * M * K  # noqa: E731
+GEMM16_BYTES = lambda M, N, K: 2 * M * K + N * K // 2 + 4 * N + 2 * N + 2 * M * N  # noqa: E731
 
 
 def _peaks():
@@ -64,10 +73,16 @@ def _peaks():
         return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "src": "fallback"}
 
 
+# the sources libconvrot.so (the W4A4 kernels) is compiled from
+W4A4_SOURCES = ("convrot.cu", "decode.cuh", "gemm.cuh", "prep.cuh", "ptx.cuh", "skinny.cuh")
+
+
 def _src_hash():
+    """Hash of the W4A4 kernel sources: the committed per-launch DRAM traffic
+    of those kernels holds while it is unchanged."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "rotated_w4a4_quantized_b200", "csrc")
-    for name in sorted(os.listdir(d)):
+    for name in sorted(W4A4_SOURCES):
         with open(os.path.join(d, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -412,6 +427,231 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
+def run_gpu_w4a16(args):
+    """The W4A16 variant: the same timing scheme as run_gpu (cold L2 through
+    rotating copies, CUDA graphs, K back-to-back steps between two events,
+    max over ranks), through convrot_w4a16_linear."""
+    import torch.distributed as dist
+
+    import rotated_w4a4_quantized_b200 as cr
+    from rotated_w4a4_quantized_b200 import build
+    build.build()
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    name = args.workload
+    spec = wl.WORKLOADS[name]
+    layers = wl.make_workload(name, seed=spec.seed + rank)
+    nl = len(layers)
+    prepared = []
+    for lt in layers:
+        w = lt.w.to(dev)
+        qw, sw = cr.convrot_quantize_weight(w, lt.spec.group)     # offline step
+        b = None if lt.b is None else lt.b.to(dev)
+        del w
+        prepared.append((lt.spec, qw, sw, b))
+    x0 = layers[0].x.to(dev)
+
+    step_bytes = sum(4 * sp.M * sp.K + sp.N * (sp.K // 2 + 6) + 2 * sp.M * sp.N
+                     for sp, *_ in prepared)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = 1 if step_bytes >= 2 * l2 else min(64, -(-2 * l2 // step_bytes))
+
+    class Copy:
+        pass
+
+    copies = []
+    for r in range(R):
+        c = Copy()
+        c.w = [(sp, qw.clone(), sw.clone(), None if b is None else b.clone())
+               for sp, qw, sw, b in prepared]
+        c.acts, c.ws, c.xr, c.outs = [x0.clone()], [], [], []
+        for i, (sp, *_) in enumerate(prepared):
+            ws = torch.empty(cr.convrot_w4a16_workspace_size(sp.M, sp.K), dtype=torch.uint8, device=dev)
+            c.ws.append(ws)
+            c.xr.append(ws[:sp.M * sp.K * 2].view(torch.bfloat16).view(sp.M, sp.K))
+            c.outs.append(torch.empty(sp.M, sp.N, dtype=torch.bfloat16, device=dev))
+            if i + 1 < nl:
+                c.acts.append(c.outs[i])
+        copies.append(c)
+
+    def step(c):
+        for i, (sp, qw, sw, b) in enumerate(c.w):
+            cr.convrot_w4a16_linear(c.acts[i], qw, sw, b, sp.group, c.ws[i], c.outs[i])
+
+    def rot_only(c, i):
+        cr.convrot_w4a16_prepare_act(c.acts[i], c.w[i][0].group, out=c.xr[i])
+
+    def gemm_only(c, i):
+        sp, qw, sw, b = c.w[i]
+        cr.convrot_w4a16_linear_prepared(c.xr[i], qw, sw, b, out=c.outs[i])
+
+    for k in range(max(args.warmup, R)):
+        step(copies[k % R])
+        for i in range(nl):
+            rot_only(copies[k % R], i)
+            gemm_only(copies[k % R], i)
+    torch.cuda.synchronize()
+    if cr.convrot_w4a16_check_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    def capture(fn, *a):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn(*a)
+        return g
+
+    def capture_all(fn, *a):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for c in copies:
+                fn(c, *a)
+        return g
+
+    progs = {"step": (step, ())}
+    for i in range(nl):
+        progs[("rot", i)] = (rot_only, (i,))
+        progs[("gemm", i)] = (gemm_only, (i,))
+    graphs = {key: ([capture(fn, c, *a) for c in copies], capture_all(fn, *a))
+              for key, (fn, a) in progs.items()}
+    for one, every in graphs.values():
+        for g in one + [every]:
+            g.replay()
+    torch.cuda.synchronize()
+
+    def timed(key, steps):
+        one, every = graphs[key]
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps // R):
+            every.replay()
+        for j in range(steps % R):
+            one[j].replay()
+        b.record()
+        b.synchronize()
+        return a.elapsed_time(b)
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = str(local)
+    with ClockSampler(gpu_id) as clocks:
+        local_ms = timed("step", args.steps)
+        torch.cuda.synchronize()
+        clocks.mark_end()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    status = cr.convrot_w4a16_check_device_error()
+    if status != 0:
+        raise RuntimeError(f"device error status {status} in the timed region")
+
+    rot_avg = [timed(("rot", i), args.steps) / args.steps for i in range(nl)]
+    gemm_avg = [timed(("gemm", i), args.steps) / args.steps for i in range(nl)]
+    flops_step = spec.ops                       # 2 M N K per layer
+    t_max, flops_total = aggregate(local_ms, flops_step * args.steps, dev)
+    value = flops_total / (t_max * 1e-3) / 1e12
+    tokens_s = spec.tokens * world * args.steps / (t_max * 1e-3)
+
+    peaks = _peaks()
+    gemm_tf = [2 * sp.M * sp.N * sp.K / (g * 1e-3) / 1e12 for (sp, *_), g in zip(prepared, gemm_avg)]
+    gemm_gbs = [GEMM16_BYTES(sp.M, sp.N, sp.K) / (g * 1e-3) / 1e9 for (sp, *_), g in zip(prepared, gemm_avg)]
+    rot_gbs = [ROT16_BYTES(sp.M, sp.K) / (r * 1e-3) / 1e9 for (sp, *_), r in zip(prepared, rot_avg)]
+    if sum(gemm_avg) >= sum(rot_avg):
+        i = max(range(nl), key=lambda j: gemm_avg[j])
+        sp = prepared[i][0]
+        # the bound of this shape: the larger of its tensor time and its byte time
+        t_tensor = 2 * sp.M * sp.N * sp.K / (peaks["bf16"] * 1e12)
+        t_bytes = GEMM16_BYTES(sp.M, sp.N, sp.K) / (peaks["hbm"] * 1e9)
+        if t_tensor >= t_bytes:
+            roof = {"kernel": "w4a16_gemm_kernel", "bound": "tensor", "achieved": round(gemm_tf[i], 2),
+                    "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": round(gemm_tf[i] / peaks["bf16"], 4),
+                    "traffic": None,
+                    "note": "bf16 tensor ops (2 per multiply-add) of the bf16 x INT4 GEMM; peak = "
+                            f"measured bf16 burst ({peaks['src']})"}
+        else:
+            roof = {"kernel": "w4a16_gemm_kernel", "bound": "hbm", "achieved": round(gemm_gbs[i], 1),
+                    "peak": peaks["hbm"], "unit": "GB/s", "frac": round(gemm_gbs[i] / peaks["hbm"], 4),
+                    "traffic": None,
+                    "note": "algorithmic bytes 2MK (xr) + NK/2 + 4N + 2N + 2MN; HBM peak "
+                            f"{peaks['src']}"}
+    else:
+        i = max(range(nl), key=lambda j: rot_avg[j])
+        roof = {"kernel": "rotate_bf16_kernel", "bound": "hbm", "achieved": round(rot_gbs[i], 1),
+                "peak": peaks["hbm"], "unit": "GB/s", "frac": round(rot_gbs[i] / peaks["hbm"], 4),
+                "traffic": None, "note": f"algorithmic bytes 4MK; HBM peak {peaks['src']}"}
+
+    # end to end: pinned host x in, pinned host y out, copies inside the interval
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    x_host = layers[0].x.pin_memory()
+    y_host = torch.empty(prepared[-1][0].M, prepared[-1][0].N, dtype=torch.bfloat16).pin_memory()
+    c = copies[0]
+    e2e_steps = max(3, min(args.steps, 200))
+
+    def e2e_step():
+        c.acts[0].copy_(x_host, non_blocking=True)
+        step(c)
+        y_host.copy_(c.outs[-1], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(e2e_steps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in ev)
+    t_e2e, fl_e2e = aggregate(e2e_ms, flops_step * e2e_steps, dev)
+
+    line = {
+        "metric": METRIC_W4A16, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded bf16, shapes and distributions of the workload; no weights)",
+        "config": {"workload": name, "variant": "w4a16",
+                   "layers": [f"{l.M}x{l.K}->{l.N} g{l.group}" for l in spec.layers],
+                   "tokens_per_rank": spec.tokens,
+                   "l2": f"cold: steps cycle through {R} copies of all step data "
+                         f"({R * step_bytes / 2**20:.0f} MiB >= 2 x L2)",
+                   "launch": f"CUDA graphs of {R} steps (each copy once), replayed back to back",
+                   "parallelism": f"dp{world}"},
+        "tokens_per_s": round(tokens_s, 1),
+        "bf16_peak_frac_path": round(value / world / peaks["bf16"], 4),
+        "gemm_tflops": [round(v, 2) for v in gemm_tf],
+        "gemm_gbs": [round(v, 1) for v in gemm_gbs],
+        "rotate_gbs": [round(v, 1) for v in rot_gbs],
+        "rotate_hbm_frac": [round(v / peaks["hbm"], 4) for v in rot_gbs],
+        "roofline": roof,
+        "e2e": {"value": round(fl_e2e / (t_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": prepared[0][0].M * prepared[0][0].K * 2,
+                "d2h_bytes_per_step": prepared[-1][0].M * prepared[-1][0].N * 2,
+                "call": "pinned host x -> device, convrot_w4a16_linear per layer, y -> pinned "
+                        "host, one stream, L2 flushed before each step"},
+        "gpu_launches": 2 * nl * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0:
+        line["cpu_baseline"] = (cpu_baseline(name, args.cpu_seconds, "w4a16")
+                                if world == 1 and not args.no_cpu else None)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def run_e2e(cr, prepared, spec, dev, stream, flush, args):
     """The public host-buffer path: pinned x in, pinned y out, through
     HostPipeline (row chunks; H2D, convrot_linear per layer and D2H overlap
@@ -446,10 +686,12 @@ def run_e2e(cr, prepared, spec, dev, stream, flush, args):
 
 class OracleSampler:
     """The oracle's per-call work on a sample of token rows: prepare those
-    activation rows, integer GEMM against the prepared weights, epilogue.
-    Weight preparation is offline (done once here, untimed), as on the GPU."""
+    activation rows, integer GEMM against the prepared weights, epilogue
+    (W4A16: rotate and round those rows, fp64 GEMM, epilogue).  Weight
+    preparation is offline (done once here, untimed), as on the GPU."""
 
-    def __init__(self, name):
+    def __init__(self, name, variant="w4a4"):
+        self.variant = variant
         import oracle as O
         O.build()
         self.O = O
@@ -465,8 +707,11 @@ class OracleSampler:
     def run(self, rows):
         O, sp = self.O, self.sp
         t0 = time.perf_counter()
-        px, sx = O.prepare_rows(self.xb[:rows], sp.group)
-        O.epilogue(O.gemm(px, self.pw, sp.K), sx, self.sw, self.bb)
+        if self.variant == "w4a16":
+            O.w4a16_linear(self.xb[:rows], self.pw, self.sw, self.bb, sp.group)
+        else:
+            px, sx = O.prepare_rows(self.xb[:rows], sp.group)
+            O.epilogue(O.gemm(px, self.pw, sp.K), sx, self.sw, self.bb)
         return time.perf_counter() - t0
 
     def calibrate(self, seconds):
@@ -487,15 +732,18 @@ class OracleSampler:
 ONE_THREAD_BASELINE = ("small_g256", "outlier_g64")
 
 
-def cpu_baseline(name, seconds):
-    s = OracleSampler(name)
+def cpu_baseline(name, seconds, variant="w4a4"):
+    s = OracleSampler(name, variant)
     rows = s.calibrate(seconds)
     t = s.run(rows)
-    out = {"value": round(s.ops(rows) / t / 1e12, 9), "unit": "TOPS", "cores": s.cores,
+    what = ("rotation + bf16 rounding + fp64 GEMM + epilogue" if variant == "w4a16"
+            else "prep + int64 GEMM + epilogue")
+    out = {"value": round(s.ops(rows) / t / 1e12, 9),
+           "unit": "TFLOP/s" if variant == "w4a16" else "TOPS", "cores": s.cores,
            "kind": "oracle",
-           "sample": f"{rows} of {s.sp.M} token rows of layer {s.layer} (prep + int64 GEMM + "
-                     f"epilogue, weights prepared offline), {t:.1f} s"}
-    if name in ONE_THREAD_BASELINE:
+           "sample": f"{rows} of {s.sp.M} token rows of layer {s.layer} ({what}, weights "
+                     f"prepared offline), {t:.1f} s"}
+    if name in ONE_THREAD_BASELINE and variant == "w4a4":
         s.O.set_num_threads(1)
         try:
             rows1 = s.calibrate(seconds / 4)
@@ -512,7 +760,8 @@ def run_reference(args):
     if rank != 0:
         return
     name = args.workload
-    s = OracleSampler(name)
+    w16 = args.variant == "w4a16"
+    s = OracleSampler(name, args.variant)
     # the whole run (warm-up + steps) stays within about --cpu-seconds x 8
     per_step = args.cpu_seconds * 8 / (args.steps + args.warmup)
     rows = s.calibrate(per_step)
@@ -523,18 +772,21 @@ def run_reference(args):
             total += t
     value = s.ops(rows) * args.steps / total / 1e12
     spec = wl.WORKLOADS[name]
+    unit = "TFLOP/s" if w16 else "TOPS"
+    what = ("rotation + bf16 rounding + fp64 GEMM + epilogue" if w16
+            else "prep + int64 GEMM + epilogue")
     line = {
-        "impl": "reference", "metric": METRIC, "value": round(value, 9), "unit": "TOPS",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "impl": "reference", "metric": METRIC_W4A16 if w16 else METRIC, "value": round(value, 9),
+        "unit": unit, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "s8",
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w16 else "s8",
         "data": "synthetic (seeded bf16, same workload)",
         "config": {"workload": name, "layers": [f"{l.M}x{l.K}->{l.N} g{l.group}" for l in spec.layers],
                    "tokens_per_rank": spec.tokens, "parallelism": "cpu"},
-        "cpu_baseline": {"value": round(value, 9), "unit": "TOPS", "cores": s.cores, "kind": "oracle",
+        "cpu_baseline": {"value": round(value, 9), "unit": unit, "cores": s.cores, "kind": "oracle",
                          "sample": f"each step: {rows} of {s.sp.M} token rows of layer {s.layer} "
-                                   "(prep + int64 GEMM + epilogue, weights prepared offline)"},
-        "e2e": {"value": round(value, 9), "unit": "TOPS", "h2d_bytes_per_step": 0,
+                                   f"({what}, weights prepared offline)"},
+        "e2e": {"value": round(value, 9), "unit": unit, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -550,11 +802,15 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time budget of the oracle baseline")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline")
+    ap.add_argument("--variant", default="w4a4", choices=["w4a4", "w4a16"],
+                    help="w4a16: the bf16-activation variant (include/convrot_w4a16.h)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.variant == "w4a16":
+        run_gpu_w4a16(args)
     else:
         run_gpu(args)
 

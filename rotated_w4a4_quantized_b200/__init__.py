@@ -8,7 +8,10 @@ turns status codes into exceptions.  There is no CPU fallback: if the
 library is missing, importing the ops raises.
 
 Names follow the C ABI: ``convrot_quantize_weight``, ``convrot_prepare_act``,
-``convrot_linear``, ``convrot_linear_prepared`` (plus the test hooks).
+``convrot_linear``, ``convrot_linear_prepared`` (plus the test hooks), and for
+the W4A16 variant (``include/convrot_w4a16.h``, library
+``libconvrot_w4a16.so``) ``convrot_w4a16_prepare_act``,
+``convrot_w4a16_linear`` and ``convrot_w4a16_linear_prepared``.
 """
 from __future__ import annotations
 
@@ -19,6 +22,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libconvrot.so")
+LIB_W4A16_PATH = os.path.join(_HERE, "libconvrot_w4a16.so")
 
 STATUS = {
     0: "CONVROT_OK", 1: "CONVROT_ERR_NULL", 2: "CONVROT_ERR_GROUP", 3: "CONVROT_ERR_SHAPE",
@@ -211,6 +215,88 @@ def convrot_check_device_error(stream=None) -> int:
 def convrot_debug_timeout_probe(timeout_ns: int, stream=None):
     _check(lib().convrot_debug_timeout_probe(int(timeout_ns), _stream(stream)),
            "convrot_debug_timeout_probe")
+
+
+# ---------------------------------------------------------------------------
+# the W4A16 variant (include/convrot_w4a16.h)
+# ---------------------------------------------------------------------------
+
+_lib_w4a16 = None
+
+
+def lib_w4a16() -> ctypes.CDLL:
+    """The loaded W4A16 library; raises if it has not been built."""
+    global _lib_w4a16
+    if _lib_w4a16 is None:
+        if not os.path.exists(LIB_W4A16_PATH):
+            raise RuntimeError(
+                f"{LIB_W4A16_PATH} is missing: build it with "
+                "`python -m rotated_w4a4_quantized_b200.build` (there is no fallback path)")
+        L = ctypes.CDLL(LIB_W4A16_PATH)
+        P, I64, I, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        sigs = {
+            "convrot_w4a16_prepare_act": [P, I64, I64, I, P, P],
+            "convrot_w4a16_linear_prepared": [P, P, P, P, I64, I64, I64, P, P],
+            "convrot_w4a16_linear": [P, P, P, P, I64, I64, I64, I, P, SZ, P, P],
+            "convrot_w4a16_check_device_error": [P],
+        }
+        for name, args in sigs.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ctypes.c_int
+        L.convrot_w4a16_workspace_size.argtypes = [I64, I64]
+        L.convrot_w4a16_workspace_size.restype = SZ
+        _lib_w4a16 = L
+    return _lib_w4a16
+
+
+def convrot_w4a16_prepare_act(x: torch.Tensor, group: int, out=None, stream=None):
+    """bf16 x [M, K] -> bf16 xr [M, K]: the rotated rows, each value rounded
+    once to bf16 (no quantisation)."""
+    _need(x, torch.bfloat16, "x")
+    M, K = x.shape
+    out = torch.empty(M, K, dtype=torch.bfloat16, device=x.device) if out is None else out
+    _check(lib_w4a16().convrot_w4a16_prepare_act(_p(x), M, K, group, _p(out), _stream(stream)),
+           "convrot_w4a16_prepare_act")
+    return out
+
+
+def convrot_w4a16_workspace_size(M: int, K: int) -> int:
+    return int(lib_w4a16().convrot_w4a16_workspace_size(M, K))
+
+
+def convrot_w4a16_linear_prepared(xr, qw, sw, bias, out=None, stream=None):
+    """bf16 xr [M, K] (rotated) x packed INT4 weights -> bf16 y [M, N]."""
+    _need(xr, torch.bfloat16, "xr")
+    M, K = xr.shape
+    N = qw.shape[0]
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=xr.device) if out is None else out
+    _check(lib_w4a16().convrot_w4a16_linear_prepared(_p(xr), _p(qw), _p(sw), _p(bias), M, N, K,
+                                                     _p(out), _stream(stream)),
+           "convrot_w4a16_linear_prepared")
+    return out
+
+
+def convrot_w4a16_linear(x, qw, sw, bias, group: int, workspace=None, out=None, stream=None):
+    """The whole W4A16 layer: bf16 x [M, K] -> bf16 y [M, N] (rotation, then
+    the bf16 x INT4 tensor-core GEMM with scale and bias)."""
+    _need(x, torch.bfloat16, "x")
+    M, K = x.shape
+    N = qw.shape[0]
+    if workspace is None:
+        workspace = torch.empty(max(1, convrot_w4a16_workspace_size(M, K)), dtype=torch.uint8,
+                                device=x.device)
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
+    _check(lib_w4a16().convrot_w4a16_linear(_p(x), _p(qw), _p(sw), _p(bias), M, N, K, group,
+                                            _p(workspace), workspace.numel(), _p(out),
+                                            _stream(stream)), "convrot_w4a16_linear")
+    return out
+
+
+def convrot_w4a16_check_device_error(stream=None) -> int:
+    """Synchronise the stream; return (and clear) the W4A16 library's device
+    error status."""
+    return int(lib_w4a16().convrot_w4a16_check_device_error(_stream(stream)))
 
 
 class HostPipeline:

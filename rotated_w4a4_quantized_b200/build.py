@@ -1,8 +1,11 @@
-"""Build the CUDA library in-tree: rotated_w4a4_quantized_b200/libconvrot.so.
+"""Build the CUDA libraries in-tree: rotated_w4a4_quantized_b200/libconvrot.so
+(the W4A4 layer, include/convrot.h) and libconvrot_w4a16.so (the W4A16
+variant, include/convrot_w4a16.h).
 
     python -m rotated_w4a4_quantized_b200.build [--verbose]
 
-Compiles csrc/convrot.cu (one translation unit) for sm_100a only, with IEEE
+Each library is one translation unit (csrc/convrot.cu, csrc/w4a16.cu)
+compiled for sm_100a only, with IEEE
 fp32 semantics (no fast-math: the epilogue and the quantiser rely on
 correctly rounded multiply, add and divide).  The CUDA runtime is linked
 statically; the driver's tensor-map encoder is looked up at run time, so no
@@ -16,11 +19,16 @@ import subprocess
 import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
+_INC = os.path.join(os.path.dirname(HERE), "include")
 SRC = os.path.join(HERE, "csrc", "convrot.cu")
 DEPS = [os.path.join(HERE, "csrc", f) for f in ("convrot.cu", "gemm.cuh", "prep.cuh", "ptx.cuh",
                                                      "skinny.cuh", "decode.cuh")]
-HEADER = os.path.join(os.path.dirname(HERE), "include", "convrot.h")
+HEADER = os.path.join(_INC, "convrot.h")
 LIB = os.path.join(HERE, "libconvrot.so")
+SRC_W4A16 = os.path.join(HERE, "csrc", "w4a16.cu")
+DEPS_W4A16 = [os.path.join(HERE, "csrc", f) for f in ("w4a16.cu", "prep.cuh", "ptx.cuh")] + [
+    HEADER, os.path.join(_INC, "convrot_w4a16.h")]
+LIB_W4A16 = os.path.join(HERE, "libconvrot_w4a16.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -37,24 +45,37 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found: the CUDA library cannot be built")
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str, deps) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
-    return any(os.path.getmtime(p) > t for p in DEPS + [HEADER])
+    t = os.path.getmtime(lib)
+    return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not stale():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, SRC, "-o", tmp]
+def stale() -> bool:
+    return _stale(LIB, DEPS + [HEADER]) or _stale(LIB_W4A16, DEPS_W4A16)
+
+
+def _build_one(src: str, lib: str, verbose: bool) -> None:
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [nvcc(), *NVCC_FLAGS, src, "-o", tmp]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Build whichever library is missing or older than its sources; returns
+    the W4A4 library's path."""
+    if force or _stale(LIB, DEPS + [HEADER]):
+        _build_one(SRC, LIB, verbose)
+    if force or _stale(LIB_W4A16, DEPS_W4A16):
+        _build_one(SRC_W4A16, LIB_W4A16, verbose)
     return LIB
 
 
 if __name__ == "__main__":
-    print(build(force=True, verbose="--verbose" in sys.argv))
+    build(force=True, verbose="--verbose" in sys.argv)
+    print(LIB)
+    print(LIB_W4A16)

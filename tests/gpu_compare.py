@@ -103,3 +103,46 @@ def check_outputs(y_gpu_bits, y_ref_bits, tol=None):
     assert not bad.any(), (f"{bad.sum()} outputs outside tolerance, e.g. at {np.argwhere(bad)[:5]}: "
                            f"gpu {g[bad][:5]} ref {r[bad][:5]}")
     return int((err > 0).sum())
+
+
+def bf16_spacing(y: np.ndarray) -> np.ndarray:
+    """Distance between the two bf16 values around |y| (2^-133 below the
+    normal range)."""
+    a = np.abs(np.asarray(y, dtype=np.float64))
+    _, e = np.frexp(a)
+    return np.ldexp(1.0, np.where(e - 1 < -126, -133, e - 8))
+
+
+def check_w4a16_outputs(y_gpu_bits, t, acc, l1, p16, sw, d_acc=0.0, scale_rtol=0.0):
+    """W4A16 outputs against the exact t = sum xr q * sw + b (oracle, fp64):
+    |y - t| <= half the bf16 spacing at max(|t|, |y|) + E, with
+      E = |sw| (2^-18 (p16 + l1) + d_acc) + 2^-23 (|acc sw| + |t|)
+          + scale_rtol |acc sw|.
+    2^-18 (p16 + l1) allows each K = 16 accumulation step of the tensor
+    cores 32 fp32 ulps of (|running sum| + its 16 |products|); d_acc is the
+    exact effect of tie-band inputs; 2^-23 (...) the two fp32 roundings of
+    the epilogue; scale_rtol the weight-scale tolerance when the GPU
+    prepared its own weights.  Returns the share of outputs equal to
+    bf16_rne(t)."""
+    y = bf16_f64(y_gpu_bits)
+    swa = np.abs(np.asarray(sw, np.float64))[None, :]
+    A = 2.0 ** -18 * (p16 + l1)
+    E = swa * (A + d_acc) + 2.0 ** -23 * (np.abs(acc) * swa + np.abs(t)) + scale_rtol * np.abs(acc) * swa
+    tol = 0.5 * np.maximum(bf16_spacing(np.abs(t) + E), bf16_spacing(y)) + E
+    err = np.abs(y - t)
+    bad = err > tol
+    assert not bad.any(), (f"{bad.sum()} outputs outside tolerance, e.g. at {np.argwhere(bad)[:5]}: "
+                           f"gpu {y[bad][:5]} exact {t[bad][:5]} tol {tol[bad][:5]}")
+    sp = bf16_spacing(t)
+    return float(np.mean(np.abs(y - t) <= 0.5 * sp))
+
+
+def w4a16_input_effect(y64_rot, xr_bits, qw_codes, tie_w, rot_band):
+    """d_acc: the largest change of sum_k xr q that the tie-band inputs
+    allow: one bf16 spacing of xr at each activation position of the band
+    (times |q| + 1), one code step at each weight position of the band
+    (times |xr| + one spacing)."""
+    sp = bf16_spacing(y64_rot)
+    qabs = np.abs(qw_codes.astype(np.float64)) + 1.0
+    xabs = np.abs(bf16_f64(xr_bits)) + sp
+    return (rot_band * sp) @ qabs.T + xabs @ tie_w.astype(np.float64).T

@@ -120,3 +120,71 @@ def test_valid_call_without_gpu_reports_cuda_error(L):
         pytest.skip("a GPU is present")
     # Arguments pass validation; the device set-up then fails cleanly.
     assert L.convrot_prepare_act(A, 4, 1024, 64, B, B, None) == 6
+
+
+# ---------------------------------------------------------------- W4A16 library
+
+HEADER_W4A16 = os.path.join(ROOT, "include", "convrot_w4a16.h")
+
+
+@pytest.fixture(scope="module")
+def L16():
+    from rotated_w4a4_quantized_b200 import build
+    build.build()
+    return cr.lib_w4a16()
+
+
+def _declared_w4a16():
+    text = open(HEADER_W4A16).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(convrot_w4a16_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_w4a16_header_declares_the_boundary():
+    assert _declared_w4a16() == sorted([
+        "convrot_w4a16_prepare_act", "convrot_w4a16_workspace_size",
+        "convrot_w4a16_linear_prepared", "convrot_w4a16_linear",
+        "convrot_w4a16_check_device_error"])
+
+
+def test_w4a16_library_exports_every_declared_symbol(L16):
+    for name in _declared_w4a16():
+        assert hasattr(L16, name), name
+
+
+def test_w4a16_workspace_size(L16):
+    assert cr.convrot_w4a16_workspace_size(0, 1024) == 0
+    assert cr.convrot_w4a16_workspace_size(3, 1024) == 6144
+    assert cr.convrot_w4a16_workspace_size(1, 64) == 256
+    assert cr.convrot_w4a16_workspace_size(5, 192) == 2048
+
+
+def test_w4a16_host_validation_without_device(L16):
+    s = None
+    assert L16.convrot_w4a16_prepare_act(A, 4, 1024, 128, B, s) == 2     # group
+    assert L16.convrot_w4a16_prepare_act(A, 4, 1000, 64, B, s) == 3      # K % group
+    assert L16.convrot_w4a16_prepare_act(A, 4, 64, 256, B, s) == 3
+    assert L16.convrot_w4a16_prepare_act(None, 0, 1024, 64, None, s) == 0
+    assert L16.convrot_w4a16_prepare_act(None, 4, 1024, 64, B, s) == 1
+    assert L16.convrot_w4a16_prepare_act(U, 4, 1024, 64, B, s) == 4
+    # prepared GEMM: K % 64, K range, sizes, NULL, alignment
+    assert L16.convrot_w4a16_linear_prepared(A, B, B, None, 4, 8, 96, B, s) == 3
+    assert L16.convrot_w4a16_linear_prepared(A, B, B, None, 4, 8, 32768 + 64, B, s) == 3
+    assert L16.convrot_w4a16_linear_prepared(A, B, B, None, -1, 8, 1024, B, s) == 3
+    assert L16.convrot_w4a16_linear_prepared(None, None, None, None, 0, 8, 1024, None, s) == 0
+    assert L16.convrot_w4a16_linear_prepared(A, None, B, None, 4, 8, 1024, B, s) == 1
+    assert L16.convrot_w4a16_linear_prepared(A, B, B, U, 4, 8, 1024, B, s) == 4
+    assert L16.convrot_w4a16_linear_prepared(A, B, U, None, 4, 8, 1024, B, s) == 4
+    # whole layer: workspace size and alignment
+    ws = cr.convrot_w4a16_workspace_size(4, 1024)
+    assert L16.convrot_w4a16_linear(A, B, B, None, 4, 8, 1024, 64, A, ws - 1, B, s) == 5
+    assert L16.convrot_w4a16_linear(A, B, B, None, 4, 8, 1024, 64, U, ws, B, s) == 5
+    assert L16.convrot_w4a16_linear(A, B, B, None, 4, 8, 1024, 32, A, ws, B, s) == 2
+    assert L16.convrot_w4a16_linear(None, None, None, None, 4, 0, 1024, 64, None, 0, None, s) == 0
+
+
+def test_w4a16_valid_call_without_gpu_reports_cuda_error(L16):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert L16.convrot_w4a16_prepare_act(A, 4, 1024, 64, B, None) == 6
