@@ -13,11 +13,13 @@
 //   rotate_bf16_kernel  the W4A4 prep kernel's row loop and butterflies
 //                       (prep.cuh helpers), writing each rotated value
 //                       rounded to bf16 instead of quantising the row;
-//   w4a16_gemm_kernel   persistent 128 x 128 output tiles, one CTA per SM.
+//   w4a16_gemm_kernel   persistent output tiles of 128 weight rows by TN
+//                       token rows (TN = 128; 16, 32 or 64 for few tokens,
+//                       with the weights on the MMA's M side), one CTA per SM.
 //
 // GEMM roles (448 threads):
 //   warp 0        TMA producer: per stage (two 64-deep K-blocks) the two
-//                 xr tiles [128 rows x 128 B], 128-byte swizzled, straight
+//                 xr tiles [TN rows x 128 B], 128-byte swizzled, straight
 //                 into the MMA layout, and the packed weight tile
 //                 [128 rows x 64 B];
 //   warp 1        TMEM allocator and MMA issuer (one thread): 4 MMAs of
@@ -25,7 +27,7 @@
 //   warps 2..5    epilogue, one per TMEM lane quarter: tcgen05.ld, scale,
 //                 bias, bf16, stores;
 //   warps 6..13   widening: packed codes -> bf16 codes in the swizzled
-//                 K-major layout of the MMA's B operand.
+//                 K-major layout of the MMA's weight operand.
 //
 // Widening a code to bf16 without the conversion unit: for a nibble u
 // (the 4-bit two's complement code c), u ^ 8 = c + 8 in [0, 15], and the
@@ -125,32 +127,50 @@ rotate_bf16_kernel(const uint16_t *__restrict__ x, int M, int K, uint16_t *__res
 
 // ------------------------------------------------------------------ GEMM
 
-constexpr int BM = 128;                  // activation rows per tile (MMA M)
-constexpr int BN = 128;                  // weight rows per tile (MMA N)
+constexpr int WR = 128;                  // weight rows per tile
 constexpr int KB = 64;                   // K per block: one 128-byte bf16 row
-constexpr int KBS = 2;                   // K-blocks per stage
-constexpr int PKB = KB * KBS / 2;        // packed weight bytes per row per stage
-constexpr int SP = 4;                    // ring stages (xr + packed weights)
-constexpr int SU = 2;                    // widened weight stages
-constexpr int A_KB = BM * 128;           // one xr K-block tile (16 KB)
-constexpr int A_ST = KBS * A_KB;
-constexpr int PB_ST = BN * PKB;          // packed weights of a stage (8 KB)
-constexpr int UB_KB = BN * 128;          // one widened K-block tile (16 KB)
-constexpr int UB_ST = KBS * UB_KB;
+constexpr int UB_KB = WR * 128;          // one widened K-block tile (16 KB)
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpEpi0 = 2, kEpiWarps = 4;
 constexpr int kWarpUnp0 = kWarpEpi0 + kEpiWarps, kUnpWarps = 8;
 constexpr int kThreads = (kWarpUnp0 + kUnpWarps) * 32;   // 448
-constexpr int OFF_A = 0;                                  // 1024-aligned tiles first
-constexpr int OFF_UB = OFF_A + SP * A_ST;
-constexpr int OFF_PB = OFF_UB + SU * UB_ST;
-constexpr int OFF_BAR = OFF_PB + SP * PB_ST;
-constexpr int NUM_BARS = 2 * SP + 2 * SU + 5;
-constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;          // + slack for 1024 alignment
-constexpr int TMEM_COLS = 2 * BN;                         // two fp32 accumulators
-static_assert(SMEM_BYTES <= 232448, "exceeds the per-CTA shared memory limit");
-static_assert((BN * 4) % (kUnpWarps * 32) == 0, "the widening covers whole stages");
-static_assert(A_KB % 1024 == 0 && UB_KB % 1024 == 0, "swizzled tiles stay 1024-aligned");
+
+// Tile forms.  TN = token rows of a tile.
+//   !SWAP (TN = 128): the token rows are the MMA's M side (A = xr, loaded by
+//     TMA) and the 128 weight rows its N side (B = widened weights).
+//   SWAP (TN = 16, 32, 64: few tokens): the 128 weight rows are the M side
+//     (A = widened weights) and the token rows the N side (B = xr), so a
+//     decode-size call still streams its weights through 128-row tiles.
+// The few-token tiles use the room their small token tiles leave for a
+// deeper ring of packed weights (8 or 6 stages).  Measured on 1 x 4096 ->
+// 14336: one K-block per stage with six widened stages and a 12-deep ring
+// was slower (897 against 1000 GB/s of weight stream) than two K-blocks per
+// stage with two widened stages, so both forms keep the latter.
+template <int TN, bool SWAP>
+struct Cfg {
+    static_assert(SWAP ? (TN == 16 || TN == 32 || TN == 64) : TN == 128, "tile forms");
+    static constexpr int MMA_N = SWAP ? TN : WR;
+    static constexpr int KBS = 2;                        // K-blocks per stage
+    static constexpr int PKB = KB * KBS / 2;             // packed weight bytes per row per stage
+    static constexpr int CPR = PKB / 16;                  // 16-byte packed chunks per row
+    static constexpr int SU = 2;                         // widened weight stages
+    static constexpr int PB_ST = WR * PKB;               // packed weights of a stage
+    static constexpr int UB_ST = KBS * UB_KB;            // widened weights of a stage
+    static constexpr int XR_KB = TN * 128;               // one xr K-block tile
+    static constexpr int XR_ST = KBS * XR_KB;
+    static constexpr int SP = !SWAP ? 4 : TN <= 32 ? 8 : 6;   // ring stages (xr + packed weights)
+    static_assert((WR * CPR) % (kUnpWarps * 32) == 0, "the widening covers whole stages");
+    static constexpr int ACC = MMA_N < 32 ? 32 : MMA_N;  // TMEM columns per accumulator
+    static constexpr int TMEM_COLS = 2 * ACC;            // two accumulators (power of two)
+    static constexpr int OFF_XR = 0;                      // 1024-aligned tiles first
+    static constexpr int OFF_UB = OFF_XR + SP * XR_ST;
+    static constexpr int OFF_PB = OFF_UB + SU * UB_ST;
+    static constexpr int OFF_BAR = OFF_PB + SP * PB_ST;
+    static constexpr int NUM_BARS = 2 * SP + 2 * SU + 5;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + slack for 1024 alignment
+    static_assert(SMEM_BYTES <= 232448, "exceeds the per-CTA shared memory limit");
+    static_assert(XR_KB % 1024 == 0 && UB_KB % 1024 == 0, "swizzled tiles stay 1024-aligned");
+};
 
 // Instruction descriptor of tcgen05.mma kind::f16: D fp32, A and B bf16,
 // both K-major, M x N.
@@ -207,17 +227,20 @@ __device__ __forceinline__ void widen_word(uint32_t w, uint32_t (&o)[4]) {
     o[3] = widen_pair(w, s, 0x7733u);
 }
 
-// tmA: xr bf16 [M][K], box 64 x 128, 128-byte swizzle.  tmB: qw u8
+// tmA: xr bf16 [M][K], box 64 x TN, 128-byte swizzle.  tmB: qw u8
 // [N][K/2], box 64 B x 128, no swizzle.  K % 64 == 0.
+template <int TN, bool SWAP>
 __global__ void __launch_bounds__(kThreads, 1)
 w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   int M, int N, int K, const float *__restrict__ sw,
                   const uint16_t *__restrict__ bias, uint16_t *__restrict__ y) {
+    using C = Cfg<TN, SWAP>;
+    constexpr int SP = C::SP, SU = C::SU, KBS = C::KBS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = ptx::smem_u32(smem);
-    const uint32_t bar0 = sbase + OFF_BAR;
+    const uint32_t bar0 = sbase + C::OFF_BAR;
     auto full_p = [&](int s) { return bar0 + 8u * s; };
     auto empty_p = [&](int s) { return bar0 + 8u * (SP + s); };
     auto full_u = [&](int s) { return bar0 + 8u * (2 * SP + s); };
@@ -225,8 +248,8 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     auto acc_full = [&](int b) { return bar0 + 8u * (2 * SP + 2 * SU + b); };
     auto acc_empty = [&](int b) { return bar0 + 8u * (2 * SP + 2 * SU + 2 + b); };
     const uint32_t drain_bar = bar0 + 8u * (2 * SP + 2 * SU + 4);
-    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + OFF_MISC);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -253,7 +276,7 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         ptx::tma_prefetch_desc(&tmB);
     }
     if (warp == kWarpMma) {
-        ptx::tmem_alloc<1>(sbase + OFF_MISC, TMEM_COLS);
+        ptx::tmem_alloc<1>(sbase + C::OFF_MISC, C::TMEM_COLS);
         ptx::tmem_relinquish<1>();
     }
     ptx::tc_fence_before();
@@ -263,8 +286,8 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     // xr comes from the preceding kernel (programmatic dependent launch)
     ptx::grid_dependency_wait();
 
-    const int tiles_a = (M + BM - 1) / BM;
-    const int tiles_b = (N + BN - 1) / BN;
+    const int tiles_a = (M + TN - 1) / TN;           // token tiles
+    const int tiles_b = (N + WR - 1) / WR;           // weight tiles
     const int num_tiles = tiles_a * tiles_b;
     const int first_tile = static_cast<int>(blockIdx.x);
     const int tile_step = static_cast<int>(gridDim.x);
@@ -284,11 +307,12 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                 // second xr tile is not loaded (and not multiplied); the
                 // packed tile's missing half reads as zeros
                 const int nk = min(KBS, nkb - kp * KBS);
-                ptx::mbar_arrive_expect_tx(full_p(ps), static_cast<uint32_t>(nk * A_KB + PB_ST));
+                ptx::mbar_arrive_expect_tx(full_p(ps), static_cast<uint32_t>(nk * C::XR_KB + C::PB_ST));
                 for (int i = 0; i < nk; ++i)
-                    ptx::tma_load_2d(sbase + OFF_A + ps * A_ST + i * A_KB, &tmA, full_p(ps),
-                                     (kp * KBS + i) * KB, ta * BM);
-                ptx::tma_load_2d(sbase + OFF_PB + ps * PB_ST, &tmB, full_p(ps), kp * PKB, tb * BN);
+                    ptx::tma_load_2d(sbase + C::OFF_XR + ps * C::XR_ST + i * C::XR_KB, &tmA,
+                                     full_p(ps), (kp * KBS + i) * KB, ta * TN);
+                ptx::tma_load_2d(sbase + C::OFF_PB + ps * C::PB_ST, &tmB, full_p(ps), kp * C::PKB,
+                                 tb * WR);
                 if (++ps == SP) { ps = 0; ph ^= 1; }
             }
         }
@@ -301,7 +325,7 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         }
     } else if (warp == kWarpMma) {
         const bool issuer = lane == 0;
-        constexpr uint32_t idesc = idesc_bf16(BM, BN);
+        constexpr uint32_t idesc = idesc_bf16(128, C::MMA_N);
         int ps = 0, us = 0;
         uint32_t pph = 0, uph = 0;
         int local = 0;
@@ -311,20 +335,22 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             const uint32_t aph = (local >> 1) & 1;
             if (!ptx::mbar_wait(acc_empty(b), aph ^ 1, abort_flag)) { ok = false; break; }
             ptx::tc_fence_after();
-            const uint32_t d = tmem_base + static_cast<uint32_t>(b * BN);
+            const uint32_t d = tmem_base + static_cast<uint32_t>(b * C::ACC);
             for (int kp = 0; kp < num_kp; ++kp) {
                 if (!ptx::mbar_wait(full_p(ps), pph, abort_flag)) { ok = false; break; }
                 if (!ptx::mbar_wait(full_u(us), uph, abort_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
                 const int nk = min(KBS, nkb - kp * KBS);
-                const uint32_t a0 = sbase + OFF_A + ps * A_ST;
-                const uint32_t b0 = sbase + OFF_UB + us * UB_ST;
+                const uint32_t x0 = sbase + C::OFF_XR + ps * C::XR_ST;
+                const uint32_t w0 = sbase + C::OFF_UB + us * C::UB_ST;
                 for (int i = 0; i < nk; ++i) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        mma_bf16_ss(d, ptx::sw128_kmajor_desc(a0 + i * A_KB + 32 * j),
-                                    ptx::sw128_kmajor_desc(b0 + i * UB_KB + 32 * j), idesc,
+                    for (int j = 0; j < 4; ++j) {
+                        const uint64_t xd = ptx::sw128_kmajor_desc(x0 + i * C::XR_KB + 32 * j);
+                        const uint64_t wd = ptx::sw128_kmajor_desc(w0 + i * UB_KB + 32 * j);
+                        mma_bf16_ss(d, SWAP ? wd : xd, SWAP ? xd : wd, idesc,
                                     (kp | i | j) != 0 ? 1u : 0u);
+                    }
                 }
                 ptx::tc_commit<1>(empty_p(ps));
                 ptx::tc_commit<1>(empty_u(us));
@@ -347,16 +373,43 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             const int ta = tile % tiles_a, tb = tile / tiles_a;
             const int b = local & 1;
             const uint32_t aph = (local >> 1) & 1;
-            const int m = ta * BM + quarter * 32 + lane;      // this lane's output row
             if (!ptx::mbar_wait(acc_full(b), aph, abort_flag)) break;
             ptx::tc_fence_after();
+            if constexpr (SWAP) {
+                // lane = output column n (a weight row), columns = tokens
+                const int n = tb * WR + quarter * 32 + lane;
+                const float swn = n < N ? sw[n] : 0.0f;
+                const float bn = (bias && n < N) ? __uint_as_float(static_cast<uint32_t>(bias[n]) << 16)
+                                                 : 0.0f;
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                const int n0 = tb * BN + c0;
+                for (int c0 = 0; c0 < C::ACC; c0 += 32) {
+                    uint32_t v[32];
+                    __syncwarp();   // tcgen05.ld is warp-collective
+                    ptx::tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                                static_cast<uint32_t>(b * C::ACC + c0),
+                                            v);
+                    ptx::tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int m = ta * TN + c0 + j;
+                        if (c0 + j < TN && m < M && n < N)
+                            y[static_cast<size_t>(m) * N + n] = static_cast<uint16_t>(
+                                bf16x2_rn(__fadd_rn(__fmul_rn(__uint_as_float(v[j]), swn), bn), 0.0f));
+                    }
+                }
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(acc_empty(b));
+                continue;
+            }
+            const int m = ta * TN + quarter * 32 + lane;      // this lane's output row
+#pragma unroll 1
+            for (int c0 = 0; c0 < WR; c0 += 32) {
+                const int n0 = tb * WR + c0;
                 uint32_t v[32];
                 __syncwarp();   // tcgen05.ld is warp-collective
                 ptx::tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                            static_cast<uint32_t>(b * BN + c0),
+                                            static_cast<uint32_t>(b * C::ACC + c0),
                                         v);
                 ptx::tmem_ld_wait();
                 // column parameters: lane l fetches column n0 + l, then broadcast
@@ -395,27 +448,29 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         }
     } else {
         // ------------------------------------------------------------ widening
-        // Stage = BN rows x 4 packed chunks of 16 bytes (chunk p = codes
+        // Stage = WR rows x CPR packed chunks of 16 bytes (chunk p = codes
         // 32p .. 32p + 31 = half p & 1 of K-block p >> 1).  Thread ut takes
-        // chunks ut, ut + 256, ...: a quarter warp reads two whole 64-byte
-        // rows (conflict-free) and writes 8 distinct 16-byte positions of
-        // the 128-byte swizzle pattern per store (the store order rotates by
-        // 2 with the K-block, and the two rows have opposite swizzle parity).
+        // chunks ut, ut + 256, ...: a quarter warp reads 128 contiguous
+        // packed bytes (two 64-byte rows, or four 32-byte rows) and writes 8
+        // distinct 16-byte positions of the 128-byte swizzle pattern per
+        // store: with two K-blocks per stage the store order rotates by 2
+        // with the K-block and the two rows have opposite swizzle parity;
+        // with one, the four rows' swizzle phases differ in their low bits.
         const int ut = threadIdx.x - kWarpUnp0 * 32;
         const int total = my_tiles * num_kp;
-        constexpr int kPer = BN * 4 / (kUnpWarps * 32);
+        constexpr int kPer = WR * C::CPR / (kUnpWarps * 32);
         for (int n = 0; n < total; ++n) {
             const int ps = n % SP, us = n % SU;
             const uint32_t pph = (n / SP) & 1, uph = (n / SU) & 1;
             if (!ptx::mbar_wait(full_p(ps), pph, abort_flag)) break;
             if (!ptx::mbar_wait(empty_u(us), uph ^ 1, abort_flag)) break;
-            const uint32_t pb = sbase + OFF_PB + ps * PB_ST;
-            const uint32_t ub = sbase + OFF_UB + us * UB_ST;
+            const uint32_t pb = sbase + C::OFF_PB + ps * C::PB_ST;
+            const uint32_t ub = sbase + C::OFF_UB + us * C::UB_ST;
 #pragma unroll
             for (int it = 0; it < kPer; ++it) {
                 const int idx = ut + it * kUnpWarps * 32;
-                const int row = idx >> 2, p = idx & 3;
-                const uint4 w = lds128(pb + static_cast<uint32_t>(row * PKB + p * 16));
+                const int row = idx / C::CPR, p = idx % C::CPR;
+                const uint4 w = lds128(pb + static_cast<uint32_t>(row * C::PKB + p * 16));
                 const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
                 const int kbi = p >> 1;
                 const uint32_t half = static_cast<uint32_t>(p & 1);
@@ -445,7 +500,7 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     ptx::tc_fence_after();
     if (warp == kWarpMma) {
         __syncwarp();
-        ptx::tmem_dealloc<1>(tmem_base, TMEM_COLS);
+        ptx::tmem_dealloc<1>(tmem_base, C::TMEM_COLS);
     }
 }
 
@@ -516,7 +571,10 @@ convrot_status device_setup(int *dev_out) {
     bool ok = true;
     ok &= set_smem(w4a16::rotate_bf16_kernel<64>, kRotSmemMax);
     ok &= set_smem(w4a16::rotate_bf16_kernel<256>, kRotSmemMax);
-    ok &= set_smem(w4a16::w4a16_gemm_kernel, w4a16::SMEM_BYTES);
+    ok &= set_smem(w4a16::w4a16_gemm_kernel<128, false>, w4a16::Cfg<128, false>::SMEM_BYTES);
+    ok &= set_smem(w4a16::w4a16_gemm_kernel<16, true>, w4a16::Cfg<16, true>::SMEM_BYTES);
+    ok &= set_smem(w4a16::w4a16_gemm_kernel<32, true>, w4a16::Cfg<32, true>::SMEM_BYTES);
+    ok &= set_smem(w4a16::w4a16_gemm_kernel<64, true>, w4a16::Cfg<64, true>::SMEM_BYTES);
     st.num_sms = sms;
     st.status = ok ? CONVROT_OK : CONVROT_ERR_CUDA;
     st.ready = true;
@@ -575,15 +633,17 @@ convrot_status launch_rotate(int num_sms, const void *x, int64_t M, int64_t K, i
     return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 
-convrot_status launch_gemm(int num_sms, const void *xr, const uint8_t *qw, const float *sw,
-                           const void *bias, int64_t M, int64_t N, int64_t K, void *y,
-                           cudaStream_t stream) {
+// TN token rows per tile; SWAP: the few-token form (weights on the MMA's M side).
+template <int TN, bool SWAP>
+convrot_status launch_gemm_cfg(int num_sms, const void *xr, const uint8_t *qw, const float *sw,
+                               const void *bias, int64_t M, int64_t N, int64_t K, void *y,
+                               cudaStream_t stream) {
+    using C = w4a16::Cfg<TN, SWAP>;
     CUtensorMap tmA, tmB;
     {
         const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
         const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-        const cuuint32_t box[2] = {static_cast<cuuint32_t>(w4a16::KB),
-                                   static_cast<cuuint32_t>(w4a16::BM)};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(w4a16::KB), static_cast<cuuint32_t>(TN)};
         const cuuint32_t estr[2] = {1, 1};
         if (g_encode(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(xr), dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -594,8 +654,8 @@ convrot_status launch_gemm(int num_sms, const void *xr, const uint8_t *qw, const
     {
         const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
         const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
-        const cuuint32_t box[2] = {static_cast<cuuint32_t>(w4a16::PKB),
-                                   static_cast<cuuint32_t>(w4a16::BN)};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(C::PKB),
+                                   static_cast<cuuint32_t>(w4a16::WR)};
         const cuuint32_t estr[2] = {1, 1};
         if (g_encode(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(qw), dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -603,12 +663,12 @@ convrot_status launch_gemm(int num_sms, const void *xr, const uint8_t *qw, const
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return CONVROT_ERR_CUDA;
     }
-    const int64_t tiles = ((M + w4a16::BM - 1) / w4a16::BM) * ((N + w4a16::BN - 1) / w4a16::BN);
+    const int64_t tiles = ((M + TN - 1) / TN) * ((N + w4a16::WR - 1) / w4a16::WR);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(w4a16::kThreads);
-    cfg.dynamicSmemBytes = w4a16::SMEM_BYTES;
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -616,9 +676,21 @@ convrot_status launch_gemm(int num_sms, const void *xr, const uint8_t *qw, const
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(
-        &cfg, w4a16::w4a16_gemm_kernel, tmA, tmB, static_cast<int>(M), static_cast<int>(N),
-        static_cast<int>(K), sw, static_cast<const uint16_t *>(bias), static_cast<uint16_t *>(y));
+        &cfg, w4a16::w4a16_gemm_kernel<TN, SWAP>, tmA, tmB, static_cast<int>(M),
+        static_cast<int>(N), static_cast<int>(K), sw, static_cast<const uint16_t *>(bias),
+        static_cast<uint16_t *>(y));
     return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
+}
+
+// Up to 64 tokens: the weights take the MMA's 128-row side and the tokens a
+// 16-, 32- or 64-wide side; beyond that, 128 x 128 token-by-weight tiles.
+convrot_status launch_gemm(int num_sms, const void *xr, const uint8_t *qw, const float *sw,
+                           const void *bias, int64_t M, int64_t N, int64_t K, void *y,
+                           cudaStream_t stream) {
+    if (M <= 16) return launch_gemm_cfg<16, true>(num_sms, xr, qw, sw, bias, M, N, K, y, stream);
+    if (M <= 32) return launch_gemm_cfg<32, true>(num_sms, xr, qw, sw, bias, M, N, K, y, stream);
+    if (M <= 64) return launch_gemm_cfg<64, true>(num_sms, xr, qw, sw, bias, M, N, K, y, stream);
+    return launch_gemm_cfg<128, false>(num_sms, xr, qw, sw, bias, M, N, K, y, stream);
 }
 
 }  // namespace

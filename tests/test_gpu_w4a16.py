@@ -71,10 +71,14 @@ def test_w4a16_rotation_matches_oracle(group, M, K):
 # step 3: the bf16 x INT4 GEMM with scale and bias
 # ---------------------------------------------------------------------------
 
-GEMM_CASES = [(1, 16, 64, True), (5, 13, 192, False), (100, 200, 320, True),
-              (130, 264, 1088, False), (257, 385, 2048, True), (300, 1000, 4096, True),
-              (128, 128, 32768, False), (1000, 40, 256, True), (256, 256, 128, False),
-              (129, 136, 960, True)]
+# token-by-weight tiles (M > 64) and the few-token forms with the weights on
+# the MMA's M side (16, 32, 64 token columns), with ragged tails everywhere
+GEMM_CASES = [(100, 200, 320, True), (130, 264, 1088, False), (257, 385, 2048, True),
+              (300, 1000, 4096, True), (128, 128, 32768, False), (1000, 40, 256, True),
+              (256, 256, 128, False), (129, 136, 960, True), (65, 72, 192, False),
+              (1, 16, 64, True), (5, 13, 192, False), (16, 14336, 4096, False),
+              (17, 130, 1088, True), (32, 300, 2048, False), (33, 257, 320, True),
+              (64, 1000, 4096, False), (48, 128, 32768, True)]
 
 
 @pytest.mark.parametrize("M,N,K,bias", GEMM_CASES)
@@ -156,8 +160,8 @@ def _sample(n, k, seed):
     return np.array(sorted(picks))
 
 
-@pytest.mark.parametrize("name", ["outlier_g64", "qkv_g256", "skinny_m1_g64", "skinny_m128_g64",
-                                  "square_g256"])
+@pytest.mark.parametrize("name", ["outlier_g64", "qkv_g256", "skinny_m1_g64", "skinny_m16_g64",
+                                  "skinny_m128_g64", "square_g256"])
 def test_w4a16_workload_full_size_sampled(name):
     """The benchmark's workloads at full size, through the same call the
     benchmark's W4A16 line times, compared on sampled rows and columns."""
