@@ -188,3 +188,13 @@ def test_w4a16_valid_call_without_gpu_reports_cuda_error(L16):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert L16.convrot_w4a16_prepare_act(A, 4, 1024, 64, B, None) == 6
+
+
+@pytest.mark.parametrize("attr,loader", [("LIB_PATH", "lib"), ("LIB_W4A16_PATH", "lib_w4a16")])
+def test_missing_library_raises_instead_of_falling_back(monkeypatch, tmp_path, attr, loader):
+    """Without the built CUDA library every op fails loudly: there is no CPU
+    path to fall back to."""
+    monkeypatch.setattr(cr, attr, str(tmp_path / "absent.so"))
+    monkeypatch.setattr(cr, "_lib" if loader == "lib" else "_lib_w4a16", None)
+    with pytest.raises(RuntimeError, match="no fallback"):
+        getattr(cr, loader)()
