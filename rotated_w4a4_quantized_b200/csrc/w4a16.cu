@@ -13,15 +13,16 @@
 //   rotate_bf16_kernel  the W4A4 prep kernel's row loop and butterflies
 //                       (prep.cuh helpers), writing each rotated value
 //                       rounded to bf16 instead of quantising the row;
-//   w4a16_gemm_kernel   persistent output tiles of 128 weight rows by TN
-//                       token rows (TN = 128; 16, 32 or 64 for few tokens,
-//                       with the weights on the MMA's M side), one CTA per SM.
+//   w4a16_gemm_kernel   persistent output tiles, one CTA per SM: 128 token
+//                       rows by 256 weight rows, or for few tokens 128
+//                       weight rows (on the MMA's M side) by 16, 32 or 64
+//                       token rows.
 //
 // GEMM roles (448 threads):
-//   warp 0        TMA producer: per stage (two 64-deep K-blocks) the two
-//                 xr tiles [TN rows x 128 B], 128-byte swizzled, straight
-//                 into the MMA layout, and the packed weight tile
-//                 [128 rows x 64 B];
+//   warp 0        TMA producer: per stage (one or two 64-deep K-blocks)
+//                 the xr tiles [TN rows x 128 B], 128-byte swizzled,
+//                 straight into the MMA layout, and the packed weight tile
+//                 [WT rows x 32 or 64 B];
 //   warp 1        TMEM allocator and MMA issuer (one thread): 4 MMAs of
 //                 K = 16 per K-block into one of two fp32 accumulators;
 //   warps 2..5    epilogue, one per TMEM lane quarter: tcgen05.ld, scale,
@@ -127,38 +128,43 @@ rotate_bf16_kernel(const uint16_t *__restrict__ x, int M, int K, uint16_t *__res
 
 // ------------------------------------------------------------------ GEMM
 
-constexpr int WR = 128;                  // weight rows per tile
 constexpr int KB = 64;                   // K per block: one 128-byte bf16 row
-constexpr int UB_KB = WR * 128;          // one widened K-block tile (16 KB)
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpEpi0 = 2, kEpiWarps = 4;
 constexpr int kWarpUnp0 = kWarpEpi0 + kEpiWarps, kUnpWarps = 8;
 constexpr int kThreads = (kWarpUnp0 + kUnpWarps) * 32;   // 448
 
-// Tile forms.  TN = token rows of a tile.
-//   !SWAP (TN = 128): the token rows are the MMA's M side (A = xr, loaded by
-//     TMA) and the 128 weight rows its N side (B = widened weights).
-//   SWAP (TN = 16, 32, 64: few tokens): the 128 weight rows are the M side
-//     (A = widened weights) and the token rows the N side (B = xr), so a
-//     decode-size call still streams its weights through 128-row tiles.
-// The few-token tiles use the room their small token tiles leave for a
-// deeper ring of packed weights (8 or 6 stages).  Measured on 1 x 4096 ->
-// 14336: one K-block per stage with six widened stages and a 12-deep ring
-// was slower (897 against 1000 GB/s of weight stream) than two K-blocks per
-// stage with two widened stages, so both forms keep the latter.
+// Tile forms.  TN = token rows of a tile, WT = weight rows.
+//   !SWAP (TN = 128, WT = 256): the token rows are the MMA's M side (A = xr,
+//     loaded by TMA) and the 256 weight rows its N side (B = widened
+//     weights).  Both operands come from shared memory, so the wide N side
+//     halves the xr bytes read per MMA flop (a 128 x 128 tile needs the
+//     whole 128 B/cycle of shared-memory bandwidth at the tensor peak).  One
+//     K-block per stage leaves room for five ring stages and three widened
+//     ones beside the 32 KB widened K-block.
+//   SWAP (TN = 16, 32, 64: few tokens; WT = 128): the weight rows are the M
+//     side (A = widened weights) and the token rows the N side (B = xr), so a
+//     decode-size call still streams its weights through 128-row tiles; they
+//     use the room their small token tiles leave for a deeper ring of packed
+//     weights (8 or 6 stages).  Measured on 1 x 4096 -> 14336: one K-block
+//     per stage with six widened stages and a 12-deep ring was slower (897
+//     against 1000 GB/s of weight stream) than two K-blocks per stage with
+//     two widened stages.
 template <int TN, bool SWAP>
 struct Cfg {
     static_assert(SWAP ? (TN == 16 || TN == 32 || TN == 64) : TN == 128, "tile forms");
-    static constexpr int MMA_N = SWAP ? TN : WR;
-    static constexpr int KBS = 2;                        // K-blocks per stage
+    static constexpr int WT = SWAP ? 128 : 256;          // weight rows per tile
+    static constexpr int MMA_N = SWAP ? TN : WT;
+    static constexpr int KBS = SWAP ? 2 : 1;             // K-blocks per stage
     static constexpr int PKB = KB * KBS / 2;             // packed weight bytes per row per stage
     static constexpr int CPR = PKB / 16;                  // 16-byte packed chunks per row
-    static constexpr int SU = 2;                         // widened weight stages
-    static constexpr int PB_ST = WR * PKB;               // packed weights of a stage
+    static constexpr int SU = SWAP ? 2 : 3;              // widened weight stages
+    static constexpr int UB_KB = WT * 128;               // one widened K-block tile
+    static constexpr int PB_ST = WT * PKB;               // packed weights of a stage
     static constexpr int UB_ST = KBS * UB_KB;            // widened weights of a stage
     static constexpr int XR_KB = TN * 128;               // one xr K-block tile
     static constexpr int XR_ST = KBS * XR_KB;
-    static constexpr int SP = !SWAP ? 4 : TN <= 32 ? 8 : 6;   // ring stages (xr + packed weights)
-    static_assert((WR * CPR) % (kUnpWarps * 32) == 0, "the widening covers whole stages");
+    static constexpr int SP = !SWAP ? 5 : TN <= 32 ? 8 : 6;   // ring stages (xr + packed weights)
+    static_assert((WT * CPR) % (kUnpWarps * 32) == 0, "the widening covers whole stages");
     static constexpr int ACC = MMA_N < 32 ? 32 : MMA_N;  // TMEM columns per accumulator
     static constexpr int TMEM_COLS = 2 * ACC;            // two accumulators (power of two)
     static constexpr int OFF_XR = 0;                      // 1024-aligned tiles first
@@ -169,7 +175,8 @@ struct Cfg {
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + slack for 1024 alignment
     static_assert(SMEM_BYTES <= 232448, "exceeds the per-CTA shared memory limit");
-    static_assert(XR_KB % 1024 == 0 && UB_KB % 1024 == 0, "swizzled tiles stay 1024-aligned");
+    static_assert(XR_KB % 1024 == 0 && UB_KB % 1024 == 0 && PB_ST % 1024 == 0,
+                  "swizzled tiles stay 1024-aligned");
 };
 
 // Instruction descriptor of tcgen05.mma kind::f16: D fp32, A and B bf16,
@@ -287,7 +294,7 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     ptx::grid_dependency_wait();
 
     const int tiles_a = (M + TN - 1) / TN;           // token tiles
-    const int tiles_b = (N + WR - 1) / WR;           // weight tiles
+    const int tiles_b = (N + C::WT - 1) / C::WT;     // weight tiles
     const int num_tiles = tiles_a * tiles_b;
     const int first_tile = static_cast<int>(blockIdx.x);
     const int tile_step = static_cast<int>(gridDim.x);
@@ -312,7 +319,7 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                     ptx::tma_load_2d(sbase + C::OFF_XR + ps * C::XR_ST + i * C::XR_KB, &tmA,
                                      full_p(ps), (kp * KBS + i) * KB, ta * TN);
                 ptx::tma_load_2d(sbase + C::OFF_PB + ps * C::PB_ST, &tmB, full_p(ps), kp * C::PKB,
-                                 tb * WR);
+                                 tb * C::WT);
                 if (++ps == SP) { ps = 0; ph ^= 1; }
             }
         }
@@ -347,7 +354,7 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const uint64_t xd = ptx::sw128_kmajor_desc(x0 + i * C::XR_KB + 32 * j);
-                        const uint64_t wd = ptx::sw128_kmajor_desc(w0 + i * UB_KB + 32 * j);
+                        const uint64_t wd = ptx::sw128_kmajor_desc(w0 + i * C::UB_KB + 32 * j);
                         mma_bf16_ss(d, SWAP ? wd : xd, SWAP ? xd : wd, idesc,
                                     (kp | i | j) != 0 ? 1u : 0u);
                     }
@@ -377,7 +384,7 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             ptx::tc_fence_after();
             if constexpr (SWAP) {
                 // lane = output column n (a weight row), columns = tokens
-                const int n = tb * WR + quarter * 32 + lane;
+                const int n = tb * C::WT + quarter * 32 + lane;
                 const float swn = n < N ? sw[n] : 0.0f;
                 const float bn = (bias && n < N) ? __uint_as_float(static_cast<uint32_t>(bias[n]) << 16)
                                                  : 0.0f;
@@ -404,8 +411,8 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             }
             const int m = ta * TN + quarter * 32 + lane;      // this lane's output row
 #pragma unroll 1
-            for (int c0 = 0; c0 < WR; c0 += 32) {
-                const int n0 = tb * WR + c0;
+            for (int c0 = 0; c0 < C::WT; c0 += 32) {
+                const int n0 = tb * C::WT + c0;
                 uint32_t v[32];
                 __syncwarp();   // tcgen05.ld is warp-collective
                 ptx::tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
@@ -448,7 +455,7 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         }
     } else {
         // ------------------------------------------------------------ widening
-        // Stage = WR rows x CPR packed chunks of 16 bytes (chunk p = codes
+        // Stage = WT rows x CPR packed chunks of 16 bytes (chunk p = codes
         // 32p .. 32p + 31 = half p & 1 of K-block p >> 1).  Thread ut takes
         // chunks ut, ut + 256, ...: a quarter warp reads 128 contiguous
         // packed bytes (two 64-byte rows, or four 32-byte rows) and writes 8
@@ -458,7 +465,7 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         // with one, the four rows' swizzle phases differ in their low bits.
         const int ut = threadIdx.x - kWarpUnp0 * 32;
         const int total = my_tiles * num_kp;
-        constexpr int kPer = WR * C::CPR / (kUnpWarps * 32);
+        constexpr int kPer = C::WT * C::CPR / (kUnpWarps * 32);
         for (int n = 0; n < total; ++n) {
             const int ps = n % SP, us = n % SU;
             const uint32_t pph = (n / SP) & 1, uph = (n / SU) & 1;
@@ -475,7 +482,7 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                 const int kbi = p >> 1;
                 const uint32_t half = static_cast<uint32_t>(p & 1);
                 const uint32_t swz = static_cast<uint32_t>(row & 7);
-                const uint32_t dst = ub + static_cast<uint32_t>(kbi * UB_KB + row * 128);
+                const uint32_t dst = ub + static_cast<uint32_t>(kbi * C::UB_KB + row * 128);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     // packed word q = widened chunk q; q = (i + 2 kbi) mod 4 = i ^ 2 kbi
@@ -655,7 +662,7 @@ convrot_status launch_gemm_cfg(int num_sms, const void *xr, const uint8_t *qw, c
         const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
         const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
         const cuuint32_t box[2] = {static_cast<cuuint32_t>(C::PKB),
-                                   static_cast<cuuint32_t>(w4a16::WR)};
+                                   static_cast<cuuint32_t>(C::WT)};
         const cuuint32_t estr[2] = {1, 1};
         if (g_encode(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(qw), dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -663,7 +670,7 @@ convrot_status launch_gemm_cfg(int num_sms, const void *xr, const uint8_t *qw, c
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return CONVROT_ERR_CUDA;
     }
-    const int64_t tiles = ((M + TN - 1) / TN) * ((N + w4a16::WR - 1) / w4a16::WR);
+    const int64_t tiles = ((M + TN - 1) / TN) * ((N + C::WT - 1) / C::WT);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
