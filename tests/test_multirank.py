@@ -68,6 +68,37 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     monkeypatch.setenv("WORLD_SIZE", "2")
     monkeypatch.setenv("RANK", "1")
     monkeypatch.setenv("LOCAL_RANK", "1")
-    args = argparse.Namespace(workload="small_g256", steps=3, warmup=3, cpu_seconds=0.1)
+    args = argparse.Namespace(workload="small_g256", steps=3, warmup=3, cpu_seconds=0.1,
+                              variant="w4a4")
     assert bench.run_reference(args) is None
     assert capsys.readouterr().out == ""
+
+
+def test_w4a16_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    args = argparse.Namespace(workload="small_g256", steps=3, warmup=3, cpu_seconds=0.1,
+                              variant="w4a16")
+    assert bench.run_reference(args) is None
+    assert capsys.readouterr().out == ""
+
+
+def test_w4a16_reference_arm_line(monkeypatch, capsys):
+    import json
+    for v in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(v, raising=False)
+    args = argparse.Namespace(workload="small_g256", steps=3, warmup=3, cpu_seconds=0.1,
+                              variant="w4a16")
+    bench.run_reference(args)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["dtype"] == "bf16"
+    assert line["metric"] == bench.METRIC_W4A16 and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_traffic_hash_covers_the_w4a4_library_sources():
+    """The per-launch DRAM traffic the benchmark reports belongs to the W4A4
+    kernels; its key hashes exactly the files that library is built from."""
+    from rotated_w4a4_quantized_b200 import build
+    assert sorted(os.path.basename(p) for p in build.DEPS) == sorted(bench.W4A4_SOURCES)
