@@ -165,3 +165,20 @@ def test_bf16_tie_band_marks_midpoints_only():
     y = np.array([[1 + 2 ** -8, 1 + 2 ** -9, 3.0, 1.5 + 2 ** -8]])
     band = O.bf16_tie_band(y, band=1e-5)
     assert band.tolist() == [[True, False, False, True]]
+
+
+def test_bf16_tie_band_is_exactly_where_rounding_can_flip():
+    """Outside the band, moving a value by up to the band width never changes
+    its bf16 rounding; every flip found that way lies inside the band."""
+    rng = np.random.default_rng(12)
+    y = rng.standard_normal((64, 256)) * np.exp2(rng.integers(-8, 8, size=(64, 1)))
+    # plant values right at and next to midpoints
+    sp = O.bf16_spacing(y[:, :32])
+    y[:, :32] = (np.floor(np.abs(y[:, :32]) / sp) + 0.5) * sp * np.sign(y[:, :32])
+    band = 1e-5
+    mask = O.bf16_tie_band(y, band)
+    eps = band * np.abs(y).max(axis=1, keepdims=True)
+    lo, mid, hi = O.round_bf16(y - eps), O.round_bf16(y), O.round_bf16(y + eps)
+    flips = (lo != mid) | (hi != mid)
+    assert not (flips & ~mask).any()
+    assert flips[:, :32].all() and mask[:, :32].all()
