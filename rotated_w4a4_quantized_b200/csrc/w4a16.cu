@@ -690,7 +690,7 @@ convrot_status launch_gemm_cfg(int num_sms, const void *xr, const uint8_t *qw, c
 }
 
 // Up to 64 tokens: the weights take the MMA's 128-row side and the tokens a
-// 16-, 32- or 64-wide side; beyond that, 128 x 128 token-by-weight tiles.
+// 16-, 32- or 64-wide side; beyond that, 128 x 256 token-by-weight tiles.
 convrot_status launch_gemm(int num_sms, const void *xr, const uint8_t *qw, const float *sw,
                            const void *bias, int64_t M, int64_t N, int64_t K, void *y,
                            cudaStream_t stream) {
