@@ -189,6 +189,25 @@ def test_quantize_matches_exhaustive_search(oracle):
     assert np.abs(q).max() <= 7
 
 
+@pytest.mark.parametrize("group,K", [(64, 512), (256, 1024), (4, 64), (16, 256)])
+def test_exact_ties_round_half_away(oracle, group, K):
+    """Rows built so that their rotation is a known sparse y of exact
+    half-integer multiples of a power-of-two scale (tests/tie_rows.py): the
+    oracle must reproduce y exactly, take s = s0, and round every .5 away
+    from zero.  Half-even, half-up or truncation would each move some of
+    the codes (0.5 -> 0, -2.5 -> -2, 6.5 -> 6), and a wrong sign or index in
+    the rotation would move y."""
+    from tests.tie_rows import exact_tie_rows
+    x, y, s0, codes = exact_tie_rows(12, K, group, seed=group + K)
+    assert np.array_equal(oracle.rotate(x, group), y)
+    p, s = oracle.prepare_rows(x, group)
+    assert np.array_equal(s, s0)
+    assert np.array_equal(oracle.unpack(p, K), codes)
+    frac = np.abs(y / s0[:, None]) % 1.0
+    assert (frac == 0.5).sum() > 10 * 12                   # many exact ties
+    assert set(np.abs(codes[frac == 0.5]).tolist()) == set(range(1, 8))
+
+
 def test_quantize_edge_rows(oracle):
     # with absmax 7, inv = 1 exactly and v = y: exact .5 ties round away
     # (the decision is taken on fp32(y): 3.4999999 would round to fp32 3.5,
@@ -281,6 +300,104 @@ def test_epilogue_exact_values_and_one_ulp(oracle):
     assert np.all(np.abs(y - ref) <= ulp)
 
 
+def _finite_bf16_table():
+    """(patterns, fp64 values) of every finite bf16, both signs."""
+    pats = np.arange(1 << 16, dtype=np.uint32)
+    pats = pats[((pats >> 7) & 0xFF) != 0xFF]
+    vals = (pats << 16).astype(np.uint32).view(np.float32).astype(np.float64)
+    return pats.astype(np.uint16), vals
+
+
+def _nearest_even_bf16_by_search(f32):
+    """Brute force over all finite bf16 of the same sign: the nearest one to
+    each fp32 value, and on an exact tie the one whose pattern is even."""
+    pats, vals = _finite_bf16_table()
+    out = np.empty(f32.shape, dtype=np.uint16)
+    v64 = f32.astype(np.float64)
+    neg = np.signbit(f32)
+    for i in range(0, f32.size, 256):
+        v = v64[i:i + 256, None]
+        same_sign = (pats[None, :] >= 0x8000) == neg[i:i + 256, None]
+        d = np.where(same_sign, np.abs(vals[None, :] - v), np.inf)
+        dmin = d.min(axis=1, keepdims=True)
+        cand = d == dmin
+        # among the nearest (at most two), prefer the even pattern
+        pref = cand & ((pats[None, :] & 1) == 0)
+        pick = np.where(pref.any(axis=1), pref.argmax(axis=1), cand.argmax(axis=1))
+        out[i:i + 256] = pats[pick]
+    return out
+
+
+def test_f32_to_bf16_is_nearest_even_by_search(oracle):
+    """The epilogue's last step.  Exact midpoints whose lower neighbour is
+    even (257 -> 256, 1 + 2^-8 -> 1) and odd (259 -> 260, 1 + 3 2^-8 ->
+    1 + 2^-6) separate ties-to-even from half-up, half-away and truncation;
+    their fp32 neighbours separate it from any rule that rounds near, not
+    at, the midpoint; subnormal midpoints check the bottom of the range."""
+    named = {257.0: 0x4380, 259.0: 0x4382, 1 + 2 ** -8: 0x3F80, 1 + 3 * 2 ** -8: 0x3F82,
+             -257.0: 0xC380, -259.0: 0xC382, 255.5: 0x437F + 1}
+    f = np.array(list(named), dtype=np.float32)
+    assert oracle.f32_to_bf16(f).tolist() == list(named.values())
+    # midpoints: fp32 patterns with the 16 dropped bits exactly 0x8000, over
+    # kept patterns with even and odd last bits, normal and subnormal, both
+    # signs, and the fp32 values one step either side of each midpoint
+    rng = np.random.default_rng(11)
+    kept = np.concatenate([np.arange(0, 8), np.arange(0x7F, 0x84), np.arange(0x3F80, 0x3F88),
+                           np.arange(0x4380, 0x4388), rng.integers(0x0080, 0x7F00, 400)])
+    kept = np.concatenate([kept, kept | 0x8000]).astype(np.uint32)
+    mids = (kept << 16) | 0x8000
+    bits = np.concatenate([mids, mids - 1, mids + 1,
+                           rng.integers(0, 0x7F000000, 600, dtype=np.uint32),
+                           rng.integers(0x80000000, 0xFF000000, 600, dtype=np.uint32)])
+    f = bits.astype(np.uint32).view(np.float32)
+    got = oracle.f32_to_bf16(f)
+    assert np.array_equal(got, _nearest_even_bf16_by_search(f))
+    # and torch's own float -> bfloat16 conversion, a library rounding
+    lib = wl.bf16_bits(torch.from_numpy(f.copy()).to(torch.bfloat16))
+    assert np.array_equal(got, lib)
+
+
+def test_quantiser_product_reading_moves_codes_only_in_the_tie_band(oracle):
+    """The pages fix no formula for a code beyond rowwise absmax INT4 in
+    [-7, 7] ("convrot-mlx" README, "What is included").  The oracle takes
+    v = fp32(y) * fp32(7 / a); the other plain reading is v = y / s with the
+    stored scale s = fp32(a / 7), evaluated either in fp32 or in fp64.  Every
+    code the readings disagree on must lie where the fp64 y / s is within
+    1e-5 of a .5 boundary (the band the parity gates excuse), so the choice
+    between them cannot decide any code a gate checks exactly.  Rows: seeded
+    normal and heavy-tailed rows at scales 2^-20 .. 2^20, plus rows built to
+    sit on and next to .5 boundaries."""
+    rng = np.random.default_rng(12)
+    rows = []
+    for e in range(-20, 21, 4):
+        rows.append(rng.standard_normal((60, 256)) * 2.0 ** e)
+        rows.append(rng.standard_cauchy((20, 256)).clip(-1e4, 1e4) * 2.0 ** e)
+    for eps in (0.0, 1e-7, -1e-7, 1e-6, -3e-6, 9e-6, -2e-5, 4e-5):
+        base = rng.integers(-7, 7, (16, 256)) + 0.5 + eps
+        base[:, 0] = 7.0
+        scale = np.float64(np.float32(rng.uniform(0.01, 3.0)))
+        rows.append(base * scale)
+    y = np.concatenate(rows)
+    q, s = oracle.quantize_rows(y)
+    s64 = s.astype(np.float64)[:, None]
+
+    def half_away(v):
+        return np.sign(v) * np.floor(np.abs(v) + 0.5)
+
+    v64 = y / s64
+    q_div64 = np.clip(half_away(v64), -7, 7)
+    v32 = (y.astype(np.float32) / s[:, None]).astype(np.float32).astype(np.float64)
+    q_div32 = np.clip(half_away(v32), -7, 7)
+    a = np.abs(v64)
+    band = np.abs(a - (np.floor(a) + 0.5)) < 1e-5
+    for alt in (q_div64, q_div32):
+        moved = alt != q
+        assert not (moved & ~band).any(), np.argwhere(moved & ~band)[:5]
+        assert np.abs(alt - q).max() <= 1
+    # the constructed rows do put values inside the band, so the check bites
+    assert band.sum() > 1000
+
+
 def test_epilogue_null_bias_is_zero_bias(oracle):
     acc = np.arange(12, dtype=np.int64).reshape(3, 4) - 5
     sx = np.array([0.1, 0.2, 0.3], dtype=np.float32)
@@ -338,7 +455,10 @@ def test_layer_brute_force_tiny(oracle, n):
     assert np.array_equal(oracle.unpack(px, 16), qx) and np.array_equal(ox, sx)
     assert np.array_equal(oracle.unpack(pw, 16), qw) and np.array_equal(ow, sw)
     y = oracle.linear_prepared_w(x, pw, ow, b, n)
-    assert np.array_equal(y, oracle.f32_to_bf16(t))
+    # the expected bf16 comes from torch's float -> bfloat16 conversion (round
+    # to nearest even), not from the oracle's own rounding
+    want = wl.bf16_bits(torch.from_numpy(np.ascontiguousarray(t)).to(torch.bfloat16))
+    assert np.array_equal(y, want)
 
 
 def test_worked_examples(oracle):

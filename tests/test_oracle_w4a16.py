@@ -182,3 +182,47 @@ def test_bf16_tie_band_is_exactly_where_rounding_can_flip():
     flips = (lo != mid) | (hi != mid)
     assert not (flips & ~mask).any()
     assert flips[:, :32].all() and mask[:, :32].all()
+
+
+def _emulate_w4a16_kernel(xr_bits, packed_w, sw, bias_bits, K, drop_block=None, block=64):
+    """The GPU GEMM's arithmetic written out on the CPU: products of bf16
+    activations and integer codes (exact in fp32), summed in fp32 sixteen at
+    a time (one tensor-core K step), each partial added to an fp32 running
+    sum; then the fp32 epilogue acc * sw + b and one rounding to bf16 (by
+    torch).  drop_block leaves out the K-block starting at that index."""
+    import torch
+    xf = _bits_to_f64(xr_bits).astype(np.float32)
+    q = decode_codes(packed_w).astype(np.float32)
+    M, N = xf.shape[0], q.shape[0]
+    run = np.zeros((M, N), dtype=np.float32)
+    for k0 in range(0, K, 16):
+        if drop_block is not None and drop_block <= k0 < drop_block + block:
+            continue
+        part = np.zeros((M, N), dtype=np.float32)
+        for k in range(k0, k0 + 16):
+            part = part + np.outer(xf[:, k], q[:, k]).astype(np.float32)
+        run = run + part
+    y = run * np.asarray(sw, np.float32)[None, :]
+    if bias_bits is not None:
+        y = y + _bits_to_f64(bias_bits).astype(np.float32)[None, :]
+    return wl.bf16_bits(torch.from_numpy(y.astype(np.float32)).to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("K,group", [(1024, 64), (4096, 256)])
+def test_w4a16_gate_accepts_the_kernel_arithmetic_and_rejects_a_dropped_block(K, group):
+    """The W4A16 output gate (check_w4a16_outputs) is a tolerance, not an
+    equality, so it is pinned from both sides: an emulation of the kernel's
+    fp32 tensor-core accumulation passes it, and the same emulation with one
+    64-deep K-block left out fails it."""
+    from tests import gpu_compare as gc
+    lt = wl.make_random_layer(20, K, 36, group, seed=K + group)
+    xb, wb, bb = wl.bf16_bits(lt.x), wl.bf16_bits(lt.w), wl.bf16_bits(lt.b)
+    xr = O.w4a16_rotate_act(xb, group)
+    pw, sw = O.prepare_rows(wb, group)
+    acc, l1, p16 = O.w4a16_gemm(xr, pw, K)
+    t, _ = O.w4a16_epilogue(acc, sw, bb)
+    gc.check_w4a16_outputs(_emulate_w4a16_kernel(xr, pw, sw, bb, K), t, acc, l1, p16, sw)
+    for drop in (0, K // 2, K - 64):
+        with pytest.raises(AssertionError):
+            gc.check_w4a16_outputs(_emulate_w4a16_kernel(xr, pw, sw, bb, K, drop_block=drop),
+                                   t, acc, l1, p16, sw)
