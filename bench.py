@@ -30,6 +30,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -60,6 +61,37 @@ METRIC_W4A16 = "W4A16 linear end-to-end TFLOP/s (bf16 x INT4 tensor ops); rotati
 # the GEMM reads xr, the packed weights, scales and bias and writes y
 ROT16_BYTES = lambda M, K: 4 * M * K  # noqa: E731
 GEMM16_BYTES = lambda M, N, K: 2 * M * K + N * K // 2 + 4 * N + 2 * N + 2 * M * N  # noqa: E731
+
+
+MIN_KERNEL_MS = 50.0          # device time of each per-kernel timing pass, at least
+NOMINAL_INT8_TOPS = 4500.0    # datasheet dense int8 (half of the 2:4-sparse figure)
+
+
+def int8_ceiling(dev, n=8192):
+    """The achieved int8 tensor-core ceiling of this GPU: torch._int_mm
+    (cuBLASLt s8 x s8 -> s32, both operands K-major) on n x n x n, best of 10
+    back-to-back launches timed with CUDA events after warm-up.  None where
+    the call is not available."""
+    try:
+        a = torch.randint(-7, 8, (n, n), dtype=torch.int8, device=dev)
+        b = torch.randint(-7, 8, (n, n), dtype=torch.int8, device=dev).t()
+        for _ in range(3):
+            c = torch._int_mm(a, b)
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            c = torch._int_mm(a, b)
+            e1.record()
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        del a, b, c
+        torch.cuda.empty_cache()
+        return {"tops": round(2 * n ** 3 / (best * 1e-3) / 1e12, 1), "shape": f"{n}^3",
+                "how": "torch._int_mm (cuBLASLt s8xs8->s32), best of 10, CUDA events"}
+    except (RuntimeError, TypeError) as e:
+        return {"tops": None, "error": str(e).splitlines()[0][:200]}
 
 
 def _peaks():
@@ -337,9 +369,22 @@ def run_gpu(args):
     if status != 0:
         raise RuntimeError(f"device error status {status} in the timed region")
 
-    # per-kernel durations: K back-to-back launches of one kernel of one layer
-    prep_ms = [[timed(("prep", i), args.steps) / args.steps] * args.steps for i in range(nl)]
-    gemm_ms = [[timed(("gemm", i), args.steps) / args.steps] * args.steps for i in range(nl)]
+    # per-kernel durations: back-to-back launches of one kernel of one layer,
+    # at least K of them and at least MIN_KERNEL_MS of device time, so that
+    # short kernels are not timed over a fraction of a millisecond
+    def timed_kernel(key):
+        n = args.steps
+        t = timed(key, n)
+        if t < MIN_KERNEL_MS:
+            n = int(math.ceil(n * MIN_KERNEL_MS * 1.05 / max(t, 1e-3)))
+            t = timed(key, n)
+        return t / n, n
+
+    prep_pass = [timed_kernel(("prep", i)) for i in range(nl)]
+    gemm_pass = [timed_kernel(("gemm", i)) for i in range(nl)]
+    prep_ms = [[avg] * args.steps for avg, _ in prep_pass]
+    gemm_ms = [[avg] * args.steps for avg, _ in gemm_pass]
+    ceiling = int8_ceiling(dev) if any(sp.M > SKINNY_MAX_M for sp, *_ in prepared) else None
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)   # e2e pass only
     ops_step = spec.ops
     t_max, ops_total = aggregate(local_ms, ops_step * args.steps, dev)
@@ -379,8 +424,13 @@ def run_gpu(args):
                     "peak": round(int8_peak, 1), "unit": "TFLOP/s",
                     "frac": round(gemm_tops[i] / int8_peak, 4),
                     "traffic": _traffic(name, "gemm_kernel"),
+                    "frac_of_nominal_int8": round(gemm_tops[i] / NOMINAL_INT8_TOPS, 4),
+                    "frac_of_int_mm": (round(gemm_tops[i] / ceiling["tops"], 4)
+                                       if ceiling and ceiling.get("tops") else None),
                     "note": "integer tensor ops (2 per multiply-add); peak = measured bf16 burst "
-                            f"x {INT8_PER_BF16} nominal int8/bf16 ratio ({peaks['src']})"}
+                            f"x {INT8_PER_BF16} nominal int8/bf16 ratio ({peaks['src']}); also "
+                            f"against the {NOMINAL_INT8_TOPS:.0f} TOPS nominal dense int8 peak "
+                            "and against torch._int_mm (cuBLASLt int8) measured in this run"}
     else:
         i = max(range(nl), key=lambda j: sum(prep_ms[j]))
         roof = {"kernel": "prep_kernel", "bound": "hbm", "achieved": round(prep_gbs[i], 1),
@@ -417,6 +467,10 @@ def run_gpu(args):
                 "call": f"HostPipeline: pinned host buffers, {e2e['chunks']} row chunks, "
                         "copies overlapped with convrot_linear on three streams"},
         "gpu_launches": launches,
+        "kernel_passes": {"prep_launches": [n for _, n in prep_pass],
+                          "gemm_launches": [n for _, n in gemm_pass],
+                          "min_device_ms": MIN_KERNEL_MS},
+        "int8_ceiling": ceiling,
         "clocks": clocks.summary(),
     }
     if rank == 0:
@@ -792,6 +846,37 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def rank_plan(gpus: int, env) -> str:
+    """'run' when this process is one of the requested ranks, 'spawn' when
+    --gpus asks for more ranks than a process group provides (none was set
+    up: start them).  A process group of another size is an error."""
+    if gpus < 1:
+        raise SystemExit(f"--gpus must be >= 1, got {gpus}")
+    world = env.get("WORLD_SIZE")
+    if world is None or world == "":
+        return "spawn" if gpus > 1 else "run"
+    if int(world) != gpus:
+        raise SystemExit(f"--gpus {gpus} but WORLD_SIZE={world}: launch one rank per GPU "
+                         f"(torchrun --nproc-per-node {gpus}) or drop --gpus")
+    return "run"
+
+
+def spawn_cmd(gpus: int, argv, port: int):
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={gpus}", "--master-addr", "127.0.0.1", f"--master-port={port}",
+            os.path.abspath(__file__), *argv]
+
+
+def spawn_ranks(gpus: int, argv) -> int:
+    """Start `gpus` ranks of this script under torchrun on 127.0.0.1; rank 0
+    prints the JSON line.  Returns their exit status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    return subprocess.call(spawn_cmd(gpus, argv, port))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -807,6 +892,9 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    plan = rank_plan(args.gpus, os.environ)
+    if plan == "spawn":
+        sys.exit(spawn_ranks(args.gpus, sys.argv[1:] if argv is None else list(argv)))
     if args.impl == "reference":
         run_reference(args)
     elif args.variant == "w4a16":

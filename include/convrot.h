@@ -22,6 +22,11 @@
  *   - All pointers are DEVICE pointers on the current CUDA device unless stated
  *     otherwise, row-major and contiguous, 16-byte aligned (CONVROT_ERR_ALIGN
  *     otherwise).  bf16 tensors are passed as const void* to raw bf16 data.
+ *     Each pointer is looked up with cudaPointerGetAttributes before anything
+ *     is launched: host memory (pinned or not), another GPU's memory or an
+ *     address the CUDA runtime does not know gives CONVROT_ERR_NOT_DEVICE.
+ *     Sizes cannot be checked through a raw pointer: buffers must hold the
+ *     bytes each entry point states.
  *   - Ownership stays with the caller: the library allocates nothing, frees
  *     nothing, never synchronises and never changes the current device.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default).
@@ -58,10 +63,13 @@ typedef enum {
     CONVROT_ERR_CUDA = 6,            /* a CUDA runtime call or launch failed */
     CONVROT_ERR_DEVICE_TIMEOUT = 7,  /* a bounded device wait ran out */
     CONVROT_ERR_UNSUPPORTED = 8,     /* device is not sm_100 */
-    CONVROT_ERR_SCRATCH_LIMIT = 9    /* needs more than the built-in scratch array */
+    CONVROT_ERR_SCRATCH_LIMIT = 9,   /* needs more than the built-in scratch array */
+    CONVROT_ERR_NOT_DEVICE = 10      /* a pointer is not memory of the current device */
 } convrot_status;
 
-/* Human-readable name of a status (static storage, never NULL). */
+/* Human-readable name of a status (static storage, never NULL).  The pages
+ * have no counterpart: their Python API raises instead ("mlx-nf4" README,
+ * "Quantize and multiply": an explicit reference path, no silent fallback). */
 const char *convrot_status_string(convrot_status s);
 
 /*
@@ -80,8 +88,11 @@ convrot_status convrot_quantize_weight(const void *w_bf16, int64_t N, int64_t K,
 convrot_status convrot_prepare_act(const void *x_bf16, int64_t M, int64_t K, int group,
                                    uint8_t *qx, float *sx, convrot_stream_t stream);
 
-/* Bytes of workspace convrot_linear needs: packed codes and scales of x,
- * each region rounded up to 256 bytes. */
+/* Bytes of workspace convrot_linear needs: the packed codes [M][K/2] and the
+ * fp32 scales [M] of the prepared activations, each region rounded up to 256
+ * bytes.  Host-only; 0 for M <= 0 or K <= 0.  Source: "convrot-mlx" README,
+ * "What is included" (fused activation preparation into the N x packed-K
+ * layout and one absmax scale per row). */
 size_t convrot_linear_workspace_size(int64_t M, int64_t K);
 
 /*
@@ -102,7 +113,9 @@ convrot_status convrot_linear(const void *x_bf16, const uint8_t *qw, const float
 /*
  * Steps 3-4 only, on prepared operands: qx [M][K/2], sx [M], qw [N][K/2],
  * sw [N], bias [N] bf16 or NULL, y [M][N] bf16.  K is the unpacked length
- * (a multiple of 64).
+ * (a multiple of 64).  Source: "convrot-mlx" README, "What is included"
+ * (the packed INT4 product) and "Install and test" (the integer product,
+ * then scaling and bias).
  */
 convrot_status convrot_linear_prepared(const uint8_t *qx, const float *sx, const uint8_t *qw,
                                        const float *sw, const void *bias_bf16, int64_t M,
@@ -111,7 +124,8 @@ convrot_status convrot_linear_prepared(const uint8_t *qx, const float *sx, const
 
 /*
  * Test hook: step 1 alone, through the same prep kernel.  Writes the
- * normalised rotated rows y_rot [M][K] as fp32.
+ * normalised rotated rows y_rot [M][K] as fp32.  Exposes the block rotation
+ * X R = [X_1 H, ..., X_G H] (Comfy-Org/comfy-quants issue, section 1).
  */
 convrot_status convrot_debug_rotate_f32(const void *x_bf16, int64_t M, int64_t K, int group,
                                         float *y_rot, convrot_stream_t stream);
@@ -119,6 +133,7 @@ convrot_status convrot_debug_rotate_f32(const void *x_bf16, int64_t M, int64_t K
 /*
  * Test hook: step 3 alone, through the same GEMM kernel.  Writes the exact
  * integer accumulators acc [M][N] as int32 (|acc| <= 49 K always fits).
+ * Exposes the integer product of "convrot-mlx" README, "Install and test".
  */
 convrot_status convrot_debug_gemm_s32(const uint8_t *qx, const uint8_t *qw, int64_t M, int64_t N,
                                       int64_t K, int32_t *acc, convrot_stream_t stream);
@@ -131,7 +146,8 @@ convrot_status convrot_debug_gemm_s32(const uint8_t *qx, const uint8_t *qw, int6
  * CUDA-core GEMV; the workspace is then not touched); 0 when it runs the
  * prep kernel and the GEMM.  Depends on (M, K, group) only.  Host-only, no
  * device work; invalid arguments give 0.  Both forms give bit-identical
- * results.
+ * results.  The pages' analogue is the skinny verification kernel that reads
+ * each weight once for a few rows ("mlx-kquant" METADATA, "Performance").
  */
 int convrot_linear_single_kernel(int64_t M, int64_t K, int group);
 
@@ -153,7 +169,8 @@ int convrot_linear_single_kernel(int64_t M, int64_t K, int group);
  *              token columns; one cta_group::2 MMA covers both slices.
  * Returns CONVROT_ERR_SHAPE for any other value or for 4 / 5 / 7 with
  * M > 128, and CONVROT_ERR_UNSUPPORTED when the device cannot co-schedule
- * CTA pairs (tiles = 3, 6, 7).
+ * CTA pairs (tiles = 3, 6, 7).  Exposes steps 3-4 ("convrot-mlx" README,
+ * "Install and test": the integer product, scaling and bias) per GEMM form.
  */
 convrot_status convrot_debug_gemm_tiles(const uint8_t *qx, const float *sx, const uint8_t *qw,
                                         const float *sw, const void *bias_bf16, int64_t M,
@@ -184,6 +201,8 @@ convrot_status convrot_debug_gemm_tiles(const uint8_t *qx, const float *sx, cons
  * device looks up the array's device address once (cudaGetSymbolAddress with
  * that device current); make that first call before any stream capture.
  * Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ * Shapes that convrot_linear runs as one kernel (convrot_linear_single_kernel)
+ * run as that kernel here too and do not touch the array.
  * Arguments, layouts and errors are otherwise those of convrot_linear.
  */
 #define CONVROT_NOALLOC_SCRATCH_BYTES (16u << 20)
@@ -192,15 +211,17 @@ convrot_status convrot_linear_noalloc(const void *x_bf16, const uint8_t *qw, con
                                       int group, void *y_bf16, convrot_stream_t stream);
 
 /*
- * Synchronises `stream`, then returns and clears the device error word of the
- * current device: CONVROT_ERR_DEVICE_TIMEOUT if a bounded wait in any kernel
+ * Failure detection (the pages have no counterpart: their kernels do not
+ * report device-side errors).  Synchronises `stream`, then returns and
+ * clears the device error word of the current device: CONVROT_ERR_DEVICE_TIMEOUT if a bounded wait in any kernel
  * of this library ran out since the last check, CONVROT_ERR_CUDA if the
  * synchronisation itself failed, CONVROT_OK otherwise.
  */
 convrot_status convrot_check_device_error(convrot_stream_t stream);
 
 /*
- * Test hook for the timeout path: launches one CTA that waits on a
+ * Test hook for the timeout path (no counterpart on the pages; it exercises
+ * the failure detection above): launches one CTA that waits on a
  * shared-memory barrier nothing ever signals, giving up after timeout_ns
  * nanoseconds (clamped to [1e3, 5e9]); it then records
  * CONVROT_ERR_DEVICE_TIMEOUT in the device error word and returns normally.

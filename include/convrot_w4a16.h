@@ -24,7 +24,8 @@
  * roundings), so results match the exact definition within the rounding of
  * that arithmetic, not bit for bit.
  *
- * Conventions are those of convrot.h: device pointers on the current device,
+ * Conventions are those of convrot.h: device pointers on the current device
+ * (CONVROT_ERR_NOT_DEVICE otherwise, checked before any launch),
  * row-major, contiguous, 16-byte aligned (CONVROT_ERR_ALIGN otherwise); the
  * caller owns every buffer and the library allocates nothing; work is
  * enqueued on `stream`; arguments are validated before any launch, so a
@@ -46,18 +47,25 @@ extern "C" {
 /*
  * Step 2 alone: xr [M][K] bf16 = bf16_rne(x R), R = I_G (x) H_group.
  * x: bf16 [M][K] (read).  xr: bf16 [M][K] (written).  One kernel.
+ * Source: the block rotation of Comfy-Org/comfy-quants issue, section 1,
+ * applied to the activations of the BF16 x INT4 path ("convrot-mlx" README,
+ * "Requirements").
  */
 convrot_status convrot_w4a16_prepare_act(const void *x_bf16, int64_t M, int64_t K, int group,
                                          void *xr_bf16, convrot_stream_t stream);
 
 /* Bytes of workspace convrot_w4a16_linear needs: the rotated activations,
- * M * K * 2 rounded up to 256 (0 for M <= 0 or K <= 0).  Host-only. */
+ * M * K * 2 rounded up to 256 (0 for M <= 0 or K <= 0).  Host-only.  It holds
+ * step 2's output, the bf16 operand of the BF16 x INT4 product ("convrot-mlx"
+ * README, "Requirements"). */
 size_t convrot_w4a16_workspace_size(int64_t M, int64_t K);
 
 /*
  * Step 3 on rotated activations: y [M][N] bf16 from xr bf16 [M][K], the
  * packed weights qw uint8 [N][K/2] and their scales sw fp32 [N], bias bf16
  * [N] or NULL (zeros).  One tensor-core kernel.  Requires K % 64 == 0.
+ * Source: "convrot-mlx" README, "What is included" (the W4A16 TensorOps path)
+ * and "Install and test" (the product, then scaling and bias).
  */
 convrot_status convrot_w4a16_linear_prepared(const void *xr_bf16, const uint8_t *qw,
                                              const float *sw, const void *bias_bf16, int64_t M,
@@ -65,7 +73,8 @@ convrot_status convrot_w4a16_linear_prepared(const void *xr_bf16, const uint8_t 
                                              convrot_stream_t stream);
 
 /*
- * The whole W4A16 layer: steps 2 and 3, two kernels on `stream` (the GEMM's
+ * The whole W4A16 layer ("convrot-mlx" README, "What is included": the
+ * W4A16 path beside W4A4): steps 2 and 3, two kernels on `stream` (the GEMM's
  * set-up overlaps the end of the rotation through programmatic dependent
  * launch).  workspace: device memory of at least
  * convrot_w4a16_workspace_size(M, K) bytes, 256-byte aligned
@@ -76,8 +85,9 @@ convrot_status convrot_w4a16_linear(const void *x_bf16, const uint8_t *qw, const
                                     int group, void *workspace, size_t ws_bytes, void *y_bf16,
                                     convrot_stream_t stream);
 
-/* Synchronise `stream`, then return and clear this library's device error
- * word (CONVROT_OK, or CONVROT_ERR_DEVICE_TIMEOUT after a wait ran out). */
+/* Failure detection (no counterpart on the pages).  Synchronise `stream`,
+ * then return and clear this library's device error word (CONVROT_OK, or
+ * CONVROT_ERR_DEVICE_TIMEOUT after a wait ran out). */
 convrot_status convrot_w4a16_check_device_error(convrot_stream_t stream);
 
 #ifdef __cplusplus

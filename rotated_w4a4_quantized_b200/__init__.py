@@ -28,6 +28,7 @@ STATUS = {
     0: "CONVROT_OK", 1: "CONVROT_ERR_NULL", 2: "CONVROT_ERR_GROUP", 3: "CONVROT_ERR_SHAPE",
     4: "CONVROT_ERR_ALIGN", 5: "CONVROT_ERR_WORKSPACE", 6: "CONVROT_ERR_CUDA",
     7: "CONVROT_ERR_DEVICE_TIMEOUT", 8: "CONVROT_ERR_UNSUPPORTED", 9: "CONVROT_ERR_SCRATCH_LIMIT",
+    10: "CONVROT_ERR_NOT_DEVICE",
 }
 MAX_K = 32768
 
@@ -93,34 +94,70 @@ def _check(rc: int, what: str):
         raise ConvRotError(rc, what)
 
 
-def _need(t: torch.Tensor, dtype, name: str):
+def _need(t, dtype, name: str, shape=None, like=None):
+    """Argument checks before any pointer reaches the library: a contiguous
+    CUDA tensor of `dtype`, on `like`'s device when given, of `shape` when
+    given (None entries match any size)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, not {type(t).__name__}")
     if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
-        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor "
+                         f"(got {t.dtype} on {t.device}, contiguous={t.is_contiguous()})")
+    if like is not None and t.device != like.device:
+        raise ValueError(f"{name} is on {t.device}, the other operands on {like.device}")
+    if shape is not None:
+        if t.dim() != len(shape) or any(w is not None and int(d) != int(w)
+                                        for d, w in zip(t.shape, shape)):
+            want = tuple("*" if w is None else int(w) for w in shape)
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {want}")
+    return t
+
+
+def _need_opt(t, dtype, name: str, shape=None, like=None):
+    return None if t is None else _need(t, dtype, name, shape, like)
+
+
+def _weights(qw, sw, bias, K: int, like):
+    """Packed weights [N, K/2] uint8, scales [N] fp32, bias [N] bf16 or None."""
+    _need(qw, torch.uint8, "qw", (None, K // 2), like)
+    N = qw.shape[0]
+    _need(sw, torch.float32, "sw", (N,), like)
+    _need_opt(bias, torch.bfloat16, "bias", (N,), like)
+    return N
+
+
+def _rows(x, dtype, name):
+    _need(x, dtype, name, (None, None))
+    return x.shape
 
 
 # ---------------------------------------------------------------------------
-# the C ABI, one wrapper each
+# the C ABI, one wrapper each; each call runs on its operands' device
 # ---------------------------------------------------------------------------
 
 def convrot_quantize_weight(w: torch.Tensor, group: int, qw=None, sw=None, stream=None):
     """bf16 [N, K] -> (packed codes uint8 [N, K/2], fp32 scales [N])."""
-    _need(w, torch.bfloat16, "w")
-    N, K = w.shape
-    qw = torch.empty(N, K // 2, dtype=torch.uint8, device=w.device) if qw is None else qw
-    sw = torch.empty(N, dtype=torch.float32, device=w.device) if sw is None else sw
-    _check(lib().convrot_quantize_weight(_p(w), N, K, group, _p(qw), _p(sw), _stream(stream)),
-           "convrot_quantize_weight")
+    N, K = _rows(w, torch.bfloat16, "w")
+    with torch.cuda.device(w.device):
+        qw = torch.empty(N, K // 2, dtype=torch.uint8, device=w.device) if qw is None else qw
+        sw = torch.empty(N, dtype=torch.float32, device=w.device) if sw is None else sw
+        _need(qw, torch.uint8, "qw", (N, K // 2), w)
+        _need(sw, torch.float32, "sw", (N,), w)
+        _check(lib().convrot_quantize_weight(_p(w), N, K, group, _p(qw), _p(sw), _stream(stream)),
+               "convrot_quantize_weight")
     return qw, sw
 
 
 def convrot_prepare_act(x: torch.Tensor, group: int, qx=None, sx=None, stream=None):
     """bf16 [M, K] -> (packed codes uint8 [M, K/2], fp32 scales [M])."""
-    _need(x, torch.bfloat16, "x")
-    M, K = x.shape
-    qx = torch.empty(M, K // 2, dtype=torch.uint8, device=x.device) if qx is None else qx
-    sx = torch.empty(M, dtype=torch.float32, device=x.device) if sx is None else sx
-    _check(lib().convrot_prepare_act(_p(x), M, K, group, _p(qx), _p(sx), _stream(stream)),
-           "convrot_prepare_act")
+    M, K = _rows(x, torch.bfloat16, "x")
+    with torch.cuda.device(x.device):
+        qx = torch.empty(M, K // 2, dtype=torch.uint8, device=x.device) if qx is None else qx
+        sx = torch.empty(M, dtype=torch.float32, device=x.device) if sx is None else sx
+        _need(qx, torch.uint8, "qx", (M, K // 2), x)
+        _need(sx, torch.float32, "sx", (M,), x)
+        _check(lib().convrot_prepare_act(_p(x), M, K, group, _p(qx), _p(sx), _stream(stream)),
+               "convrot_prepare_act")
     return qx, sx
 
 
@@ -135,15 +172,20 @@ def convrot_linear_workspace_size(M: int, K: int) -> int:
 
 def convrot_linear(x, qw, sw, bias, group: int, workspace=None, out=None, stream=None):
     """The whole layer: bf16 x [M, K] -> bf16 y [M, N]."""
-    _need(x, torch.bfloat16, "x")
-    M, K = x.shape
-    N = qw.shape[0]
-    if workspace is None:
-        workspace = torch.empty(max(1, convrot_linear_workspace_size(M, K)), dtype=torch.uint8,
-                                device=x.device)
-    out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
-    _check(lib().convrot_linear(_p(x), _p(qw), _p(sw), _p(bias), M, N, K, group, _p(workspace),
-                                workspace.numel(), _p(out), _stream(stream)), "convrot_linear")
+    M, K = _rows(x, torch.bfloat16, "x")
+    N = _weights(qw, sw, bias, K, x)
+    with torch.cuda.device(x.device):
+        need = convrot_linear_workspace_size(M, K)
+        if workspace is None:
+            workspace = torch.empty(max(1, need), dtype=torch.uint8, device=x.device)
+        _need(workspace, torch.uint8, "workspace", None, x)
+        if workspace.numel() < need:
+            raise ValueError(f"workspace holds {workspace.numel()} bytes, {need} needed")
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
+        _need(out, torch.bfloat16, "out", (M, N), x)
+        _check(lib().convrot_linear(_p(x), _p(qw), _p(sw), _p(bias), M, N, K, group,
+                                    _p(workspace), workspace.numel(), _p(out), _stream(stream)),
+               "convrot_linear")
     return out
 
 
@@ -153,36 +195,55 @@ def convrot_linear_noalloc(x, qw, sw, bias, group: int, out=None, stream=None):
     callers that cannot allocate device memory (a plugin whose host runtime
     owns every allocation, or a path that must not call cudaMalloc).  Calls
     that overlap on the GPU share that array and race; order them."""
-    _need(x, torch.bfloat16, "x")
-    M, K = x.shape
-    N = qw.shape[0]
-    out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
-    _check(lib().convrot_linear_noalloc(_p(x), _p(qw), _p(sw), _p(bias), M, N, K, group, _p(out),
-                                        _stream(stream)), "convrot_linear_noalloc")
+    M, K = _rows(x, torch.bfloat16, "x")
+    N = _weights(qw, sw, bias, K, x)
+    with torch.cuda.device(x.device):
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
+        _need(out, torch.bfloat16, "out", (M, N), x)
+        _check(lib().convrot_linear_noalloc(_p(x), _p(qw), _p(sw), _p(bias), M, N, K, group,
+                                            _p(out), _stream(stream)), "convrot_linear_noalloc")
     return out
 
 
+def _prepared(qx, sx, K: int):
+    _need(qx, torch.uint8, "qx", (None, K // 2))
+    M = qx.shape[0]
+    _need_opt(sx, torch.float32, "sx", (M,), qx)
+    return M
+
+
 def convrot_linear_prepared(qx, sx, qw, sw, bias, K: int, out=None, stream=None):
-    M, N = qx.shape[0], qw.shape[0]
-    out = torch.empty(M, N, dtype=torch.bfloat16, device=qx.device) if out is None else out
-    _check(lib().convrot_linear_prepared(_p(qx), _p(sx), _p(qw), _p(sw), _p(bias), M, N, K,
-                                         _p(out), _stream(stream)), "convrot_linear_prepared")
+    """Steps 3-4 on prepared operands -> bf16 y [M, N]."""
+    M = _prepared(qx, sx, K)
+    _need(sx, torch.float32, "sx", (M,), qx)
+    N = _weights(qw, sw, bias, K, qx)
+    with torch.cuda.device(qx.device):
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=qx.device) if out is None else out
+        _need(out, torch.bfloat16, "out", (M, N), qx)
+        _check(lib().convrot_linear_prepared(_p(qx), _p(sx), _p(qw), _p(sw), _p(bias), M, N, K,
+                                             _p(out), _stream(stream)), "convrot_linear_prepared")
     return out
 
 
 def convrot_debug_rotate_f32(x, group: int, out=None, stream=None):
-    M, K = x.shape
-    out = torch.empty(M, K, dtype=torch.float32, device=x.device) if out is None else out
-    _check(lib().convrot_debug_rotate_f32(_p(x), M, K, group, _p(out), _stream(stream)),
-           "convrot_debug_rotate_f32")
+    M, K = _rows(x, torch.bfloat16, "x")
+    with torch.cuda.device(x.device):
+        out = torch.empty(M, K, dtype=torch.float32, device=x.device) if out is None else out
+        _need(out, torch.float32, "out", (M, K), x)
+        _check(lib().convrot_debug_rotate_f32(_p(x), M, K, group, _p(out), _stream(stream)),
+               "convrot_debug_rotate_f32")
     return out
 
 
 def convrot_debug_gemm_s32(qx, qw, K: int, out=None, stream=None):
-    M, N = qx.shape[0], qw.shape[0]
-    out = torch.empty(M, N, dtype=torch.int32, device=qx.device) if out is None else out
-    _check(lib().convrot_debug_gemm_s32(_p(qx), _p(qw), M, N, K, _p(out), _stream(stream)),
-           "convrot_debug_gemm_s32")
+    M = _prepared(qx, None, K)
+    _need(qw, torch.uint8, "qw", (None, K // 2), qx)
+    N = qw.shape[0]
+    with torch.cuda.device(qx.device):
+        out = torch.empty(M, N, dtype=torch.int32, device=qx.device) if out is None else out
+        _need(out, torch.int32, "out", (M, N), qx)
+        _check(lib().convrot_debug_gemm_s32(_p(qx), _p(qw), M, N, K, _p(out), _stream(stream)),
+               "convrot_debug_gemm_s32")
     return out
 
 
@@ -198,12 +259,20 @@ def convrot_debug_gemm_tiles(qx, sx, qw, sw, bias, K: int, tiles: int, out_s32: 
                              out=None, stream=None):
     """Steps 3-4 (bf16 y) or step 3 alone (int32 acc, out_s32=True) with the
     GEMM forced to one tile shape (TILES_*)."""
-    M, N = qx.shape[0], qw.shape[0]
+    M = _prepared(qx, sx, K)
+    if out_s32:
+        _need(qw, torch.uint8, "qw", (None, K // 2), qx)
+        N = qw.shape[0]
+    else:
+        _need(sx, torch.float32, "sx", (M,), qx)
+        N = _weights(qw, sw, bias, K, qx)
     dt = torch.int32 if out_s32 else torch.bfloat16
-    out = torch.empty(M, N, dtype=dt, device=qx.device) if out is None else out
-    _check(lib().convrot_debug_gemm_tiles(_p(qx), _p(sx), _p(qw), _p(sw), _p(bias), M, N, K,
-                                          int(tiles), int(bool(out_s32)), _p(out),
-                                          _stream(stream)), "convrot_debug_gemm_tiles")
+    with torch.cuda.device(qx.device):
+        out = torch.empty(M, N, dtype=dt, device=qx.device) if out is None else out
+        _need(out, dt, "out", (M, N), qx)
+        _check(lib().convrot_debug_gemm_tiles(_p(qx), _p(sx), _p(qw), _p(sw), _p(bias), M, N, K,
+                                              int(tiles), int(bool(out_s32)), _p(out),
+                                              _stream(stream)), "convrot_debug_gemm_tiles")
     return out
 
 
@@ -253,11 +322,13 @@ def lib_w4a16() -> ctypes.CDLL:
 def convrot_w4a16_prepare_act(x: torch.Tensor, group: int, out=None, stream=None):
     """bf16 x [M, K] -> bf16 xr [M, K]: the rotated rows, each value rounded
     once to bf16 (no quantisation)."""
-    _need(x, torch.bfloat16, "x")
-    M, K = x.shape
-    out = torch.empty(M, K, dtype=torch.bfloat16, device=x.device) if out is None else out
-    _check(lib_w4a16().convrot_w4a16_prepare_act(_p(x), M, K, group, _p(out), _stream(stream)),
-           "convrot_w4a16_prepare_act")
+    M, K = _rows(x, torch.bfloat16, "x")
+    with torch.cuda.device(x.device):
+        out = torch.empty(M, K, dtype=torch.bfloat16, device=x.device) if out is None else out
+        _need(out, torch.bfloat16, "out", (M, K), x)
+        _check(lib_w4a16().convrot_w4a16_prepare_act(_p(x), M, K, group, _p(out),
+                                                     _stream(stream)),
+               "convrot_w4a16_prepare_act")
     return out
 
 
@@ -267,29 +338,34 @@ def convrot_w4a16_workspace_size(M: int, K: int) -> int:
 
 def convrot_w4a16_linear_prepared(xr, qw, sw, bias, out=None, stream=None):
     """bf16 xr [M, K] (rotated) x packed INT4 weights -> bf16 y [M, N]."""
-    _need(xr, torch.bfloat16, "xr")
-    M, K = xr.shape
-    N = qw.shape[0]
-    out = torch.empty(M, N, dtype=torch.bfloat16, device=xr.device) if out is None else out
-    _check(lib_w4a16().convrot_w4a16_linear_prepared(_p(xr), _p(qw), _p(sw), _p(bias), M, N, K,
-                                                     _p(out), _stream(stream)),
-           "convrot_w4a16_linear_prepared")
+    M, K = _rows(xr, torch.bfloat16, "xr")
+    N = _weights(qw, sw, bias, K, xr)
+    with torch.cuda.device(xr.device):
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=xr.device) if out is None else out
+        _need(out, torch.bfloat16, "out", (M, N), xr)
+        _check(lib_w4a16().convrot_w4a16_linear_prepared(_p(xr), _p(qw), _p(sw), _p(bias), M, N,
+                                                         K, _p(out), _stream(stream)),
+               "convrot_w4a16_linear_prepared")
     return out
 
 
 def convrot_w4a16_linear(x, qw, sw, bias, group: int, workspace=None, out=None, stream=None):
     """The whole W4A16 layer: bf16 x [M, K] -> bf16 y [M, N] (rotation, then
     the bf16 x INT4 tensor-core GEMM with scale and bias)."""
-    _need(x, torch.bfloat16, "x")
-    M, K = x.shape
-    N = qw.shape[0]
-    if workspace is None:
-        workspace = torch.empty(max(1, convrot_w4a16_workspace_size(M, K)), dtype=torch.uint8,
-                                device=x.device)
-    out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
-    _check(lib_w4a16().convrot_w4a16_linear(_p(x), _p(qw), _p(sw), _p(bias), M, N, K, group,
-                                            _p(workspace), workspace.numel(), _p(out),
-                                            _stream(stream)), "convrot_w4a16_linear")
+    M, K = _rows(x, torch.bfloat16, "x")
+    N = _weights(qw, sw, bias, K, x)
+    with torch.cuda.device(x.device):
+        need = convrot_w4a16_workspace_size(M, K)
+        if workspace is None:
+            workspace = torch.empty(max(1, need), dtype=torch.uint8, device=x.device)
+        _need(workspace, torch.uint8, "workspace", None, x)
+        if workspace.numel() < need:
+            raise ValueError(f"workspace holds {workspace.numel()} bytes, {need} needed")
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
+        _need(out, torch.bfloat16, "out", (M, N), x)
+        _check(lib_w4a16().convrot_w4a16_linear(_p(x), _p(qw), _p(sw), _p(bias), M, N, K, group,
+                                                _p(workspace), workspace.numel(), _p(out),
+                                                _stream(stream)), "convrot_w4a16_linear")
     return out
 
 

@@ -8,6 +8,7 @@
 #include <stdio.h>
 
 #include <atomic>
+#include <initializer_list>
 #include <mutex>
 
 #include "../../include/convrot.h"
@@ -24,8 +25,11 @@ constexpr int kSmemOptin = 232448;   // per-CTA shared memory limit (sm_100)
 // dynamic shared memory the prep kernels may use (their static part is < 1 KB)
 constexpr int kPrepSmemMax = kSmemOptin - 1024;
 
+// `ready` is stored (release) only after every other field is written and
+// read (acquire) before any of them, so a thread that sees it set sees the
+// whole state; the first set-up on each device runs under g_mu.
 struct DeviceState {
-    bool ready = false;
+    std::atomic<bool> ready{false};
     convrot_status status = CONVROT_OK;
     int num_sms = 0;
     int pair_clusters = 0;   // co-resident 2-CTA clusters of the pair GEMM (0: none)
@@ -52,20 +56,20 @@ convrot_status device_setup(int *dev_out) {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CONVROT_ERR_CUDA;
     *dev_out = dev;
     DeviceState &st = g_dev[dev];
-    if (st.ready) return st.status;
+    if (st.ready.load(std::memory_order_acquire)) return st.status;
     std::lock_guard<std::mutex> lock(g_mu);
-    if (st.ready) return st.status;
+    if (st.ready.load(std::memory_order_relaxed)) return st.status;
     int major = 0, minor = 0, sms = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
         st.status = CONVROT_ERR_CUDA;
-        st.ready = true;
+        st.ready.store(true, std::memory_order_release);
         return st.status;
     }
     if (major != 10 || minor != 0) {
         st.status = CONVROT_ERR_UNSUPPORTED;
-        st.ready = true;
+        st.ready.store(true, std::memory_order_release);
         return st.status;
     }
     if (!g_encode) {
@@ -75,7 +79,7 @@ convrot_status device_setup(int *dev_out) {
                                              &q) != cudaSuccess ||
             q != cudaDriverEntryPointSuccess || !fn) {
             st.status = CONVROT_ERR_CUDA;
-            st.ready = true;
+            st.ready.store(true, std::memory_order_release);
             return st.status;
         }
         g_encode = reinterpret_cast<EncodeTiledFn>(fn);
@@ -145,11 +149,29 @@ convrot_status device_setup(int *dev_out) {
     }
     st.num_sms = sms;
     st.status = ok ? CONVROT_OK : CONVROT_ERR_CUDA;
-    st.ready = true;
+    st.ready.store(true, std::memory_order_release);
     return st.status;
 }
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// CONVROT_OK when every non-null pointer is device (or managed) memory of
+// device `dev`, CONVROT_ERR_NOT_DEVICE otherwise: host memory, another GPU's
+// memory, or an address the runtime does not know.  Run before any launch,
+// so a bad pointer is never handed to a tensor map or a kernel.
+convrot_status check_device_ptrs(int dev, std::initializer_list<const void *> ptrs) {
+    for (const void *p : ptrs) {
+        if (!p) continue;
+        cudaPointerAttributes a;
+        if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+            cudaGetLastError();   // clear the lookup error (it is not sticky)
+            return CONVROT_ERR_NOT_DEVICE;
+        }
+        if ((a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) || a.device != dev)
+            return CONVROT_ERR_NOT_DEVICE;
+    }
+    return CONVROT_OK;
+}
 
 convrot_status check_shape(int64_t rows, int64_t K, int group) {
     if (group != 64 && group != 256) return CONVROT_ERR_GROUP;
@@ -164,11 +186,14 @@ size_t prep_smem(int64_t K, int group) {
     return static_cast<size_t>(K) * (group == 256 ? 6 : 2);
 }
 
-// Resident prep CTAs per SM for a (group, mode, K) launch, cached.
+// Resident prep CTAs per SM for a (group, mode, K) launch, cached.  The
+// cache entries are atomics: concurrent first callers may both compute an
+// entry, and they store the same value.
 int prep_ctas_per_sm(int group, int mode, int64_t K) {
-    static int cache[2][2][prep::kMaxThreads + 1];
+    static std::atomic<int> cache[2][2][prep::kMaxThreads + 1];
     const int T = static_cast<int>(K / prep::kElemsPerThread);
-    int &slot = cache[group == 256][mode][T];
+    std::atomic<int> &entry = cache[group == 256][mode][T];
+    int slot = entry.load(std::memory_order_relaxed);
     if (slot == 0) {
         int n = 0;
         cudaError_t e;
@@ -180,15 +205,17 @@ int prep_ctas_per_sm(int group, int mode, int64_t K) {
             e = mode ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, prep::prep_kernel<256, 1>, T, smem)
                      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, prep::prep_kernel<256, 0>, T, smem);
         slot = (e == cudaSuccess && n > 0) ? n : 1;
+        entry.store(slot, std::memory_order_relaxed);
     }
     return slot;
 }
 
-// Resident 16-channel prep CTAs (K/16 threads) per SM, cached.
+// Resident 16-channel prep CTAs (K/16 threads) per SM, cached (as above).
 int prep16_ctas_per_sm(int group, int mode, int64_t K) {
-    static int cache[2][2][1025];
+    static std::atomic<int> cache[2][2][1025];
     const int T = static_cast<int>((K / 16 + 31) / 32 * 32);
-    int &slot = cache[group == 256][mode][T];
+    std::atomic<int> &entry = cache[group == 256][mode][T];
+    int slot = entry.load(std::memory_order_relaxed);
     if (slot == 0) {
         int n = 0;
         cudaError_t e;
@@ -199,6 +226,7 @@ int prep16_ctas_per_sm(int group, int mode, int64_t K) {
             e = mode ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, prep::prep16_kernel<256, 1>, T, 0)
                      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, prep::prep16_kernel<256, 0>, T, 0);
         slot = (e == cudaSuccess && n > 0) ? n : 1;
+        entry.store(slot, std::memory_order_relaxed);
     }
     return slot;
 }
@@ -540,6 +568,8 @@ const char *convrot_status_string(convrot_status s) {
         case CONVROT_ERR_UNSUPPORTED: return "CONVROT_ERR_UNSUPPORTED: needs an sm_100 device";
         case CONVROT_ERR_SCRATCH_LIMIT:
             return "CONVROT_ERR_SCRATCH_LIMIT: larger than the built-in scratch array";
+        case CONVROT_ERR_NOT_DEVICE:
+            return "CONVROT_ERR_NOT_DEVICE: a pointer is not memory of the current device";
     }
     return "CONVROT_ERR_UNKNOWN";
 }
@@ -554,6 +584,7 @@ convrot_status convrot_quantize_weight(const void *w_bf16, int64_t N, int64_t K,
         return CONVROT_ERR_ALIGN;
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    if ((st = check_device_ptrs(dev, {w_bf16, qw, sw})) != CONVROT_OK) return st;
     return launch_prep(g_dev[dev].num_sms, w_bf16, N, K, group, qw, sw, nullptr, stream);
 }
 
@@ -581,6 +612,7 @@ convrot_status convrot_linear_prepared(const uint8_t *qx, const float *sx, const
         return CONVROT_ERR_ALIGN;
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    if ((st = check_device_ptrs(dev, {qx, sx, qw, sw, bias_bf16, y_bf16})) != CONVROT_OK) return st;
     return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream);
 }
 
@@ -602,6 +634,8 @@ convrot_status convrot_linear(const void *x_bf16, const uint8_t *qw, const float
     if ((st = check_gemm_args(qw, qw, M, N, K)) != CONVROT_OK) return st;
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    if ((st = check_device_ptrs(dev, {x_bf16, qw, sw, bias_bf16, workspace, y_bf16})) != CONVROT_OK)
+        return st;
     // 1..4 tokens: one kernel (the workspace is not touched).  Eligibility
     // is decided for the largest slice (128 rows), so that it depends on
     // (M, K, group) alone, as convrot_linear_single_kernel reports it; the
@@ -632,6 +666,7 @@ convrot_status convrot_debug_rotate_f32(const void *x_bf16, int64_t M, int64_t K
     if (!aligned16(x_bf16) || !aligned16(y_rot)) return CONVROT_ERR_ALIGN;
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    if ((st = check_device_ptrs(dev, {x_bf16, y_rot})) != CONVROT_OK) return st;
     return launch_prep(g_dev[dev].num_sms, x_bf16, M, K, group, nullptr, nullptr, y_rot, stream);
 }
 
@@ -645,6 +680,7 @@ convrot_status convrot_debug_gemm_s32(const uint8_t *qx, const uint8_t *qw, int6
     if (!aligned16(acc)) return CONVROT_ERR_ALIGN;
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    if ((st = check_device_ptrs(dev, {qx, qw, acc})) != CONVROT_OK) return st;
     return launch_gemm<true>(g_dev[dev], qx, nullptr, qw, nullptr, nullptr, M, N, K, acc,
                              stream);
 }
@@ -664,6 +700,8 @@ convrot_status convrot_debug_gemm_tiles(const uint8_t *qx, const float *sx, cons
         return CONVROT_ERR_ALIGN;
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    if ((st = check_device_ptrs(dev, {qx, qw, out})) != CONVROT_OK) return st;
+    if (!out_s32 && (st = check_device_ptrs(dev, {sx, sw, bias_bf16})) != CONVROT_OK) return st;
     if (out_s32)
         return launch_gemm<true>(g_dev[dev], qx, nullptr, qw, nullptr, nullptr, M, N, K, out, stream,
                                  tiles);
@@ -762,6 +800,13 @@ extern "C" convrot_status convrot_linear_noalloc(const void *x_bf16, const uint8
         return CONVROT_ERR_SCRATCH_LIMIT;
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    if ((st = check_device_ptrs(dev, {x_bf16, qw, sw, bias_bf16, y_bf16})) != CONVROT_OK) return st;
+    // 1..4 tokens: the same one-kernel form as convrot_linear, which needs no
+    // scratch at all.
+    if (decode_stages(M, K, group) > 0)
+        if (const int sp = decode_stages(M, K, group, skinny::rows_per_cta(N, g_dev[dev].num_sms)))
+            return launch_decode(g_dev[dev].num_sms, sp, x_bf16, qw, sw, bias_bf16, M, N, K,
+                                 group, y_bf16, stream);
     uint8_t *qx = nullptr;
     if ((st = noalloc_scratch(dev, &qx)) != CONVROT_OK) return st;
     // Every byte of qx and sx read by the GEMM is written by the prep kernel

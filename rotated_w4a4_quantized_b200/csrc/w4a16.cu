@@ -44,6 +44,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <initializer_list>
 #include <mutex>
 
 #include "../../include/convrot_w4a16.h"
@@ -521,8 +523,11 @@ constexpr int kMaxDevices = 64;
 constexpr int kSmemOptin = 232448;
 constexpr int kRotSmemMax = kSmemOptin - 1024;
 
+// `ready` is stored (release) only after every other field is written and
+// read (acquire) before any of them, so a thread that sees it set sees the
+// whole state; the first set-up on each device runs under g_mu.
 struct DeviceState {
-    bool ready = false;
+    std::atomic<bool> ready{false};
     convrot_status status = CONVROT_OK;
     int num_sms = 0;
 };
@@ -547,20 +552,20 @@ convrot_status device_setup(int *dev_out) {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CONVROT_ERR_CUDA;
     *dev_out = dev;
     DeviceState &st = g_dev[dev];
-    if (st.ready) return st.status;
+    if (st.ready.load(std::memory_order_acquire)) return st.status;
     std::lock_guard<std::mutex> lock(g_mu);
-    if (st.ready) return st.status;
+    if (st.ready.load(std::memory_order_relaxed)) return st.status;
     int major = 0, minor = 0, sms = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
         st.status = CONVROT_ERR_CUDA;
-        st.ready = true;
+        st.ready.store(true, std::memory_order_release);
         return st.status;
     }
     if (major != 10 || minor != 0) {
         st.status = CONVROT_ERR_UNSUPPORTED;
-        st.ready = true;
+        st.ready.store(true, std::memory_order_release);
         return st.status;
     }
     if (!g_encode) {
@@ -570,7 +575,7 @@ convrot_status device_setup(int *dev_out) {
                                              &q) != cudaSuccess ||
             q != cudaDriverEntryPointSuccess || !fn) {
             st.status = CONVROT_ERR_CUDA;
-            st.ready = true;
+            st.ready.store(true, std::memory_order_release);
             return st.status;
         }
         g_encode = reinterpret_cast<EncodeTiledFn>(fn);
@@ -584,11 +589,29 @@ convrot_status device_setup(int *dev_out) {
     ok &= set_smem(w4a16::w4a16_gemm_kernel<64, true>, w4a16::Cfg<64, true>::SMEM_BYTES);
     st.num_sms = sms;
     st.status = ok ? CONVROT_OK : CONVROT_ERR_CUDA;
-    st.ready = true;
+    st.ready.store(true, std::memory_order_release);
     return st.status;
 }
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// CONVROT_OK when every non-null pointer is device (or managed) memory of
+// device `dev`, CONVROT_ERR_NOT_DEVICE otherwise: host memory, another GPU's
+// memory, or an address the runtime does not know.  Run before any launch,
+// so a bad pointer is never handed to a tensor map or a kernel.
+convrot_status check_device_ptrs(int dev, std::initializer_list<const void *> ptrs) {
+    for (const void *p : ptrs) {
+        if (!p) continue;
+        cudaPointerAttributes a;
+        if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+            cudaGetLastError();   // clear the lookup error (it is not sticky)
+            return CONVROT_ERR_NOT_DEVICE;
+        }
+        if ((a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) || a.device != dev)
+            return CONVROT_ERR_NOT_DEVICE;
+    }
+    return CONVROT_OK;
+}
 inline size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 convrot_status check_shape(int64_t rows, int64_t K, int group) {
@@ -605,11 +628,13 @@ convrot_status check_gemm_shape(int64_t M, int64_t N, int64_t K) {
     return CONVROT_OK;
 }
 
-// Resident rotation CTAs (K/64 threads, K * (2 or 6) bytes) per SM, cached.
+// Resident rotation CTAs (K/64 threads, K * (2 or 6) bytes) per SM, cached
+// in atomics (concurrent first callers store the same value).
 int rot_ctas_per_sm(int group, int64_t K) {
-    static int cache[2][prep::kMaxThreads + 1];
+    static std::atomic<int> cache[2][prep::kMaxThreads + 1];
     const int T = static_cast<int>(K / prep::kElemsPerThread);
-    int &slot = cache[group == 256][T];
+    std::atomic<int> &entry = cache[group == 256][T];
+    int slot = entry.load(std::memory_order_relaxed);
     if (slot == 0) {
         int n = 0;
         const size_t smem = static_cast<size_t>(K) * (group == 256 ? 6 : 2);
@@ -618,6 +643,7 @@ int rot_ctas_per_sm(int group, int64_t K) {
                 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, w4a16::rotate_bf16_kernel<64>, T, smem)
                 : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, w4a16::rotate_bf16_kernel<256>, T, smem);
         slot = (e == cudaSuccess && n > 0) ? n : 1;
+        entry.store(slot, std::memory_order_relaxed);
     }
     return slot;
 }
@@ -713,6 +739,7 @@ convrot_status convrot_w4a16_prepare_act(const void *x_bf16, int64_t M, int64_t 
     if (!aligned16(x_bf16) || !aligned16(xr_bf16)) return CONVROT_ERR_ALIGN;
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    if ((st = check_device_ptrs(dev, {x_bf16, xr_bf16})) != CONVROT_OK) return st;
     return launch_rotate(g_dev[dev].num_sms, x_bf16, M, K, group, xr_bf16, stream);
 }
 
@@ -734,6 +761,7 @@ convrot_status convrot_w4a16_linear_prepared(const void *xr_bf16, const uint8_t 
         return CONVROT_ERR_ALIGN;
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    if ((st = check_device_ptrs(dev, {xr_bf16, qw, sw, bias_bf16, y_bf16})) != CONVROT_OK) return st;
     return launch_gemm(g_dev[dev].num_sms, xr_bf16, qw, sw, bias_bf16, M, N, K, y_bf16, stream);
 }
 
@@ -754,6 +782,8 @@ convrot_status convrot_w4a16_linear(const void *x_bf16, const uint8_t *qw, const
         return CONVROT_ERR_ALIGN;
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    if ((st = check_device_ptrs(dev, {x_bf16, qw, sw, bias_bf16, workspace, y_bf16})) != CONVROT_OK)
+        return st;
     if ((st = launch_rotate(g_dev[dev].num_sms, x_bf16, M, K, group, workspace, stream)) !=
         CONVROT_OK)
         return st;

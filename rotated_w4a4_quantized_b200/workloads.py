@@ -78,8 +78,10 @@ for _m in (1, 16, 128, 512):
         f"skinny_m{_m}_g64", (Linear(_m, 4096, 14336, 64, bias=False),),
         f"skinny {_m} x 4096 -> 14336, group 64, bias zero")
 
-# The workload a single benchmark step runs by default: the outlier layer.
-DEFAULT_BENCH = "outlier_g64"
+# The workload a single benchmark step runs by default: the square 8192^3
+# layer, the largest single-GPU configuration and the one whose GEMM target
+# (>= 60% of the dense int8 peak at M >= 4096) the layer is measured against.
+DEFAULT_BENCH = "square_g256"
 
 
 def _bf16(t: torch.Tensor) -> torch.Tensor:

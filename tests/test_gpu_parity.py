@@ -93,6 +93,55 @@ def test_prepare_edge_rows():
     assert np.all(qx.cpu().numpy()[0] == 0x77)
 
 
+# Exact ties, no band: rows whose rotation is a known sparse y of exact
+# half-integer multiples of a power-of-two scale (tests/tie_rows.py), so the
+# fp32 butterflies reproduce y bit for bit and every nonzero code below 7 is
+# decided by the round-half-away rule alone.  Up to 1024 rows of K <= 16384
+# run the 16-channel prep kernel, longer launches or rows the 64-channel one.
+TIE_PREP_CASES = [(40, 1024, 64), (40, 4096, 256), (5, 16384, 256), (1100, 1024, 64),
+                  (1100, 2048, 256), (3, 32768, 256), (2, 20480, 64)]
+
+
+@pytest.mark.parametrize("M,K,group", TIE_PREP_CASES)
+def test_exact_ties_bit_exact_without_band(M, K, group):
+    from tests.tie_rows import exact_tie_rows
+    xb, y, s0, codes = exact_tie_rows(M, K, group, seed=M + K + group)
+    x = _dev(torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16))
+    q_ref, s_ref = O.prepare_rows(xb, group)
+    assert np.array_equal(O.unpack(q_ref, K), codes) and np.array_equal(s_ref, s0)
+    yr = cr.convrot_debug_rotate_f32(x, group)
+    qx, sx = cr.convrot_prepare_act(x, group)
+    qw, sw = cr.convrot_quantize_weight(x, group)
+    torch.cuda.synchronize()
+    assert np.array_equal(yr.cpu().numpy().astype(np.float64), y)
+    for q, s in ((qx, sx), (qw, sw)):
+        assert np.array_equal(q.cpu().numpy(), q_ref)
+        assert np.array_equal(s.cpu().numpy(), s_ref)
+
+
+# The whole layer on exact-tie activations and weights: every code is fixed,
+# so the outputs must equal the oracle's bit for bit on every path (the
+# one-kernel decode form for 1-4 tokens, the few-token GEMM, the tiled GEMM).
+@pytest.mark.parametrize("M,K,N,group", [(1, 2048, 300, 64), (2, 4096, 520, 256),
+                                         (4, 8192, 136, 64), (16, 1024, 400, 256),
+                                         (100, 2048, 264, 64), (300, 1024, 392, 256),
+                                         (1100, 1024, 200, 64)])
+def test_exact_ties_whole_layer_bit_exact(M, K, N, group):
+    from tests.tie_rows import exact_tie_rows
+    xb, _, _, _ = exact_tie_rows(M, K, group, seed=3 * M + K)
+    wb, _, _, _ = exact_tie_rows(N, K, group, seed=5 * N + K + 1)
+    bb = wl.bf16_bits(wl.make_random_layer(1, 64, N, 64, seed=N).b)
+    dev = lambda a: _dev(torch.from_numpy(a.view(np.int16)).view(torch.bfloat16))
+    qw, sw = cr.convrot_quantize_weight(dev(wb), group)
+    y = cr.convrot_linear(dev(xb), qw, sw, dev(bb), group)
+    torch.cuda.synchronize()
+    assert cr.convrot_check_device_error() == 0
+    px, sx = O.prepare_rows(xb, group)
+    pw, swr = O.prepare_rows(wb, group)
+    y_ref = O.epilogue(O.gemm(px, pw, K), sx, swr, bb)
+    assert np.array_equal(gc.to_np_u16(y), y_ref)
+
+
 @pytest.mark.parametrize("M,N,K", [(1, 16, 64), (5, 72, 192), (16, 128, 1024), (17, 300, 512),
                                    (64, 1000, 768), (100, 256, 256), (128, 384, 1024),
                                    (129, 257, 320), (300, 600, 1536), (513, 96, 128),
@@ -339,10 +388,16 @@ def test_linear_deterministic():
 # full-size workloads, sampled outputs
 # ---------------------------------------------------------------------------
 
-def _sample(n, k, seed):
+def _sample(n, k, seed, block=None):
+    """k random indices of n, the first and last, the edges of the first
+    128- and 256-blocks, and (block given) one random index in every block of
+    that many, so that every output tile of the launch is checked."""
     rng = np.random.default_rng(seed)
     pick = set(rng.choice(n, size=min(n, k), replace=False).tolist())
     pick |= {0, n - 1, min(n - 1, 127), min(n - 1, 128), min(n - 1, 255), min(n - 1, 256)}
+    if block:
+        for b0 in range(0, n, block):
+            pick.add(int(rng.integers(b0, min(n, b0 + block))))
     return np.array(sorted(pick))
 
 
@@ -352,15 +407,19 @@ def _sample(n, k, seed):
 def test_workload_full_size_sampled(name):
     lt = wl.make_workload(name)[0]
     M, N = lt.x.shape[0], lt.w.shape[0]
-    _full_path_case(lt, lt.spec.group, rows=_sample(M, 48, 1), cols=_sample(N, 48, 2))
+    # one row in every 128-token block (the M side of every tile form) and
+    # one column in every 64 columns (tiles are 128, 192 or 256 wide, and
+    # the few-token form's weight slices are >= 64 rows)
+    _full_path_case(lt, lt.spec.group, rows=_sample(M, 48, 1, block=128),
+                    cols=_sample(N, 48, 2, block=64))
 
 
 def test_dit_mlp_pair_full_size_sampled():
     up, down = wl.make_workload("dit_mlp_g256")
     group = 256
-    rows = _sample(up.x.shape[0], 32, 3)
-    # up-projection, sampled
-    _full_path_case(up, group, rows=rows, cols=_sample(up.w.shape[0], 48, 4))
+    rows = _sample(up.x.shape[0], 32, 3, block=128)
+    # up-projection, sampled (every output tile)
+    _full_path_case(up, group, rows=rows, cols=_sample(up.w.shape[0], 48, 4, block=64))
     # down-projection: its input rows at the sampled positions are the
     # oracle's own up-projection output; other rows are seeded noise of the
     # same spread.  The GPU runs the full 1536 x 12288 -> 3072 layer.
@@ -373,7 +432,7 @@ def test_dit_mlp_pair_full_size_sampled():
     h_np = wl.bf16_bits(h).copy()
     h_np[rows] = h_rows
     down.x = torch.from_numpy(h_np.view(np.int16)).view(torch.bfloat16)
-    _full_path_case(down, group, rows=rows, cols=_sample(down.w.shape[0], 48, 5))
+    _full_path_case(down, group, rows=rows, cols=_sample(down.w.shape[0], 48, 5, block=64))
 
 
 # ---------------------------------------------------------------------------
@@ -402,6 +461,96 @@ def test_bad_arguments_raise():
     with pytest.raises(cr.ConvRotError) as e:
         cr.convrot_debug_rotate_f32(misaligned, 64)
     assert e.value.status == 4
+
+
+def test_binding_rejects_bad_tensors_before_any_launch():
+    """Every entry point checks every tensor (device, dtype, contiguity,
+    shape) before a pointer reaches the library; the output buffer stays
+    untouched."""
+    K, N, M, group = 256, 32, 8, 64
+    lt = _layer(M, K, N, group, seed=2)
+    x, w, b = _dev(lt.x), _dev(lt.w), _dev(lt.b)
+    qw, sw = cr.convrot_quantize_weight(w, group)
+    qx, sx = cr.convrot_prepare_act(x, group)
+    xr = cr.convrot_w4a16_prepare_act(x, group)
+    torch.cuda.synchronize()
+    out = torch.full((M, N), 3.0, dtype=torch.bfloat16, device="cuda")
+    sentinel = out.clone()
+    bad_weights = [dict(qw=qw.cpu()), dict(bias=b[:16]), dict(sw=sw.double()),
+                   dict(qw=qw[:, :64].contiguous()), dict(sw=sw[:16]), dict(out=out[:, :16]),
+                   dict(out=out.float()), dict(qw=qw.t())]
+    calls = {
+        "linear": lambda a: cr.convrot_linear(x, a["qw"], a["sw"], a["bias"], group, out=a["out"]),
+        "noalloc": lambda a: cr.convrot_linear_noalloc(x, a["qw"], a["sw"], a["bias"], group,
+                                                       out=a["out"]),
+        "prepared": lambda a: cr.convrot_linear_prepared(qx, sx, a["qw"], a["sw"], a["bias"], K,
+                                                         out=a["out"]),
+        "tiles": lambda a: cr.convrot_debug_gemm_tiles(qx, sx, a["qw"], a["sw"], a["bias"], K,
+                                                       cr.TILES_AUTO, out=a["out"]),
+        "w4a16": lambda a: cr.convrot_w4a16_linear(x, a["qw"], a["sw"], a["bias"], group,
+                                                   out=a["out"]),
+        "w4a16_prepared": lambda a: cr.convrot_w4a16_linear_prepared(xr, a["qw"], a["sw"],
+                                                                     a["bias"], out=a["out"]),
+    }
+    for name, call in calls.items():
+        for change in bad_weights:
+            a = dict(qw=qw, sw=sw, bias=b, out=out)
+            a.update(change)
+            with pytest.raises((ValueError, TypeError)):
+                call(a)
+    with pytest.raises(ValueError):
+        cr.convrot_linear(x.cpu(), qw, sw, b, group, out=out)
+    with pytest.raises(ValueError):
+        cr.convrot_linear_prepared(qx, sx[:4], qw, sw, b, K, out=out)
+    with pytest.raises(ValueError):
+        cr.convrot_prepare_act(x, group, qx=qx[:4])
+    with pytest.raises(ValueError):
+        cr.convrot_linear(x, qw, sw, b, group, workspace=torch.empty(16, dtype=torch.uint8,
+                                                                    device="cuda"), out=out)
+    torch.cuda.synchronize()
+    assert torch.equal(out, sentinel)
+    assert cr.convrot_check_device_error() == 0
+
+
+def test_c_abi_rejects_host_pointers_before_any_launch():
+    """Below the binding, each entry point looks its pointers up before any
+    launch: pinned and pageable host memory give CONVROT_ERR_NOT_DEVICE (10)
+    and the output stays untouched."""
+    import ctypes
+    K, N, M, group = 256, 32, 8, 64
+    lt = _layer(M, K, N, group, seed=4)
+    x, w, b = _dev(lt.x), _dev(lt.w), _dev(lt.b)
+    qw, sw = cr.convrot_quantize_weight(w, group)
+    qx, sx = cr.convrot_prepare_act(x, group)
+    ws = torch.empty(cr.convrot_linear_workspace_size(M, K), dtype=torch.uint8, device="cuda")
+    ws16 = torch.empty(cr.convrot_w4a16_workspace_size(M, K), dtype=torch.uint8, device="cuda")
+    out = torch.full((M, N), 3.0, dtype=torch.bfloat16, device="cuda")
+    sentinel = out.clone()
+    torch.cuda.synchronize()
+    pinned = lt.x.pin_memory()
+    pageable = np.zeros(M * K, dtype=np.uint16)
+    hosts = [ctypes.c_void_p(pinned.data_ptr()), pageable.ctypes.data_as(ctypes.c_void_p)]
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    L, L16 = cr.lib(), cr.lib_w4a16()
+    for h in hosts:
+        assert L.convrot_linear(h, P(qw), P(sw), P(b), M, N, K, group, P(ws), ws.numel(), P(out),
+                                s) == 10
+        assert L.convrot_linear(P(x), P(qw), P(sw), h, M, N, K, group, P(ws), ws.numel(),
+                                P(out), s) == 10
+        assert L.convrot_linear_noalloc(P(x), h, P(sw), P(b), M, N, K, group, P(out), s) == 10
+        assert L.convrot_linear_prepared(P(qx), P(sx), P(qw), h, P(b), M, N, K, P(out), s) == 10
+        assert L.convrot_prepare_act(h, M, K, group, P(qx), P(sx), s) == 10
+        assert L.convrot_quantize_weight(P(w), N, K, group, h, P(sw), s) == 10
+        assert L.convrot_debug_gemm_tiles(P(qx), P(sx), P(qw), P(sw), P(b), M, N, K, 0, 0, h,
+                                          s) == 10
+        assert L16.convrot_w4a16_linear(h, P(qw), P(sw), P(b), M, N, K, group, P(ws16),
+                                        ws16.numel(), P(out), s) == 10
+        assert L16.convrot_w4a16_linear_prepared(P(x), P(qw), h, P(b), M, N, K, P(out), s) == 10
+    torch.cuda.synchronize()
+    assert torch.equal(out, sentinel)
+    assert cr.convrot_check_device_error() == 0
+    assert L.convrot_status_string(10).startswith(b"CONVROT_ERR_NOT_DEVICE")
 
 
 # ---------------------------------------------------------------------------

@@ -102,3 +102,40 @@ def test_traffic_hash_covers_the_w4a4_library_sources():
     kernels; its key hashes exactly the files that library is built from."""
     from rotated_w4a4_quantized_b200 import build
     assert sorted(os.path.basename(p) for p in build.DEPS) == sorted(bench.W4A4_SOURCES)
+
+
+def test_rank_plan_spawns_runs_or_refuses():
+    import pytest
+    assert bench.rank_plan(1, {}) == "run"
+    assert bench.rank_plan(4, {}) == "spawn"
+    assert bench.rank_plan(2, {"WORLD_SIZE": "2"}) == "run"
+    assert bench.rank_plan(1, {"WORLD_SIZE": "1"}) == "run"
+    with pytest.raises(SystemExit):
+        bench.rank_plan(8, {"WORLD_SIZE": "2"})      # a process group of another size
+    with pytest.raises(SystemExit):
+        bench.rank_plan(0, {})
+    cmd = bench.spawn_cmd(4, ["--gpus", "4", "--steps", "7"], 29512)
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "127.0.0.1" in cmd and cmd[-4:] == [
+        "--gpus", "4", "--steps", "7"]
+
+
+def test_gpus_without_torchrun_launches_the_ranks_itself():
+    """`bench.py --gpus 2` outside torchrun starts two ranks; the reference
+    arm (the CPU oracle, no GPU needed) runs on rank 0 alone, which prints
+    the only JSON line, with n_gpus = 2."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.abspath(bench.__file__))
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "1", "--warmup", "3", "--workload", "small_g256",
+                        "--cpu-seconds", "0.2"], capture_output=True, text=True, timeout=600,
+                       cwd=root, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2
