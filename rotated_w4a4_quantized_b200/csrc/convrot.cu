@@ -180,10 +180,10 @@ convrot_status check_shape(int64_t rows, int64_t K, int group) {
     return CONVROT_OK;
 }
 
-// Shared memory of one prep CTA: one staged bf16 row (+ the group-256
-// exchange area of 4 bytes per channel).
+// Shared memory of one prep CTA: one or two staged bf16 rows (the group-256
+// exchange reuses the current row's buffer).
 size_t prep_smem(int64_t K, int group) {
-    return static_cast<size_t>(K) * (group == 256 ? 6 : 2);
+    return static_cast<size_t>(K) * 2 * prep::stage_buffers(group);
 }
 
 // Resident prep CTAs per SM for a (group, mode, K) launch, cached.  The

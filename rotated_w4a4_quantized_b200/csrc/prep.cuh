@@ -106,6 +106,11 @@ __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
+// All but the most recent of this thread's committed groups have landed.
+__device__ __forceinline__ void cp_async_wait_prior() {
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+
 // ------------------------------------------------------------------------
 // The steps of one row, shared by prep_kernel and the fused decode kernel
 // (same instructions in the same order, so both give identical codes).
@@ -167,6 +172,58 @@ __device__ __forceinline__ void rotate_row(float (&v)[kElemsPerThread], float4 *
     }
 }
 
+// The same rotation for prep_kernel, whose digit-3 exchange reuses the
+// row's own stage buffer (128 bytes per thread: the thread's 64 bf16
+// channels, already in registers) instead of a separate 256-byte-per-thread
+// area.  It runs in two passes over halves of each quarter: in pass p every
+// thread stores registers 16 qq + 8 p + (0..7) of each quarter qq (8 float4)
+// and reads back, from each of the four threads of its group, the 8 values
+// of its own quarter j.  (Skipping the thread's own quarter diverges the
+// warp, since the four lanes of a group would take different branches, and
+// measured 25% slower.)  Slot key k(w) = 2 (w mod 4) + (w / 4 mod 2): the
+// 8 threads of a quarter warp then store to 8 distinct slots and read from
+// 8 distinct slots, so neither side has bank conflicts.  The values and the
+// order of every addition are those of rotate_row, so results are identical.
+__device__ __forceinline__ int stage_key(int w) { return ((w & 3) << 1) | ((w >> 2) & 1); }
+
+template <int G>
+__device__ __forceinline__ void rotate_row_staged(float (&v)[kElemsPerThread],
+                                                  float4 *__restrict__ xb, int t, uint32_t mask) {
+    radix4_digit0(v);
+    radix4_stage<4>(v);
+    radix4_stage<16>(v);
+    if (G == 256) {
+        const int j = t & 3, gb = t & ~3, kt = stage_key(t);
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            __syncwarp(mask);     // the group's reads of the buffer (row load or pass 0) are done
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq)
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const int e = 16 * qq + 8 * p + 4 * c;
+                    xb[t * 8 + ((2 * qq + c) ^ kt)] = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                }
+            __syncwarp(mask);
+#pragma unroll
+            for (int d3 = 0; d3 < 4; ++d3) {
+                const int w = gb + d3;
+                const int kw = stage_key(w);
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const float4 f = xb[w * 8 + ((2 * j + c) ^ kw)];
+                    const int e = 16 * d3 + 8 * p + 4 * c;
+                    v[e] = f.x;
+                    v[e + 1] = f.y;
+                    v[e + 2] = f.z;
+                    v[e + 3] = f.w;
+                }
+            }
+        }
+        radix4_stage<16>(v);
+    }
+}
+
 // Channel of register e of thread t after rotate_row.
 template <int G>
 __device__ __forceinline__ int row_chan(int t, int e) {
@@ -211,15 +268,25 @@ __device__ __forceinline__ void quantize_pack(const float (&v)[E], float inv,
     }
 }
 
+// Stage buffers of prep_kernel: two where the digit-3 exchange reuses the
+// current row's buffer (n = 256), one otherwise.
+__host__ __device__ constexpr int stage_buffers(int G) { return G == 256 ? 2 : 1; }
+
 // MODE 0: quantise + pack (q, s).  MODE 1: write the normalised rotated row
 // as fp32 (yrot) instead.
 //
-// Persistent: CTA b handles rows b, b + gridDim.x, ...  Loads are
-// asynchronous: while a row is rotated and quantised, the next row of the
-// same CTA is already on its way into the stage buffer.  Each row is read with coalesced 16-byte copies (consecutive
+// Persistent: CTA b handles rows b, b + gridDim.x, ...  Rows arrive by
+// asynchronous copies while the previous row is rotated and quantised.  For
+// n = 256, two stage buffers of one bf16 row each: the CTA's next two rows
+// are on their way during the arithmetic.  For n = 64 (no exchange), one
+// buffer: the next row is requested as soon as the current one is in
+// registers (measured faster there than two buffers).  Each row is read with coalesced 16-byte copies (consecutive
 // threads, consecutive chunks) that land so that chunk c of thread t's
 // 128-byte slice sits at position c ^ (t mod 8); each thread then reads its
-// own 64 channels with conflict-free 128-bit loads.
+// own 64 channels with conflict-free 128-bit loads.  For n = 256 the
+// digit-3 exchange then reuses the same buffer (rotate_row_staged), and the
+// barrier of the row maximum also tells that every warp is done with the
+// buffer, which then receives the row after next.
 template <int G, int MODE>
 __global__ void __launch_bounds__(kMaxThreads)
 prep_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ q,
@@ -227,8 +294,9 @@ prep_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ 
     static_assert(G == 64 || G == 256, "group 64 or 256");
     constexpr int kDigits = (G == 64) ? 3 : 4;
     constexpr float kNorm = (G == 64) ? 0.125f : 0.0625f;   // 2^-kDigits
+    constexpr int NBUF = stage_buffers(G);   // one buffer only without an exchange
 
-    // K * 2 bytes of stage buffer, then (group 256) K * 4 bytes of exchange
+    // NBUF stage buffers of K * 2 bytes
     extern __shared__ uint4 stage[];
     __shared__ uint32_t red[kMaxThreads / 32];
 
@@ -241,41 +309,44 @@ prep_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ 
     const uint32_t stage_s = ptx::smem_u32(stage);
 
     auto issue_row = [&](int r, int buf) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(r) * K);
-        const uint32_t base = stage_s;
-        (void)buf;
+        if (r < M) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(r) * K);
+            const uint32_t base = stage_s + static_cast<uint32_t>(buf * row_chunks * 16);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int g = t + j * nthreads;              // chunk index in the row
-            const int owner = g >> 3, c = g & 7;
-            cp_async16(base + static_cast<uint32_t>((owner * 8 + (c ^ (owner & 7))) * 16), src + g);
+            for (int j = 0; j < 8; ++j) {
+                const int g = t + j * nthreads;          // chunk index in the row
+                const int owner = g >> 3, c = g & 7;
+                cp_async16(base + static_cast<uint32_t>((owner * 8 + (c ^ (owner & 7))) * 16),
+                           src + g);
+            }
         }
+        cp_async_commit();   // one group per row, empty past the end
     };
 
-    // One stage buffer: a row is read into registers, then (after a barrier)
-    // the next row of this CTA is requested into the same buffer, so the copy
-    // overlaps all of the arithmetic on the current row.
     int row = blockIdx.x;
-    if (row < M) issue_row(row, 0);
-    cp_async_commit();
+    issue_row(row, 0);
+    if (NBUF == 2) issue_row(row + gridDim.x, 1);
     // The GEMM that follows may be scheduled on the SMs this grid leaves
     // free from now on (all of this grid's CTAs are resident: the grid is
     // sized to the resident capacity).  It sets up, and streams weights that
     // do not depend on this grid, but reads these rows only after its
     // griddepcontrol.wait, which waits for this whole grid to complete.
     ptx::launch_dependents();
-    for (; row < M; row += gridDim.x) {
-        const int next = row + gridDim.x;
-        cp_async_wait_all();      // this row's copies (by this thread) have landed
+    for (int it = 0; row < M; row += gridDim.x, ++it) {
+        const int b = NBUF == 2 ? (it & 1) : 0;
+        uint4 *sb = stage + b * row_chunks;
+        // this row's copies (by this thread) have landed ...
+        if (NBUF == 2) cp_async_wait_prior();
+        else cp_async_wait_all();
         __syncthreads();          // ... and everyone else's
 
         float v[kElemsPerThread];
-        load_row(stage, t, v);
-        __syncthreads();          // the stage buffer is free again
-        if (next < M) issue_row(next, 0);
-        cp_async_commit();
-
-        rotate_row<G>(v, reinterpret_cast<float4 *>(stage + row_chunks), t, mask);
+        load_row(sb, t, v);
+        if (NBUF == 1) {
+            __syncthreads();      // the stage buffer is free again
+            issue_row(row + gridDim.x, 0);
+        }
+        rotate_row_staged<G>(v, reinterpret_cast<float4 *>(sb), t, mask);
         auto chan = [&](int e) -> int { return row_chan<G>(t, e); };
 
         if (MODE == 1) {
@@ -285,6 +356,10 @@ prep_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ 
                 *reinterpret_cast<float4 *>(dst + chan(4 * i)) =
                     make_float4(v[4 * i] * kNorm, v[4 * i + 1] * kNorm, v[4 * i + 2] * kNorm,
                                 v[4 * i + 3] * kNorm);
+            if (NBUF == 2) {
+                __syncthreads();  // every warp is done with buffer b
+                issue_row(row + 2 * gridDim.x, b);
+            }
             continue;
         }
 
@@ -292,7 +367,8 @@ prep_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ 
         // non-negative floats order like their bit patterns
         uint32_t mb = __reduce_max_sync(mask, __float_as_uint(m));
         if (lane == 0) red[warp] = mb;
-        __syncthreads();
+        __syncthreads();          // the row maximum is complete (and buffer b is free)
+        if (NBUF == 2) issue_row(row + 2 * gridDim.x, b);
         const int nwarps = (nthreads + 31) >> 5;
         for (int w = 0; w < nwarps; ++w) mb = max(mb, red[w]);
         const float a_u = __uint_as_float(mb);
@@ -315,6 +391,7 @@ prep_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ 
                     make_uint2(packed[2 * d3], packed[2 * d3 + 1]);
         }
     }
+    cp_async_wait_all();          // no copy outlives the CTA (empty groups past the end)
 }
 
 
