@@ -62,6 +62,8 @@ def lib():
             "oracle_w4a16_gemm": [P, P, I64, I64, I64, P, P, P],
             "oracle_w4a16_epilogue": [P, P, P, I64, I64, P, P],
             "oracle_w4a16_linear": [P, P, P, P, I64, I64, I64, I, P],
+            "oracle_repack_weight": [P, I64, I64, P],
+            "oracle_unpack_weight": [P, I64, I64, P],
             "oracle_num_threads": [],
         }
         for name, args in sig.items():
@@ -218,6 +220,30 @@ def tie_band(y: np.ndarray, s: np.ndarray, band: float = 1e-5) -> np.ndarray:
         v = np.where(s64 > 0, y / np.where(s64 > 0, s64, 1.0), 0.0)
     a = np.abs(v)
     return np.abs(a - (np.floor(a) + 0.5)) < band
+
+
+def repacked_size(N: int, K: int) -> int:
+    """Bytes of the repacked weights: N rows x ceil(K/256) blocks x 128."""
+    return N * ((K // 2 + 127) // 128) * 128
+
+
+def repack_weight(qw: np.ndarray, K: int) -> np.ndarray:
+    """Canonical packed weights [N][K/2] -> the block-major layout (flat
+    uint8 of repacked_size bytes): 128-byte column block b of every row,
+    rows in order, before block b + 1; a short last block is zero-padded."""
+    qw = np.ascontiguousarray(qw, dtype=np.uint8)
+    N = qw.shape[0]
+    rep = np.empty(repacked_size(N, K), dtype=np.uint8)
+    _check(lib().oracle_repack_weight(_ptr(qw), N, K, _ptr(rep)), "repack_weight")
+    return rep
+
+
+def unpack_weight(rep: np.ndarray, N: int, K: int) -> np.ndarray:
+    """The inverse of repack_weight: [N][K/2] canonical packed weights."""
+    rep = np.ascontiguousarray(rep, dtype=np.uint8).reshape(-1)
+    qw = np.empty((N, K // 2), dtype=np.uint8)
+    _check(lib().oracle_unpack_weight(_ptr(rep), N, K, _ptr(qw)), "unpack_weight")
+    return qw
 
 
 # --------------------------------------------------------------------------

@@ -52,6 +52,11 @@
  *    and y = bf16_rne(sum_k xr[m][k] q[n][k] * sw[n] + b[n]) with the sum,
  *    the scaling and the bias exact (fp64 here), rounded once at the end.
  *
+ *  - The reversible weight repack (oracle_repack_weight / _unpack_weight).
+ *    "convrot-mlx" README, "What is included" (lossless repacking) and
+ *    "Install and test" (repack_nk_weight_for_mpp): the packed bytes in
+ *    128-byte column blocks, block-major, and back.
+ *
  * Every function returns 0 on success or a negative number for bad
  * arguments.  Buffers are caller-owned, row-major and contiguous.
  * bf16 values travel as their raw 16-bit patterns (uint16_t).
@@ -477,6 +482,43 @@ int oracle_w4a16_linear(const uint16_t *x, const uint8_t *qw, const float *sw,
     free(xr);
     free(acc);
     return rc;
+}
+
+/* ----------------------------------------------------------------------- */
+/* The reversible weight repack.                                            */
+/* ----------------------------------------------------------------------- */
+
+/* "convrot-mlx" README, "What is included" (lossless repacking of the
+ * packed weights for the kernels that read them) and "Install and test"
+ * (repack_nk_weight_for_mpp).  The pages repack for Apple's layout; the
+ * reading taken here: the same bytes, reordered without loss into the order
+ * the reading kernel streams them.  The canonical layout is N x packed-K
+ * (row n holds bytes 0 .. K/2 - 1).  The repacked one cuts every row into
+ * 128-byte column blocks (256 codes) and stores block b of all rows before
+ * block b + 1:
+ *     rep[(b * N + n) * 128 + j] = qw[n * (K/2) + b * 128 + j]
+ * for b < ceil(K / 256), j < 128; bytes past the end of a row (K not a
+ * multiple of 256) are zero. */
+int oracle_repack_weight(const uint8_t *qw, int64_t N, int64_t K, uint8_t *rep) {
+    if (!qw || !rep || N < 0 || K <= 0 || K % 2) return -1;
+    const int64_t row = K / 2, nblk = (row + 127) / 128;
+    for (int64_t b = 0; b < nblk; ++b)
+        for (int64_t n = 0; n < N; ++n)
+            for (int64_t j = 0; j < 128; ++j) {
+                const int64_t c = b * 128 + j;
+                rep[(b * N + n) * 128 + j] = c < row ? qw[n * row + c] : 0;
+            }
+    return 0;
+}
+
+/* The inverse: qw[n * (K/2) + c] = rep[((c / 128) * N + n) * 128 + c % 128]. */
+int oracle_unpack_weight(const uint8_t *rep, int64_t N, int64_t K, uint8_t *qw) {
+    if (!qw || !rep || N < 0 || K <= 0 || K % 2) return -1;
+    const int64_t row = K / 2;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t c = 0; c < row; ++c)
+            qw[n * row + c] = rep[((c / 128) * N + n) * 128 + c % 128];
+    return 0;
 }
 
 int oracle_num_threads(void) {

@@ -508,3 +508,48 @@ def test_rotation_reduces_outlier_error(oracle):
     e_plain = np.linalg.norm(plain - dense) / np.linalg.norm(dense)
     assert err(64) < e_plain
     assert err(256) < e_plain
+
+
+# ---------------------------------------------------------------------------
+# The reversible weight repack
+# ---------------------------------------------------------------------------
+
+def test_repack_layout_by_hand(oracle):
+    """K = 512 (two 128-byte blocks per row), N = 3: block 0 of rows 0, 1, 2,
+    then block 1 of rows 0, 1, 2, written out by hand from the definition."""
+    N, K = 3, 512
+    qw = (np.arange(N * K // 2) % 251).astype(np.uint8).reshape(N, K // 2)
+    rep = oracle.repack_weight(qw, K)
+    want = np.concatenate([qw[0, :128], qw[1, :128], qw[2, :128],
+                           qw[0, 128:], qw[1, 128:], qw[2, 128:]])
+    assert np.array_equal(rep, want)
+
+
+@pytest.mark.parametrize("K", [64, 192, 256, 320, 4096])
+def test_repack_pads_the_last_block_with_zeros(oracle, K):
+    N = 5
+    qw = np.random.default_rng(K).integers(1, 256, (N, K // 2)).astype(np.uint8)
+    rep = oracle.repack_weight(qw, K).reshape(-1, N, 128)
+    assert rep.shape[0] == -(-K // 256)
+    tail = (K // 2) % 128
+    if tail:
+        assert np.all(rep[-1, :, tail:] == 0) and np.all(rep[-1, :, :tail] != 0)
+    assert np.count_nonzero(rep) == N * K // 2        # every byte once, nothing else
+
+
+def test_repack_round_trip_over_all_byte_patterns(oracle):
+    """Every byte value in every position class of a row (both halves of a
+    block, a short last block) survives repack then unpack."""
+    for N, K in [(256, 512), (7, 320), (256, 64)]:
+        rng = np.random.default_rng(N + K)
+        qw = rng.permutation(np.resize(np.arange(256, dtype=np.uint8), N * K // 2)).reshape(N, K // 2)
+        qw[:, 0] = np.arange(N) % 256                  # all 256 values in column 0 as well
+        back = oracle.unpack_weight(oracle.repack_weight(qw, K), N, K)
+        assert np.array_equal(back, qw)
+    # and a brute-force check of the index map on a tiny case
+    N, K = 2, 320
+    qw = np.arange(N * K // 2, dtype=np.uint8).reshape(N, K // 2)
+    rep = oracle.repack_weight(qw, K)
+    for n in range(N):
+        for c in range(K // 2):
+            assert rep[((c // 128) * N + n) * 128 + c % 128] == qw[n, c]
