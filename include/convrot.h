@@ -64,7 +64,8 @@ typedef enum {
     CONVROT_ERR_DEVICE_TIMEOUT = 7,  /* a bounded device wait ran out */
     CONVROT_ERR_UNSUPPORTED = 8,     /* device is not sm_100 */
     CONVROT_ERR_SCRATCH_LIMIT = 9,   /* needs more than the built-in scratch array */
-    CONVROT_ERR_NOT_DEVICE = 10      /* a pointer is not memory of the current device */
+    CONVROT_ERR_NOT_DEVICE = 10,     /* a pointer is not memory of the current device */
+    CONVROT_ERR_OVERLAP = 11         /* input and output buffers overlap */
 } convrot_status;
 
 /* Human-readable name of a status (static storage, never NULL).  The pages
@@ -123,6 +124,45 @@ convrot_status convrot_linear_prepared(const uint8_t *qx, const float *sx, const
                                        convrot_stream_t stream);
 
 /*
+ * The reversible weight repack.  "convrot-mlx" README, "What is included"
+ * (lossless repacking of the packed weights for the kernels that read them)
+ * and "Install and test" (repack_nk_weight_for_mpp).  The pages repack for
+ * Apple's MPP layout; here the same bytes are reordered, without loss, into
+ * the order the B200 kernels stream them: every row of the canonical
+ * N x packed-K layout qw [N][K/2] is cut into 128-byte column blocks (256
+ * codes), and block b of all N rows is stored before block b + 1:
+ *     qw_rep[(b * N + n) * 128 + j] = qw[n * (K/2) + b * 128 + j],
+ * b < ceil(K / 256), j < 128, zero where b * 128 + j >= K/2.  A kernel's
+ * slice of rows then reads each block as one contiguous run instead of N
+ * strided 128-byte pieces.
+ *
+ * convrot_repacked_weight_size: bytes of qw_rep, N * ceil(K/256) * 128
+ * (host-only; 0 for N <= 0 or K <= 0).
+ * convrot_repack_weight: qw [N][K/2] -> qw_rep.  convrot_unpack_weight: the
+ * exact inverse, qw_rep -> qw.  Device pointers, 16-byte aligned, the two
+ * buffers must not overlap (CONVROT_ERR_OVERLAP); K a multiple of 64 up to
+ * CONVROT_MAX_K.  One kernel on `stream`.
+ *
+ * convrot_linear_repacked / convrot_linear_prepared_repacked: convrot_linear
+ * and convrot_linear_prepared with the weights given as qw_rep (same
+ * arguments otherwise); the results are bit-identical to the canonical
+ * calls on the unpacked weights.
+ */
+size_t convrot_repacked_weight_size(int64_t N, int64_t K);
+convrot_status convrot_repack_weight(const uint8_t *qw, int64_t N, int64_t K, uint8_t *qw_rep,
+                                     convrot_stream_t stream);
+convrot_status convrot_unpack_weight(const uint8_t *qw_rep, int64_t N, int64_t K, uint8_t *qw,
+                                     convrot_stream_t stream);
+convrot_status convrot_linear_repacked(const void *x_bf16, const uint8_t *qw_rep, const float *sw,
+                                       const void *bias_bf16, int64_t M, int64_t N, int64_t K,
+                                       int group, void *workspace, size_t ws_bytes, void *y_bf16,
+                                       convrot_stream_t stream);
+convrot_status convrot_linear_prepared_repacked(const uint8_t *qx, const float *sx,
+                                                const uint8_t *qw_rep, const float *sw,
+                                                const void *bias_bf16, int64_t M, int64_t N,
+                                                int64_t K, void *y_bf16, convrot_stream_t stream);
+
+/*
  * Test hook: step 1 alone, through the same prep kernel.  Writes the
  * normalised rotated rows y_rot [M][K] as fp32.  Exposes the block rotation
  * X R = [X_1 H, ..., X_G H] (Comfy-Org/comfy-quants issue, section 1).
@@ -167,11 +207,15 @@ int convrot_linear_single_kernel(int64_t M, int64_t K, int group);
  *           7  few-token form on CTA pairs (M <= 128): each CTA widens its
  *              slice of weight rows into its TMEM and holds half of the
  *              token columns; one cta_group::2 MMA covers both slices.
+ * tiles | CONVROT_TILES_REPACKED takes qw in the repacked layout
+ * (convrot_repack_weight); form 5 with M <= 16 reads 256-byte boxes and
+ * does not take it (CONVROT_ERR_UNSUPPORTED).
  * Returns CONVROT_ERR_SHAPE for any other value or for 4 / 5 / 7 with
  * M > 128, and CONVROT_ERR_UNSUPPORTED when the device cannot co-schedule
  * CTA pairs (tiles = 3, 6, 7).  Exposes steps 3-4 ("convrot-mlx" README,
  * "Install and test": the integer product, scaling and bias) per GEMM form.
  */
+#define CONVROT_TILES_REPACKED 0x100
 convrot_status convrot_debug_gemm_tiles(const uint8_t *qx, const float *sx, const uint8_t *qw,
                                         const float *sw, const void *bias_bf16, int64_t M,
                                         int64_t N, int64_t K, int tiles, int out_s32, void *out,

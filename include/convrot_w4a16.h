@@ -85,6 +85,22 @@ convrot_status convrot_w4a16_linear(const void *x_bf16, const uint8_t *qw, const
                                     int group, void *workspace, size_t ws_bytes, void *y_bf16,
                                     convrot_stream_t stream);
 
+/*
+ * convrot_w4a16_linear and convrot_w4a16_linear_prepared with the weights
+ * given in the repacked layout of convrot_repack_weight (include/convrot.h;
+ * "convrot-mlx" README, "What is included": lossless repacking), same
+ * arguments otherwise, bit-identical results.
+ */
+convrot_status convrot_w4a16_linear_repacked(const void *x_bf16, const uint8_t *qw_rep,
+                                             const float *sw, const void *bias_bf16, int64_t M,
+                                             int64_t N, int64_t K, int group, void *workspace,
+                                             size_t ws_bytes, void *y_bf16,
+                                             convrot_stream_t stream);
+convrot_status convrot_w4a16_linear_prepared_repacked(const void *xr_bf16, const uint8_t *qw_rep,
+                                                      const float *sw, const void *bias_bf16,
+                                                      int64_t M, int64_t N, int64_t K,
+                                                      void *y_bf16, convrot_stream_t stream);
+
 /* Failure detection (no counterpart on the pages).  Synchronise `stream`,
  * then return and clear this library's device error word (CONVROT_OK, or
  * CONVROT_ERR_DEVICE_TIMEOUT after a wait ran out). */

@@ -28,7 +28,7 @@ STATUS = {
     0: "CONVROT_OK", 1: "CONVROT_ERR_NULL", 2: "CONVROT_ERR_GROUP", 3: "CONVROT_ERR_SHAPE",
     4: "CONVROT_ERR_ALIGN", 5: "CONVROT_ERR_WORKSPACE", 6: "CONVROT_ERR_CUDA",
     7: "CONVROT_ERR_DEVICE_TIMEOUT", 8: "CONVROT_ERR_UNSUPPORTED", 9: "CONVROT_ERR_SCRATCH_LIMIT",
-    10: "CONVROT_ERR_NOT_DEVICE",
+    10: "CONVROT_ERR_NOT_DEVICE", 11: "CONVROT_ERR_OVERLAP",
 }
 MAX_K = 32768
 
@@ -63,6 +63,10 @@ def lib() -> ctypes.CDLL:
             "convrot_debug_timeout_probe": [I64, P],
             "convrot_linear_noalloc": [P, P, P, P, I64, I64, I64, I, P, P],
             "convrot_debug_gemm_tiles": [P, P, P, P, P, I64, I64, I64, I, I, P, P],
+            "convrot_repack_weight": [P, I64, I64, P, P],
+            "convrot_unpack_weight": [P, I64, I64, P, P],
+            "convrot_linear_repacked": [P, P, P, P, I64, I64, I64, I, P, SZ, P, P],
+            "convrot_linear_prepared_repacked": [P, P, P, P, P, I64, I64, I64, P, P],
         }
         for name, args in sigs.items():
             f = getattr(L, name)
@@ -72,6 +76,8 @@ def lib() -> ctypes.CDLL:
         L.convrot_linear_single_kernel.restype = I
         L.convrot_linear_workspace_size.argtypes = [I64, I64]
         L.convrot_linear_workspace_size.restype = SZ
+        L.convrot_repacked_weight_size.argtypes = [I64, I64]
+        L.convrot_repacked_weight_size.restype = SZ
         L.convrot_status_string.argtypes = [I]
         L.convrot_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -189,6 +195,82 @@ def convrot_linear(x, qw, sw, bias, group: int, workspace=None, out=None, stream
     return out
 
 
+# ---------------------------------------------------------------------------
+# the reversible weight repack (block-major layout, include/convrot.h)
+# ---------------------------------------------------------------------------
+
+def convrot_repacked_weight_size(N: int, K: int) -> int:
+    return int(lib().convrot_repacked_weight_size(N, K))
+
+
+def convrot_repack_weight(qw, out=None, stream=None):
+    """Packed weights uint8 [N, K/2] -> the block-major repacked layout (a
+    flat uint8 tensor of convrot_repacked_weight_size(N, K) bytes)."""
+    N, half = _rows(qw, torch.uint8, "qw")
+    K = 2 * half
+    with torch.cuda.device(qw.device):
+        size = convrot_repacked_weight_size(N, K)
+        out = torch.empty(size, dtype=torch.uint8, device=qw.device) if out is None else out
+        _need(out, torch.uint8, "out", (size,), qw)
+        _check(lib().convrot_repack_weight(_p(qw), N, K, _p(out), _stream(stream)),
+               "convrot_repack_weight")
+    return out
+
+
+def convrot_unpack_weight(qw_rep, N: int, K: int, out=None, stream=None):
+    """The exact inverse of convrot_repack_weight -> uint8 [N, K/2]."""
+    _need(qw_rep, torch.uint8, "qw_rep", (convrot_repacked_weight_size(N, K),))
+    with torch.cuda.device(qw_rep.device):
+        out = torch.empty(N, K // 2, dtype=torch.uint8, device=qw_rep.device) if out is None else out
+        _need(out, torch.uint8, "out", (N, K // 2), qw_rep)
+        _check(lib().convrot_unpack_weight(_p(qw_rep), N, K, _p(out), _stream(stream)),
+               "convrot_unpack_weight")
+    return out
+
+
+def _weights_rep(qw_rep, sw, bias, K: int, like):
+    """Repacked weights (flat, sized for N = len(sw) rows), scales, bias."""
+    _need(sw, torch.float32, "sw", (None,), like)
+    N = sw.shape[0]
+    _need(qw_rep, torch.uint8, "qw_rep", (convrot_repacked_weight_size(N, K),), like)
+    _need_opt(bias, torch.bfloat16, "bias", (N,), like)
+    return N
+
+
+def convrot_linear_repacked(x, qw_rep, sw, bias, group: int, workspace=None, out=None,
+                            stream=None):
+    """convrot_linear with the weights in the repacked layout."""
+    M, K = _rows(x, torch.bfloat16, "x")
+    N = _weights_rep(qw_rep, sw, bias, K, x)
+    with torch.cuda.device(x.device):
+        need = convrot_linear_workspace_size(M, K)
+        if workspace is None:
+            workspace = torch.empty(max(1, need), dtype=torch.uint8, device=x.device)
+        _need(workspace, torch.uint8, "workspace", None, x)
+        if workspace.numel() < need:
+            raise ValueError(f"workspace holds {workspace.numel()} bytes, {need} needed")
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
+        _need(out, torch.bfloat16, "out", (M, N), x)
+        _check(lib().convrot_linear_repacked(_p(x), _p(qw_rep), _p(sw), _p(bias), M, N, K, group,
+                                             _p(workspace), workspace.numel(), _p(out),
+                                             _stream(stream)), "convrot_linear_repacked")
+    return out
+
+
+def convrot_linear_prepared_repacked(qx, sx, qw_rep, sw, bias, K: int, out=None, stream=None):
+    """convrot_linear_prepared with the weights in the repacked layout."""
+    M = _prepared(qx, sx, K)
+    _need(sx, torch.float32, "sx", (M,), qx)
+    N = _weights_rep(qw_rep, sw, bias, K, qx)
+    with torch.cuda.device(qx.device):
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=qx.device) if out is None else out
+        _need(out, torch.bfloat16, "out", (M, N), qx)
+        _check(lib().convrot_linear_prepared_repacked(_p(qx), _p(sx), _p(qw_rep), _p(sw), _p(bias),
+                                                      M, N, K, _p(out), _stream(stream)),
+               "convrot_linear_prepared_repacked")
+    return out
+
+
 def convrot_linear_noalloc(x, qw, sw, bias, group: int, out=None, stream=None):
     """The whole layer without a caller workspace: the library's fixed
     16 MiB scratch array holds the packed activations instead.  Meant for
@@ -255,12 +337,24 @@ TILES_256x128_PAIR = 6
 SKINNY_PAIR = 7
 
 
+TILES_REPACKED = 0x100
+
+
 def convrot_debug_gemm_tiles(qx, sx, qw, sw, bias, K: int, tiles: int, out_s32: bool = False,
-                             out=None, stream=None):
+                             out=None, stream=None, N: int | None = None):
     """Steps 3-4 (bf16 y) or step 3 alone (int32 acc, out_s32=True) with the
-    GEMM forced to one tile shape (TILES_*)."""
+    GEMM forced to one tile shape (TILES_*); tiles | TILES_REPACKED takes
+    qw in the repacked layout (a flat tensor; give N then)."""
     M = _prepared(qx, sx, K)
-    if out_s32:
+    if tiles & TILES_REPACKED:
+        if N is None:
+            raise ValueError("N is needed with repacked weights")
+        _need(qw, torch.uint8, "qw_rep", (convrot_repacked_weight_size(N, K),), qx)
+        if not out_s32:
+            _need(sx, torch.float32, "sx", (M,), qx)
+            _need(sw, torch.float32, "sw", (N,), qx)
+            _need_opt(bias, torch.bfloat16, "bias", (N,), qx)
+    elif out_s32:
         _need(qw, torch.uint8, "qw", (None, K // 2), qx)
         N = qw.shape[0]
     else:
@@ -308,6 +402,8 @@ def lib_w4a16() -> ctypes.CDLL:
             "convrot_w4a16_linear_prepared": [P, P, P, P, I64, I64, I64, P, P],
             "convrot_w4a16_linear": [P, P, P, P, I64, I64, I64, I, P, SZ, P, P],
             "convrot_w4a16_check_device_error": [P],
+            "convrot_w4a16_linear_prepared_repacked": [P, P, P, P, I64, I64, I64, P, P],
+            "convrot_w4a16_linear_repacked": [P, P, P, P, I64, I64, I64, I, P, SZ, P, P],
         }
         for name, args in sigs.items():
             f = getattr(L, name)
@@ -366,6 +462,39 @@ def convrot_w4a16_linear(x, qw, sw, bias, group: int, workspace=None, out=None, 
         _check(lib_w4a16().convrot_w4a16_linear(_p(x), _p(qw), _p(sw), _p(bias), M, N, K, group,
                                                 _p(workspace), workspace.numel(), _p(out),
                                                 _stream(stream)), "convrot_w4a16_linear")
+    return out
+
+
+def convrot_w4a16_linear_repacked(x, qw_rep, sw, bias, group: int, workspace=None, out=None,
+                                  stream=None):
+    """convrot_w4a16_linear with the weights in the repacked layout."""
+    M, K = _rows(x, torch.bfloat16, "x")
+    N = _weights_rep(qw_rep, sw, bias, K, x)
+    with torch.cuda.device(x.device):
+        need = convrot_w4a16_workspace_size(M, K)
+        if workspace is None:
+            workspace = torch.empty(max(1, need), dtype=torch.uint8, device=x.device)
+        _need(workspace, torch.uint8, "workspace", None, x)
+        if workspace.numel() < need:
+            raise ValueError(f"workspace holds {workspace.numel()} bytes, {need} needed")
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
+        _need(out, torch.bfloat16, "out", (M, N), x)
+        _check(lib_w4a16().convrot_w4a16_linear_repacked(
+            _p(x), _p(qw_rep), _p(sw), _p(bias), M, N, K, group, _p(workspace), workspace.numel(),
+            _p(out), _stream(stream)), "convrot_w4a16_linear_repacked")
+    return out
+
+
+def convrot_w4a16_linear_prepared_repacked(xr, qw_rep, sw, bias, out=None, stream=None):
+    """convrot_w4a16_linear_prepared with the weights in the repacked layout."""
+    M, K = _rows(xr, torch.bfloat16, "xr")
+    N = _weights_rep(qw_rep, sw, bias, K, xr)
+    with torch.cuda.device(xr.device):
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=xr.device) if out is None else out
+        _need(out, torch.bfloat16, "out", (M, N), xr)
+        _check(lib_w4a16().convrot_w4a16_linear_prepared_repacked(
+            _p(xr), _p(qw_rep), _p(sw), _p(bias), M, N, K, _p(out), _stream(stream)),
+            "convrot_w4a16_linear_prepared_repacked")
     return out
 
 

@@ -270,8 +270,25 @@ convrot_status launch_prep(int num_sms, const void *x, int64_t rows, int64_t K, 
     return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 
+// Packed rows [rows][K/2] (rep = false), or the block-major repacked layout
+// of the same bytes (rep = true): 3-D {128 bytes, rows, ceil(K/256) blocks},
+// boxes of box_bytes <= 128 inside one block.
 bool make_map(CUtensorMap *map, const uint8_t *base, int64_t rows, int64_t K, int box_bytes,
-              int box_rows, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE) {
+              int box_rows, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE,
+              bool rep = false) {
+    if (rep) {
+        if (box_bytes > 128) return false;
+        const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(rows),
+                                    static_cast<cuuint64_t>((K / 2 + 127) / 128)};
+        const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(rows) * 128};
+        const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_bytes),
+                                   static_cast<cuuint32_t>(box_rows), 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    }
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_bytes), static_cast<cuuint32_t>(box_rows)};
@@ -297,17 +314,20 @@ bool make_out_map(CUtensorMap *map, void *y, int64_t M, int64_t N) {
 }
 
 // slots: CTAs (CTA pairs when PAIR) the persistent grid may use.
+// wrep: the weights (qB, or qA in the swapped forms) are repacked.
 template <int BN, bool SWAP, bool OUT_S32, bool PAIR = false>
 convrot_status launch_gemm_cfg(int slots, const uint8_t *qA, const uint8_t *qB, int64_t rowsA,
                                int64_t rowsB, int64_t K, const float *sx, const float *sw,
                                const void *bias, void *out, int64_t M, int64_t N,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, bool wrep = false) {
     using C = gemm::Cfg<BN, SWAP, PAIR>;
     CUtensorMap tmA, tmB, tmY;
     constexpr int pkb = C::PKB;
     // A widened into TMEM reads its packed rows 128-byte swizzled.
     const CUtensorMapSwizzle swa = C::ATM ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
-    if (!make_map(&tmA, qA, rowsA, K, pkb, gemm::BM, swa) || !make_map(&tmB, qB, rowsB, K, pkb, C::BR))
+    if (wrep && pkb > 128) return CONVROT_ERR_UNSUPPORTED;   // boxes wider than a block
+    if (!make_map(&tmA, qA, rowsA, K, pkb, gemm::BM, swa, SWAP && wrep) ||
+        !make_map(&tmB, qB, rowsB, K, pkb, C::BR, CU_TENSOR_MAP_SWIZZLE_NONE, !SWAP && wrep))
         return CONVROT_ERR_CUDA;
     int use_tma_store = 0;
     if (!SWAP && !OUT_S32 && N % 8 == 0) {
@@ -339,7 +359,8 @@ convrot_status launch_gemm_cfg(int slots, const uint8_t *qA, const uint8_t *qB, 
     const cudaError_t e = cudaLaunchKernelEx(
         &cfg, gemm::gemm_kernel<BN, SWAP, OUT_S32, PAIR>, tmA, tmB, tmY, use_tma_store,
         static_cast<int>(rowsA), static_cast<int>(rowsB), static_cast<int>(K), sx, sw,
-        static_cast<const uint16_t *>(bias), out, static_cast<int>(M), static_cast<int>(N));
+        static_cast<const uint16_t *>(bias), out, static_cast<int>(M), static_cast<int>(N),
+        wrep ? 1 : 0);
     return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 
@@ -351,11 +372,11 @@ template <int BN, bool OUT_S32, bool PAIR = false>
 convrot_status launch_skinny_cfg(int num_sms, const uint8_t *qx, const float *sx,
                                  const uint8_t *qw, const float *sw, const void *bias, int64_t M,
                                  int64_t N, int64_t K, void *out, bool weights_ready,
-                                 cudaStream_t stream) {
+                                 cudaStream_t stream, bool wrep) {
     using C = skinny::Cfg<BN, PAIR>;
     const int R = skinny::rows_per_cta(N, num_sms);
     CUtensorMap tmA, tmB;
-    if (!make_map(&tmA, qw, N, K, skinny::kPKB, R, CU_TENSOR_MAP_SWIZZLE_128B) ||
+    if (!make_map(&tmA, qw, N, K, skinny::kPKB, R, CU_TENSOR_MAP_SWIZZLE_128B, wrep) ||
         !make_map(&tmB, qx, M, K, skinny::kPKB, C::BR))
         return CONVROT_ERR_CUDA;
     int64_t ctas = (N + R - 1) / R;
@@ -376,7 +397,7 @@ convrot_status launch_skinny_cfg(int num_sms, const uint8_t *qx, const float *sx
     cfg.numAttrs = PAIR ? 2 : 1;
     const cudaError_t e = cudaLaunchKernelEx(
         &cfg, skinny::skinny_kernel<BN, OUT_S32, PAIR>, tmA, tmB, R, weights_ready ? 1 : 0,
-        static_cast<int>(K), sx, sw, static_cast<const uint16_t *>(bias), out, static_cast<int>(M),
+        static_cast<int>(K), wrep ? 1 : 0, sx, sw, static_cast<const uint16_t *>(bias), out, static_cast<int>(M),
         static_cast<int>(N));
     return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
@@ -384,28 +405,29 @@ convrot_status launch_skinny_cfg(int num_sms, const uint8_t *qx, const float *sx
 template <bool OUT_S32>
 convrot_status launch_skinny(int num_sms, const uint8_t *qx, const float *sx, const uint8_t *qw,
                              const float *sw, const void *bias, int64_t M, int64_t N, int64_t K,
-                             void *out, bool weights_ready, cudaStream_t stream, bool pair = false) {
+                             void *out, bool weights_ready, cudaStream_t stream, bool pair = false,
+                             bool wrep = false) {
     if (pair) {
         if (M <= 32)
             return launch_skinny_cfg<32, OUT_S32, true>(num_sms, qx, sx, qw, sw, bias, M, N, K, out,
-                                                        weights_ready, stream);
+                                                        weights_ready, stream, wrep);
         if (M <= 64)
             return launch_skinny_cfg<64, OUT_S32, true>(num_sms, qx, sx, qw, sw, bias, M, N, K, out,
-                                                        weights_ready, stream);
+                                                        weights_ready, stream, wrep);
         return launch_skinny_cfg<128, OUT_S32, true>(num_sms, qx, sx, qw, sw, bias, M, N, K, out,
-                                                     weights_ready, stream);
+                                                     weights_ready, stream, wrep);
     }
     if (M <= 16)
         return launch_skinny_cfg<16, OUT_S32>(num_sms, qx, sx, qw, sw, bias, M, N, K, out,
-                                              weights_ready, stream);
+                                              weights_ready, stream, wrep);
     if (M <= 32)
         return launch_skinny_cfg<32, OUT_S32>(num_sms, qx, sx, qw, sw, bias, M, N, K, out,
-                                              weights_ready, stream);
+                                              weights_ready, stream, wrep);
     if (M <= 64)
         return launch_skinny_cfg<64, OUT_S32>(num_sms, qx, sx, qw, sw, bias, M, N, K, out,
-                                              weights_ready, stream);
+                                              weights_ready, stream, wrep);
     return launch_skinny_cfg<128, OUT_S32>(num_sms, qx, sx, qw, sw, bias, M, N, K, out,
-                                           weights_ready, stream);
+                                           weights_ready, stream, wrep);
 }
 
 // GEMM forms: the automatic choice, the three token-major tile shapes, and
@@ -422,7 +444,8 @@ template <bool OUT_S32>
 convrot_status launch_gemm(const DeviceState &ds, const uint8_t *qx, const float *sx,
                            const uint8_t *qw, const float *sw, const void *bias, int64_t M,
                            int64_t N, int64_t K, void *out, cudaStream_t stream,
-                           int tiles = kTilesAuto, bool weights_ready = false) {
+                           int tiles = kTilesAuto, bool weights_ready = false,
+                           bool wrep = false) {
     const int num_sms = ds.num_sms;
     // Few tokens: the weight-streaming form.  (The CTA-pair form measured
     // the same at 128 tokens and slower below: each SM's tensor core does
@@ -434,19 +457,19 @@ convrot_status launch_gemm(const DeviceState &ds, const uint8_t *qx, const float
     if (tiles == kSkinnyPair && ds.pair_clusters <= 0) return CONVROT_ERR_UNSUPPORTED;
     if (tiles == kSkinnyTmem || tiles == kSkinnyPair)
         return launch_skinny<OUT_S32>(num_sms, qx, sx, qw, sw, bias, M, N, K, out, weights_ready,
-                                      stream, tiles == kSkinnyPair);
+                                      stream, tiles == kSkinnyPair, wrep);
     if (tiles == kSkinnySmem) {
         if (M <= 16)
             return launch_gemm_cfg<16, true, OUT_S32>(num_sms, qw, qx, N, M, K, sx, sw, bias, out, M,
-                                                      N, stream);
+                                                      N, stream, wrep);
         if (M <= 32)
             return launch_gemm_cfg<32, true, OUT_S32>(num_sms, qw, qx, N, M, K, sx, sw, bias, out, M,
-                                                      N, stream);
+                                                      N, stream, wrep);
         if (M <= 64)
             return launch_gemm_cfg<64, true, OUT_S32>(num_sms, qw, qx, N, M, K, sx, sw, bias, out, M,
-                                                      N, stream);
+                                                      N, stream, wrep);
         return launch_gemm_cfg<128, true, OUT_S32>(num_sms, qw, qx, N, M, K, sx, sw, bias, out, M, N,
-                                                   stream);
+                                                   stream, wrep);
     }
     if (tiles == kTilesAuto) {
         // Measured on layers of 1024-8192 tokens and K 3072-12288: the
@@ -476,19 +499,19 @@ convrot_status launch_gemm(const DeviceState &ds, const uint8_t *qx, const float
     if (tiles == kTiles256x128Pair) {
         if (ds.pair_clusters <= 0) return CONVROT_ERR_UNSUPPORTED;
         return launch_gemm_cfg<128, false, OUT_S32, true>(ds.pair_clusters, qx, qw, M, N, K, sx, sw,
-                                                          bias, out, M, N, stream);
+                                                          bias, out, M, N, stream, wrep);
     }
     if (tiles == kTiles256x192Pair) {
         if (ds.pair_clusters <= 0) return CONVROT_ERR_UNSUPPORTED;
         return launch_gemm_cfg<192, false, OUT_S32, true>(ds.pair_clusters, qx, qw, M, N, K, sx, sw,
-                                                          bias, out, M, N, stream);
+                                                          bias, out, M, N, stream, wrep);
     }
     if (tiles == kTiles128x192)
         return launch_gemm_cfg<192, false, OUT_S32>(num_sms, qx, qw, M, N, K, sx, sw, bias, out, M,
-                                                    N, stream);
+                                                    N, stream, wrep);
     if (tiles == kTiles128x256)
         return launch_gemm_cfg<256, false, OUT_S32>(num_sms, qx, qw, M, N, K, sx, sw, bias, out, M,
-                                                    N, stream);
+                                                    N, stream, wrep);
     return CONVROT_ERR_SHAPE;
 }
 
@@ -513,30 +536,31 @@ int decode_stages(int64_t M, int64_t K, int group, int R = decode::kRows) {
 template <int MT, int G>
 convrot_status launch_decode_cfg(int num_sms, int SP, const void *x, const uint8_t *qw,
                                  const float *sw, const void *bias, int64_t M, int64_t N,
-                                 int64_t K, void *y, cudaStream_t stream) {
+                                 int64_t K, void *y, cudaStream_t stream, bool wrep) {
     const int R = skinny::rows_per_cta(N, num_sms);
     CUtensorMap tmW;
-    if (!make_map(&tmW, qw, N, K, decode::kPKB, R, CU_TENSOR_MAP_SWIZZLE_128B)) return CONVROT_ERR_CUDA;
+    if (!make_map(&tmW, qw, N, K, decode::kPKB, R, CU_TENSOR_MAP_SWIZZLE_128B, wrep))
+        return CONVROT_ERR_CUDA;
     const size_t smem = decode::smem_bytes(MT, G, static_cast<int>(K), SP, R) + 1024;
     const dim3 grid(static_cast<unsigned>((N + R - 1) / R));
     decode::decode_kernel<MT, G><<<grid, decode::kThreads, smem, stream>>>(
         tmW, static_cast<const uint16_t *>(x), static_cast<int>(M), static_cast<int>(N),
-        static_cast<int>(K), R, SP, sw, static_cast<const uint16_t *>(bias),
+        static_cast<int>(K), R, SP, wrep ? 1 : 0, sw, static_cast<const uint16_t *>(bias),
         static_cast<uint16_t *>(y));
     return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 
 convrot_status launch_decode(int num_sms, int SP, const void *x, const uint8_t *qw, const float *sw,
                              const void *bias, int64_t M, int64_t N, int64_t K, int group, void *y,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, bool wrep = false) {
     if (group == 64) {
-        if (M <= 1) return launch_decode_cfg<1, 64>(num_sms, SP, x, qw, sw, bias, M, N, K, y, stream);
-        if (M <= 2) return launch_decode_cfg<2, 64>(num_sms, SP, x, qw, sw, bias, M, N, K, y, stream);
-        return launch_decode_cfg<4, 64>(num_sms, SP, x, qw, sw, bias, M, N, K, y, stream);
+        if (M <= 1) return launch_decode_cfg<1, 64>(num_sms, SP, x, qw, sw, bias, M, N, K, y, stream, wrep);
+        if (M <= 2) return launch_decode_cfg<2, 64>(num_sms, SP, x, qw, sw, bias, M, N, K, y, stream, wrep);
+        return launch_decode_cfg<4, 64>(num_sms, SP, x, qw, sw, bias, M, N, K, y, stream, wrep);
     }
-    if (M <= 1) return launch_decode_cfg<1, 256>(num_sms, SP, x, qw, sw, bias, M, N, K, y, stream);
-    if (M <= 2) return launch_decode_cfg<2, 256>(num_sms, SP, x, qw, sw, bias, M, N, K, y, stream);
-    return launch_decode_cfg<4, 256>(num_sms, SP, x, qw, sw, bias, M, N, K, y, stream);
+    if (M <= 1) return launch_decode_cfg<1, 256>(num_sms, SP, x, qw, sw, bias, M, N, K, y, stream, wrep);
+    if (M <= 2) return launch_decode_cfg<2, 256>(num_sms, SP, x, qw, sw, bias, M, N, K, y, stream, wrep);
+    return launch_decode_cfg<4, 256>(num_sms, SP, x, qw, sw, bias, M, N, K, y, stream, wrep);
 }
 
 convrot_status check_gemm_args(const uint8_t *qx, const uint8_t *qw, int64_t M, int64_t N,
@@ -550,6 +574,107 @@ convrot_status check_gemm_args(const uint8_t *qx, const uint8_t *qw, int64_t M, 
 }
 
 inline size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+// steps 3-4 on prepared operands; wrep: qw is in the repacked layout
+convrot_status linear_prepared_impl(const uint8_t *qx, const float *sx, const uint8_t *qw,
+                                    const float *sw, const void *bias_bf16, int64_t M, int64_t N,
+                                    int64_t K, void *y_bf16, cudaStream_t stream, bool wrep) {
+    if (M < 0 || N < 0) return CONVROT_ERR_SHAPE;
+    if (M == 0 || N == 0) return CONVROT_OK;
+    convrot_status st = check_gemm_args(qx, qw, M, N, K);
+    if (st != CONVROT_OK) return st;
+    if (!sx || !sw || !y_bf16) return CONVROT_ERR_NULL;
+    if (!aligned16(sx) || !aligned16(sw) || !aligned16(y_bf16) ||
+        (bias_bf16 && !aligned16(bias_bf16)))
+        return CONVROT_ERR_ALIGN;
+    int dev;
+    if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    if ((st = check_device_ptrs(dev, {qx, sx, qw, sw, bias_bf16, y_bf16})) != CONVROT_OK) return st;
+    return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream,
+                              kTilesAuto, false, wrep);
+}
+
+// steps 1-4; wrep: qw is in the repacked layout
+convrot_status linear_impl(const void *x_bf16, const uint8_t *qw, const float *sw,
+                           const void *bias_bf16, int64_t M, int64_t N, int64_t K, int group,
+                           void *workspace, size_t ws_bytes, void *y_bf16, cudaStream_t stream,
+                           bool wrep) {
+    convrot_status st = check_shape(M, K, group);
+    if (st != CONVROT_OK) return st;
+    if (N < 0) return CONVROT_ERR_SHAPE;
+    if (M == 0 || N == 0) return CONVROT_OK;
+    if (!x_bf16 || !qw || !sw || !y_bf16 || !workspace) return CONVROT_ERR_NULL;
+    if (ws_bytes < convrot_linear_workspace_size(M, K) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return CONVROT_ERR_WORKSPACE;
+    if (!aligned16(x_bf16) || !aligned16(qw) || !aligned16(sw) || !aligned16(y_bf16) ||
+        (bias_bf16 && !aligned16(bias_bf16)))
+        return CONVROT_ERR_ALIGN;
+    if ((st = check_gemm_args(qw, qw, M, N, K)) != CONVROT_OK) return st;
+    int dev;
+    if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    if ((st = check_device_ptrs(dev, {x_bf16, qw, sw, bias_bf16, workspace, y_bf16})) != CONVROT_OK)
+        return st;
+    // 1..4 tokens: one kernel (the workspace is not touched).  Eligibility
+    // is decided for the largest slice (128 rows), so that it depends on
+    // (M, K, group) alone, as convrot_linear_single_kernel reports it; the
+    // ring then takes what the actual slice leaves.
+    if (decode_stages(M, K, group) > 0)
+        if (const int sp = decode_stages(M, K, group, skinny::rows_per_cta(N, g_dev[dev].num_sms)))
+            return launch_decode(g_dev[dev].num_sms, sp, x_bf16, qw, sw, bias_bf16, M, N, K,
+                                 group, y_bf16, stream, wrep);
+    uint8_t *qx = static_cast<uint8_t *>(workspace);
+    float *sx = reinterpret_cast<float *>(qx + round256(static_cast<size_t>(M) * (K / 2)));
+    if ((st = launch_prep(g_dev[dev].num_sms, x_bf16, M, K, group, qx, sx, nullptr, stream)) != CONVROT_OK)
+        return st;
+    return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream,
+                              kTilesAuto, true, wrep);
+}
+
+// The reversible block-major repack (16 bytes per thread, grid-stride).
+// Forward: chunk i of the repacked layout is 16-byte chunk j = i mod 8 of
+// 128-byte block b of row n, (b, n) = (i / 8) divmod N, zero past the row's
+// end.  Inverse: chunk i of the canonical layout (row n = i / row16) reads
+// its chunk of its block.
+__global__ void repack_kernel(const uint4 *__restrict__ in, uint4 *__restrict__ out, int64_t N,
+                              int64_t row16, int64_t nblk, int inverse) {
+    const int64_t total = inverse ? N * row16 : nblk * N * 8;
+    const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += step) {
+        if (!inverse) {
+            const int64_t j = i & 7, t = i >> 3;
+            const int64_t b = t / N, n = t - b * N;
+            const int64_t c16 = b * 8 + j;               // 16-byte chunk of the row
+            out[i] = c16 < row16 ? in[n * row16 + c16] : make_uint4(0u, 0u, 0u, 0u);
+        } else {
+            const int64_t n = i / row16, c16 = i - n * row16;
+            out[i] = in[((c16 >> 3) * N + n) * 8 + (c16 & 7)];
+        }
+    }
+}
+
+convrot_status repack_common(const uint8_t *in, int64_t N, int64_t K, uint8_t *out,
+                             cudaStream_t stream, int inverse) {
+    if (N < 0 || K < 64 || K > CONVROT_MAX_K || K % 64 || N > (int64_t(1) << 30))
+        return CONVROT_ERR_SHAPE;
+    if (N == 0) return CONVROT_OK;
+    if (!in || !out) return CONVROT_ERR_NULL;
+    if (!aligned16(in) || !aligned16(out)) return CONVROT_ERR_ALIGN;
+    const size_t canon = static_cast<size_t>(N) * static_cast<size_t>(K / 2);
+    const size_t rep = convrot_repacked_weight_size(N, K);
+    const uintptr_t a = reinterpret_cast<uintptr_t>(in), b = reinterpret_cast<uintptr_t>(out);
+    const size_t na = inverse ? rep : canon, nb = inverse ? canon : rep;
+    if (a < b + nb && b < a + na) return CONVROT_ERR_OVERLAP;
+    int dev;
+    convrot_status st = device_setup(&dev);
+    if (st != CONVROT_OK) return st;
+    if ((st = check_device_ptrs(dev, {in, out})) != CONVROT_OK) return st;
+    const int64_t row16 = K / 32, nblk = (K / 2 + 127) / 128;
+    repack_kernel<<<g_dev[dev].num_sms * 8, 256, 0, stream>>>(
+        reinterpret_cast<const uint4 *>(in), reinterpret_cast<uint4 *>(out), N, row16, nblk, inverse);
+    return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -570,6 +695,8 @@ const char *convrot_status_string(convrot_status s) {
             return "CONVROT_ERR_SCRATCH_LIMIT: larger than the built-in scratch array";
         case CONVROT_ERR_NOT_DEVICE:
             return "CONVROT_ERR_NOT_DEVICE: a pointer is not memory of the current device";
+        case CONVROT_ERR_OVERLAP:
+            return "CONVROT_ERR_OVERLAP: input and output buffers overlap";
     }
     return "CONVROT_ERR_UNKNOWN";
 }
@@ -602,54 +729,45 @@ size_t convrot_linear_workspace_size(int64_t M, int64_t K) {
 convrot_status convrot_linear_prepared(const uint8_t *qx, const float *sx, const uint8_t *qw,
                                        const float *sw, const void *bias_bf16, int64_t M, int64_t N,
                                        int64_t K, void *y_bf16, convrot_stream_t stream) {
-    if (M < 0 || N < 0) return CONVROT_ERR_SHAPE;
-    if (M == 0 || N == 0) return CONVROT_OK;
-    convrot_status st = check_gemm_args(qx, qw, M, N, K);
-    if (st != CONVROT_OK) return st;
-    if (!sx || !sw || !y_bf16) return CONVROT_ERR_NULL;
-    if (!aligned16(sx) || !aligned16(sw) || !aligned16(y_bf16) ||
-        (bias_bf16 && !aligned16(bias_bf16)))
-        return CONVROT_ERR_ALIGN;
-    int dev;
-    if ((st = device_setup(&dev)) != CONVROT_OK) return st;
-    if ((st = check_device_ptrs(dev, {qx, sx, qw, sw, bias_bf16, y_bf16})) != CONVROT_OK) return st;
-    return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream);
+    return linear_prepared_impl(qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream, false);
 }
 
 convrot_status convrot_linear(const void *x_bf16, const uint8_t *qw, const float *sw,
                               const void *bias_bf16, int64_t M, int64_t N, int64_t K, int group,
                               void *workspace, size_t ws_bytes, void *y_bf16,
                               convrot_stream_t stream) {
-    convrot_status st = check_shape(M, K, group);
-    if (st != CONVROT_OK) return st;
-    if (N < 0) return CONVROT_ERR_SHAPE;
-    if (M == 0 || N == 0) return CONVROT_OK;
-    if (!x_bf16 || !qw || !sw || !y_bf16 || !workspace) return CONVROT_ERR_NULL;
-    if (ws_bytes < convrot_linear_workspace_size(M, K) ||
-        (reinterpret_cast<uintptr_t>(workspace) & 255u))
-        return CONVROT_ERR_WORKSPACE;
-    if (!aligned16(x_bf16) || !aligned16(qw) || !aligned16(sw) || !aligned16(y_bf16) ||
-        (bias_bf16 && !aligned16(bias_bf16)))
-        return CONVROT_ERR_ALIGN;
-    if ((st = check_gemm_args(qw, qw, M, N, K)) != CONVROT_OK) return st;
-    int dev;
-    if ((st = device_setup(&dev)) != CONVROT_OK) return st;
-    if ((st = check_device_ptrs(dev, {x_bf16, qw, sw, bias_bf16, workspace, y_bf16})) != CONVROT_OK)
-        return st;
-    // 1..4 tokens: one kernel (the workspace is not touched).  Eligibility
-    // is decided for the largest slice (128 rows), so that it depends on
-    // (M, K, group) alone, as convrot_linear_single_kernel reports it; the
-    // ring then takes what the actual slice leaves.
-    if (decode_stages(M, K, group) > 0)
-        if (const int sp = decode_stages(M, K, group, skinny::rows_per_cta(N, g_dev[dev].num_sms)))
-            return launch_decode(g_dev[dev].num_sms, sp, x_bf16, qw, sw, bias_bf16, M, N, K,
-                                 group, y_bf16, stream);
-    uint8_t *qx = static_cast<uint8_t *>(workspace);
-    float *sx = reinterpret_cast<float *>(qx + round256(static_cast<size_t>(M) * (K / 2)));
-    if ((st = launch_prep(g_dev[dev].num_sms, x_bf16, M, K, group, qx, sx, nullptr, stream)) != CONVROT_OK)
-        return st;
-    return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream,
-                              kTilesAuto, true);
+    return linear_impl(x_bf16, qw, sw, bias_bf16, M, N, K, group, workspace, ws_bytes, y_bf16,
+                       stream, false);
+}
+
+size_t convrot_repacked_weight_size(int64_t N, int64_t K) {
+    if (N <= 0 || K <= 0) return 0;
+    return static_cast<size_t>(N) * static_cast<size_t>((K / 2 + 127) / 128) * 128;
+}
+
+convrot_status convrot_repack_weight(const uint8_t *qw, int64_t N, int64_t K, uint8_t *qw_rep,
+                                     convrot_stream_t stream) {
+    return repack_common(qw, N, K, qw_rep, stream, 0);
+}
+
+convrot_status convrot_unpack_weight(const uint8_t *qw_rep, int64_t N, int64_t K, uint8_t *qw,
+                                     convrot_stream_t stream) {
+    return repack_common(qw_rep, N, K, qw, stream, 1);
+}
+
+convrot_status convrot_linear_repacked(const void *x_bf16, const uint8_t *qw_rep, const float *sw,
+                                       const void *bias_bf16, int64_t M, int64_t N, int64_t K,
+                                       int group, void *workspace, size_t ws_bytes, void *y_bf16,
+                                       convrot_stream_t stream) {
+    return linear_impl(x_bf16, qw_rep, sw, bias_bf16, M, N, K, group, workspace, ws_bytes, y_bf16,
+                       stream, true);
+}
+
+convrot_status convrot_linear_prepared_repacked(const uint8_t *qx, const float *sx,
+                                                const uint8_t *qw_rep, const float *sw,
+                                                const void *bias_bf16, int64_t M, int64_t N,
+                                                int64_t K, void *y_bf16, convrot_stream_t stream) {
+    return linear_prepared_impl(qx, sx, qw_rep, sw, bias_bf16, M, N, K, y_bf16, stream, true);
 }
 
 int convrot_linear_single_kernel(int64_t M, int64_t K, int group) {
@@ -690,6 +808,8 @@ convrot_status convrot_debug_gemm_tiles(const uint8_t *qx, const float *sx, cons
                                         int64_t N, int64_t K, int tiles, int out_s32, void *out,
                                         convrot_stream_t stream) {
     if (M < 0 || N < 0) return CONVROT_ERR_SHAPE;
+    const bool wrep = (tiles & CONVROT_TILES_REPACKED) != 0;
+    tiles &= ~CONVROT_TILES_REPACKED;
     if (tiles < kTilesAuto || tiles > kSkinnyPair) return CONVROT_ERR_SHAPE;
     if (M == 0 || N == 0) return CONVROT_OK;
     convrot_status st = check_gemm_args(qx, qw, M, N, K);
@@ -704,8 +824,9 @@ convrot_status convrot_debug_gemm_tiles(const uint8_t *qx, const float *sx, cons
     if (!out_s32 && (st = check_device_ptrs(dev, {sx, sw, bias_bf16})) != CONVROT_OK) return st;
     if (out_s32)
         return launch_gemm<true>(g_dev[dev], qx, nullptr, qw, nullptr, nullptr, M, N, K, out, stream,
-                                 tiles);
-    return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, out, stream, tiles);
+                                 tiles, false, wrep);
+    return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, out, stream, tiles,
+                              false, wrep);
 }
 
 convrot_status convrot_check_device_error(convrot_stream_t stream) {

@@ -139,12 +139,13 @@ __device__ __forceinline__ bool gemv(uint32_t sbase, int slot, int blk, uint32_t
     return ok;
 }
 
-// tmW: packed weights [N][K/2], box 128 B x R rows, 128-byte swizzle.
+// tmW: packed weights [N][K/2], box 128 B x R rows, 128-byte swizzle (3-D
+// over the block-major repacked layout when wrep).
 // x: bf16 [M][K]; y: bf16 [M][N]; sw: fp32 [N]; bias: bf16 [N] or null.
 template <int MT, int G>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t *__restrict__ x, int M,
-              int N, int K, int R, int SP, const float *__restrict__ sw,
+              int N, int K, int R, int SP, int wrep, const float *__restrict__ sw,
               const uint16_t *__restrict__ bias, uint16_t *__restrict__ y) {
     static_assert(MT == 1 || MT == 2 || MT == 4, "1, 2 or 4 tokens");
     constexpr float kNorm = (G == 64) ? 0.125f : 0.0625f;   // 2^-digits
@@ -204,8 +205,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t *__restric
         for (int kp = 0; kp < SP && kp < num_kp; ++kp) {
             ptx::mbar_arrive_expect_tx(full_p(kp), stage_tx);
             for (int q = 0; q < kBlocks; ++q)
-                ptx::tma_load_2d(sbase + kp * slot + q * blk, &tmW, full_p(kp),
-                                 (kp * kBlocks + q) * kPKB, n0);
+                ptx::tma_load_rows(sbase + kp * slot + q * blk, &tmW, full_p(kp),
+                                   (kp * kBlocks + q) * kPKB, n0, wrep);
         }
     }
     __syncthreads();
@@ -218,8 +219,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t *__restric
                 if (!ptx::mbar_wait(empty_p(s), ((kp / SP) - 1) & 1, abort_flag)) break;
                 ptx::mbar_arrive_expect_tx(full_p(s), stage_tx);
                 for (int q = 0; q < kBlocks; ++q)
-                    ptx::tma_load_2d(sbase + s * slot + q * blk, &tmW, full_p(s),
-                                     (kp * kBlocks + q) * kPKB, n0);
+                    ptx::tma_load_rows(sbase + s * slot + q * blk, &tmW, full_p(s),
+                                       (kp * kBlocks + q) * kPKB, n0, wrep);
             }
         }
         return;

@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmY, int use_tma_store, int rowsA, int rowsB,
             int K, const float *__restrict__ sx, const float *__restrict__ sw,
-            const uint16_t *__restrict__ bias, void *__restrict__ out, int M, int N) {
+            const uint16_t *__restrict__ bias, void *__restrict__ out, int M, int N, int wrep) {
     using C = Cfg<BN, SWAP, PAIR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -293,10 +293,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             for (int kp = 0; kp < num_kp; ++kp) {
                 if (!ptx::mbar_wait(empty_p(ps), ph ^ 1, abort_flag)) { ok = false; break; }
                 ptx::mbar_arrive_expect_tx(full_p(ps), C::PA + C::PB);
-                ptx::tma_load_2d(sbase + C::OFF_PA + ps * C::PA, &tmA, full_p(ps), kp * C::PKB,
-                                 ta * C::TM + static_cast<int>(rank) * BM);
-                ptx::tma_load_2d(sbase + C::OFF_PB + ps * C::PB, &tmB, full_p(ps), kp * C::PKB,
-                                 tb * BN + static_cast<int>(rank) * C::BR);
+                // the weights (B, or A in the swapped form) may be repacked
+                ptx::tma_load_rows(sbase + C::OFF_PA + ps * C::PA, &tmA, full_p(ps), kp * C::PKB,
+                                   ta * C::TM + static_cast<int>(rank) * BM, SWAP ? wrep : 0);
+                ptx::tma_load_rows(sbase + C::OFF_PB + ps * C::PB, &tmB, full_p(ps), kp * C::PKB,
+                                   tb * BN + static_cast<int>(rank) * C::BR, SWAP ? 0 : wrep);
                 if (++ps == C::SP) { ps = 0; ph ^= 1; }
             }
         }

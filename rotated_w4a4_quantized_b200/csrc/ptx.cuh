@@ -205,6 +205,28 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
+// 3-D tiled load, this CTA only (no multicast).  x is the innermost
+// coordinate in bytes; callers keep it a multiple of 16.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
+// A box of packed weight rows: bytes [x, x + box) of rows y .. y + box rows.
+// rep = 0: the canonical N x packed-K layout through a 2-D map.  rep = 1:
+// the block-major repacked layout (128-byte column block b of all rows
+// before block b + 1) through a 3-D map {128 bytes, rows, blocks}; the box
+// stays inside one block (x % 128 + box width <= 128).
+__device__ __forceinline__ void tma_load_rows(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                              int x, int y, int rep) {
+    if (rep) tma_load_3d(dst, map, bar, x & 127, y, x >> 7);
+    else tma_load_2d(dst, map, bar, x, y);
+}
+
 // 2-D tiled store of a shared-memory box to global memory (parts of the box
 // outside the tensor are skipped), tracked by this thread's bulk async-group.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int x, int y) {

@@ -107,13 +107,14 @@ inline int rows_per_cta(int64_t N, int num_sms) {
 
 // tmA: packed weights [N][K/2], box 128 B x R rows, 128-byte swizzle.
 // tmB: packed tokens [M][K/2], box 128 B x Cfg::BR rows.
+// wrep: the weights are in the block-major repacked layout (3-D tmA).
 // early_a: the weights were complete before the preceding kernel on the
 // stream started, so they may be loaded before waiting for it.
 // OUT_S32: write the integer accumulators (test hook) instead of bf16.
 template <int BN, bool OUT_S32, bool PAIR = false>
 __global__ void __launch_bounds__(kThreads, 1)
 skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              int R, int early_a, int K, const float *__restrict__ sx,
+              int R, int early_a, int K, int wrep, const float *__restrict__ sx,
               const float *__restrict__ sw, const uint16_t *__restrict__ bias,
               void *__restrict__ out, int M, int N) {
     using C = Cfg<BN, PAIR>;
@@ -171,7 +172,8 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         ptx::fence_mbar_init();
         for (int kp = 0; kp < early; ++kp) {
             ptx::mbar_arrive_expect_tx(full_a(kp), a_tx);
-            ptx::tma_load_2d(sbase + C::OFF_PA + kp * C::PA, &tmA, full_a(kp), kp * kPKB, n0);
+            ptx::tma_load_rows(sbase + C::OFF_PA + kp * C::PA, &tmA, full_a(kp), kp * kPKB, n0,
+                               wrep);
         }
     }
     if (warp == kWarpMma) {
@@ -205,7 +207,8 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 const int s = kp % C::SP;
                 if (!ptx::mbar_wait(empty_a(s), ((kp / C::SP) & 1) ^ 1, abort_flag)) break;
                 ptx::mbar_arrive_expect_tx(full_a(s), a_tx);
-                ptx::tma_load_2d(sbase + C::OFF_PA + s * C::PA, &tmA, full_a(s), kp * kPKB, n0);
+                ptx::tma_load_rows(sbase + C::OFF_PA + s * C::PA, &tmA, full_a(s), kp * kPKB, n0,
+                                   wrep);
             }
             if (kp < num_kp) drain(full_a, kp, C::SP);
         }

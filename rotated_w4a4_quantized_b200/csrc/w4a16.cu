@@ -237,11 +237,12 @@ __device__ __forceinline__ void widen_word(uint32_t w, uint32_t (&o)[4]) {
 }
 
 // tmA: xr bf16 [M][K], box 64 x TN, 128-byte swizzle.  tmB: qw u8
-// [N][K/2], box 64 B x 128, no swizzle.  K % 64 == 0.
+// [N][K/2], box 64 B x 128, no swizzle (3-D over the block-major repacked
+// layout when wrep).  K % 64 == 0.
 template <int TN, bool SWAP>
 __global__ void __launch_bounds__(kThreads, 1)
 w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                  int M, int N, int K, const float *__restrict__ sw,
+                  int M, int N, int K, int wrep, const float *__restrict__ sw,
                   const uint16_t *__restrict__ bias, uint16_t *__restrict__ y) {
     using C = Cfg<TN, SWAP>;
     constexpr int SP = C::SP, SU = C::SU, KBS = C::KBS;
@@ -320,8 +321,8 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                 for (int i = 0; i < nk; ++i)
                     ptx::tma_load_2d(sbase + C::OFF_XR + ps * C::XR_ST + i * C::XR_KB, &tmA,
                                      full_p(ps), (kp * KBS + i) * KB, ta * TN);
-                ptx::tma_load_2d(sbase + C::OFF_PB + ps * C::PB_ST, &tmB, full_p(ps), kp * C::PKB,
-                                 tb * C::WT);
+                ptx::tma_load_rows(sbase + C::OFF_PB + ps * C::PB_ST, &tmB, full_p(ps),
+                                   kp * C::PKB, tb * C::WT, wrep);
                 if (++ps == SP) { ps = 0; ph ^= 1; }
             }
         }
@@ -670,7 +671,7 @@ convrot_status launch_rotate(int num_sms, const void *x, int64_t M, int64_t K, i
 template <int TN, bool SWAP>
 convrot_status launch_gemm_cfg(int num_sms, const void *xr, const uint8_t *qw, const float *sw,
                                const void *bias, int64_t M, int64_t N, int64_t K, void *y,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, bool wrep) {
     using C = w4a16::Cfg<TN, SWAP>;
     CUtensorMap tmA, tmB;
     {
@@ -684,7 +685,20 @@ convrot_status launch_gemm_cfg(int num_sms, const void *xr, const uint8_t *qw, c
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return CONVROT_ERR_CUDA;
     }
-    {
+    if (wrep) {
+        // the block-major repacked weights: {128 bytes, N rows, ceil(K/256)
+        // blocks}; a box of PKB <= 128 bytes stays inside one block
+        const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(N),
+                                    static_cast<cuuint64_t>((K / 2 + 127) / 128)};
+        const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(N) * 128};
+        const cuuint32_t box[3] = {static_cast<cuuint32_t>(C::PKB), static_cast<cuuint32_t>(C::WT), 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (g_encode(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(qw), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONVROT_ERR_CUDA;
+    } else {
         const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
         const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
         const cuuint32_t box[2] = {static_cast<cuuint32_t>(C::PKB),
@@ -710,7 +724,8 @@ convrot_status launch_gemm_cfg(int num_sms, const void *xr, const uint8_t *qw, c
     cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(
         &cfg, w4a16::w4a16_gemm_kernel<TN, SWAP>, tmA, tmB, static_cast<int>(M),
-        static_cast<int>(N), static_cast<int>(K), sw, static_cast<const uint16_t *>(bias),
+        static_cast<int>(N), static_cast<int>(K), wrep ? 1 : 0, sw,
+        static_cast<const uint16_t *>(bias),
         static_cast<uint16_t *>(y));
     return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
@@ -719,11 +734,11 @@ convrot_status launch_gemm_cfg(int num_sms, const void *xr, const uint8_t *qw, c
 // 16-, 32- or 64-wide side; beyond that, 128 x 256 token-by-weight tiles.
 convrot_status launch_gemm(int num_sms, const void *xr, const uint8_t *qw, const float *sw,
                            const void *bias, int64_t M, int64_t N, int64_t K, void *y,
-                           cudaStream_t stream) {
-    if (M <= 16) return launch_gemm_cfg<16, true>(num_sms, xr, qw, sw, bias, M, N, K, y, stream);
-    if (M <= 32) return launch_gemm_cfg<32, true>(num_sms, xr, qw, sw, bias, M, N, K, y, stream);
-    if (M <= 64) return launch_gemm_cfg<64, true>(num_sms, xr, qw, sw, bias, M, N, K, y, stream);
-    return launch_gemm_cfg<128, false>(num_sms, xr, qw, sw, bias, M, N, K, y, stream);
+                           cudaStream_t stream, bool wrep = false) {
+    if (M <= 16) return launch_gemm_cfg<16, true>(num_sms, xr, qw, sw, bias, M, N, K, y, stream, wrep);
+    if (M <= 32) return launch_gemm_cfg<32, true>(num_sms, xr, qw, sw, bias, M, N, K, y, stream, wrep);
+    if (M <= 64) return launch_gemm_cfg<64, true>(num_sms, xr, qw, sw, bias, M, N, K, y, stream, wrep);
+    return launch_gemm_cfg<128, false>(num_sms, xr, qw, sw, bias, M, N, K, y, stream, wrep);
 }
 
 }  // namespace
@@ -748,10 +763,10 @@ size_t convrot_w4a16_workspace_size(int64_t M, int64_t K) {
     return round256(static_cast<size_t>(M) * static_cast<size_t>(K) * 2);
 }
 
-convrot_status convrot_w4a16_linear_prepared(const void *xr_bf16, const uint8_t *qw,
-                                             const float *sw, const void *bias_bf16, int64_t M,
-                                             int64_t N, int64_t K, void *y_bf16,
-                                             convrot_stream_t stream) {
+static convrot_status linear_prepared_impl(const void *xr_bf16, const uint8_t *qw,
+                                           const float *sw, const void *bias_bf16, int64_t M,
+                                           int64_t N, int64_t K, void *y_bf16,
+                                           cudaStream_t stream, bool wrep) {
     convrot_status st = check_gemm_shape(M, N, K);
     if (st != CONVROT_OK) return st;
     if (M == 0 || N == 0) return CONVROT_OK;
@@ -762,13 +777,14 @@ convrot_status convrot_w4a16_linear_prepared(const void *xr_bf16, const uint8_t 
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
     if ((st = check_device_ptrs(dev, {xr_bf16, qw, sw, bias_bf16, y_bf16})) != CONVROT_OK) return st;
-    return launch_gemm(g_dev[dev].num_sms, xr_bf16, qw, sw, bias_bf16, M, N, K, y_bf16, stream);
+    return launch_gemm(g_dev[dev].num_sms, xr_bf16, qw, sw, bias_bf16, M, N, K, y_bf16, stream,
+                       wrep);
 }
 
-convrot_status convrot_w4a16_linear(const void *x_bf16, const uint8_t *qw, const float *sw,
-                                    const void *bias_bf16, int64_t M, int64_t N, int64_t K,
-                                    int group, void *workspace, size_t ws_bytes, void *y_bf16,
-                                    convrot_stream_t stream) {
+static convrot_status linear_impl(const void *x_bf16, const uint8_t *qw, const float *sw,
+                                  const void *bias_bf16, int64_t M, int64_t N, int64_t K,
+                                  int group, void *workspace, size_t ws_bytes, void *y_bf16,
+                                  cudaStream_t stream, bool wrep) {
     convrot_status st = check_shape(M, K, group);
     if (st != CONVROT_OK) return st;
     if ((st = check_gemm_shape(M, N, K)) != CONVROT_OK) return st;
@@ -787,7 +803,39 @@ convrot_status convrot_w4a16_linear(const void *x_bf16, const uint8_t *qw, const
     if ((st = launch_rotate(g_dev[dev].num_sms, x_bf16, M, K, group, workspace, stream)) !=
         CONVROT_OK)
         return st;
-    return launch_gemm(g_dev[dev].num_sms, workspace, qw, sw, bias_bf16, M, N, K, y_bf16, stream);
+    return launch_gemm(g_dev[dev].num_sms, workspace, qw, sw, bias_bf16, M, N, K, y_bf16, stream,
+                       wrep);
+}
+
+convrot_status convrot_w4a16_linear_prepared(const void *xr_bf16, const uint8_t *qw,
+                                             const float *sw, const void *bias_bf16, int64_t M,
+                                             int64_t N, int64_t K, void *y_bf16,
+                                             convrot_stream_t stream) {
+    return linear_prepared_impl(xr_bf16, qw, sw, bias_bf16, M, N, K, y_bf16, stream, false);
+}
+
+convrot_status convrot_w4a16_linear_prepared_repacked(const void *xr_bf16, const uint8_t *qw_rep,
+                                                      const float *sw, const void *bias_bf16,
+                                                      int64_t M, int64_t N, int64_t K,
+                                                      void *y_bf16, convrot_stream_t stream) {
+    return linear_prepared_impl(xr_bf16, qw_rep, sw, bias_bf16, M, N, K, y_bf16, stream, true);
+}
+
+convrot_status convrot_w4a16_linear(const void *x_bf16, const uint8_t *qw, const float *sw,
+                                    const void *bias_bf16, int64_t M, int64_t N, int64_t K,
+                                    int group, void *workspace, size_t ws_bytes, void *y_bf16,
+                                    convrot_stream_t stream) {
+    return linear_impl(x_bf16, qw, sw, bias_bf16, M, N, K, group, workspace, ws_bytes, y_bf16,
+                       stream, false);
+}
+
+convrot_status convrot_w4a16_linear_repacked(const void *x_bf16, const uint8_t *qw_rep,
+                                             const float *sw, const void *bias_bf16, int64_t M,
+                                             int64_t N, int64_t K, int group, void *workspace,
+                                             size_t ws_bytes, void *y_bf16,
+                                             convrot_stream_t stream) {
+    return linear_impl(x_bf16, qw_rep, sw, bias_bf16, M, N, K, group, workspace, ws_bytes, y_bf16,
+                       stream, true);
 }
 
 convrot_status convrot_w4a16_check_device_error(convrot_stream_t stream) {

@@ -144,7 +144,8 @@ def test_w4a16_header_declares_the_boundary():
     assert _declared_w4a16() == sorted([
         "convrot_w4a16_prepare_act", "convrot_w4a16_workspace_size",
         "convrot_w4a16_linear_prepared", "convrot_w4a16_linear",
-        "convrot_w4a16_check_device_error"])
+        "convrot_w4a16_check_device_error", "convrot_w4a16_linear_repacked",
+        "convrot_w4a16_linear_prepared_repacked"])
 
 
 def test_w4a16_library_exports_every_declared_symbol(L16):
@@ -198,3 +199,24 @@ def test_missing_library_raises_instead_of_falling_back(monkeypatch, tmp_path, a
     monkeypatch.setattr(cr, "_lib" if loader == "lib" else "_lib_w4a16", None)
     with pytest.raises(RuntimeError, match="no fallback"):
         getattr(cr, loader)()
+
+
+def test_status_strings_cover_every_code(L):
+    for code in range(12):
+        assert L.convrot_status_string(code).decode().startswith("CONVROT_")
+    assert L.convrot_status_string(11).decode().startswith("CONVROT_ERR_OVERLAP")
+
+
+def test_repacked_size_and_host_checks(L):
+    assert cr.convrot_repacked_weight_size(3, 512) == 3 * 2 * 128
+    assert cr.convrot_repacked_weight_size(5, 320) == 5 * 2 * 128     # short last block padded
+    assert cr.convrot_repacked_weight_size(0, 512) == 0
+    f = L.convrot_repack_weight
+    assert f(A, 4, 100, B, None) == 3          # K not a multiple of 64
+    assert f(A, -1, 512, B, None) == 3
+    assert f(None, 4, 512, B, None) == 1
+    assert f(A, 4, 512, U, None) == 4          # misaligned output
+    assert f(A, 4, 512, A, None) == 11         # the same buffer
+    assert f(A, 4, 512, ctypes.c_void_p(0x10000 + 512), None) == 11   # overlapping tails
+    assert L.convrot_unpack_weight(A, 4, 512, A, None) == 11
+    assert f(A, 0, 512, B, None) == 0          # nothing to do
