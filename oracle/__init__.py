@@ -63,6 +63,15 @@ def lib():
             "oracle_w4a16_epilogue": [P, P, P, I64, I64, P, P],
             "oracle_w4a16_linear": [P, P, P, P, I64, I64, I64, I, P],
             "oracle_repack_weight": [P, I64, I64, P],
+            "oracle_e2m1_round": [P, I64, P],
+            "oracle_e4m3_round": [P, I64, P],
+            "oracle_e2m1_value": [P, I64, P],
+            "oracle_e4m3_value": [P, I64, P],
+            "oracle_nvfp4_quantize_rows": [P, I64, I64, P, P, P],
+            "oracle_nvfp4_pack": [P, I64, I64, P],
+            "oracle_nvfp4_sf_layout": [P, I64, I64, P],
+            "oracle_nvfp4_gemm": [P, P, P, P, I64, I64, I64, P, P, P],
+            "oracle_nvfp4_epilogue": [P, P, P, P, I64, I64, P, P],
             "oracle_unpack_weight": [P, I64, I64, P],
             "oracle_num_threads": [],
         }
@@ -327,3 +336,104 @@ def bf16_tie_band(y: np.ndarray, band: float = 1e-5) -> np.ndarray:
     mid = (np.floor(a / sp) + 0.5) * sp
     amax = a.max(axis=-1, keepdims=True) if a.ndim > 1 else a.max()
     return np.abs(a - mid) <= band * amax
+
+
+# --------------------------------------------------------------------------
+# The NVFP4 variant
+# --------------------------------------------------------------------------
+
+def e2m1_round(v: np.ndarray) -> np.ndarray:
+    """E2M1 codes (sign bit 3) of fp32 values: nearest, ties to even, saturating."""
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, dtype=np.uint8)
+    _check(lib().oracle_e2m1_round(_ptr(v), v.size, _ptr(out)), "e2m1_round")
+    return out
+
+
+def e4m3_round(v: np.ndarray) -> np.ndarray:
+    """Unsigned E4M3 codes of non-negative fp32 values (nearest, ties to even, saturating)."""
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, dtype=np.uint8)
+    _check(lib().oracle_e4m3_round(_ptr(v), v.size, _ptr(out)), "e4m3_round")
+    return out
+
+
+def e2m1_value(c: np.ndarray) -> np.ndarray:
+    c = np.ascontiguousarray(c, dtype=np.uint8)
+    out = np.empty(c.shape, dtype=np.float64)
+    _check(lib().oracle_e2m1_value(_ptr(c), c.size, _ptr(out)), "e2m1_value")
+    return out
+
+
+def e4m3_value(c: np.ndarray) -> np.ndarray:
+    c = np.ascontiguousarray(c, dtype=np.uint8)
+    out = np.empty(c.shape, dtype=np.float64)
+    _check(lib().oracle_e4m3_value(_ptr(c), c.size, _ptr(out)), "e4m3_value")
+    return out
+
+
+def nvfp4_quantize_rows(y: np.ndarray):
+    """(codes uint8 [rows][K] one per byte, block scales uint8 [rows][K/16],
+    row scales fp32 [rows]) of fp64 rotated rows."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    rows, K = y.shape
+    codes = np.empty((rows, K), dtype=np.uint8)
+    sf = np.empty((rows, K // 16), dtype=np.uint8)
+    sc = np.empty((rows,), dtype=np.float32)
+    _check(lib().oracle_nvfp4_quantize_rows(_ptr(y), rows, K, _ptr(codes), _ptr(sf), _ptr(sc)),
+           "nvfp4_quantize_rows")
+    return codes, sf, sc
+
+
+def nvfp4_pack(codes: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    rows, K = codes.shape
+    p = np.empty((rows, K // 2), dtype=np.uint8)
+    _check(lib().oracle_nvfp4_pack(_ptr(codes), rows, K, _ptr(p)), "nvfp4_pack")
+    return p
+
+
+def nvfp4_prepare_rows(x_bf16: np.ndarray, group: int):
+    """Rotate, quantise to NVFP4 and pack: (packed codes [rows][K/2], block
+    scales row-major [rows][K/16], row scales fp32 [rows])."""
+    codes, sf, sc = nvfp4_quantize_rows(rotate(x_bf16, group))
+    return nvfp4_pack(codes), sf, sc
+
+
+def nvfp4_sf_layout(sf: np.ndarray, K: int) -> np.ndarray:
+    """Row-major block scales [rows][K/16] -> the boundary's atom layout
+    (flat, rows padded to a multiple of 128)."""
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    rows = sf.shape[0]
+    out = np.empty(((rows + 127) // 128) * 128 * (K // 16), dtype=np.uint8)
+    _check(lib().oracle_nvfp4_sf_layout(_ptr(sf), rows, K, _ptr(out)), "nvfp4_sf_layout")
+    return out
+
+
+def nvfp4_gemm(qx, sfx, qw, sfw, K: int):
+    """(acc, l1, p64) fp64 [M][N] from packed codes and row-major block scales."""
+    qx = np.ascontiguousarray(qx, dtype=np.uint8)
+    qw = np.ascontiguousarray(qw, dtype=np.uint8)
+    sfx = np.ascontiguousarray(sfx, dtype=np.uint8)
+    sfw = np.ascontiguousarray(sfw, dtype=np.uint8)
+    M, N = qx.shape[0], qw.shape[0]
+    acc = np.empty((M, N), dtype=np.float64)
+    l1 = np.empty((M, N), dtype=np.float64)
+    p64 = np.empty((M, N), dtype=np.float64)
+    _check(lib().oracle_nvfp4_gemm(_ptr(qx), _ptr(sfx), _ptr(qw), _ptr(sfw), M, N, K, _ptr(acc),
+                                   _ptr(l1), _ptr(p64)), "nvfp4_gemm")
+    return acc, l1, p64
+
+
+def nvfp4_epilogue(acc, sx, sw, bias_bf16):
+    """(t fp64, y bf16 bits): t = acc sx sw + b exactly, y = bf16_rne(t)."""
+    acc = np.ascontiguousarray(acc, dtype=np.float64)
+    sx = np.ascontiguousarray(sx, dtype=np.float32)
+    sw = np.ascontiguousarray(sw, dtype=np.float32)
+    b = None if bias_bf16 is None else np.ascontiguousarray(bias_bf16, dtype=np.uint16)
+    M, N = acc.shape
+    t = np.empty((M, N), dtype=np.float64)
+    y = np.empty((M, N), dtype=np.uint16)
+    _check(lib().oracle_nvfp4_epilogue(_ptr(acc), _ptr(sx), _ptr(sw), _ptr(b), M, N, _ptr(t),
+                                       _ptr(y)), "nvfp4_epilogue")
+    return t, y

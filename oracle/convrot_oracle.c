@@ -57,6 +57,11 @@
  *    "Install and test" (repack_nk_weight_for_mpp): the packed bytes in
  *    128-byte column blocks, block-major, and back.
  *
+ *  - The NVFP4 variant (oracle_nvfp4_*).  "convrot-mlx" README, "Why this
+ *    repository exists" (the official ConvRot targets NVFP4 on Blackwell);
+ *    the format itself is not on the pages: E2M1 codes with one E4M3 scale
+ *    per 16 values and one fp32 scale per row (reading in the function).
+ *
  * Every function returns 0 on success or a negative number for bad
  * arguments.  Buffers are caller-owned, row-major and contiguous.
  * bf16 values travel as their raw 16-bit patterns (uint16_t).
@@ -518,6 +523,201 @@ int oracle_unpack_weight(const uint8_t *rep, int64_t N, int64_t K, uint8_t *qw) 
     for (int64_t n = 0; n < N; ++n)
         for (int64_t c = 0; c < row; ++c)
             qw[n * row + c] = rep[((c / 128) * N + n) * 128 + c % 128];
+    return 0;
+}
+
+/* ----------------------------------------------------------------------- */
+/* The NVFP4 variant.                                                       */
+/* ----------------------------------------------------------------------- */
+
+/* E2M1 (4-bit float): bit 3 sign, bits 2..1 exponent (bias 1), bit 0
+ * mantissa; codes 0..7 are the magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
+static double e2m1_value(unsigned code) {
+    static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    double v = mag[code & 7u];
+    return (code & 8u) ? -v : v;
+}
+
+/* Nearest E2M1 value by search over the eight magnitudes, ties to the even
+ * code (mantissa bit 0), magnitudes past 6 to 6 (saturation); the sign bit
+ * of v is kept, so a negative value that rounds to zero gives code 8. */
+static unsigned e2m1_round(float v) {
+    double a = fabs((double)v), bd = INFINITY;
+    unsigned best = 0;
+    for (unsigned c = 0; c < 8; ++c) {
+        double d = fabs(a - e2m1_value(c));
+        if (d < bd || (d == bd && (c & 1u) == 0)) {
+            best = c;
+            bd = d;
+        }
+    }
+    return (signbit(v) ? 8u : 0u) | best;
+}
+
+/* Unsigned E4M3 scale: bits 6..3 exponent (bias 7), bits 2..0 mantissa;
+ * exponent 0 is subnormal (m 2^-9); code 127 is not a number (not used).
+ * The largest value, code 126, is 448. */
+static double e4m3_value(unsigned code) {
+    unsigned e = (code >> 3) & 15u, m = code & 7u;
+    if (e == 0) return ldexp((double)m, -9);
+    return ldexp((double)(8u + m), (int)e - 10);
+}
+
+/* Nearest E4M3 value of a non-negative v by search over codes 0..126, ties
+ * to the even code, values past 448 to 448 (saturation). */
+static unsigned e4m3_round(float v) {
+    double a = (double)v, bd = INFINITY;
+    unsigned best = 0;
+    for (unsigned c = 0; c < 127; ++c) {
+        double d = fabs(a - e4m3_value(c));
+        if (d < bd || (d == bd && (c & 1u) == 0)) {
+            best = c;
+            bd = d;
+        }
+    }
+    return best;
+}
+
+int oracle_e2m1_round(const float *v, int64_t count, uint8_t *codes) {
+    if (!v || !codes || count < 0) return -1;
+    for (int64_t i = 0; i < count; ++i) codes[i] = (uint8_t)e2m1_round(v[i]);
+    return 0;
+}
+
+int oracle_e4m3_round(const float *v, int64_t count, uint8_t *codes) {
+    if (!v || !codes || count < 0) return -1;
+    for (int64_t i = 0; i < count; ++i) {
+        if (!(v[i] >= 0.0f)) return -1;
+        codes[i] = (uint8_t)e4m3_round(v[i]);
+    }
+    return 0;
+}
+
+int oracle_e2m1_value(const uint8_t *codes, int64_t count, double *v) {
+    if (!v || !codes || count < 0) return -1;
+    for (int64_t i = 0; i < count; ++i) v[i] = e2m1_value(codes[i]);
+    return 0;
+}
+
+int oracle_e4m3_value(const uint8_t *codes, int64_t count, double *v) {
+    if (!v || !codes || count < 0) return -1;
+    for (int64_t i = 0; i < count; ++i) {
+        if (codes[i] > 126) return -1;
+        v[i] = e4m3_value(codes[i]);
+    }
+    return 0;
+}
+
+/* NVFP4 quantisation of rotated rows.  The NVFP4 format (E2M1 elements, one
+ * E4M3 scale per 16 elements, one fp32 scale above it) is named by the pages
+ * ("convrot-mlx" README, "Why this repository exists": the official
+ * implementation targets NVFP4 on Blackwell) but not spelled out; the
+ * plainest reading, with the row as the unit of the fp32 scale as in the
+ * W4A4 quantiser, decided in fp32:
+ *   a    = fp32(max_k |y_k|),  s = a / 2688 (6 x 448, so the block scales
+ *          span E4M3 up to 448), r = 448 / a;  a == 0 gives s = r = 0;
+ *   per block b of 16: a_b = fp32(max |y_k|), sf_b = e4m3(a_b * r),
+ *   d_b  = fp32(value(sf_b) * s), inv_b = 1 / d_b (0 when d_b == 0),
+ *   q_k  = e2m1(fp32(y_k) * inv_b).
+ * Outputs: codes, one per byte [rows][K]; sf [rows][K/16] (E4M3 codes);
+ * s [rows]. */
+int oracle_nvfp4_quantize_rows(const double *y, int64_t rows, int64_t K, uint8_t *codes,
+                               uint8_t *sf, float *s) {
+    if (!y || !codes || !sf || !s || rows < 0 || K <= 0 || K % 16) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const double *yr = y + r * K;
+        double amax = 0.0;
+        for (int64_t k = 0; k < K; ++k)
+            if (fabs(yr[k]) > amax) amax = fabs(yr[k]);
+        const float a = (float)amax;
+        const float sr = a > 0.0f ? a / 2688.0f : 0.0f;
+        const float rr = a > 0.0f ? 448.0f / a : 0.0f;
+        s[r] = sr;
+        for (int64_t b = 0; b < K / 16; ++b) {
+            double bmax = 0.0;
+            for (int64_t k = 16 * b; k < 16 * b + 16; ++k)
+                if (fabs(yr[k]) > bmax) bmax = fabs(yr[k]);
+            const float t = (float)bmax * rr;
+            const unsigned c = e4m3_round(t);
+            sf[r * (K / 16) + b] = (uint8_t)c;
+            const float d = (float)e4m3_value(c) * sr;
+            const float inv = d > 0.0f ? 1.0f / d : 0.0f;
+            for (int64_t k = 16 * b; k < 16 * b + 16; ++k)
+                codes[r * K + k] = (uint8_t)e2m1_round((float)yr[k] * inv);
+        }
+    }
+    return 0;
+}
+
+/* Two E2M1 codes per byte, low nibble = even k (as the INT4 packing). */
+int oracle_nvfp4_pack(const uint8_t *codes, int64_t rows, int64_t K, uint8_t *p) {
+    if (!codes || !p || rows < 0 || K <= 0 || K % 2) return -1;
+    for (int64_t i = 0; i < rows * (K / 2); ++i)
+        p[i] = (uint8_t)((codes[2 * i] & 0xFu) | ((codes[2 * i + 1] & 0xFu) << 4));
+    return 0;
+}
+
+/* The block-scale storage layout of the GPU boundary (include/convrot_nvfp4.h):
+ * 512-byte atoms of 128 rows x 4 blocks, atom (row / 128, block / 4) at
+ * ((row / 128) * (K / 64) + block / 4) * 512, and inside an atom row r,
+ * block j at 16 (r mod 32) + 4 (r / 32 mod 4) + j.  rows are padded to a
+ * multiple of 128 (padding bytes 0).  sf: [rows][K/16] row-major. */
+int oracle_nvfp4_sf_layout(const uint8_t *sf, int64_t rows, int64_t K, uint8_t *out) {
+    if (!sf || !out || rows < 0 || K <= 0 || K % 64) return -1;
+    const int64_t tiles = (rows + 127) / 128, ka = K / 64;
+    memset(out, 0, (size_t)(tiles * 128 * (K / 16)));
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < K / 16; ++b) {
+            const int64_t atom = (r / 128) * ka + b / 4;
+            const int64_t rr = r % 128;
+            out[atom * 512 + 16 * (rr % 32) + 4 * (rr / 32) + b % 4] = sf[r * (K / 16) + b];
+        }
+    return 0;
+}
+
+/* acc[m][n] = sum over blocks b of value(sfx[m][b]) value(sfw[n][b])
+ *             sum_{k in b} e2m1(qx[m][k]) e2m1(qw[n][k])    (fp64, exact:
+ * every product has at most 12 significant bits and the sums stay far below
+ * 2^53 of its spacing), plus l1 = the sum of the |terms| and p64 = the sum
+ * of |running sums| at every 64th k, for the accumulation bound.  Packed
+ * codes [rows][K/2], block scales row-major [rows][K/16]. */
+int oracle_nvfp4_gemm(const uint8_t *qx, const uint8_t *sfx, const uint8_t *qw,
+                      const uint8_t *sfw, int64_t M, int64_t N, int64_t K, double *acc,
+                      double *l1, double *p64) {
+    if (!qx || !sfx || !qw || !sfw || !acc || M < 0 || N < 0 || K <= 0 || K % 64) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double sum = 0.0, a1 = 0.0, pr = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                const unsigned cx = (qx[m * (K / 2) + k / 2] >> (4 * (k & 1))) & 0xFu;
+                const unsigned cw = (qw[n * (K / 2) + k / 2] >> (4 * (k & 1))) & 0xFu;
+                const double t = e2m1_value(cx) * e2m1_value(cw) *
+                                 e4m3_value(sfx[m * (K / 16) + k / 16]) *
+                                 e4m3_value(sfw[n * (K / 16) + k / 16]);
+                sum += t;
+                a1 += fabs(t);
+                if (k % 64 == 63) pr += fabs(sum);
+            }
+            acc[m * N + n] = sum;
+            if (l1) l1[m * N + n] = a1;
+            if (p64) p64[m * N + n] = pr;
+        }
+    return 0;
+}
+
+/* t = acc sx sw + b exactly (fp64) and y = bf16_rne(t). */
+int oracle_nvfp4_epilogue(const double *acc, const float *sx, const float *sw,
+                          const uint16_t *bias, int64_t M, int64_t N, double *t, uint16_t *y) {
+    if (!acc || !sx || !sw || !y || M < 0 || N < 0) return -1;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double v = acc[m * N + n] * (double)sx[m] * (double)sw[n];
+            v += bias ? bf16_bits_to_double(bias[n]) : 0.0;
+            if (t) t[m * N + n] = v;
+            y[m * N + n] = double_to_bf16_bits_rne(v);
+        }
     return 0;
 }
 
