@@ -11,7 +11,10 @@ Names follow the C ABI: ``convrot_quantize_weight``, ``convrot_prepare_act``,
 ``convrot_linear``, ``convrot_linear_prepared`` (plus the test hooks), and for
 the W4A16 variant (``include/convrot_w4a16.h``, library
 ``libconvrot_w4a16.so``) ``convrot_w4a16_prepare_act``,
-``convrot_w4a16_linear`` and ``convrot_w4a16_linear_prepared``.
+``convrot_w4a16_linear`` and ``convrot_w4a16_linear_prepared``, and for the
+NVFP4 variant (``include/convrot_nvfp4.h``, library ``libconvrot_nvfp4.so``)
+``convrot_nvfp4_quantize``, ``convrot_nvfp4_linear`` and
+``convrot_nvfp4_linear_prepared``.
 """
 from __future__ import annotations
 
@@ -23,6 +26,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libconvrot.so")
 LIB_W4A16_PATH = os.path.join(_HERE, "libconvrot_w4a16.so")
+LIB_NVFP4_PATH = os.path.join(_HERE, "libconvrot_nvfp4.so")
 
 STATUS = {
     0: "CONVROT_OK", 1: "CONVROT_ERR_NULL", 2: "CONVROT_ERR_GROUP", 3: "CONVROT_ERR_SHAPE",
@@ -502,6 +506,114 @@ def convrot_w4a16_check_device_error(stream=None) -> int:
     """Synchronise the stream; return (and clear) the W4A16 library's device
     error status."""
     return int(lib_w4a16().convrot_w4a16_check_device_error(_stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# the NVFP4 variant (include/convrot_nvfp4.h)
+# ---------------------------------------------------------------------------
+
+_lib_nvfp4 = None
+
+
+def lib_nvfp4() -> ctypes.CDLL:
+    """The loaded NVFP4 library; raises if it has not been built."""
+    global _lib_nvfp4
+    if _lib_nvfp4 is None:
+        if not os.path.exists(LIB_NVFP4_PATH):
+            raise RuntimeError(
+                f"{LIB_NVFP4_PATH} is missing: build it with "
+                "`python -m rotated_w4a4_quantized_b200.build` (there is no fallback path)")
+        L = ctypes.CDLL(LIB_NVFP4_PATH)
+        P, I64, I, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        sigs = {
+            "convrot_nvfp4_quantize": [P, I64, I64, I, P, P, P, P],
+            "convrot_nvfp4_linear_prepared": [P, P, P, P, P, P, P, I64, I64, I64, P, P],
+            "convrot_nvfp4_linear": [P, P, P, P, P, I64, I64, I64, I, P, SZ, P, P],
+            "convrot_nvfp4_check_device_error": [P],
+        }
+        for name, args in sigs.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ctypes.c_int
+        for name in ("convrot_nvfp4_scale_bytes", "convrot_nvfp4_workspace_size"):
+            getattr(L, name).argtypes = [I64, I64]
+            getattr(L, name).restype = SZ
+        _lib_nvfp4 = L
+    return _lib_nvfp4
+
+
+def convrot_nvfp4_scale_bytes(rows: int, K: int) -> int:
+    return int(lib_nvfp4().convrot_nvfp4_scale_bytes(rows, K))
+
+
+def convrot_nvfp4_workspace_size(M: int, K: int) -> int:
+    return int(lib_nvfp4().convrot_nvfp4_workspace_size(M, K))
+
+
+def convrot_nvfp4_quantize(x: torch.Tensor, group: int, q=None, sf=None, s=None, stream=None):
+    """bf16 [rows, K] -> (E2M1 codes uint8 [rows, K/2], E4M3 block scales
+    uint8 [scale_bytes] in the tensor cores' atom layout, fp32 row scales [rows])."""
+    rows, K = _rows(x, torch.bfloat16, "x")
+    with torch.cuda.device(x.device):
+        nsf = convrot_nvfp4_scale_bytes(rows, K)
+        q = torch.empty(rows, K // 2, dtype=torch.uint8, device=x.device) if q is None else q
+        sf = torch.empty(max(1, nsf), dtype=torch.uint8, device=x.device) if sf is None else sf
+        s = torch.empty(rows, dtype=torch.float32, device=x.device) if s is None else s
+        _need(q, torch.uint8, "q", (rows, K // 2), x)
+        _need(sf, torch.uint8, "sf", (max(1, nsf),), x)
+        _need(s, torch.float32, "s", (rows,), x)
+        _check(lib_nvfp4().convrot_nvfp4_quantize(_p(x), rows, K, group, _p(q), _p(sf), _p(s),
+                                                  _stream(stream)), "convrot_nvfp4_quantize")
+    return q, sf, s
+
+
+def _nvfp4_operand(q, sf, s, K: int, name: str, like=None):
+    _need(q, torch.uint8, name, (None, K // 2), like)
+    rows = q.shape[0]
+    _need(sf, torch.uint8, name + " scales", (convrot_nvfp4_scale_bytes(rows, K),), like)
+    _need(s, torch.float32, name + " row scales", (rows,), like)
+    return rows
+
+
+def convrot_nvfp4_linear_prepared(qx, sfx, sx, qw, sfw, sw, bias, K: int, out=None, stream=None):
+    """The block-scaled FP4 product on prepared operands -> bf16 y [M, N]."""
+    M = _nvfp4_operand(qx, sfx, sx, K, "qx")
+    N = _nvfp4_operand(qw, sfw, sw, K, "qw", qx)
+    _need_opt(bias, torch.bfloat16, "bias", (N,), qx)
+    with torch.cuda.device(qx.device):
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=qx.device) if out is None else out
+        _need(out, torch.bfloat16, "out", (M, N), qx)
+        _check(lib_nvfp4().convrot_nvfp4_linear_prepared(
+            _p(qx), _p(sfx), _p(sx), _p(qw), _p(sfw), _p(sw), _p(bias), M, N, K, _p(out),
+            _stream(stream)), "convrot_nvfp4_linear_prepared")
+    return out
+
+
+def convrot_nvfp4_linear(x, qw, sfw, sw, bias, group: int, workspace=None, out=None, stream=None):
+    """The whole NVFP4 layer: bf16 x [M, K] -> bf16 y [M, N] (rotation and
+    NVFP4 quantisation of x, then the block-scaled FP4 product)."""
+    M, K = _rows(x, torch.bfloat16, "x")
+    N = _nvfp4_operand(qw, sfw, sw, K, "qw", x)
+    _need_opt(bias, torch.bfloat16, "bias", (N,), x)
+    with torch.cuda.device(x.device):
+        need = convrot_nvfp4_workspace_size(M, K)
+        if workspace is None:
+            workspace = torch.empty(max(1, need), dtype=torch.uint8, device=x.device)
+        _need(workspace, torch.uint8, "workspace", None, x)
+        if workspace.numel() < need:
+            raise ValueError(f"workspace holds {workspace.numel()} bytes, {need} needed")
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
+        _need(out, torch.bfloat16, "out", (M, N), x)
+        _check(lib_nvfp4().convrot_nvfp4_linear(
+            _p(x), _p(qw), _p(sfw), _p(sw), _p(bias), M, N, K, group, _p(workspace),
+            workspace.numel(), _p(out), _stream(stream)), "convrot_nvfp4_linear")
+    return out
+
+
+def convrot_nvfp4_check_device_error(stream=None) -> int:
+    """Synchronise the stream; return (and clear) the NVFP4 library's device
+    error status."""
+    return int(lib_nvfp4().convrot_nvfp4_check_device_error(_stream(stream)))
 
 
 class HostPipeline:

@@ -1,10 +1,12 @@
 """Build the CUDA libraries in-tree: rotated_w4a4_quantized_b200/libconvrot.so
-(the W4A4 layer, include/convrot.h) and libconvrot_w4a16.so (the W4A16
-variant, include/convrot_w4a16.h).
+(the W4A4 layer, include/convrot.h), libconvrot_w4a16.so (the W4A16
+variant, include/convrot_w4a16.h) and libconvrot_nvfp4.so (the NVFP4
+variant, include/convrot_nvfp4.h).
 
     python -m rotated_w4a4_quantized_b200.build [--verbose]
 
-Each library is one translation unit (csrc/convrot.cu, csrc/w4a16.cu)
+Each library is one translation unit (csrc/convrot.cu, csrc/w4a16.cu,
+csrc/nvfp4.cu)
 compiled for sm_100a only, with IEEE
 fp32 semantics (no fast-math: the epilogue and the quantiser rely on
 correctly rounded multiply, add and divide).  The CUDA runtime is linked
@@ -29,6 +31,10 @@ SRC_W4A16 = os.path.join(HERE, "csrc", "w4a16.cu")
 DEPS_W4A16 = [os.path.join(HERE, "csrc", f) for f in ("w4a16.cu", "prep.cuh", "ptx.cuh")] + [
     HEADER, os.path.join(_INC, "convrot_w4a16.h")]
 LIB_W4A16 = os.path.join(HERE, "libconvrot_w4a16.so")
+SRC_NVFP4 = os.path.join(HERE, "csrc", "nvfp4.cu")
+DEPS_NVFP4 = [os.path.join(HERE, "csrc", f) for f in ("nvfp4.cu", "prep.cuh", "ptx.cuh")] + [
+    HEADER, os.path.join(_INC, "convrot_nvfp4.h")]
+LIB_NVFP4 = os.path.join(HERE, "libconvrot_nvfp4.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -53,7 +59,8 @@ def _stale(lib: str, deps) -> bool:
 
 
 def stale() -> bool:
-    return _stale(LIB, DEPS + [HEADER]) or _stale(LIB_W4A16, DEPS_W4A16)
+    return (_stale(LIB, DEPS + [HEADER]) or _stale(LIB_W4A16, DEPS_W4A16)
+            or _stale(LIB_NVFP4, DEPS_NVFP4))
 
 
 def _build_one(src: str, lib: str, verbose: bool) -> None:
@@ -72,6 +79,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
         _build_one(SRC, LIB, verbose)
     if force or _stale(LIB_W4A16, DEPS_W4A16):
         _build_one(SRC_W4A16, LIB_W4A16, verbose)
+    if force or _stale(LIB_NVFP4, DEPS_NVFP4):
+        _build_one(SRC_NVFP4, LIB_NVFP4, verbose)
     return LIB
 
 
@@ -79,3 +88,4 @@ if __name__ == "__main__":
     build(force=True, verbose="--verbose" in sys.argv)
     print(LIB)
     print(LIB_W4A16)
+    print(LIB_NVFP4)

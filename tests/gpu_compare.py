@@ -146,3 +146,44 @@ def w4a16_input_effect(y64_rot, xr_bits, qw_codes, tie_w, rot_band):
     qabs = np.abs(qw_codes.astype(np.float64)) + 1.0
     xabs = np.abs(bf16_f64(xr_bits)) + sp
     return (rot_band * sp) @ qabs.T + xabs @ tie_w.astype(np.float64).T
+
+
+def check_nvfp4_outputs(y_gpu_bits, t, acc, l1, p64, sx, sw):
+    """NVFP4 outputs against the exact t = acc sx sw + b (oracle, fp64):
+    |y - t| <= half the bf16 spacing at max(|t|, |y|) + E, with
+      E = |sx sw| 2^-20 (p64 + l1) + 2^-23 (|acc sx sw| + |t|).
+    Every product of two E2M1 codes and two E4M3 scales is exact in fp32;
+    2^-20 (p64 + l1) lets each 64-deep tensor-core step err by 8 fp32 ulps
+    of its |running sum| and of the |products| it adds; 2^-23 (...) covers the
+    three fp32 roundings of the epilogue ((acc sx) sw + b).  Returns the
+    share of outputs equal to bf16_rne(t)."""
+    y = bf16_f64(y_gpu_bits)
+    sxw = np.abs(np.asarray(sx, np.float64))[:, None] * np.abs(np.asarray(sw, np.float64))[None, :]
+    E = sxw * 2.0 ** -20 * (p64 + l1) + 2.0 ** -23 * (np.abs(acc) * sxw + np.abs(t)) * 1.5
+    tol = 0.5 * np.maximum(bf16_spacing(np.abs(t) + E), bf16_spacing(y)) + E
+    err = np.abs(y - t)
+    bad = err > tol
+    assert not bad.any(), (f"{bad.sum()} outputs outside tolerance, e.g. at {np.argwhere(bad)[:5]}: "
+                           f"gpu {y[bad][:5]} exact {t[bad][:5]} tol {tol[bad][:5]}")
+    return float(np.mean(np.abs(y - t) <= 0.5 * bf16_spacing(t)))
+
+
+def nvfp4_sf_rowmajor(sf_atoms: np.ndarray, rows: int, K: int) -> np.ndarray:
+    """The boundary's scale atoms -> row-major [rows][K/16] (the index map of
+    include/convrot_nvfp4.h, restated here)."""
+    r = np.arange(rows)[:, None]
+    j = np.arange(K // 16)[None, :]
+    off = ((r // 128) * (K // 64) + j // 4) * 512 + 16 * (r % 32) + 4 * ((r // 32) % 4) + j % 4
+    return sf_atoms[off]
+
+
+def nvfp4_codes_equal(a_packed: np.ndarray, b_packed: np.ndarray) -> np.ndarray:
+    """Per code (unpacked, [rows][K]): equal, counting the two encodings of
+    zero (0 and 8) as the same value."""
+    def unpack(p):
+        out = np.empty((p.shape[0], 2 * p.shape[1]), np.uint8)
+        out[:, 0::2] = p & 0xF
+        out[:, 1::2] = p >> 4
+        out[out == 8] = 0
+        return out
+    return unpack(a_packed) == unpack(b_packed)

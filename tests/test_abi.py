@@ -220,3 +220,29 @@ def test_repacked_size_and_host_checks(L):
     assert f(A, 4, 512, ctypes.c_void_p(0x10000 + 512), None) == 11   # overlapping tails
     assert L.convrot_unpack_weight(A, 4, 512, A, None) == 11
     assert f(A, 0, 512, B, None) == 0          # nothing to do
+
+
+HEADER_NVFP4 = os.path.join(ROOT, "include", "convrot_nvfp4.h")
+
+
+def test_nvfp4_library_exports_every_declared_symbol():
+    from rotated_w4a4_quantized_b200 import build
+    build.build()
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER_NVFP4).read(), flags=re.S)
+    names = sorted(set(re.findall(r"\b(convrot_nvfp4_[a-z0-9_]+)\s*\(", text)))
+    assert names == sorted(["convrot_nvfp4_scale_bytes", "convrot_nvfp4_quantize",
+                            "convrot_nvfp4_workspace_size", "convrot_nvfp4_linear_prepared",
+                            "convrot_nvfp4_linear", "convrot_nvfp4_check_device_error"])
+    L = cr.lib_nvfp4()
+    for name in names:
+        assert hasattr(L, name), name
+    assert cr.convrot_nvfp4_scale_bytes(200, 192) == 256 * 12
+    assert cr.convrot_nvfp4_scale_bytes(0, 192) == 0
+    assert cr.convrot_nvfp4_workspace_size(3, 1024) == 1536 + 128 * 64 + 256
+    # host-side validation before any device work
+    A, B = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x20000)
+    assert L.convrot_nvfp4_quantize(A, 4, 100, 64, B, B, B, None) == 3     # K % 64
+    assert L.convrot_nvfp4_quantize(A, 4, 1024, 32, B, B, B, None) == 2    # group
+    assert L.convrot_nvfp4_quantize(None, 4, 1024, 64, B, B, B, None) == 1
+    assert L.convrot_nvfp4_linear_prepared(A, A, A, A, A, A, None, 4, 4, 100, B, None) == 3
+    assert L.convrot_nvfp4_linear(A, A, A, A, None, 4, 4, 1024, 64, B, 16, B, None) == 5

@@ -226,3 +226,52 @@ def test_nvfp4_error_below_int4_rowwise_on_outlier_layer():
     y_int4 = f64(O.linear_prepared_w(xb, qw, sww, None, 64))
     e_int4 = np.linalg.norm(y_int4 - dense) / np.linalg.norm(dense)
     assert e_fp4 < e_int4
+
+
+def _emulate_nvfp4_kernel(px, sfx, sx, pw, sfw, sw, bias_bits, K, drop_block=None):
+    """The GPU product's arithmetic on the CPU: products of two E2M1 codes
+    and two E4M3 scales (exact in fp32), summed in fp32 sixteen at a time,
+    each 64-deep step added to an fp32 running sum; then the fp32 epilogue
+    ((acc sx) sw + b) and one rounding to bf16 (torch).  drop_block leaves
+    out the 16-value block starting at that k."""
+    cx = O.e2m1_value(np.stack([px & 0xF, px >> 4], -1).reshape(px.shape[0], -1))
+    cw = O.e2m1_value(np.stack([pw & 0xF, pw >> 4], -1).reshape(pw.shape[0], -1))
+    xs = (cx * O.e4m3_value(sfx).repeat(16, axis=1)).astype(np.float32)
+    ws = (cw * O.e4m3_value(sfw).repeat(16, axis=1)).astype(np.float32)
+    M, N = xs.shape[0], ws.shape[0]
+    run = np.zeros((M, N), np.float32)
+    for k0 in range(0, K, 64):
+        step = np.zeros((M, N), np.float32)
+        for k in range(k0, k0 + 64):
+            if drop_block is not None and drop_block <= k < drop_block + 16:
+                continue
+            step = step + np.outer(xs[:, k], ws[:, k]).astype(np.float32)
+        run = run + step
+    y = (run * sx[:, None]).astype(np.float32) * sw[None, :]
+    if bias_bits is not None:
+        y = y + ((bias_bits.astype(np.uint32) << 16).view(np.float32))[None, :]
+    return wl.bf16_bits(torch.from_numpy(y.astype(np.float32)).to(torch.bfloat16))
+
+
+def test_nvfp4_gate_accepts_the_kernel_arithmetic_and_rejects_a_dropped_block():
+    from tests import gpu_compare as gc
+    M, N, K = 12, 20, 1024
+    lt = wl.make_random_layer(M, K, N, 64, seed=21)
+    xb, wb, bb = wl.bf16_bits(lt.x), wl.bf16_bits(lt.w), wl.bf16_bits(lt.b)
+    px, sfx, sx = O.nvfp4_prepare_rows(xb, 64)
+    pw, sfw, sw = O.nvfp4_prepare_rows(wb, 64)
+    acc, l1, p64 = O.nvfp4_gemm(px, sfx, pw, sfw, K)
+    t, _ = O.nvfp4_epilogue(acc, sx, sw, bb)
+    gc.check_nvfp4_outputs(_emulate_nvfp4_kernel(px, sfx, sx, pw, sfw, sw, bb, K), t, acc, l1,
+                           p64, sx, sw)
+    for drop in (0, 512, K - 16):
+        with pytest.raises(AssertionError):
+            gc.check_nvfp4_outputs(_emulate_nvfp4_kernel(px, sfx, sx, pw, sfw, sw, bb, K, drop),
+                                   t, acc, l1, p64, sx, sw)
+
+
+def test_scale_atom_index_maps_agree():
+    from tests import gpu_compare as gc
+    rows, K = 300, 320
+    sf = np.random.default_rng(9).integers(0, 127, (rows, K // 16)).astype(np.uint8)
+    assert np.array_equal(gc.nvfp4_sf_rowmajor(O.nvfp4_sf_layout(sf, K), rows, K), sf)
