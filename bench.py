@@ -61,6 +61,14 @@ METRIC_W4A16 = "W4A16 linear end-to-end TFLOP/s (bf16 x INT4 tensor ops); rotati
 # the GEMM reads xr, the packed weights, scales and bias and writes y
 ROT16_BYTES = lambda M, K: 4 * M * K  # noqa: E731
 GEMM16_BYTES = lambda M, N, K: 2 * M * K + N * K // 2 + 4 * N + 2 * N + 2 * M * N  # noqa: E731
+METRIC_NVFP4 = ("NVFP4 linear end-to-end TFLOP/s (E2M1 x E2M1 block-scaled tensor ops); "
+                "quantisation kernel HBM GB/s")
+FP4_PER_BF16 = 4.0    # nominal dense ratio (9 / 2.25 PFLOP/s)
+# NVFP4 algorithmic bytes: the quantisation reads x (bf16) and writes codes,
+# block scales and row scales; the GEMM reads both operands' codes and
+# scales, the bias, and writes y
+FP4_QUANT_BYTES = lambda M, K: 2 * M * K + M * K // 2 + M * K // 16 + 4 * M  # noqa: E731
+FP4_GEMM_BYTES = lambda M, N, K: (M + N) * (K // 2 + K // 16 + 4) + 2 * N + 2 * M * N  # noqa: E731
 
 
 MIN_KERNEL_MS = 50.0          # device time of each per-kernel timing pass, at least
@@ -465,7 +473,8 @@ def run_gpu(args):
         "e2e": {"value": round(ops_e2e / (t_e2e * 1e-3) / 1e12, 3), "unit": "TOPS",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                 "call": f"HostPipeline: pinned host buffers, {e2e['chunks']} row chunks, "
-                        "copies overlapped with convrot_linear on three streams"},
+                        "copies overlapped with convrot_linear on three streams",
+                "link": e2e["link"]},
         "gpu_launches": launches,
         "kernel_passes": {"prep_launches": [n for _, n in prep_pass],
                           "gemm_launches": [n for _, n in gemm_pass],
@@ -481,10 +490,93 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
-def run_gpu_w4a16(args):
-    """The W4A16 variant: the same timing scheme as run_gpu (cold L2 through
-    rotating copies, CUDA graphs, K back-to-back steps between two events,
-    max over ranks), through convrot_w4a16_linear."""
+class W4A16Variant:
+    """bf16 activations x the W4A4 packed weights (include/convrot_w4a16.h)."""
+    name, metric, dtype = "w4a16", METRIC_W4A16, "bf16"
+    peak_ratio, peak_note = 1.0, "measured bf16 burst"
+    prep_kernel, gemm_kernel = "rotate_bf16_kernel", "w4a16_gemm_kernel"
+    prep_bytes = staticmethod(ROT16_BYTES)
+    gemm_bytes = staticmethod(GEMM16_BYTES)
+    prep_desc = "algorithmic bytes 4MK"
+    gemm_desc = "2MK (xr) + NK/2 + 4N + 2N + 2MN"
+
+    @staticmethod
+    def weights(cr, w, group):
+        return cr.convrot_quantize_weight(w, group)
+
+    @staticmethod
+    def buffers(cr, sp, dev):
+        ws = torch.empty(cr.convrot_w4a16_workspace_size(sp.M, sp.K), dtype=torch.uint8, device=dev)
+        return {"ws": ws, "xr": ws[:sp.M * sp.K * 2].view(torch.bfloat16).view(sp.M, sp.K)}
+
+    @staticmethod
+    def step(cr, x, wt, b, sp, bufs, out):
+        cr.convrot_w4a16_linear(x, *wt, b, sp.group, bufs["ws"], out)
+
+    @staticmethod
+    def prep(cr, x, sp, bufs):
+        cr.convrot_w4a16_prepare_act(x, sp.group, out=bufs["xr"])
+
+    @staticmethod
+    def gemm(cr, wt, b, sp, bufs, out):
+        cr.convrot_w4a16_linear_prepared(bufs["xr"], *wt, b, out=out)
+
+    @staticmethod
+    def check(cr):
+        return cr.convrot_w4a16_check_device_error()
+
+
+class NVFP4Variant:
+    """E2M1 activations and weights with E4M3 block scales (include/convrot_nvfp4.h)."""
+    name, metric, dtype = "nvfp4", METRIC_NVFP4, "e2m1"
+    peak_ratio = FP4_PER_BF16
+    peak_note = f"measured bf16 burst x {FP4_PER_BF16} nominal fp4/bf16 ratio"
+    prep_kernel, gemm_kernel = "quant_kernel", "nvfp4_gemm_kernel"
+    prep_bytes = staticmethod(FP4_QUANT_BYTES)
+    gemm_bytes = staticmethod(FP4_GEMM_BYTES)
+    prep_desc = "algorithmic bytes 2MK + MK/2 + MK/16 + 4M"
+    gemm_desc = "(M+N)(K/2 + K/16 + 4) + 2N + 2MN"
+
+    @staticmethod
+    def weights(cr, w, group):
+        return cr.convrot_nvfp4_quantize(w, group)
+
+    @staticmethod
+    def buffers(cr, sp, dev):
+        M, K = sp.M, sp.K
+        ws = torch.empty(cr.convrot_nvfp4_workspace_size(M, K), dtype=torch.uint8, device=dev)
+        r256 = lambda v: (v + 255) // 256 * 256  # noqa: E731
+        nsf = cr.convrot_nvfp4_scale_bytes(M, K)
+        o1 = r256(M * K // 2)
+        o2 = o1 + r256(nsf)
+        return {"ws": ws, "q": ws[:M * K // 2].view(M, K // 2), "sf": ws[o1:o1 + nsf],
+                "s": ws[o2:o2 + 4 * M].view(torch.float32)}
+
+    @staticmethod
+    def step(cr, x, wt, b, sp, bufs, out):
+        cr.convrot_nvfp4_linear(x, *wt, b, sp.group, bufs["ws"], out)
+
+    @staticmethod
+    def prep(cr, x, sp, bufs):
+        cr.convrot_nvfp4_quantize(x, sp.group, bufs["q"], bufs["sf"], bufs["s"])
+
+    @staticmethod
+    def gemm(cr, wt, b, sp, bufs, out):
+        cr.convrot_nvfp4_linear_prepared(bufs["q"], bufs["sf"], bufs["s"], *wt, b, sp.K, out=out)
+
+    @staticmethod
+    def check(cr):
+        return cr.convrot_nvfp4_check_device_error()
+
+
+VARIANTS = {"w4a16": W4A16Variant, "nvfp4": NVFP4Variant}
+
+
+def run_gpu_variant(args, V):
+    """A variant on the bf16 tensor path (W4A16, NVFP4): the same timing
+    scheme as run_gpu (cold L2 through rotating copies, CUDA graphs, K
+    back-to-back steps between two events, max over ranks), through the
+    variant's public whole-layer call."""
     import torch.distributed as dist
 
     import rotated_w4a4_quantized_b200 as cr
@@ -505,14 +597,13 @@ def run_gpu_w4a16(args):
     prepared = []
     for lt in layers:
         w = lt.w.to(dev)
-        qw, sw = cr.convrot_quantize_weight(w, lt.spec.group)     # offline step
+        wt = V.weights(cr, w, lt.spec.group)             # offline step
         b = None if lt.b is None else lt.b.to(dev)
         del w
-        prepared.append((lt.spec, qw, sw, b))
+        prepared.append((lt.spec, wt, b))
     x0 = layers[0].x.to(dev)
 
-    step_bytes = sum(4 * sp.M * sp.K + sp.N * (sp.K // 2 + 6) + 2 * sp.M * sp.N
-                     for sp, *_ in prepared)
+    step_bytes = sum(V.prep_bytes(sp.M, sp.K) + V.gemm_bytes(sp.M, sp.N, sp.K) for sp, *_ in prepared)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     R = 1 if step_bytes >= 2 * l2 else min(64, -(-2 * l2 // step_bytes))
 
@@ -522,36 +613,34 @@ def run_gpu_w4a16(args):
     copies = []
     for r in range(R):
         c = Copy()
-        c.w = [(sp, qw.clone(), sw.clone(), None if b is None else b.clone())
-               for sp, qw, sw, b in prepared]
-        c.acts, c.ws, c.xr, c.outs = [x0.clone()], [], [], []
+        c.w = [(sp, tuple(t.clone() for t in wt), None if b is None else b.clone())
+               for sp, wt, b in prepared]
+        c.acts, c.bufs, c.outs = [x0.clone()], [], []
         for i, (sp, *_) in enumerate(prepared):
-            ws = torch.empty(cr.convrot_w4a16_workspace_size(sp.M, sp.K), dtype=torch.uint8, device=dev)
-            c.ws.append(ws)
-            c.xr.append(ws[:sp.M * sp.K * 2].view(torch.bfloat16).view(sp.M, sp.K))
+            c.bufs.append(V.buffers(cr, sp, dev))
             c.outs.append(torch.empty(sp.M, sp.N, dtype=torch.bfloat16, device=dev))
             if i + 1 < nl:
                 c.acts.append(c.outs[i])
         copies.append(c)
 
     def step(c):
-        for i, (sp, qw, sw, b) in enumerate(c.w):
-            cr.convrot_w4a16_linear(c.acts[i], qw, sw, b, sp.group, c.ws[i], c.outs[i])
+        for i, (sp, wt, b) in enumerate(c.w):
+            V.step(cr, c.acts[i], wt, b, sp, c.bufs[i], c.outs[i])
 
-    def rot_only(c, i):
-        cr.convrot_w4a16_prepare_act(c.acts[i], c.w[i][0].group, out=c.xr[i])
+    def prep_only(c, i):
+        V.prep(cr, c.acts[i], c.w[i][0], c.bufs[i])
 
     def gemm_only(c, i):
-        sp, qw, sw, b = c.w[i]
-        cr.convrot_w4a16_linear_prepared(c.xr[i], qw, sw, b, out=c.outs[i])
+        sp, wt, b = c.w[i]
+        V.gemm(cr, wt, b, sp, c.bufs[i], c.outs[i])
 
     for k in range(max(args.warmup, R)):
         step(copies[k % R])
         for i in range(nl):
-            rot_only(copies[k % R], i)
+            prep_only(copies[k % R], i)
             gemm_only(copies[k % R], i)
     torch.cuda.synchronize()
-    if cr.convrot_w4a16_check_device_error() != 0:
+    if V.check(cr) != 0:
         raise RuntimeError("device error during warm-up")
 
     def capture(fn, *a):
@@ -569,7 +658,7 @@ def run_gpu_w4a16(args):
 
     progs = {"step": (step, ())}
     for i in range(nl):
-        progs[("rot", i)] = (rot_only, (i,))
+        progs[("prep", i)] = (prep_only, (i,))
         progs[("gemm", i)] = (gemm_only, (i,))
     graphs = {key: ([capture(fn, c, *a) for c in copies], capture_all(fn, *a))
               for key, (fn, a) in progs.items()}
@@ -590,6 +679,14 @@ def run_gpu_w4a16(args):
         b.synchronize()
         return a.elapsed_time(b)
 
+    def timed_kernel(key):
+        n = args.steps
+        t = timed(key, n)
+        if t < MIN_KERNEL_MS:
+            n = int(math.ceil(n * MIN_KERNEL_MS * 1.05 / max(t, 1e-3)))
+            t = timed(key, n)
+        return t / n
+
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -604,44 +701,44 @@ def run_gpu_w4a16(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    status = cr.convrot_w4a16_check_device_error()
+    status = V.check(cr)
     if status != 0:
         raise RuntimeError(f"device error status {status} in the timed region")
 
-    rot_avg = [timed(("rot", i), args.steps) / args.steps for i in range(nl)]
-    gemm_avg = [timed(("gemm", i), args.steps) / args.steps for i in range(nl)]
+    prep_avg = [timed_kernel(("prep", i)) for i in range(nl)]
+    gemm_avg = [timed_kernel(("gemm", i)) for i in range(nl)]
     flops_step = spec.ops                       # 2 M N K per layer
     t_max, flops_total = aggregate(local_ms, flops_step * args.steps, dev)
     value = flops_total / (t_max * 1e-3) / 1e12
     tokens_s = spec.tokens * world * args.steps / (t_max * 1e-3)
 
     peaks = _peaks()
+    tensor_peak = peaks["bf16"] * V.peak_ratio
     gemm_tf = [2 * sp.M * sp.N * sp.K / (g * 1e-3) / 1e12 for (sp, *_), g in zip(prepared, gemm_avg)]
-    gemm_gbs = [GEMM16_BYTES(sp.M, sp.N, sp.K) / (g * 1e-3) / 1e9 for (sp, *_), g in zip(prepared, gemm_avg)]
-    rot_gbs = [ROT16_BYTES(sp.M, sp.K) / (r * 1e-3) / 1e9 for (sp, *_), r in zip(prepared, rot_avg)]
-    if sum(gemm_avg) >= sum(rot_avg):
+    gemm_gbs = [V.gemm_bytes(sp.M, sp.N, sp.K) / (g * 1e-3) / 1e9
+                for (sp, *_), g in zip(prepared, gemm_avg)]
+    prep_gbs = [V.prep_bytes(sp.M, sp.K) / (r * 1e-3) / 1e9 for (sp, *_), r in zip(prepared, prep_avg)]
+    if sum(gemm_avg) >= sum(prep_avg):
         i = max(range(nl), key=lambda j: gemm_avg[j])
         sp = prepared[i][0]
         # the bound of this shape: the larger of its tensor time and its byte time
-        t_tensor = 2 * sp.M * sp.N * sp.K / (peaks["bf16"] * 1e12)
-        t_bytes = GEMM16_BYTES(sp.M, sp.N, sp.K) / (peaks["hbm"] * 1e9)
+        t_tensor = 2 * sp.M * sp.N * sp.K / (tensor_peak * 1e12)
+        t_bytes = V.gemm_bytes(sp.M, sp.N, sp.K) / (peaks["hbm"] * 1e9)
         if t_tensor >= t_bytes:
-            roof = {"kernel": "w4a16_gemm_kernel", "bound": "tensor", "achieved": round(gemm_tf[i], 2),
-                    "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": round(gemm_tf[i] / peaks["bf16"], 4),
-                    "traffic": None,
-                    "note": "bf16 tensor ops (2 per multiply-add) of the bf16 x INT4 GEMM; peak = "
-                            f"measured bf16 burst ({peaks['src']})"}
+            roof = {"kernel": V.gemm_kernel, "bound": "tensor", "achieved": round(gemm_tf[i], 2),
+                    "peak": round(tensor_peak, 1), "unit": "TFLOP/s",
+                    "frac": round(gemm_tf[i] / tensor_peak, 4), "traffic": None,
+                    "note": f"tensor ops (2 per multiply-add); peak = {V.peak_note} ({peaks['src']})"}
         else:
-            roof = {"kernel": "w4a16_gemm_kernel", "bound": "hbm", "achieved": round(gemm_gbs[i], 1),
+            roof = {"kernel": V.gemm_kernel, "bound": "hbm", "achieved": round(gemm_gbs[i], 1),
                     "peak": peaks["hbm"], "unit": "GB/s", "frac": round(gemm_gbs[i] / peaks["hbm"], 4),
                     "traffic": None,
-                    "note": "algorithmic bytes 2MK (xr) + NK/2 + 4N + 2N + 2MN; HBM peak "
-                            f"{peaks['src']}"}
+                    "note": f"algorithmic bytes {V.gemm_desc}; HBM peak {peaks['src']}"}
     else:
-        i = max(range(nl), key=lambda j: rot_avg[j])
-        roof = {"kernel": "rotate_bf16_kernel", "bound": "hbm", "achieved": round(rot_gbs[i], 1),
-                "peak": peaks["hbm"], "unit": "GB/s", "frac": round(rot_gbs[i] / peaks["hbm"], 4),
-                "traffic": None, "note": f"algorithmic bytes 4MK; HBM peak {peaks['src']}"}
+        i = max(range(nl), key=lambda j: prep_avg[j])
+        roof = {"kernel": V.prep_kernel, "bound": "hbm", "achieved": round(prep_gbs[i], 1),
+                "peak": peaks["hbm"], "unit": "GB/s", "frac": round(prep_gbs[i] / peaks["hbm"], 4),
+                "traffic": None, "note": f"{V.prep_desc}; HBM peak {peaks['src']}"}
 
     # end to end: pinned host x in, pinned host y out, copies inside the interval
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -671,11 +768,11 @@ def run_gpu_w4a16(args):
     t_e2e, fl_e2e = aggregate(e2e_ms, flops_step * e2e_steps, dev)
 
     line = {
-        "metric": METRIC_W4A16, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "metric": V.metric, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": V.dtype,
         "data": "synthetic (seeded bf16, shapes and distributions of the workload; no weights)",
-        "config": {"workload": name, "variant": "w4a16",
+        "config": {"workload": name, "variant": V.name,
                    "layers": [f"{l.M}x{l.K}->{l.N} g{l.group}" for l in spec.layers],
                    "tokens_per_rank": spec.tokens,
                    "l2": f"cold: steps cycle through {R} copies of all step data "
@@ -683,27 +780,69 @@ def run_gpu_w4a16(args):
                    "launch": f"CUDA graphs of {R} steps (each copy once), replayed back to back",
                    "parallelism": f"dp{world}"},
         "tokens_per_s": round(tokens_s, 1),
-        "bf16_peak_frac_path": round(value / world / peaks["bf16"], 4),
+        "tensor_peak_frac_path": round(value / world / tensor_peak, 4),
         "gemm_tflops": [round(v, 2) for v in gemm_tf],
         "gemm_gbs": [round(v, 1) for v in gemm_gbs],
-        "rotate_gbs": [round(v, 1) for v in rot_gbs],
-        "rotate_hbm_frac": [round(v / peaks["hbm"], 4) for v in rot_gbs],
+        "prep_gbs": [round(v, 1) for v in prep_gbs],
+        "prep_hbm_frac": [round(v / peaks["hbm"], 4) for v in prep_gbs],
         "roofline": roof,
         "e2e": {"value": round(fl_e2e / (t_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": prepared[0][0].M * prepared[0][0].K * 2,
                 "d2h_bytes_per_step": prepared[-1][0].M * prepared[-1][0].N * 2,
-                "call": "pinned host x -> device, convrot_w4a16_linear per layer, y -> pinned "
-                        "host, one stream, L2 flushed before each step"},
+                "call": f"pinned host x -> device, the {V.name} whole-layer call per layer, y -> "
+                        "pinned host, one stream, L2 flushed before each step"},
         "gpu_launches": 2 * nl * args.steps,
         "clocks": clocks.summary(),
     }
     if rank == 0:
-        line["cpu_baseline"] = (cpu_baseline(name, args.cpu_seconds, "w4a16")
+        line["cpu_baseline"] = (cpu_baseline(name, args.cpu_seconds, V.name)
                                 if world == 1 and not args.no_cpu else None)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def link_bandwidth(x_host, y_host, dev, reps=5):
+    """Pinned host <-> device copy bandwidth of this step's byte counts: H2D
+    alone, D2H alone, and both at once on two streams (GB/s, best of
+    `reps`, CUDA events): the bound the end-to-end figure is judged against."""
+    xd = torch.empty_like(x_host, device=dev)
+    yd = torch.empty_like(y_host, device=dev)
+    s1, s2 = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+
+    def best(fn):
+        t = float("inf")
+        for _ in range(reps):
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            t = min(t, a.elapsed_time(b))
+        return t
+
+    def both():
+        cur = torch.cuda.current_stream()
+        e = torch.cuda.Event()
+        e.record(cur)
+        s1.wait_event(e)
+        s2.wait_event(e)
+        with torch.cuda.stream(s1):
+            xd.copy_(x_host, non_blocking=True)
+        with torch.cuda.stream(s2):
+            y_host.copy_(yd, non_blocking=True)
+        cur.wait_stream(s1)
+        cur.wait_stream(s2)
+
+    t_in = best(lambda: xd.copy_(x_host, non_blocking=True))
+    t_out = best(lambda: y_host.copy_(yd, non_blocking=True))
+    t_both = best(both)
+    bi, bo = x_host.numel() * x_host.element_size(), y_host.numel() * y_host.element_size()
+    return {"h2d_gbs": round(bi / (t_in * 1e-3) / 1e9, 1), "d2h_gbs": round(bo / (t_out * 1e-3) / 1e9, 1),
+            "both_gbs": round((bi + bo) / (t_both * 1e-3) / 1e9, 1),
+            "bound_ms": round(max(t_in, t_out, t_both), 4)}
 
 
 def run_e2e(cr, prepared, spec, dev, stream, flush, args):
@@ -713,8 +852,12 @@ def run_e2e(cr, prepared, spec, dev, stream, flush, args):
     sp0 = prepared[0][0]
     x_host = wl.make_workload(args.workload)[0].x.pin_memory()
     y_host = torch.empty(prepared[-1][0].M, prepared[-1][0].N, dtype=torch.bfloat16).pin_memory()
+    # chunks of at least 1024 rows, up to 8: on the 8192-token layer 8 chunks
+    # measured 3.37 ms per step against 3.49 (4), 3.51 (16) and 3.92 (32):
+    # pipeline fill and drain are one chunk's copy each, and every chunk adds
+    # its own copy and launch overheads
     pipe = cr.HostPipeline(sp0.M, sp0.K, [(qw, sw, b, sp.group) for sp, qw, sw, b in prepared],
-                           chunks=max(1, min(8, sp0.M // 256)), device=dev)
+                           chunks=max(1, min(8, sp0.M // 1024)), device=dev)
     steps = max(3, min(args.steps, 200))
     for _ in range(3):
         pipe(x_host, y_host, stream)
@@ -730,19 +873,19 @@ def run_e2e(cr, prepared, spec, dev, stream, flush, args):
         b.record(stream)
     torch.cuda.synchronize()
     total = sum(a.elapsed_time(b) for a, b in ev)
+    link = link_bandwidth(x_host, y_host, dev)
+    link["e2e_over_bound"] = round(total / steps / link["bound_ms"], 3)
     return {"ms": total, "steps": steps, "h2d": sp0.M * sp0.K * 2,
-            "d2h": prepared[-1][0].M * prepared[-1][0].N * 2, "chunks": len(pipe.ranges)}
+            "d2h": prepared[-1][0].M * prepared[-1][0].N * 2, "chunks": len(pipe.ranges),
+            "link": link}
 
-
-# ---------------------------------------------------------------------------
-# the CPU oracle as a timed baseline
-# ---------------------------------------------------------------------------
 
 class OracleSampler:
     """The oracle's per-call work on a sample of token rows: prepare those
     activation rows, integer GEMM against the prepared weights, epilogue
-    (W4A16: rotate and round those rows, fp64 GEMM, epilogue).  Weight
-    preparation is offline (done once here, untimed), as on the GPU."""
+    (W4A16: rotate and round those rows, fp64 GEMM, epilogue; NVFP4: rotate
+    and quantise those rows to NVFP4, fp64 block-scaled GEMM, epilogue).
+    Weight preparation is offline (done once here, untimed), as on the GPU."""
 
     def __init__(self, name, variant="w4a4"):
         self.variant = variant
@@ -752,7 +895,10 @@ class OracleSampler:
         self.spec = wl.WORKLOADS[name]
         l0 = wl.make_workload(name)[0]
         self.sp = l0.spec
-        self.pw, self.sw = O.prepare_rows(wl.bf16_bits(l0.w), self.sp.group)
+        if variant == "nvfp4":
+            self.pw, self.sfw, self.sw = O.nvfp4_prepare_rows(wl.bf16_bits(l0.w), self.sp.group)
+        else:
+            self.pw, self.sw = O.prepare_rows(wl.bf16_bits(l0.w), self.sp.group)
         self.bb = None if l0.b is None else wl.bf16_bits(l0.b)
         self.xb = wl.bf16_bits(l0.x)
         self.cores = O.num_threads()
@@ -763,6 +909,10 @@ class OracleSampler:
         t0 = time.perf_counter()
         if self.variant == "w4a16":
             O.w4a16_linear(self.xb[:rows], self.pw, self.sw, self.bb, sp.group)
+        elif self.variant == "nvfp4":
+            px, sfx, sx = O.nvfp4_prepare_rows(self.xb[:rows], sp.group)
+            acc, _, _ = O.nvfp4_gemm(px, sfx, self.pw, self.sfw, sp.K)
+            O.nvfp4_epilogue(acc, sx, self.sw, self.bb)
         else:
             px, sx = O.prepare_rows(self.xb[:rows], sp.group)
             O.epilogue(O.gemm(px, self.pw, sp.K), sx, self.sw, self.bb)
@@ -782,6 +932,10 @@ class OracleSampler:
         return 2 * rows * self.sp.N * self.sp.K
 
 
+# what the oracle computes per sampled row, by variant
+VARIANT_WORK = {"w4a16": "rotation + bf16 rounding + fp64 GEMM + epilogue",
+                "nvfp4": "rotation + NVFP4 quantisation + fp64 block-scaled GEMM + epilogue"}
+
 # workloads whose baseline also gets a one-thread figure
 ONE_THREAD_BASELINE = ("small_g256", "outlier_g64")
 
@@ -790,10 +944,9 @@ def cpu_baseline(name, seconds, variant="w4a4"):
     s = OracleSampler(name, variant)
     rows = s.calibrate(seconds)
     t = s.run(rows)
-    what = ("rotation + bf16 rounding + fp64 GEMM + epilogue" if variant == "w4a16"
-            else "prep + int64 GEMM + epilogue")
+    what = VARIANT_WORK.get(variant, "prep + int64 GEMM + epilogue")
     out = {"value": round(s.ops(rows) / t / 1e12, 9),
-           "unit": "TFLOP/s" if variant == "w4a16" else "TOPS", "cores": s.cores,
+           "unit": "TOPS" if variant == "w4a4" else "TFLOP/s", "cores": s.cores,
            "kind": "oracle",
            "sample": f"{rows} of {s.sp.M} token rows of layer {s.layer} ({what}, weights "
                      f"prepared offline), {t:.1f} s"}
@@ -814,7 +967,7 @@ def run_reference(args):
     if rank != 0:
         return
     name = args.workload
-    w16 = args.variant == "w4a16"
+    V = VARIANTS.get(args.variant)
     s = OracleSampler(name, args.variant)
     # the whole run (warm-up + steps) stays within about --cpu-seconds x 8
     per_step = args.cpu_seconds * 8 / (args.steps + args.warmup)
@@ -826,14 +979,13 @@ def run_reference(args):
             total += t
     value = s.ops(rows) * args.steps / total / 1e12
     spec = wl.WORKLOADS[name]
-    unit = "TFLOP/s" if w16 else "TOPS"
-    what = ("rotation + bf16 rounding + fp64 GEMM + epilogue" if w16
-            else "prep + int64 GEMM + epilogue")
+    unit = "TOPS" if V is None else "TFLOP/s"
+    what = VARIANT_WORK.get(args.variant, "prep + int64 GEMM + epilogue")
     line = {
-        "impl": "reference", "metric": METRIC_W4A16 if w16 else METRIC, "value": round(value, 9),
+        "impl": "reference", "metric": METRIC if V is None else V.metric, "value": round(value, 9),
         "unit": unit, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w16 else "s8",
+        "scaling": "weak", "vs_baseline": None, "dtype": "s8" if V is None else V.dtype,
         "data": "synthetic (seeded bf16, same workload)",
         "config": {"workload": name, "layers": [f"{l.M}x{l.K}->{l.N} g{l.group}" for l in spec.layers],
                    "tokens_per_rank": spec.tokens, "parallelism": "cpu"},
@@ -887,8 +1039,9 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time budget of the oracle baseline")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline")
-    ap.add_argument("--variant", default="w4a4", choices=["w4a4", "w4a16"],
-                    help="w4a16: the bf16-activation variant (include/convrot_w4a16.h)")
+    ap.add_argument("--variant", default="w4a4", choices=["w4a4", "w4a16", "nvfp4"],
+                    help="w4a16: the bf16-activation variant (include/convrot_w4a16.h); "
+                         "nvfp4: the NVFP4 variant (include/convrot_nvfp4.h)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -897,8 +1050,8 @@ def main(argv=None):
         sys.exit(spawn_ranks(args.gpus, sys.argv[1:] if argv is None else list(argv)))
     if args.impl == "reference":
         run_reference(args)
-    elif args.variant == "w4a16":
-        run_gpu_w4a16(args)
+    elif args.variant in VARIANTS:
+        run_gpu_variant(args, VARIANTS[args.variant])
     else:
         run_gpu(args)
 
