@@ -270,7 +270,9 @@ def run_gpu(args):
     # of everything a step touches (activations, workspace, weights, outputs),
     # with R copies together at least twice the L2 size, so no step finds its
     # data in L2 from an earlier one.
-    step_bytes = sum(sp.M * sp.K * 2 + cr.convrot_linear_workspace_size(sp.M, sp.K)
+    # (the workspace's codes and scales; its split area is touched only by
+    # the partial sums of one wave, a small share of a step)
+    step_bytes = sum(sp.M * sp.K * 2 + sp.M * (sp.K // 2 + 4)
                      + sp.N * (sp.K // 2 + 6) + sp.M * sp.N * 2 for sp, *_ in prepared)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     R = 1 if step_bytes >= 2 * l2 else min(64, -(-2 * l2 // step_bytes))
@@ -304,9 +306,14 @@ def run_gpu(args):
         sp, qw, sw, b = c.w[i]
         cr.convrot_prepare_act(c.acts[i], sp.group, c.ws[i][0], c.ws[i][1])
 
+    # the GEMM alone with a split area, so it runs the split-K plan of the
+    # whole-layer call (steps on one stream may share one area)
+    areas = [cr.new_split_area(dev) for _ in prepared]
+
     def gemm_only(c, i):
         sp, qw, sw, b = c.w[i]
-        cr.convrot_linear_prepared(c.ws[i][0], c.ws[i][1], qw, sw, b, sp.K, out=c.outs[i])
+        cr.convrot_linear_prepared_split(c.ws[i][0], c.ws[i][1], qw, sw, b, sp.K, areas[i],
+                                         out=c.outs[i])
 
     for k in range(max(args.warmup, R)):
         step(copies[k % R])

@@ -89,11 +89,27 @@ convrot_status convrot_quantize_weight(const void *w_bf16, int64_t N, int64_t K,
 convrot_status convrot_prepare_act(const void *x_bf16, int64_t M, int64_t K, int group,
                                    uint8_t *qx, float *sx, convrot_stream_t stream);
 
+/*
+ * Split K (the pages have no counterpart: it is how the integer product is
+ * scheduled on 148 SMs, not what it computes).  Where the output tiles leave
+ * the last wave of the persistent GEMM part-filled, the tiles of that wave
+ * are split into 2-4 ranges of K; each part writes its int32 partial sums to
+ * a split area, and the part that finishes last adds them and runs the
+ * epilogue.  Integer addition is exact, so the result is bit-identical to
+ * the unsplit product.  A split area is CONVROT_SPLIT_AREA_BYTES bytes,
+ * 256-byte aligned: CONVROT_SPLIT_COUNTER_BYTES of counters that must be
+ * zero before a launch (each launch that completes leaves them zero), then
+ * the partial slots (one wave of 256 x 256 int32 tiles).
+ */
+#define CONVROT_SPLIT_COUNTER_BYTES ((size_t)8192)
+#define CONVROT_SPLIT_AREA_BYTES (CONVROT_SPLIT_COUNTER_BYTES + (size_t)160 * 128 * 256 * 4)
+
 /* Bytes of workspace convrot_linear needs: the packed codes [M][K/2] and the
  * fp32 scales [M] of the prepared activations, each region rounded up to 256
- * bytes.  Host-only; 0 for M <= 0 or K <= 0.  Source: "convrot-mlx" README,
- * "What is included" (fused activation preparation into the N x packed-K
- * layout and one absmax scale per row). */
+ * bytes, then (M > 128, where the token-major GEMM runs) a split area of
+ * CONVROT_SPLIT_AREA_BYTES.  Host-only; 0 for M <= 0 or K <= 0.  Source:
+ * "convrot-mlx" README, "What is included" (fused activation preparation
+ * into the N x packed-K layout and one absmax scale per row). */
 size_t convrot_linear_workspace_size(int64_t M, int64_t K);
 
 /*
@@ -102,9 +118,12 @@ size_t convrot_linear_workspace_size(int64_t M, int64_t K);
  * x_bf16 [M][K] bf16; qw [N][K/2] and sw [N] from convrot_quantize_weight
  * with the same group; bias_bf16 [N] bf16 or NULL (zeros); y_bf16 [M][N].
  * workspace: ws_bytes >= convrot_linear_workspace_size(M, K), 256-byte
- * aligned.  Source: "convrot-mlx" README, "Install and test" (the complete
- * path is rotation, activation quantisation, the integer product, scaling
- * and bias).
+ * aligned.  A workspace that holds the codes and scales but not the split
+ * area (ws_bytes >= the size less CONVROT_SPLIT_AREA_BYTES) is accepted and
+ * runs without split K, with the same results.  The prep kernel zeroes the
+ * split counters, so the workspace needs no initialisation.  Source:
+ * "convrot-mlx" README, "Install and test" (the complete path is rotation,
+ * activation quantisation, the integer product, scaling and bias).
  */
 convrot_status convrot_linear(const void *x_bf16, const uint8_t *qw, const float *sw,
                               const void *bias_bf16, int64_t M, int64_t N, int64_t K, int group,
@@ -122,6 +141,21 @@ convrot_status convrot_linear_prepared(const uint8_t *qx, const float *sx, const
                                        const float *sw, const void *bias_bf16, int64_t M,
                                        int64_t N, int64_t K, void *y_bf16,
                                        convrot_stream_t stream);
+
+/*
+ * convrot_linear_prepared with a split area (split_ws, split_bytes >=
+ * CONVROT_SPLIT_AREA_BYTES, 256-byte aligned, else CONVROT_ERR_WORKSPACE),
+ * so that the GEMM may split K as convrot_linear does.  Its counters must be
+ * zero before the first call (e.g. one memset when the area is allocated);
+ * every call that completes leaves them zero, so later calls need nothing.
+ * After CONVROT_ERR_DEVICE_TIMEOUT zero them again.  Calls that use one area
+ * must be ordered on the GPU.  split_ws = NULL runs without split K.
+ */
+convrot_status convrot_linear_prepared_split(const uint8_t *qx, const float *sx,
+                                             const uint8_t *qw, const float *sw,
+                                             const void *bias_bf16, int64_t M, int64_t N,
+                                             int64_t K, void *split_ws, size_t split_bytes,
+                                             void *y_bf16, convrot_stream_t stream);
 
 /*
  * The reversible weight repack.  "convrot-mlx" README, "What is included"
@@ -222,6 +256,26 @@ convrot_status convrot_debug_gemm_tiles(const uint8_t *qx, const float *sx, cons
                                         convrot_stream_t stream);
 
 /*
+ * Test hook: convrot_debug_gemm_tiles for a token-major form (tiles 0-3 or
+ * 6, optionally | CONVROT_TILES_REPACKED) with a given split-K plan: the
+ * first split_tiles output tiles (tile t covers rows (t mod TA) x TM and
+ * columns (t / TA) x BN, TA = ceil(M / TM)) are each cut into `splits`
+ * contiguous ranges of K-stages; split_tiles = 0 runs every tile whole,
+ * split_tiles = -1 takes the planner's choice for this area.  The split area
+ * is that of convrot_linear_prepared_split (counters zero on entry, zero
+ * again when the call completes).  CONVROT_ERR_SHAPE when the plan does not
+ * fit: split_tiles above the tile count, splits outside 2 .. the K-stages of
+ * a tile, or slots or counters beyond the area.  Exposes the scheduling of
+ * step 3 ("convrot-mlx" README, "Install and test": the integer product) and
+ * shows it does not change a bit of the result.
+ */
+convrot_status convrot_debug_gemm_split(const uint8_t *qx, const float *sx, const uint8_t *qw,
+                                        const float *sw, const void *bias_bf16, int64_t M,
+                                        int64_t N, int64_t K, int tiles, int split_tiles,
+                                        int splits, void *split_ws, size_t split_bytes,
+                                        int out_s32, void *out, convrot_stream_t stream);
+
+/*
  * The whole layer, like convrot_linear, for callers that cannot give the
  * library any device memory of their own: a plugin called by a host runtime
  * that owns every allocation and passes no workspace, or a caller on a
@@ -232,8 +286,9 @@ convrot_status convrot_debug_gemm_tiles(const uint8_t *qx, const float *sx, cons
  * Instead of a caller-provided workspace it uses one fixed array of
  * CONVROT_NOALLOC_SCRATCH_BYTES in the library's own device memory.  Every
  * GPU that loads the library holds that array until the process exits.
- * Requests needing more (round256(M*K/2) + round256(4*M) bytes, the same
- * layout as convrot_linear_workspace_size) fail with
+ * Requests needing more (round256(M*K/2) + round256(4*M) bytes, the codes
+ * and scales of convrot_linear_workspace_size without its split area; this
+ * entry point does not split K) fail with
  * CONVROT_ERR_SCRATCH_LIMIT before anything is launched; e.g. M = 4096 with
  * K = 4096 fits (8 MiB), M = 8192 with K = 4096 (16 MiB + 32 KiB) does not.
  *

@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
             "convrot_unpack_weight": [P, I64, I64, P, P],
             "convrot_linear_repacked": [P, P, P, P, I64, I64, I64, I, P, SZ, P, P],
             "convrot_linear_prepared_repacked": [P, P, P, P, P, I64, I64, I64, P, P],
+            "convrot_linear_prepared_split": [P, P, P, P, P, I64, I64, I64, P, SZ, P, P],
+            "convrot_debug_gemm_split": [P, P, P, P, P, I64, I64, I64, I, I, I, P, SZ, I, P, P],
         }
         for name, args in sigs.items():
             f = getattr(L, name)
@@ -180,6 +182,12 @@ def convrot_linear_workspace_size(M: int, K: int) -> int:
     return int(lib().convrot_linear_workspace_size(M, K))
 
 
+def _base_workspace(M: int, need: int) -> int:
+    # the codes and scales alone: a workspace without the split area runs
+    # the layer unsplit, with the same results
+    return need - SPLIT_AREA_BYTES if M > 128 and need else need
+
+
 def convrot_linear(x, qw, sw, bias, group: int, workspace=None, out=None, stream=None):
     """The whole layer: bf16 x [M, K] -> bf16 y [M, N]."""
     M, K = _rows(x, torch.bfloat16, "x")
@@ -189,8 +197,9 @@ def convrot_linear(x, qw, sw, bias, group: int, workspace=None, out=None, stream
         if workspace is None:
             workspace = torch.empty(max(1, need), dtype=torch.uint8, device=x.device)
         _need(workspace, torch.uint8, "workspace", None, x)
-        if workspace.numel() < need:
-            raise ValueError(f"workspace holds {workspace.numel()} bytes, {need} needed")
+        if workspace.numel() < _base_workspace(M, need):
+            raise ValueError(f"workspace holds {workspace.numel()} bytes, {need} needed "
+                             f"({_base_workspace(M, need)} without split K)")
         out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
         _need(out, torch.bfloat16, "out", (M, N), x)
         _check(lib().convrot_linear(_p(x), _p(qw), _p(sw), _p(bias), M, N, K, group,
@@ -251,8 +260,9 @@ def convrot_linear_repacked(x, qw_rep, sw, bias, group: int, workspace=None, out
         if workspace is None:
             workspace = torch.empty(max(1, need), dtype=torch.uint8, device=x.device)
         _need(workspace, torch.uint8, "workspace", None, x)
-        if workspace.numel() < need:
-            raise ValueError(f"workspace holds {workspace.numel()} bytes, {need} needed")
+        if workspace.numel() < _base_workspace(M, need):
+            raise ValueError(f"workspace holds {workspace.numel()} bytes, {need} needed "
+                             f"({_base_workspace(M, need)} without split K)")
         out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
         _need(out, torch.bfloat16, "out", (M, N), x)
         _check(lib().convrot_linear_repacked(_p(x), _p(qw_rep), _p(sw), _p(bias), M, N, K, group,
@@ -308,6 +318,45 @@ def convrot_linear_prepared(qx, sx, qw, sw, bias, K: int, out=None, stream=None)
         _need(out, torch.bfloat16, "out", (M, N), qx)
         _check(lib().convrot_linear_prepared(_p(qx), _p(sx), _p(qw), _p(sw), _p(bias), M, N, K,
                                              _p(out), _stream(stream)), "convrot_linear_prepared")
+    return out
+
+
+# Split-K area (include/convrot.h): counters, then one wave of partial slots.
+SPLIT_COUNTER_BYTES = 8192
+SPLIT_AREA_BYTES = SPLIT_COUNTER_BYTES + 160 * 128 * 256 * 4
+
+
+def new_split_area(device) -> torch.Tensor:
+    """A split area for convrot_linear_prepared_split: its counters start at
+    zero (every call that completes leaves them zero)."""
+    a = torch.empty(SPLIT_AREA_BYTES, dtype=torch.uint8, device=device)
+    a[:SPLIT_COUNTER_BYTES].zero_()
+    return a
+
+
+def _split_area(area, like):
+    if area is None:
+        return None, 0
+    _need(area, torch.uint8, "split area", None, like)
+    if area.numel() < SPLIT_AREA_BYTES or area.data_ptr() % 256:
+        raise ValueError("the split area needs SPLIT_AREA_BYTES bytes, 256-byte aligned")
+    return _p(area), area.numel()
+
+
+def convrot_linear_prepared_split(qx, sx, qw, sw, bias, K: int, split_area, out=None,
+                                  stream=None):
+    """convrot_linear_prepared with a split area (new_split_area), so that
+    the GEMM may split K where its last wave is part-filled."""
+    M = _prepared(qx, sx, K)
+    _need(sx, torch.float32, "sx", (M,), qx)
+    N = _weights(qw, sw, bias, K, qx)
+    with torch.cuda.device(qx.device):
+        pa, na = _split_area(split_area, qx)
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=qx.device) if out is None else out
+        _need(out, torch.bfloat16, "out", (M, N), qx)
+        _check(lib().convrot_linear_prepared_split(_p(qx), _p(sx), _p(qw), _p(sw), _p(bias), M, N,
+                                                   K, pa, na, _p(out), _stream(stream)),
+               "convrot_linear_prepared_split")
     return out
 
 
@@ -721,3 +770,30 @@ class ConvRotLinear:
             self._ws = torch.empty(max(1, need), dtype=torch.uint8, device=x2.device)
         y = convrot_linear(x2, self.qweight, self.scales, self.bias, self.group, self._ws)
         return y.reshape(*lead, self.out_features)
+
+
+def convrot_debug_gemm_split(qx, sx, qw, sw, bias, K: int, tiles: int, split_tiles: int,
+                             splits: int, split_area, out_s32: bool = False, out=None,
+                             stream=None):
+    """convrot_debug_gemm_tiles for a token-major form with a given split-K
+    plan: the first split_tiles output tiles cut into `splits` ranges of K
+    (split_tiles = 0: none; -1: the planner's choice).  split_area as for
+    convrot_linear_prepared_split."""
+    M = _prepared(qx, sx, K)
+    if out_s32:
+        _need(qw, torch.uint8, "qw", (None, K // 2), qx)
+        N = qw.shape[0]
+    else:
+        _need(sx, torch.float32, "sx", (M,), qx)
+        N = _weights(qw, sw, bias, K, qx)
+    dt = torch.int32 if out_s32 else torch.bfloat16
+    with torch.cuda.device(qx.device):
+        _need(split_area, torch.uint8, "split area", None, qx)
+        out = torch.empty(M, N, dtype=dt, device=qx.device) if out is None else out
+        _need(out, dt, "out", (M, N), qx)
+        _check(lib().convrot_debug_gemm_split(_p(qx), _p(sx), _p(qw), _p(sw), _p(bias), M, N, K,
+                                              int(tiles), int(split_tiles), int(splits),
+                                              _p(split_area), split_area.numel(),
+                                              int(bool(out_s32)), _p(out), _stream(stream)),
+               "convrot_debug_gemm_split")
+    return out

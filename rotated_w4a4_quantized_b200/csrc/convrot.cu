@@ -7,6 +7,7 @@
 #include <stdint.h>
 #include <stdio.h>
 
+#include <algorithm>
 #include <atomic>
 #include <initializer_list>
 #include <mutex>
@@ -231,8 +232,11 @@ int prep16_ctas_per_sm(int group, int mode, int64_t K) {
     return slot;
 }
 
+// zero / nzero: words the kernel sets to 0 on the way (the split counters
+// of the GEMM that follows), or nullptr / 0.
 convrot_status launch_prep(int num_sms, const void *x, int64_t rows, int64_t K, int group,
-                           uint8_t *q, float *s, float *yrot, cudaStream_t stream) {
+                           uint8_t *q, float *s, float *yrot, cudaStream_t stream,
+                           uint32_t *zero = nullptr, int nzero = 0) {
     if (rows == 0) return CONVROT_OK;
     const int mode = yrot ? 1 : 0;
     // Up to 1024 rows the launch is latency-bound (a row or two per CTA):
@@ -246,11 +250,11 @@ convrot_status launch_prep(int num_sms, const void *x, int64_t rows, int64_t K, 
         const uint16_t *xx = static_cast<const uint16_t *>(x);
         const int m = static_cast<int>(rows), k = static_cast<int>(K);
         if (yrot) {
-            if (group == 64) prep::prep16_kernel<64, 1><<<grid16, block16, 0, stream>>>(xx, m, k, q, s, yrot);
-            else prep::prep16_kernel<256, 1><<<grid16, block16, 0, stream>>>(xx, m, k, q, s, yrot);
+            if (group == 64) prep::prep16_kernel<64, 1><<<grid16, block16, 0, stream>>>(xx, m, k, q, s, yrot, zero, nzero);
+            else prep::prep16_kernel<256, 1><<<grid16, block16, 0, stream>>>(xx, m, k, q, s, yrot, zero, nzero);
         } else {
-            if (group == 64) prep::prep16_kernel<64, 0><<<grid16, block16, 0, stream>>>(xx, m, k, q, s, yrot);
-            else prep::prep16_kernel<256, 0><<<grid16, block16, 0, stream>>>(xx, m, k, q, s, yrot);
+            if (group == 64) prep::prep16_kernel<64, 0><<<grid16, block16, 0, stream>>>(xx, m, k, q, s, yrot, zero, nzero);
+            else prep::prep16_kernel<256, 0><<<grid16, block16, 0, stream>>>(xx, m, k, q, s, yrot, zero, nzero);
         }
         return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
     }
@@ -261,11 +265,11 @@ convrot_status launch_prep(int num_sms, const void *x, int64_t rows, int64_t K, 
     const uint16_t *xx = static_cast<const uint16_t *>(x);
     const int m = static_cast<int>(rows), k = static_cast<int>(K);
     if (yrot) {
-        if (group == 64) prep::prep_kernel<64, 1><<<grid, block, smem, stream>>>(xx, m, k, q, s, yrot);
-        else prep::prep_kernel<256, 1><<<grid, block, smem, stream>>>(xx, m, k, q, s, yrot);
+        if (group == 64) prep::prep_kernel<64, 1><<<grid, block, smem, stream>>>(xx, m, k, q, s, yrot, zero, nzero);
+        else prep::prep_kernel<256, 1><<<grid, block, smem, stream>>>(xx, m, k, q, s, yrot, zero, nzero);
     } else {
-        if (group == 64) prep::prep_kernel<64, 0><<<grid, block, smem, stream>>>(xx, m, k, q, s, yrot);
-        else prep::prep_kernel<256, 0><<<grid, block, smem, stream>>>(xx, m, k, q, s, yrot);
+        if (group == 64) prep::prep_kernel<64, 0><<<grid, block, smem, stream>>>(xx, m, k, q, s, yrot, zero, nzero);
+        else prep::prep_kernel<256, 0><<<grid, block, smem, stream>>>(xx, m, k, q, s, yrot, zero, nzero);
     }
     return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
@@ -315,11 +319,14 @@ bool make_out_map(CUtensorMap *map, void *y, int64_t M, int64_t N) {
 
 // slots: CTAs (CTA pairs when PAIR) the persistent grid may use.
 // wrep: the weights (qB, or qA in the swapped forms) are repacked.
+// split_tiles, splits, split_ws: the split-K plan (gemm.cuh, "Split K");
+// split_tiles = 0 runs every tile whole.
 template <int BN, bool SWAP, bool OUT_S32, bool PAIR = false>
 convrot_status launch_gemm_cfg(int slots, const uint8_t *qA, const uint8_t *qB, int64_t rowsA,
                                int64_t rowsB, int64_t K, const float *sx, const float *sw,
                                const void *bias, void *out, int64_t M, int64_t N,
-                               cudaStream_t stream, bool wrep = false) {
+                               cudaStream_t stream, bool wrep = false, int split_tiles = 0,
+                               int splits = 1, uint32_t *split_ws = nullptr) {
     using C = gemm::Cfg<BN, SWAP, PAIR>;
     CUtensorMap tmA, tmB, tmY;
     constexpr int pkb = C::PKB;
@@ -336,8 +343,10 @@ convrot_status launch_gemm_cfg(int slots, const uint8_t *qA, const uint8_t *qB, 
     } else {
         tmY = tmA;   // unused by the kernel
     }
+    if (split_tiles > 0 && (SWAP || BN < 64 || !split_ws || splits < 2)) return CONVROT_ERR_UNSUPPORTED;
     const int64_t tiles = ((rowsA + C::TM - 1) / C::TM) * ((rowsB + BN - 1) / BN);
-    const int grid = static_cast<int>(tiles < slots ? tiles : slots) * C::CG;
+    const int64_t units = tiles + static_cast<int64_t>(split_tiles) * (splits - 1);
+    const int grid = static_cast<int>(units < slots ? units : slots) * C::CG;
     // Programmatic dependent launch: the GEMM's set-up (barriers, TMEM,
     // descriptor prefetch) overlaps the end of the preceding kernel on the
     // stream (normally the prep kernel); the kernel waits for that grid's
@@ -360,7 +369,7 @@ convrot_status launch_gemm_cfg(int slots, const uint8_t *qA, const uint8_t *qB, 
         &cfg, gemm::gemm_kernel<BN, SWAP, OUT_S32, PAIR>, tmA, tmB, tmY, use_tma_store,
         static_cast<int>(rowsA), static_cast<int>(rowsB), static_cast<int>(K), sx, sw,
         static_cast<const uint16_t *>(bias), out, static_cast<int>(M), static_cast<int>(N),
-        wrep ? 1 : 0);
+        wrep ? 1 : 0, split_tiles, split_tiles > 0 ? splits : 1, split_ws);
     return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 
@@ -430,6 +439,9 @@ convrot_status launch_skinny(int num_sms, const uint8_t *qx, const float *sx, co
                                            weights_ready, stream, wrep);
 }
 
+// Up to this many tokens the GEMM is the few-token (weight-streaming) form.
+constexpr int64_t kSkinnyMaxM = 128;
+
 // GEMM forms: the automatic choice, the three token-major tile shapes, and
 // the two few-token forms (M <= 128).
 enum TileChoice {
@@ -437,20 +449,75 @@ enum TileChoice {
     kSkinnyTmem = 4, kSkinnySmem = 5, kTiles256x128Pair = 6, kSkinnyPair = 7
 };
 
+// Split-K area handed to the token-major GEMM: counters, then partial slots
+// (gemm.cuh, "Split K").  bytes = 0: no split.
+struct SplitArea {
+    uint32_t *ws = nullptr;
+    size_t bytes = 0;
+    int force_tiles = -1;   // >= 0: this plan instead of the planner's (test hook)
+    int force_splits = 1;
+};
+
+// Partial slots (one per split unit and CTA) of BM x BN int32 that fit.
+int64_t split_capacity(const SplitArea &a, int BN) {
+    if (!a.ws || a.bytes < CONVROT_SPLIT_COUNTER_BYTES) return 0;
+    return static_cast<int64_t>((a.bytes - CONVROT_SPLIT_COUNTER_BYTES) /
+                                (static_cast<size_t>(gemm::BM) * BN * 4));
+}
+
+// The planner: `tiles` output tiles (BM x bn int32 accumulators per CTA) of
+// `num_kp` packed K-stages each on `slots` CTAs (pairs of cg CTAs).  Whole
+// waves stay whole; the `rem` tiles of a part-filled last wave may be split
+// into s parts (2 <= s <= 4, every part at least two stages, rem * s units
+// within one wave and the area), which the schedule runs first.  `cost` =
+// the busiest CTA's K-stages plus the split's own cost in stages: writing,
+// fencing and reading back the partial sums, measured on a B200 as about 3
+// stages plus 0.6 stage per MB of partials (e.g. the 1536 x 12288 -> 3072
+// layer: 59.7 us unsplit, 44.1 us in 3 parts; the 512 x 4096 -> 2048 layer,
+// one part-filled wave of 16-stage tiles: 14.8 us unsplit, 15.7 us in 3
+// parts).  The split with the lowest cost is taken if it beats no split.
+struct SplitPlan {
+    int split_tiles = 0, splits = 1;
+    int64_t cost = 0;   // K-stages of the busiest CTA, plus the split's cost
+};
+
+SplitPlan plan_split(int64_t tiles, int64_t slots, int64_t num_kp, int64_t capacity, int cg,
+                     int bn) {
+    SplitPlan p;
+    const int64_t full = tiles / slots, rem = tiles % slots;
+    p.cost = (full + (rem ? 1 : 0)) * num_kp;
+    if (rem == 0 || capacity <= 0 || rem * cg * gemm::kEpiWarps > gemm::kSplitCounters) return p;
+    int64_t smax = std::min<int64_t>(slots / rem, 4);
+    smax = std::min<int64_t>(smax, num_kp / 2);
+    smax = std::min<int64_t>(smax, capacity / (rem * cg));
+    for (int64_t sp = 2; sp <= smax; ++sp) {
+        const int64_t partial_bytes = rem * sp * cg * gemm::BM * bn * 4;
+        const int64_t cost = full * num_kp + (num_kp + sp - 1) / sp + 3 +
+                             (partial_bytes * 6 + 5000000) / 10000000;
+        if (cost < p.cost) {
+            p.split_tiles = static_cast<int>(rem);
+            p.splits = static_cast<int>(sp);
+            p.cost = cost;
+        }
+    }
+    return p;
+}
+
 // Path choice: up to 128 tokens the few-token form (weights on the 128-row
 // MMA side, widened into TMEM, one CTA per slice of weight rows); otherwise
-// tokens on the M side, with the tile shape that finishes first.
+// tokens on the M side, with the tile shape (and split-K plan) that finishes
+// first.
 template <bool OUT_S32>
 convrot_status launch_gemm(const DeviceState &ds, const uint8_t *qx, const float *sx,
                            const uint8_t *qw, const float *sw, const void *bias, int64_t M,
                            int64_t N, int64_t K, void *out, cudaStream_t stream,
                            int tiles = kTilesAuto, bool weights_ready = false,
-                           bool wrep = false) {
+                           bool wrep = false, const SplitArea &area = SplitArea()) {
     const int num_sms = ds.num_sms;
     // Few tokens: the weight-streaming form.  (The CTA-pair form measured
     // the same at 128 tokens and slower below: each SM's tensor core does
     // the same work per weight byte either way.)
-    if (tiles == kTilesAuto && M <= 128) tiles = kSkinnyTmem;
+    if (tiles == kTilesAuto && M <= kSkinnyMaxM) tiles = kSkinnyTmem;
     if (tiles == kSkinnyTmem && M > 128) return CONVROT_ERR_SHAPE;
     if (tiles == kSkinnySmem && M > 128) return CONVROT_ERR_SHAPE;
     if (tiles == kSkinnyPair && M > 128) return CONVROT_ERR_SHAPE;
@@ -471,48 +538,84 @@ convrot_status launch_gemm(const DeviceState &ds, const uint8_t *qx, const float
         return launch_gemm_cfg<128, true, OUT_S32>(num_sms, qw, qx, N, M, K, sx, sw, bias, out, M, N,
                                                    stream, wrep);
     }
+    // Token-major shapes: {BN, rows of A per tile, CTAs per tile, packed
+    // bytes per K-stage} of each choice, and its plan.
+    struct Shape {
+        int64_t ntiles, slots, num_kp, capacity;
+        int cg, bn;
+    };
+    const auto shape_of = [&](int t) {
+        const bool pair = t == kTiles256x128Pair || t == kTiles256x192Pair;
+        const int bn = (t == kTiles256x128Pair) ? 128 : (t == kTiles128x256) ? 256 : 192;
+        const int tm = pair ? 256 : 128;
+        const int pkb = (t == kTiles128x256) ? 64 : 128;
+        return Shape{((M + tm - 1) / tm) * ((N + bn - 1) / bn),
+                     pair ? static_cast<int64_t>(ds.pair_clusters) : static_cast<int64_t>(num_sms),
+                     (K / 2 + pkb - 1) / pkb, split_capacity(area, bn), pair ? 2 : 1, bn};
+    };
+    const auto shape_plan = [&](int t) {
+        const Shape h = shape_of(t);
+        return plan_split(h.ntiles, h.slots, h.num_kp, h.capacity, h.cg, h.bn);
+    };
     if (tiles == kTilesAuto) {
         // Measured on layers of 1024-8192 tokens and K 3072-12288: the
         // 256 x 192 pair beats both single-CTA shapes everywhere (each SM
-        // widens half of B and the tensor core reads A from TMEM).  Without CTA
-        // pairs the cost is wave-weighted (a tile count just above a multiple
-        // of the SMs wastes a wave): one 256-code stage of a wave takes ~1880
-        // cycles on 128 x 256 tiles (both operands widened in shared memory)
-        // and ~1340 on 128 x 192 (A in TMEM).
+        // widens half of B and the tensor core reads A from TMEM).  The cost
+        // of a choice is the busiest CTA's K-stages (waves, less what split K
+        // takes off the last one) times a stage's time.
         if (ds.pair_clusters > 0) {
             // A 256 x 128 pair tile takes ~0.9 of a 256 x 192 one's time
             // (measured on 1024-8192 tokens), so the narrower tile wins only
-            // where the 192-wide grid wastes most of a last wave: e.g. 96
-            // tiles on 74 pairs (1536 x 3072) against 144.
-            const auto waves = [](int64_t t, int64_t slots) { return (t + slots - 1) / slots; };
-            const int64_t ta = (M + 255) / 256;
-            const int64_t c192 = waves(ta * ((N + 191) / 192), ds.pair_clusters) * 10;
-            const int64_t c128 = waves(ta * ((N + 127) / 128), ds.pair_clusters) * 9;
+            // where the 192-wide grid wastes most of a last wave that split K
+            // does not recover.
+            const int64_t c192 = shape_plan(kTiles256x192Pair).cost * 10;
+            const int64_t c128 = shape_plan(kTiles256x128Pair).cost * 9;
             tiles = c128 < c192 ? kTiles256x128Pair : kTiles256x192Pair;
         } else {
-            const auto waves = [](int64_t t, int64_t slots) { return (t + slots - 1) / slots; };
-            const int64_t c_ss = waves(((M + 127) / 128) * ((N + 255) / 256), num_sms) * 1880;
-            const int64_t c_atm = waves(((M + 127) / 128) * ((N + 191) / 192), num_sms) * 1340;
+            // a 128-code stage takes ~940 cycles on 128 x 256 tiles (both
+            // operands widened in shared memory), a 256-code stage ~1340 on
+            // 128 x 192 (A in TMEM)
+            const int64_t c_ss = shape_plan(kTiles128x256).cost * 940;
+            const int64_t c_atm = shape_plan(kTiles128x192).cost * 1340;
             tiles = c_atm <= c_ss ? kTiles128x192 : kTiles128x256;
         }
     }
+    if (tiles != kTiles256x128Pair && tiles != kTiles256x192Pair && tiles != kTiles128x192 &&
+        tiles != kTiles128x256)
+        return CONVROT_ERR_SHAPE;
+    SplitPlan plan = shape_plan(tiles);
+    if (area.force_tiles > 0) {
+        // a given plan: every part at least one K-stage, every slot and
+        // counter inside the area
+        const Shape h = shape_of(tiles);
+        const int64_t ft = area.force_tiles, fs = area.force_splits;
+        if (ft > h.ntiles || fs < 2 || fs > h.num_kp || ft * h.cg * gemm::kEpiWarps > gemm::kSplitCounters ||
+            ft * fs * h.cg > h.capacity)
+            return CONVROT_ERR_SHAPE;
+        plan.split_tiles = area.force_tiles;
+        plan.splits = area.force_splits;
+    } else if (area.force_tiles == 0) {
+        plan.split_tiles = 0;
+        plan.splits = 1;
+    }
+    const int st = plan.split_tiles, sp = plan.splits;
     if (tiles == kTiles256x128Pair) {
         if (ds.pair_clusters <= 0) return CONVROT_ERR_UNSUPPORTED;
         return launch_gemm_cfg<128, false, OUT_S32, true>(ds.pair_clusters, qx, qw, M, N, K, sx, sw,
-                                                          bias, out, M, N, stream, wrep);
+                                                          bias, out, M, N, stream, wrep, st, sp,
+                                                          area.ws);
     }
     if (tiles == kTiles256x192Pair) {
         if (ds.pair_clusters <= 0) return CONVROT_ERR_UNSUPPORTED;
         return launch_gemm_cfg<192, false, OUT_S32, true>(ds.pair_clusters, qx, qw, M, N, K, sx, sw,
-                                                          bias, out, M, N, stream, wrep);
+                                                          bias, out, M, N, stream, wrep, st, sp,
+                                                          area.ws);
     }
     if (tiles == kTiles128x192)
         return launch_gemm_cfg<192, false, OUT_S32>(num_sms, qx, qw, M, N, K, sx, sw, bias, out, M,
-                                                    N, stream, wrep);
-    if (tiles == kTiles128x256)
-        return launch_gemm_cfg<256, false, OUT_S32>(num_sms, qx, qw, M, N, K, sx, sw, bias, out, M,
-                                                    N, stream, wrep);
-    return CONVROT_ERR_SHAPE;
+                                                    N, stream, wrep, st, sp, area.ws);
+    return launch_gemm_cfg<256, false, OUT_S32>(num_sms, qx, qw, M, N, K, sx, sw, bias, out, M, N,
+                                                stream, wrep, st, sp, area.ws);
 }
 
 // The one-kernel path for 1..4 tokens (decode.cuh): token rows prepared in
@@ -575,10 +678,20 @@ convrot_status check_gemm_args(const uint8_t *qx, const uint8_t *qw, int64_t M, 
 
 inline size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
+static_assert(gemm::kSplitCounters * 4 == CONVROT_SPLIT_COUNTER_BYTES, "split counter bytes");
+
+// Workspace of the prepared activations (codes, then scales); the split
+// area, where there is one, follows.
+size_t prepared_bytes(int64_t M, int64_t K) {
+    return round256(static_cast<size_t>(M) * static_cast<size_t>(K / 2)) +
+           round256(static_cast<size_t>(M) * sizeof(float));
+}
+
 // steps 3-4 on prepared operands; wrep: qw is in the repacked layout
 convrot_status linear_prepared_impl(const uint8_t *qx, const float *sx, const uint8_t *qw,
                                     const float *sw, const void *bias_bf16, int64_t M, int64_t N,
-                                    int64_t K, void *y_bf16, cudaStream_t stream, bool wrep) {
+                                    int64_t K, void *y_bf16, cudaStream_t stream, bool wrep,
+                                    const SplitArea &area = SplitArea()) {
     if (M < 0 || N < 0) return CONVROT_ERR_SHAPE;
     if (M == 0 || N == 0) return CONVROT_OK;
     convrot_status st = check_gemm_args(qx, qw, M, N, K);
@@ -589,9 +702,10 @@ convrot_status linear_prepared_impl(const uint8_t *qx, const float *sx, const ui
         return CONVROT_ERR_ALIGN;
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
-    if ((st = check_device_ptrs(dev, {qx, sx, qw, sw, bias_bf16, y_bf16})) != CONVROT_OK) return st;
+    if ((st = check_device_ptrs(dev, {qx, sx, qw, sw, bias_bf16, y_bf16, area.ws})) != CONVROT_OK)
+        return st;
     return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream,
-                              kTilesAuto, false, wrep);
+                              kTilesAuto, false, wrep, area);
 }
 
 // steps 1-4; wrep: qw is in the repacked layout
@@ -604,8 +718,8 @@ convrot_status linear_impl(const void *x_bf16, const uint8_t *qw, const float *s
     if (N < 0) return CONVROT_ERR_SHAPE;
     if (M == 0 || N == 0) return CONVROT_OK;
     if (!x_bf16 || !qw || !sw || !y_bf16 || !workspace) return CONVROT_ERR_NULL;
-    if (ws_bytes < convrot_linear_workspace_size(M, K) ||
-        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    const size_t base = prepared_bytes(M, K);
+    if (ws_bytes < base || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return CONVROT_ERR_WORKSPACE;
     if (!aligned16(x_bf16) || !aligned16(qw) || !aligned16(sw) || !aligned16(y_bf16) ||
         (bias_bf16 && !aligned16(bias_bf16)))
@@ -625,10 +739,18 @@ convrot_status linear_impl(const void *x_bf16, const uint8_t *qw, const float *s
                                  group, y_bf16, stream, wrep);
     uint8_t *qx = static_cast<uint8_t *>(workspace);
     float *sx = reinterpret_cast<float *>(qx + round256(static_cast<size_t>(M) * (K / 2)));
-    if ((st = launch_prep(g_dev[dev].num_sms, x_bf16, M, K, group, qx, sx, nullptr, stream)) != CONVROT_OK)
+    // The split area, when the workspace holds one and the token-major GEMM
+    // runs; the prep kernel zeroes its counters.
+    SplitArea area;
+    if (M > kSkinnyMaxM && ws_bytes >= base + CONVROT_SPLIT_AREA_BYTES) {
+        area.ws = reinterpret_cast<uint32_t *>(qx + base);
+        area.bytes = CONVROT_SPLIT_AREA_BYTES;
+    }
+    if ((st = launch_prep(g_dev[dev].num_sms, x_bf16, M, K, group, qx, sx, nullptr, stream,
+                          area.ws, area.ws ? gemm::kSplitCounters : 0)) != CONVROT_OK)
         return st;
     return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream,
-                              kTilesAuto, true, wrep);
+                              kTilesAuto, true, wrep, area);
 }
 
 // The reversible block-major repack (16 bytes per thread, grid-stride).
@@ -722,14 +844,28 @@ convrot_status convrot_prepare_act(const void *x_bf16, int64_t M, int64_t K, int
 
 size_t convrot_linear_workspace_size(int64_t M, int64_t K) {
     if (M <= 0 || K <= 0) return 0;
-    return round256(static_cast<size_t>(M) * static_cast<size_t>(K / 2)) +
-           round256(static_cast<size_t>(M) * sizeof(float));
+    return prepared_bytes(M, K) + (M > kSkinnyMaxM ? CONVROT_SPLIT_AREA_BYTES : 0);
 }
 
 convrot_status convrot_linear_prepared(const uint8_t *qx, const float *sx, const uint8_t *qw,
                                        const float *sw, const void *bias_bf16, int64_t M, int64_t N,
                                        int64_t K, void *y_bf16, convrot_stream_t stream) {
     return linear_prepared_impl(qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream, false);
+}
+
+convrot_status convrot_linear_prepared_split(const uint8_t *qx, const float *sx,
+                                             const uint8_t *qw, const float *sw,
+                                             const void *bias_bf16, int64_t M, int64_t N,
+                                             int64_t K, void *split_ws, size_t split_bytes,
+                                             void *y_bf16, convrot_stream_t stream) {
+    SplitArea area;
+    if (split_ws) {
+        if (split_bytes < CONVROT_SPLIT_AREA_BYTES || (reinterpret_cast<uintptr_t>(split_ws) & 255u))
+            return CONVROT_ERR_WORKSPACE;
+        area.ws = static_cast<uint32_t *>(split_ws);
+        area.bytes = CONVROT_SPLIT_AREA_BYTES;
+    }
+    return linear_prepared_impl(qx, sx, qw, sw, bias_bf16, M, N, K, y_bf16, stream, false, area);
 }
 
 convrot_status convrot_linear(const void *x_bf16, const uint8_t *qw, const float *sw,
@@ -829,6 +965,44 @@ convrot_status convrot_debug_gemm_tiles(const uint8_t *qx, const float *sx, cons
                               false, wrep);
 }
 
+convrot_status convrot_debug_gemm_split(const uint8_t *qx, const float *sx, const uint8_t *qw,
+                                        const float *sw, const void *bias_bf16, int64_t M,
+                                        int64_t N, int64_t K, int tiles, int split_tiles,
+                                        int splits, void *split_ws, size_t split_bytes,
+                                        int out_s32, void *out, convrot_stream_t stream) {
+    if (M < 0 || N < 0) return CONVROT_ERR_SHAPE;
+    const bool wrep = (tiles & CONVROT_TILES_REPACKED) != 0;
+    tiles &= ~CONVROT_TILES_REPACKED;
+    if (tiles != kTilesAuto && tiles != kTiles128x256 && tiles != kTiles128x192 &&
+        tiles != kTiles256x192Pair && tiles != kTiles256x128Pair)
+        return CONVROT_ERR_SHAPE;
+    if (split_tiles < -1 || (split_tiles > 0 && splits < 2)) return CONVROT_ERR_SHAPE;
+    if (M <= kSkinnyMaxM) return CONVROT_ERR_SHAPE;   // the token-major forms only
+    if (N == 0) return CONVROT_OK;
+    convrot_status st = check_gemm_args(qx, qw, M, N, K);
+    if (st != CONVROT_OK) return st;
+    if (!out || !split_ws || (!out_s32 && (!sx || !sw))) return CONVROT_ERR_NULL;
+    if (split_bytes < CONVROT_SPLIT_COUNTER_BYTES || (reinterpret_cast<uintptr_t>(split_ws) & 255u))
+        return CONVROT_ERR_WORKSPACE;
+    if (!aligned16(out) || (!out_s32 && (!aligned16(sx) || !aligned16(sw) ||
+                                         (bias_bf16 && !aligned16(bias_bf16)))))
+        return CONVROT_ERR_ALIGN;
+    int dev;
+    if ((st = device_setup(&dev)) != CONVROT_OK) return st;
+    if ((st = check_device_ptrs(dev, {qx, qw, out, split_ws})) != CONVROT_OK) return st;
+    if (!out_s32 && (st = check_device_ptrs(dev, {sx, sw, bias_bf16})) != CONVROT_OK) return st;
+    SplitArea area;
+    area.ws = static_cast<uint32_t *>(split_ws);
+    area.bytes = split_bytes;
+    area.force_tiles = split_tiles;
+    area.force_splits = splits;
+    if (out_s32)
+        return launch_gemm<true>(g_dev[dev], qx, nullptr, qw, nullptr, nullptr, M, N, K, out, stream,
+                                 tiles, false, wrep, area);
+    return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, out, stream, tiles,
+                              false, wrep, area);
+}
+
 convrot_status convrot_check_device_error(convrot_stream_t stream) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return CONVROT_ERR_CUDA;
     int v = 0;
@@ -917,8 +1091,7 @@ extern "C" convrot_status convrot_linear_noalloc(const void *x_bf16, const uint8
         (bias_bf16 && !aligned16(bias_bf16)))
         return CONVROT_ERR_ALIGN;
     if ((st = check_gemm_args(qw, qw, M, N, K)) != CONVROT_OK) return st;
-    if (convrot_linear_workspace_size(M, K) > CONVROT_NOALLOC_SCRATCH_BYTES)
-        return CONVROT_ERR_SCRATCH_LIMIT;
+    if (prepared_bytes(M, K) > CONVROT_NOALLOC_SCRATCH_BYTES) return CONVROT_ERR_SCRATCH_LIMIT;
     int dev;
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
     if ((st = check_device_ptrs(dev, {x_bf16, qw, sw, bias_bf16, y_bf16})) != CONVROT_OK) return st;

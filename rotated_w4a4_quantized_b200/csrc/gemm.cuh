@@ -33,6 +33,20 @@
 // Accumulators are double-buffered in TMEM so the epilogue of one tile runs
 // under the main loop of the next.
 //
+// Split K.  Where the tiles leave the last wave of the persistent grid
+// part-filled, the host may split the first `split_tiles` tiles into
+// `splits` contiguous ranges of K-blocks each.  These split units come first
+// in the schedule (one per CTA or pair), so their fix-up overlaps the whole
+// tiles that follow.  Each epilogue warp of a split unit writes its region
+// of the raw accumulators (256 x a partial sum; 32 rows x half the columns)
+// to the unit's slot in the split area, then counts itself in on the
+// region's counter with one atomic.  The warp that arrives last adds the
+// other parts' copies of its region to its own accumulators and runs the
+// epilogue on it: integer addition is exact and associative, so the result
+// is bit-identical to the unsplit one in any arrival order, and no warp or
+// CTA ever waits for another.  The counter wraps back to zero on the last
+// arrival (atom.inc), so it is ready for the next launch.
+//
 // SWAP selects the skinny-M form: the weights become the 128-row MMA operand
 // and the few token rows the N-side operand (BN = 16 .. 128), so the weight
 // stream is split over many CTAs; the epilogue writes the transposed tile
@@ -54,6 +68,34 @@ constexpr int kWarpTma = 0, kWarpMma = 1, kWarpEpi0 = 2, kEpiWarps = 8;
 constexpr int kWarpUnp0 = kWarpEpi0 + kEpiWarps, kUnpWarps = 8;
 constexpr int kThreads = (kWarpUnp0 + kUnpWarps) * 32;    // 576
 constexpr int kStoreBox = 32;    // epilogue TMA-store box: 32 rows x 32 bf16
+// Split area: kSplitCounters counter words (one per split tile, CTA and
+// epilogue warp), then one slot of BM x BN int32 per split unit and CTA.
+constexpr int kSplitCounters = 2048;
+
+// One unit of the persistent schedule: output tile `tile`, packed K-stages
+// [kp0, kp1), and its part index (-1 for a whole tile).  Units
+// 0 .. split_tiles * splits - 1 are the parts of tiles 0 .. split_tiles - 1
+// (part p of tile t is unit t * splits + p); the rest are whole tiles.
+struct Unit {
+    int tile, kp0, kp1, part;
+};
+
+__device__ __forceinline__ Unit unit_at(int u, int split_tiles, int splits, int num_kp) {
+    Unit w;
+    const int nsu = split_tiles * splits;
+    if (u < nsu) {
+        w.tile = u / splits;
+        w.part = u - w.tile * splits;
+        w.kp0 = w.part * num_kp / splits;
+        w.kp1 = (w.part + 1) * num_kp / splits;
+    } else {
+        w.tile = u - nsu + split_tiles;
+        w.part = -1;
+        w.kp0 = 0;
+        w.kp1 = num_kp;
+    }
+    return w;
+}
 
 // PAIR: a 2-CTA cluster computes one 256 x BN tile with cta_group::2 MMAs;
 // each CTA holds 128 rows of A (in its TMEM), BN / 2 rows of B (in its
@@ -210,7 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmY, int use_tma_store, int rowsA, int rowsB,
             int K, const float *__restrict__ sx, const float *__restrict__ sw,
-            const uint16_t *__restrict__ bias, void *__restrict__ out, int M, int N, int wrep) {
+            const uint16_t *__restrict__ bias, void *__restrict__ out, int M, int N, int wrep,
+            int split_tiles, int splits, uint32_t *__restrict__ split_ws) {
     using C = Cfg<BN, SWAP, PAIR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -276,11 +319,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     const int tiles_a = (rowsA + C::TM - 1) / C::TM;
     const int tiles_b = (rowsB + BN - 1) / BN;
     const int num_tiles = tiles_a * tiles_b;
-    // Persistent schedule: tile t goes to CTA (pair) t mod the grid.
+    // Persistent schedule: unit u goes to CTA (pair) u mod the grid.
+    const int num_units = num_tiles + split_tiles * (splits - 1);
     const int first_tile = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
     const int tile_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
     const int num_kp = (K / 2 + C::PKB - 1) / C::PKB;   // packed stages per tile
-    const int num_kb = num_kp * C::PSUB;                // widened K-blocks per tile
 
     // The producer and MMA loops run in one thread each (lane 0): a warp-wide
     // mbarrier operation costs a multiple of one thread's.
@@ -288,9 +331,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         int ps = 0;
         uint32_t ph = 0;
         bool ok = true;
-        for (int tile = first_tile; lane == 0 && tile < num_tiles && ok; tile += tile_step) {
-            const int ta = tile % tiles_a, tb = tile / tiles_a;
-            for (int kp = 0; kp < num_kp; ++kp) {
+        for (int u = first_tile; lane == 0 && u < num_units && ok; u += tile_step) {
+            const Unit w = unit_at(u, split_tiles, splits, num_kp);
+            const int ta = w.tile % tiles_a, tb = w.tile / tiles_a;
+            for (int kp = w.kp0; kp < w.kp1; ++kp) {
                 if (!ptx::mbar_wait(empty_p(ps), ph ^ 1, abort_flag)) { ok = false; break; }
                 ptx::mbar_arrive_expect_tx(full_p(ps), C::PA + C::PB);
                 // the weights (B, or A in the swapped form) may be repacked
@@ -321,7 +365,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         uint32_t ph = 0;
         int local = 0;
         bool ok = true;
-        for (int tile = first_tile; issuer && tile < num_tiles && ok; tile += tile_step, ++local) {
+        for (int u = first_tile; issuer && u < num_units && ok; u += tile_step, ++local) {
+            const Unit w = unit_at(u, split_tiles, splits, num_kp);
+            const int num_kb = (w.kp1 - w.kp0) * C::PSUB;   // widened K-blocks of the unit
             const int b = local & 1;
             const uint32_t aph = (local >> 1) & 1;
             if (!ptx::mbar_wait<PAIR>(acc_empty(b), aph ^ 1, abort_flag)) { ok = false; break; }
@@ -370,8 +416,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         const uint32_t box0 = sbase + C::OFF_ST + e * (C::SB * kStoreBox * kStoreBox * 2);
         int nstores = 0;
         int local = 0;
-        for (int tile = first_tile; tile < num_tiles; tile += tile_step, ++local) {
-            const int ta = tile % tiles_a, tb = tile / tiles_a;
+        for (int u = first_tile; u < num_units; u += tile_step, ++local) {
+            const Unit w = unit_at(u, split_tiles, splits, num_kp);
+            const int ta = w.tile % tiles_a, tb = w.tile / tiles_a;
             const int b = local & 1;
             const uint32_t aph = (local >> 1) & 1;
             const int row0 = ta * C::TM + static_cast<int>(rank) * BM;   // this CTA's first A row
@@ -396,17 +443,76 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             }
             if (!ptx::mbar_wait<PAIR>(acc_full(b), aph, abort_flag)) break;
             ptx::tc_fence_after();
-            if (active) {
+            const uint32_t acc_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                      static_cast<uint32_t>(b * C::ACC_STRIDE);
+            bool emit = true;
+            if constexpr (!SWAP && BN >= 64) {
+                if (w.part >= 0) {
+                    // A part of a split tile: this warp's region of the raw
+                    // accumulators goes to the unit's slot, 32 columns at a
+                    // time as eight 16-byte words per row, word j4 of column
+                    // block c of row r at ((c * 8 + j4) * BM + r) * 4
+                    // (coalesced across the warp).
+                    uint32_t *slot = split_ws + kSplitCounters +
+                                     static_cast<size_t>(u * C::CG + static_cast<int>(rank)) * (BM * BN);
+#pragma unroll 1
+                    for (int c0 = col_begin; c0 < col_begin + kCols; c0 += 32) {
+                        uint32_t v[32];
+                        __syncwarp();
+                        ptx::tmem_ld_32x32b_x32(acc_lane + static_cast<uint32_t>(c0), v);
+                        ptx::tmem_ld_wait();
+                        uint32_t *dst = slot + (static_cast<size_t>(c0 / 32) * 8 * BM + r) * 4;
+#pragma unroll
+                        for (int j4 = 0; j4 < 8; ++j4)
+                            ptx::st_cg_v4(dst + j4 * BM * 4, v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2],
+                                          v[4 * j4 + 3]);
+                    }
+                    // The region is in the slot before the counter moves; the
+                    // last arrival then sees every other part's copy of it.
+                    __threadfence();
+                    __syncwarp();
+                    uint32_t old = 0;
+                    if (lane == 0)
+                        old = ptx::atom_inc_acq_rel(
+                            split_ws + (w.tile * C::CG + static_cast<int>(rank)) * kEpiWarps + e,
+                            static_cast<uint32_t>(splits - 1));
+                    old = __shfl_sync(0xFFFFFFFFu, old, 0);
+                    emit = old == static_cast<uint32_t>(splits - 1);
+                    if (emit) __threadfence();
+                }
+            }
+            if (active && emit) {
 #pragma unroll 1
                 for (int c0 = col_begin; c0 < col_begin + kCols; c0 += 32) {
                     const int bcol0 = tb * BN + c0;   // first B row of these 32 columns
                     uint32_t v[32];
                     __syncwarp();   // tcgen05.ld is warp-collective
-                    ptx::tmem_ld_32x32b_x32(
-                        tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                            static_cast<uint32_t>(b * C::ACC_STRIDE + c0),
-                        v);
+                    ptx::tmem_ld_32x32b_x32(acc_lane + static_cast<uint32_t>(c0), v);
                     ptx::tmem_ld_wait();
+                    if constexpr (!SWAP && BN >= 64) {
+                        if (w.part >= 0) {
+                            // last part of a split tile: add the other parts
+                            for (int p = 0; p < splits; ++p) {
+                                if (p == w.part) continue;
+                                const uint32_t *src =
+                                    split_ws + kSplitCounters +
+                                    static_cast<size_t>((w.tile * splits + p) * C::CG +
+                                                        static_cast<int>(rank)) * (BM * BN) +
+                                    (static_cast<size_t>(c0 / 32) * 8 * BM + r) * 4;
+                                // all eight loads in flight before the first add
+                                uint4 q[8];
+#pragma unroll
+                                for (int j4 = 0; j4 < 8; ++j4) q[j4] = ptx::ld_cg_v4(src + j4 * BM * 4);
+#pragma unroll
+                                for (int j4 = 0; j4 < 8; ++j4) {
+                                    v[4 * j4] += q[j4].x;
+                                    v[4 * j4 + 1] += q[j4].y;
+                                    v[4 * j4 + 2] += q[j4].z;
+                                    v[4 * j4 + 3] += q[j4].w;
+                                }
+                            }
+                        }
+                    }
                     if (!SWAP && !OUT_S32 && tma_out) {
                         // 32 rows x 32 columns through a swizzled box, one TMA store
                         const int n0 = bcol0;
@@ -505,8 +611,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         // Warps 4..7 widen B into the swizzled shared-memory stage, one
         // 128-byte-row tile per K-block.
         const int uw = warp - kWarpUnp0;
-        const int my_tiles = num_tiles > first_tile ? (num_tiles - 1 - first_tile) / tile_step + 1 : 0;
-        const int total = my_tiles * num_kb;
+        int total = 0;   // widened stages this CTA runs
+        for (int u = first_tile; u < num_units; u += tile_step) {
+            const Unit w = unit_at(u, split_tiles, splits, num_kp);
+            total += (w.kp1 - w.kp0) * C::PSUB;
+        }
         const uint32_t hm = 0xF0F0F0F0u;
         if (uw < 4) {
             const int quarter = warp & 3;             // TMEM lanes 32*quarter ..
@@ -612,8 +721,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         const uint32_t sw8 = static_cast<uint32_t>((ut >> 2) & 7);
         const uint32_t lo_off = ((2u * c) ^ sw8) << 4;
         const uint32_t hi_off = ((2u * c + 1u) ^ sw8) << 4;
-        const int my_tiles = num_tiles > first_tile ? (num_tiles - 1 - first_tile) / tile_step + 1 : 0;
-        const int total = my_tiles * num_kb;            // stages this CTA runs
+        int total = 0;                                  // stages this CTA runs
+        for (int u = first_tile; u < num_units; u += tile_step) {
+            const Unit w = unit_at(u, split_tiles, splits, num_kp);
+            total += (w.kp1 - w.kp0) * C::PSUB;
+        }
         for (int n = ug; n < total; n += C::UG) {
             const int np = n / C::PSUB, sub = n % C::PSUB;   // packed stage, K-block in it
             const int ps = np % C::SP, us = n % C::SU;

@@ -290,9 +290,13 @@ __host__ __device__ constexpr int stage_buffers(int G) { return G == 256 ? 2 : 1
 template <int G, int MODE>
 __global__ void __launch_bounds__(kMaxThreads)
 prep_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ q,
-            float *__restrict__ s, float *__restrict__ yrot) {
+            float *__restrict__ s, float *__restrict__ yrot, uint32_t *__restrict__ zero,
+            int nzero) {
     static_assert(G == 64 || G == 256, "group 64 or 256");
     constexpr int kDigits = (G == 64) ? 3 : 4;
+    // side job for the GEMM that follows: clear its split counters
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0u;
     constexpr float kNorm = (G == 64) ? 0.125f : 0.0625f;   // 2^-kDigits
     constexpr int NBUF = stage_buffers(G);   // one buffer only without an exchange
 
@@ -420,10 +424,14 @@ __device__ __forceinline__ void radix4_lanes(float (&v)[16], int m1, int m2) {
 template <int G, int MODE>
 __global__ void __maxnreg__(40)
 prep16_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ q,
-              float *__restrict__ s, float *__restrict__ yrot) {
+              float *__restrict__ s, float *__restrict__ yrot, uint32_t *__restrict__ zero,
+              int nzero) {
     static_assert(G == 64 || G == 256, "group 64 or 256");
     constexpr float kNorm = (G == 64) ? 0.125f : 0.0625f;   // 2^-digits
     __shared__ uint32_t red[2][32];
+    // side job for the GEMM that follows: clear its split counters
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0u;
     // blockDim.x = K/16 rounded up to whole warps; K is a multiple of 256, so
     // the padding lanes form whole 16-lane groups: they hold zeros, take part
     // in the shuffles and the maximum, and store nothing.

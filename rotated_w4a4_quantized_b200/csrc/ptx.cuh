@@ -189,6 +189,36 @@ __device__ __forceinline__ void launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// ------------------------------------------------- cross-CTA exchange
+// 16-byte global store and load cached in L2 only: data that another CTA
+// exchanges through global memory never sits in this SM's L1.
+__device__ __forceinline__ void st_cg_v4(uint32_t *p, uint32_t a, uint32_t b, uint32_t c,
+                                         uint32_t d) {
+    asm volatile("st.global.cg.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_cg_v4(const uint32_t *p) {
+    uint4 r;
+    asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p)
+                 : "memory");
+    return r;
+}
+
+// old = *p; *p = old >= limit ? 0 : old + 1 (one atomic, GPU scope, with
+// acquire and release semantics).  Returns old.
+__device__ __forceinline__ uint32_t atom_inc_acq_rel(uint32_t *p, uint32_t limit) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.inc.u32 %0, [%1], %2;"
+                 : "=r"(old)
+                 : "l"(p), "r"(limit)
+                 : "memory");
+    return old;
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -51,7 +51,26 @@ def test_workspace_size(L):
     assert cr.convrot_linear_workspace_size(0, 1024) == 0
     assert cr.convrot_linear_workspace_size(3, 1024) == 1536 + 256
     assert cr.convrot_linear_workspace_size(1, 64) == 256 + 256
-    assert cr.convrot_linear_workspace_size(1024, 3072) == 1024 * 1536 + 4096
+    # the few-token GEMM (M <= 128) never splits K: codes and scales only
+    assert cr.convrot_linear_workspace_size(128, 1024) == 128 * 512 + 512
+    # beyond it the split area follows the codes and scales
+    assert cr.convrot_linear_workspace_size(129, 1024) == 129 * 512 + 768 + cr.SPLIT_AREA_BYTES
+    assert (cr.convrot_linear_workspace_size(1024, 3072)
+            == 1024 * 1536 + 4096 + cr.SPLIT_AREA_BYTES)
+
+
+def test_split_area_constants_match_the_header():
+    text = open(HEADER).read()
+    counters = int(re.search(r"#define CONVROT_SPLIT_COUNTER_BYTES \(\(size_t\)(\d+)\)", text).group(1))
+    m = re.search(r"#define CONVROT_SPLIT_AREA_BYTES \(CONVROT_SPLIT_COUNTER_BYTES \+ "
+                  r"\(size_t\)(\d+) \* (\d+) \* (\d+) \* (\d+)\)", text)
+    slots, rows, cols, word = map(int, m.groups())
+    assert counters == cr.SPLIT_COUNTER_BYTES
+    assert counters + slots * rows * cols * word == cr.SPLIT_AREA_BYTES
+    # one counter per split tile, CTA and epilogue warp (8): a wave of 148
+    # CTAs fits, and so does one wave of 128 x 256 int32 partial slots
+    assert counters // 4 >= 148 * 8
+    assert slots >= 148 and rows * cols * word == 128 * 256 * 4
 
 
 A = ctypes.c_void_p(0x10000)    # fake, aligned, never dereferenced: checks fail first
@@ -91,6 +110,24 @@ def test_host_validation_without_device(L):
     assert L.convrot_debug_gemm_tiles(A, None, A, None, None, 4, 8, 128, 3, 1, U, s) == 4
     assert L.convrot_debug_gemm_tiles(A, B, A, B, U, 4, 8, 128, 1, 0, B, s) == 4
     assert L.convrot_debug_gemm_tiles(None, None, None, None, None, 0, 8, 128, 3, 1, None, s) == 0
+    # split K: the area is checked before anything else of the call
+    area = cr.SPLIT_AREA_BYTES
+    assert L.convrot_linear_prepared_split(A, B, A, B, None, 400, 8, 1024, B, area - 1, B, s) == 5
+    assert L.convrot_linear_prepared_split(A, B, A, B, None, 400, 8, 1024, U, area, B, s) == 5
+    assert L.convrot_linear_prepared_split(A, B, A, B, None, 400, 8, 1000, B, area, B, s) == 3
+    # forced plans: token-major forms and M > 128 only, a split count of 2 or
+    # more, the area present and holding its counters
+    g = L.convrot_debug_gemm_split
+    assert g(A, B, A, B, None, 400, 8, 1024, 4, 1, 2, B, area, 0, B, s) == 3      # few-token form
+    assert g(A, B, A, B, None, 400, 8, 1024, 7, 1, 2, B, area, 0, B, s) == 3
+    assert g(A, B, A, B, None, 128, 8, 1024, 3, 1, 2, B, area, 0, B, s) == 3      # M <= 128
+    assert g(A, B, A, B, None, 400, 8, 1024, 3, 1, 1, B, area, 0, B, s) == 3      # splits < 2
+    assert g(A, B, A, B, None, 400, 8, 1024, 3, -2, 2, B, area, 0, B, s) == 3
+    assert g(A, B, A, B, None, 400, 8, 1024, 3, 1, 2, None, area, 0, B, s) == 1
+    assert g(A, B, A, B, None, 400, 8, 1024, 3, 1, 2, B, 8191, 0, B, s) == 5
+    assert g(A, B, A, B, None, 400, 8, 1024, 3, 1, 2, U, area, 0, B, s) == 5
+    assert g(A, B, A, B, None, 400, 8, 1024, 3, 1, 2, B, area, 0, U, s) == 4
+    assert g(A, B, A, B, None, 400, 0, 1024, 3, 1, 2, None, 0, 0, None, s) == 0  # empty
 
 
 def test_single_kernel_rule(L):
@@ -120,6 +157,11 @@ def test_valid_call_without_gpu_reports_cuda_error(L):
         pytest.skip("a GPU is present")
     # Arguments pass validation; the device set-up then fails cleanly.
     assert L.convrot_prepare_act(A, 4, 1024, 64, B, B, None) == 6
+    # a workspace without the split area is accepted (the call runs unsplit);
+    # one byte less than the codes and scales is not
+    base = cr.convrot_linear_workspace_size(200, 1024) - cr.SPLIT_AREA_BYTES
+    assert L.convrot_linear(A, B, B, None, 200, 8, 1024, 64, A, base, B, None) == 6
+    assert L.convrot_linear(A, B, B, None, 200, 8, 1024, 64, A, base - 1, B, None) == 5
 
 
 # ---------------------------------------------------------------- W4A16 library
