@@ -101,6 +101,27 @@ convrot_status convrot_w4a16_linear_prepared_repacked(const void *xr_bf16, const
                                                       int64_t M, int64_t N, int64_t K,
                                                       void *y_bf16, convrot_stream_t stream);
 
+/*
+ * Test hook: the product on prepared operands (as
+ * convrot_w4a16_linear_prepared) with the GEMM forced to one form, so that
+ * every form is checked whatever the automatic choice for (M, N, K):
+ *   form = 0  automatic (as the entry points above: form 3 up to 64 tokens,
+ *             form 1 beyond);
+ *          1  128 x 256 token-by-weight tiles;
+ *          2  few tokens (M <= 64), weights widened to bf16 in shared memory
+ *             on the MMA's 128-row side;
+ *          3  few tokens (M <= 64), weights widened to bf16 straight into
+ *             TMEM (the MMA's A operand), one CTA per slice of weight rows.
+ * form | CONVROT_TILES_REPACKED takes qw in the repacked layout.  Returns
+ * CONVROT_ERR_SHAPE for any other form or for 2 / 3 with M > 64.  Exposes
+ * the product of "convrot-mlx" README, "What is included" (the W4A16 path)
+ * per GEMM form.
+ */
+convrot_status convrot_w4a16_debug_gemm_form(const void *xr_bf16, const uint8_t *qw,
+                                             const float *sw, const void *bias_bf16, int64_t M,
+                                             int64_t N, int64_t K, int form, void *y_bf16,
+                                             convrot_stream_t stream);
+
 /* Failure detection (no counterpart on the pages).  Synchronise `stream`,
  * then return and clear this library's device error word (CONVROT_OK, or
  * CONVROT_ERR_DEVICE_TIMEOUT after a wait ran out). */

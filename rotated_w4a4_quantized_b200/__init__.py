@@ -457,6 +457,7 @@ def lib_w4a16() -> ctypes.CDLL:
             "convrot_w4a16_check_device_error": [P],
             "convrot_w4a16_linear_prepared_repacked": [P, P, P, P, I64, I64, I64, P, P],
             "convrot_w4a16_linear_repacked": [P, P, P, P, I64, I64, I64, I, P, SZ, P, P],
+            "convrot_w4a16_debug_gemm_form": [P, P, P, P, I64, I64, I64, I, P, P],
         }
         for name, args in sigs.items():
             f = getattr(L, name)
@@ -495,6 +496,34 @@ def convrot_w4a16_linear_prepared(xr, qw, sw, bias, out=None, stream=None):
         _check(lib_w4a16().convrot_w4a16_linear_prepared(_p(xr), _p(qw), _p(sw), _p(bias), M, N,
                                                          K, _p(out), _stream(stream)),
                "convrot_w4a16_linear_prepared")
+    return out
+
+
+# GEMM forms of convrot_w4a16_debug_gemm_form: automatic, 128 x 256 tiles,
+# few tokens (M <= 64) with the weights widened in shared memory or in TMEM
+W4A16_AUTO, W4A16_TILES, W4A16_FEW_SMEM, W4A16_FEW_TMEM = 0, 1, 2, 3
+
+
+def convrot_w4a16_debug_gemm_form(xr, qw, sw, bias, form: int, out=None, stream=None,
+                                  N: int | None = None):
+    """convrot_w4a16_linear_prepared with the GEMM forced to one form
+    (W4A16_*); form | TILES_REPACKED takes qw in the repacked layout (a flat
+    tensor; give N then)."""
+    M, K = _rows(xr, torch.bfloat16, "xr")
+    if form & TILES_REPACKED:
+        if N is None:
+            raise ValueError("N is needed with repacked weights")
+        _need(qw, torch.uint8, "qw_rep", (convrot_repacked_weight_size(N, K),), xr)
+        _need(sw, torch.float32, "sw", (N,), xr)
+        _need_opt(bias, torch.bfloat16, "bias", (N,), xr)
+    else:
+        N = _weights(qw, sw, bias, K, xr)
+    with torch.cuda.device(xr.device):
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=xr.device) if out is None else out
+        _need(out, torch.bfloat16, "out", (M, N), xr)
+        _check(lib_w4a16().convrot_w4a16_debug_gemm_form(_p(xr), _p(qw), _p(sw), _p(bias), M, N, K,
+                                                         int(form), _p(out), _stream(stream)),
+               "convrot_w4a16_debug_gemm_form")
     return out
 
 

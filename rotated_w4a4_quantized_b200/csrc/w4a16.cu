@@ -514,6 +514,301 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     }
 }
 
+
+// ------------------------------------------------ few tokens, weights in TMEM
+// The few-token form of the W4A4 skinny kernel, for bf16 tokens: the packed
+// weights are widened to bf16 straight into TMEM (the MMA's A operand,
+// 128 lanes = weight rows), so a weight byte is written once by TMA and
+// read once from shared memory; the rotated tokens xr are already bf16 and
+// go by TMA straight into the 128-byte swizzled K-major layout of the MMA's
+// B operand.  CTA i owns weight rows [i R, i R + R) over the whole of K
+// (R spreads N over the SMs): one wave, no split K.  A stage is 256 codes:
+// 128 packed bytes per weight row, four 64-deep xr K-blocks.
+//
+// CTA organisation (12 warps):
+//   warp 0      weight TMA producer (one thread), a ring as deep as shared
+//               memory allows; in the whole-layer call the first stages are
+//               requested before waiting for the rotation kernel;
+//   warp 2      token TMA producer (one thread), a ring of three;
+//   warp 1      TMEM allocator and MMA issuer: 16 MMAs of K = 16 per stage,
+//               A from TMEM, B from shared memory;
+//   warps 4..11 weight widening, two warps per TMEM lane quarter (thread =
+//               weight row = TMEM lane; warp 4 + q takes codes 0..127 of
+//               each stage, warp 8 + q codes 128..255), then the epilogue
+//               (lane = output column, accumulator columns = tokens).
+// Widening: packed chunk p of row r arrives at p ^ (r & 7) (128-byte
+// swizzle); its 32 codes become 16 bf16 pairs in natural K order
+// (widen_word), TMEM columns 16 p .. 16 p + 15 of the stage.
+namespace sk {
+
+constexpr int kWarpTmaW = 0, kWarpMma = 1, kWarpTmaX = 2, kWarpW0 = 4, kWidenWarps = 8;
+constexpr int kThreads = (kWarpW0 + kWidenWarps) * 32;   // 384
+constexpr int kMaxRows = 128;          // weight rows per CTA: the TMEM lanes
+constexpr int kPKB = 128;              // packed weight bytes per row per stage (256 codes)
+constexpr int kXKB = 4;                // 64-deep xr K-blocks per stage
+constexpr int kSU = 3;                 // TMEM A stages
+constexpr int kSX = 3;                 // token stages (from L2)
+
+template <int BN>
+struct Cfg {
+    static_assert(BN == 16 || BN == 32 || BN == 64, "token tile of 16, 32 or 64");
+    static constexpr int XKB = BN * 128;                 // one xr K-block tile (BN rows x 64 bf16)
+    static constexpr int XST = kXKB * XKB;               // token stage
+    static constexpr int PA = kMaxRows * kPKB;           // weight stage (up to 128 rows)
+    static constexpr int SP_FIT = (232448 - (kSX * XST + 2048)) / PA;
+    static constexpr int SP = SP_FIT > 12 ? 12 : SP_FIT;
+    static_assert(SP >= 3, "at least three weight stages in flight");
+    static constexpr int OFF_X = 0;                      // 1024-aligned tiles first
+    static constexpr int OFF_PA = OFF_X + kSX * XST;
+    static constexpr int OFF_BAR = OFF_PA + SP * PA;
+    static constexpr int NUM_BARS = 2 * SP + 2 * kSX + 2 * kSU + 1;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;     // TMEM base, abort flag
+    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;    // + slack for 1024 alignment
+    static constexpr int ACC_COLS = BN < 32 ? 32 : BN;         // read 32 columns at a time
+    static constexpr int A_COLS = kPKB;                        // 256 bf16 = 128 columns
+    static constexpr int A_OFF = ACC_COLS;
+    static constexpr int TMEM_NEED = A_OFF + kSU * A_COLS;
+    static constexpr int TMEM_COLS = TMEM_NEED <= 256 ? 256 : 512;
+    static_assert(TMEM_NEED <= 512, "TMEM holds 512 columns");
+    static_assert(XKB % 1024 == 0 && PA % 1024 == 0, "swizzled tiles stay 1024-aligned");
+    static_assert(SMEM_BYTES <= 232448, "exceeds the per-CTA shared memory limit");
+};
+
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, bf16 x bf16 -> f32, K = 16: A holds
+// 8 columns (16 bf16, two per column, low half first) of each of 128 lanes.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// tmX: xr bf16 [M][K], box 64 x BN, 128-byte swizzle.  tmW: qw u8 [N][K/2],
+// box 128 B x R rows, 128-byte swizzle (3-D over the repacked layout when
+// wrep).  early_w: the weights were complete before the preceding kernel on
+// the stream started.  K % 64 == 0; K tails past a stage read zeros.
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+w4a16_skinny_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                    int R, int early_w, int M, int N, int K, int wrep, const float *__restrict__ sw,
+                    const uint16_t *__restrict__ bias, uint16_t *__restrict__ y) {
+    using C = Cfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = ptx::smem_u32(smem);
+    const uint32_t bar0 = sbase + C::OFF_BAR;
+    auto full_a = [&](int s) { return bar0 + 8u * s; };                  // weight stages
+    auto empty_a = [&](int s) { return bar0 + 8u * (C::SP + s); };
+    auto full_x = [&](int s) { return bar0 + 8u * (2 * C::SP + s); };    // token stages
+    auto empty_x = [&](int s) { return bar0 + 8u * (2 * C::SP + kSX + s); };
+    const uint32_t bar_u = bar0 + 8u * (2 * C::SP + 2 * kSX);
+    auto full_u = [&](int s) { return bar_u + 8u * s; };                 // TMEM A stages
+    auto empty_u = [&](int s) { return bar_u + 8u * (kSU + s); };
+    const uint32_t acc_full = bar_u + 8u * (2 * kSU);
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = static_cast<int>(blockIdx.x) * R;      // first weight row of this CTA
+    const int num_kp = (K / 2 + kPKB - 1) / kPKB;         // stages
+    const uint32_t a_tx = static_cast<uint32_t>(R * kPKB);
+
+    const int early = early_w ? (num_kp < C::SP ? num_kp : C::SP) : 0;
+    if (threadIdx.x == 0) {
+        ptx::tma_prefetch_desc(&tmX);
+        ptx::tma_prefetch_desc(&tmW);
+        for (int s = 0; s < C::SP; ++s) {
+            ptx::mbar_init(full_a(s), 1);
+            ptx::mbar_init(empty_a(s), kWidenWarps);
+        }
+        for (int s = 0; s < kSX; ++s) {
+            ptx::mbar_init(full_x(s), 1);
+            ptx::mbar_init(empty_x(s), 1);     // the MMAs read the tokens in place
+        }
+        for (int s = 0; s < kSU; ++s) {
+            ptx::mbar_init(full_u(s), kWidenWarps);
+            ptx::mbar_init(empty_u(s), 1);
+        }
+        ptx::mbar_init(acc_full, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+        for (int kp = 0; kp < early; ++kp) {
+            ptx::mbar_arrive_expect_tx(full_a(kp), a_tx);
+            ptx::tma_load_rows(sbase + C::OFF_PA + kp * C::PA, &tmW, full_a(kp), kp * kPKB, n0, wrep);
+        }
+    }
+    if (warp == kWarpMma) {
+        ptx::tmem_alloc<1>(sbase + C::OFF_MISC, C::TMEM_COLS);
+        ptx::tmem_relinquish<1>();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    // Let a producer's copies already in flight land before the CTA exits:
+    // `issued` stages went into a ring of S slots.
+    auto drain = [&](auto full, int issued, int S) {
+        const int ps = issued % S;
+        const uint32_t ph = static_cast<uint32_t>(issued / S) & 1u;
+        for (int s = 0; s < S; ++s) {
+            volatile int never = 0;
+            ptx::mbar_wait(full(s), ph ^ (s < ps ? 0u : 1u), &never, 10000000ull);
+        }
+    };
+
+    if (warp == kWarpTmaW) {
+        if (lane == 0) {
+            if (!early_w) ptx::grid_dependency_wait();
+            int kp = early;
+            for (; kp < num_kp; ++kp) {
+                const int s = kp % C::SP;
+                if (!ptx::mbar_wait(empty_a(s), ((kp / C::SP) & 1) ^ 1, abort_flag)) break;
+                ptx::mbar_arrive_expect_tx(full_a(s), a_tx);
+                ptx::tma_load_rows(sbase + C::OFF_PA + s * C::PA, &tmW, full_a(s), kp * kPKB, n0, wrep);
+            }
+            if (kp < num_kp) drain(full_a, kp, C::SP);
+        }
+    } else if (warp == kWarpTmaX) {
+        if (lane == 0) {
+            ptx::grid_dependency_wait();   // xr comes from the preceding kernel
+            int kp = 0;
+            for (; kp < num_kp; ++kp) {
+                const int s = kp % kSX;
+                if (!ptx::mbar_wait(empty_x(s), ((kp / kSX) & 1) ^ 1, abort_flag)) break;
+                ptx::mbar_arrive_expect_tx(full_x(s), static_cast<uint32_t>(C::XST));
+#pragma unroll
+                for (int i = 0; i < kXKB; ++i)   // K-blocks past K arrive as zeros
+                    ptx::tma_load_2d(sbase + C::OFF_X + s * C::XST + i * C::XKB, &tmX, full_x(s),
+                                     (kp * kXKB + i) * KB, 0);
+            }
+            if (kp < num_kp) drain(full_x, kp, kSX);
+        }
+    } else if (warp == kWarpMma) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(128, BN);
+            int us = 0, xs = 0;
+            uint32_t uph = 0, xph = 0;
+            for (int kp = 0; kp < num_kp; ++kp) {
+                if (!ptx::mbar_wait(full_u(us), uph, abort_flag)) break;
+                if (!ptx::mbar_wait(full_x(xs), xph, abort_flag)) break;
+                ptx::tc_fence_after();
+                const uint32_t a0 = tmem_base + static_cast<uint32_t>(C::A_OFF + us * C::A_COLS);
+                const uint32_t x0 = sbase + C::OFF_X + xs * C::XST;
+#pragma unroll
+                for (int j = 0; j < kXKB * KB / 16; ++j)   // A stage: 8 columns per MMA
+                    mma_bf16_ts(tmem_base, a0 + static_cast<uint32_t>(8 * j),
+                                ptx::sw128_kmajor_desc(x0 + (j >> 2) * C::XKB + 32 * (j & 3)), idesc,
+                                (kp | j) != 0 ? 1u : 0u);
+                ptx::tc_commit<1>(empty_u(us));
+                ptx::tc_commit<1>(empty_x(xs));
+                if (++us == kSU) { us = 0; uph ^= 1; }
+                if (++xs == kSX) { xs = 0; xph ^= 1; }
+            }
+            // Also the drain: TMEM is released only after every MMA completed.
+            ptx::tc_commit<1>(acc_full);
+            volatile int never = 0;
+            ptx::mbar_wait(acc_full, 0, &never, 100000000ull);
+        }
+    } else if (warp >= kWarpW0) {
+        const int quarter = warp & 3;                  // TMEM lanes 32 quarter ..
+        const int hh = (warp - kWarpW0) >> 2;          // which 128 codes of a stage
+        const int r = quarter * 32 + lane;
+        const bool live = r < R;
+        const uint32_t rsw = static_cast<uint32_t>(r & 7);
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+        // ------------------------------------------------- weight widening
+        for (int kp = 0; kp < num_kp; ++kp) {
+            const int ps = kp % C::SP, us = kp % kSU;
+            const uint32_t pph = (kp / C::SP) & 1, uph = (kp / kSU) & 1;
+            if (!ptx::mbar_wait(full_a(ps), pph, abort_flag)) break;
+            if (!ptx::mbar_wait(empty_u(us), uph ^ 1, abort_flag)) break;
+            ptx::tc_fence_after();
+            const uint32_t src = sbase + C::OFF_PA + ps * C::PA + r * kPKB;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t t[32];
+                if (live) {
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const uint32_t chunk = static_cast<uint32_t>(4 * hh + 2 * half + cc) ^ rsw;
+                        const uint4 w = lds128(src + (chunk << 4));
+                        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) {
+                            uint32_t o[4];
+                            widen_word(wv[x], o);
+#pragma unroll
+                            for (int z = 0; z < 4; ++z) t[16 * cc + 4 * x + z] = o[z];
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) t[i] = 0u;
+                }
+                __syncwarp();   // tcgen05.st is warp-collective
+                ptx::tmem_st_32x32b_x32(
+                    lane_base + static_cast<uint32_t>(C::A_OFF + us * C::A_COLS + 64 * hh + 32 * half), t);
+            }
+            ptx::tmem_st_wait();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                ptx::mbar_arrive(empty_a(ps));
+                ptx::mbar_arrive(full_u(us));
+            }
+        }
+        // --------------------------------------------------------- epilogue
+        // lane = output column n (a weight row), accumulator columns =
+        // tokens; with 64 tokens the two warps of a quarter take 32 each.
+        const bool active = BN >= 64 || hh == 0;
+        if (active && !*abort_flag && ptx::mbar_wait(acc_full, 0, abort_flag)) {
+            ptx::tc_fence_after();
+            const int n = n0 + r;
+            const bool store = live && n < N;
+            const float swn = store ? sw[n] : 0.0f;
+            const float bn = (store && bias) ? __uint_as_float(static_cast<uint32_t>(bias[n]) << 16) : 0.0f;
+            const int c0 = 32 * hh;
+            uint32_t v[32];
+            __syncwarp();   // tcgen05.ld is warp-collective
+            ptx::tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(c0), v);
+            ptx::tmem_ld_wait();
+            constexpr int JW = BN < 32 ? BN : 32;
+            if (store) {
+#pragma unroll
+                for (int j = 0; j < JW; ++j) {
+                    const int m = c0 + j;
+                    if (m < M)
+                        y[static_cast<size_t>(m) * N + n] = static_cast<uint16_t>(
+                            bf16x2_rn(__fadd_rn(__fmul_rn(__uint_as_float(v[j]), swn), bn), 0.0f));
+                }
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == kWarpMma) {
+        __syncwarp();
+        ptx::tmem_dealloc<1>(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// Weight rows per CTA for N output columns on num_sms SMs (a multiple of 8,
+// at most 128).
+inline int rows_per_cta(int64_t N, int num_sms) {
+    int64_t r = (N + num_sms - 1) / num_sms;
+    r = (r + 7) / 8 * 8;
+    return static_cast<int>(r < 8 ? 8 : r > kMaxRows ? kMaxRows : r);
+}
+
+}  // namespace sk
+
 }  // namespace w4a16
 
 // ====================================================================== host
@@ -588,6 +883,9 @@ convrot_status device_setup(int *dev_out) {
     ok &= set_smem(w4a16::w4a16_gemm_kernel<16, true>, w4a16::Cfg<16, true>::SMEM_BYTES);
     ok &= set_smem(w4a16::w4a16_gemm_kernel<32, true>, w4a16::Cfg<32, true>::SMEM_BYTES);
     ok &= set_smem(w4a16::w4a16_gemm_kernel<64, true>, w4a16::Cfg<64, true>::SMEM_BYTES);
+    ok &= set_smem(w4a16::sk::w4a16_skinny_kernel<16>, w4a16::sk::Cfg<16>::SMEM_BYTES);
+    ok &= set_smem(w4a16::sk::w4a16_skinny_kernel<32>, w4a16::sk::Cfg<32>::SMEM_BYTES);
+    ok &= set_smem(w4a16::sk::w4a16_skinny_kernel<64>, w4a16::sk::Cfg<64>::SMEM_BYTES);
     st.num_sms = sms;
     st.status = ok ? CONVROT_OK : CONVROT_ERR_CUDA;
     st.ready.store(true, std::memory_order_release);
@@ -730,15 +1028,99 @@ convrot_status launch_gemm_cfg(int num_sms, const void *xr, const uint8_t *qw, c
     return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 
-// Up to 64 tokens: the weights take the MMA's 128-row side and the tokens a
-// 16-, 32- or 64-wide side; beyond that, 128 x 256 token-by-weight tiles.
+// The few-token form with the weights widened into TMEM (M <= BN).
+// early_w: the weights were complete before the preceding kernel on the
+// stream started (the whole-layer call), so the kernel streams them before
+// waiting for it.
+template <int BN>
+convrot_status launch_skinny_cfg(int num_sms, const void *xr, const uint8_t *qw, const float *sw,
+                                 const void *bias, int64_t M, int64_t N, int64_t K, void *y,
+                                 cudaStream_t stream, bool wrep, bool early_w) {
+    using C = w4a16::sk::Cfg<BN>;
+    const int R = w4a16::sk::rows_per_cta(N, num_sms);
+    CUtensorMap tmX, tmW;
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(w4a16::KB), static_cast<cuuint32_t>(BN)};
+        const cuuint32_t estr[2] = {1, 1};
+        if (g_encode(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(xr), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONVROT_ERR_CUDA;
+    }
+    if (wrep) {
+        // the block-major repacked weights: {128 bytes, N rows, ceil(K/256) blocks}
+        const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(N),
+                                    static_cast<cuuint64_t>((K / 2 + 127) / 128)};
+        const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(N) * 128};
+        const cuuint32_t box[3] = {static_cast<cuuint32_t>(w4a16::sk::kPKB),
+                                   static_cast<cuuint32_t>(R), 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (g_encode(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(qw), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONVROT_ERR_CUDA;
+    } else {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(w4a16::sk::kPKB),
+                                   static_cast<cuuint32_t>(R)};
+        const cuuint32_t estr[2] = {1, 1};
+        if (g_encode(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(qw), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CONVROT_ERR_CUDA;
+    }
+    const int64_t ctas = (N + R - 1) / R;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+    cfg.blockDim = dim3(w4a16::sk::kThreads);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(
+        &cfg, w4a16::sk::w4a16_skinny_kernel<BN>, tmX, tmW, R, early_w ? 1 : 0,
+        static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), wrep ? 1 : 0, sw,
+        static_cast<const uint16_t *>(bias), static_cast<uint16_t *>(y));
+    return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
+}
+
+// GEMM forms: the automatic choice, the 128 x 256 token-by-weight tiles, and
+// the two few-token forms (M <= 64): weights widened in shared memory (the
+// 128-row tiles of w4a16_gemm_kernel) or into TMEM (w4a16_skinny_kernel).
+enum Form { kFormAuto = 0, kFormTiles = 1, kFormFewSmem = 2, kFormFewTmem = 3 };
+
+// Up to 64 tokens the few-token form with the weights in TMEM; beyond
+// that, 128 x 256 token-by-weight tiles.
 convrot_status launch_gemm(int num_sms, const void *xr, const uint8_t *qw, const float *sw,
                            const void *bias, int64_t M, int64_t N, int64_t K, void *y,
-                           cudaStream_t stream, bool wrep = false) {
-    if (M <= 16) return launch_gemm_cfg<16, true>(num_sms, xr, qw, sw, bias, M, N, K, y, stream, wrep);
-    if (M <= 32) return launch_gemm_cfg<32, true>(num_sms, xr, qw, sw, bias, M, N, K, y, stream, wrep);
-    if (M <= 64) return launch_gemm_cfg<64, true>(num_sms, xr, qw, sw, bias, M, N, K, y, stream, wrep);
-    return launch_gemm_cfg<128, false>(num_sms, xr, qw, sw, bias, M, N, K, y, stream, wrep);
+                           cudaStream_t stream, bool wrep = false, bool early_w = false,
+                           int form = kFormAuto) {
+    if (form == kFormAuto) form = M <= 64 ? kFormFewTmem : kFormTiles;
+    if ((form == kFormFewSmem || form == kFormFewTmem) && M > 64) return CONVROT_ERR_SHAPE;
+    if (form == kFormFewTmem) {
+        if (M <= 16)
+            return launch_skinny_cfg<16>(num_sms, xr, qw, sw, bias, M, N, K, y, stream, wrep, early_w);
+        if (M <= 32)
+            return launch_skinny_cfg<32>(num_sms, xr, qw, sw, bias, M, N, K, y, stream, wrep, early_w);
+        return launch_skinny_cfg<64>(num_sms, xr, qw, sw, bias, M, N, K, y, stream, wrep, early_w);
+    }
+    if (form == kFormFewSmem) {
+        if (M <= 16) return launch_gemm_cfg<16, true>(num_sms, xr, qw, sw, bias, M, N, K, y, stream, wrep);
+        if (M <= 32) return launch_gemm_cfg<32, true>(num_sms, xr, qw, sw, bias, M, N, K, y, stream, wrep);
+        return launch_gemm_cfg<64, true>(num_sms, xr, qw, sw, bias, M, N, K, y, stream, wrep);
+    }
+    if (form == kFormTiles)
+        return launch_gemm_cfg<128, false>(num_sms, xr, qw, sw, bias, M, N, K, y, stream, wrep);
+    return CONVROT_ERR_SHAPE;
 }
 
 }  // namespace
@@ -766,7 +1148,7 @@ size_t convrot_w4a16_workspace_size(int64_t M, int64_t K) {
 static convrot_status linear_prepared_impl(const void *xr_bf16, const uint8_t *qw,
                                            const float *sw, const void *bias_bf16, int64_t M,
                                            int64_t N, int64_t K, void *y_bf16,
-                                           cudaStream_t stream, bool wrep) {
+                                           cudaStream_t stream, bool wrep, int form = kFormAuto) {
     convrot_status st = check_gemm_shape(M, N, K);
     if (st != CONVROT_OK) return st;
     if (M == 0 || N == 0) return CONVROT_OK;
@@ -778,7 +1160,7 @@ static convrot_status linear_prepared_impl(const void *xr_bf16, const uint8_t *q
     if ((st = device_setup(&dev)) != CONVROT_OK) return st;
     if ((st = check_device_ptrs(dev, {xr_bf16, qw, sw, bias_bf16, y_bf16})) != CONVROT_OK) return st;
     return launch_gemm(g_dev[dev].num_sms, xr_bf16, qw, sw, bias_bf16, M, N, K, y_bf16, stream,
-                       wrep);
+                       wrep, false, form);
 }
 
 static convrot_status linear_impl(const void *x_bf16, const uint8_t *qw, const float *sw,
@@ -803,8 +1185,9 @@ static convrot_status linear_impl(const void *x_bf16, const uint8_t *qw, const f
     if ((st = launch_rotate(g_dev[dev].num_sms, x_bf16, M, K, group, workspace, stream)) !=
         CONVROT_OK)
         return st;
+    // the weights were complete before the rotation kernel started
     return launch_gemm(g_dev[dev].num_sms, workspace, qw, sw, bias_bf16, M, N, K, y_bf16, stream,
-                       wrep);
+                       wrep, true);
 }
 
 convrot_status convrot_w4a16_linear_prepared(const void *xr_bf16, const uint8_t *qw,
@@ -836,6 +1219,17 @@ convrot_status convrot_w4a16_linear_repacked(const void *x_bf16, const uint8_t *
                                              convrot_stream_t stream) {
     return linear_impl(x_bf16, qw_rep, sw, bias_bf16, M, N, K, group, workspace, ws_bytes, y_bf16,
                        stream, true);
+}
+
+convrot_status convrot_w4a16_debug_gemm_form(const void *xr_bf16, const uint8_t *qw,
+                                             const float *sw, const void *bias_bf16, int64_t M,
+                                             int64_t N, int64_t K, int form, void *y_bf16,
+                                             convrot_stream_t stream) {
+    const bool wrep = (form & CONVROT_TILES_REPACKED) != 0;
+    form &= ~CONVROT_TILES_REPACKED;
+    if (form < kFormAuto || form > kFormFewTmem) return CONVROT_ERR_SHAPE;
+    if ((form == kFormFewSmem || form == kFormFewTmem) && M > 64) return CONVROT_ERR_SHAPE;
+    return linear_prepared_impl(xr_bf16, qw, sw, bias_bf16, M, N, K, y_bf16, stream, wrep, form);
 }
 
 convrot_status convrot_w4a16_check_device_error(convrot_stream_t stream) {

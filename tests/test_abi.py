@@ -187,7 +187,7 @@ def test_w4a16_header_declares_the_boundary():
         "convrot_w4a16_prepare_act", "convrot_w4a16_workspace_size",
         "convrot_w4a16_linear_prepared", "convrot_w4a16_linear",
         "convrot_w4a16_check_device_error", "convrot_w4a16_linear_repacked",
-        "convrot_w4a16_linear_prepared_repacked"])
+        "convrot_w4a16_linear_prepared_repacked", "convrot_w4a16_debug_gemm_form"])
 
 
 def test_w4a16_library_exports_every_declared_symbol(L16):
@@ -224,6 +224,15 @@ def test_w4a16_host_validation_without_device(L16):
     assert L16.convrot_w4a16_linear(A, B, B, None, 4, 8, 1024, 64, U, ws, B, s) == 5
     assert L16.convrot_w4a16_linear(A, B, B, None, 4, 8, 1024, 32, A, ws, B, s) == 2
     assert L16.convrot_w4a16_linear(None, None, None, None, 4, 0, 1024, 64, None, 0, None, s) == 0
+    # forced GEMM forms: 0..3 (| repacked), the few-token forms up to 64 tokens
+    f = L16.convrot_w4a16_debug_gemm_form
+    assert f(A, B, B, None, 4, 8, 1024, 4, B, s) == 3
+    assert f(A, B, B, None, 4, 8, 1024, -1, B, s) == 3
+    assert f(A, B, B, None, 65, 8, 1024, 2, B, s) == 3
+    assert f(A, B, B, None, 65, 8, 1024, 3 | 0x100, B, s) == 3
+    assert f(A, B, B, None, 4, 8, 96, 3, B, s) == 3                    # K % 64
+    assert f(A, None, B, None, 4, 8, 1024, 3, B, s) == 1
+    assert f(A, B, B, U, 4, 8, 1024, 3, B, s) == 4
 
 
 def test_w4a16_valid_call_without_gpu_reports_cuda_error(L16):

@@ -125,3 +125,10 @@ def test_w4a16_on_repacked_weights(M, K, N):
     torch.cuda.synchronize()
     assert cr.convrot_w4a16_check_device_error() == 0
     assert _eq16(y, yr) and _eq16(y, yp)
+    # every form that runs this shape, forced, on both layouts
+    forms = [cr.W4A16_TILES] + ([cr.W4A16_FEW_SMEM, cr.W4A16_FEW_TMEM] if M <= 64 else [])
+    for form in forms:
+        yc = cr.convrot_w4a16_debug_gemm_form(xr, qw, sw, b, form)
+        yf = cr.convrot_w4a16_debug_gemm_form(xr, rep, sw, b, form | cr.TILES_REPACKED, N=N)
+        torch.cuda.synchronize()
+        assert _eq16(yc, yf), form

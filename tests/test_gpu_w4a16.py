@@ -97,6 +97,42 @@ def test_w4a16_gemm_matches_oracle(M, N, K, bias):
     gc.check_w4a16_outputs(gc.to_np_u16(y), t, acc, l1, p16, sw)
 
 
+# The two few-token forms, each forced: weights widened to bf16 in shared
+# memory (form 2) or straight into TMEM (form 3), with token counts at and
+# around the 16 / 32 / 64 tile widths, slices of weight rows with a ragged
+# last slice, K tails inside a 256-code stage (K = 64, 192, 1088) and
+# stages whose xr K-blocks lie past K.
+FEW_CASES = [(1, 16, 64, True), (1, 14336, 4096, False), (3, 1000, 192, True),
+             (16, 777, 1088, False), (17, 300, 2048, True), (32, 4000, 3072, False),
+             (33, 130, 320, True), (64, 1024, 4096, True), (50, 9, 12288, False)]
+
+
+@pytest.mark.parametrize("form", [cr.W4A16_FEW_SMEM, cr.W4A16_FEW_TMEM], ids=["smem", "tmem"])
+@pytest.mark.parametrize("M,N,K,bias", FEW_CASES)
+def test_w4a16_few_token_forms_match_oracle(form, M, N, K, bias):
+    lt = wl.make_random_layer(M, K, N, 64, seed=7 * M + N + K, bias=bias)
+    xb, wb = wl.bf16_bits(lt.x), wl.bf16_bits(lt.w)
+    bb = None if lt.b is None else wl.bf16_bits(lt.b)
+    pw, sw = O.prepare_rows(wb, 64)
+    y = cr.convrot_w4a16_debug_gemm_form(
+        lt.x.cuda(), torch.from_numpy(pw).cuda(), torch.from_numpy(sw).cuda(),
+        None if lt.b is None else lt.b.cuda(), form)
+    torch.cuda.synchronize()
+    assert cr.convrot_w4a16_check_device_error() == 0
+    acc, l1, p16 = O.w4a16_gemm(xb, pw, K)
+    t, _ = O.w4a16_epilogue(acc, sw, bb)
+    gc.check_w4a16_outputs(gc.to_np_u16(y), t, acc, l1, p16, sw)
+
+
+def test_w4a16_forms_refuse_what_they_cannot_run():
+    lt = wl.make_random_layer(65, 256, 32, 64, seed=3)
+    qw, sw = cr.convrot_quantize_weight(lt.w.cuda(), 64)
+    for form in (cr.W4A16_FEW_SMEM, cr.W4A16_FEW_TMEM, 4):
+        with pytest.raises(cr.ConvRotError) as e:
+            cr.convrot_w4a16_debug_gemm_form(lt.x.cuda(), qw, sw, None, form)
+        assert e.value.status == 3
+
+
 def test_w4a16_zero_rows_give_exactly_the_bias():
     M, N, K = 140, 96, 512
     lt = wl.make_random_layer(M, K, N, 64, seed=9)
