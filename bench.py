@@ -501,8 +501,14 @@ class W4A16Variant:
     """bf16 activations x the W4A4 packed weights (include/convrot_w4a16.h)."""
     name, metric, dtype = "w4a16", METRIC_W4A16, "bf16"
     peak_ratio, peak_note = 1.0, "measured bf16 burst"
-    prep_kernel, gemm_kernel = "rotate_bf16_kernel", "w4a16_gemm_kernel"
+    prep_kernel = "rotate_bf16_kernel"
     prep_bytes = staticmethod(ROT16_BYTES)
+
+    @staticmethod
+    def gemm_kernel_for(sp):
+        # up to 64 tokens the few-token form with the weights widened into TMEM
+        return "w4a16_skinny_kernel" if sp.M <= 64 else "w4a16_gemm_kernel"
+
     gemm_bytes = staticmethod(GEMM16_BYTES)
     prep_desc = "algorithmic bytes 4MK"
     gemm_desc = "2MK (xr) + NK/2 + 4N + 2N + 2MN"
@@ -538,8 +544,13 @@ class NVFP4Variant:
     name, metric, dtype = "nvfp4", METRIC_NVFP4, "e2m1"
     peak_ratio = FP4_PER_BF16
     peak_note = f"measured bf16 burst x {FP4_PER_BF16} nominal fp4/bf16 ratio"
-    prep_kernel, gemm_kernel = "quant_kernel", "nvfp4_gemm_kernel"
+    prep_kernel = "quant_kernel"
     prep_bytes = staticmethod(FP4_QUANT_BYTES)
+
+    @staticmethod
+    def gemm_kernel_for(sp):
+        return "nvfp4_gemm_kernel"
+
     gemm_bytes = staticmethod(FP4_GEMM_BYTES)
     prep_desc = "algorithmic bytes 2MK + MK/2 + MK/16 + 4M"
     gemm_desc = "(M+N)(K/2 + K/16 + 4) + 2N + 2MN"
@@ -732,12 +743,12 @@ def run_gpu_variant(args, V):
         t_tensor = 2 * sp.M * sp.N * sp.K / (tensor_peak * 1e12)
         t_bytes = V.gemm_bytes(sp.M, sp.N, sp.K) / (peaks["hbm"] * 1e9)
         if t_tensor >= t_bytes:
-            roof = {"kernel": V.gemm_kernel, "bound": "tensor", "achieved": round(gemm_tf[i], 2),
+            roof = {"kernel": V.gemm_kernel_for(sp), "bound": "tensor", "achieved": round(gemm_tf[i], 2),
                     "peak": round(tensor_peak, 1), "unit": "TFLOP/s",
                     "frac": round(gemm_tf[i] / tensor_peak, 4), "traffic": None,
                     "note": f"tensor ops (2 per multiply-add); peak = {V.peak_note} ({peaks['src']})"}
         else:
-            roof = {"kernel": V.gemm_kernel, "bound": "hbm", "achieved": round(gemm_gbs[i], 1),
+            roof = {"kernel": V.gemm_kernel_for(sp), "bound": "hbm", "achieved": round(gemm_gbs[i], 1),
                     "peak": peaks["hbm"], "unit": "GB/s", "frac": round(gemm_gbs[i] / peaks["hbm"], 4),
                     "traffic": None,
                     "note": f"algorithmic bytes {V.gemm_desc}; HBM peak {peaks['src']}"}
