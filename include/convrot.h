@@ -256,6 +256,22 @@ convrot_status convrot_debug_gemm_tiles(const uint8_t *qx, const float *sx, cons
                                         convrot_stream_t stream);
 
 /*
+ * Test hook, host-only (no device work): the GEMM form and split-K plan
+ * convrot_linear chooses for (M, N, K) on a device with `pairs` co-resident
+ * CTA pairs (0: none) and `sms` SMs, given a split area of split_bytes
+ * (0: none).  *tiles is the form as numbered for convrot_debug_gemm_tiles
+ * (4 for the few-token form, M <= 128); the first *split_tiles output tiles
+ * are cut into *splits ranges of K (0 and 1: no split).  CONVROT_ERR_NULL
+ * for a NULL output, CONVROT_ERR_SHAPE for K outside 64 .. CONVROT_MAX_K or
+ * not a multiple of 64, negative sizes, pairs < 0 or sms <= 0.  Exposes the
+ * scheduling of step 3 ("convrot-mlx" README, "Install and test": the
+ * integer product), which changes no result.
+ */
+convrot_status convrot_debug_gemm_plan(int64_t M, int64_t N, int64_t K, int pairs, int sms,
+                                       size_t split_bytes, int *tiles, int *split_tiles,
+                                       int *splits);
+
+/*
  * Test hook: convrot_debug_gemm_tiles for a token-major form (tiles 0-3 or
  * 6, optionally | CONVROT_TILES_REPACKED) with a given split-K plan: the
  * first split_tiles output tiles (tile t covers rows (t mod TA) x TM and

@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
             "convrot_linear_prepared_repacked": [P, P, P, P, P, I64, I64, I64, P, P],
             "convrot_linear_prepared_split": [P, P, P, P, P, I64, I64, I64, P, SZ, P, P],
             "convrot_debug_gemm_split": [P, P, P, P, P, I64, I64, I64, I, I, I, P, SZ, I, P, P],
+            "convrot_debug_gemm_plan": [I64, I64, I64, I, I, SZ, P, P, P],
         }
         for name, args in sigs.items():
             f = getattr(L, name)
@@ -826,3 +827,16 @@ def convrot_debug_gemm_split(qx, sx, qw, sw, bias, K: int, tiles: int, split_til
                                               int(bool(out_s32)), _p(out), _stream(stream)),
                "convrot_debug_gemm_split")
     return out
+
+
+def convrot_debug_gemm_plan(M: int, N: int, K: int, pairs: int = 74, sms: int = 148,
+                            split_bytes: int | None = None):
+    """Host-only: the GEMM form (numbered as for convrot_debug_gemm_tiles) and
+    split-K plan (split_tiles, splits) convrot_linear takes for (M, N, K) on a
+    device with `pairs` CTA pairs and `sms` SMs (a B200: 74 and 148)."""
+    t, st, sp = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    nb = SPLIT_AREA_BYTES if split_bytes is None else split_bytes
+    _check(lib().convrot_debug_gemm_plan(M, N, K, pairs, sms, nb, ctypes.byref(t),
+                                         ctypes.byref(st), ctypes.byref(sp)),
+           "convrot_debug_gemm_plan")
+    return t.value, st.value, sp.value

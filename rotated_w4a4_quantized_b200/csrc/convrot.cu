@@ -458,12 +458,14 @@ struct SplitArea {
     int force_splits = 1;
 };
 
-// Partial slots (one per split unit and CTA) of BM x BN int32 that fit.
-int64_t split_capacity(const SplitArea &a, int BN) {
-    if (!a.ws || a.bytes < CONVROT_SPLIT_COUNTER_BYTES) return 0;
-    return static_cast<int64_t>((a.bytes - CONVROT_SPLIT_COUNTER_BYTES) /
+// Partial slots (one per split unit and CTA) of BM x BN int32 that fit in
+// a split area of `bytes` (0: no area).
+int64_t split_capacity(size_t bytes, int BN) {
+    if (bytes < CONVROT_SPLIT_COUNTER_BYTES) return 0;
+    return static_cast<int64_t>((bytes - CONVROT_SPLIT_COUNTER_BYTES) /
                                 (static_cast<size_t>(gemm::BM) * BN * 4));
 }
+int64_t split_capacity(const SplitArea &a, int BN) { return a.ws ? split_capacity(a.bytes, BN) : 0; }
 
 // The planner: `tiles` output tiles (BM x bn int32 accumulators per CTA) of
 // `num_kp` packed K-stages each on `slots` CTAs (pairs of cg CTAs).  Whole
@@ -484,6 +486,10 @@ struct SplitPlan {
 SplitPlan plan_split(int64_t tiles, int64_t slots, int64_t num_kp, int64_t capacity, int cg,
                      int bn) {
     SplitPlan p;
+    if (slots <= 0) {   // no co-resident CTAs of this form: one tile after another
+        p.cost = tiles * num_kp;
+        return p;
+    }
     const int64_t full = tiles / slots, rem = tiles % slots;
     p.cost = (full + (rem ? 1 : 0)) * num_kp;
     if (rem == 0 || capacity <= 0 || rem * cg * gemm::kEpiWarps > gemm::kSplitCounters) return p;
@@ -503,10 +509,67 @@ SplitPlan plan_split(int64_t tiles, int64_t slots, int64_t num_kp, int64_t capac
     return p;
 }
 
+// The token-major tile shape and split-K plan for (M, N, K) on `pairs` CTA
+// pairs (0: none) and `sms` SMs, with a split area of `area_bytes`
+// (host-only: no device needed).  tiles = kTilesAuto picks the shape.
+struct GemmPlan {
+    int tiles = kTilesAuto;
+    SplitPlan split;
+};
+
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int64_t pairs, int64_t sms, size_t area_bytes,
+                   int tiles) {
+    struct Shape {
+        int64_t ntiles, slots, num_kp, capacity;
+        int cg, bn;
+    };
+    const auto shape_of = [&](int t) {
+        const bool pair = t == kTiles256x128Pair || t == kTiles256x192Pair;
+        const int bn = (t == kTiles256x128Pair) ? 128 : (t == kTiles128x256) ? 256 : 192;
+        const int tm = pair ? 256 : 128;
+        const int pkb = (t == kTiles128x256) ? 64 : 128;
+        return Shape{((M + tm - 1) / tm) * ((N + bn - 1) / bn), pair ? pairs : sms,
+                     (K / 2 + pkb - 1) / pkb, split_capacity(area_bytes, bn), pair ? 2 : 1, bn};
+    };
+    const auto shape_plan = [&](int t) {
+        const Shape h = shape_of(t);
+        return plan_split(h.ntiles, h.slots, h.num_kp, h.capacity, h.cg, h.bn);
+    };
+    GemmPlan g;
+    g.tiles = tiles;
+    if (g.tiles == kTilesAuto) {
+        // Measured on layers of 1024-8192 tokens and K 3072-12288: the
+        // 256 x 192 pair beats both single-CTA shapes everywhere (each SM
+        // widens half of B and the tensor core reads A from TMEM).  The cost
+        // of a choice is the busiest CTA's K-stages (waves, less what split K
+        // takes off the last one) times a stage's time.
+        if (pairs > 0) {
+            // A 256 x 128 pair tile takes ~0.9 of a 256 x 192 one's time
+            // (measured on 1024-8192 tokens), so the narrower tile wins only
+            // where the 192-wide grid wastes most of a last wave that split K
+            // does not recover.
+            const int64_t c192 = shape_plan(kTiles256x192Pair).cost * 10;
+            const int64_t c128 = shape_plan(kTiles256x128Pair).cost * 9;
+            g.tiles = c128 < c192 ? kTiles256x128Pair : kTiles256x192Pair;
+        } else {
+            // a 128-code stage takes ~940 cycles on 128 x 256 tiles (both
+            // operands widened in shared memory), a 256-code stage ~1340 on
+            // 128 x 192 (A in TMEM)
+            const int64_t c_ss = shape_plan(kTiles128x256).cost * 940;
+            const int64_t c_atm = shape_plan(kTiles128x192).cost * 1340;
+            g.tiles = c_atm <= c_ss ? kTiles128x192 : kTiles128x256;
+        }
+    }
+    if (g.tiles == kTiles256x128Pair || g.tiles == kTiles256x192Pair || g.tiles == kTiles128x192 ||
+        g.tiles == kTiles128x256)
+        g.split = shape_plan(g.tiles);
+    return g;
+}
+
 // Path choice: up to 128 tokens the few-token form (weights on the 128-row
 // MMA side, widened into TMEM, one CTA per slice of weight rows); otherwise
 // tokens on the M side, with the tile shape (and split-K plan) that finishes
-// first.
+// first (plan_gemm).
 template <bool OUT_S32>
 convrot_status launch_gemm(const DeviceState &ds, const uint8_t *qx, const float *sx,
                            const uint8_t *qw, const float *sw, const void *bias, int64_t M,
@@ -538,59 +601,25 @@ convrot_status launch_gemm(const DeviceState &ds, const uint8_t *qx, const float
         return launch_gemm_cfg<128, true, OUT_S32>(num_sms, qw, qx, N, M, K, sx, sw, bias, out, M, N,
                                                    stream, wrep);
     }
-    // Token-major shapes: {BN, rows of A per tile, CTAs per tile, packed
-    // bytes per K-stage} of each choice, and its plan.
-    struct Shape {
-        int64_t ntiles, slots, num_kp, capacity;
-        int cg, bn;
-    };
-    const auto shape_of = [&](int t) {
-        const bool pair = t == kTiles256x128Pair || t == kTiles256x192Pair;
-        const int bn = (t == kTiles256x128Pair) ? 128 : (t == kTiles128x256) ? 256 : 192;
-        const int tm = pair ? 256 : 128;
-        const int pkb = (t == kTiles128x256) ? 64 : 128;
-        return Shape{((M + tm - 1) / tm) * ((N + bn - 1) / bn),
-                     pair ? static_cast<int64_t>(ds.pair_clusters) : static_cast<int64_t>(num_sms),
-                     (K / 2 + pkb - 1) / pkb, split_capacity(area, bn), pair ? 2 : 1, bn};
-    };
-    const auto shape_plan = [&](int t) {
-        const Shape h = shape_of(t);
-        return plan_split(h.ntiles, h.slots, h.num_kp, h.capacity, h.cg, h.bn);
-    };
-    if (tiles == kTilesAuto) {
-        // Measured on layers of 1024-8192 tokens and K 3072-12288: the
-        // 256 x 192 pair beats both single-CTA shapes everywhere (each SM
-        // widens half of B and the tensor core reads A from TMEM).  The cost
-        // of a choice is the busiest CTA's K-stages (waves, less what split K
-        // takes off the last one) times a stage's time.
-        if (ds.pair_clusters > 0) {
-            // A 256 x 128 pair tile takes ~0.9 of a 256 x 192 one's time
-            // (measured on 1024-8192 tokens), so the narrower tile wins only
-            // where the 192-wide grid wastes most of a last wave that split K
-            // does not recover.
-            const int64_t c192 = shape_plan(kTiles256x192Pair).cost * 10;
-            const int64_t c128 = shape_plan(kTiles256x128Pair).cost * 9;
-            tiles = c128 < c192 ? kTiles256x128Pair : kTiles256x192Pair;
-        } else {
-            // a 128-code stage takes ~940 cycles on 128 x 256 tiles (both
-            // operands widened in shared memory), a 256-code stage ~1340 on
-            // 128 x 192 (A in TMEM)
-            const int64_t c_ss = shape_plan(kTiles128x256).cost * 940;
-            const int64_t c_atm = shape_plan(kTiles128x192).cost * 1340;
-            tiles = c_atm <= c_ss ? kTiles128x192 : kTiles128x256;
-        }
-    }
-    if (tiles != kTiles256x128Pair && tiles != kTiles256x192Pair && tiles != kTiles128x192 &&
-        tiles != kTiles128x256)
+    if (tiles != kTilesAuto && tiles != kTiles256x128Pair && tiles != kTiles256x192Pair &&
+        tiles != kTiles128x192 && tiles != kTiles128x256)
         return CONVROT_ERR_SHAPE;
-    SplitPlan plan = shape_plan(tiles);
+    const GemmPlan gp = plan_gemm(M, N, K, ds.pair_clusters, num_sms, area.ws ? area.bytes : 0, tiles);
+    tiles = gp.tiles;
+    SplitPlan plan = gp.split;
     if (area.force_tiles > 0) {
         // a given plan: every part at least one K-stage, every slot and
         // counter inside the area
-        const Shape h = shape_of(tiles);
+        const bool pair = tiles == kTiles256x128Pair || tiles == kTiles256x192Pair;
+        const int bn = (tiles == kTiles256x128Pair) ? 128 : (tiles == kTiles128x256) ? 256 : 192;
+        const int tm = pair ? 256 : 128;
+        const int pkb = (tiles == kTiles128x256) ? 64 : 128;
+        const int64_t ntiles = ((M + tm - 1) / tm) * ((N + bn - 1) / bn);
+        const int64_t num_kp = (K / 2 + pkb - 1) / pkb;
+        const int64_t cg = pair ? 2 : 1;
         const int64_t ft = area.force_tiles, fs = area.force_splits;
-        if (ft > h.ntiles || fs < 2 || fs > h.num_kp || ft * h.cg * gemm::kEpiWarps > gemm::kSplitCounters ||
-            ft * fs * h.cg > h.capacity)
+        if (ft > ntiles || fs < 2 || fs > num_kp || ft * cg * gemm::kEpiWarps > gemm::kSplitCounters ||
+            ft * fs * cg > split_capacity(area, bn))
             return CONVROT_ERR_SHAPE;
         plan.split_tiles = area.force_tiles;
         plan.splits = area.force_splits;
@@ -963,6 +992,25 @@ convrot_status convrot_debug_gemm_tiles(const uint8_t *qx, const float *sx, cons
                                  tiles, false, wrep);
     return launch_gemm<false>(g_dev[dev], qx, sx, qw, sw, bias_bf16, M, N, K, out, stream, tiles,
                               false, wrep);
+}
+
+convrot_status convrot_debug_gemm_plan(int64_t M, int64_t N, int64_t K, int pairs, int sms,
+                                       size_t split_bytes, int *tiles, int *split_tiles,
+                                       int *splits) {
+    if (!tiles || !split_tiles || !splits) return CONVROT_ERR_NULL;
+    if (M < 0 || N < 0 || K < 64 || K > CONVROT_MAX_K || K % 64 || pairs < 0 || sms <= 0)
+        return CONVROT_ERR_SHAPE;
+    if (M <= kSkinnyMaxM) {   // the few-token form: one CTA per slice of weight rows
+        *tiles = kSkinnyTmem;
+        *split_tiles = 0;
+        *splits = 1;
+        return CONVROT_OK;
+    }
+    const GemmPlan g = plan_gemm(M, N, K, pairs, sms, split_bytes, kTilesAuto);
+    *tiles = g.tiles;
+    *split_tiles = g.split.split_tiles;
+    *splits = g.split.splits;
+    return CONVROT_OK;
 }
 
 convrot_status convrot_debug_gemm_split(const uint8_t *qx, const float *sx, const uint8_t *qw,
