@@ -224,7 +224,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 2-D tiled load, this CTA only (no multicast).  x is the innermost
+// 2-D tiled load into this CTA's shared memory only.  x is the innermost
 // coordinate in elements (bytes here); callers keep it a multiple of 16.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
                                             int x, int y) {
@@ -235,7 +235,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
-// 3-D tiled load, this CTA only (no multicast).  x is the innermost
+// 3-D tiled load into this CTA's shared memory only.  x is the innermost
 // coordinate in bytes; callers keep it a multiple of 16.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
                                             int x, int y, int z) {
