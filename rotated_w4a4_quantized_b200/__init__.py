@@ -804,13 +804,22 @@ class ConvRotLinear:
 
 def convrot_debug_gemm_split(qx, sx, qw, sw, bias, K: int, tiles: int, split_tiles: int,
                              splits: int, split_area, out_s32: bool = False, out=None,
-                             stream=None):
+                             stream=None, N: int | None = None):
     """convrot_debug_gemm_tiles for a token-major form with a given split-K
     plan: the first split_tiles output tiles cut into `splits` ranges of K
     (split_tiles = 0: none; -1: the planner's choice).  split_area as for
-    convrot_linear_prepared_split."""
+    convrot_linear_prepared_split; tiles | TILES_REPACKED takes qw in the
+    repacked layout (a flat tensor; give N then)."""
     M = _prepared(qx, sx, K)
-    if out_s32:
+    if tiles & TILES_REPACKED:
+        if N is None:
+            raise ValueError("N is needed with repacked weights")
+        _need(qw, torch.uint8, "qw_rep", (convrot_repacked_weight_size(N, K),), qx)
+        if not out_s32:
+            _need(sx, torch.float32, "sx", (M,), qx)
+            _need(sw, torch.float32, "sw", (N,), qx)
+            _need_opt(bias, torch.bfloat16, "bias", (N,), qx)
+    elif out_s32:
         _need(qw, torch.uint8, "qw", (None, K // 2), qx)
         N = qw.shape[0]
     else:

@@ -172,3 +172,38 @@ def test_prepared_split_area_serves_calls_in_a_row():
         torch.cuda.synchronize()
         assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16)), (M, K, N)
         assert not area[:cr.SPLIT_COUNTER_BYTES].any()
+
+
+def test_split_on_repacked_weights():
+    """Forced plans and the whole layer on repacked weights (the block-major
+    layout of include/convrot.h) against the canonical unsplit product."""
+    M, N, K = 1000, 2000, 3136
+    lt = wl.make_random_layer(M, K, N, 64, seed=31)
+    x, w, b = lt.x.cuda(), lt.w.cuda(), lt.b.cuda()
+    qw, sw = cr.convrot_quantize_weight(w, 64)
+    rep = cr.convrot_repack_weight(qw)
+    qx, sx = cr.convrot_prepare_act(x, 64)
+    area = cr.new_split_area(x.device)
+    for tiles in (cr.TILES_256x192_PAIR, cr.TILES_128x192):
+        whole = cr.convrot_debug_gemm_tiles(qx, sx, qw, sw, b, K, tiles)
+        acc = cr.convrot_debug_gemm_tiles(qx, None, qw, None, None, K, tiles, out_s32=True)
+        for st, sp in [(-1, 1), (3, 2), (5, 4)]:
+            y = cr.convrot_debug_gemm_split(qx, sx, rep, sw, b, K, tiles | cr.TILES_REPACKED, st, sp,
+                                            area, N=N)
+            a = cr.convrot_debug_gemm_split(qx, None, rep, None, None, K, tiles | cr.TILES_REPACKED,
+                                            st, sp, area, out_s32=True, N=N)
+            torch.cuda.synchronize()
+            assert torch.equal(y.view(torch.int16), whole.view(torch.int16)), (tiles, st, sp)
+            assert torch.equal(a, acc), (tiles, st, sp)
+            assert not area[:cr.SPLIT_COUNTER_BYTES].any()
+    # the whole layer on repacked weights, where the planner splits
+    M, K, N = 1536, 12288, 3072
+    lt = wl.make_random_layer(M, K, N, 256, seed=32)
+    x, w, b = lt.x.cuda(), lt.w.cuda(), lt.b.cuda()
+    qw, sw = cr.convrot_quantize_weight(w, 256)
+    rep = cr.convrot_repack_weight(qw)
+    y_can = cr.convrot_linear(x, qw, sw, b, 256)
+    y_rep = cr.convrot_linear_repacked(x, rep, sw, b, 256)
+    torch.cuda.synchronize()
+    assert cr.convrot_check_device_error() == 0
+    assert torch.equal(y_can.view(torch.int16), y_rep.view(torch.int16))
