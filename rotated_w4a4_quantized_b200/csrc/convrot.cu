@@ -90,6 +90,8 @@ convrot_status device_setup(int *dev_out) {
     ok &= set_smem(prep::prep_kernel<256, 0>, kPrepSmemMax);
     ok &= set_smem(prep::prep_kernel<64, 1>, kPrepSmemMax);
     ok &= set_smem(prep::prep_kernel<256, 1>, kPrepSmemMax);
+    ok &= set_smem(prep::prep32_kernel<256, 0>, kPrepSmemMax);
+    ok &= set_smem(prep::prep32_kernel<256, 1>, kPrepSmemMax);
     ok &= set_smem(gemm::gemm_kernel<256, false, false>, gemm::Cfg<256, false>::SMEM_BYTES);
     ok &= set_smem(gemm::gemm_kernel<256, false, true>, gemm::Cfg<256, false>::SMEM_BYTES);
     ok &= set_smem(gemm::gemm_kernel<192, false, false>, gemm::Cfg<192, false>::SMEM_BYTES);
@@ -211,6 +213,25 @@ int prep_ctas_per_sm(int group, int mode, int64_t K) {
     return slot;
 }
 
+// Resident 32-channel prep CTAs (K/32 threads, two staged rows) per SM for
+// group 256, cached (as above).
+int prep32_ctas_per_sm(int mode, int64_t K) {
+    static std::atomic<int> cache[2][1025];
+    const int T = static_cast<int>(K / 32);
+    std::atomic<int> &entry = cache[mode][T];
+    int slot = entry.load(std::memory_order_relaxed);
+    if (slot == 0) {
+        int n = 0;
+        const size_t smem = static_cast<size_t>(K) * 4;
+        const cudaError_t e =
+            mode ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, prep::prep32_kernel<256, 1>, T, smem)
+                 : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, prep::prep32_kernel<256, 0>, T, smem);
+        slot = (e == cudaSuccess && n > 0) ? n : 1;
+        entry.store(slot, std::memory_order_relaxed);
+    }
+    return slot;
+}
+
 // Resident 16-channel prep CTAs (K/16 threads) per SM, cached (as above).
 int prep16_ctas_per_sm(int group, int mode, int64_t K) {
     static std::atomic<int> cache[2][2][1025];
@@ -256,6 +277,25 @@ convrot_status launch_prep(int num_sms, const void *x, int64_t rows, int64_t K, 
             if (group == 64) prep::prep16_kernel<64, 0><<<grid16, block16, 0, stream>>>(xx, m, k, q, s, yrot, zero, nzero);
             else prep::prep16_kernel<256, 0><<<grid16, block16, 0, stream>>>(xx, m, k, q, s, yrot, zero, nzero);
         }
+        return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
+    }
+    if (group == 256 && K <= 3072) {
+        // Beyond 1024 rows of up to 3072 channels, group 256: 32 channels per
+        // thread, twice the resident warps of the 64-channel kernel.  Measured
+        // (rows x K, us, 64- against 32-channel): 4608 x 3072 13.9 / 12.9,
+        // 1536 x 3072 6.5 / 6.0, 3000 x 1024 6.1 / 4.7; on longer rows the
+        // per-row costs spread over fewer channels per thread lose:
+        // 2048 x 4096 8.4 / 8.7, 8192 x 8192 45.1 / 50.6.
+        const int64_t resident32 = static_cast<int64_t>(num_sms) * prep32_ctas_per_sm(mode, K);
+        const dim3 grid32(static_cast<unsigned>(rows < resident32 ? rows : resident32));
+        const dim3 block32(static_cast<unsigned>(K / 32));
+        const size_t smem32 = static_cast<size_t>(K) * 4;   // two staged bf16 rows
+        const uint16_t *xx = static_cast<const uint16_t *>(x);
+        const int m = static_cast<int>(rows), k = static_cast<int>(K);
+        if (yrot)
+            prep::prep32_kernel<256, 1><<<grid32, block32, smem32, stream>>>(xx, m, k, q, s, yrot, zero, nzero);
+        else
+            prep::prep32_kernel<256, 0><<<grid32, block32, smem32, stream>>>(xx, m, k, q, s, yrot, zero, nzero);
         return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
     }
     const size_t smem = prep_smem(K, group);

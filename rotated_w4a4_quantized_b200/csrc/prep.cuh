@@ -484,4 +484,200 @@ prep16_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict_
     }
 }
 
+
+// ------------------------------------------------------------------------
+// The same preparation with 32 channels per thread (K/32 threads per row),
+// for launches of many rows: half the registers of prep_kernel per thread
+// (its 64 channels need 128), so an SM holds twice the warps to hide the
+// latency of the row's dependency chains.  Thread t owns channels
+// [32t, 32t + 32): digits 0 and 1 of the rotation run in registers; digit 2
+// (stride 16) spans the thread pair t, t ^ 1, which swap the partial sums
+// x0 + x1 and x2 + x3 of each quadruple with one shuffle; for n = 256,
+// digit 3 (stride 64) spans threads t, t ^ 2, t ^ 4, t ^ 6, which exchange
+// quarters of their values through the row's stage buffer, so that digit 3
+// becomes a register stride of 8.  Every sum is formed from the same
+// operands in the same order as in prep_kernel (floating-point addition
+// commutes bitwise), so codes, scales and rotated values are bit-identical
+// to prep_kernel's.
+//
+// Shared-memory layouts (16-byte slots; thread t owns slots 4t .. 4t + 3,
+// key(t) = (t >> 1) & 3):
+//   row stage: chunk c (8 bf16) of thread t's 64 bytes at slot
+//              4t + (c ^ key(t));
+//   exchange:  in pass p, the four values 8k + 4p .. 8k + 4p + 3 of thread
+//              t at slot 4t + (k ^ key(t)).
+// Eight consecutive threads (a quarter warp) then touch eight distinct
+// slots modulo 8 in every load and store (even threads slots 0-3, odd ones
+// 4-7, each set distinct through the key): no bank conflicts.  Each thread
+// writes only its own four slots, so one warp barrier per pass suffices.
+__device__ __forceinline__ uint32_t key32(int t) { return static_cast<uint32_t>((t >> 1) & 3); }
+
+// Registers v[0..31] <- the thread's 32 channels of a staged bf16 row.
+__device__ __forceinline__ void load_row32(const uint4 *__restrict__ sb, int t, float (&v)[32]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 raw = sb[4 * t + (static_cast<uint32_t>(i) ^ key32(t))];
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+            v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+    }
+}
+
+// The unnormalised rotation of the thread's 32 channels.  On return, for
+// n = 64, v[e] is channel 32 t + e; for n = 256, v[8 d3 + q] is channel
+// 256 g + 64 d3 + 32 h + 8 j + q, with g = t / 8, h = t mod 2 and
+// j = (t / 2) mod 4 (row32_chan).
+template <int G>
+__device__ __forceinline__ void rotate_row32(float (&v)[32], float4 *__restrict__ xb, int t,
+                                             uint32_t mask) {
+    radix4_digit0(v);
+    radix4_stage<4>(v);
+    // digit 2: v[r] and v[16 + r] are x0, x1 (even thread) or x2, x3 (odd)
+#pragma unroll
+    for (int r = 0; r < 16; r += 2) {
+        float a0, a1;
+        add2(a0, a1, v[r], v[r + 1], v[r + 16], v[r + 17]);
+        const float b0 = __shfl_xor_sync(mask, a0, 1);
+        const float b1 = __shfl_xor_sync(mask, a1, 1);
+        float s0, s1;
+        add2(s0, s1, a0, a1, b0, b1);
+        bfly2(v[r], v[r + 1], s0, s1);
+        bfly2(v[r + 16], v[r + 17], s0, s1);
+    }
+    if (G == 256) {
+        const int j = (t >> 1) & 3, gb = t & ~7, h = t & 1;
+        const uint32_t kt = key32(t);
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            __syncwarp(mask);     // the group's reads of the buffer (row load or pass 0) are done
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int e = 8 * k + 4 * p;
+                xb[4 * t + (static_cast<uint32_t>(k) ^ kt)] = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+            }
+            __syncwarp(mask);
+#pragma unroll
+            for (int d3 = 0; d3 < 4; ++d3) {
+                const int w = gb + 2 * d3 + h;
+                const float4 f = xb[4 * w + (static_cast<uint32_t>(j) ^ key32(w))];
+                const int e = 8 * d3 + 4 * p;
+                v[e] = f.x;
+                v[e + 1] = f.y;
+                v[e + 2] = f.z;
+                v[e + 3] = f.w;
+            }
+        }
+        radix4_stage<8>(v);
+    }
+}
+
+// Channel of register e of thread t after rotate_row32.
+template <int G>
+__device__ __forceinline__ int row32_chan(int t, int e) {
+    if (G == 64) return t * 32 + e;
+    return (t & ~7) * 32 + 64 * (e >> 3) + 32 * (t & 1) + 8 * ((t >> 1) & 3) + (e & 7);
+}
+
+// Persistent over rows with two stage buffers, as prep_kernel for n = 256:
+// the next two rows arrive by asynchronous copies during the arithmetic,
+// and the barrier of the row maximum also frees the buffer for the row
+// after next.
+template <int G, int MODE>
+__global__ void __maxnreg__(64)
+prep32_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ q,
+              float *__restrict__ s, float *__restrict__ yrot, uint32_t *__restrict__ zero,
+              int nzero) {
+    static_assert(G == 64 || G == 256, "group 64 or 256");
+    // side job for the GEMM that follows: clear its split counters
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0u;
+    constexpr float kNorm = (G == 64) ? 0.125f : 0.0625f;   // 2^-digits
+
+    extern __shared__ uint4 stage[];                       // two buffers of K * 2 bytes
+    __shared__ uint32_t red[32];
+
+    const int t = threadIdx.x;
+    const int nthreads = blockDim.x;                       // K / 32
+    const int warp = t >> 5, lane = t & 31;
+    const int warp_lanes = min(32, nthreads - warp * 32);
+    const uint32_t mask = warp_lanes == 32 ? 0xFFFFFFFFu : ((1u << warp_lanes) - 1u);
+    const int row_chunks = nthreads * 4;                   // 16-byte chunks per row
+    const uint32_t stage_s = ptx::smem_u32(stage);
+
+    auto issue_row = [&](int r, int buf) {
+        if (r < M) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(r) * K);
+            const uint32_t base = stage_s + static_cast<uint32_t>(buf * row_chunks * 16);
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int g = t + jj * nthreads;           // chunk index in the row
+                const int owner = g >> 2;
+                const uint32_t c = static_cast<uint32_t>(g & 3);
+                cp_async16(base + static_cast<uint32_t>((owner * 4 + (c ^ key32(owner))) * 16), src + g);
+            }
+        }
+        cp_async_commit();   // one group per row, empty past the end
+    };
+
+    int row = blockIdx.x;
+    issue_row(row, 0);
+    issue_row(row + gridDim.x, 1);
+    // The GEMM that follows may be scheduled on the SMs this grid leaves
+    // free; it reads these rows only after its griddepcontrol.wait.
+    ptx::launch_dependents();
+    for (int it = 0; row < M; row += gridDim.x, ++it) {
+        const int b = it & 1;
+        uint4 *sb = stage + b * row_chunks;
+        cp_async_wait_prior();    // this row's copies (by this thread) have landed ...
+        __syncthreads();          // ... and everyone else's
+
+        float v[32];
+        load_row32(sb, t, v);
+        rotate_row32<G>(v, reinterpret_cast<float4 *>(sb), t, mask);
+        auto chan = [&](int e) -> int { return row32_chan<G>(t, e); };
+
+        if (MODE == 1) {
+            float *dst = yrot + static_cast<size_t>(row) * K;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                *reinterpret_cast<float4 *>(dst + chan(4 * i)) =
+                    make_float4(v[4 * i] * kNorm, v[4 * i + 1] * kNorm, v[4 * i + 2] * kNorm,
+                                v[4 * i + 3] * kNorm);
+            __syncthreads();      // every warp is done with buffer b
+            issue_row(row + 2 * gridDim.x, b);
+            continue;
+        }
+
+        const float m = thread_absmax(v);
+        uint32_t mb = __reduce_max_sync(mask, __float_as_uint(m));
+        if (lane == 0) red[warp] = mb;
+        __syncthreads();          // the row maximum is complete (and buffer b is free)
+        issue_row(row + 2 * gridDim.x, b);
+        const int nwarps = (nthreads + 31) >> 5;
+        for (int w = 0; w < nwarps; ++w) mb = max(mb, red[w]);
+        const float a_u = __uint_as_float(mb);
+
+        const float inv = a_u > 0.0f ? __fdiv_rn(7.0f, a_u) : 0.0f;
+        if (t == 0) s[row] = __fdiv_rn(a_u * kNorm, 7.0f);
+
+        uint32_t packed[4];
+        quantize_pack(v, inv, packed);
+        uint8_t *qrow = q + static_cast<size_t>(row) * (K / 2);
+        if (G == 64) {
+            *reinterpret_cast<uint4 *>(qrow + t * 16) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        } else {
+            // registers 8 d3 .. 8 d3 + 7 are 8 consecutive channels: 4 bytes
+#pragma unroll
+            for (int d3 = 0; d3 < 4; ++d3)
+                *reinterpret_cast<uint32_t *>(qrow + chan(8 * d3) / 2) = packed[d3];
+        }
+        // red[] is rewritten only after the next row's first barrier, which
+        // every thread passes after reading it here
+    }
+    cp_async_wait_all();          // no copy outlives the CTA (empty groups past the end)
+}
+
 }  // namespace prep

@@ -72,6 +72,25 @@ def test_prepare_matches_oracle(group, M, K):
         assert sx[0].item() == 0.0 and int(qx[0].abs().sum()) == 0
 
 
+# The three prep kernels give the same codes and scales bit for bit: up to
+# 1024 rows (K <= 16384) the 16-channel kernel runs, beyond that the
+# 32-channel one (group 256, K <= 3072) or the 64-channel one.  The first
+# rows of a long launch must equal the same rows prepared alone.
+@pytest.mark.parametrize("K,group", [(1024, 256), (3072, 256), (4096, 256), (8192, 256),
+                                     (3072, 64)])
+def test_prep_kernels_agree_bit_for_bit(K, group):
+    M, head = 2100, 1000
+    x = _dev(_layer(M, K, 1, group, seed=K + group).x)
+    qx, sx = cr.convrot_prepare_act(x, group)
+    qh, sh = cr.convrot_prepare_act(x[:head].contiguous(), group)
+    yr = cr.convrot_debug_rotate_f32(x, group)
+    yh = cr.convrot_debug_rotate_f32(x[:head].contiguous(), group)
+    torch.cuda.synchronize()
+    assert torch.equal(qx[:head], qh)
+    assert torch.equal(sx[:head].view(torch.int32), sh.view(torch.int32))
+    assert torch.equal(yr[:head].view(torch.int32), yh.view(torch.int32))
+
+
 def test_prepare_edge_rows():
     # exact ties and saturation: absmax 7 after rotation makes inv = 1
     K, group = 256, 256
