@@ -871,9 +871,10 @@ def run_e2e(cr, prepared, spec, dev, stream, flush, args):
     x_host = wl.make_workload(args.workload)[0].x.pin_memory()
     y_host = torch.empty(prepared[-1][0].M, prepared[-1][0].N, dtype=torch.bfloat16).pin_memory()
     # chunks of at least 256 rows, up to 8: on the 8192-token layer 8 chunks
-    # measured 3.37 ms per step against 3.49 (4), 3.51 (16) and 3.92 (32):
-    # pipeline fill and drain are one chunk's copy each, and every chunk adds
-    # its own copy and launch overheads; one chunk would not overlap at all
+    # measured 3.36 ms per step against 3.49 (4), 3.41 (12) and 3.47 (16), on
+    # QKV 1.68 ms against 1.75 (4) and 1.74 (16): pipeline fill and drain are
+    # one chunk's copy each, and every chunk adds its own copy and launch
+    # overheads; one chunk would not overlap at all
     pipe = cr.HostPipeline(sp0.M, sp0.K, [(qw, sw, b, sp.group) for sp, qw, sw, b in prepared],
                            chunks=max(1, min(8, sp0.M // 256)), device=dev)
     steps = max(3, min(args.steps, 200))
