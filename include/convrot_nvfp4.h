@@ -33,7 +33,8 @@
  *     in 512-byte atoms of 128 rows x 4 blocks: the scale of row r, block j
  *     is at ((r / 128) * (K / 64) + j / 4) * 512 + 16 (r mod 32)
  *     + 4 ((r / 32) mod 4) + j mod 4, rows padded to a multiple of 128 (the
- *     layout the tensor cores read, so atoms go to them unchanged);
+ *     layout the tensor cores read, so atoms go to them unchanged); the
+ *     quantisation writes every byte, code 0 for the padding rows;
  *   - row scales: fp32 [rows].
  * Conventions are those of convrot.h: device pointers on the current device
  * (CONVROT_ERR_NOT_DEVICE otherwise), 16-byte aligned (CONVROT_ERR_ALIGN),

@@ -168,6 +168,13 @@ quant_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__
             *reinterpret_cast<uint2 *>(qrow + c0 / 2) = make_uint2(words[2 * b], words[2 * b + 1]);
         }
     }
+    // The padding rows of the last 128-row atom get scale code 0 (the value
+    // 0), so that every byte of sf is a function of x alone.
+    const int padded = (M + 127) & ~127;
+    for (int r = M + static_cast<int>(blockIdx.x); r < padded; r += gridDim.x) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) sf[sf_offset(r, prep::row_chan<G>(t, 16 * b) / 16, K)] = 0;
+    }
 }
 
 // ------------------------------------------------------------------ GEMM

@@ -52,6 +52,7 @@ def test_quantize_bit_exact_on_the_gpu_rotation(group, M, K):
     codes, sf_ref, s_ref = O.nvfp4_quantize_rows(y32)
     assert np.array_equal(s, s_ref)
     assert np.array_equal(gc.nvfp4_sf_rowmajor(sf, M, K), sf_ref)
+    assert np.array_equal(sf, O.nvfp4_sf_layout(sf_ref, K))      # padding rows included
     assert gc.nvfp4_codes_equal(q, O.nvfp4_pack(codes)).all()
     if M > 2:
         assert s[1] == 0 and not (q[1] & 0x77).any()
