@@ -236,9 +236,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t *__restric
             prep::cp_async_wait_all();
             bar_named(bid, gt);                          // the row has landed
             float v[prep::kElemsPerThread];
-            prep::load_row(stg, t, v);
+            prep::load_row<G>(stg, t, v);
             bar_named(bid, gt);                          // the stage may be overwritten
-            prep::rotate_row<G>(v, reinterpret_cast<float4 *>(stg), t, 0xFFFFFFFFu);
+            prep::rotate_row<G>(v, 0xFFFFFFFFu);
             const float m = prep::thread_absmax(v);
             uint32_t mb = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m));
             if (lane == 0) red[tok][t >> 5] = mb;

@@ -86,7 +86,7 @@ __host__ __device__ __forceinline__ size_t sf_offset(int64_t r, int64_t j, int64
 // Persistent over rows like the W4A4 prep kernel: K/64 threads per CTA,
 // thread t owns 64 channels; the next row's copy into the stage buffer
 // overlaps the current row's arithmetic.  Shared memory: K * 2 bytes of
-// stage, then (group 256) K * 4 bytes of exchange.
+// stage (the digit-3 swap of group 256 runs on lane shuffles).
 template <int G>
 __global__ void __launch_bounds__(prep::kMaxThreads)
 quant_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ q,
@@ -101,7 +101,6 @@ quant_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__
     const int warp = t >> 5, lane = t & 31;
     const int warp_lanes = min(32, nthreads - warp * 32);
     const uint32_t mask = warp_lanes == 32 ? 0xFFFFFFFFu : ((1u << warp_lanes) - 1u);
-    const int row_chunks = nthreads * 8;                 // 16-byte chunks per row
     const uint32_t stage_s = ptx::smem_u32(stage);
 
     // chunk c of owner thread o's 128-byte slice lands at o * 8 + (c ^ (o mod 8))
@@ -127,12 +126,12 @@ quant_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__
         prep::cp_async_wait_all();
         __syncthreads();
         float v[prep::kElemsPerThread];
-        prep::load_row(stage, t, v);
+        prep::load_row<G>(stage, t, v);
         __syncthreads();          // the stage buffer is free again
         if (next < M) issue_row(next);
         prep::cp_async_commit();
 
-        prep::rotate_row<G>(v, reinterpret_cast<float4 *>(stage + row_chunks), t, mask);
+        prep::rotate_row<G>(v, mask);
 #pragma unroll
         for (int e = 0; e < prep::kElemsPerThread; ++e) v[e] *= kNorm;   // exact
 
@@ -148,7 +147,7 @@ quant_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__
         if (t == 0) s[row] = sr;
 
         // registers 16 b .. 16 b + 15 hold 16 consecutive channels: one block
-        uint32_t words[8];
+        uint32_t words[8], codes[4];
         uint8_t *qrow = q + static_cast<size_t>(row) * (K / 2);
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
@@ -163,9 +162,19 @@ quant_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__
             for (int i = 0; i < 16; ++i) w8[i] = __fmul_rn(v[16 * b + i], inv);
             words[2 * b] = e2m1x8(w8);
             words[2 * b + 1] = e2m1x8(w8 + 8);
-            const int c0 = prep::row_chan<G>(t, 16 * b);   // first channel of the block
-            sf[sf_offset(row, c0 / 16, K)] = static_cast<uint8_t>(code);
-            *reinterpret_cast<uint2 *>(qrow + c0 / 2) = make_uint2(words[2 * b], words[2 * b + 1]);
+            codes[b] = code;
+        }
+        // with group 256 store d writes digit 3 = d, register block d ^ (t mod 4)
+        const int jg = (G == 256) ? (t & 3) : 0;
+#pragma unroll
+        for (int d = 0; d < 4; ++d) {
+            const int m = d ^ jg;
+            const int c0 = prep::row_chan<G>(t, 16 * m);   // first channel of the block
+            sf[sf_offset(row, c0 / 16, K)] =
+                static_cast<uint8_t>(prep::pick4(codes[0], codes[1], codes[2], codes[3], m));
+            *reinterpret_cast<uint2 *>(qrow + c0 / 2) =
+                make_uint2(prep::pick4(words[0], words[2], words[4], words[6], m),
+                           prep::pick4(words[1], words[3], words[5], words[7], m));
         }
     }
     // The padding rows of the last 128-row atom get scale code 0 (the value
@@ -549,7 +558,7 @@ convrot_status check_shape(int64_t rows, int64_t K, int group) {
     return CONVROT_OK;
 }
 
-// Resident quantisation CTAs (K/64 threads, K * (2 or 6) bytes) per SM, cached
+// Resident quantisation CTAs (K/64 threads, K * 2 bytes) per SM, cached
 // in atomics (concurrent first callers store the same value).
 int quant_ctas_per_sm(int group, int64_t K) {
     static std::atomic<int> cache[2][prep::kMaxThreads + 1];
@@ -558,7 +567,7 @@ int quant_ctas_per_sm(int group, int64_t K) {
     int slot = entry.load(std::memory_order_relaxed);
     if (slot == 0) {
         int n = 0;
-        const size_t smem = static_cast<size_t>(K) * (group == 256 ? 6 : 2);
+        const size_t smem = static_cast<size_t>(K) * 2;
         const cudaError_t e =
             group == 64
                 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nvfp4::quant_kernel<64>, T, smem)
@@ -572,7 +581,7 @@ int quant_ctas_per_sm(int group, int64_t K) {
 convrot_status launch_quant(int num_sms, const void *x, int64_t rows, int64_t K, int group,
                             uint8_t *q, uint8_t *sf, float *s, cudaStream_t stream) {
     if (rows == 0) return CONVROT_OK;
-    const size_t smem = static_cast<size_t>(K) * (group == 256 ? 6 : 2);
+    const size_t smem = static_cast<size_t>(K) * 2;
     const int64_t resident = static_cast<int64_t>(num_sms) * quant_ctas_per_sm(group, K);
     const dim3 grid(static_cast<unsigned>(rows < resident ? rows : resident));
     const dim3 block(static_cast<unsigned>(K / prep::kElemsPerThread));

@@ -13,10 +13,10 @@
 // that differ only in digit d, y_i = (x_0 + x_1 + x_2 + x_3) - 2 x_i.  The k
 // butterflies commute (every factor is the same symmetric T), so they run in
 // any order: digits 0, 1, 2 live inside one thread's 64 registers; for
-// n = 256 digit 3 spans the 4 threads of the group, which swap quarters of
-// their data through shared memory so that digit 3 also becomes a register
-// stride.  The 1/2^k normalisation is exact and is folded into the scale
-// (see below), so the butterflies run on unnormalised values.
+// n = 256 digit 3 spans the 4 threads of the group (four lanes of a warp),
+// which swap quarters of their data with lane shuffles so that digit 3 also
+// becomes a register stride.  The 1/2^k normalisation is exact and is folded
+// into the scale (see below), so the butterflies run on unnormalised values.
 //
 // Quantisation ("convrot-mlx" README, "What is included": symmetric rowwise
 // absmax to [-7, 7]).  With u the unnormalised rotated row and y = u 2^-k:
@@ -118,11 +118,19 @@ __device__ __forceinline__ void cp_async_wait_prior() {
 
 // Registers v[0..63] <- the thread's 64 channels of a staged bf16 row (the
 // stage layout: chunk c of thread t's 128-byte slice at position c ^ (t & 7)).
+// For n = 64 register e holds channel 64 t + e.  For n = 256 the quarters
+// come in the order the digit-3 swap of rotate_row needs: registers
+// 16 m .. 16 m + 15 hold the thread's quarter m ^ (t mod 4), i.e. slice
+// chunks i ^ 2 (t mod 4) for register chunk i.  The read key
+// (t mod 8) ^ 2 (t mod 4) still differs between the 8 lanes of a quarter
+// warp, so the 128-bit reads stay free of bank conflicts.
+template <int G>
 __device__ __forceinline__ void load_row(const uint4 *__restrict__ sb, int t,
                                          float (&v)[kElemsPerThread]) {
+    const int key = (G == 256) ? ((t & 7) ^ ((t & 3) << 1)) : (t & 7);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const uint4 raw = sb[t * 8 + (i ^ (t & 7))];
+        const uint4 raw = sb[t * 8 + (i ^ key)];
         const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -132,103 +140,57 @@ __device__ __forceinline__ void load_row(const uint4 *__restrict__ sb, int t,
     }
 }
 
-// The unnormalised rotation of the thread's channels: digits 0-2 in
-// registers; for n = 256 the four threads of a group (lanes of one warp)
-// hold digit 3 = 0..3 and swap quarters through xb (16 float4 per thread)
-// so that each thread then holds, for its j = t mod 4, the channels
-// 64 d3 + 16 j + r (d3 = 0..3, r = 0..15): digit 3 becomes a register
-// stride of 16 and the last butterfly runs in registers.  Chunk i = 4a + b
-// (4 floats) of thread t is stored at slot (4b + a) ^ (t mod 16) of t's
-// 16-slot row, which keeps both the stores and the transposed loads free of
-// bank conflicts.  mask: the lanes of the warp that take part.
+// The unnormalised rotation of the thread's channels (registers as load_row
+// leaves them): digits 0-2 in registers; for n = 256 the four threads of a
+// group (lanes 4g .. 4g + 3 of one warp, j = t mod 4 the thread's digit 3)
+// then swap quarters with lane shuffles so that digit 3 is a register
+// stride too, and the last butterfly runs in registers.
+//
+// Why the sums are unchanged by load_row's quarter order: every radix-4
+// butterfly adds its quadruple as (x_0 + x_1) + (x_2 + x_3).  With quarter
+// m ^ j in register block m, the digit-2 butterfly pairs blocks {0, 1} and
+// {2, 3}, i.e. quarters {j, j ^ 1} = {0, 1} or {2, 3} and the other pair:
+// the same two pair sums, added the same way up to the order of operands,
+// and IEEE addition is commutative bit for bit.
+//
+// The swap: in round m = 1, 2, 3 a thread sends block m (its quarter m ^ j,
+// which lane j ^ m needs) to lane j ^ m and receives that lane's block m (its
+// quarter (j ^ m) ^ m = j).  Every register index is static, so each round
+// is 16 shuffles in place.  Afterwards block m holds quarter j of the thread
+// with digit 3 = j ^ m, and the digit-3 butterfly pairs those threads as
+// {j, j ^ 1} and {j ^ 2, j ^ 3}, again the pairs {0, 1} and {2, 3}.
+// mask: the lanes of the warp that take part (whole groups).
 template <int G>
-__device__ __forceinline__ void rotate_row(float (&v)[kElemsPerThread], float4 *__restrict__ xb,
-                                           int t, uint32_t mask) {
+__device__ __forceinline__ void rotate_row(float (&v)[kElemsPerThread], uint32_t mask) {
     radix4_digit0(v);
     radix4_stage<4>(v);
     radix4_stage<16>(v);
     if (G == 256) {
-        const int key = t & 15;
-        __syncwarp(mask);     // the group finished reading the previous swap
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-            xb[t * 16 + ((((i & 3) << 2) | (i >> 2)) ^ key)] =
-                make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-        __syncwarp(mask);
-        const int j = t & 3, gb = t & ~3;
+        for (int m = 1; m < 4; ++m)
 #pragma unroll
-        for (int d3 = 0; d3 < 4; ++d3) {
-            const int w = gb + d3;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const float4 f = xb[w * 16 + (((c << 2) | j) ^ (w & 15))];
-                v[16 * d3 + 4 * c] = f.x;
-                v[16 * d3 + 4 * c + 1] = f.y;
-                v[16 * d3 + 4 * c + 2] = f.z;
-                v[16 * d3 + 4 * c + 3] = f.w;
-            }
-        }
+            for (int r = 0; r < 16; ++r) v[16 * m + r] = __shfl_xor_sync(mask, v[16 * m + r], m);
         radix4_stage<16>(v);
     }
 }
 
-// The same rotation for prep_kernel, whose digit-3 exchange reuses the
-// row's own stage buffer (128 bytes per thread: the thread's 64 bf16
-// channels, already in registers) instead of a separate 256-byte-per-thread
-// area.  It runs in two passes over halves of each quarter: in pass p every
-// thread stores registers 16 qq + 8 p + (0..7) of each quarter qq (8 float4)
-// and reads back, from each of the four threads of its group, the 8 values
-// of its own quarter j.  (Skipping the thread's own quarter diverges the
-// warp, since the four lanes of a group would take different branches, and
-// measured 25% slower.)  Slot key k(w) = 2 (w mod 4) + (w / 4 mod 2): the
-// 8 threads of a quarter warp then store to 8 distinct slots and read from
-// 8 distinct slots, so neither side has bank conflicts.  The values and the
-// order of every addition are those of rotate_row, so results are identical.
-__device__ __forceinline__ int stage_key(int w) { return ((w & 3) << 1) | ((w >> 2) & 1); }
-
-template <int G>
-__device__ __forceinline__ void rotate_row_staged(float (&v)[kElemsPerThread],
-                                                  float4 *__restrict__ xb, int t, uint32_t mask) {
-    radix4_digit0(v);
-    radix4_stage<4>(v);
-    radix4_stage<16>(v);
-    if (G == 256) {
-        const int j = t & 3, gb = t & ~3, kt = stage_key(t);
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            __syncwarp(mask);     // the group's reads of the buffer (row load or pass 0) are done
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq)
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const int e = 16 * qq + 8 * p + 4 * c;
-                    xb[t * 8 + ((2 * qq + c) ^ kt)] = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-                }
-            __syncwarp(mask);
-#pragma unroll
-            for (int d3 = 0; d3 < 4; ++d3) {
-                const int w = gb + d3;
-                const int kw = stage_key(w);
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const float4 f = xb[w * 8 + ((2 * j + c) ^ kw)];
-                    const int e = 16 * d3 + 8 * p + 4 * c;
-                    v[e] = f.x;
-                    v[e + 1] = f.y;
-                    v[e + 2] = f.z;
-                    v[e + 3] = f.w;
-                }
-            }
-        }
-        radix4_stage<16>(v);
-    }
+// a[m] for a lane-dependent m in 0..3, by selects (registers cannot be
+// indexed at run time).  After rotate_row (n = 256) block m of thread t holds
+// digit 3 = m ^ (t mod 4); picking block d ^ (t mod 4) in store d makes one
+// store instruction cover digit 3 = d of every group, four contiguous runs of
+// a group's lanes, instead of four places apart.
+__device__ __forceinline__ uint32_t pick4(uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          int m) {
+    return (m & 2) ? ((m & 1) ? a3 : a2) : ((m & 1) ? a1 : a0);
 }
 
-// Channel of register e of thread t after rotate_row.
+// Channel of register e of thread t after rotate_row: for n = 256, block
+// e / 16 holds digit 3 = (e / 16) ^ j, quarter j = t mod 4 of the group's
+// 64-channel blocks.
 template <int G>
 __device__ __forceinline__ int row_chan(int t, int e) {
     if (G == 64) return t * 64 + e;
-    return (t & ~3) * 64 + 64 * (e >> 4) + 16 * (t & 3) + (e & 15);
+    return (t & ~3) * 64 + 64 * ((e >> 4) ^ (t & 3)) + 16 * (t & 3) + (e & 15);
 }
 
 // The thread's max |v|: four independent chains of three-input maxima.
@@ -268,8 +230,9 @@ __device__ __forceinline__ void quantize_pack(const float (&v)[E], float inv,
     }
 }
 
-// Stage buffers of prep_kernel: two where the digit-3 exchange reuses the
-// current row's buffer (n = 256), one otherwise.
+// Stage buffers of prep_kernel: two for n = 256, one for n = 64 (each
+// measured faster than the other count on 8192 x 8192: 43.9 against 45.1 us
+// for n = 256; for n = 64 one buffer is 5% faster).
 __host__ __device__ constexpr int stage_buffers(int G) { return G == 256 ? 2 : 1; }
 
 // MODE 0: quantise + pack (q, s).  MODE 1: write the normalised rotated row
@@ -278,15 +241,14 @@ __host__ __device__ constexpr int stage_buffers(int G) { return G == 256 ? 2 : 1
 // Persistent: CTA b handles rows b, b + gridDim.x, ...  Rows arrive by
 // asynchronous copies while the previous row is rotated and quantised.  For
 // n = 256, two stage buffers of one bf16 row each: the CTA's next two rows
-// are on their way during the arithmetic.  For n = 64 (no exchange), one
-// buffer: the next row is requested as soon as the current one is in
-// registers (measured faster there than two buffers).  Each row is read with coalesced 16-byte copies (consecutive
-// threads, consecutive chunks) that land so that chunk c of thread t's
-// 128-byte slice sits at position c ^ (t mod 8); each thread then reads its
-// own 64 channels with conflict-free 128-bit loads.  For n = 256 the
-// digit-3 exchange then reuses the same buffer (rotate_row_staged), and the
-// barrier of the row maximum also tells that every warp is done with the
-// buffer, which then receives the row after next.
+// are on their way during the arithmetic, and the barrier of the row maximum
+// also tells that every warp has read the current buffer, which then
+// receives the row after next.  For n = 64, one buffer: the next row is
+// requested as soon as the current one is in registers.  Each row is read
+// with coalesced 16-byte copies (consecutive threads, consecutive chunks)
+// that land so that chunk c of thread t's 128-byte slice sits at position
+// c ^ (t mod 8); each thread then reads its own 64 channels with
+// conflict-free 128-bit loads (load_row).
 template <int G, int MODE>
 __global__ void __launch_bounds__(kMaxThreads)
 prep_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ q,
@@ -298,7 +260,7 @@ prep_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ 
     if (blockIdx.x == 0)
         for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0u;
     constexpr float kNorm = (G == 64) ? 0.125f : 0.0625f;   // 2^-kDigits
-    constexpr int NBUF = stage_buffers(G);   // one buffer only without an exchange
+    constexpr int NBUF = stage_buffers(G);
 
     // NBUF stage buffers of K * 2 bytes
     extern __shared__ uint4 stage[];
@@ -345,12 +307,12 @@ prep_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ 
         __syncthreads();          // ... and everyone else's
 
         float v[kElemsPerThread];
-        load_row(sb, t, v);
+        load_row<G>(sb, t, v);
         if (NBUF == 1) {
             __syncthreads();      // the stage buffer is free again
             issue_row(row + gridDim.x, 0);
         }
-        rotate_row_staged<G>(v, reinterpret_cast<float4 *>(sb), t, mask);
+        rotate_row<G>(v, mask);
         auto chan = [&](int e) -> int { return row_chan<G>(t, e); };
 
         if (MODE == 1) {
@@ -388,11 +350,16 @@ prep_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__ 
             dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
             dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
         } else {
-            // registers 16 d3 .. 16 d3 + 15 are 16 consecutive channels: 8 bytes
+            // each register block is 16 consecutive channels (8 bytes); store d
+            // writes digit 3 = d, the block d ^ j
+            const int j = t & 3;
 #pragma unroll
-            for (int d3 = 0; d3 < 4; ++d3)
-                *reinterpret_cast<uint2 *>(qrow + chan(16 * d3) / 2) =
-                    make_uint2(packed[2 * d3], packed[2 * d3 + 1]);
+            for (int d = 0; d < 4; ++d) {
+                const int m = d ^ j;
+                *reinterpret_cast<uint2 *>(qrow + ((t & ~3) * 64 + 64 * d + 16 * j) / 2) =
+                    make_uint2(pick4(packed[0], packed[2], packed[4], packed[6], m),
+                               pick4(packed[1], packed[3], packed[5], packed[7], m));
+            }
         }
     }
     cp_async_wait_all();          // no copy outlives the CTA (empty groups past the end)

@@ -71,7 +71,7 @@ rotate_bf16_kernel(const uint16_t *__restrict__ x, int M, int K, uint16_t *__res
     static_assert(G == 64 || G == 256, "group 64 or 256");
     constexpr float kNorm = (G == 64) ? 0.125f : 0.0625f;   // 1/sqrt(G), exact
 
-    // K * 2 bytes of stage buffer, then (group 256) K * 4 bytes of exchange
+    // K * 2 bytes of stage buffer
     extern __shared__ uint4 stage[];
 
     const int t = threadIdx.x;
@@ -79,7 +79,6 @@ rotate_bf16_kernel(const uint16_t *__restrict__ x, int M, int K, uint16_t *__res
     const int warp = t >> 5;
     const int warp_lanes = min(32, nthreads - warp * 32);
     const uint32_t mask = warp_lanes == 32 ? 0xFFFFFFFFu : ((1u << warp_lanes) - 1u);
-    const int row_chunks = nthreads * 8;                 // 16-byte chunks per row
     const uint32_t stage_s = ptx::smem_u32(stage);
 
     // chunk c of owner thread o's 128-byte slice lands at o * 8 + (c ^ (o mod 8))
@@ -106,24 +105,32 @@ rotate_bf16_kernel(const uint16_t *__restrict__ x, int M, int K, uint16_t *__res
         __syncthreads();
 
         float v[prep::kElemsPerThread];
-        prep::load_row(stage, t, v);
+        prep::load_row<G>(stage, t, v);
         __syncthreads();          // the stage buffer is free again
         if (next < M) issue_row(next);
         prep::cp_async_commit();
 
-        prep::rotate_row<G>(v, reinterpret_cast<float4 *>(stage + row_chunks), t, mask);
+        prep::rotate_row<G>(v, mask);
 
-        // registers 16 b .. 16 b + 15 hold 16 consecutive channels
+        // registers 16 b .. 16 b + 15 hold 16 consecutive channels; with
+        // group 256 store d writes digit 3 = d, register block d ^ (t mod 4)
         uint16_t *dst = xr + static_cast<size_t>(row) * K;
+        uint32_t w[4][8];
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            uint32_t w[8];
+        for (int b = 0; b < 4; ++b)
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                w[j] = bf16x2_rn(v[16 * b + 2 * j] * kNorm, v[16 * b + 2 * j + 1] * kNorm);
-            uint4 *d = reinterpret_cast<uint4 *>(dst + prep::row_chan<G>(t, 16 * b));
-            d[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            for (int i = 0; i < 8; ++i)
+                w[b][i] = bf16x2_rn(v[16 * b + 2 * i] * kNorm, v[16 * b + 2 * i + 1] * kNorm);
+        const int jg = (G == 256) ? (t & 3) : 0;
+#pragma unroll
+        for (int d = 0; d < 4; ++d) {
+            const int m = d ^ jg;
+            uint32_t o[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[i] = prep::pick4(w[0][i], w[1][i], w[2][i], w[3][i], m);
+            uint4 *p = reinterpret_cast<uint4 *>(dst + prep::row_chan<G>(t, 16 * m));
+            p[0] = make_uint4(o[0], o[1], o[2], o[3]);
+            p[1] = make_uint4(o[4], o[5], o[6], o[7]);
         }
     }
 }
@@ -927,7 +934,7 @@ convrot_status check_gemm_shape(int64_t M, int64_t N, int64_t K) {
     return CONVROT_OK;
 }
 
-// Resident rotation CTAs (K/64 threads, K * (2 or 6) bytes) per SM, cached
+// Resident rotation CTAs (K/64 threads, K * 2 bytes) per SM, cached
 // in atomics (concurrent first callers store the same value).
 int rot_ctas_per_sm(int group, int64_t K) {
     static std::atomic<int> cache[2][prep::kMaxThreads + 1];
@@ -936,7 +943,7 @@ int rot_ctas_per_sm(int group, int64_t K) {
     int slot = entry.load(std::memory_order_relaxed);
     if (slot == 0) {
         int n = 0;
-        const size_t smem = static_cast<size_t>(K) * (group == 256 ? 6 : 2);
+        const size_t smem = static_cast<size_t>(K) * 2;
         const cudaError_t e =
             group == 64
                 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, w4a16::rotate_bf16_kernel<64>, T, smem)
@@ -950,7 +957,7 @@ int rot_ctas_per_sm(int group, int64_t K) {
 convrot_status launch_rotate(int num_sms, const void *x, int64_t M, int64_t K, int group, void *xr,
                              cudaStream_t stream) {
     if (M == 0) return CONVROT_OK;
-    const size_t smem = static_cast<size_t>(K) * (group == 256 ? 6 : 2);
+    const size_t smem = static_cast<size_t>(K) * 2;
     const int64_t resident = static_cast<int64_t>(num_sms) * rot_ctas_per_sm(group, K);
     const dim3 grid(static_cast<unsigned>(M < resident ? M : resident));
     const dim3 block(static_cast<unsigned>(K / prep::kElemsPerThread));
