@@ -16,13 +16,14 @@
 //                     rows, one CTA per SM:
 //     warp 0      producer (one thread): per stage of 256 codes, the packed
 //                 token and weight tiles by TMA (128-byte swizzle) and the
-//                 tiles' scale atoms by bulk copies, on one barrier;
+//                 tiles' scale atoms by TMA as four replicas of each copy
+//                 source (see make_sf_map), all on one barrier;
 //     warp 1      TMEM allocator and MMA issuer (one thread): per stage it
-//                 copies the scale atoms into TMEM (tcgen05.cp 32x128b,
-//                 broadcast to the four lane quarters: row n's four scales of
-//                 one 64-code step sit in lane n mod 32, column n / 32) and
-//                 issues four MMAs of K = 64 (M = 128, N = 256) into one
-//                 fp32 accumulator of 256 columns;
+//                 copies the scales into TMEM (tcgen05.cp 128x256b: lane
+//                 quarter q receives replica q, so row n's four scales of one
+//                 64-code step sit in lane n mod 32 of every quarter, column
+//                 n / 32) and issues four MMAs of K = 64 (M = 128, N = 256)
+//                 into one fp32 accumulator of 256 columns;
 //     warps 2..5  epilogue, one per TMEM lane quarter: tcgen05.ld, (acc * sx)
 //                 * sw + b, bf16, stores; then the accumulator is free.
 #include <cuda.h>
@@ -192,11 +193,19 @@ constexpr int BM = 128;                  // token rows per tile (the MMA's M)
 constexpr int BN = 256;                  // weight rows per tile (the MMA's N)
 constexpr int PKB = 128;                 // packed bytes per row per stage: 256 codes
 constexpr int KB = 4;                    // MMAs (K = 64) per stage
-constexpr int SP = 4;                    // ring stages
+constexpr int SP = 3;                    // ring stages
 constexpr int A_ST = BM * PKB;           // 16 KB
 constexpr int B_ST = BN * PKB;           // 32 KB
-constexpr int SFA_ST = KB * 512;         // one scale atom per 64 codes
-constexpr int SFB_ST = 2 * KB * 512;     // two 128-row atoms per 64 codes
+// Scales are staged for 128-lane copies (tcgen05.cp 128x256b): a copy
+// source is 128 rows x 32 bytes, row i = 32 q + l holding lane l's 16 bytes
+// of two scale atoms (so each lane quarter q receives the same values, as
+// the MMA reads them).  In core-matrix order (8 rows x 16 bytes) with the
+// two 16-byte halves 2 KB apart and 8-row groups 128 bytes apart, replica q
+// of an atom is the atom's 512 bytes verbatim at half * 2048 + q * 512, so
+// one TMA (make_sf_map) fills a whole 4 KB source.
+constexpr int SF_SRC = 4096;
+constexpr int SFA_ST = (KB / 2) * SF_SRC;   // A: the atoms of steps 2p, 2p + 1 per source
+constexpr int SFB_ST = KB * SF_SRC;         // B: the two 128-row atoms of one step per source
 constexpr int OFF_A = 0;                 // 1024-aligned tiles first
 constexpr int OFF_B = OFF_A + SP * A_ST;
 constexpr int OFF_SFA = OFF_B + SP * B_ST;
@@ -222,23 +231,38 @@ __host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N) {
            | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
 }
 
-// Shared-memory descriptor of a scale atom for tcgen05.cp: 32 rows of 16
-// bytes, no swizzle, K-major core matrices of 8 rows x 16 bytes 128 bytes
-// apart in the row direction.
-__device__ __forceinline__ uint64_t sf_atom_desc(uint32_t smem_addr) {
+// Shared-memory descriptor of a scale copy source for tcgen05.cp: 128 rows
+// of 32 bytes, no swizzle, core matrices of 8 rows x 16 bytes, the two
+// 16-byte halves of a row 2 KB apart (leading offset), 8-row groups 128
+// bytes apart (stride offset).
+__device__ __forceinline__ uint64_t sf_src_desc(uint32_t smem_addr) {
     uint64_t d = 0;
     d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);   // start address
-    d |= static_cast<uint64_t>(16 >> 4) << 16;                 // leading offset (one core matrix)
+    d |= static_cast<uint64_t>(2048 >> 4) << 16;               // leading offset: the second half
     d |= static_cast<uint64_t>(128 >> 4) << 32;                // stride between 8-row groups
     d |= static_cast<uint64_t>(1) << 46;                       // descriptor version (sm_100)
     return d;                                                  // swizzle mode 0: none
 }
 
-// TMEM <- 32 rows x 128 bits of shared memory, broadcast to the four lane
-// quarters.
+// TMEM lanes 0..127, 8 columns <- 128 rows x 256 bits of shared memory.
+// One instruction instead of the two four-column broadcast copies
+// (32x128b.warpx4) it replaces: the tensor pipe spends about the same time
+// on a copy of either size.
 __device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc)
                  : "memory");
+}
+
+// One 4 KB scale copy source by TMA (4-D map, box 512 B x 4 replicas x 2 x 1;
+// see make_sf_map).
+__device__ __forceinline__ void tma_load_sf(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(0), "r"(c2), "r"(c3),
+          "r"(bar)
+        : "memory");
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T with per-16 E4M3 scales from TMEM.
@@ -253,16 +277,6 @@ __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint6
         : "memory");
 }
 
-// Bulk copy of `bytes` (a multiple of 16) contiguous global bytes into
-// shared memory, completing on the barrier's transaction count.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
-                                          uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-        : "memory");
-}
-
 __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t *>(&h);
@@ -270,10 +284,12 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
 
 // tmA: codes of the tokens [M][K/2], box 128 B x 128 rows, 128-byte swizzle.
 // tmB: codes of the weights [N][K/2], box 128 B x 256 rows, 128-byte swizzle.
-// sfx, sfw: scale atoms (rows padded to 128); sx, sw: row scales.
+// tmSA, tmSB: the scale atoms of the tokens and of the weights (rows padded
+// to 128) as copy-source replicas (make_sf_map); sx, sw: row scales.
 __global__ void __launch_bounds__(kThreads, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                  const uint8_t *__restrict__ sfx, const uint8_t *__restrict__ sfw,
+                  const __grid_constant__ CUtensorMap tmSA,
+                  const __grid_constant__ CUtensorMap tmSB,
                   const float *__restrict__ sx, const float *__restrict__ sw,
                   const uint16_t *__restrict__ bias, uint16_t *__restrict__ y, int M, int N, int K) {
     extern __shared__ uint8_t smem_raw[];
@@ -302,6 +318,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         ptx::fence_mbar_init();
         ptx::tma_prefetch_desc(&tmA);
         ptx::tma_prefetch_desc(&tmB);
+        ptx::tma_prefetch_desc(&tmSA);
+        ptx::tma_prefetch_desc(&tmSB);
     }
     if (warp == kWarpMma) {
         ptx::tmem_alloc<1>(sbase + OFF_MISC, TMEM_COLS);
@@ -318,8 +336,6 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     const int num_tiles = tiles_m * tiles_n;
     const int nkb = K / 64;                          // MMAs over K
     const int num_kp = (nkb + KB - 1) / KB;          // stages per tile
-    const int ka = K / 64;                           // scale atoms per 128 rows
-    const int npad = (N + 127) / 128 * 128;          // weight rows of the scale buffer
 
     if (warp == kWarpTma) {
         int ps = 0;
@@ -328,21 +344,23 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         for (int tile = blockIdx.x; lane == 0 && ok && tile < num_tiles; tile += gridDim.x) {
             const int ta = tile % tiles_m, tb = tile / tiles_m;
             const int m0 = ta * BM, n0 = tb * BN;
-            const int nsfb = (n0 + 128 < npad) ? 2 : 1;   // weight scale atoms present
             for (int kp = 0; kp < num_kp; ++kp) {
                 if (!ptx::mbar_wait(empty_p(ps), ph ^ 1, abort_flag)) { ok = false; break; }
-                const int nk = min(KB, nkb - kp * KB);
-                const uint32_t sfb_bytes = static_cast<uint32_t>(nk * 512);
-                ptx::mbar_arrive_expect_tx(full_p(ps), A_ST + B_ST + sfb_bytes * (1 + nsfb));
+                const int nk = min(KB, nkb - kp * KB);       // MMA steps of this stage
+                const int npairs = (nk + 1) / 2;             // token scale sources
+                const int s0 = kp * KB;                      // first scale atom (step)
+                // one 4 KB copy source per TMA; steps past K are not requested
+                // (a pair's second step past K reads as zeros)
+                ptx::mbar_arrive_expect_tx(full_p(ps),
+                                           A_ST + B_ST + (npairs + nk) * SF_SRC);
                 ptx::tma_load_2d(sbase + OFF_A + ps * A_ST, &tmA, full_p(ps), kp * PKB, m0);
                 ptx::tma_load_2d(sbase + OFF_B + ps * B_ST, &tmB, full_p(ps), kp * PKB, n0);
-                bulk_load(sbase + OFF_SFA + ps * SFA_ST,
-                          sfx + (static_cast<size_t>(m0 / 128) * ka + kp * KB) * 512, sfb_bytes,
-                          full_p(ps));
-                for (int h = 0; h < nsfb; ++h)
-                    bulk_load(sbase + OFF_SFB + ps * SFB_ST + h * KB * 512,
-                              sfw + (static_cast<size_t>(n0 / 128 + h) * ka + kp * KB) * 512,
-                              sfb_bytes, full_p(ps));
+                for (int pr = 0; pr < npairs; ++pr)
+                    tma_load_sf(sbase + OFF_SFA + ps * SFA_ST + pr * SF_SRC, &tmSA, full_p(ps),
+                                s0 + 2 * pr, m0 / 128);
+                for (int j = 0; j < nk; ++j)
+                    tma_load_sf(sbase + OFF_SFB + ps * SFB_ST + j * SF_SRC, &tmSB, full_p(ps),
+                                n0 / 128, s0 + j);
                 if (++ps == SP) { ps = 0; ph ^= 1; }
             }
         }
@@ -372,11 +390,13 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                     const uint32_t sfb_t = sfa_t + KB * 4;
                     const uint32_t sa = sbase + OFF_SFA + ps * SFA_ST;
                     const uint32_t sb = sbase + OFF_SFB + ps * SFB_ST;
-                    for (int j = 0; j < nk; ++j) {
-                        tmem_cp_sf(sfa_t + 4 * j, sf_atom_desc(sa + 512 * j));
-                        tmem_cp_sf(sfb_t + 8 * j, sf_atom_desc(sb + 512 * j));
-                        tmem_cp_sf(sfb_t + 8 * j + 4, sf_atom_desc(sb + KB * 512 + 512 * j));
-                    }
+                    // step j's scales: token columns sfa_t + 4 j (two steps per
+                    // copy), weight columns sfb_t + 8 j (both 128-row halves
+                    // of the tile per copy)
+                    for (int pr = 0; 2 * pr < nk; ++pr)
+                        tmem_cp_sf(sfa_t + 8 * pr, sf_src_desc(sa + pr * SF_SRC));
+                    for (int j = 0; j < nk; ++j)
+                        tmem_cp_sf(sfb_t + 8 * j, sf_src_desc(sb + j * SF_SRC));
                     const uint32_t a0 = sbase + OFF_A + ps * A_ST, b0 = sbase + OFF_B + ps * B_ST;
                     for (int j = 0; j < nk; ++j)
                         mma_mxf4(tmem_base, ptx::sw128_kmajor_desc(a0 + 32 * j),
@@ -606,12 +626,38 @@ bool make_code_map(CUtensorMap *map, const uint8_t *base, int64_t rows, int64_t 
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The scale atoms of `rows` rows (padded to 128) as tcgen05.cp sources: a
+// 4-D view of the atom layout (32-bit elements) whose 128 x 4 x 2 x 1 box is
+// one 4 KB source in shared memory, [pair member][replica][atom, 512 bytes].
+// The replica dimension has global stride 0: the same atom four times.
+//   token side (b_side false): pair member = two consecutive steps,
+//     dims {atom, replica, step, row group of 128}, coordinates (step, group);
+//   weight side: pair member = two consecutive 128-row groups,
+//     dims {atom, replica, group, step}, coordinates (group, step).
+// The atom of step s, group g starts at (g * K/64 + s) * 512.
+bool make_sf_map(CUtensorMap *map, const uint8_t *sf, int64_t rows, int64_t K, bool b_side) {
+    const cuuint64_t ka = static_cast<cuuint64_t>(K / 64);
+    const cuuint64_t groups = static_cast<cuuint64_t>((rows + 127) / 128);
+    const cuuint64_t dims_a[4] = {128, 4, ka, groups};
+    const cuuint64_t str_a[3] = {0, 512, ka * 512};
+    const cuuint64_t dims_b[4] = {128, 4, groups, ka};
+    const cuuint64_t str_b[3] = {0, ka * 512, 512};
+    const cuuint32_t box[4] = {128, 4, 2, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, const_cast<uint8_t *>(sf),
+                    b_side ? dims_b : dims_a, b_side ? str_b : str_a, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 convrot_status launch_gemm(int num_sms, const uint8_t *qx, const uint8_t *sfx, const float *sx,
                            const uint8_t *qw, const uint8_t *sfw, const float *sw,
                            const void *bias, int64_t M, int64_t N, int64_t K, void *y,
                            cudaStream_t stream) {
     CUtensorMap tmA, tmB;
-    if (!make_code_map(&tmA, qx, M, K, nvfp4::BM) || !make_code_map(&tmB, qw, N, K, nvfp4::BN))
+    CUtensorMap tmSA, tmSB;
+    if (!make_code_map(&tmA, qx, M, K, nvfp4::BM) || !make_code_map(&tmB, qw, N, K, nvfp4::BN) ||
+        !make_sf_map(&tmSA, sfx, M, K, false) || !make_sf_map(&tmSB, sfw, N, K, true))
         return CONVROT_ERR_CUDA;
     const int64_t tiles = ((M + nvfp4::BM - 1) / nvfp4::BM) * ((N + nvfp4::BN - 1) / nvfp4::BN);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
@@ -626,7 +672,7 @@ convrot_status launch_gemm(int num_sms, const uint8_t *qx, const uint8_t *sfx, c
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(
-        &cfg, nvfp4::nvfp4_gemm_kernel, tmA, tmB, sfx, sfw, sx, sw,
+        &cfg, nvfp4::nvfp4_gemm_kernel, tmA, tmB, tmSA, tmSB, sx, sw,
         static_cast<const uint16_t *>(bias), static_cast<uint16_t *>(y), static_cast<int>(M),
         static_cast<int>(N), static_cast<int>(K));
     return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
