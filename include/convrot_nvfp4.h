@@ -84,6 +84,24 @@ convrot_status convrot_nvfp4_linear_prepared(const uint8_t *qx, const uint8_t *s
                                              int64_t K, void *y_bf16, convrot_stream_t stream);
 
 /*
+ * Test hook: convrot_nvfp4_linear_prepared with the GEMM's tile width
+ * forced.  form:
+ *          0  automatic: 128-wide weight tiles where twice the number of
+ *             256-wide tiles fits in one wave of CTAs (one per SM), else
+ *             256-wide;
+ *          1  tiles of 128 tokens x 256 weight rows;
+ *          2  tiles of 128 tokens x 128 weight rows.
+ * Returns CONVROT_ERR_SHAPE for any other form.  Exposes the product of
+ * "convrot-mlx" README, "Install and test" per tile width.
+ */
+convrot_status convrot_nvfp4_debug_gemm_form(const uint8_t *qx, const uint8_t *sfx,
+                                             const float *sx, const uint8_t *qw,
+                                             const uint8_t *sfw, const float *sw,
+                                             const void *bias_bf16, int64_t M, int64_t N,
+                                             int64_t K, int form, void *y_bf16,
+                                             convrot_stream_t stream);
+
+/*
  * The whole NVFP4 layer: quantisation of x into `workspace`
  * (ws_bytes >= convrot_nvfp4_workspace_size(M, K), 256-byte aligned,
  * CONVROT_ERR_WORKSPACE otherwise), then the product.  Two kernels.

@@ -609,6 +609,7 @@ def lib_nvfp4() -> ctypes.CDLL:
             "convrot_nvfp4_linear_prepared": [P, P, P, P, P, P, P, I64, I64, I64, P, P],
             "convrot_nvfp4_linear": [P, P, P, P, P, I64, I64, I64, I, P, SZ, P, P],
             "convrot_nvfp4_check_device_error": [P],
+            "convrot_nvfp4_debug_gemm_form": [P, P, P, P, P, P, P, I64, I64, I64, I, P, P],
         }
         for name, args in sigs.items():
             f = getattr(L, name)
@@ -665,6 +666,27 @@ def convrot_nvfp4_linear_prepared(qx, sfx, sx, qw, sfw, sw, bias, K: int, out=No
         _check(lib_nvfp4().convrot_nvfp4_linear_prepared(
             _p(qx), _p(sfx), _p(sx), _p(qw), _p(sfw), _p(sw), _p(bias), M, N, K, _p(out),
             _stream(stream)), "convrot_nvfp4_linear_prepared")
+    return out
+
+
+# GEMM forms of convrot_nvfp4_debug_gemm_form: automatic, 256- or 128-wide
+# weight tiles
+NVFP4_AUTO, NVFP4_TILES_256, NVFP4_TILES_128 = 0, 1, 2
+
+
+def convrot_nvfp4_debug_gemm_form(qx, sfx, sx, qw, sfw, sw, bias, K: int, form: int, out=None,
+                                  stream=None):
+    """convrot_nvfp4_linear_prepared with the GEMM's tile width forced
+    (NVFP4_*)."""
+    M = _nvfp4_operand(qx, sfx, sx, K, "qx")
+    N = _nvfp4_operand(qw, sfw, sw, K, "qw", qx)
+    _need_opt(bias, torch.bfloat16, "bias", (N,), qx)
+    with torch.cuda.device(qx.device):
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=qx.device) if out is None else out
+        _need(out, torch.bfloat16, "out", (M, N), qx)
+        _check(lib_nvfp4().convrot_nvfp4_debug_gemm_form(
+            _p(qx), _p(sfx), _p(sx), _p(qw), _p(sfw), _p(sw), _p(bias), M, N, K, int(form),
+            _p(out), _stream(stream)), "convrot_nvfp4_debug_gemm_form")
     return out
 
 

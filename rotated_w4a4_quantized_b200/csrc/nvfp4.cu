@@ -190,12 +190,9 @@ quant_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__
 // ------------------------------------------------------------------ GEMM
 
 constexpr int BM = 128;                  // token rows per tile (the MMA's M)
-constexpr int BN = 256;                  // weight rows per tile (the MMA's N)
 constexpr int PKB = 128;                 // packed bytes per row per stage: 256 codes
 constexpr int KB = 4;                    // MMAs (K = 64) per stage
-constexpr int SP = 3;                    // ring stages
 constexpr int A_ST = BM * PKB;           // 16 KB
-constexpr int B_ST = BN * PKB;           // 32 KB
 // Scales are staged for 128-lane copies (tcgen05.cp 128x256b): a copy
 // source is 128 rows x 32 bytes, row i = 32 q + l holding lane l's 16 bytes
 // of two scale atoms (so each lane quarter q receives the same values, as
@@ -205,21 +202,36 @@ constexpr int B_ST = BN * PKB;           // 32 KB
 // one TMA (make_sf_map) fills a whole 4 KB source.
 constexpr int SF_SRC = 4096;
 constexpr int SFA_ST = (KB / 2) * SF_SRC;   // A: the atoms of steps 2p, 2p + 1 per source
-constexpr int SFB_ST = KB * SF_SRC;         // B: the two 128-row atoms of one step per source
-constexpr int OFF_A = 0;                 // 1024-aligned tiles first
-constexpr int OFF_B = OFF_A + SP * A_ST;
-constexpr int OFF_SFA = OFF_B + SP * B_ST;
-constexpr int OFF_SFB = OFF_SFA + SP * SFA_ST;
-constexpr int OFF_BAR = OFF_SFB + SP * SFB_ST;
-constexpr int NUM_BARS = 2 * SP + 3;
-constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + slack for 1024 alignment
-static_assert(SMEM_BYTES <= 232448, "exceeds the per-CTA shared memory limit");
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpEpi0 = 2, kEpiWarps = 4;
 constexpr int kThreads = (kWarpEpi0 + kEpiWarps) * 32;   // 192
-constexpr int TMEM_COLS = 512;
-constexpr int SF_COL = BN;               // scale regions after the accumulator
-constexpr int SF_REGION = KB * 4 + KB * 8;   // 16 columns of A scales + 32 of B scales
+
+// Tiles of 128 tokens x BN weight rows (the MMA's N): 256, or 128 where the
+// 256-wide grid would leave most SMs idle (few tokens, small layers).
+//   BN = 256: a weight copy source holds the two 128-row atoms of one step;
+//   BN = 128: like the tokens, the atoms of steps 2p, 2p + 1.
+template <int BN>
+struct GCfg {
+    static_assert(BN == 128 || BN == 256, "128- or 256-wide weight tiles");
+    static constexpr int B_ST = BN * PKB;                         // 32 or 16 KB
+    static constexpr int SFB_ST = (BN == 256 ? KB : KB / 2) * SF_SRC;
+    static constexpr int ST = A_ST + B_ST + SFA_ST + SFB_ST;       // 72 or 48 KB
+    static constexpr int SP = BN == 256 ? 3 : 4;                   // ring stages
+    static constexpr int OFF_A = 0;                                // 1024-aligned tiles first
+    static constexpr int OFF_B = OFF_A + SP * A_ST;
+    static constexpr int OFF_SFA = OFF_B + SP * B_ST;
+    static constexpr int OFF_SFB = OFF_SFA + SP * SFA_ST;
+    static constexpr int OFF_BAR = OFF_SFB + SP * SFB_ST;
+    static constexpr int NUM_BARS = 2 * SP + 3;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;       // + slack for 1024 alignment
+    static_assert(SMEM_BYTES <= 232448, "exceeds the per-CTA shared memory limit");
+    static constexpr int SFB_COLS = BN / 32;                       // TMEM columns per step
+    static constexpr int SF_COL = BN;                              // scales after the accumulator
+    static constexpr int SF_REGION = KB * 4 + KB * SFB_COLS;       // A then B scales of a stage
+    static constexpr int TMEM_NEED = SF_COL + 2 * SF_REGION;
+    static constexpr int TMEM_COLS = TMEM_NEED <= 256 ? 256 : 512;
+    static_assert(TMEM_NEED <= 512, "TMEM holds 512 columns");
+};
 
 // Instruction descriptor of tcgen05.mma kind::mxf4nvf4: A and B E2M1 (1),
 // both K-major, E4M3 scales (scale format 0), scale-factor ids 0, M x N,
@@ -283,31 +295,33 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
 }
 
 // tmA: codes of the tokens [M][K/2], box 128 B x 128 rows, 128-byte swizzle.
-// tmB: codes of the weights [N][K/2], box 128 B x 256 rows, 128-byte swizzle.
+// tmB: codes of the weights [N][K/2], box 128 B x BN rows, 128-byte swizzle.
 // tmSA, tmSB: the scale atoms of the tokens and of the weights (rows padded
 // to 128) as copy-source replicas (make_sf_map); sx, sw: row scales.
+template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmSA,
                   const __grid_constant__ CUtensorMap tmSB,
                   const float *__restrict__ sx, const float *__restrict__ sw,
                   const uint16_t *__restrict__ bias, uint16_t *__restrict__ y, int M, int N, int K) {
+    using C = GCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = ptx::smem_u32(smem);
-    const uint32_t bar0 = sbase + OFF_BAR;
+    const uint32_t bar0 = sbase + C::OFF_BAR;
     auto full_p = [&](int st) { return bar0 + 8u * st; };
-    auto empty_p = [&](int st) { return bar0 + 8u * (SP + st); };
-    const uint32_t acc_full = bar0 + 8u * (2 * SP);
-    const uint32_t acc_empty = bar0 + 8u * (2 * SP + 1);
-    const uint32_t drain_bar = bar0 + 8u * (2 * SP + 2);
-    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + OFF_MISC);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+    auto empty_p = [&](int st) { return bar0 + 8u * (C::SP + st); };
+    const uint32_t acc_full = bar0 + 8u * (2 * C::SP);
+    const uint32_t acc_empty = bar0 + 8u * (2 * C::SP + 1);
+    const uint32_t drain_bar = bar0 + 8u * (2 * C::SP + 2);
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int st = 0; st < SP; ++st) {
+        for (int st = 0; st < C::SP; ++st) {
             ptx::mbar_init(full_p(st), 1);
             ptx::mbar_init(empty_p(st), 1);
         }
@@ -322,7 +336,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         ptx::tma_prefetch_desc(&tmSB);
     }
     if (warp == kWarpMma) {
-        ptx::tmem_alloc<1>(sbase + OFF_MISC, TMEM_COLS);
+        ptx::tmem_alloc<1>(sbase + C::OFF_MISC, C::TMEM_COLS);
         ptx::tmem_relinquish<1>();
     }
     ptx::tc_fence_before();
@@ -351,22 +365,28 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                 const int s0 = kp * KB;                      // first scale atom (step)
                 // one 4 KB copy source per TMA; steps past K are not requested
                 // (a pair's second step past K reads as zeros)
+                const int nsrc_b = BN == 256 ? nk : npairs;  // weight scale sources
                 ptx::mbar_arrive_expect_tx(full_p(ps),
-                                           A_ST + B_ST + (npairs + nk) * SF_SRC);
-                ptx::tma_load_2d(sbase + OFF_A + ps * A_ST, &tmA, full_p(ps), kp * PKB, m0);
-                ptx::tma_load_2d(sbase + OFF_B + ps * B_ST, &tmB, full_p(ps), kp * PKB, n0);
+                                           A_ST + C::B_ST + (npairs + nsrc_b) * SF_SRC);
+                ptx::tma_load_2d(sbase + C::OFF_A + ps * A_ST, &tmA, full_p(ps), kp * PKB, m0);
+                ptx::tma_load_2d(sbase + C::OFF_B + ps * C::B_ST, &tmB, full_p(ps), kp * PKB, n0);
                 for (int pr = 0; pr < npairs; ++pr)
-                    tma_load_sf(sbase + OFF_SFA + ps * SFA_ST + pr * SF_SRC, &tmSA, full_p(ps),
+                    tma_load_sf(sbase + C::OFF_SFA + ps * SFA_ST + pr * SF_SRC, &tmSA, full_p(ps),
                                 s0 + 2 * pr, m0 / 128);
-                for (int j = 0; j < nk; ++j)
-                    tma_load_sf(sbase + OFF_SFB + ps * SFB_ST + j * SF_SRC, &tmSB, full_p(ps),
-                                n0 / 128, s0 + j);
-                if (++ps == SP) { ps = 0; ph ^= 1; }
+                for (int j = 0; j < nsrc_b; ++j) {
+                    if (BN == 256)       // step s0 + j, both 128-row halves
+                        tma_load_sf(sbase + C::OFF_SFB + ps * C::SFB_ST + j * SF_SRC, &tmSB,
+                                    full_p(ps), n0 / 128, s0 + j);
+                    else                 // steps s0 + 2 j, + 1 of the one 128-row group
+                        tma_load_sf(sbase + C::OFF_SFB + ps * C::SFB_ST + j * SF_SRC, &tmSB,
+                                    full_p(ps), s0 + 2 * j, n0 / 128);
+                }
+                if (++ps == C::SP) { ps = 0; ph ^= 1; }
             }
         }
         if (!ok) {
             // let copies already in flight land before the CTA exits
-            for (int st = 0; st < SP; ++st) {
+            for (int st = 0; st < C::SP; ++st) {
                 volatile int never = 0;
                 ptx::mbar_wait(full_p(st), ph ^ (st < ps ? 0u : 1u), &never, 10000000ull);
             }
@@ -386,24 +406,25 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                     if (!ptx::mbar_wait(full_p(ps), pph, abort_flag)) { ok = false; break; }
                     ptx::tc_fence_after();
                     const int nk = min(KB, nkb - kp * KB);
-                    const uint32_t sfa_t = tmem_base + static_cast<uint32_t>(SF_COL + (kglob & 1) * SF_REGION);
+                    const uint32_t sfa_t = tmem_base + static_cast<uint32_t>(C::SF_COL + (kglob & 1) * C::SF_REGION);
                     const uint32_t sfb_t = sfa_t + KB * 4;
-                    const uint32_t sa = sbase + OFF_SFA + ps * SFA_ST;
-                    const uint32_t sb = sbase + OFF_SFB + ps * SFB_ST;
+                    const uint32_t sa = sbase + C::OFF_SFA + ps * SFA_ST;
+                    const uint32_t sb = sbase + C::OFF_SFB + ps * C::SFB_ST;
                     // step j's scales: token columns sfa_t + 4 j (two steps per
-                    // copy), weight columns sfb_t + 8 j (both 128-row halves
-                    // of the tile per copy)
+                    // copy); weight columns sfb_t + 8 j (BN = 256: both 128-row
+                    // halves of the tile per copy) or sfb_t + 4 j (BN = 128: two
+                    // steps per copy)
                     for (int pr = 0; 2 * pr < nk; ++pr)
                         tmem_cp_sf(sfa_t + 8 * pr, sf_src_desc(sa + pr * SF_SRC));
-                    for (int j = 0; j < nk; ++j)
+                    for (int j = 0; j < (BN == 256 ? nk : (nk + 1) / 2); ++j)
                         tmem_cp_sf(sfb_t + 8 * j, sf_src_desc(sb + j * SF_SRC));
-                    const uint32_t a0 = sbase + OFF_A + ps * A_ST, b0 = sbase + OFF_B + ps * B_ST;
+                    const uint32_t a0 = sbase + C::OFF_A + ps * A_ST, b0 = sbase + C::OFF_B + ps * C::B_ST;
                     for (int j = 0; j < nk; ++j)
                         mma_mxf4(tmem_base, ptx::sw128_kmajor_desc(a0 + 32 * j),
                                  ptx::sw128_kmajor_desc(b0 + 32 * j), idesc, sfa_t + 4 * j,
-                                 sfb_t + 8 * j, (kp | j) != 0 ? 1u : 0u);
+                                 sfb_t + C::SFB_COLS * j, (kp | j) != 0 ? 1u : 0u);
                     ptx::tc_commit<1>(empty_p(ps));
-                    if (++ps == SP) { ps = 0; pph ^= 1; }
+                    if (++ps == C::SP) { ps = 0; pph ^= 1; }
                 }
                 if (ok) ptx::tc_commit<1>(acc_full);
             }
@@ -471,7 +492,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     ptx::tc_fence_after();
     if (warp == kWarpMma) {
         __syncwarp();
-        ptx::tmem_dealloc<1>(tmem_base, TMEM_COLS);
+        ptx::tmem_dealloc<1>(tmem_base, C::TMEM_COLS);
     }
 }
 
@@ -545,7 +566,8 @@ convrot_status device_setup(int *dev_out) {
     bool ok = true;
     ok &= set_smem(nvfp4::quant_kernel<64>, kQuantSmemMax);
     ok &= set_smem(nvfp4::quant_kernel<256>, kQuantSmemMax);
-    ok &= set_smem(nvfp4::nvfp4_gemm_kernel, nvfp4::SMEM_BYTES);
+    ok &= set_smem(nvfp4::nvfp4_gemm_kernel<256>, nvfp4::GCfg<256>::SMEM_BYTES);
+    ok &= set_smem(nvfp4::nvfp4_gemm_kernel<128>, nvfp4::GCfg<128>::SMEM_BYTES);
     st.num_sms = sms;
     st.status = ok ? CONVROT_OK : CONVROT_ERR_CUDA;
     st.ready.store(true, std::memory_order_release);
@@ -650,21 +672,25 @@ bool make_sf_map(CUtensorMap *map, const uint8_t *sf, int64_t rows, int64_t K, b
                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-convrot_status launch_gemm(int num_sms, const uint8_t *qx, const uint8_t *sfx, const float *sx,
-                           const uint8_t *qw, const uint8_t *sfw, const float *sw,
-                           const void *bias, int64_t M, int64_t N, int64_t K, void *y,
-                           cudaStream_t stream) {
+template <int BN>
+convrot_status launch_gemm_bn(int num_sms, const uint8_t *qx, const uint8_t *sfx, const float *sx,
+                              const uint8_t *qw, const uint8_t *sfw, const float *sw,
+                              const void *bias, int64_t M, int64_t N, int64_t K, void *y,
+                              cudaStream_t stream) {
+    using C = nvfp4::GCfg<BN>;
     CUtensorMap tmA, tmB;
     CUtensorMap tmSA, tmSB;
-    if (!make_code_map(&tmA, qx, M, K, nvfp4::BM) || !make_code_map(&tmB, qw, N, K, nvfp4::BN) ||
-        !make_sf_map(&tmSA, sfx, M, K, false) || !make_sf_map(&tmSB, sfw, N, K, true))
+    // weight copy sources: the two 128-row halves of a step (BN = 256) or
+    // two steps of the one 128-row group (BN = 128, as on the token side)
+    if (!make_code_map(&tmA, qx, M, K, nvfp4::BM) || !make_code_map(&tmB, qw, N, K, BN) ||
+        !make_sf_map(&tmSA, sfx, M, K, false) || !make_sf_map(&tmSB, sfw, N, K, BN == 256))
         return CONVROT_ERR_CUDA;
-    const int64_t tiles = ((M + nvfp4::BM - 1) / nvfp4::BM) * ((N + nvfp4::BN - 1) / nvfp4::BN);
+    const int64_t tiles = ((M + nvfp4::BM - 1) / nvfp4::BM) * ((N + BN - 1) / BN);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(nvfp4::kThreads);
-    cfg.dynamicSmemBytes = nvfp4::SMEM_BYTES;
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -672,10 +698,31 @@ convrot_status launch_gemm(int num_sms, const uint8_t *qx, const uint8_t *sfx, c
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(
-        &cfg, nvfp4::nvfp4_gemm_kernel, tmA, tmB, tmSA, tmSB, sx, sw,
+        &cfg, nvfp4::nvfp4_gemm_kernel<BN>, tmA, tmB, tmSA, tmSB, sx, sw,
         static_cast<const uint16_t *>(bias), static_cast<uint16_t *>(y), static_cast<int>(M),
         static_cast<int>(N), static_cast<int>(K));
     return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
+}
+
+// GEMM forms: automatic, 256- or 128-wide weight tiles.
+enum GemmForm { kFormAuto = 0, kForm256 = 1, kForm128 = 2 };
+
+// The automatic width: 128 where twice the 256-wide tiles still fit in one
+// wave (few tokens, small layers: twice the SMs then stream the weights),
+// else 256 (fewer scale copies per flop).
+int auto_width(int64_t M, int64_t N, int num_sms) {
+    const int64_t t256 = ((M + nvfp4::BM - 1) / nvfp4::BM) * ((N + 255) / 256);
+    return 2 * t256 <= num_sms ? 128 : 256;
+}
+
+convrot_status launch_gemm(int num_sms, const uint8_t *qx, const uint8_t *sfx, const float *sx,
+                           const uint8_t *qw, const uint8_t *sfw, const float *sw,
+                           const void *bias, int64_t M, int64_t N, int64_t K, void *y,
+                           cudaStream_t stream, int form = kFormAuto) {
+    const int width = form == kForm256 ? 256 : form == kForm128 ? 128 : auto_width(M, N, num_sms);
+    if (width == 128)
+        return launch_gemm_bn<128>(num_sms, qx, sfx, sx, qw, sfw, sw, bias, M, N, K, y, stream);
+    return launch_gemm_bn<256>(num_sms, qx, sfx, sx, qw, sfw, sw, bias, M, N, K, y, stream);
 }
 
 convrot_status check_gemm_shape(int64_t M, int64_t N, int64_t K) {
@@ -715,11 +762,11 @@ convrot_status convrot_nvfp4_quantize(const void *x_bf16, int64_t rows, int64_t 
     return launch_quant(g_dev[dev].num_sms, x_bf16, rows, K, group, q, sf, s, stream);
 }
 
-convrot_status convrot_nvfp4_linear_prepared(const uint8_t *qx, const uint8_t *sfx,
-                                             const float *sx, const uint8_t *qw,
-                                             const uint8_t *sfw, const float *sw,
-                                             const void *bias_bf16, int64_t M, int64_t N,
-                                             int64_t K, void *y_bf16, convrot_stream_t stream) {
+static convrot_status linear_prepared_impl(const uint8_t *qx, const uint8_t *sfx, const float *sx,
+                                           const uint8_t *qw, const uint8_t *sfw, const float *sw,
+                                           const void *bias_bf16, int64_t M, int64_t N, int64_t K,
+                                           void *y_bf16, cudaStream_t stream, int form) {
+    if (form < kFormAuto || form > kForm128) return CONVROT_ERR_SHAPE;
     convrot_status st = check_gemm_shape(M, N, K);
     if (st != CONVROT_OK) return st;
     if (M == 0 || N == 0) return CONVROT_OK;
@@ -733,7 +780,26 @@ convrot_status convrot_nvfp4_linear_prepared(const uint8_t *qx, const uint8_t *s
     if ((st = check_device_ptrs(dev, {qx, sfx, sx, qw, sfw, sw, bias_bf16, y_bf16})) != CONVROT_OK)
         return st;
     return launch_gemm(g_dev[dev].num_sms, qx, sfx, sx, qw, sfw, sw, bias_bf16, M, N, K, y_bf16,
-                       stream);
+                       stream, form);
+}
+
+convrot_status convrot_nvfp4_linear_prepared(const uint8_t *qx, const uint8_t *sfx,
+                                             const float *sx, const uint8_t *qw,
+                                             const uint8_t *sfw, const float *sw,
+                                             const void *bias_bf16, int64_t M, int64_t N,
+                                             int64_t K, void *y_bf16, convrot_stream_t stream) {
+    return linear_prepared_impl(qx, sfx, sx, qw, sfw, sw, bias_bf16, M, N, K, y_bf16, stream,
+                                kFormAuto);
+}
+
+convrot_status convrot_nvfp4_debug_gemm_form(const uint8_t *qx, const uint8_t *sfx,
+                                             const float *sx, const uint8_t *qw,
+                                             const uint8_t *sfw, const float *sw,
+                                             const void *bias_bf16, int64_t M, int64_t N,
+                                             int64_t K, int form, void *y_bf16,
+                                             convrot_stream_t stream) {
+    return linear_prepared_impl(qx, sfx, sx, qw, sfw, sw, bias_bf16, M, N, K, y_bf16, stream,
+                                form);
 }
 
 convrot_status convrot_nvfp4_linear(const void *x_bf16, const uint8_t *qw, const uint8_t *sfw,

@@ -283,7 +283,8 @@ def test_nvfp4_library_exports_every_declared_symbol():
     names = sorted(set(re.findall(r"\b(convrot_nvfp4_[a-z0-9_]+)\s*\(", text)))
     assert names == sorted(["convrot_nvfp4_scale_bytes", "convrot_nvfp4_quantize",
                             "convrot_nvfp4_workspace_size", "convrot_nvfp4_linear_prepared",
-                            "convrot_nvfp4_linear", "convrot_nvfp4_check_device_error"])
+                            "convrot_nvfp4_linear", "convrot_nvfp4_check_device_error",
+                            "convrot_nvfp4_debug_gemm_form"])
     L = cr.lib_nvfp4()
     for name in names:
         assert hasattr(L, name), name
@@ -297,3 +298,10 @@ def test_nvfp4_library_exports_every_declared_symbol():
     assert L.convrot_nvfp4_quantize(None, 4, 1024, 64, B, B, B, None) == 1
     assert L.convrot_nvfp4_linear_prepared(A, A, A, A, A, A, None, 4, 4, 100, B, None) == 3
     assert L.convrot_nvfp4_linear(A, A, A, A, None, 4, 4, 1024, 64, B, 16, B, None) == 5
+    # forced tile widths: forms 0..2 only; the shape checks as for the product
+    f = L.convrot_nvfp4_debug_gemm_form
+    assert f(A, A, A, A, A, A, None, 4, 4, 1024, 3, B, None) == 3
+    assert f(A, A, A, A, A, A, None, 4, 4, 1024, -1, B, None) == 3
+    assert f(A, A, A, A, A, A, None, 4, 4, 100, 1, B, None) == 3      # K % 64
+    assert f(None, A, A, A, A, A, None, 4, 4, 1024, 2, B, None) == 1
+    assert f(A, A, A, A, A, A, None, 0, 4, 1024, 2, B, None) == 0     # no tokens: nothing to do

@@ -20,7 +20,7 @@ to run:
   when N % 8 == 0, direct stores otherwise);
 - split K, with the planner's and forced plans;
 - the repacked-weight forms and the no-alloc entry point;
-- the W4A16 and NVFP4 variants.
+- the W4A16 and NVFP4 variants, with each NVFP4 tile width.
 
 Empty inputs (M = 0) must write nothing."""
 import numpy as np
@@ -358,3 +358,9 @@ def test_nvfp4_writes_only_its_outputs(M, K, N, group):
     _verify("nvfp4 linear", [ws, y1, y2], inp, [(y1.t, y_ref)] + ([(y2.t, y_ref)] if M else []),
             chk)
     assert inp2.unchanged()
+    if M:                           # each tile width, forced
+        for form in (cr.NVFP4_TILES_256, cr.NVFP4_TILES_128):
+            want = cr.convrot_nvfp4_debug_gemm_form(qx_ref, sfx_ref, sx_ref, qw, sfw, sw, b, K, form)
+            y3 = Guarded((M, N), torch.bfloat16)
+            cr.convrot_nvfp4_debug_gemm_form(qx_ref, sfx_ref, sx_ref, qw, sfw, sw, b, K, form, y3.t)
+            _verify(f"nvfp4 form {form}", [y3], inp2, [(y3.t, want)], chk)

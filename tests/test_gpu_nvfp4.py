@@ -101,15 +101,35 @@ def _prepared_case(M, N, K, group, seed, bias=True):
     return ops, (t, acc, l1, p64, sx, sw), lt
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (1, 16, 64), (130, 200, 192), (300, 520, 1024),
-                                   (64, 1000, 3072), (257, 256, 4096), (40, 136, 12288)])
-def test_gemm_matches_oracle(M, N, K):
+GEMM_CASES = [(128, 256, 256), (1, 16, 64), (130, 200, 192), (300, 520, 1024), (64, 1000, 3072),
+              (257, 256, 4096), (40, 136, 12288), (600, 1300, 320)]
+
+
+# Every tile width, forced (128 tokens x 256 or 128 weight rows; K tails
+# inside a 256-code stage at K = 64, 192, 320; a last weight tile holding
+# one 128-row group of scales or less), and the automatic choice.
+@pytest.mark.parametrize("form", [cr.NVFP4_AUTO, cr.NVFP4_TILES_256, cr.NVFP4_TILES_128],
+                         ids=["auto", "w256", "w128"])
+@pytest.mark.parametrize("M,N,K", GEMM_CASES)
+def test_gemm_matches_oracle(form, M, N, K):
     ops, (t, acc, l1, p64, sx, sw), _ = _prepared_case(M, N, K, 64, seed=M * N + K)
-    y = cr.convrot_nvfp4_linear_prepared(*ops, K)
+    y = cr.convrot_nvfp4_debug_gemm_form(*ops, K, form)
     torch.cuda.synchronize()
     assert cr.convrot_nvfp4_check_device_error() == 0
     share = gc.check_nvfp4_outputs(gc.to_np_u16(y), t, acc, l1, p64, sx, sw)
     assert share > 0.9
+    if form == cr.NVFP4_AUTO:     # the public call runs the same kernel
+        y2 = cr.convrot_nvfp4_linear_prepared(*ops, K)
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+
+
+def test_gemm_form_hook_refuses_other_forms():
+    ops, _, _ = _prepared_case(4, 16, 64, 64, seed=1)
+    for form in (3, -1):
+        with pytest.raises(cr.ConvRotError) as e:
+            cr.convrot_nvfp4_debug_gemm_form(*ops, 64, form)
+        assert e.value.status == 3
 
 
 def test_zero_rows_give_exactly_the_bias():
