@@ -178,12 +178,29 @@ quant_kernel(const uint16_t *__restrict__ x, int M, int K, uint8_t *__restrict__
                            prep::pick4(words[1], words[3], words[5], words[7], m));
         }
     }
-    // The padding rows of the last 128-row atom get scale code 0 (the value
-    // 0), so that every byte of sf is a function of x alone.
-    const int padded = (M + 127) & ~127;
-    for (int r = M + static_cast<int>(blockIdx.x); r < padded; r += gridDim.x) {
-#pragma unroll
-        for (int b = 0; b < 4; ++b) sf[sf_offset(r, prep::row_chan<G>(t, 16 * b) / 16, K)] = 0;
+    // The padding rows of the last 128-row group get scale code 0 (the value
+    // 0), so that every byte of sf is a function of x alone.  In an atom, the
+    // 16-byte chunk l holds the four scales (one 32-bit word) of each of rows
+    // l, l + 32, l + 64, l + 96 of the group: a chunk whose rows are all
+    // padding is cleared with one 16-byte store, the padding words of the
+    // others one by one.  These stores touch no byte of a real row.  A warp
+    // takes whole atoms, a lane the chunks l = lane, lane + (warp's lanes).
+    const int m = M & 127;                               // real rows of the last group
+    if (m != 0) {
+        uint8_t *grp = sf + static_cast<size_t>(M >> 7) * (K / 64) * 512;
+        const int nw = (nthreads + 31) >> 5;
+        for (int a = warp + static_cast<int>(blockIdx.x) * nw; a < K / 64;
+             a += static_cast<int>(gridDim.x) * nw) {
+            uint8_t *atom = grp + static_cast<size_t>(a) * 512;
+            for (int l = lane; l < 32; l += warp_lanes) {
+                const int c0 = l >= m ? 0 : (m - l + 31) / 32;   // first padding word
+                if (c0 == 0)
+                    *reinterpret_cast<uint4 *>(atom + 16 * l) = make_uint4(0u, 0u, 0u, 0u);
+                else
+                    for (int c = c0; c < 4; ++c)
+                        *reinterpret_cast<uint32_t *>(atom + 16 * l + 4 * c) = 0u;
+            }
+        }
     }
 }
 
@@ -625,7 +642,12 @@ convrot_status launch_quant(int num_sms, const void *x, int64_t rows, int64_t K,
     if (rows == 0) return CONVROT_OK;
     const size_t smem = static_cast<size_t>(K) * 2;
     const int64_t resident = static_cast<int64_t>(num_sms) * quant_ctas_per_sm(group, K);
-    const dim3 grid(static_cast<unsigned>(rows < resident ? rows : resident));
+    int64_t ctas = rows < resident ? rows : resident;
+    // With padding rows in the last 128-row group, at least 16 CTAs, so that
+    // each warp clears about two scale atoms of it (CTAs past the last row do
+    // only that): one CTA clearing all K/64 atoms took ~4 us more at one row.
+    if ((rows & 127) != 0 && ctas < 16) ctas = 16;
+    const dim3 grid(static_cast<unsigned>(ctas));
     const dim3 block(static_cast<unsigned>(K / prep::kElemsPerThread));
     const uint16_t *xx = static_cast<const uint16_t *>(x);
     if (group == 64)
