@@ -12,7 +12,8 @@
 //                     block maximum -> E4M3 scale (cvt ... e4m3x2), codes by
 //                     cvt ... e2m1x2 (round to nearest even, saturating), the
 //                     scales written in the tensor cores' atom layout;
-//   nvfp4_gemm_kernel persistent output tiles of 128 tokens x 256 weight
+//   nvfp4_gemm_kernel persistent output tiles of 128 tokens x BN = 256 (or,
+//                     where that grid is under half a wave, 128) weight
 //                     rows, one CTA per SM:
 //     warp 0      producer (one thread): per stage of 256 codes, the packed
 //                 token and weight tiles by TMA (128-byte swizzle) and the
@@ -22,8 +23,8 @@
 //                 copies the scales into TMEM (tcgen05.cp 128x256b: lane
 //                 quarter q receives replica q, so row n's four scales of one
 //                 64-code step sit in lane n mod 32 of every quarter, column
-//                 n / 32) and issues four MMAs of K = 64 (M = 128, N = 256)
-//                 into one fp32 accumulator of 256 columns;
+//                 n / 32) and issues four MMAs of K = 64 (M = 128, N = BN)
+//                 into one fp32 accumulator of BN columns;
 //     warps 2..5  epilogue, one per TMEM lane quarter: tcgen05.ld, (acc * sx)
 //                 * sw + b, bf16, stores; then the accumulator is free.
 #include <cuda.h>
