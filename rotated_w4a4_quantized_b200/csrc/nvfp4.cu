@@ -232,8 +232,7 @@ struct GCfg {
     static_assert(BN == 128 || BN == 256, "128- or 256-wide weight tiles");
     static constexpr int B_ST = BN * PKB;                         // 32 or 16 KB
     static constexpr int SFB_ST = (BN == 256 ? KB : KB / 2) * SF_SRC;
-    static constexpr int ST = A_ST + B_ST + SFA_ST + SFB_ST;       // 72 or 48 KB
-    static constexpr int SP = BN == 256 ? 3 : 4;                   // ring stages
+    static constexpr int SP = BN == 256 ? 3 : 4;                   // ring stages of 72 or 48 KB
     static constexpr int OFF_A = 0;                                // 1024-aligned tiles first
     static constexpr int OFF_B = OFF_A + SP * A_ST;
     static constexpr int OFF_SFA = OFF_B + SP * B_ST;
